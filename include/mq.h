@@ -1,0 +1,287 @@
+/*
+ * mq — quantized-KV decode attention for NVIDIA B200 (sm_100a).
+ *
+ * A C ABI over hand-written CUDA kernels for the per-token decode step of an
+ * inference engine whose KV cache stores keys as int8 and values as int4:
+ *
+ *   mq_kv_append    quantize-on-append of new K/V tokens into a paged cache
+ *   mq_decode_attn  attention of a few query tokens per sequence (1 = decode,
+ *                   n > 1 = verification of n speculative draft tokens, causal
+ *                   among the drafts) against the cache, split over the
+ *                   sequence and merged by log-sum-exp
+ *   mq_tune         on-device choice of the decode launch shape under a
+ *                   wall-clock budget, accepting only bit-identical candidates
+ *
+ * Where the operations come from.  The blog.123qwe.co.kr deep dive on
+ * magnitudedev/magnitude, section 5 ("core mechanism 3: speculative decoding,
+ * quantized KV, prefix sharing"), reports the decode attention unit
+ * attention_decode_k8v4 with the codec "Key 8-bit, Value 4-bit, group 32, f16
+ * scale", the guarantee that verifying several draft tokens costs one decode
+ * step because decode is bandwidth-bound, and sessions sharing a prefix cache.
+ * Its section 3 ("core mechanism 1: the 60 s first-load tuner") describes the
+ * tuner: a 60 s wall-clock budget, candidates measured on the device, a cost
+ * summed over serving shapes (4k/64k decode, verification width) weighted by
+ * their time at the default configuration, and timing passes sized beyond the
+ * last-level cache.  The paper-digest.app summary ("Core Mechanics") adds that
+ * the tuner keeps only configurations that do not change model output.
+ *
+ * The codec's arithmetic is this library's fixed reading (the pages name the
+ * codec only):
+ *   K, per (token, kv-head) vector: s = fp16_rn(max|x| / 127), computed as an
+ *     IEEE fp32 division then rounded to fp16; code = clamp(rne(x / s), -127,
+ *     127) with an IEEE fp32 division; s == 0 gives code 0.
+ *   V, per (token, kv-head, 32 consecutive channels): s = fp16_rn(max|x| / 7),
+ *     code = clamp(rne(x / s), -8, 7); two codes per byte, the even channel in
+ *     the low nibble, two's complement nibbles.
+ *   Symmetric (no zero point).  NaN inputs give code 0; scales that overflow
+ *     fp16 become +inf and give code 0 (inputs beyond 65504*127 for K or
+ *     65504*7 for V are outside the codec's domain).
+ *
+ * Conventions
+ *   - Every pointer argument is a DEVICE pointer owned by the caller unless
+ *     stated otherwise; the library never frees caller memory.  The opaque
+ *     mq_cache handle is a host object allocated by mq_cache_create.
+ *   - Every call returns an mq_status and never throws.  Host-side validation
+ *     happens before any CUDA call; a failed validation launches nothing.
+ *   - Calls that launch work are asynchronous on `stream` (a cudaStream_t; NULL
+ *     is the legacy default stream).  Faults inside kernels surface at the next
+ *     synchronization; conditions a kernel detects itself (an out-of-range
+ *     block id or position, a wait that ran out of time) set a device error
+ *     word that mq_device_status() reads and clears.
+ *   - A cache handle is not thread-safe; distinct handles are independent.
+ */
+#ifndef MQ_H
+#define MQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (CUDA's runtime stream handle); NULL is the legacy default stream. */
+typedef struct CUstream_st* mq_stream;
+
+typedef enum mq_status {
+    MQ_OK = 0,
+    MQ_ERR_INVALID_ARG = 1,     /* null pointer, bad size or count, inconsistent arguments     */
+    MQ_ERR_UNSUPPORTED = 2,     /* head_dim not 128/256, page size not 16, dtype, too many rows  */
+    MQ_ERR_CAPACITY = 3,        /* pool too small for n_blocks, max_seq_len beyond the table     */
+    MQ_ERR_WORKSPACE = 4,       /* workspace null, too small or misaligned                      */
+    MQ_ERR_CUDA = 5,            /* a CUDA runtime call or kernel launch failed                   */
+    MQ_ERR_DEVICE = 6,          /* a kernel flagged a bad block id/position/length or a timeout  */
+    MQ_TUNE_BUDGET_EXHAUSTED = 7 /* warning: the tuner's budget ran out before every candidate    */
+} mq_status;
+
+typedef enum mq_dtype { MQ_F32 = 0, MQ_BF16 = 1, MQ_F16 = 2 } mq_dtype;
+
+/* Tokens per page; fixed. */
+#define MQ_PAGE_TOKENS 16
+
+/* ---------------------------------------------------------------------------
+ * Cache layout
+ *
+ * The pool is an array of n_blocks blocks; a block holds MQ_PAGE_TOKENS
+ * consecutive token positions of one sequence for every kv-head, as n_kv_heads
+ * pages of mq_page_bytes(head_dim) bytes: page (block, h) starts at byte
+ * (block * n_kv_heads + h) * mq_page_bytes(head_dim).  A page holds the 16
+ * tokens of one (block, kv-head):
+ *     K codes   16*D bytes      int8
+ *     K scales  16 * 2 bytes    fp16, one per token
+ *     V codes   16*D/2 bytes    int4 pairs
+ *     V scales  16*D/32 * 2     fp16, one per (token, 32-channel group)
+ * = 25*D + 32 bytes (3232 for D = 128, 6432 for D = 256), against 64*D for
+ * fp16 K+V: 0.395x (D = 128) and 0.393x (D = 256) — "more than half" smaller,
+ * as the trawling.dev Launch HN page (per-device tuning and performance claims)
+ * reports for this codec.  Within each region the bytes are permuted so that
+ * the decode kernel's tensor-core fragments load with 16-byte shared-memory
+ * reads (lane L = 4g + t, g = 0..7, t = 0..3; NG = D/32 groups):
+ *     K code of token tau, channel c: byte (k*32 + L)*16 + (o % 16) with
+ *       L = 4*(tau % 8) + c / (D/4), o = c % (D/4), k = (tau / 8)*(D/64) + o/16
+ *     K scale of token tau: half-word tau of the K-scale region
+ *     V codes: 32-bit word w = 2q + p of lane L sits at ((w/4)*32 + L)*16 +
+ *       (w%4)*4 of the V-code region and holds, byte by byte, channels
+ *       (c, c+1), (c+2, c+3) of token 8p + 2t, then the same channels of token
+ *       8p + 2t + 1, with c = 32q + 4g and the even channel in the low nibble
+ *     V scale of token tau, group q: half-word ((t'*NG + q)*2 + tau/8)*2 + tau%2
+ *       of the V-scale region, t' = (tau % 8)/2
+ * The codes and scales themselves are exactly the codec's.
+ *
+ * A block_table is int32 [n_seqs][max_blocks_per_seq]: entry [b][i] is the
+ * physical block holding positions [16 i, 16 i + 16) of sequence b.  Several
+ * sequences may name the same physical block (a shared prefix: the deep dive's
+ * section 5 and the Launch HN page describe sessions sharing a prefix cache);
+ * the library only reads through block tables and never owns blocks.
+ * ------------------------------------------------------------------------- */
+typedef struct mq_cache mq_cache;
+
+typedef struct mq_cache_desc {
+    int32_t n_kv_heads;   /* >= 1                                                     */
+    int32_t head_dim;     /* 128 or 256                                               */
+    int32_t page_tokens;  /* must be MQ_PAGE_TOKENS                                   */
+    int64_t n_blocks;     /* >= 1                                                     */
+    void* pool;           /* device memory, caller-owned, 256-byte aligned            */
+    size_t pool_bytes;    /* >= mq_cache_pool_bytes(n_kv_heads, head_dim, n_blocks)   */
+} mq_cache_desc;
+
+/* Bytes of one page: 25*head_dim + 32, or 0 for an unsupported head_dim. */
+size_t mq_page_bytes(int32_t head_dim);
+
+/* Bytes the pool must hold: n_blocks * n_kv_heads * mq_page_bytes(head_dim)
+ * (0 for invalid arguments). */
+size_t mq_cache_pool_bytes(int32_t n_kv_heads, int32_t head_dim, int64_t n_blocks);
+
+/* Validates the descriptor and returns a new host handle in *out (which is set
+ * to NULL on error).  Binds the handle to the current CUDA device.  Does not
+ * touch the pool's contents.  Errors: INVALID_ARG (null, n_kv_heads < 1,
+ * n_blocks < 1, misaligned pool), UNSUPPORTED (head_dim, page_tokens),
+ * CAPACITY (pool_bytes too small), CUDA. */
+mq_status mq_cache_create(const mq_cache_desc* desc, mq_cache** out);
+
+/* Frees the handle (never the pool).  NULL is accepted. */
+mq_status mq_cache_destroy(mq_cache* cache);
+
+/* ---------------------------------------------------------------------------
+ * mq_kv_append — quantize-on-append
+ *
+ * Quantizes n_tokens new K/V vectors and writes them into their pages.
+ *   k, v         [n_tokens][n_kv_heads][head_dim], dtype `dtype` (F32, BF16 or
+ *                F16), packed by sequence in order b = 0 .. n_seqs-1
+ *   cu_new       int32 [n_seqs + 1], exclusive prefix sum of the tokens each
+ *                sequence appends (cu_new[0] = 0, cu_new[n_seqs] = n_tokens)
+ *   start_pos    int32 [n_seqs], the position of sequence b's first new token
+ *   block_table  int32 [n_seqs][max_blocks_per_seq] (see above)
+ * Token i of sequence b goes to position start_pos[b] + i, i.e. page
+ * block_table[b][pos / 16], slot pos % 16.  Two calls (or two tokens) that
+ * write the same position race; writing a position of a shared block changes
+ * it for every sequence that names the block.
+ * Errors: INVALID_ARG (null pointers, n_seqs < 1, n_tokens < 0, dtype),
+ * CUDA.  n_tokens == 0 launches nothing.  A position beyond
+ * max_blocks_per_seq*16 or a block id outside [0, n_blocks) is skipped by the
+ * kernel and reported through mq_device_status() as MQ_ERR_DEVICE.
+ * ------------------------------------------------------------------------- */
+mq_status mq_kv_append(mq_cache* cache, const void* k, const void* v, mq_dtype dtype, int32_t n_seqs,
+                       int32_t n_tokens, const int32_t* cu_new, const int32_t* start_pos,
+                       const int32_t* block_table, int32_t max_blocks_per_seq, mq_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * mq_decode_attn — attention of n_q_per_seq[b] query tokens of every sequence
+ * against its quantized cache
+ *
+ *   q            [sum_b n_q_per_seq[b]][n_q_heads][head_dim], dtype q_dtype
+ *                (F32, BF16 or F16), packed by sequence in order
+ *   seq_lens     int32 [n_seqs]: L_b, the tokens in sequence b's cache,
+ *                INCLUDING its n_q_per_seq[b] query tokens, whose K/V must
+ *                already be appended
+ *   n_q_per_seq  int32 [n_seqs]: n_b, 1 <= n_b <= min(L_b, max_q_per_seq)
+ *   total_q      host: the rows of q and out (sum_b n_b); a row index at or beyond
+ *                it is never read or written (such rows are reported through
+ *                mq_device_status())
+ *   max_q_per_seq, max_seq_len   host bounds on n_b and L_b (they size the grid)
+ *   block_table  int32 [n_seqs][max_blocks_per_seq]
+ *   softmax_scale  the logit scale (1/sqrt(head_dim) for standard attention)
+ *   out          fp32 [sum_b n_b][n_q_heads][head_dim]
+ *   lse          fp32 [sum_b n_b][n_q_heads], natural-log log-sum-exp of the
+ *                scaled logits; may be NULL
+ *   workspace    device scratch of at least mq_decode_workspace_bytes(...)
+ *                bytes, 256-byte aligned.  It must be zero-filled before its
+ *                first use; every call that completes leaves its counter
+ *                region zero again, so it can be reused across calls on the
+ *                same stream without clearing.  After MQ_ERR_DEVICE, zero it
+ *                again.  Calls that share a workspace must not overlap.
+ * Query token j of sequence b (0-based) attends to positions 0 .. L_b - n_b + j:
+ * the history plus drafts 0..j (causal among the drafts).  q-head h reads
+ * kv-head h / (n_q_heads / n_kv_heads).  The result is bit-identical for every
+ * launch configuration the tuner may choose (see mq_tune).
+ * Errors: INVALID_ARG (null pointers, n_seqs < 1 or > 65535, n_q_heads not a
+ * multiple of n_kv_heads, total_q < 1, max_q_per_seq < 1, max_seq_len <
+ * max_q_per_seq, a non-finite softmax_scale, out not 16-byte aligned), UNSUPPORTED
+ * (n_q_heads/n_kv_heads * max_q_per_seq > 64, q dtype), CAPACITY (max_seq_len >
+ * max_blocks_per_seq * 16), WORKSPACE, CUDA.  A sequence whose L_b / n_b break
+ * the bounds above is skipped by the kernel and reported by mq_device_status().
+ * ------------------------------------------------------------------------- */
+size_t mq_decode_workspace_bytes(const mq_cache* cache, int32_t n_seqs, int32_t n_q_heads, int32_t max_q_per_seq,
+                                 int32_t max_seq_len);
+
+mq_status mq_decode_attn(const mq_cache* cache, const void* q, mq_dtype q_dtype, int32_t n_seqs, int32_t n_q_heads,
+                         int32_t total_q, int32_t max_q_per_seq, int32_t max_seq_len, const int32_t* block_table,
+                         int32_t max_blocks_per_seq, const int32_t* seq_lens, const int32_t* n_q_per_seq,
+                         float softmax_scale, float* out, float* lse, void* workspace, size_t workspace_bytes,
+                         mq_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * Launch configuration and tuning
+ *
+ * The decode kernel's arithmetic is fixed: every sequence is cut into chunks of
+ * 128 tokens, each chunk is reduced by one warp in token order with an online
+ * softmax, and chunk results are combined by one fixed binary tree.  The launch
+ * configuration only decides which warp and CTA computes which subtree, so all
+ * configurations give bit-identical outputs.
+ *   warps_per_cta    4 or 8: chunks a CTA reduces concurrently
+ *   pages_per_stage  2 .. 4: pages each warp keeps in flight (TMA ring depth)
+ *   ctas_per_sm      1, 2 or 4: target CTAs per SM; fixes how many chunks one
+ *                    CTA takes (the split count along the sequence)
+ * There is one configuration per row class (query rows per kv-head, padded):
+ * rows_class 0 = up to 8 rows, 1 = up to 16, 2 = up to 32.
+ * ------------------------------------------------------------------------- */
+typedef struct mq_decode_config {
+    int32_t warps_per_cta;
+    int32_t pages_per_stage;
+    int32_t ctas_per_sm;
+} mq_decode_config;
+
+mq_status mq_get_decode_config(const mq_cache* cache, int32_t rows_class, mq_decode_config* cfg);
+mq_status mq_set_decode_config(mq_cache* cache, int32_t rows_class, const mq_decode_config* cfg);
+
+typedef struct mq_tune_params {
+    double budget_s;        /* wall-clock budget for everything the tuner does (e.g. 60) */
+    int32_t n_q_heads;      /* query heads of the model the cache serves                */
+    const char* log_path;   /* host path for the JSON evidence log, or NULL             */
+} mq_tune_params;
+
+typedef struct mq_tune_result {
+    mq_decode_config chosen[3];   /* per rows_class (unchanged if that class was not probed) */
+    double cost;                  /* weighted cost of the chosen set (1.0 = the defaults)   */
+    int32_t n_tried;              /* candidates measured                                      */
+    int32_t n_rejected;           /* candidates rejected as not bit-identical                 */
+    int32_t n_skipped;            /* candidates not reached inside the budget                 */
+    double elapsed_s;
+} mq_tune_result;
+
+/* On-device tuner.  Within params->budget_s of wall-clock time (allocation,
+ * probe set-up, every measurement included) it measures the candidate launch
+ * configurations on three probe shapes built from the cache's geometry and
+ * params->n_q_heads — decode at 4K and at 64K tokens, and verification of 8
+ * drafts at 64K — rejects any candidate whose output bytes differ from the
+ * default configuration's, and keeps the candidate set with the lowest cost
+ *     cost(c) = sum_p median_time(c, p) / median_time(default, p).
+ * Timed launches read probe caches that together exceed twice the L2 size, so
+ * no launch finds its data warm in L2.  The probes use their own device
+ * buffers (allocated and freed here; the cache's pool is not touched).  The
+ * chosen configurations are stored in the cache handle.  Returns MQ_OK, or
+ * MQ_TUNE_BUDGET_EXHAUSTED when the budget ended the search early (the best
+ * configuration measured so far is kept; the defaults if none).  Synchronizes
+ * the device.  Writes a JSON record of every candidate to params->log_path
+ * when it is not NULL. */
+mq_status mq_tune(mq_cache* cache, const mq_tune_params* params, mq_tune_result* result);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics
+ * ------------------------------------------------------------------------- */
+/* Synchronizes `stream`, then reads and clears the device error word of the
+ * cache's device: MQ_OK, MQ_ERR_DEVICE (a kernel flagged bad input or a timed
+ * out wait since the last call), or MQ_ERR_CUDA. */
+mq_status mq_device_status(const mq_cache* cache, mq_stream stream);
+
+/* Static description of a status code. */
+const char* mq_status_string(mq_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t mq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MQ_H */

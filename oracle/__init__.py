@@ -11,8 +11,8 @@ function computes, and which page passage it follows, is stated in the C file's
 header: the blog.123qwe.co.kr deep dive on magnitudedev/magnitude, section 5
 (core mechanism 3: speculative decoding, quantized KV, prefix sharing) names the
 ``attention_decode_k8v4`` unit and its codec (K 8 bit, V 4 bit, group 32, f16
-scale); the scheme's exact arithmetic is this library's reading, listed in
-DESIGN.md.
+scale); the pages give no formula, so the exact arithmetic is a fixed reading
+of them, stated in the C file's header.
 
 Parity status: quantization and dequantized attention are pinned by
 ``tests/test_oracle_*.py`` (hand-worked cases, brute force, closed forms,

@@ -12,8 +12,8 @@
  * `attention_decode_k8v4` with keys at 8 bit and values at 4 bit, groups of 32
  * and f16 scales; the trawling.dev "Launch HN: Magnitude" page (section on
  * per-device kernel tuning and performance claims) calls the KV codec
- * TurboQuant-inspired, 8-bit keys / 4-bit values.  This library fixes the
- * scheme as follows (every reading is listed in the design doc):
+ * TurboQuant-inspired, 8-bit keys / 4-bit values.  The pages give no formula,
+ * so the scheme is fixed as follows (each choice is a reading of the pages):
  *
  *   K, per (token, kv-head) vector of D channels:
  *       a = max_c |x_c|                 (fp32, exact)

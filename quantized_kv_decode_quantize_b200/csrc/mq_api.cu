@@ -1,0 +1,332 @@
+// C ABI of the mq library: argument validation, the cache handle, the choice of
+// launch shape, and the device error word.  Every entry point validates its
+// arguments on the host before making any CUDA call.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include "../../include/mq.h"
+#include "mq_device.cuh"
+#include "mq_kernels.h"
+#include "mq_host.h"
+
+namespace mq {
+
+// One error word per device (every device that loads the library holds its own copy).
+__device__ unsigned g_err_word;
+
+cudaError_t error_word_address(unsigned** out) {
+    return cudaGetSymbolAddress(reinterpret_cast<void**>(out), g_err_word);
+}
+
+int rows_class_rows(int head_dim, int cls) {
+    if (cls == 0) return 8;
+    if (cls == 1) return 16;
+    return head_dim == 128 ? 32 : 16;
+}
+
+int rows_class_for(int head_dim, int rows_total) {
+    if (rows_total <= 8) return 0;
+    if (rows_total <= 16) return 1;
+    return head_dim == 128 ? 2 : 1;
+}
+
+mq_decode_config default_config(int head_dim, int cls) {
+    mq_decode_config c{};
+    if (head_dim == 128) {
+        c.warps_per_cta = cls == 2 ? 4 : 8;
+        c.pages_per_stage = 2;
+        c.ctas_per_sm = cls == 0 ? 2 : 1;
+    } else {
+        c.warps_per_cta = cls == 0 ? 8 : 4;
+        c.pages_per_stage = 2;
+        c.ctas_per_sm = 1;
+    }
+    return c;
+}
+
+bool config_valid(const mq_decode_config& c) {
+    return (c.warps_per_cta == 4 || c.warps_per_cta == 8) && c.pages_per_stage >= 2 && c.pages_per_stage <= 4 &&
+           (c.ctas_per_sm == 1 || c.ctas_per_sm == 2 || c.ctas_per_sm == 4);
+}
+
+DevGuard::DevGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != dev) {
+        cudaSetDevice(dev);
+        switched = true;
+    }
+}
+DevGuard::~DevGuard() {
+    if (switched && prev >= 0) cudaSetDevice(prev);
+}
+
+DecodePlan plan_decode(const mq_cache* c, int n_seqs, int n_q_heads, int max_q, int max_seq_len) {
+    DecodePlan pl{};
+    const int G = n_q_heads / c->n_kv_heads;
+    const int rows_total = G * max_q;
+    pl.cls = rows_class_for(c->head_dim, rows_total);
+    pl.rows = rows_class_rows(c->head_dim, pl.cls);
+    pl.n_rb = (rows_total + pl.rows - 1) / pl.rows;
+    const mq_decode_config cfg = c->cfg[pl.cls];
+    pl.warps = cfg.warps_per_cta;
+    pl.pages_per_stage = cfg.pages_per_stage;
+    const long long max_chunks = (max_seq_len + kChunkTokens - 1) / kChunkTokens;
+    long long cpc = pl.warps;
+    while ((max_chunks + cpc - 1) / cpc > kMaxSplits) cpc *= 2;
+    const long long units = (long long)n_seqs * c->n_kv_heads * pl.n_rb;
+    const long long target = (long long)cfg.ctas_per_sm * c->n_sm;
+    while (cpc < max_chunks && units * ((max_chunks + cpc - 1) / cpc) > target) cpc *= 2;
+    pl.cpc = (int)cpc;
+    pl.max_splits = (int)std::max<long long>(1, (max_chunks + cpc - 1) / cpc);
+    if (pl.cpc < pl.warps) pl.cpc = pl.warps;
+    auto fit = [&]() {
+        const int rounds = (int)((pl.cpc + pl.warps - 1) / pl.warps);
+        int sd = 1;
+        while ((1 << (sd - 1)) < rounds) sd++;
+        pl.stack_depth = sd;
+        pl.smem = decode_smem_bytes(c->head_dim, pl.rows, pl.warps, pl.pages_per_stage, pl.stack_depth);
+    };
+    fit();
+    // A configuration that does not fit in shared memory runs with a shallower ring,
+    // then with 4 warps; the arithmetic (and so the output) is the same.
+    while (pl.smem > (size_t)c->max_smem && pl.pages_per_stage > 2) {
+        pl.pages_per_stage--;
+        fit();
+    }
+    if (pl.smem > (size_t)c->max_smem && pl.warps > 4) {
+        pl.warps = 4;
+        fit();
+    }
+    return pl;
+}
+
+size_t workspace_bytes_for(const mq_cache* c, int n_seqs, int n_rb, int rows) {
+    const size_t units = (size_t)n_seqs * c->n_kv_heads * n_rb;
+    size_t off = (units * 4 + 255) / 256 * 256;
+    off += (units * kMaxSplits * rows * 2 * 4 + 255) / 256 * 256;
+    off += units * kMaxSplits * (size_t)rows * c->head_dim * 4;
+    return off;
+}
+
+mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void* q, mq_dtype q_dtype, int n_seqs,
+                             int n_q_heads, int total_q, int max_q, const int32_t* block_table, int max_blocks,
+                             const int32_t* seq_lens, const int32_t* n_q_per_seq, float softmax_scale, float* out,
+                             float* lse, void* workspace, cudaStream_t st) {
+    if (pl.smem == 0 || pl.smem > (size_t)c->max_smem) return MQ_ERR_UNSUPPORTED;
+    cudaError_t e = ensure_decode_smem(c->device, c->head_dim, pl.rows, pl.smem);
+    if (e != cudaSuccess) return MQ_ERR_CUDA;
+    DecodeParams p{};
+    p.pool = static_cast<const uint8_t*>(c->pool);
+    p.n_kv_heads = c->n_kv_heads;
+    p.n_blocks = c->n_blocks;
+    p.q = q;
+    p.q_dtype = (int)q_dtype;
+    p.n_q_heads = n_q_heads;
+    p.group = n_q_heads / c->n_kv_heads;
+    p.total_q = total_q;
+    p.max_q = max_q;
+    p.n_seqs = n_seqs;
+    p.block_table = block_table;
+    p.max_blocks_per_seq = max_blocks;
+    p.seq_lens = seq_lens;
+    p.n_q_per_seq = n_q_per_seq;
+    p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
+    p.out = out;
+    p.lse = lse;
+    const size_t units = (size_t)n_seqs * c->n_kv_heads * pl.n_rb;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.counters = reinterpret_cast<unsigned*>(ws);
+    size_t off = (units * 4 + 255) / 256 * 256;
+    p.part_ml = reinterpret_cast<float*>(ws + off);
+    off += (units * kMaxSplits * pl.rows * 2 * 4 + 255) / 256 * 256;
+    p.part_o = reinterpret_cast<float*>(ws + off);
+    p.n_rb = pl.n_rb;
+    p.cpc = pl.cpc;
+    p.pages_per_stage = pl.pages_per_stage;
+    p.stack_depth = pl.stack_depth;
+    p.err = c->err_word;
+    e = launch_decode(p, c->head_dim, pl.rows, pl.warps, pl.max_splits, pl.smem, st);
+    return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
+}
+
+cudaError_t ensure_decode_smem(int device, int head_dim, int rows, size_t smem) {
+    // raised limit per (device, kernel variant); the attribute only grows
+    static size_t done[64][2][3] = {};
+    const int di = device & 63, hi = head_dim == 128 ? 0 : 1, ri = rows == 8 ? 0 : (rows == 16 ? 1 : 2);
+    if (done[di][hi][ri] >= smem) return cudaSuccess;
+    cudaError_t e = decode_prepare(head_dim, rows, smem);
+    if (e == cudaSuccess) done[di][hi][ri] = smem;
+    return e;
+}
+
+}  // namespace mq
+
+using namespace mq;
+
+extern "C" {
+
+const char* mq_status_string(mq_status s) {
+    switch (s) {
+        case MQ_OK: return "ok";
+        case MQ_ERR_INVALID_ARG: return "invalid argument";
+        case MQ_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MQ_ERR_CAPACITY: return "capacity exceeded";
+        case MQ_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+        case MQ_ERR_CUDA: return "CUDA error";
+        case MQ_ERR_DEVICE: return "a kernel flagged bad input or a timed-out wait";
+        case MQ_TUNE_BUDGET_EXHAUSTED: return "tuning budget exhausted before every candidate was measured";
+    }
+    return "unknown status";
+}
+
+int32_t mq_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+size_t mq_page_bytes(int32_t head_dim) {
+    return (head_dim == 128 || head_dim == 256) ? (size_t)page_bytes(head_dim) : 0;
+}
+
+size_t mq_cache_pool_bytes(int32_t n_kv_heads, int32_t head_dim, int64_t n_blocks) {
+    const size_t pb = mq_page_bytes(head_dim);
+    if (pb == 0 || n_kv_heads < 1 || n_blocks < 1) return 0;
+    return (size_t)n_blocks * (size_t)n_kv_heads * pb;
+}
+
+mq_status mq_cache_create(const mq_cache_desc* d, mq_cache** out) {
+    if (out == nullptr) return MQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (d == nullptr || d->pool == nullptr || d->n_kv_heads < 1 || d->n_blocks < 1) return MQ_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(d->pool) % 256 != 0) return MQ_ERR_INVALID_ARG;
+    if (d->head_dim != 128 && d->head_dim != 256) return MQ_ERR_UNSUPPORTED;
+    if (d->page_tokens != MQ_PAGE_TOKENS) return MQ_ERR_UNSUPPORTED;
+    if (d->pool_bytes < mq_cache_pool_bytes(d->n_kv_heads, d->head_dim, d->n_blocks)) return MQ_ERR_CAPACITY;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MQ_ERR_CUDA;
+    int n_sm = 0, max_smem = 0;
+    if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MQ_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return MQ_ERR_CUDA;
+    unsigned* err = nullptr;
+    if (error_word_address(&err) != cudaSuccess) return MQ_ERR_CUDA;
+    mq_cache* c = new (std::nothrow) mq_cache;
+    if (c == nullptr) return MQ_ERR_INVALID_ARG;
+    c->n_kv_heads = d->n_kv_heads;
+    c->head_dim = d->head_dim;
+    c->n_blocks = d->n_blocks;
+    c->pool = d->pool;
+    c->pool_bytes = d->pool_bytes;
+    c->device = dev;
+    c->n_sm = n_sm;
+    c->max_smem = max_smem;
+    c->err_word = err;
+    for (int k = 0; k < 3; k++) c->cfg[k] = default_config(d->head_dim, k);
+    *out = c;
+    return MQ_OK;
+}
+
+mq_status mq_cache_destroy(mq_cache* c) {
+    delete c;
+    return MQ_OK;
+}
+
+mq_status mq_kv_append(mq_cache* c, const void* k, const void* v, mq_dtype dtype, int32_t n_seqs, int32_t n_tokens,
+                       const int32_t* cu_new, const int32_t* start_pos, const int32_t* block_table,
+                       int32_t max_blocks_per_seq, mq_stream stream) {
+    if (c == nullptr || n_seqs < 1 || n_tokens < 0 || max_blocks_per_seq < 1) return MQ_ERR_INVALID_ARG;
+    if (dtype != MQ_F32 && dtype != MQ_BF16 && dtype != MQ_F16) return MQ_ERR_INVALID_ARG;
+    if (n_tokens == 0) return MQ_OK;
+    if (k == nullptr || v == nullptr || cu_new == nullptr || start_pos == nullptr || block_table == nullptr)
+        return MQ_ERR_INVALID_ARG;
+    const size_t esz = dtype == MQ_F32 ? 4 : 2;
+    const size_t align = esz * c->head_dim / 32;   // one lane's vector load
+    if (reinterpret_cast<uintptr_t>(k) % align || reinterpret_cast<uintptr_t>(v) % align) return MQ_ERR_INVALID_ARG;
+    DevGuard guard(c->device);
+    AppendParams p{};
+    p.pool = static_cast<uint8_t*>(c->pool);
+    p.n_kv_heads = c->n_kv_heads;
+    p.n_blocks = c->n_blocks;
+    p.k = k;
+    p.v = v;
+    p.dtype = (int)dtype;
+    p.n_seqs = n_seqs;
+    p.n_tokens = n_tokens;
+    p.cu_new = cu_new;
+    p.start_pos = start_pos;
+    p.block_table = block_table;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.err = c->err_word;
+    return launch_append(p, c->head_dim, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MQ_OK
+                                                                                               : MQ_ERR_CUDA;
+}
+
+size_t mq_decode_workspace_bytes(const mq_cache* c, int32_t n_seqs, int32_t n_q_heads, int32_t max_q_per_seq,
+                                 int32_t max_seq_len) {
+    if (c == nullptr || n_seqs < 1 || n_q_heads < 1 || n_q_heads % c->n_kv_heads != 0 || max_q_per_seq < 1 ||
+        max_seq_len < max_q_per_seq)
+        return 0;
+    const int G = n_q_heads / c->n_kv_heads;
+    const int rows_total = G * max_q_per_seq;
+    if (rows_total > 64) return 0;
+    const int cls = rows_class_for(c->head_dim, rows_total);
+    const int rows = rows_class_rows(c->head_dim, cls);
+    const int n_rb = (rows_total + rows - 1) / rows;
+    return workspace_bytes_for(c, n_seqs, n_rb, rows);
+}
+
+mq_status mq_decode_attn(const mq_cache* c, const void* q, mq_dtype q_dtype, int32_t n_seqs, int32_t n_q_heads,
+                         int32_t total_q, int32_t max_q_per_seq, int32_t max_seq_len, const int32_t* block_table,
+                         int32_t max_blocks_per_seq, const int32_t* seq_lens, const int32_t* n_q_per_seq,
+                         float softmax_scale, float* out, float* lse, void* workspace, size_t workspace_bytes,
+                         mq_stream stream) {
+    if (c == nullptr || q == nullptr || block_table == nullptr || seq_lens == nullptr || n_q_per_seq == nullptr ||
+        out == nullptr)
+        return MQ_ERR_INVALID_ARG;
+    if (n_seqs < 1 || n_seqs > 65535 || n_q_heads < 1 || n_q_heads % c->n_kv_heads != 0) return MQ_ERR_INVALID_ARG;
+    if (max_q_per_seq < 1 || max_seq_len < max_q_per_seq || total_q < 1 || max_blocks_per_seq < 1)
+        return MQ_ERR_INVALID_ARG;
+    if (!(std::isfinite(softmax_scale))) return MQ_ERR_INVALID_ARG;
+    if (q_dtype != MQ_F32 && q_dtype != MQ_BF16 && q_dtype != MQ_F16) return MQ_ERR_UNSUPPORTED;
+    const int G = n_q_heads / c->n_kv_heads;
+    if (G * max_q_per_seq > 64) return MQ_ERR_UNSUPPORTED;
+    if ((long long)max_seq_len > (long long)max_blocks_per_seq * MQ_PAGE_TOKENS) return MQ_ERR_CAPACITY;
+    if ((long long)c->n_kv_heads * ((G * max_q_per_seq + 7) / 8) > 65535) return MQ_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(out) % 16 != 0) return MQ_ERR_INVALID_ARG;
+    const size_t need = mq_decode_workspace_bytes(c, n_seqs, n_q_heads, max_q_per_seq, max_seq_len);
+    if (workspace == nullptr || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256 != 0)
+        return MQ_ERR_WORKSPACE;
+    DevGuard guard(c->device);
+    const DecodePlan pl = plan_decode(c, n_seqs, n_q_heads, max_q_per_seq, max_seq_len);
+    return launch_decode_plan(c, pl, q, q_dtype, n_seqs, n_q_heads, total_q, max_q_per_seq, block_table,
+                              max_blocks_per_seq, seq_lens, n_q_per_seq, softmax_scale, out, lse, workspace,
+                              reinterpret_cast<cudaStream_t>(stream));
+}
+
+mq_status mq_get_decode_config(const mq_cache* c, int32_t cls, mq_decode_config* cfg) {
+    if (c == nullptr || cfg == nullptr || cls < 0 || cls > 2) return MQ_ERR_INVALID_ARG;
+    *cfg = c->cfg[cls];
+    return MQ_OK;
+}
+
+mq_status mq_set_decode_config(mq_cache* c, int32_t cls, const mq_decode_config* cfg) {
+    if (c == nullptr || cfg == nullptr || cls < 0 || cls > 2) return MQ_ERR_INVALID_ARG;
+    if (!config_valid(*cfg)) return MQ_ERR_INVALID_ARG;
+    c->cfg[cls] = *cfg;
+    return MQ_OK;
+}
+
+mq_status mq_device_status(const mq_cache* c, mq_stream stream) {
+    if (c == nullptr) return MQ_ERR_INVALID_ARG;
+    DevGuard guard(c->device);
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MQ_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, c->err_word, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MQ_ERR_CUDA;
+    if (v != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpy(c->err_word, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess) return MQ_ERR_CUDA;
+        return MQ_ERR_DEVICE;
+    }
+    return MQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,770 @@
+// Split-K flash-decode over the K8/V4 paged cache, with draft verification.
+//
+// What it computes (the deep dive on magnitudedev/magnitude at blog.123qwe.co.kr,
+// section 5: the decode attention unit attention_decode_k8v4 over the 8-bit-key /
+// 4-bit-value cache, and the guarantee that verifying several draft tokens is
+// one launch against the cache): for query token j of sequence b (n_b query
+// tokens, L_b cached tokens including the drafts) and q-head h,
+//     z_t = scale * <q, s_k[t] * kcode_t>,  t = 0 .. L_b - n_b + j
+//     out = sum_t softmax(z)_t * (s_v[t, group] * vcode_t),  lse = log sum_t exp z_t
+//
+// How, on sm_100a:
+//  * One CTA takes an aligned block of 128-token chunks of one (sequence, kv-head,
+//    row block); every warp of the CTA takes one chunk per round.  Pages (16
+//    tokens of one kv-head, 3232 or 6432 bytes) stream into a per-warp shared-memory
+//    ring by 1-D bulk TMA copies (cp.async.bulk + mbarrier, L2 evict-first), looked
+//    up through the block table.
+//  * QK^T on the tensor cores in int8: q is held as a 23-bit fixed-point value per
+//    row (q = Q * 2^(E-22), |Q| <= 2^22) split into three 8-bit limbs, so the int8
+//    key codes feed mma.m16n8k32 straight from shared memory with no conversion and
+//    the int32 products are exact; the limbs are combined once per score in fp32.
+//  * P.V on the tensor cores in fp16: the int4 value codes become exact fp16
+//    integers with two LOP3 + one HADD2/HFMA2 per pair; the weights
+//    p * s_v[token, group] are rounded to fp16 (relative error <= 2^-11 per weight).
+//  * Within a chunk one warp keeps an online softmax (running max in log2 units).
+//    Chunk results are combined by ONE fixed binary tree over chunk indices
+//    (warps of a round, rounds of a CTA, CTAs of a sequence), so the output does
+//    not depend on warps per CTA, ring depth or split count.  The last CTA of each
+//    (sequence, kv-head, row block) to finish — found with one atomic counter —
+//    completes the tree over the CTA partials and writes out and lse; there is no
+//    second kernel and no CTA ever waits for another.
+#include <cfloat>
+
+#include "mq_device.cuh"
+#include "mq_kernels.h"
+
+namespace mq {
+
+template <int D, int ROWS>
+struct Cfg {
+    static constexpr int PB = page_bytes(D);
+    static constexpr int NG = D / 32;            // V groups (= int8 k-steps of 32 channels)
+    static constexpr int KS = D / 32;
+    static constexpr int MTQ = (ROWS + 15) / 16; // QK m-tiles (16 query rows each)
+    static constexpr int NTP = ROWS / 8;         // PV n-tiles (8 query rows each)
+    static constexpr int MTP = D / 16;           // PV m-tiles (16 channels each)
+    static constexpr int SLOTS = ROWS / 8;       // query rows owned by a lane: 8k + g
+    static constexpr int KCH = D / 32;           // K 16-byte chunks per lane per page
+    static constexpr int VCH = D / 64;           // V code chunks per lane per page
+    static constexpr int SCH = D / 64;           // V scale chunks per lane per page
+    static constexpr bool HI = ROWS > 8;         // rows g+8 of a QK m-tile are real rows
+    static constexpr bool QREG = MTQ * KS * 3 * (HI ? 4 : 2) <= 48;  // q fragments in registers
+    static constexpr int PART = ROWS * D + 2 * ROWS;                 // floats of one partial
+};
+
+struct Smem {
+    size_t ring, part, stack, coef, qfrag, flags, mbar, bt, misc, heap, total;
+};
+
+template <int D, int ROWS>
+__host__ __device__ inline Smem smem_layout(int W, int R, int SD) {
+    using C = Cfg<D, ROWS>;
+    Smem s{};
+    size_t off = 0;
+    auto al = [](size_t x, size_t a) { return (x + a - 1) / a * a; };
+    s.ring = off;
+    off += (size_t)W * R * C::PB;
+    off = al(off, 16);
+    s.part = off;
+    off += (size_t)W * C::PART * 4;
+    s.heap = 0;  // the final merge reuses ring + part
+    const size_t heap_bytes = (size_t)2 * kMaxSplits * ROWS * 4 * 4;
+    if (off < heap_bytes) off = heap_bytes;
+    off = al(off, 16);
+    s.stack = off;
+    off += (size_t)SD * C::PART * 4;
+    s.coef = off;
+    off += (size_t)8 * ROWS * 2 * 4;  // up to 8 merges per phase
+    s.qfrag = off;
+    off += C::QREG ? 0 : (size_t)C::MTQ * C::KS * 3 * 32 * 16;
+    s.flags = off;
+    off += 64 * 4;
+    off = al(off, 8);
+    s.mbar = off;
+    off += (size_t)W * R * 8;
+    s.bt = off;
+    off += (size_t)W * 2 * kChunkPages * 4;
+    s.misc = off;
+    off += 64;
+    s.total = al(off, 128);
+    return s;
+}
+
+// ---- merge of two partial results (one binary-tree node) ------------------
+__device__ __forceinline__ void merge_coef(float ml, float ll, float mr, float lr, float& m, float& l, float& a,
+                                           float& b) {
+    m = fmaxf(ml, mr);
+    a = (ml == m) ? 1.0f : exp2f(__fsub_rn(ml, m));
+    b = (mr == m) ? 1.0f : exp2f(__fsub_rn(mr, m));
+    l = __fadd_rn(__fmul_rn(ll, a), __fmul_rn(lr, b));
+}
+__device__ __forceinline__ float merge_val(float ol, float orr, float a, float b) {
+    return __fadd_rn(__fmul_rn(ol, a), __fmul_rn(orr, b));
+}
+
+// dst[k] = dst[k] (+) src[k] for k < n_merges, cooperative over the CTA.  A partial
+// is O[ROWS][D] followed by m[ROWS], l[ROWS].  empty flags: an empty right side
+// leaves dst unchanged, an empty left side takes a copy of the right side.
+template <int D, int ROWS>
+__device__ void cta_merge(float* const* dst, const float* const* src, int n_merges, int* dst_empty,
+                          const int* src_empty, float* coef) {
+    const int T = blockDim.x;
+    for (int i = threadIdx.x; i < n_merges * ROWS; i += T) {
+        const int k = i / ROWS, r = i % ROWS;
+        float* d = dst[k];
+        const float* s = src[k];
+        if (src_empty[k]) continue;
+        if (dst_empty[k]) {
+            d[ROWS * D + r] = s[ROWS * D + r];
+            d[ROWS * D + ROWS + r] = s[ROWS * D + ROWS + r];
+            continue;
+        }
+        float m, l, a, b;
+        merge_coef(d[ROWS * D + r], d[ROWS * D + ROWS + r], s[ROWS * D + r], s[ROWS * D + ROWS + r], m, l, a, b);
+        coef[2 * i] = a;
+        coef[2 * i + 1] = b;
+        d[ROWS * D + r] = m;
+        d[ROWS * D + ROWS + r] = l;
+    }
+    __syncthreads();
+    constexpr int V4 = ROWS * D / 4;
+    for (int i = threadIdx.x; i < n_merges * V4; i += T) {
+        const int k = i / V4, e = i % V4, r = (4 * e) / D;
+        if (src_empty[k]) continue;
+        float4* d = reinterpret_cast<float4*>(dst[k]) + e;
+        const float4 s = reinterpret_cast<const float4*>(src[k])[e];
+        if (dst_empty[k]) {
+            *d = s;
+            continue;
+        }
+        const float a = coef[2 * (k * ROWS + r)], b = coef[2 * (k * ROWS + r) + 1];
+        float4 o = *d;
+        o.x = merge_val(o.x, s.x, a, b);
+        o.y = merge_val(o.y, s.y, a, b);
+        o.z = merge_val(o.z, s.z, a, b);
+        o.w = merge_val(o.w, s.w, a, b);
+        *d = o;
+    }
+    __syncthreads();
+    if (threadIdx.x < n_merges && !src_empty[threadIdx.x]) dst_empty[threadIdx.x] = 0;
+    __syncthreads();
+}
+
+template <typename T>
+__device__ __forceinline__ float ld_f32(const void* base, size_t i);
+template <>
+__device__ __forceinline__ float ld_f32<float>(const void* base, size_t i) {
+    return __ldg(reinterpret_cast<const float*>(base) + i);
+}
+template <>
+__device__ __forceinline__ float ld_f32<__nv_bfloat16>(const void* base, size_t i) {
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+}
+template <>
+__device__ __forceinline__ float ld_f32<__half>(const void* base, size_t i) {
+    return __half2float(reinterpret_cast<const __half*>(base)[i]);
+}
+
+__device__ __forceinline__ float load_q(const DecodeParams& p, size_t i) {
+    if (p.q_dtype == 0) return ld_f32<float>(p.q, i);
+    if (p.q_dtype == 1) return ld_f32<__nv_bfloat16>(p.q, i);
+    return ld_f32<__half>(p.q, i);
+}
+
+template <int D, int ROWS>
+__global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
+    using C = Cfg<D, ROWS>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int W = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int R = p.pages_per_stage;
+    const Smem S = smem_layout<D, ROWS>(W, R, p.stack_depth);
+    const int b = blockIdx.z, hk = blockIdx.y / p.n_rb, rb = blockIdx.y % p.n_rb, sp = blockIdx.x;
+    const unsigned FULL = 0xffffffffu;
+
+    // ---- sequence bounds (uniform per CTA) ----
+    const int L = __ldg(p.seq_lens + b), nq = __ldg(p.n_q_per_seq + b);
+    if (nq < 1 || nq > p.max_q || nq > L || (long long)L > (long long)p.max_blocks_per_seq * kPageTokens) {
+        if (sp == 0 && rb == 0 && hk == 0 && threadIdx.x == 0) atomicOr(p.err, kErrBadSeq);
+        return;
+    }
+    const int rows_b = p.group * nq, row0 = rb * ROWS;
+    if (row0 >= rows_b) return;
+    const int rows_here = min(ROWS, rows_b - row0);
+    const int n_pages = (L + kPageTokens - 1) / kPageTokens;
+    const int n_chunks = (L + kChunkTokens - 1) / kChunkTokens;
+    const int c0 = sp * p.cpc;
+    if (c0 >= n_chunks) return;
+    const int c1 = min(c0 + p.cpc, n_chunks);
+    const int n_splits = (n_chunks + p.cpc - 1) / p.cpc;
+    const int n_rounds = (c1 - c0 + W - 1) / W;
+
+    int* misc = reinterpret_cast<int*>(smem + S.misc);
+    int* flags = reinterpret_cast<int*>(smem + S.flags);   // [0..W): warp partial empty
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S.mbar) + warp * R;
+    int* bt = reinterpret_cast<int*>(smem + S.bt) + warp * 2 * kChunkPages;
+    uint8_t* ring = smem + S.ring + (size_t)warp * R * C::PB;
+    float* part = reinterpret_cast<float*>(smem + S.part);
+    float* stack = reinterpret_cast<float*>(smem + S.stack);
+    float* coef = reinterpret_cast<float*>(smem + S.coef);
+
+    // ---- query-row offset of this sequence (sum of n_q of earlier sequences) ----
+    if (warp == 0) {
+        int s = 0;
+        for (int i = lane; i < b; i += 32) s += min(max(__ldg(p.n_q_per_seq + i), 0), p.max_q);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
+        if (lane == 0) misc[0] = s;
+    }
+    if (lane == 0) {
+        for (int s = 0; s < R; s++) mbar_init(smem_u32(&bars[s]), 1);
+        mbar_fence_init();
+    }
+    if (threadIdx.x == 0) misc[1] = 0;
+    __syncthreads();
+    const int qoff = misc[0];
+
+    // ---- q -> three 8-bit limbs of a 23-bit fixed-point value per row ----------
+    // Lane (g, t) owns rows 16*mt + 8*h + g and channels [t*D/4, (t+1)*D/4).  The
+    // A fragment of mma.m16n8k32 for k-step ks holds, for row g (h = 0) and g + 8
+    // (h = 1), channels t*D/4 + 8*ks + {0..3} (regs 0/1) and + {4..7} (regs 2/3).
+    uint32_t qa[C::QREG ? C::MTQ : 1][C::QREG ? C::KS : 1][3][4];
+    float crow[C::SLOTS];
+    int lim[C::SLOTS];
+    uint32_t* qfrag_s = reinterpret_cast<uint32_t*>(smem + S.qfrag);
+    if constexpr (C::QREG) {
+#pragma unroll
+        for (int mt = 0; mt < C::MTQ; mt++)
+#pragma unroll
+            for (int ks = 0; ks < C::KS; ks++)
+#pragma unroll
+                for (int lb = 0; lb < 3; lb++)
+#pragma unroll
+                    for (int r = 0; r < 4; r++) qa[mt][ks][lb][r] = 0u;
+    }
+#pragma unroll
+    for (int k = 0; k < C::SLOTS; k++) {
+        const int mt = k >> 1, h = k & 1;
+        const int rl = 8 * k + g;  // local row
+        const int r = row0 + rl;
+        const bool real = rl < rows_here;
+        const int j = real ? r / p.group : 0, hq = real ? r % p.group : 0;
+        const long long qrow = (long long)qoff + j;
+        const bool qok = real && qrow < p.total_q;
+        if (real && !qok && t == 0) atomicOr(p.err, kErrBadRow);
+        constexpr int CH = D / 4;
+        float qv[CH];
+        float amax = 0.0f;
+        const size_t base = ((size_t)qrow * p.n_q_heads + (size_t)hk * p.group + hq) * D + (size_t)t * CH;
+#pragma unroll
+        for (int c = 0; c < CH; c++) {
+            qv[c] = qok ? load_q(p, base + c) : 0.0f;
+            amax = fmaxf(amax, fabsf(qv[c]));
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
+        int E = 0;
+        if (amax > 0.0f) frexpf(amax, &E);  // amax < 2^E
+        const bool zero_row = !(amax >= 0x1p-100f);
+        const float up = zero_row ? 0.0f : ldexpf(1.0f, 22 - E);
+        crow[k] = zero_row ? 0.0f : ldexpf(p.scale_log2, E - 22);
+        lim[k] = real ? (L - nq + j + 1) : L;
+#pragma unroll
+        for (int ks = 0; ks < C::KS; ks++) {
+            uint32_t w[3][2];
+#pragma unroll
+            for (int half = 0; half < 2; half++) {
+                uint32_t l2 = 0, l1 = 0, l0 = 0;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const int Q = (int)rintf(__fmul_rn(qv[8 * ks + 4 * half + i], up));
+                    l2 |= (uint32_t)((Q >> 16) & 0xFF) << (8 * i);
+                    l1 |= (uint32_t)((Q >> 8) & 0xFF) << (8 * i);
+                    l0 |= (uint32_t)(Q & 0xFF) << (8 * i);
+                }
+                w[0][half] = l2;
+                w[1][half] = l1;
+                w[2][half] = l0;
+            }
+#pragma unroll
+            for (int lb = 0; lb < 3; lb++) {
+                if constexpr (C::QREG) {
+                    qa[mt][ks][lb][h] = w[lb][0];
+                    qa[mt][ks][lb][2 + h] = w[lb][1];
+                } else if (warp == 0) {
+                    uint32_t* f = qfrag_s + ((((size_t)mt * C::KS + ks) * 3 + lb) * 32 + lane) * 4;
+                    f[h] = w[lb][0];
+                    f[2 + h] = w[lb][1];
+                    if constexpr (!C::HI) {
+                        f[1] = 0u;
+                        f[3] = 0u;
+                    }
+                }
+            }
+        }
+    }
+    if constexpr (!C::QREG) __syncthreads();
+
+    // ---- per-warp chunk sequence and page ring ----
+    const uint64_t policy = l2_evict_first_policy();
+    auto chunk_of = [&](int ro) { return c0 + ro * W + warp; };
+    // pages of this warp, in order: all its chunks are full except possibly the last
+    // chunk of the sequence
+    int my_pages = 0;
+    for (int ro = 0; ro < n_rounds; ro++) {
+        const int c = chunk_of(ro);
+        if (c < c1) my_pages += min(kChunkPages, n_pages - c * kChunkPages);
+    }
+    auto load_bt = [&](int ro) {
+        const int c = chunk_of(ro);
+        if (ro < n_rounds && c < c1 && lane < kChunkPages) {
+            const int lp = c * kChunkPages + lane;
+            int blk = -1;
+            if (lp < n_pages) {
+                blk = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + lp);
+                if (blk < 0 || (long long)blk >= p.n_blocks) {
+                    atomicOr(p.err, kErrBadBlock);
+                    blk = -1;
+                }
+            }
+            bt[(ro & 1) * kChunkPages + lane] = blk;
+        }
+    };
+    auto issue = [&](int k) {  // lane 0 only: page k of this warp's sequence
+        const int ro = k / kChunkPages, pi = k % kChunkPages, slot = k % R;
+        const int blk = bt[(ro & 1) * kChunkPages + pi];
+        const uint8_t* src = p.pool + ((long long)(blk < 0 ? 0 : blk) * p.n_kv_heads + hk) * C::PB;
+        mbar_arrive_expect_tx(smem_u32(&bars[slot]), C::PB);
+        tma_load_1d(smem_u32(ring + (size_t)slot * C::PB), src, C::PB, smem_u32(&bars[slot]), policy);
+    };
+    load_bt(0);
+    load_bt(1);
+    __syncwarp();
+    if (lane == 0)
+        for (int k = 0; k < R && k < my_pages; k++) issue(k);
+
+    bool aborted = false;
+    int k_abort = 0;       // first page not waited for after a timeout
+    int k_next = 0;        // next page of this warp to consume
+    int n_stack = 0;       // round-stack entries (uniform)
+    int* stack_level = misc + 4;   // levels of stack entries (up to 16)
+
+    for (int ro = 0; ro < n_rounds; ro++) {
+        const int c = chunk_of(ro);
+        const bool active = c < c1;
+        if (active) {
+            if (ro >= 1) {
+                load_bt(ro + 1);
+                __syncwarp();
+            }
+            float O[C::MTP][C::NTP][4];
+#pragma unroll
+            for (int j = 0; j < C::MTP; j++)
+#pragma unroll
+                for (int n = 0; n < C::NTP; n++)
+#pragma unroll
+                    for (int e = 0; e < 4; e++) O[j][n][e] = 0.0f;
+            float mrun[C::SLOTS], lrun[C::SLOTS];
+#pragma unroll
+            for (int k = 0; k < C::SLOTS; k++) {
+                mrun[k] = -INFINITY;
+                lrun[k] = 0.0f;
+            }
+            const int pages_here = min(kChunkPages, n_pages - c * kChunkPages);
+            for (int pi = 0; pi < pages_here; pi++, k_next++) {
+                const int slot = k_next % R;
+                const uint32_t par = (uint32_t)((k_next / R) & 1);
+                if (!aborted && !mbar_wait_bounded(smem_u32(&bars[slot]), par)) {
+                    aborted = true;
+                    k_abort = k_next;
+                    if (lane == 0) atomicOr(p.err, kErrTimeout);
+                }
+                const uint8_t* pp = ring + (size_t)slot * C::PB;
+                const int lp = c * kChunkPages + pi;
+                const bool bad = bt[(ro & 1) * kChunkPages + pi] < 0;
+
+                // ---- scores: int8 QK^T on the tensor cores ----
+                uint4 kc[C::KCH];
+#pragma unroll
+                for (int i = 0; i < C::KCH; i++) kc[i] = lds128(pp + (size_t)(i * 32 + lane) * 16);
+                const float2 skA = __half22float2(u32_as_h2(lds32(pp + k_scale_off(D) + 4 * t)));
+                const float2 skB = __half22float2(u32_as_h2(lds32(pp + k_scale_off(D) + 16 + 4 * t)));
+                const float sk[2][2] = {{skA.x, skA.y}, {skB.x, skB.y}};
+                float z[C::SLOTS][2][2];
+#pragma unroll
+                for (int mt = 0; mt < C::MTQ; mt++) {
+#pragma unroll
+                    for (int nt = 0; nt < 2; nt++) {
+                        int d21[4] = {0, 0, 0, 0}, d0[4] = {0, 0, 0, 0};
+#pragma unroll
+                        for (int lb = 0; lb < 3; lb++) {
+#pragma unroll
+                            for (int ks = 0; ks < C::KS; ks++) {
+                                const uint4 ch = kc[nt * (D / 64) + ks / 2];
+                                const uint32_t b0 = (ks & 1) ? ch.z : ch.x;
+                                const uint32_t b1 = (ks & 1) ? ch.w : ch.y;
+                                uint32_t a[4];
+                                if constexpr (C::QREG) {
+#pragma unroll
+                                    for (int r = 0; r < 4; r++) a[r] = qa[mt][ks][lb][r];
+                                } else {
+                                    const uint4 f = lds128(qfrag_s + ((((size_t)mt * C::KS + ks) * 3 + lb) * 32 + lane) * 4);
+                                    a[0] = f.x;
+                                    a[1] = f.y;
+                                    a[2] = f.z;
+                                    a[3] = f.w;
+                                }
+                                if (lb == 0) mma_s8s8(d21, a, b0, b1);
+                                else if (lb == 1) mma_u8s8(d21, a, b0, b1);
+                                else mma_u8s8(d0, a, b0, b1);
+                            }
+                            if (lb == 0) {
+#pragma unroll
+                                for (int i = 0; i < 4; i++) d21[i] <<= 8;
+                            }
+                        }
+#pragma unroll
+                        for (int h = 0; h < 2; h++) {
+                            if (16 * mt + 8 * h < ROWS) {
+                                const int k = 2 * mt + h;
+#pragma unroll
+                                for (int e = 0; e < 2; e++) {
+                                    const float s = __fmaf_rn((float)d21[2 * h + e], 256.0f, (float)d0[2 * h + e]);
+                                    z[k][nt][e] = __fmul_rn(__fmul_rn(s, crow[k]), sk[nt][e]);
+                                }
+                            }
+                        }
+                    }
+                }
+
+                // ---- online softmax (log2 units) ----
+                const int tok0 = lp * kPageTokens + 2 * t;
+                float pw[C::SLOTS][2][2], alph[C::SLOTS];
+#pragma unroll
+                for (int k = 0; k < C::SLOTS; k++) {
+                    float pm = -INFINITY;
+#pragma unroll
+                    for (int nt = 0; nt < 2; nt++)
+#pragma unroll
+                        for (int e = 0; e < 2; e++) {
+                            const bool valid = !bad && (tok0 + 8 * nt + e) < lim[k];
+                            z[k][nt][e] = valid ? z[k][nt][e] : -INFINITY;
+                            pm = fmaxf(pm, z[k][nt][e]);
+                        }
+                    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 1));
+                    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 2));
+                    const float mnew = fmaxf(mrun[k], pm);
+                    alph[k] = (mnew == mrun[k]) ? 1.0f : exp2f(__fsub_rn(mrun[k], mnew));
+#pragma unroll
+                    for (int nt = 0; nt < 2; nt++)
+#pragma unroll
+                        for (int e = 0; e < 2; e++)
+                            pw[k][nt][e] = (z[k][nt][e] == -INFINITY) ? 0.0f : exp2f(__fsub_rn(z[k][nt][e], mnew));
+                    const float ps = __fadd_rn(__fadd_rn(pw[k][0][0], pw[k][0][1]), __fadd_rn(pw[k][1][0], pw[k][1][1]));
+                    lrun[k] = __fadd_rn(__fmul_rn(lrun[k], alph[k]), ps);
+                    mrun[k] = mnew;
+                }
+#pragma unroll
+                for (int n = 0; n < C::NTP; n++) {
+                    const float a0 = __shfl_sync(FULL, alph[n], 8 * t);
+                    const float a1 = __shfl_sync(FULL, alph[n], 8 * t + 4);
+#pragma unroll
+                    for (int j = 0; j < C::MTP; j++) {
+                        O[j][n][0] = __fmul_rn(O[j][n][0], a0);
+                        O[j][n][1] = __fmul_rn(O[j][n][1], a1);
+                        O[j][n][2] = __fmul_rn(O[j][n][2], a0);
+                        O[j][n][3] = __fmul_rn(O[j][n][3], a1);
+                    }
+                }
+
+                // ---- P.V: int4 codes as exact fp16, weights p * s_v in fp16 ----
+                uint4 vcw[C::VCH], svw[C::SCH];
+#pragma unroll
+                for (int i = 0; i < C::VCH; i++) vcw[i] = lds128(pp + v_code_off(D) + (size_t)(i * 32 + lane) * 16);
+#pragma unroll
+                for (int i = 0; i < C::SCH; i++)
+                    svw[i] = lds128(pp + v_scale_off(D) + (size_t)t * C::NG * 8 + (size_t)i * 16);
+                const uint32_t* vwd = reinterpret_cast<const uint32_t*>(vcw);
+                const uint32_t* swd = reinterpret_cast<const uint32_t*>(svw);
+#pragma unroll
+                for (int q = 0; q < C::NG; q++) {
+                    const float2 s0 = __half22float2(u32_as_h2(swd[2 * q]));
+                    const float2 s1 = __half22float2(u32_as_h2(swd[2 * q + 1]));
+                    const uint32_t x0 = vwd[2 * q] ^ 0x88888888u, x1 = vwd[2 * q + 1] ^ 0x88888888u;
+                    const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
+                    const uint32_t A0 = nib_lo_to_h2(x0), A1 = nib_hi_to_h2(x0);
+                    const uint32_t A2 = nib_lo_to_h2(x1), A3 = nib_hi_to_h2(x1);
+                    const uint32_t B0 = nib_lo_to_h2(y0), B1 = nib_hi_to_h2(y0);
+                    const uint32_t B2 = nib_lo_to_h2(y1), B3 = nib_hi_to_h2(y1);
+#pragma unroll
+                    for (int n = 0; n < C::NTP; n++) {
+                        const float w00 = pw[n][0][0] == 0.0f ? 0.0f : __fmul_rn(pw[n][0][0], s0.x);
+                        const float w01 = pw[n][0][1] == 0.0f ? 0.0f : __fmul_rn(pw[n][0][1], s0.y);
+                        const float w10 = pw[n][1][0] == 0.0f ? 0.0f : __fmul_rn(pw[n][1][0], s1.x);
+                        const float w11 = pw[n][1][1] == 0.0f ? 0.0f : __fmul_rn(pw[n][1][1], s1.y);
+                        const uint32_t bb0 = pack_h2(w00, w01), bb1 = pack_h2(w10, w11);
+                        mma_f16(O[2 * q][n], A0, A1, A2, A3, bb0, bb1);
+                        mma_f16(O[2 * q + 1][n], B0, B1, B2, B3, bb0, bb1);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0 && !aborted && k_next + R < my_pages) {
+                    fence_proxy_async_smem();
+                    issue(k_next + R);
+                }
+            }
+            // ---- chunk partial -> shared memory (natural layout) ----
+            float* mine = part + (size_t)warp * C::PART;
+#pragma unroll
+            for (int k = 0; k < C::SLOTS; k++) {
+                float l = lrun[k];
+                l = __fadd_rn(l, __shfl_xor_sync(FULL, l, 1));
+                l = __fadd_rn(l, __shfl_xor_sync(FULL, l, 2));
+                if (t == 0) {
+                    mine[ROWS * D + 8 * k + g] = mrun[k];
+                    mine[ROWS * D + ROWS + 8 * k + g] = l;
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < C::NTP; n++)
+#pragma unroll
+                for (int q = 0; q < C::NG; q++) {
+                    const int ch = 32 * q + 4 * g;
+                    const int r0 = 8 * n + 2 * t;
+                    *reinterpret_cast<float4*>(mine + (size_t)r0 * D + ch) =
+                        make_float4(O[2 * q][n][0], O[2 * q][n][2], O[2 * q + 1][n][0], O[2 * q + 1][n][2]);
+                    *reinterpret_cast<float4*>(mine + (size_t)(r0 + 1) * D + ch) =
+                        make_float4(O[2 * q][n][1], O[2 * q][n][3], O[2 * q + 1][n][1], O[2 * q + 1][n][3]);
+                }
+        }
+        if (lane == 0) flags[warp] = active ? 0 : 1;
+        __syncthreads();
+
+        // ---- tree over the W chunk partials of this round -> part[0] ----
+        for (int s = 1; s < W; s <<= 1) {
+            float* dsts[8];
+            const float* srcs[8];
+            int n_m = 0;
+            for (int w = 0; w + s < W; w += 2 * s) {
+                dsts[n_m] = part + (size_t)w * C::PART;
+                srcs[n_m] = part + (size_t)(w + s) * C::PART;
+                n_m++;
+            }
+            // gather empty flags of this level into flags[16..]
+            if (threadIdx.x < n_m) {
+                flags[16 + threadIdx.x] = flags[threadIdx.x * 2 * s];
+                flags[32 + threadIdx.x] = flags[threadIdx.x * 2 * s + s];
+            }
+            __syncthreads();
+            cta_merge<D, ROWS>(dsts, srcs, n_m, flags + 16, flags + 32, coef);
+            if (threadIdx.x < n_m) flags[threadIdx.x * 2 * s] = flags[16 + threadIdx.x];
+            __syncthreads();
+        }
+        // ---- push the round result onto the round stack (binary counter) ----
+        {
+            int level = 0;
+            bool in_part = true;
+            float* cur = part;
+            while (n_stack > 0 && stack_level[n_stack - 1] == level) {
+                float* left = stack + (size_t)(n_stack - 1) * C::PART;
+                float* dsts[1] = {left};
+                const float* srcs[1] = {cur};
+                if (threadIdx.x == 0) {
+                    flags[16] = 0;
+                    flags[32] = 0;
+                }
+                __syncthreads();
+                cta_merge<D, ROWS>(dsts, srcs, 1, flags + 16, flags + 32, coef);
+                cur = left;
+                in_part = false;
+                level++;
+                n_stack--;
+            }
+            if (in_part) {
+                float* dst = stack + (size_t)n_stack * C::PART;
+                for (int i = threadIdx.x; i < C::PART / 2; i += blockDim.x)
+                    reinterpret_cast<float2*>(dst)[i] = reinterpret_cast<const float2*>(part)[i];
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) stack_level[n_stack] = level;
+            n_stack++;
+            __syncthreads();
+        }
+    }
+    // ---- fold the round stack right to left -> stack[0] ----
+    for (int i = n_stack - 2; i >= 0; i--) {
+        float* dsts[1] = {stack + (size_t)i * C::PART};
+        const float* srcs[1] = {stack + (size_t)(i + 1) * C::PART};
+        if (threadIdx.x == 0) {
+            flags[16] = 0;
+            flags[32] = 0;
+        }
+        __syncthreads();
+        cta_merge<D, ROWS>(dsts, srcs, 1, flags + 16, flags + 32, coef);
+    }
+    // any warp that gave up on a wait: drain its copies still in flight, then stop
+    if (aborted) {
+        for (int k = k_abort; k < my_pages && k < k_abort + R; k++)
+            mbar_wait_bounded(smem_u32(&bars[k % R]), (uint32_t)((k / R) & 1));
+        misc[1] = 1;
+    }
+    __syncthreads();
+    if (misc[1] == 1) return;
+
+    const float* res = stack;
+    const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
+    auto finalize = [&](const float* o_src, const float* m_src, const float* l_src) {
+        for (int i = threadIdx.x; i < rows_here * (D / 4); i += blockDim.x) {
+            const int rl = i / (D / 4), c4 = i % (D / 4);
+            const int r = row0 + rl, j = r / p.group, hq = r % p.group;
+            const long long qrow = (long long)qoff + j;
+            if (qrow >= p.total_q) continue;
+            const float l = l_src[rl];
+            float4 o = reinterpret_cast<const float4*>(o_src + (size_t)rl * D)[c4];
+            o.x = __fdiv_rn(o.x, l);
+            o.y = __fdiv_rn(o.y, l);
+            o.z = __fdiv_rn(o.z, l);
+            o.w = __fdiv_rn(o.w, l);
+            const size_t orow = (size_t)qrow * p.n_q_heads + (size_t)hk * p.group + hq;
+            reinterpret_cast<float4*>(p.out + orow * D)[c4] = o;
+            if (c4 == 0 && p.lse != nullptr)
+                p.lse[orow] = __fmul_rn(__fadd_rn(m_src[rl], log2f(l)), 0.69314718055994531f);
+        }
+    };
+
+    if (n_splits == 1) {
+        finalize(res, res + ROWS * D, res + ROWS * D + ROWS);
+        return;
+    }
+    // ---- publish this CTA's partial; the last CTA completes the tree ----
+    float* go = p.part_o + (pidx * kMaxSplits + sp) * (size_t)(ROWS * D);
+    float* gml = p.part_ml + (pidx * kMaxSplits + sp) * (size_t)(2 * ROWS);
+    for (int i = threadIdx.x; i < ROWS * D / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(go)[i] = reinterpret_cast<const float4*>(res)[i];
+    for (int i = threadIdx.x; i < 2 * ROWS; i += blockDim.x) gml[i] = res[ROWS * D + i];
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) misc[2] = (atomicAdd(p.counters + pidx, 1u) == (unsigned)(n_splits - 1)) ? 1 : 0;
+    __syncthreads();
+    if (misc[2] == 0) return;
+    __threadfence();
+
+    // Coefficients of every node of the padded tree over the n_splits CTA partials,
+    // heap-indexed (node (level, i) at 2^(H-level) + i), per row: m, l, alpha, beta.
+    int H = 0;
+    while ((1 << H) < n_splits) H++;
+    float* hp = reinterpret_cast<float*>(smem + S.heap);
+    auto hidx = [&](int level, int i) { return (1 << (H - level)) + i; };
+    const float* gml0 = p.part_ml + pidx * kMaxSplits * (size_t)(2 * ROWS);
+    const float* go0 = p.part_o + pidx * kMaxSplits * (size_t)(ROWS * D);
+    for (int i = threadIdx.x; i < n_splits * ROWS; i += blockDim.x) {
+        const int s = i / ROWS, r = i % ROWS;
+        float* nd = hp + ((size_t)hidx(0, s) * ROWS + r) * 4;
+        nd[0] = __ldcg(gml0 + (size_t)s * 2 * ROWS + r);
+        nd[1] = __ldcg(gml0 + (size_t)s * 2 * ROWS + ROWS + r);
+    }
+    __syncthreads();
+    for (int lv = 1; lv <= H; lv++) {
+        const int n_here = (n_splits + (1 << lv) - 1) >> lv;
+        for (int i = threadIdx.x; i < n_here * ROWS; i += blockDim.x) {
+            const int ni = i / ROWS, r = i % ROWS;
+            float* nd = hp + ((size_t)hidx(lv, ni) * ROWS + r) * 4;
+            const float* lf = hp + ((size_t)hidx(lv - 1, 2 * ni) * ROWS + r) * 4;
+            const bool has_right = (2 * ni + 1) * (1 << (lv - 1)) < n_splits;
+            if (has_right) {
+                const float* rt = hp + ((size_t)hidx(lv - 1, 2 * ni + 1) * ROWS + r) * 4;
+                merge_coef(lf[0], lf[1], rt[0], rt[1], nd[0], nd[1], nd[2], nd[3]);
+            } else {
+                nd[0] = lf[0];
+                nd[1] = lf[1];
+                nd[2] = 1.0f;
+                nd[3] = 0.0f;
+            }
+        }
+        __syncthreads();
+    }
+    // Elements: binary counter over the leaves, merging at the padded-tree nodes.
+    float* fin = stack;   // final O [ROWS][D], m, l (this CTA's own partial is in global memory now)
+    const float* root = hp + (size_t)hidx(H, 0) * ROWS * 4;
+    for (int e4 = threadIdx.x; e4 < ROWS * D / 4; e4 += blockDim.x) {
+        const int r = (4 * e4) / D;
+        float4 st[kMaxSplits == 64 ? 7 : 12];
+        int lvl[kMaxSplits == 64 ? 7 : 12], beg[kMaxSplits == 64 ? 7 : 12];
+        int n_st = 0;
+        for (int s = 0; s < n_splits; s++) {
+            float4 cur = __ldcg(reinterpret_cast<const float4*>(go0 + (size_t)s * ROWS * D) + e4);
+            int cl = 0, cb = s;
+            while (n_st > 0 && lvl[n_st - 1] == cl) {
+                const int a = beg[n_st - 1];
+                const float* nd = hp + ((size_t)hidx(cl + 1, a >> (cl + 1)) * ROWS + r) * 4;
+                const float4 lf = st[n_st - 1];
+                cur.x = merge_val(lf.x, cur.x, nd[2], nd[3]);
+                cur.y = merge_val(lf.y, cur.y, nd[2], nd[3]);
+                cur.z = merge_val(lf.z, cur.z, nd[2], nd[3]);
+                cur.w = merge_val(lf.w, cur.w, nd[2], nd[3]);
+                cl++;
+                cb = a;
+                n_st--;
+            }
+            st[n_st] = cur;
+            lvl[n_st] = cl;
+            beg[n_st] = cb;
+            n_st++;
+        }
+        float4 acc = st[n_st - 1];
+        for (int i = n_st - 2; i >= 0; i--) {
+            const int a = beg[i], cl = lvl[i];
+            const float* nd = hp + ((size_t)hidx(cl + 1, a >> (cl + 1)) * ROWS + r) * 4;
+            const float4 lf = st[i];
+            acc.x = merge_val(lf.x, acc.x, nd[2], nd[3]);
+            acc.y = merge_val(lf.y, acc.y, nd[2], nd[3]);
+            acc.z = merge_val(lf.z, acc.z, nd[2], nd[3]);
+            acc.w = merge_val(lf.w, acc.w, nd[2], nd[3]);
+        }
+        reinterpret_cast<float4*>(fin)[e4] = acc;
+    }
+    float* fml = fin + ROWS * D;
+    for (int r = threadIdx.x; r < ROWS; r += blockDim.x) {
+        fml[r] = root[r * 4 + 0];
+        fml[ROWS + r] = root[r * 4 + 1];
+    }
+    __syncthreads();
+    finalize(fin, fml, fml + ROWS);
+    if (threadIdx.x == 0) p.counters[pidx] = 0u;
+}
+
+size_t decode_smem_bytes(int head_dim, int rows, int warps, int pages_per_stage, int stack_depth) {
+#define MQ_SMEM(DD, RR) \
+    if (head_dim == DD && rows == RR) return smem_layout<DD, RR>(warps, pages_per_stage, stack_depth).total;
+    MQ_SMEM(128, 8) MQ_SMEM(128, 16) MQ_SMEM(128, 32) MQ_SMEM(256, 8) MQ_SMEM(256, 16)
+#undef MQ_SMEM
+    return 0;
+}
+
+template <int D, int ROWS>
+static cudaError_t set_smem(size_t smem) {
+    return cudaFuncSetAttribute(decode_kernel<D, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}
+
+cudaError_t decode_prepare(int head_dim, int rows, size_t smem) {
+    if (head_dim == 128 && rows == 8) return set_smem<128, 8>(smem);
+    if (head_dim == 128 && rows == 16) return set_smem<128, 16>(smem);
+    if (head_dim == 128 && rows == 32) return set_smem<128, 32>(smem);
+    if (head_dim == 256 && rows == 8) return set_smem<256, 8>(smem);
+    if (head_dim == 256 && rows == 16) return set_smem<256, 16>(smem);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int warps, int max_splits, size_t smem,
+                          cudaStream_t st) {
+    const dim3 grid((unsigned)max_splits, (unsigned)(p.n_kv_heads * p.n_rb), (unsigned)p.n_seqs);
+    const dim3 block((unsigned)(warps * 32));
+#define MQ_LAUNCH(DD, RR) \
+    if (head_dim == DD && rows == RR) decode_kernel<DD, RR><<<grid, block, smem, st>>>(p); else
+    MQ_LAUNCH(128, 8) MQ_LAUNCH(128, 16) MQ_LAUNCH(128, 32) MQ_LAUNCH(256, 8) MQ_LAUNCH(256, 16)
+    return cudaErrorInvalidValue;
+#undef MQ_LAUNCH
+    return cudaGetLastError();
+}
+
+}  // namespace mq

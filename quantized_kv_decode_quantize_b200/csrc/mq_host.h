@@ -1,0 +1,49 @@
+// Host-side internals shared by the C-ABI layer and the tuner.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/mq.h"
+
+struct mq_cache {
+    int n_kv_heads;
+    int head_dim;
+    int64_t n_blocks;
+    void* pool;
+    size_t pool_bytes;
+    int device;
+    int n_sm;
+    int max_smem;
+    unsigned* err_word;         // device address of this device's error word
+    mq_decode_config cfg[3];    // per rows class
+};
+
+namespace mq {
+
+struct DecodePlan {
+    int cls, rows, n_rb, warps, pages_per_stage, cpc, max_splits, stack_depth;
+    size_t smem;
+};
+
+// Switches to `dev` for the lifetime of the guard when it is not current.
+struct DevGuard {
+    int prev = -1;
+    bool switched = false;
+    explicit DevGuard(int dev);
+    ~DevGuard();
+};
+
+int rows_class_rows(int head_dim, int cls);
+int rows_class_for(int head_dim, int rows_total);
+mq_decode_config default_config(int head_dim, int cls);
+bool config_valid(const mq_decode_config& c);
+DecodePlan plan_decode(const mq_cache* c, int n_seqs, int n_q_heads, int max_q, int max_seq_len);
+size_t workspace_bytes_for(const mq_cache* c, int n_seqs, int n_rb, int rows);
+cudaError_t ensure_decode_smem(int device, int head_dim, int rows, size_t smem);
+mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void* q, mq_dtype q_dtype, int n_seqs,
+                             int n_q_heads, int total_q, int max_q, const int32_t* block_table, int max_blocks,
+                             const int32_t* seq_lens, const int32_t* n_q_per_seq, float softmax_scale, float* out,
+                             float* lse, void* workspace, cudaStream_t st);
+
+}  // namespace mq

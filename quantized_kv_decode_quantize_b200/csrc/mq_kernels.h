@@ -1,0 +1,71 @@
+// Internal launch interface between the C-ABI layer (mq_api.cu) and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace mq {
+
+struct AppendParams {
+    uint8_t* pool;
+    int n_kv_heads;
+    long long n_blocks;
+    const void* k;
+    const void* v;
+    int dtype;  // 0 f32, 1 bf16, 2 f16
+    int n_seqs;
+    int n_tokens;
+    const int32_t* cu_new;
+    const int32_t* start_pos;
+    const int32_t* block_table;
+    int max_blocks_per_seq;
+    unsigned* err;
+};
+
+cudaError_t launch_append(const AppendParams& p, int head_dim, cudaStream_t st);
+
+struct DecodeParams {
+    const uint8_t* pool;
+    int n_kv_heads;
+    long long n_blocks;
+    const void* q;
+    int q_dtype;  // 0 f32, 1 bf16, 2 f16
+    int n_q_heads;
+    int group;    // n_q_heads / n_kv_heads
+    int total_q;
+    int max_q;
+    int n_seqs;
+    const int32_t* block_table;
+    int max_blocks_per_seq;
+    const int32_t* seq_lens;
+    const int32_t* n_q_per_seq;
+    float scale_log2;  // softmax_scale * log2(e)
+    float* out;
+    float* lse;
+    // workspace
+    unsigned* counters;  // [n_seqs][n_kv_heads][n_rb]
+    float* part_ml;      // [n_seqs][n_kv_heads][n_rb][kMaxSplits][rows][2]
+    float* part_o;       // [n_seqs][n_kv_heads][n_rb][kMaxSplits][rows][D]
+    int n_rb;            // row blocks per kv-head
+    int cpc;             // chunks per CTA (power of two >= warps)
+    int pages_per_stage; // TMA ring depth per warp
+    int stack_depth;     // round-stack entries in shared memory
+    unsigned* err;
+};
+
+// rows: 8, 16 or 32 (padded query rows per kv-head handled by one CTA)
+size_t decode_smem_bytes(int head_dim, int rows, int warps, int pages_per_stage, int stack_depth);
+cudaError_t decode_prepare(int head_dim, int rows, size_t smem);  // raises the dynamic smem limit
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int warps, int max_splits, size_t smem,
+                          cudaStream_t st);
+
+// Fills n values of dtype with a deterministic pseudo-random pattern (uniform in
+// [-2, 2), channels 0..3 of every head_dim vector scaled by 10).  Used by the tuner
+// to build probe caches; not part of any computed result.
+cudaError_t launch_fill_random(void* dst, int dtype, long long n, int head_dim, unsigned long long seed,
+                               cudaStream_t st);
+// Writes a buffer (L2 flush between timed launches).
+cudaError_t launch_scribble(void* dst, size_t bytes, unsigned v, cudaStream_t st);
+// out[0] = 1 if a[i] != b[i] for some i < n32 (32-bit words), else unchanged.
+cudaError_t launch_compare(const uint32_t* a, const uint32_t* b, long long n32, unsigned* out, cudaStream_t st);
+
+}  // namespace mq

@@ -1,0 +1,359 @@
+// mq_tune: on-device choice of the decode launch configuration.
+//
+// Follows the first-load tuner of the blog.123qwe.co.kr deep dive on
+// magnitudedev/magnitude, section 3 ("core mechanism 1: the 60 s first-load
+// tuner"): one wall-clock budget covers everything (probe set-up, every launch,
+// every comparison); candidates are measured on the device over serving shapes
+// (decode at 4k and 64k history, the verification width), and the cost of a
+// configuration c is
+//     cost(c) = sum_p weight(p) * median_time(c, p),  weight(p) = 1 / median_time(default, p)
+// (each probe is one launch of its term); timing passes read data sized beyond the
+// last-level cache (here: rotating probe caches that together exceed twice the L2
+// size), so no launch finds its data warm; structurally different candidates are
+// tried before refinements of one; a candidate is started only when the budget
+// left covers its estimated cost.  Admission follows the paper-digest.app summary
+// ("Core Mechanics": only configurations that do not change the output are
+// kept): a candidate's out and lse bytes must equal the default's exactly.
+#include <algorithm>
+#include <chrono>
+#include <cstdio>
+#include <string>
+#include <vector>
+
+#include "../../include/mq.h"
+#include "mq_device.cuh"
+#include "mq_host.h"
+#include "mq_kernels.h"
+
+namespace mq {
+namespace {
+
+using Clock = std::chrono::steady_clock;
+
+struct Probe {
+    const char* name;
+    int seq_len, n_q, cls;
+    double t_default = 0;   // median seconds at the default configuration
+};
+
+struct Cand {
+    mq_decode_config cfg;
+    int cls;
+    double t[3] = {0, 0, 0};
+    bool identical = true, measured = false, rejected = false, valid = true;
+};
+
+double seconds_since(Clock::time_point t0) {
+    return std::chrono::duration<double>(Clock::now() - t0).count();
+}
+
+struct Buffers {
+    void* pool = nullptr;
+    int32_t* bt = nullptr;       // [n_copies][blocks_per_copy]
+    int32_t* lens = nullptr;     // one per probe
+    int32_t* nq = nullptr;
+    int32_t* cu = nullptr;
+    int32_t* start = nullptr;
+    void* kv = nullptr;          // staging for K and V
+    void* q = nullptr;
+    float* out_ref[3] = {nullptr, nullptr, nullptr};
+    float* lse_ref[3] = {nullptr, nullptr, nullptr};
+    float* out = nullptr;
+    float* lse = nullptr;
+    void* ws = nullptr;
+    unsigned* flag = nullptr;
+    cudaEvent_t ev[2] = {nullptr, nullptr};
+    cudaStream_t st = nullptr;
+    ~Buffers() {
+        void* ptrs[] = {pool, bt, lens, nq, cu, start, kv, q, out, lse, ws, flag,
+                        out_ref[0], out_ref[1], out_ref[2], lse_ref[0], lse_ref[1], lse_ref[2]};
+        for (void* p : ptrs)
+            if (p) cudaFree(p);
+        for (auto e : ev)
+            if (e) cudaEventDestroy(e);
+        if (st) cudaStreamDestroy(st);
+    }
+};
+
+}  // namespace
+}  // namespace mq
+
+using namespace mq;
+
+extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune_result* res) {
+    const auto t0 = Clock::now();
+    if (cache == nullptr || prm == nullptr || res == nullptr) return MQ_ERR_INVALID_ARG;
+    if (!(prm->budget_s >= 0.0) || prm->n_q_heads < 1 || prm->n_q_heads % cache->n_kv_heads != 0)
+        return MQ_ERR_INVALID_ARG;
+    const int Hkv = cache->n_kv_heads, D = cache->head_dim, Hq = prm->n_q_heads, G = Hq / Hkv;
+    if (G > 64) return MQ_ERR_UNSUPPORTED;
+    *res = mq_tune_result{};
+    for (int k = 0; k < 3; k++) res->chosen[k] = cache->cfg[k];
+    res->cost = 1.0;
+    if (prm->budget_s < 0.5) {   // not even the probe set-up fits: keep the defaults
+        res->elapsed_s = seconds_since(t0);
+        return MQ_TUNE_BUDGET_EXHAUSTED;
+    }
+    DevGuard guard(cache->device);
+
+    std::vector<Probe> probes = {{"decode_4k", 4096, 1, rows_class_for(D, G)},
+                                 {"decode_64k", 65536, 1, rows_class_for(D, G)}};
+    if (G * 8 <= 64) probes.push_back({"verify8_64k", 65544, 8, rows_class_for(D, G * 8)});
+    const int P = (int)probes.size();
+
+    // ---- probe caches: enough rotating copies to exceed 2x L2 ----
+    int l2 = 0;
+    cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, cache->device);
+    const int max_len = 65544;
+    const int blocks_per_copy = (max_len + MQ_PAGE_TOKENS - 1) / MQ_PAGE_TOKENS;
+    const size_t copy_bytes = (size_t)blocks_per_copy * Hkv * page_bytes(D);
+    int n_copies = (int)std::min<size_t>(64, std::max<size_t>(2, (size_t)(2.0 * l2 / copy_bytes) + 1));
+    Buffers B;
+    auto ck = [](cudaError_t e) { return e == cudaSuccess; };
+    if (!ck(cudaStreamCreateWithFlags(&B.st, cudaStreamNonBlocking)) || !ck(cudaEventCreate(&B.ev[0])) ||
+        !ck(cudaEventCreate(&B.ev[1])))
+        return MQ_ERR_CUDA;
+    size_t ws_bytes = 0;
+    for (auto& pr : probes) {
+        const int rows_total = G * pr.n_q;
+        const int rows = rows_class_rows(D, rows_class_for(D, rows_total));
+        ws_bytes = std::max(ws_bytes, workspace_bytes_for(cache, 1, (rows_total + rows - 1) / rows, rows));
+    }
+    const size_t kv_elems = (size_t)max_len * Hkv * D;
+    if (!ck(cudaMalloc(&B.pool, copy_bytes * n_copies)) ||
+        !ck(cudaMalloc(&B.bt, sizeof(int32_t) * blocks_per_copy * n_copies)) ||
+        !ck(cudaMalloc(&B.lens, sizeof(int32_t) * 4)) || !ck(cudaMalloc(&B.nq, sizeof(int32_t) * 4)) ||
+        !ck(cudaMalloc(&B.cu, sizeof(int32_t) * 2)) || !ck(cudaMalloc(&B.start, sizeof(int32_t))) ||
+        !ck(cudaMalloc(&B.kv, kv_elems * 2 * 2)) || !ck(cudaMalloc(&B.q, (size_t)8 * Hq * D * 2)) ||
+        !ck(cudaMalloc(&B.out, (size_t)8 * Hq * D * 4)) || !ck(cudaMalloc(&B.lse, (size_t)8 * Hq * 4)) ||
+        !ck(cudaMalloc(&B.ws, ws_bytes)) || !ck(cudaMalloc(&B.flag, sizeof(unsigned))))
+        return MQ_ERR_CUDA;
+    for (int p = 0; p < P; p++)
+        if (!ck(cudaMalloc(&B.out_ref[p], (size_t)8 * Hq * D * 4)) || !ck(cudaMalloc(&B.lse_ref[p], (size_t)8 * Hq * 4)))
+            return MQ_ERR_CUDA;
+    if (!ck(cudaMemsetAsync(B.ws, 0, ws_bytes, B.st))) return MQ_ERR_CUDA;
+    {
+        std::vector<int32_t> bt((size_t)blocks_per_copy * n_copies);
+        for (size_t i = 0; i < bt.size(); i++) bt[i] = (int32_t)i;
+        int32_t h[6] = {0, max_len, 0, 0, 0, 0};
+        if (!ck(cudaMemcpy(B.bt, bt.data(), sizeof(int32_t) * bt.size(), cudaMemcpyHostToDevice)) ||
+            !ck(cudaMemcpy(B.cu, h, sizeof(int32_t) * 2, cudaMemcpyHostToDevice)) ||
+            !ck(cudaMemcpy(B.start, h + 2, sizeof(int32_t), cudaMemcpyHostToDevice)))
+            return MQ_ERR_CUDA;
+        int32_t lens[4], nq[4];
+        for (int p = 0; p < P; p++) {
+            lens[p] = probes[p].seq_len;
+            nq[p] = probes[p].n_q;
+        }
+        if (!ck(cudaMemcpy(B.lens, lens, sizeof(int32_t) * P, cudaMemcpyHostToDevice)) ||
+            !ck(cudaMemcpy(B.nq, nq, sizeof(int32_t) * P, cudaMemcpyHostToDevice)))
+            return MQ_ERR_CUDA;
+    }
+    // random K/V for one copy, quantized by the append kernel, then replicated
+    mq_cache probe_cache = *cache;
+    probe_cache.pool = B.pool;
+    probe_cache.pool_bytes = copy_bytes * n_copies;
+    probe_cache.n_blocks = (int64_t)blocks_per_copy * n_copies;
+    {
+        void* kbuf = B.kv;
+        void* vbuf = static_cast<uint8_t*>(B.kv) + kv_elems * 2;
+        if (!ck(launch_fill_random(kbuf, 1, (long long)kv_elems, D, 0x6B65ull, B.st)) ||
+            !ck(launch_fill_random(vbuf, 1, (long long)kv_elems, D, 0x7631ull, B.st)) ||
+            !ck(launch_fill_random(B.q, 1, (long long)8 * Hq * D, D, 0x7131ull, B.st)))
+            return MQ_ERR_CUDA;
+        AppendParams ap{};
+        ap.pool = static_cast<uint8_t*>(B.pool);
+        ap.n_kv_heads = Hkv;
+        ap.n_blocks = probe_cache.n_blocks;
+        ap.k = kbuf;
+        ap.v = vbuf;
+        ap.dtype = 1;
+        ap.n_seqs = 1;
+        ap.n_tokens = max_len;
+        ap.cu_new = B.cu;
+        ap.start_pos = B.start;
+        ap.block_table = B.bt;
+        ap.max_blocks_per_seq = blocks_per_copy;
+        ap.err = cache->err_word;
+        if (!ck(launch_append(ap, D, B.st))) return MQ_ERR_CUDA;
+        for (int i = 1; i < n_copies; i++)
+            if (!ck(cudaMemcpyAsync(static_cast<uint8_t*>(B.pool) + copy_bytes * i, B.pool, copy_bytes,
+                                    cudaMemcpyDeviceToDevice, B.st)))
+                return MQ_ERR_CUDA;
+        if (!ck(cudaStreamSynchronize(B.st))) return MQ_ERR_CUDA;
+    }
+
+    int rot = 0;
+    // one launch of probe p with configuration cfg on copy `rot`; returns status
+    auto launch = [&](int p, const mq_decode_config& cfg, float* out, float* lse) -> mq_status {
+        mq_cache pc = probe_cache;
+        pc.cfg[probes[p].cls] = cfg;
+        const DecodePlan pl = plan_decode(&pc, 1, Hq, probes[p].n_q, probes[p].seq_len);
+        const int32_t* bt = B.bt + (size_t)(rot % n_copies) * blocks_per_copy;
+        rot++;
+        return launch_decode_plan(&pc, pl, B.q, MQ_BF16, 1, Hq, probes[p].n_q, probes[p].n_q, bt, blocks_per_copy,
+                                  B.lens + p, B.nq + p, 1.0f / std::sqrt((float)D), out, lse, B.ws, B.st);
+    };
+    const int reps = 7;
+    // median device time of `reps` launches (events around each launch)
+    auto time_probe = [&](int p, const mq_decode_config& cfg, double* out_t) -> mq_status {
+        std::vector<float> ts;
+        for (int r = 0; r < reps; r++) {
+            cudaEventRecord(B.ev[0], B.st);
+            mq_status s = launch(p, cfg, B.out, B.lse);
+            if (s != MQ_OK) return s;
+            cudaEventRecord(B.ev[1], B.st);
+            if (!ck(cudaEventSynchronize(B.ev[1]))) return MQ_ERR_CUDA;
+            float ms = 0;
+            cudaEventElapsedTime(&ms, B.ev[0], B.ev[1]);
+            ts.push_back(ms);
+        }
+        std::sort(ts.begin(), ts.end());
+        *out_t = ts[ts.size() / 2] * 1e-3;
+        return MQ_OK;
+    };
+
+    // ---- defaults: reference outputs and times ----
+    for (int p = 0; p < P; p++) {
+        mq_status s = launch(p, cache->cfg[probes[p].cls], B.out_ref[p], B.lse_ref[p]);
+        if (s != MQ_OK) return s;
+        if ((s = time_probe(p, cache->cfg[probes[p].cls], &probes[p].t_default)) != MQ_OK) return s;
+    }
+    if (!ck(cudaStreamSynchronize(B.st))) return MQ_ERR_CUDA;
+    if (seconds_since(t0) > prm->budget_s) {
+        res->elapsed_s = seconds_since(t0);
+        return MQ_TUNE_BUDGET_EXHAUSTED;
+    }
+
+    // ---- candidates: structure (warps, ctas_per_sm) first, then ring depth ----
+    std::vector<Cand> cands;
+    bool class_used[3] = {false, false, false};
+    for (auto& pr : probes) class_used[pr.cls] = true;
+    const int Rs[3] = {2, 3, 4};
+    for (int ri = 0; ri < 3; ri++)
+        for (int w : {8, 4})
+            for (int cps : {1, 2, 4})
+                for (int cls = 0; cls < 3; cls++) {
+                    if (!class_used[cls]) continue;
+                    Cand cd;
+                    cd.cfg = mq_decode_config{w, Rs[ri], cps};
+                    cd.cls = cls;
+                    const mq_decode_config& d = cache->cfg[cls];
+                    if (cd.cfg.warps_per_cta == d.warps_per_cta && cd.cfg.pages_per_stage == d.pages_per_stage &&
+                        cd.cfg.ctas_per_sm == d.ctas_per_sm)
+                        continue;
+                    cands.push_back(cd);
+                }
+    bool exhausted = false;
+    for (auto& cd : cands) {
+        double est = 0;
+        for (int p = 0; p < P; p++)
+            if (probes[p].cls == cd.cls) est += probes[p].t_default * (reps + 2) * 2 + 2e-3;
+        if (seconds_since(t0) + est > prm->budget_s) {
+            exhausted = true;
+            res->n_skipped++;
+            continue;
+        }
+        mq_cache pc = probe_cache;
+        pc.cfg[cd.cls] = cd.cfg;
+        bool ok = true;
+        for (int p = 0; p < P && ok; p++) {
+            if (probes[p].cls != cd.cls) continue;
+            const DecodePlan pl = plan_decode(&pc, 1, Hq, probes[p].n_q, probes[p].seq_len);
+            if (pl.smem == 0 || pl.smem > (size_t)cache->max_smem) {
+                cd.valid = false;
+                ok = false;
+                break;
+            }
+            // admission: bit-identical out and lse
+            if (launch(p, cd.cfg, B.out, B.lse) != MQ_OK) return MQ_ERR_CUDA;
+            if (!ck(cudaMemsetAsync(B.flag, 0, sizeof(unsigned), B.st))) return MQ_ERR_CUDA;
+            const long long n_out = (long long)probes[p].n_q * Hq * D, n_lse = (long long)probes[p].n_q * Hq;
+            if (!ck(launch_compare(reinterpret_cast<const uint32_t*>(B.out), reinterpret_cast<const uint32_t*>(B.out_ref[p]),
+                                   n_out, B.flag, B.st)) ||
+                !ck(launch_compare(reinterpret_cast<const uint32_t*>(B.lse), reinterpret_cast<const uint32_t*>(B.lse_ref[p]),
+                                   n_lse, B.flag, B.st)))
+                return MQ_ERR_CUDA;
+            unsigned differ = 0;
+            if (!ck(cudaMemcpyAsync(&differ, B.flag, sizeof differ, cudaMemcpyDeviceToHost, B.st)) ||
+                !ck(cudaStreamSynchronize(B.st)))
+                return MQ_ERR_CUDA;
+            if (differ) {
+                cd.identical = false;
+                cd.rejected = true;
+                res->n_rejected++;
+                ok = false;
+                break;
+            }
+            if (time_probe(p, cd.cfg, &cd.t[p]) != MQ_OK) return MQ_ERR_CUDA;
+        }
+        if (cd.valid) {
+            cd.measured = true;
+            res->n_tried++;
+        }
+    }
+
+    // ---- choose per rows class ----
+    double total = 0;
+    int n_terms = 0;
+    for (int cls = 0; cls < 3; cls++) {
+        if (!class_used[cls]) continue;
+        double best = 0;
+        int terms = 0;
+        for (int p = 0; p < P; p++)
+            if (probes[p].cls == cls) {
+                best += 1.0;
+                terms++;
+            }
+        mq_decode_config pick = cache->cfg[cls];
+        for (auto& cd : cands) {
+            if (cd.cls != cls || !cd.measured || cd.rejected || !cd.valid) continue;
+            double cost = 0;
+            for (int p = 0; p < P; p++)
+                if (probes[p].cls == cls) cost += cd.t[p] / probes[p].t_default;
+            if (cost < best) {
+                best = cost;
+                pick = cd.cfg;
+            }
+        }
+        res->chosen[cls] = pick;
+        cache->cfg[cls] = pick;
+        total += best;
+        n_terms += terms;
+    }
+    res->cost = n_terms ? total / n_terms : 1.0;
+    res->elapsed_s = seconds_since(t0);
+
+    if (prm->log_path != nullptr) {
+        FILE* f = std::fopen(prm->log_path, "w");
+        if (f != nullptr) {
+            std::fprintf(f, "{\n  \"budget_s\": %.3f, \"elapsed_s\": %.3f, \"n_copies\": %d, \"l2_bytes\": %d,\n",
+                         prm->budget_s, res->elapsed_s, n_copies, l2);
+            std::fprintf(f, "  \"probes\": [");
+            for (int p = 0; p < P; p++)
+                std::fprintf(f, "%s{\"name\": \"%s\", \"seq_len\": %d, \"n_q\": %d, \"rows_class\": %d, \"default_us\": %.3f}",
+                             p ? ", " : "", probes[p].name, probes[p].seq_len, probes[p].n_q, probes[p].cls,
+                             probes[p].t_default * 1e6);
+            std::fprintf(f, "],\n  \"candidates\": [\n");
+            for (size_t i = 0; i < cands.size(); i++) {
+                const Cand& cd = cands[i];
+                std::fprintf(f,
+                             "    {\"rows_class\": %d, \"warps_per_cta\": %d, \"pages_per_stage\": %d, \"ctas_per_sm\": %d, "
+                             "\"measured\": %s, \"valid\": %s, \"bit_identical\": %s, \"times_us\": [%.3f, %.3f, %.3f]}%s\n",
+                             cd.cls, cd.cfg.warps_per_cta, cd.cfg.pages_per_stage, cd.cfg.ctas_per_sm,
+                             cd.measured ? "true" : "false", cd.valid ? "true" : "false",
+                             cd.identical ? "true" : "false", cd.t[0] * 1e6, cd.t[1] * 1e6, cd.t[2] * 1e6,
+                             i + 1 < cands.size() ? "," : "");
+            }
+            std::fprintf(f, "  ],\n  \"chosen\": [");
+            for (int cls = 0; cls < 3; cls++)
+                std::fprintf(f, "%s{\"rows_class\": %d, \"warps_per_cta\": %d, \"pages_per_stage\": %d, \"ctas_per_sm\": %d}",
+                             cls ? ", " : "", cls, res->chosen[cls].warps_per_cta, res->chosen[cls].pages_per_stage,
+                             res->chosen[cls].ctas_per_sm);
+            std::fprintf(f, "],\n  \"cost\": %.4f, \"n_tried\": %d, \"n_rejected\": %d, \"n_skipped\": %d\n}\n", res->cost,
+                         res->n_tried, res->n_rejected, res->n_skipped);
+            std::fclose(f);
+        }
+    }
+    return exhausted ? MQ_TUNE_BUDGET_EXHAUSTED : MQ_OK;
+}

@@ -1,0 +1,174 @@
+"""mq_decode_attn (CUDA) against the CPU oracle's fp64 attention over the same
+quantized cache: every output within max-abs 1e-3 (and lse within 1e-3)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_kv_decode_quantize_b200 as mq
+from quantized_kv_decode_quantize_b200 import workloads as wl
+from tests.gpu_harness import GpuCase, oracle_outputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3          # max-abs on out (the stated tolerance)
+TOL_LSE = 1e-3
+
+
+def _check(case, seqs=None):
+    out, lse = case.decode()
+    assert case.status() == mq.MQ_OK
+    eo, el = oracle_outputs(case.w, case.inp, seqs=seqs)
+    o, l = out.cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+    mask = ~np.isnan(el)
+    err = np.max(np.abs(o[mask] - eo[mask])) if mask.any() else 0.0
+    lerr = np.max(np.abs(l[mask] - el[mask])) if mask.any() else 0.0
+    assert np.all(np.isfinite(o[mask]))
+    assert err <= TOL, f"max-abs error {err:.3e}"
+    assert lerr <= TOL_LSE, f"lse error {lerr:.3e}"
+    return err
+
+
+@pytest.mark.parametrize("name", ["tiny", "long", "prefix", "verify", "mixed"])
+def test_decode_reduced_workloads(name):
+    _check(GpuCase(wl.reduced(name)))
+
+
+@pytest.mark.parametrize("name", ["tiny", "long", "prefix", "verify", "mixed"])
+def test_decode_full_size_workloads(name):
+    """Full sizes (64K history etc.), default launch configuration, every output row
+    compared (the C oracle with OpenMP computes them all)."""
+    _check(GpuCase(wl.FULL[name]()))
+
+
+@pytest.mark.parametrize("L", [1, 2, 15, 16, 17, 127, 128, 129, 255, 1025])
+def test_decode_lengths(L):
+    w = wl.long_decode(L=L)
+    _check(GpuCase(w))
+
+
+def test_single_token_cache_returns_its_value():
+    """L = 1: the weight is exactly 1, so out equals the dequantized v_0 exactly."""
+    w = wl.long_decode(L=1)
+    case = GpuCase(w)
+    out, _ = case.decode()
+    vp, vs = oracle.quantize_v(case.inp.seq_v(0).float().numpy())
+    v0 = oracle.dequantize_v(vp, vs)[0]                     # [Hkv, D]
+    G = w.n_q_heads // w.n_kv_heads
+    exp = np.repeat(v0, G, axis=0)
+    assert np.array_equal(out.cpu().numpy()[0].astype(np.float64), exp)
+
+
+@pytest.mark.parametrize("Hq,Hkv,n,D", [(8, 8, 1, 128), (16, 2, 1, 128), (4, 2, 8, 128), (32, 8, 8, 128),
+                                         (64, 8, 8, 128), (16, 4, 8, 256), (8, 4, 3, 256), (12, 4, 5, 128)])
+def test_decode_gqa_and_draft_shapes(Hq, Hkv, n, D):
+    """Every row class (8, 16, 32 rows per kv-head) and several row blocks."""
+    w = wl.Workload("shape", Hq, Hkv, D, [700, 1300], [n, max(1, n - 1)], [n, max(1, n - 1)])
+    _check(GpuCase(w))
+
+
+def test_drafts_equal_cache_length():
+    """n_q = L: the first draft sees one token."""
+    w = wl.Workload("all_drafts", 32, 8, 128, [8, 3], [8, 3], [8, 3])
+    _check(GpuCase(w))
+
+
+def test_f16_queries():
+    w = wl.reduced("long")
+    inp = wl.make_inputs(w)
+    case = GpuCase(w, inp)
+    q16 = inp.q.to(torch.float16)
+    mq.mq_decode_attn(case.cache.handle, q16.cuda(), mq.MQ_F16, w.n_seqs, w.n_q_heads, w.total_q, w.max_q,
+                      w.max_seq_len, case.tabs[0], w.max_blocks(), case.seq_lens, case.n_q,
+                      1 / math.sqrt(w.head_dim), case.out, case.lse, case.ws, case.ws.numel())
+    inp.q = q16
+    eo, _ = oracle_outputs(w, inp)
+    assert np.max(np.abs(case.out.cpu().numpy() - eo)) <= TOL
+
+
+def test_ragged_grid_and_null_lse():
+    """max_seq_len far above the actual lengths (empty CTAs exit), lse = NULL."""
+    w = wl.reduced("mixed")
+    case = GpuCase(w)
+    mq.mq_decode_attn(case.cache.handle, case.q, mq.MQ_BF16, w.n_seqs, w.n_q_heads, w.total_q, w.max_q,
+                      w.max_seq_len, case.tabs[0], w.max_blocks(), case.seq_lens, case.n_q,
+                      1 / math.sqrt(w.head_dim), case.out, None, case.ws, case.ws.numel())
+    assert case.status() == mq.MQ_OK
+    eo, _ = oracle_outputs(w, case.inp)
+    assert np.max(np.abs(case.out.cpu().numpy() - eo)) <= TOL
+
+
+def test_shared_prefix_equals_private_copies():
+    """Sessions that alias the same physical prefix blocks get bit-identical outputs
+    to the same sessions holding private copies of the prefix."""
+    w = wl.reduced("prefix")
+    inp = wl.make_inputs(w)
+    shared = GpuCase(w, inp)
+    o1 = shared.decode()[0].clone()
+    wp = wl.Workload("private", w.n_q_heads, w.n_kv_heads, w.head_dim, list(w.seq_lens), list(w.n_q),
+                     list(w.n_append), shared_prefix=0)
+    inp2 = wl.Inputs(None, None, [inp.seq_k(b) for b in range(w.n_seqs)], [inp.seq_v(b) for b in range(w.n_seqs)],
+                     inp.q)
+    private = GpuCase(wp, inp2)
+    o2 = private.decode()[0]
+    assert torch.equal(o1, o2)
+
+
+CONFIGS = [(w, r, c) for w in (4, 8) for r in (2, 3, 4) for c in (1, 2, 4)]
+
+
+@pytest.mark.parametrize("name", ["long", "verify", "mixed"])
+def test_launch_configs_bit_identical(name):
+    """Every launch configuration the tuner may pick gives the same bytes."""
+    w = wl.reduced(name)
+    if name == "long":
+        w = wl.long_decode(L=20000)
+    case = GpuCase(w)
+    ref = [t.clone() for t in case.decode()]
+    cls = {8: 0, 16: 1, 32: 2}
+    for cfg in CONFIGS:
+        for k in range(3):
+            mq.mq_set_decode_config(case.cache.handle, k, *cfg)
+        out, lse = case.decode()
+        assert case.status() == mq.MQ_OK
+        assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1]), cfg
+
+
+def test_repeated_calls_reuse_workspace():
+    """The counter region returns to zero: many calls on one workspace agree."""
+    case = GpuCase(wl.reduced("verify"))
+    ref = case.decode()[0].clone()
+    for _ in range(20):
+        assert torch.equal(case.decode()[0], ref)
+    assert int(case.ws[:64].count_nonzero()) == 0
+
+
+def test_bad_sequence_is_flagged_not_faulted():
+    w = wl.reduced("long")
+    case = GpuCase(w)
+    bad_len = torch.tensor([w.max_blocks() * 16 + 5], dtype=torch.int32, device="cuda")
+    mq.mq_decode_attn(case.cache.handle, case.q, mq.MQ_BF16, 1, w.n_q_heads, 1, 1, w.max_seq_len, case.tabs[0],
+                      w.max_blocks(), bad_len, case.n_q, 0.1, case.out, case.lse, case.ws, case.ws.numel())
+    assert case.status() == mq.MQ_ERR_DEVICE
+    bad_tab = case.tabs[0].clone()
+    bad_tab[0, 3] = 10 ** 8
+    case.ws.zero_()
+    mq.mq_decode_attn(case.cache.handle, case.q, mq.MQ_BF16, 1, w.n_q_heads, 1, 1, w.max_seq_len, bad_tab,
+                      w.max_blocks(), case.seq_lens, case.n_q, 0.1, case.out, case.lse, case.ws, case.ws.numel())
+    assert case.status() == mq.MQ_ERR_DEVICE
+
+
+def test_error_against_unquantized_is_reported():
+    """Reported, not gated: error of the quantized path against fp64 attention over
+    the original (unquantized) K/V on the long workload shape (parity unpinned)."""
+    w = wl.long_decode(L=4096)
+    case = GpuCase(w)
+    out, _ = case.decode()
+    eo, _ = oracle_outputs(w, case.inp, unquantized=True)
+    o = out.cpu().numpy()
+    err = float(np.max(np.abs(o - eo)))
+    rel = float(np.linalg.norm(o - eo) / np.linalg.norm(eo))
+    print(f"\nvs unquantized fp64 attention: max-abs {err:.3e}, relative L2 {rel:.3e}")
+    assert np.isfinite(err)
