@@ -1,0 +1,478 @@
+"""Benchmark of the quantized-KV decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {mq,reference}] [--workload long]
+
+A step is one pass of the whole hot path over the workload: quantize-on-append of
+the step's new K/V token(s) into the paged cache (mq_kv_append), then split-K decode
+attention of the step's query token(s) against the whole cache (mq_decode_attn).
+The default workload is the 64K-context single-stream decode (batch 1, 32 q / 8 kv
+heads, head_dim 128, 65536 cached tokens including the step's own, shuffled
+16-token blocks, bf16 inputs).  Inputs are seeded synthetic tensors.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier +
+torch.cuda.synchronize() on both sides, replayed from a CUDA graph of steps; the
+caches read by successive steps rotate over copies that together exceed 4x the L2
+size, so no step finds its KV in L2.  Each decode launch is bracketed by CUDA events
+recorded in the graph on the launching stream (the kernel's own duration feeds the
+roofline figure).  Multi-GPU (torchrun): every rank runs its own replica (the work
+shards over independent sessions; no collective on the data path), the time is
+the max over ranks, and the value is the whole job's bytes / that time.
+
+`e2e` times the same step through the C ABI from pinned HOST buffers: per step an
+H2D copy of q and the new K/V, the two calls, a D2H copy of out and lse, and a
+stream synchronize.  `--impl reference` runs the CPU oracle (the reference arm) on
+a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-KV decode attention: KV GB/s (% of HBM peak) and µs/step at 64K ctx"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=500)
+    ap.add_argument("--impl", default="mq", choices=["mq", "reference"])
+    ap.add_argument("--workload", default="long", choices=["tiny", "long", "prefix", "verify", "mixed"])
+    ap.add_argument("--graph-steps", type=int, default=0, help="steps per captured graph (0: one rotation)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tune", type=float, default=0.0, help="run mq_tune with this budget (s) first")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0=None, t1=None):
+        rows = [r for t, r in self.rows if (t0 is None or t >= t0) and (t1 is None or t <= t1)]
+        if not rows:
+            rows = [r for _, r in self.rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "quantized_kv_decode_quantize_b200", "csrc")
+    for n in sorted(os.listdir(d)):
+        with open(os.path.join(d, n), "rb") as f:
+            h.update(n.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload_name: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload_name)
+    if not e or e.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------------
+def max_over_ranks(x: float, device) -> float:
+    """The max of x over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def algorithmic_bytes(w, bytes_per_token_head: int):
+    """Bytes a decode launch must move: every (token, kv-head) of every sequence once
+    (a shared prefix counted once per sequence: the logical figure), q, out, lse and
+    the block-table entries read; plus the append of the step's tokens (bf16 K/V
+    read, quantized form written)."""
+    esz = 4 if w.dtype == "f32" else 2
+    kv = sum(w.seq_lens) * w.n_kv_heads * bytes_per_token_head
+    q = w.total_q * w.n_q_heads * w.head_dim * esz
+    out = w.total_q * w.n_q_heads * (w.head_dim + 1) * 4
+    bt = sum((L + 15) // 16 for L in w.seq_lens) * 4 + 8 * w.n_seqs
+    decode = kv + q + out + bt
+    n_app = sum(w.n_append)
+    append = n_app * w.n_kv_heads * (2 * w.head_dim * esz + bytes_per_token_head)
+    return decode, append
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle on the host cores, on a bounded sample of
+    the workload per step."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from quantized_kv_decode_quantize_b200 import workloads as wl
+
+    if rank != 0:
+        return
+    w = wl.FULL[args.workload]()
+    inp = wl.make_inputs(w)
+    cores = oracle.max_threads()
+    bpt = oracle.kv_bytes_per_token_head(w.head_dim)
+    # sample: query heads of kv-head 0 of sequence 0 over a token slice sized so that the
+    # whole run stays within a few minutes
+    L = w.seq_lens[0]
+    G = w.n_q_heads // w.n_kv_heads
+    kf = inp.seq_k(0)[:, :1].float().numpy()
+    vf = inp.seq_v(0)[:, :1].float().numpy()
+    kc, ks = oracle.quantize_k(kf)
+    vp, vs = oracle.quantize_v(vf)
+    q = inp.q[: w.n_q[0], :G].float().numpy().astype(np.float64)
+    scale = 1.0 / math.sqrt(w.head_dim)
+
+    def step(n_tok):
+        # quantize the step's token (the append) and attend over the first n_tok tokens
+        oracle.quantize_k(kf[L - 1: L])
+        oracle.quantize_v(vf[L - 1: L])
+        oracle.attention_quant(q, kc[:n_tok], ks[:n_tok], vp[:n_tok], vs[:n_tok], scale, cores)
+
+    t = time.perf_counter()
+    step(min(L, 8192))
+    per_tok = (time.perf_counter() - t) / min(L, 8192)
+    budget = 150.0
+    n_tok = int(max(w.n_q[0] + 16, min(L, budget / max(1, args.steps + args.warmup) / max(per_tok, 1e-9))))
+    for _ in range(args.warmup):
+        step(n_tok)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step(n_tok)
+    dt = time.perf_counter() - t0
+    bytes_step = n_tok * bpt
+    val = bytes_step * args.steps / dt / 1e9
+    line = {
+        "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": w.name, "note": w.note},
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"per step: quantize of the step's K/V token, then fp64 attention of the "
+                                   f"{G} q-heads of kv-head 0 over the first {n_tok} of {L} tokens"},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w, inp, steps_budget_s=20.0):
+    """The oracle as it stands, on all host cores: full decode steps of the workload
+    (every sequence, every head) until ~steps_budget_s of work; GB/s of KV read."""
+    import numpy as np
+
+    import oracle
+
+    cores = oracle.max_threads()
+    bpt = oracle.kv_bytes_per_token_head(w.head_dim)
+    codes = []
+    for b in range(w.n_seqs):
+        kc, ks = oracle.quantize_k(inp.seq_k(b).float().numpy())
+        vp, vs = oracle.quantize_v(inp.seq_v(b).float().numpy())
+        codes.append((kc, ks, vp, vs))
+    q = inp.q.float().numpy().astype(np.float64)
+    qoff = np.concatenate([[0], np.cumsum(w.n_q)]).astype(int)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        for b in range(w.n_seqs):
+            oracle.attention_quant(q[qoff[b]: qoff[b + 1]], *codes[b], scale, cores)
+        n += 1
+        if time.perf_counter() - t0 > steps_budget_s or n >= 50:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": sum(w.seq_lens) * w.n_kv_heads * bpt * n / dt / 1e9, "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{n} full decode step(s) of {w.name} (all sequences and heads, fp64 attention over the "
+                      f"quantized cache), {dt:.1f} s"}
+
+
+def run_mq(args, rank, world, local):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import quantized_kv_decode_quantize_b200 as mq
+    from quantized_kv_decode_quantize_b200 import workloads as wl
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    w = wl.FULL[args.workload]()
+    inp = wl.make_inputs(w)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = props.L2_cache_size
+    bpt = mq.mq_page_bytes(w.head_dim) // 16
+    copy_bytes = w.kv_bytes_unique(bpt)
+    copies = max(2, math.ceil(4 * l2 / copy_bytes))
+    tabs_np, n_blocks = wl.block_tables(w, copies=copies)
+    cache = mq.Cache(w.n_kv_heads, w.head_dim, n_blocks)
+    tabs = torch.from_numpy(tabs_np).to(dev)
+    dt_code = mq.MQ_F32 if w.dtype == "f32" else mq.MQ_BF16
+    i32 = dict(dtype=torch.int32, device=dev)
+
+    # history: everything but the step's own appended tokens, in every copy
+    hist_k, hist_v, step_k, step_v = [], [], [], []
+    for b in range(w.n_seqs):
+        n_app = w.n_append[b]
+        kb, vb = inp.own_k[b], inp.own_v[b]
+        hist_k.append(kb[: kb.shape[0] - n_app])
+        hist_v.append(vb[: vb.shape[0] - n_app])
+        step_k.append(kb[kb.shape[0] - n_app:])
+        step_v.append(vb[vb.shape[0] - n_app:])
+    for c in range(copies):
+        if w.shared_prefix:
+            mq.mq_kv_append(cache.handle, inp.prefix_k.to(dev), inp.prefix_v.to(dev), dt_code, 1, w.shared_prefix,
+                            torch.tensor([0, w.shared_prefix], **i32), torch.tensor([0], **i32), tabs[c][:1].contiguous(),
+                            w.max_blocks())
+        n_h = [int(x.shape[0]) for x in hist_k]
+        if sum(n_h):
+            mq.mq_kv_append(cache.handle, torch.cat(hist_k).to(dev), torch.cat(hist_v).to(dev), dt_code, w.n_seqs,
+                            sum(n_h), torch.tensor(np.concatenate([[0], np.cumsum(n_h)]).astype(np.int32), device=dev),
+                            torch.tensor([w.shared_prefix] * w.n_seqs, **i32), tabs[c], w.max_blocks())
+    torch.cuda.synchronize(dev)
+    assert mq.mq_device_status(cache.handle) == mq.MQ_OK
+
+    if args.tune > 0:
+        mq.mq_tune(cache.handle, args.tune, w.n_q_heads)
+
+    n_new = [int(x.shape[0]) for x in step_k]
+    new_k = torch.cat(step_k).to(dev).contiguous()
+    new_v = torch.cat(step_v).to(dev).contiguous()
+    cu_new = torch.tensor(np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32), device=dev)
+    start = torch.tensor([L - a for L, a in zip(w.seq_lens, w.n_append)], **i32)
+    q = inp.q.to(dev).contiguous()
+    seq_lens = torch.tensor(w.seq_lens, **i32)
+    n_q = torch.tensor(w.n_q, **i32)
+    out = torch.empty((w.total_q, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.total_q, w.n_q_heads), dtype=torch.float32, device=dev)
+    ws_bytes = mq.mq_decode_workspace_bytes(cache.handle, w.n_seqs, w.n_q_heads, w.max_q, w.max_seq_len)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    tab_c = [tabs[c] for c in range(copies)]
+
+    def step(c, stream, ev=None):
+        mq.mq_kv_append(cache.handle, new_k, new_v, dt_code, w.n_seqs, sum(n_new), cu_new, start, tab_c[c],
+                        w.max_blocks(), stream)
+        if ev is not None:
+            ev[0].record(stream)
+        mq.mq_decode_attn(cache.handle, q, dt_code, w.n_seqs, w.n_q_heads, w.total_q, w.max_q, w.max_seq_len,
+                          tab_c[c], w.max_blocks(), seq_lens, n_q, scale, out, lse, ws, ws_bytes, stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    # ---- capture S steps (one rotation over the copies, or more) in a graph ----
+    S = args.graph_steps or copies * max(1, math.ceil(24 / copies))
+    stream = torch.cuda.Stream(dev)
+    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+           for _ in range(S)]
+    with torch.cuda.stream(stream):
+        for i in range(3):                        # eager warm-up before capture
+            step(i % copies, stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(S):
+            step(i % copies, stream, evs[i])
+    torch.cuda.synchronize(dev)
+
+    # warm-up: W steps (whole graphs, rounded up), then ~1 s of untimed soak for clocks
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(max(1, math.ceil(args.warmup / S))):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    t_soak = time.time()
+    while time.time() - t_soak < 1.0:
+        g.replay()
+        torch.cuda.synchronize(dev)
+    reps, rem = divmod(args.steps, S)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.time()
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for _ in range(reps):
+            g.replay()
+        for i in range(rem):                      # the remainder eagerly: exactly K steps
+            step(i % copies, stream)
+        t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    # decode-kernel durations of the last graph replay inside the timed region
+    kern_ms = [a.elapsed_time(b) for a, b in evs] if reps > 0 else []
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
+    assert mq.mq_device_status(cache.handle, stream) == mq.MQ_OK
+
+    dec_bytes, app_bytes = algorithmic_bytes(w, bpt)
+    step_bytes = dec_bytes + app_bytes
+    value = world * step_bytes * args.steps / (elapsed_ms * 1e-3) / 1e9
+    peak, peak_kind = load_peaks()
+    kern_avg = statistics.mean(kern_ms) if kern_ms else None
+    achieved = dec_bytes / (kern_avg * 1e-3) / 1e9 if kern_avg else None
+
+    # ---- e2e through the C ABI from pinned host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        h_q = inp.q.contiguous().pin_memory()
+        h_k = torch.cat(step_k).contiguous().pin_memory()
+        h_v = torch.cat(step_v).contiguous().pin_memory()
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        K2 = min(args.steps, 2000)
+        with torch.cuda.stream(stream):
+            for i in range(min(args.warmup, 50)):
+                q.copy_(h_q, non_blocking=True)
+                new_k.copy_(h_k, non_blocking=True)
+                new_v.copy_(h_v, non_blocking=True)
+                step(i % copies, stream)
+                h_out.copy_(out, non_blocking=True)
+                h_lse.copy_(lse, non_blocking=True)
+                stream.synchronize()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize(dev)
+            e0 = time.perf_counter()
+            for i in range(K2):
+                q.copy_(h_q, non_blocking=True)
+                new_k.copy_(h_k, non_blocking=True)
+                new_v.copy_(h_v, non_blocking=True)
+                step(i % copies, stream)
+                h_out.copy_(out, non_blocking=True)
+                h_lse.copy_(lse, non_blocking=True)
+                stream.synchronize()
+            e_dt = time.perf_counter() - e0
+        e_dt = max_over_ranks(e_dt, dev)
+        h2d = h_q.numel() * h_q.element_size() + h_k.numel() * h_k.element_size() * 2
+        d2h = h_out.numel() * 4 + h_lse.numel() * 4
+        e2e = {"value": world * step_bytes * K2 / e_dt / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": K2, "ms_per_step": e_dt / K2 * 1e3}
+
+    if rank == 0:
+        cfg = mq.mq_get_decode_config(cache.handle, 0)
+        clocks = sampler.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8/int4 KV, fp32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": w.name, "note": w.note, "n_seqs": w.n_seqs, "seq_lens_sum": int(sum(w.seq_lens)),
+                       "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+                       "l2_policy": f"inputs larger than L2: {copies} rotating cache copies "
+                                    f"({copies * copy_bytes / 1e6:.0f} MB, L2 {l2 / 1e6:.0f} MB)",
+                       "parallelism": f"replica x{world}", "step": "mq_kv_append + mq_decode_attn",
+                       "decode_config": cfg, "us_per_step": elapsed_ms / args.steps * 1e3,
+                       "pct_of_8TBps": 100 * value / world / 8000.0},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": (achieved / peak) if achieved else None, "peak_kind": peak_kind,
+                         "traffic": ncu_traffic(w.name), "kernel": "mq::decode_kernel",
+                         "bytes_per_launch": dec_bytes, "kernel_us_mean": kern_avg * 1e3 if kern_avg else None,
+                         "kernel_us_median": statistics.median(kern_ms) * 1e3 if kern_ms else None},
+            "e2e": e2e,
+            "gpu_launches": 2 * args.steps,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
+                       "samples": clocks["samples"]},
+            "wall_s": wall1 - wall0,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline(w, inp)
+        print(json.dumps(line), flush=True)
+    del g
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_mq(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()
