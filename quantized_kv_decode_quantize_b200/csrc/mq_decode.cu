@@ -48,7 +48,6 @@ struct Cfg {
     static constexpr int VCH = D / 64;           // V code chunks per lane per page
     static constexpr int SCH = D / 64;           // V scale chunks per lane per page
     static constexpr bool HI = ROWS > 8;         // rows g+8 of a QK m-tile are real rows
-    static constexpr bool QREG = MTQ * KS * 3 * (HI ? 4 : 2) <= 48;  // q fragments in registers
     static constexpr int PART = ROWS * D + 2 * ROWS;                 // floats of one partial
 };
 
@@ -76,7 +75,7 @@ __host__ __device__ inline Smem smem_layout(int W, int R, int SD) {
     s.coef = off;
     off += (size_t)8 * ROWS * 2 * 4;  // up to 8 merges per phase
     s.qfrag = off;
-    off += C::QREG ? 0 : (size_t)C::MTQ * C::KS * 3 * 32 * 16;
+    off += (size_t)C::MTQ * C::KS * 3 * 32 * 16;
     s.flags = off;
     off += 64 * 4;
     off = al(off, 8);
@@ -94,8 +93,8 @@ __host__ __device__ inline Smem smem_layout(int W, int R, int SD) {
 __device__ __forceinline__ void merge_coef(float ml, float ll, float mr, float lr, float& m, float& l, float& a,
                                            float& b) {
     m = fmaxf(ml, mr);
-    a = (ml == m) ? 1.0f : exp2f(__fsub_rn(ml, m));
-    b = (mr == m) ? 1.0f : exp2f(__fsub_rn(mr, m));
+    a = (ml == m) ? 1.0f : ex2(__fsub_rn(ml, m));
+    b = (mr == m) ? 1.0f : ex2(__fsub_rn(mr, m));
     l = __fadd_rn(__fmul_rn(ll, a), __fmul_rn(lr, b));
 }
 __device__ __forceinline__ float merge_val(float ol, float orr, float a, float b) {
@@ -172,7 +171,7 @@ __device__ __forceinline__ float load_q(const DecodeParams& p, size_t i) {
 }
 
 template <int D, int ROWS>
-__global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_kernel(const DecodeParams p) {
     using C = Cfg<D, ROWS>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int W = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -228,20 +227,9 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
     // Lane (g, t) owns rows 16*mt + 8*h + g and channels [t*D/4, (t+1)*D/4).  The
     // A fragment of mma.m16n8k32 for k-step ks holds, for row g (h = 0) and g + 8
     // (h = 1), channels t*D/4 + 8*ks + {0..3} (regs 0/1) and + {4..7} (regs 2/3).
-    uint32_t qa[C::QREG ? C::MTQ : 1][C::QREG ? C::KS : 1][3][4];
     float crow[C::SLOTS];
     int lim[C::SLOTS];
     uint32_t* qfrag_s = reinterpret_cast<uint32_t*>(smem + S.qfrag);
-    if constexpr (C::QREG) {
-#pragma unroll
-        for (int mt = 0; mt < C::MTQ; mt++)
-#pragma unroll
-            for (int ks = 0; ks < C::KS; ks++)
-#pragma unroll
-                for (int lb = 0; lb < 3; lb++)
-#pragma unroll
-                    for (int r = 0; r < 4; r++) qa[mt][ks][lb][r] = 0u;
-    }
 #pragma unroll
     for (int k = 0; k < C::SLOTS; k++) {
         const int mt = k >> 1, h = k & 1;
@@ -253,14 +241,11 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
         const bool qok = real && qrow < p.total_q;
         if (real && !qok && t == 0) atomicOr(p.err, kErrBadRow);
         constexpr int CH = D / 4;
-        float qv[CH];
         float amax = 0.0f;
         const size_t base = ((size_t)qrow * p.n_q_heads + (size_t)hk * p.group + hq) * D + (size_t)t * CH;
-#pragma unroll
-        for (int c = 0; c < CH; c++) {
-            qv[c] = qok ? load_q(p, base + c) : 0.0f;
-            amax = fmaxf(amax, fabsf(qv[c]));
-        }
+        // two passes over the lane's channels (max, then limbs) keep few values live
+#pragma unroll 8
+        for (int c = 0; c < CH; c++) amax = fmaxf(amax, fabsf(qok ? load_q(p, base + c) : 0.0f));
         amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
         int E = 0;
@@ -277,7 +262,8 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
                 uint32_t l2 = 0, l1 = 0, l0 = 0;
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
-                    const int Q = (int)rintf(__fmul_rn(qv[8 * ks + 4 * half + i], up));
+                    const float qv = qok ? load_q(p, base + 8 * ks + 4 * half + i) : 0.0f;
+                    const int Q = (int)rintf(__fmul_rn(qv, up));
                     l2 |= (uint32_t)((Q >> 16) & 0xFF) << (8 * i);
                     l1 |= (uint32_t)((Q >> 8) & 0xFF) << (8 * i);
                     l0 |= (uint32_t)(Q & 0xFF) << (8 * i);
@@ -288,28 +274,26 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
             }
 #pragma unroll
             for (int lb = 0; lb < 3; lb++) {
-                if constexpr (C::QREG) {
-                    qa[mt][ks][lb][h] = w[lb][0];
-                    qa[mt][ks][lb][2 + h] = w[lb][1];
-                } else if (warp == 0) {
+                if (warp == 0) {
                     uint32_t* f = qfrag_s + ((((size_t)mt * C::KS + ks) * 3 + lb) * 32 + lane) * 4;
-                    f[h] = w[lb][0];
-                    f[2 + h] = w[lb][1];
-                    if constexpr (!C::HI) {
-                        f[1] = 0u;
-                        f[3] = 0u;
+                    if constexpr (C::HI) {
+                        f[h] = w[lb][0];
+                        f[2 + h] = w[lb][1];
+                    } else {   // rows g + 8 are padding: keep regs 0 and 2 only, as 64 bits
+                        f[0] = w[lb][0];
+                        f[1] = w[lb][1];
                     }
                 }
             }
         }
     }
-    if constexpr (!C::QREG) __syncthreads();
+    __syncthreads();
 
     // ---- per-warp chunk sequence and page ring ----
     const uint64_t policy = l2_evict_first_policy();
     auto chunk_of = [&](int ro) { return c0 + ro * W + warp; };
     // pages of this warp, in order: all its chunks are full except possibly the last
-    // chunk of the sequence
+    // chunk of the sequence, which is the warp's last
     int my_pages = 0;
     for (int ro = 0; ro < n_rounds; ro++) {
         const int c = chunk_of(ro);
@@ -330,9 +314,8 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
             bt[(ro & 1) * kChunkPages + lane] = blk;
         }
     };
-    auto issue = [&](int k) {  // lane 0 only: page k of this warp's sequence
-        const int ro = k / kChunkPages, pi = k % kChunkPages, slot = k % R;
-        const int blk = bt[(ro & 1) * kChunkPages + pi];
+    auto issue = [&](int k, int slot) {  // lane 0 only: page k of this warp's sequence into `slot`
+        const int blk = bt[((k / kChunkPages) & 1) * kChunkPages + (k % kChunkPages)];
         const uint8_t* src = p.pool + ((long long)(blk < 0 ? 0 : blk) * p.n_kv_heads + hk) * C::PB;
         mbar_arrive_expect_tx(smem_u32(&bars[slot]), C::PB);
         tma_load_1d(smem_u32(ring + (size_t)slot * C::PB), src, C::PB, smem_u32(&bars[slot]), policy);
@@ -341,13 +324,18 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
     load_bt(1);
     __syncwarp();
     if (lane == 0)
-        for (int k = 0; k < R && k < my_pages; k++) issue(k);
+        for (int k = 0; k < R && k < my_pages; k++) issue(k, k);
+
+    // the smallest visibility limit of the real rows of this row block
+    const int lim_min = L - nq + row0 / p.group + 1;
 
     bool aborted = false;
     int k_abort = 0;       // first page not waited for after a timeout
     int k_next = 0;        // next page of this warp to consume
+    int slot = 0;          // its ring slot (k_next % R) and mbarrier phase ((k_next / R) & 1)
+    uint32_t phase = 0;
     int n_stack = 0;       // round-stack entries (uniform)
-    int* stack_level = misc + 4;   // levels of stack entries (up to 16)
+    int* stack_level = misc + 4;   // levels of stack entries (up to 12)
 
     for (int ro = 0; ro < n_rounds; ro++) {
         const int c = chunk_of(ro);
@@ -372,9 +360,7 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
             }
             const int pages_here = min(kChunkPages, n_pages - c * kChunkPages);
             for (int pi = 0; pi < pages_here; pi++, k_next++) {
-                const int slot = k_next % R;
-                const uint32_t par = (uint32_t)((k_next / R) & 1);
-                if (!aborted && !mbar_wait_bounded(smem_u32(&bars[slot]), par)) {
+                if (!aborted && !mbar_wait_bounded(smem_u32(&bars[slot]), phase)) {
                     aborted = true;
                     k_abort = k_next;
                     if (lane == 0) atomicOr(p.err, kErrTimeout);
@@ -382,98 +368,123 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
                 const uint8_t* pp = ring + (size_t)slot * C::PB;
                 const int lp = c * kChunkPages + pi;
                 const bool bad = bt[(ro & 1) * kChunkPages + pi] < 0;
+                // every token of the page visible to every row: no per-element masking
+                const bool full = !bad && (lp + 1) * kPageTokens <= lim_min;
 
                 // ---- scores: int8 QK^T on the tensor cores ----
-                uint4 kc[C::KCH];
-#pragma unroll
-                for (int i = 0; i < C::KCH; i++) kc[i] = lds128(pp + (size_t)(i * 32 + lane) * 16);
                 const float2 skA = __half22float2(u32_as_h2(lds32(pp + k_scale_off(D) + 4 * t)));
                 const float2 skB = __half22float2(u32_as_h2(lds32(pp + k_scale_off(D) + 16 + 4 * t)));
-                const float sk[2][2] = {{skA.x, skA.y}, {skB.x, skB.y}};
                 float z[C::SLOTS][2][2];
 #pragma unroll
                 for (int mt = 0; mt < C::MTQ; mt++) {
+                    // the lane's key chunks: token g (n-tile 0) and token g + 8 (n-tile 1)
+                    uint4 kc[C::KCH];
 #pragma unroll
-                    for (int nt = 0; nt < 2; nt++) {
-                        int d21[4] = {0, 0, 0, 0}, d0[4] = {0, 0, 0, 0};
+                    for (int i = 0; i < C::KCH; i++) kc[i] = lds128(pp + (size_t)(i * 32 + lane) * 16);
+                    int d2[2][4], d0[2][4];
 #pragma unroll
-                        for (int lb = 0; lb < 3; lb++) {
+                    for (int nt = 0; nt < 2; nt++)
 #pragma unroll
-                            for (int ks = 0; ks < C::KS; ks++) {
+                        for (int i = 0; i < 4; i++) d2[nt][i] = d0[nt][i] = 0;
+#pragma unroll
+                    for (int lb = 0; lb < 3; lb++) {
+#pragma unroll
+                        for (int ks = 0; ks < C::KS; ks++) {
+                            uint32_t a[4];
+                            const uint32_t* f = qfrag_s + ((((size_t)mt * C::KS + ks) * 3 + lb) * 32 + lane) * 4;
+                            if constexpr (C::HI) {
+                                const uint4 v = lds128(f);
+                                a[0] = v.x;
+                                a[1] = v.y;
+                                a[2] = v.z;
+                                a[3] = v.w;
+                            } else {   // rows g + 8 are padding: their fragment registers are zero
+                                const uint2 v = lds64(f);
+                                a[0] = v.x;
+                                a[1] = 0u;
+                                a[2] = v.y;
+                                a[3] = 0u;
+                            }
+#pragma unroll
+                            for (int nt = 0; nt < 2; nt++) {
                                 const uint4 ch = kc[nt * (D / 64) + ks / 2];
                                 const uint32_t b0 = (ks & 1) ? ch.z : ch.x;
                                 const uint32_t b1 = (ks & 1) ? ch.w : ch.y;
-                                uint32_t a[4];
-                                if constexpr (C::QREG) {
-#pragma unroll
-                                    for (int r = 0; r < 4; r++) a[r] = qa[mt][ks][lb][r];
-                                } else {
-                                    const uint4 f = lds128(qfrag_s + ((((size_t)mt * C::KS + ks) * 3 + lb) * 32 + lane) * 4);
-                                    a[0] = f.x;
-                                    a[1] = f.y;
-                                    a[2] = f.z;
-                                    a[3] = f.w;
-                                }
-                                if (lb == 0) mma_s8s8(d21, a, b0, b1);
-                                else if (lb == 1) mma_u8s8(d21, a, b0, b1);
-                                else mma_u8s8(d0, a, b0, b1);
-                            }
-                            if (lb == 0) {
-#pragma unroll
-                                for (int i = 0; i < 4; i++) d21[i] <<= 8;
+                                if (lb == 0) mma_s8s8(d2[nt], a, b0, b1);
+                                else if (lb == 1) mma_u8s8(d2[nt], a, b0, b1);
+                                else mma_u8s8(d0[nt], a, b0, b1);
                             }
                         }
+                        if (lb == 0) {
+#pragma unroll
+                            for (int nt = 0; nt < 2; nt++)
+#pragma unroll
+                                for (int i = 0; i < 4; i++)
+                                    if (16 * mt + 8 * (i / 2) < ROWS) d2[nt][i] <<= 8;
+                        }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < 2; nt++)
 #pragma unroll
                         for (int h = 0; h < 2; h++) {
                             if (16 * mt + 8 * h < ROWS) {
                                 const int k = 2 * mt + h;
 #pragma unroll
                                 for (int e = 0; e < 2; e++) {
-                                    const float s = __fmaf_rn((float)d21[2 * h + e], 256.0f, (float)d0[2 * h + e]);
-                                    z[k][nt][e] = __fmul_rn(__fmul_rn(s, crow[k]), sk[nt][e]);
+                                    const float s = __fmaf_rn((float)d2[nt][2 * h + e], 256.0f, (float)d0[nt][2 * h + e]);
+                                    const float skv = nt == 0 ? (e == 0 ? skA.x : skA.y) : (e == 0 ? skB.x : skB.y);
+                                    z[k][nt][e] = __fmul_rn(__fmul_rn(s, crow[k]), skv);
                                 }
                             }
                         }
-                    }
                 }
 
                 // ---- online softmax (log2 units) ----
                 const int tok0 = lp * kPageTokens + 2 * t;
                 float pw[C::SLOTS][2][2], alph[C::SLOTS];
+                bool resc = false;
 #pragma unroll
                 for (int k = 0; k < C::SLOTS; k++) {
-                    float pm = -INFINITY;
+                    if (!full) {
+#pragma unroll
+                        for (int nt = 0; nt < 2; nt++)
+#pragma unroll
+                            for (int e = 0; e < 2; e++) {
+                                const bool valid = !bad && (tok0 + 8 * nt + e) < lim[k];
+                                z[k][nt][e] = valid ? z[k][nt][e] : -INFINITY;
+                            }
+                    }
+                    float pm = fmaxf(fmaxf(z[k][0][0], z[k][0][1]), fmaxf(z[k][1][0], z[k][1][1]));
+                    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 1));
+                    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 2));
+                    const float mnew = fmaxf(mrun[k], pm);
+                    alph[k] = (mnew == mrun[k]) ? 1.0f : ex2(__fsub_rn(mrun[k], mnew));
+                    resc |= alph[k] != 1.0f;
 #pragma unroll
                     for (int nt = 0; nt < 2; nt++)
 #pragma unroll
                         for (int e = 0; e < 2; e++) {
-                            const bool valid = !bad && (tok0 + 8 * nt + e) < lim[k];
-                            z[k][nt][e] = valid ? z[k][nt][e] : -INFINITY;
-                            pm = fmaxf(pm, z[k][nt][e]);
+                            const float pv = ex2(__fsub_rn(z[k][nt][e], mnew));
+                            pw[k][nt][e] = full ? pv : (z[k][nt][e] == -INFINITY ? 0.0f : pv);
                         }
-                    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 1));
-                    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 2));
-                    const float mnew = fmaxf(mrun[k], pm);
-                    alph[k] = (mnew == mrun[k]) ? 1.0f : exp2f(__fsub_rn(mrun[k], mnew));
-#pragma unroll
-                    for (int nt = 0; nt < 2; nt++)
-#pragma unroll
-                        for (int e = 0; e < 2; e++)
-                            pw[k][nt][e] = (z[k][nt][e] == -INFINITY) ? 0.0f : exp2f(__fsub_rn(z[k][nt][e], mnew));
                     const float ps = __fadd_rn(__fadd_rn(pw[k][0][0], pw[k][0][1]), __fadd_rn(pw[k][1][0], pw[k][1][1]));
                     lrun[k] = __fadd_rn(__fmul_rn(lrun[k], alph[k]), ps);
                     mrun[k] = mnew;
                 }
+                // rescaling by exactly 1 changes nothing, so it is skipped when no row's
+                // running max moved (the common case after the first pages of a chunk)
+                if (__any_sync(FULL, resc)) {
 #pragma unroll
-                for (int n = 0; n < C::NTP; n++) {
-                    const float a0 = __shfl_sync(FULL, alph[n], 8 * t);
-                    const float a1 = __shfl_sync(FULL, alph[n], 8 * t + 4);
+                    for (int n = 0; n < C::NTP; n++) {
+                        const float a0 = __shfl_sync(FULL, alph[n], 8 * t);
+                        const float a1 = __shfl_sync(FULL, alph[n], 8 * t + 4);
 #pragma unroll
-                    for (int j = 0; j < C::MTP; j++) {
-                        O[j][n][0] = __fmul_rn(O[j][n][0], a0);
-                        O[j][n][1] = __fmul_rn(O[j][n][1], a1);
-                        O[j][n][2] = __fmul_rn(O[j][n][2], a0);
-                        O[j][n][3] = __fmul_rn(O[j][n][3], a1);
+                        for (int j = 0; j < C::MTP; j++) {
+                            O[j][n][0] = __fmul_rn(O[j][n][0], a0);
+                            O[j][n][1] = __fmul_rn(O[j][n][1], a1);
+                            O[j][n][2] = __fmul_rn(O[j][n][2], a0);
+                            O[j][n][3] = __fmul_rn(O[j][n][3], a1);
+                        }
                     }
                 }
 
@@ -484,13 +495,12 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
 #pragma unroll
                 for (int i = 0; i < C::SCH; i++)
                     svw[i] = lds128(pp + v_scale_off(D) + (size_t)t * C::NG * 8 + (size_t)i * 16);
-                const uint32_t* vwd = reinterpret_cast<const uint32_t*>(vcw);
-                const uint32_t* swd = reinterpret_cast<const uint32_t*>(svw);
 #pragma unroll
                 for (int q = 0; q < C::NG; q++) {
-                    const float2 s0 = __half22float2(u32_as_h2(swd[2 * q]));
-                    const float2 s1 = __half22float2(u32_as_h2(swd[2 * q + 1]));
-                    const uint32_t x0 = vwd[2 * q] ^ 0x88888888u, x1 = vwd[2 * q + 1] ^ 0x88888888u;
+                    const float2 s0 = __half22float2(u32_as_h2(comp(svw[(2 * q) / 4], (2 * q) % 4)));
+                    const float2 s1 = __half22float2(u32_as_h2(comp(svw[(2 * q + 1) / 4], (2 * q + 1) % 4)));
+                    const uint32_t x0 = comp(vcw[(2 * q) / 4], (2 * q) % 4);
+                    const uint32_t x1 = comp(vcw[(2 * q + 1) / 4], (2 * q + 1) % 4);
                     const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
                     const uint32_t A0 = nib_lo_to_h2(x0), A1 = nib_hi_to_h2(x0);
                     const uint32_t A2 = nib_lo_to_h2(x1), A3 = nib_hi_to_h2(x1);
@@ -498,10 +508,14 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
                     const uint32_t B2 = nib_lo_to_h2(y1), B3 = nib_hi_to_h2(y1);
 #pragma unroll
                     for (int n = 0; n < C::NTP; n++) {
-                        const float w00 = pw[n][0][0] == 0.0f ? 0.0f : __fmul_rn(pw[n][0][0], s0.x);
-                        const float w01 = pw[n][0][1] == 0.0f ? 0.0f : __fmul_rn(pw[n][0][1], s0.y);
-                        const float w10 = pw[n][1][0] == 0.0f ? 0.0f : __fmul_rn(pw[n][1][0], s1.x);
-                        const float w11 = pw[n][1][1] == 0.0f ? 0.0f : __fmul_rn(pw[n][1][1], s1.y);
+                        float w00 = __fmul_rn(pw[n][0][0], s0.x), w01 = __fmul_rn(pw[n][0][1], s0.y);
+                        float w10 = __fmul_rn(pw[n][1][0], s1.x), w11 = __fmul_rn(pw[n][1][1], s1.y);
+                        if (!full) {  // masked tokens may sit next to unwritten (non-finite) scales
+                            w00 = pw[n][0][0] == 0.0f ? 0.0f : w00;
+                            w01 = pw[n][0][1] == 0.0f ? 0.0f : w01;
+                            w10 = pw[n][1][0] == 0.0f ? 0.0f : w10;
+                            w11 = pw[n][1][1] == 0.0f ? 0.0f : w11;
+                        }
                         const uint32_t bb0 = pack_h2(w00, w01), bb1 = pack_h2(w10, w11);
                         mma_f16(O[2 * q][n], A0, A1, A2, A3, bb0, bb1);
                         mma_f16(O[2 * q + 1][n], B0, B1, B2, B3, bb0, bb1);
@@ -510,7 +524,11 @@ __global__ void __launch_bounds__(256, 1) decode_kernel(const DecodeParams p) {
                 __syncwarp();
                 if (lane == 0 && !aborted && k_next + R < my_pages) {
                     fence_proxy_async_smem();
-                    issue(k_next + R);
+                    issue(k_next + R, slot);
+                }
+                if (++slot == R) {
+                    slot = 0;
+                    phase ^= 1u;
                 }
             }
             // ---- chunk partial -> shared memory (natural layout) ----

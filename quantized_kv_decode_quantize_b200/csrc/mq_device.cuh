@@ -128,6 +128,12 @@ __device__ __forceinline__ uint4 lds128(const void* p) {
     return v;
 }
 
+__device__ __forceinline__ uint2 lds64(const void* p) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_u32(p)));
+    return v;
+}
+
 __device__ __forceinline__ uint32_t lds32(const void* p) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)));
@@ -136,7 +142,7 @@ __device__ __forceinline__ uint32_t lds32(const void* p) {
 
 // D = A(16x32, s8) * B(32x8, s8) + C, int32 accumulate
 __device__ __forceinline__ void mma_s8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -144,7 +150,7 @@ __device__ __forceinline__ void mma_s8s8(int (&d)[4], const uint32_t (&a)[4], ui
 
 // D = A(16x32, u8) * B(32x8, s8) + C, int32 accumulate
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -153,7 +159,7 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], ui
 // D = A(16x16, f16) * B(16x8, f16) + D, fp32 accumulate
 __device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                         uint32_t b0, uint32_t b1) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -169,17 +175,39 @@ __device__ __forceinline__ uint32_t lop_and_or(uint32_t x, uint32_t mask, uint32
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-// Two signed 4-bit codes at bit positions (0..3, 16..19) of x (already XOR 0x8
-// biased, i.e. code + 8) -> fp16x2 holding the exact integer codes.
-__device__ __forceinline__ uint32_t nib_lo_to_h2(uint32_t xb) {
-    const uint32_t m = lop_and_or(xb, 0x000F000Fu, 0x64006400u);       // 1024 + u
+// (x & mask) ^ flip in one LOP3
+__device__ __forceinline__ uint32_t lop_and_xor(uint32_t x, uint32_t mask, uint32_t flip) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(x), "r"(mask), "r"(flip));
+    return d;
+}
+
+// Two two's-complement 4-bit codes at bit positions (0..3, 16..19) of x -> fp16x2
+// holding the exact integer codes.  One LOP3 forms 1024 + (n ^ 8) = 1032 + code in
+// each half (0x6400 is 1024; flipping bit 3 turns the two's-complement nibble into
+// code + 8), one HSUB2 removes the 1032.
+__device__ __forceinline__ uint32_t nib_lo_to_h2(uint32_t x) {
+    const uint32_t m = lop_and_xor(x, 0x000F000Fu, 0x64086408u);
     return h2_as_u32(__hsub2(u32_as_h2(m), u32_as_h2(0x64086408u)));   // - 1032
 }
-// Same for bit positions (4..7, 20..23).
-__device__ __forceinline__ uint32_t nib_hi_to_h2(uint32_t xb) {
-    const uint32_t m = lop_and_or(xb, 0x00F000F0u, 0x64006400u);       // 1024 + 16u
-    // (1024 + 16u) / 16 - 72 = u - 8
+// Same for bit positions (4..7, 20..23): 1024 + 16 (code + 8), then /16 - 72.
+__device__ __forceinline__ uint32_t nib_hi_to_h2(uint32_t x) {
+    const uint32_t m = lop_and_xor(x, 0x00F000F0u, 0x64806480u);
     return h2_as_u32(__hfma2(u32_as_h2(m), u32_as_h2(0x2C002C00u), u32_as_h2(0xD480D480u)));
+}
+
+// 2^x with the SFU instruction (ex2.approx.ftz.f32: relative error ~2^-22, subnormal
+// results flushed to zero, ex2(-inf) = +0).  Every exponential of the decode kernel
+// goes through this one function.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// component i (compile-time after unrolling) of a uint4
+__device__ __forceinline__ uint32_t comp(const uint4& v, int i) {
+    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
