@@ -6,7 +6,7 @@
 #include <cstring>
 #include <new>
 
-#include "../../include/mq.h"
+#include "mq.h"
 #include "mq_device.cuh"
 #include "mq_kernels.h"
 #include "mq_host.h"

@@ -4,7 +4,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/mq.h"
+#include "mq.h"
 
 struct mq_cache {
     int n_kv_heads;

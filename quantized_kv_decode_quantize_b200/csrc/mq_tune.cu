@@ -20,7 +20,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/mq.h"
+#include "mq.h"
 #include "mq_device.cuh"
 #include "mq_host.h"
 #include "mq_kernels.h"
