@@ -35,6 +35,9 @@
 
 namespace mq {
 
+// lazy-max threshold of the online softmax, in log2 units (weights stay <= 2^4)
+constexpr float kLazy = 4.0f;
+
 template <int D, int ROWS>
 struct Cfg {
     static constexpr int PB = page_bytes(D);
@@ -328,6 +331,9 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
 
     // the smallest visibility limit of the real rows of this row block
     const int lim_min = L - nq + row0 / p.group + 1;
+    // 32-bit shared-window addresses: ring slot 0 and this lane's q fragments
+    const uint32_t ring_s = smem_u32(ring), lane16 = (uint32_t)lane * 16u;
+    const uint32_t qf_s = smem_u32(qfrag_s) + lane16;
 
     bool aborted = false;
     int k_abort = 0;       // first page not waited for after a timeout
@@ -365,22 +371,23 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
                     k_abort = k_next;
                     if (lane == 0) atomicOr(p.err, kErrTimeout);
                 }
-                const uint8_t* pp = ring + (size_t)slot * C::PB;
+                const uint32_t pg = ring_s + (uint32_t)slot * C::PB;   // this page
+                const uint32_t pgl = pg + lane16;
                 const int lp = c * kChunkPages + pi;
                 const bool bad = bt[(ro & 1) * kChunkPages + pi] < 0;
                 // every token of the page visible to every row: no per-element masking
                 const bool full = !bad && (lp + 1) * kPageTokens <= lim_min;
 
                 // ---- scores: int8 QK^T on the tensor cores ----
-                const float2 skA = __half22float2(u32_as_h2(lds32(pp + k_scale_off(D) + 4 * t)));
-                const float2 skB = __half22float2(u32_as_h2(lds32(pp + k_scale_off(D) + 16 + 4 * t)));
+                const float2 skA = __half22float2(u32_as_h2(ldsa32(pg + k_scale_off(D) + 4 * t)));
+                const float2 skB = __half22float2(u32_as_h2(ldsa32(pg + k_scale_off(D) + 16 + 4 * t)));
                 float z[C::SLOTS][2][2];
 #pragma unroll
                 for (int mt = 0; mt < C::MTQ; mt++) {
                     // the lane's key chunks: token g (n-tile 0) and token g + 8 (n-tile 1)
                     uint4 kc[C::KCH];
 #pragma unroll
-                    for (int i = 0; i < C::KCH; i++) kc[i] = lds128(pp + (size_t)(i * 32 + lane) * 16);
+                    for (int i = 0; i < C::KCH; i++) kc[i] = ldsa128(pgl + i * 512);
                     int d2[2][4], d0[2][4];
 #pragma unroll
                     for (int nt = 0; nt < 2; nt++)
@@ -391,15 +398,15 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
 #pragma unroll
                         for (int ks = 0; ks < C::KS; ks++) {
                             uint32_t a[4];
-                            const uint32_t* f = qfrag_s + ((((size_t)mt * C::KS + ks) * 3 + lb) * 32 + lane) * 4;
+                            const uint32_t f = qf_s + (((mt * C::KS + ks) * 3 + lb) * 512);
                             if constexpr (C::HI) {
-                                const uint4 v = lds128(f);
+                                const uint4 v = ldsa128(f);
                                 a[0] = v.x;
                                 a[1] = v.y;
                                 a[2] = v.z;
                                 a[3] = v.w;
                             } else {   // rows g + 8 are padding: their fragment registers are zero
-                                const uint2 v = lds64(f);
+                                const uint2 v = ldsa64(f);
                                 a[0] = v.x;
                                 a[1] = 0u;
                                 a[2] = v.y;
@@ -457,9 +464,13 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
                     float pm = fmaxf(fmaxf(z[k][0][0], z[k][0][1]), fmaxf(z[k][1][0], z[k][1][1]));
                     pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 1));
                     pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 2));
-                    const float mnew = fmaxf(mrun[k], pm);
+                    // Lazy reference: the row's reference max moves only when a page max
+                    // exceeds it by more than kLazy (log2 units), so p = 2^(z - m) <= 2^kLazy
+                    // and a rescale of O is rare.  The first finite page max always moves it
+                    // (O is still zero then, so that rescale is skipped).
+                    const float mnew = (pm > __fadd_rn(mrun[k], kLazy)) ? pm : mrun[k];
                     alph[k] = (mnew == mrun[k]) ? 1.0f : ex2(__fsub_rn(mrun[k], mnew));
-                    resc |= alph[k] != 1.0f;
+                    resc |= (alph[k] != 1.0f) && (mrun[k] != -INFINITY);
 #pragma unroll
                     for (int nt = 0; nt < 2; nt++)
 #pragma unroll
@@ -491,10 +502,9 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
                 // ---- P.V: int4 codes as exact fp16, weights p * s_v in fp16 ----
                 uint4 vcw[C::VCH], svw[C::SCH];
 #pragma unroll
-                for (int i = 0; i < C::VCH; i++) vcw[i] = lds128(pp + v_code_off(D) + (size_t)(i * 32 + lane) * 16);
+                for (int i = 0; i < C::VCH; i++) vcw[i] = ldsa128(pgl + v_code_off(D) + i * 512);
 #pragma unroll
-                for (int i = 0; i < C::SCH; i++)
-                    svw[i] = lds128(pp + v_scale_off(D) + (size_t)t * C::NG * 8 + (size_t)i * 16);
+                for (int i = 0; i < C::SCH; i++) svw[i] = ldsa128(pg + v_scale_off(D) + t * (C::NG * 8) + i * 16);
 #pragma unroll
                 for (int q = 0; q < C::NG; q++) {
                     const float2 s0 = __half22float2(u32_as_h2(comp(svw[(2 * q) / 4], (2 * q) % 4)));
