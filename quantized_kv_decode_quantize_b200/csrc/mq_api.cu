@@ -82,10 +82,12 @@ DecodePlan plan_decode(const mq_cache* c, int n_seqs, int n_q_heads, int max_q, 
     pl.max_splits = (int)std::max<long long>(1, (max_chunks + cpc - 1) / cpc);
     if (pl.cpc < pl.warps) pl.cpc = pl.warps;
     auto fit = [&]() {
-        const int rounds = (int)((pl.cpc + pl.warps - 1) / pl.warps);
-        int sd = 1;
-        while ((1 << (sd - 1)) < rounds) sd++;
-        pl.stack_depth = sd;
+        // each warp reduces an aligned run of cpc / warps chunks; its binary counter
+        // keeps at most log2(run) left siblings (at least one entry: its result)
+        const int run = (int)(pl.cpc / pl.warps);
+        int sd = 0;
+        while ((1 << sd) < run) sd++;
+        pl.stack_depth = sd < 1 ? 1 : sd;
         pl.smem = decode_smem_bytes(c->head_dim, pl.rows, pl.warps, pl.pages_per_stage, pl.stack_depth);
     };
     fit();

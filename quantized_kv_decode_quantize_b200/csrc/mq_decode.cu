@@ -29,6 +29,7 @@
 //    completes the tree over the CTA partials and writes out and lse; there is no
 //    second kernel and no CTA ever waits for another.
 #include <cfloat>
+#include <climits>
 
 #include "mq_device.cuh"
 #include "mq_kernels.h"
@@ -55,9 +56,11 @@ struct Cfg {
 };
 
 struct Smem {
-    size_t ring, part, stack, coef, qfrag, flags, mbar, bt, misc, heap, total;
+    size_t ring, part, fin, coef, qfrag, flags, mbar, bt, misc, heap, total;
 };
 
+// W warps, R ring slots per warp, SD partial entries per warp (entry 0 holds the warp's
+// result for the CTA tree; the others are left siblings of its binary counter).
 template <int D, int ROWS>
 __host__ __device__ inline Smem smem_layout(int W, int R, int SD) {
     using C = Cfg<D, ROWS>;
@@ -68,13 +71,13 @@ __host__ __device__ inline Smem smem_layout(int W, int R, int SD) {
     off += (size_t)W * R * C::PB;
     off = al(off, 16);
     s.part = off;
-    off += (size_t)W * C::PART * 4;
+    off += (size_t)W * SD * C::PART * 4;
     s.heap = 0;  // the final merge reuses ring + part
     const size_t heap_bytes = (size_t)2 * kMaxSplits * ROWS * 4 * 4;
     if (off < heap_bytes) off = heap_bytes;
     off = al(off, 16);
-    s.stack = off;
-    off += (size_t)SD * C::PART * 4;
+    s.fin = off;                      // the final merge's result (outside the heap)
+    off += (size_t)C::PART * 4;
     s.coef = off;
     off += (size_t)8 * ROWS * 2 * 4;  // up to 8 merges per phase
     s.qfrag = off;
@@ -85,7 +88,7 @@ __host__ __device__ inline Smem smem_layout(int W, int R, int SD) {
     s.mbar = off;
     off += (size_t)W * R * 8;
     s.bt = off;
-    off += (size_t)W * 2 * kChunkPages * 4;
+    off += (size_t)W * 4 * kChunkPages * 4;
     s.misc = off;
     off += 64;
     s.total = al(off, 128);
@@ -204,10 +207,9 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
     int* misc = reinterpret_cast<int*>(smem + S.misc);
     int* flags = reinterpret_cast<int*>(smem + S.flags);   // [0..W): warp partial empty
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S.mbar) + warp * R;
-    int* bt = reinterpret_cast<int*>(smem + S.bt) + warp * 2 * kChunkPages;
+    int* bt = reinterpret_cast<int*>(smem + S.bt) + warp * 4 * kChunkPages;
     uint8_t* ring = smem + S.ring + (size_t)warp * R * C::PB;
     float* part = reinterpret_cast<float*>(smem + S.part);
-    float* stack = reinterpret_cast<float*>(smem + S.stack);
     float* coef = reinterpret_cast<float*>(smem + S.coef);
 
     // ---- query-row offset of this sequence (sum of n_q of earlier sequences) ----
@@ -292,40 +294,43 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
     }
     __syncthreads();
 
-    // ---- per-warp chunk sequence and page ring ----
+    // ---- this warp's chunks: an aligned run [wc0, wc1) of Q = cpc / W chunks ----
     const uint64_t policy = l2_evict_first_policy();
-    auto chunk_of = [&](int ro) { return c0 + ro * W + warp; };
-    // pages of this warp, in order: all its chunks are full except possibly the last
-    // chunk of the sequence, which is the warp's last
-    int my_pages = 0;
-    for (int ro = 0; ro < n_rounds; ro++) {
-        const int c = chunk_of(ro);
-        if (c < c1) my_pages += min(kChunkPages, n_pages - c * kChunkPages);
-    }
-    auto load_bt = [&](int ro) {
-        const int c = chunk_of(ro);
-        if (ro < n_rounds && c < c1 && lane < kChunkPages) {
-            const int lp = c * kChunkPages + lane;
-            int blk = -1;
-            if (lp < n_pages) {
-                blk = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + lp);
-                if (blk < 0 || (long long)blk >= p.n_blocks) {
-                    atomicOr(p.err, kErrBadBlock);
-                    blk = -1;
-                }
+    const int Q = p.cpc / W;
+    const int SD = p.stack_depth;                  // partial entries per warp
+    const int wc0 = c0 + warp * Q;
+    const int my_chunks = max(0, min(wc0 + Q, c1) - wc0);
+    const int my_pages = my_chunks > 0 ? min((wc0 + my_chunks) * kChunkPages, n_pages) - wc0 * kChunkPages : 0;
+    // Block-table entries of the run: a ring of four chunks' entries in shared memory,
+    // fetched two chunks ahead into a register, so that no load is ever waited for.
+    constexpr int kUnused = INT_MIN;
+    auto bt_fetch = [&](int i) -> int {   // entry of page `lane` of the run's chunk i (lanes < 8)
+        int blk = kUnused;
+        if (i < my_chunks && lane < kChunkPages) {
+            const int lp = (wc0 + i) * kChunkPages + lane;
+            if (lp < n_pages) blk = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + lp);
+        }
+        return blk;
+    };
+    auto bt_store = [&](int i, int blk) {
+        if (i < my_chunks && lane < kChunkPages) {
+            if (blk != kUnused && (blk < 0 || (long long)blk >= p.n_blocks)) {
+                atomicOr(p.err, kErrBadBlock);
+                blk = -1;
             }
-            bt[(ro & 1) * kChunkPages + lane] = blk;
+            bt[(i & 3) * kChunkPages + lane] = blk == kUnused ? -1 : blk;
         }
     };
-    auto issue = [&](int k, int slot) {  // lane 0 only: page k of this warp's sequence into `slot`
-        const int blk = bt[((k / kChunkPages) & 1) * kChunkPages + (k % kChunkPages)];
+    bt_store(0, bt_fetch(0));
+    bt_store(1, bt_fetch(1));
+    int bt_next = bt_fetch(2);
+    __syncwarp();
+    auto issue = [&](int k, int slot) {  // lane 0 only: page k of this warp's run into `slot`
+        const int blk = bt[((k / kChunkPages) & 3) * kChunkPages + (k % kChunkPages)];
         const uint8_t* src = p.pool + ((long long)(blk < 0 ? 0 : blk) * p.n_kv_heads + hk) * C::PB;
         mbar_arrive_expect_tx(smem_u32(&bars[slot]), C::PB);
         tma_load_1d(smem_u32(ring + (size_t)slot * C::PB), src, C::PB, smem_u32(&bars[slot]), policy);
     };
-    load_bt(0);
-    load_bt(1);
-    __syncwarp();
     if (lane == 0)
         for (int k = 0; k < R && k < my_pages; k++) issue(k, k);
 
@@ -334,301 +339,340 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
     // 32-bit shared-window addresses: ring slot 0 and this lane's q fragments
     const uint32_t ring_s = smem_u32(ring), lane16 = (uint32_t)lane * 16u;
     const uint32_t qf_s = smem_u32(qfrag_s) + lane16;
+    float* my_ent = part + (size_t)warp * SD * C::PART;   // this warp's partial entries
 
     bool aborted = false;
     int k_abort = 0;       // first page not waited for after a timeout
     int k_next = 0;        // next page of this warp to consume
     int slot = 0;          // its ring slot (k_next % R) and mbarrier phase ((k_next / R) & 1)
     uint32_t phase = 0;
-    int n_stack = 0;       // round-stack entries (uniform)
-    int* stack_level = misc + 4;   // levels of stack entries (up to 12)
 
-    for (int ro = 0; ro < n_rounds; ro++) {
-        const int c = chunk_of(ro);
-        const bool active = c < c1;
-        if (active) {
-            if (ro >= 1) {
-                load_bt(ro + 1);
-                __syncwarp();
+    // The run's result, as (O fragments, m and l of the lane's O rows 8n + 2t + e).
+    float O[C::MTP][C::NTP][4];
+    float mo[C::NTP][2], lo[C::NTP][2];
+    int n_ent = 0;            // binary-counter entries in shared memory (warp-uniform)
+    uint32_t ent_lvl = 0;     // their levels, 4 bits each
+
+    // entry e (left sibling) (+) registers (right sibling) -> registers
+    auto merge_entry = [&](int e) {
+        __syncwarp();
+        const float* ent = my_ent + (size_t)e * C::PART;
+        float ca[C::NTP][2], cb[C::NTP][2];
+#pragma unroll
+        for (int n = 0; n < C::NTP; n++)
+#pragma unroll
+            for (int e2 = 0; e2 < 2; e2++) {
+                const int r = 8 * n + 2 * t + e2;
+                float m, l;
+                merge_coef(ent[ROWS * D + r], ent[ROWS * D + ROWS + r], mo[n][e2], lo[n][e2], m, l, ca[n][e2],
+                           cb[n][e2]);
+                mo[n][e2] = m;
+                lo[n][e2] = l;
             }
-            float O[C::MTP][C::NTP][4];
 #pragma unroll
-            for (int j = 0; j < C::MTP; j++)
+        for (int n = 0; n < C::NTP; n++)
 #pragma unroll
-                for (int n = 0; n < C::NTP; n++)
-#pragma unroll
-                    for (int e = 0; e < 4; e++) O[j][n][e] = 0.0f;
-            float mrun[C::SLOTS], lrun[C::SLOTS];
-#pragma unroll
-            for (int k = 0; k < C::SLOTS; k++) {
-                mrun[k] = -INFINITY;
-                lrun[k] = 0.0f;
+            for (int q = 0; q < C::NG; q++) {
+                const int ch = 32 * q + 4 * g, r0 = 8 * n + 2 * t;
+                const float4 L0 = *reinterpret_cast<const float4*>(ent + (size_t)r0 * D + ch);
+                const float4 L1 = *reinterpret_cast<const float4*>(ent + (size_t)(r0 + 1) * D + ch);
+                O[2 * q][n][0] = merge_val(L0.x, O[2 * q][n][0], ca[n][0], cb[n][0]);
+                O[2 * q][n][2] = merge_val(L0.y, O[2 * q][n][2], ca[n][0], cb[n][0]);
+                O[2 * q + 1][n][0] = merge_val(L0.z, O[2 * q + 1][n][0], ca[n][0], cb[n][0]);
+                O[2 * q + 1][n][2] = merge_val(L0.w, O[2 * q + 1][n][2], ca[n][0], cb[n][0]);
+                O[2 * q][n][1] = merge_val(L1.x, O[2 * q][n][1], ca[n][1], cb[n][1]);
+                O[2 * q][n][3] = merge_val(L1.y, O[2 * q][n][3], ca[n][1], cb[n][1]);
+                O[2 * q + 1][n][1] = merge_val(L1.z, O[2 * q + 1][n][1], ca[n][1], cb[n][1]);
+                O[2 * q + 1][n][3] = merge_val(L1.w, O[2 * q + 1][n][3], ca[n][1], cb[n][1]);
             }
-            const int pages_here = min(kChunkPages, n_pages - c * kChunkPages);
-            for (int pi = 0; pi < pages_here; pi++, k_next++) {
-                if (!aborted && !mbar_wait_bounded(smem_u32(&bars[slot]), phase)) {
-                    aborted = true;
-                    k_abort = k_next;
-                    if (lane == 0) atomicOr(p.err, kErrTimeout);
+    };
+    // registers -> entry e (natural layout: O [ROWS][D], m [ROWS], l [ROWS])
+    auto write_entry = [&](int e) {
+        float* ent = my_ent + (size_t)e * C::PART;
+#pragma unroll
+        for (int n = 0; n < C::NTP; n++)
+#pragma unroll
+            for (int q = 0; q < C::NG; q++) {
+                const int ch = 32 * q + 4 * g, r0 = 8 * n + 2 * t;
+                *reinterpret_cast<float4*>(ent + (size_t)r0 * D + ch) =
+                    make_float4(O[2 * q][n][0], O[2 * q][n][2], O[2 * q + 1][n][0], O[2 * q + 1][n][2]);
+                *reinterpret_cast<float4*>(ent + (size_t)(r0 + 1) * D + ch) =
+                    make_float4(O[2 * q][n][1], O[2 * q][n][3], O[2 * q + 1][n][1], O[2 * q + 1][n][3]);
+            }
+        if (g == 0) {
+#pragma unroll
+            for (int n = 0; n < C::NTP; n++)
+#pragma unroll
+                for (int e2 = 0; e2 < 2; e2++) {
+                    ent[ROWS * D + 8 * n + 2 * t + e2] = mo[n][e2];
+                    ent[ROWS * D + ROWS + 8 * n + 2 * t + e2] = lo[n][e2];
                 }
-                const uint32_t pg = ring_s + (uint32_t)slot * C::PB;   // this page
-                const uint32_t pgl = pg + lane16;
-                const int lp = c * kChunkPages + pi;
-                const bool bad = bt[(ro & 1) * kChunkPages + pi] < 0;
-                // every token of the page visible to every row: no per-element masking
-                const bool full = !bad && (lp + 1) * kPageTokens <= lim_min;
+        }
+        __syncwarp();
+    };
 
-                // ---- scores: int8 QK^T on the tensor cores ----
-                const float2 skA = __half22float2(u32_as_h2(ldsa32(pg + k_scale_off(D) + 4 * t)));
-                const float2 skB = __half22float2(u32_as_h2(ldsa32(pg + k_scale_off(D) + 16 + 4 * t)));
-                float z[C::SLOTS][2][2];
+    for (int i = 0; i < my_chunks; i++) {
+        if (i >= 1) {
+            bt_store(i + 1, bt_next);
+            bt_next = bt_fetch(i + 2);
+            __syncwarp();
+        }
+        const int c = wc0 + i;
 #pragma unroll
-                for (int mt = 0; mt < C::MTQ; mt++) {
-                    // the lane's key chunks: token g (n-tile 0) and token g + 8 (n-tile 1)
-                    uint4 kc[C::KCH];
+        for (int j = 0; j < C::MTP; j++)
 #pragma unroll
-                    for (int i = 0; i < C::KCH; i++) kc[i] = ldsa128(pgl + i * 512);
-                    int d2[2][4], d0[2][4];
+            for (int n = 0; n < C::NTP; n++)
 #pragma unroll
-                    for (int nt = 0; nt < 2; nt++)
+                for (int e = 0; e < 4; e++) O[j][n][e] = 0.0f;
+        float mrun[C::SLOTS], lrun[C::SLOTS];
 #pragma unroll
-                        for (int i = 0; i < 4; i++) d2[nt][i] = d0[nt][i] = 0;
+        for (int k = 0; k < C::SLOTS; k++) {
+            mrun[k] = -INFINITY;
+            lrun[k] = 0.0f;
+        }
+        const int pages_here = min(kChunkPages, n_pages - c * kChunkPages);
+        for (int pi = 0; pi < pages_here; pi++, k_next++) {
+            if (!aborted && !mbar_wait_bounded(smem_u32(&bars[slot]), phase)) {
+                aborted = true;
+                k_abort = k_next;
+                if (lane == 0) atomicOr(p.err, kErrTimeout);
+            }
+            const uint32_t pg = ring_s + (uint32_t)slot * C::PB;   // this page
+            const uint32_t pgl = pg + lane16;
+            const int lp = c * kChunkPages + pi;
+            const bool bad = bt[(i & 3) * kChunkPages + pi] < 0;
+            // every token of the page visible to every row: no per-element masking
+            const bool full = !bad && (lp + 1) * kPageTokens <= lim_min;
+
+            // ---- scores: int8 QK^T on the tensor cores ----
+            const float2 skA = __half22float2(u32_as_h2(ldsa32(pg + k_scale_off(D) + 4 * t)));
+            const float2 skB = __half22float2(u32_as_h2(ldsa32(pg + k_scale_off(D) + 16 + 4 * t)));
+            float z[C::SLOTS][2][2];
 #pragma unroll
-                    for (int lb = 0; lb < 3; lb++) {
+            for (int mt = 0; mt < C::MTQ; mt++) {
+                // the lane's key chunks: token g (n-tile 0) and token g + 8 (n-tile 1)
+                uint4 kc[C::KCH];
 #pragma unroll
-                        for (int ks = 0; ks < C::KS; ks++) {
-                            uint32_t a[4];
-                            const uint32_t f = qf_s + (((mt * C::KS + ks) * 3 + lb) * 512);
-                            if constexpr (C::HI) {
-                                const uint4 v = ldsa128(f);
-                                a[0] = v.x;
-                                a[1] = v.y;
-                                a[2] = v.z;
-                                a[3] = v.w;
-                            } else {   // rows g + 8 are padding: their fragment registers are zero
-                                const uint2 v = ldsa64(f);
-                                a[0] = v.x;
-                                a[1] = 0u;
-                                a[2] = v.y;
-                                a[3] = 0u;
-                            }
+                for (int ii = 0; ii < C::KCH; ii++) kc[ii] = ldsa128(pgl + ii * 512);
+                // int32 chains per limb and n-tile (exact, so any order).  The 8-row class
+                // keeps the three limbs apart for ILP; the larger classes, short of
+                // registers, shift the top limb in place before the middle one joins it.
+                constexpr bool SPLIT3 = ROWS == 8;
+                int d2[2][4], d1[SPLIT3 ? 2 : 1][4], d0[2][4];
 #pragma unroll
-                            for (int nt = 0; nt < 2; nt++) {
-                                const uint4 ch = kc[nt * (D / 64) + ks / 2];
-                                const uint32_t b0 = (ks & 1) ? ch.z : ch.x;
-                                const uint32_t b1 = (ks & 1) ? ch.w : ch.y;
-                                if (lb == 0) mma_s8s8(d2[nt], a, b0, b1);
-                                else if (lb == 1) mma_u8s8(d2[nt], a, b0, b1);
-                                else mma_u8s8(d0[nt], a, b0, b1);
-                            }
+                for (int nt = 0; nt < 2; nt++)
+#pragma unroll
+                    for (int ii = 0; ii < 4; ii++) {
+                        d2[nt][ii] = d0[nt][ii] = 0;
+                        if constexpr (SPLIT3) d1[nt][ii] = 0;
+                    }
+#pragma unroll
+                for (int lb = 0; lb < 3; lb++) {
+#pragma unroll
+                    for (int ks = 0; ks < C::KS; ks++) {
+                        uint32_t a[4];
+                        const uint32_t f = qf_s + (((mt * C::KS + ks) * 3 + lb) * 512);
+                        if constexpr (C::HI) {
+                            const uint4 v = ldsa128(f);
+                            a[0] = v.x;
+                            a[1] = v.y;
+                            a[2] = v.z;
+                            a[3] = v.w;
+                        } else {   // rows g + 8 are padding: their fragment registers are zero
+                            const uint2 v = ldsa64(f);
+                            a[0] = v.x;
+                            a[1] = 0u;
+                            a[2] = v.y;
+                            a[3] = 0u;
                         }
+#pragma unroll
+                        for (int nt = 0; nt < 2; nt++) {
+                            const uint4 ch = kc[nt * (D / 64) + ks / 2];
+                            const uint32_t b0 = (ks & 1) ? ch.z : ch.x;
+                            const uint32_t b1 = (ks & 1) ? ch.w : ch.y;
+                            if (lb == 0) mma_s8s8(d2[nt], a, b0, b1);
+                            else if (lb == 1) {
+                                if constexpr (SPLIT3) mma_u8s8(d1[nt], a, b0, b1);
+                                else mma_u8s8(d2[nt], a, b0, b1);
+                            } else mma_u8s8(d0[nt], a, b0, b1);
+                        }
+                    }
+                    if constexpr (!SPLIT3) {
                         if (lb == 0) {
 #pragma unroll
                             for (int nt = 0; nt < 2; nt++)
 #pragma unroll
-                                for (int i = 0; i < 4; i++)
-                                    if (16 * mt + 8 * (i / 2) < ROWS) d2[nt][i] <<= 8;
+                                for (int ii = 0; ii < 4; ii++)
+                                    if (16 * mt + 8 * (ii / 2) < ROWS) d2[nt][ii] <<= 8;
                         }
                     }
-#pragma unroll
-                    for (int nt = 0; nt < 2; nt++)
-#pragma unroll
-                        for (int h = 0; h < 2; h++) {
-                            if (16 * mt + 8 * h < ROWS) {
-                                const int k = 2 * mt + h;
-#pragma unroll
-                                for (int e = 0; e < 2; e++) {
-                                    const float s = __fmaf_rn((float)d2[nt][2 * h + e], 256.0f, (float)d0[nt][2 * h + e]);
-                                    const float skv = nt == 0 ? (e == 0 ? skA.x : skA.y) : (e == 0 ? skB.x : skB.y);
-                                    z[k][nt][e] = __fmul_rn(__fmul_rn(s, crow[k]), skv);
-                                }
-                            }
-                        }
                 }
-
-                // ---- online softmax (log2 units) ----
-                const int tok0 = lp * kPageTokens + 2 * t;
-                float pw[C::SLOTS][2][2], alph[C::SLOTS];
-                bool resc = false;
 #pragma unroll
-                for (int k = 0; k < C::SLOTS; k++) {
-                    if (!full) {
+                for (int nt = 0; nt < 2; nt++)
 #pragma unroll
-                        for (int nt = 0; nt < 2; nt++)
+                    for (int h = 0; h < 2; h++) {
+                        if (16 * mt + 8 * h < ROWS) {
+                            const int k = 2 * mt + h;
 #pragma unroll
                             for (int e = 0; e < 2; e++) {
-                                const bool valid = !bad && (tok0 + 8 * nt + e) < lim[k];
-                                z[k][nt][e] = valid ? z[k][nt][e] : -INFINITY;
+                                int d21;
+                                if constexpr (SPLIT3) d21 = (d2[nt][2 * h + e] << 8) + d1[nt][2 * h + e];
+                                else d21 = d2[nt][2 * h + e];
+                                const float sc = __fmaf_rn((float)d21, 256.0f, (float)d0[nt][2 * h + e]);
+                                const float skv = nt == 0 ? (e == 0 ? skA.x : skA.y) : (e == 0 ? skB.x : skB.y);
+                                z[k][nt][e] = __fmul_rn(__fmul_rn(sc, crow[k]), skv);
                             }
+                        }
                     }
-                    float pm = fmaxf(fmaxf(z[k][0][0], z[k][0][1]), fmaxf(z[k][1][0], z[k][1][1]));
-                    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 1));
-                    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 2));
-                    // Lazy reference: the row's reference max moves only when a page max
-                    // exceeds it by more than kLazy (log2 units), so p = 2^(z - m) <= 2^kLazy
-                    // and a rescale of O is rare.  The first finite page max always moves it
-                    // (O is still zero then, so that rescale is skipped).
-                    const float mnew = (pm > __fadd_rn(mrun[k], kLazy)) ? pm : mrun[k];
-                    alph[k] = (mnew == mrun[k]) ? 1.0f : ex2(__fsub_rn(mrun[k], mnew));
-                    resc |= (alph[k] != 1.0f) && (mrun[k] != -INFINITY);
+            }
+
+            // ---- online softmax (log2 units) ----
+            const int tok0 = lp * kPageTokens + 2 * t;
+            float pw[C::SLOTS][2][2], alph[C::SLOTS];
+            bool resc = false;
+#pragma unroll
+            for (int k = 0; k < C::SLOTS; k++) {
+                if (!full) {
 #pragma unroll
                     for (int nt = 0; nt < 2; nt++)
 #pragma unroll
                         for (int e = 0; e < 2; e++) {
-                            const float pv = ex2(__fsub_rn(z[k][nt][e], mnew));
-                            pw[k][nt][e] = full ? pv : (z[k][nt][e] == -INFINITY ? 0.0f : pv);
+                            const bool valid = !bad && (tok0 + 8 * nt + e) < lim[k];
+                            z[k][nt][e] = valid ? z[k][nt][e] : -INFINITY;
                         }
-                    const float ps = __fadd_rn(__fadd_rn(pw[k][0][0], pw[k][0][1]), __fadd_rn(pw[k][1][0], pw[k][1][1]));
-                    lrun[k] = __fadd_rn(__fmul_rn(lrun[k], alph[k]), ps);
-                    mrun[k] = mnew;
                 }
-                // rescaling by exactly 1 changes nothing, so it is skipped when no row's
-                // running max moved (the common case after the first pages of a chunk)
-                if (__any_sync(FULL, resc)) {
+                float pm = fmaxf(fmaxf(z[k][0][0], z[k][0][1]), fmaxf(z[k][1][0], z[k][1][1]));
+                pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 1));
+                pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 2));
+                // Lazy reference: the row's reference max moves only when a page max
+                // exceeds it by more than kLazy (log2 units), so p = 2^(z - m) <= 2^kLazy
+                // and a rescale of O is rare.  The first finite page max always moves it
+                // (O is still zero then, so that rescale is skipped).
+                const float mnew = (pm > __fadd_rn(mrun[k], kLazy)) ? pm : mrun[k];
+                alph[k] = (mnew == mrun[k]) ? 1.0f : ex2(__fsub_rn(mrun[k], mnew));
+                resc |= (alph[k] != 1.0f) && (mrun[k] != -INFINITY);
 #pragma unroll
-                    for (int n = 0; n < C::NTP; n++) {
-                        const float a0 = __shfl_sync(FULL, alph[n], 8 * t);
-                        const float a1 = __shfl_sync(FULL, alph[n], 8 * t + 4);
+                for (int nt = 0; nt < 2; nt++)
 #pragma unroll
-                        for (int j = 0; j < C::MTP; j++) {
-                            O[j][n][0] = __fmul_rn(O[j][n][0], a0);
-                            O[j][n][1] = __fmul_rn(O[j][n][1], a1);
-                            O[j][n][2] = __fmul_rn(O[j][n][2], a0);
-                            O[j][n][3] = __fmul_rn(O[j][n][3], a1);
-                        }
+                    for (int e = 0; e < 2; e++) {
+                        const float pv = ex2(__fsub_rn(z[k][nt][e], mnew));
+                        pw[k][nt][e] = full ? pv : (z[k][nt][e] == -INFINITY ? 0.0f : pv);
+                    }
+                const float ps = __fadd_rn(__fadd_rn(pw[k][0][0], pw[k][0][1]), __fadd_rn(pw[k][1][0], pw[k][1][1]));
+                lrun[k] = __fadd_rn(__fmul_rn(lrun[k], alph[k]), ps);
+                mrun[k] = mnew;
+            }
+            // rescaling by exactly 1 changes nothing, so it is skipped when no row's
+            // reference moved (the common case)
+            if (__any_sync(FULL, resc)) {
+#pragma unroll
+                for (int n = 0; n < C::NTP; n++) {
+                    const float a0 = __shfl_sync(FULL, alph[n], 8 * t);
+                    const float a1 = __shfl_sync(FULL, alph[n], 8 * t + 4);
+#pragma unroll
+                    for (int j = 0; j < C::MTP; j++) {
+                        O[j][n][0] = __fmul_rn(O[j][n][0], a0);
+                        O[j][n][1] = __fmul_rn(O[j][n][1], a1);
+                        O[j][n][2] = __fmul_rn(O[j][n][2], a0);
+                        O[j][n][3] = __fmul_rn(O[j][n][3], a1);
                     }
                 }
+            }
 
-                // ---- P.V: int4 codes as exact fp16, weights p * s_v in fp16 ----
-                uint4 vcw[C::VCH], svw[C::SCH];
+            // ---- P.V: int4 codes as exact fp16, weights p * s_v in fp16 ----
+            uint4 vcw[C::VCH], svw[C::SCH];
 #pragma unroll
-                for (int i = 0; i < C::VCH; i++) vcw[i] = ldsa128(pgl + v_code_off(D) + i * 512);
+            for (int ii = 0; ii < C::VCH; ii++) vcw[ii] = ldsa128(pgl + v_code_off(D) + ii * 512);
 #pragma unroll
-                for (int i = 0; i < C::SCH; i++) svw[i] = ldsa128(pg + v_scale_off(D) + t * (C::NG * 8) + i * 16);
+            for (int ii = 0; ii < C::SCH; ii++) svw[ii] = ldsa128(pg + v_scale_off(D) + t * (C::NG * 8) + ii * 16);
 #pragma unroll
-                for (int q = 0; q < C::NG; q++) {
-                    const float2 s0 = __half22float2(u32_as_h2(comp(svw[(2 * q) / 4], (2 * q) % 4)));
-                    const float2 s1 = __half22float2(u32_as_h2(comp(svw[(2 * q + 1) / 4], (2 * q + 1) % 4)));
-                    const uint32_t x0 = comp(vcw[(2 * q) / 4], (2 * q) % 4);
-                    const uint32_t x1 = comp(vcw[(2 * q + 1) / 4], (2 * q + 1) % 4);
-                    const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
-                    const uint32_t A0 = nib_lo_to_h2(x0), A1 = nib_hi_to_h2(x0);
-                    const uint32_t A2 = nib_lo_to_h2(x1), A3 = nib_hi_to_h2(x1);
-                    const uint32_t B0 = nib_lo_to_h2(y0), B1 = nib_hi_to_h2(y0);
-                    const uint32_t B2 = nib_lo_to_h2(y1), B3 = nib_hi_to_h2(y1);
+            for (int q = 0; q < C::NG; q++) {
+                const float2 s0 = __half22float2(u32_as_h2(comp(svw[(2 * q) / 4], (2 * q) % 4)));
+                const float2 s1 = __half22float2(u32_as_h2(comp(svw[(2 * q + 1) / 4], (2 * q + 1) % 4)));
+                const uint32_t x0 = comp(vcw[(2 * q) / 4], (2 * q) % 4);
+                const uint32_t x1 = comp(vcw[(2 * q + 1) / 4], (2 * q + 1) % 4);
+                const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
+                const uint32_t A0 = nib_lo_to_h2(x0), A1 = nib_hi_to_h2(x0);
+                const uint32_t A2 = nib_lo_to_h2(x1), A3 = nib_hi_to_h2(x1);
+                const uint32_t B0 = nib_lo_to_h2(y0), B1 = nib_hi_to_h2(y0);
+                const uint32_t B2 = nib_lo_to_h2(y1), B3 = nib_hi_to_h2(y1);
 #pragma unroll
-                    for (int n = 0; n < C::NTP; n++) {
-                        float w00 = __fmul_rn(pw[n][0][0], s0.x), w01 = __fmul_rn(pw[n][0][1], s0.y);
-                        float w10 = __fmul_rn(pw[n][1][0], s1.x), w11 = __fmul_rn(pw[n][1][1], s1.y);
-                        if (!full) {  // masked tokens may sit next to unwritten (non-finite) scales
-                            w00 = pw[n][0][0] == 0.0f ? 0.0f : w00;
-                            w01 = pw[n][0][1] == 0.0f ? 0.0f : w01;
-                            w10 = pw[n][1][0] == 0.0f ? 0.0f : w10;
-                            w11 = pw[n][1][1] == 0.0f ? 0.0f : w11;
-                        }
-                        const uint32_t bb0 = pack_h2(w00, w01), bb1 = pack_h2(w10, w11);
-                        mma_f16(O[2 * q][n], A0, A1, A2, A3, bb0, bb1);
-                        mma_f16(O[2 * q + 1][n], B0, B1, B2, B3, bb0, bb1);
+                for (int n = 0; n < C::NTP; n++) {
+                    float w00 = __fmul_rn(pw[n][0][0], s0.x), w01 = __fmul_rn(pw[n][0][1], s0.y);
+                    float w10 = __fmul_rn(pw[n][1][0], s1.x), w11 = __fmul_rn(pw[n][1][1], s1.y);
+                    if (!full) {  // masked tokens may sit next to unwritten (non-finite) scales
+                        w00 = pw[n][0][0] == 0.0f ? 0.0f : w00;
+                        w01 = pw[n][0][1] == 0.0f ? 0.0f : w01;
+                        w10 = pw[n][1][0] == 0.0f ? 0.0f : w10;
+                        w11 = pw[n][1][1] == 0.0f ? 0.0f : w11;
                     }
-                }
-                __syncwarp();
-                if (lane == 0 && !aborted && k_next + R < my_pages) {
-                    fence_proxy_async_smem();
-                    issue(k_next + R, slot);
-                }
-                if (++slot == R) {
-                    slot = 0;
-                    phase ^= 1u;
+                    const uint32_t bb0 = pack_h2(w00, w01), bb1 = pack_h2(w10, w11);
+                    mma_f16(O[2 * q][n], A0, A1, A2, A3, bb0, bb1);
+                    mma_f16(O[2 * q + 1][n], B0, B1, B2, B3, bb0, bb1);
                 }
             }
-            // ---- chunk partial -> shared memory (natural layout) ----
-            float* mine = part + (size_t)warp * C::PART;
-#pragma unroll
-            for (int k = 0; k < C::SLOTS; k++) {
-                float l = lrun[k];
-                l = __fadd_rn(l, __shfl_xor_sync(FULL, l, 1));
-                l = __fadd_rn(l, __shfl_xor_sync(FULL, l, 2));
-                if (t == 0) {
-                    mine[ROWS * D + 8 * k + g] = mrun[k];
-                    mine[ROWS * D + ROWS + 8 * k + g] = l;
-                }
+            // every lane has consumed the page (its loads fed the math above): refill
+            // the slot.  The reads are complete, so the bulk copy cannot overtake them.
+            __syncwarp();
+            if (lane == 0 && !aborted && k_next + R < my_pages) issue(k_next + R, slot);
+            if (++slot == R) {
+                slot = 0;
+                phase ^= 1u;
             }
-#pragma unroll
-            for (int n = 0; n < C::NTP; n++)
-#pragma unroll
-                for (int q = 0; q < C::NG; q++) {
-                    const int ch = 32 * q + 4 * g;
-                    const int r0 = 8 * n + 2 * t;
-                    *reinterpret_cast<float4*>(mine + (size_t)r0 * D + ch) =
-                        make_float4(O[2 * q][n][0], O[2 * q][n][2], O[2 * q + 1][n][0], O[2 * q + 1][n][2]);
-                    *reinterpret_cast<float4*>(mine + (size_t)(r0 + 1) * D + ch) =
-                        make_float4(O[2 * q][n][1], O[2 * q][n][3], O[2 * q + 1][n][1], O[2 * q + 1][n][3]);
-                }
         }
-        if (lane == 0) flags[warp] = active ? 0 : 1;
-        __syncthreads();
-
-        // ---- tree over the W chunk partials of this round -> part[0] ----
-        for (int s = 1; s < W; s <<= 1) {
-            float* dsts[8];
-            const float* srcs[8];
-            int n_m = 0;
-            for (int w = 0; w + s < W; w += 2 * s) {
-                dsts[n_m] = part + (size_t)w * C::PART;
-                srcs[n_m] = part + (size_t)(w + s) * C::PART;
-                n_m++;
-            }
-            // gather empty flags of this level into flags[16..]
-            if (threadIdx.x < n_m) {
-                flags[16 + threadIdx.x] = flags[threadIdx.x * 2 * s];
-                flags[32 + threadIdx.x] = flags[threadIdx.x * 2 * s + s];
-            }
-            __syncthreads();
-            cta_merge<D, ROWS>(dsts, srcs, n_m, flags + 16, flags + 32, coef);
-            if (threadIdx.x < n_m) flags[threadIdx.x * 2 * s] = flags[16 + threadIdx.x];
-            __syncthreads();
+        // ---- chunk result: slot form (rows 8k + g) -> O-row form (rows 8n + 2t + e) ----
+        float lrow[C::SLOTS];
+#pragma unroll
+        for (int k = 0; k < C::SLOTS; k++) {
+            float l = lrun[k];
+            l = __fadd_rn(l, __shfl_xor_sync(FULL, l, 1));
+            l = __fadd_rn(l, __shfl_xor_sync(FULL, l, 2));
+            lrow[k] = l;
         }
-        // ---- push the round result onto the round stack (binary counter) ----
-        {
-            int level = 0;
-            bool in_part = true;
-            float* cur = part;
-            while (n_stack > 0 && stack_level[n_stack - 1] == level) {
-                float* left = stack + (size_t)(n_stack - 1) * C::PART;
-                float* dsts[1] = {left};
-                const float* srcs[1] = {cur};
-                if (threadIdx.x == 0) {
-                    flags[16] = 0;
-                    flags[32] = 0;
-                }
-                __syncthreads();
-                cta_merge<D, ROWS>(dsts, srcs, 1, flags + 16, flags + 32, coef);
-                cur = left;
-                in_part = false;
-                level++;
-                n_stack--;
+#pragma unroll
+        for (int n = 0; n < C::NTP; n++)
+#pragma unroll
+            for (int e2 = 0; e2 < 2; e2++) {
+                mo[n][e2] = __shfl_sync(FULL, mrun[n], 8 * t + 4 * e2);
+                lo[n][e2] = __shfl_sync(FULL, lrow[n], 8 * t + 4 * e2);
             }
-            if (in_part) {
-                float* dst = stack + (size_t)n_stack * C::PART;
-                for (int i = threadIdx.x; i < C::PART / 2; i += blockDim.x)
-                    reinterpret_cast<float2*>(dst)[i] = reinterpret_cast<const float2*>(part)[i];
-            }
-            __syncthreads();
-            if (threadIdx.x == 0) stack_level[n_stack] = level;
-            n_stack++;
-            __syncthreads();
+        // ---- binary counter over the run's chunks (aligned, so it closes the subtree) ----
+        int lvl = 0;
+        while (n_ent > 0 && (int)((ent_lvl >> (4 * (n_ent - 1))) & 15u) == lvl) {
+            merge_entry(n_ent - 1);
+            n_ent--;
+            lvl++;
+        }
+        if (i + 1 < my_chunks) {
+            write_entry(n_ent);
+            ent_lvl = (ent_lvl & ~(15u << (4 * n_ent))) | ((uint32_t)lvl << (4 * n_ent));
+            n_ent++;
         }
     }
-    // ---- fold the round stack right to left -> stack[0] ----
-    for (int i = n_stack - 2; i >= 0; i--) {
-        float* dsts[1] = {stack + (size_t)i * C::PART};
-        const float* srcs[1] = {stack + (size_t)(i + 1) * C::PART};
-        if (threadIdx.x == 0) {
-            flags[16] = 0;
-            flags[32] = 0;
+    // a run cut short by the end of the sequence: fold what is left, right to left
+    for (int e = n_ent - 1; e >= 0; e--) merge_entry(e);
+    if (my_chunks > 0) write_entry(0);
+    if (lane == 0) flags[warp] = my_chunks > 0 ? 0 : 1;
+    __syncthreads();
+
+    // ---- tree over the W warp results (entry 0 of each warp) -> warp 0's entry 0 ----
+    for (int s = 1; s < W; s <<= 1) {
+        float* dsts[8];
+        const float* srcs[8];
+        int n_m = 0;
+        for (int w = 0; w + s < W; w += 2 * s) {
+            dsts[n_m] = part + (size_t)w * SD * C::PART;
+            srcs[n_m] = part + (size_t)(w + s) * SD * C::PART;
+            n_m++;
+        }
+        if (threadIdx.x < n_m) {
+            flags[16 + threadIdx.x] = flags[threadIdx.x * 2 * s];
+            flags[32 + threadIdx.x] = flags[threadIdx.x * 2 * s + s];
         }
         __syncthreads();
-        cta_merge<D, ROWS>(dsts, srcs, 1, flags + 16, flags + 32, coef);
+        cta_merge<D, ROWS>(dsts, srcs, n_m, flags + 16, flags + 32, coef);
+        if (threadIdx.x < n_m) flags[threadIdx.x * 2 * s] = flags[16 + threadIdx.x];
+        __syncthreads();
     }
     // any warp that gave up on a wait: drain its copies still in flight, then stop
     if (aborted) {
@@ -639,7 +683,7 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
     __syncthreads();
     if (misc[1] == 1) return;
 
-    const float* res = stack;
+    const float* res = part;
     const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
     auto finalize = [&](const float* o_src, const float* m_src, const float* l_src) {
         for (int i = threadIdx.x; i < rows_here * (D / 4); i += blockDim.x) {
@@ -670,12 +714,12 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
     for (int i = threadIdx.x; i < ROWS * D / 4; i += blockDim.x)
         reinterpret_cast<float4*>(go)[i] = reinterpret_cast<const float4*>(res)[i];
     for (int i = threadIdx.x; i < 2 * ROWS; i += blockDim.x) gml[i] = res[ROWS * D + i];
-    __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) misc[2] = (atomicAdd(p.counters + pidx, 1u) == (unsigned)(n_splits - 1)) ? 1 : 0;
+    // release: this CTA's partial (written by all threads, ordered by the barrier)
+    // happens-before the count; acquire: the last CTA sees every other CTA's partial
+    if (threadIdx.x == 0) misc[2] = (atom_add_acq_rel_gpu(p.counters + pidx, 1u) == (unsigned)(n_splits - 1)) ? 1 : 0;
     __syncthreads();
     if (misc[2] == 0) return;
-    __threadfence();
 
     // Coefficients of every node of the padded tree over the n_splits CTA partials,
     // heap-indexed (node (level, i) at 2^(H-level) + i), per row: m, l, alpha, beta.
@@ -712,7 +756,7 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
         __syncthreads();
     }
     // Elements: binary counter over the leaves, merging at the padded-tree nodes.
-    float* fin = stack;   // final O [ROWS][D], m, l (this CTA's own partial is in global memory now)
+    float* fin = reinterpret_cast<float*>(smem + S.fin);   // final O [ROWS][D], m, l
     const float* root = hp + (size_t)hidx(H, 0) * ROWS * 4;
     for (int e4 = threadIdx.x; e4 < ROWS * D / 4; e4 += blockDim.x) {
         const int r = (4 * e4) / D;

@@ -48,7 +48,7 @@ struct DecodeParams {
     int n_rb;            // row blocks per kv-head
     int cpc;             // chunks per CTA (power of two >= warps)
     int pages_per_stage; // TMA ring depth per warp
-    int stack_depth;     // round-stack entries in shared memory
+    int stack_depth;     // partial entries per warp in shared memory
     unsigned* err;
 };
 
