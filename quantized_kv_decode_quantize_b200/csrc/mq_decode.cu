@@ -107,54 +107,6 @@ __device__ __forceinline__ float merge_val(float ol, float orr, float a, float b
     return __fadd_rn(__fmul_rn(ol, a), __fmul_rn(orr, b));
 }
 
-// dst[k] = dst[k] (+) src[k] for k < n_merges, cooperative over the CTA.  A partial
-// is O[ROWS][D] followed by m[ROWS], l[ROWS].  empty flags: an empty right side
-// leaves dst unchanged, an empty left side takes a copy of the right side.
-template <int D, int ROWS>
-__device__ void cta_merge(float* const* dst, const float* const* src, int n_merges, int* dst_empty,
-                          const int* src_empty, float* coef) {
-    const int T = blockDim.x;
-    for (int i = threadIdx.x; i < n_merges * ROWS; i += T) {
-        const int k = i / ROWS, r = i % ROWS;
-        float* d = dst[k];
-        const float* s = src[k];
-        if (src_empty[k]) continue;
-        if (dst_empty[k]) {
-            d[ROWS * D + r] = s[ROWS * D + r];
-            d[ROWS * D + ROWS + r] = s[ROWS * D + ROWS + r];
-            continue;
-        }
-        float m, l, a, b;
-        merge_coef(d[ROWS * D + r], d[ROWS * D + ROWS + r], s[ROWS * D + r], s[ROWS * D + ROWS + r], m, l, a, b);
-        coef[2 * i] = a;
-        coef[2 * i + 1] = b;
-        d[ROWS * D + r] = m;
-        d[ROWS * D + ROWS + r] = l;
-    }
-    __syncthreads();
-    constexpr int V4 = ROWS * D / 4;
-    for (int i = threadIdx.x; i < n_merges * V4; i += T) {
-        const int k = i / V4, e = i % V4, r = (4 * e) / D;
-        if (src_empty[k]) continue;
-        float4* d = reinterpret_cast<float4*>(dst[k]) + e;
-        const float4 s = reinterpret_cast<const float4*>(src[k])[e];
-        if (dst_empty[k]) {
-            *d = s;
-            continue;
-        }
-        const float a = coef[2 * (k * ROWS + r)], b = coef[2 * (k * ROWS + r) + 1];
-        float4 o = *d;
-        o.x = merge_val(o.x, s.x, a, b);
-        o.y = merge_val(o.y, s.y, a, b);
-        o.z = merge_val(o.z, s.z, a, b);
-        o.w = merge_val(o.w, s.w, a, b);
-        *d = o;
-    }
-    __syncthreads();
-    if (threadIdx.x < n_merges && !src_empty[threadIdx.x]) dst_empty[threadIdx.x] = 0;
-    __syncthreads();
-}
-
 template <typename T>
 __device__ __forceinline__ float ld_f32(const void* base, size_t i);
 template <>
@@ -411,6 +363,64 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
         __syncwarp();
     };
 
+    // registers (left sibling) (+) entry (right sibling) -> registers
+    auto merge_right = [&](const float* ent) {
+        float ca[C::NTP][2], cb[C::NTP][2];
+#pragma unroll
+        for (int n = 0; n < C::NTP; n++)
+#pragma unroll
+            for (int e2 = 0; e2 < 2; e2++) {
+                const int r = 8 * n + 2 * t + e2;
+                float m, l;
+                merge_coef(mo[n][e2], lo[n][e2], ent[ROWS * D + r], ent[ROWS * D + ROWS + r], m, l, ca[n][e2],
+                           cb[n][e2]);
+                mo[n][e2] = m;
+                lo[n][e2] = l;
+            }
+#pragma unroll
+        for (int n = 0; n < C::NTP; n++)
+#pragma unroll
+            for (int q = 0; q < C::NG; q++) {
+                const int ch = 32 * q + 4 * g, r0 = 8 * n + 2 * t;
+                const float4 R0 = *reinterpret_cast<const float4*>(ent + (size_t)r0 * D + ch);
+                const float4 R1 = *reinterpret_cast<const float4*>(ent + (size_t)(r0 + 1) * D + ch);
+                O[2 * q][n][0] = merge_val(O[2 * q][n][0], R0.x, ca[n][0], cb[n][0]);
+                O[2 * q][n][2] = merge_val(O[2 * q][n][2], R0.y, ca[n][0], cb[n][0]);
+                O[2 * q + 1][n][0] = merge_val(O[2 * q + 1][n][0], R0.z, ca[n][0], cb[n][0]);
+                O[2 * q + 1][n][2] = merge_val(O[2 * q + 1][n][2], R0.w, ca[n][0], cb[n][0]);
+                O[2 * q][n][1] = merge_val(O[2 * q][n][1], R1.x, ca[n][1], cb[n][1]);
+                O[2 * q][n][3] = merge_val(O[2 * q][n][3], R1.y, ca[n][1], cb[n][1]);
+                O[2 * q + 1][n][1] = merge_val(O[2 * q + 1][n][1], R1.z, ca[n][1], cb[n][1]);
+                O[2 * q + 1][n][3] = merge_val(O[2 * q + 1][n][3], R1.w, ca[n][1], cb[n][1]);
+            }
+    };
+    // entry -> registers
+    auto load_entry = [&](const float* ent) {
+#pragma unroll
+        for (int n = 0; n < C::NTP; n++)
+#pragma unroll
+            for (int e2 = 0; e2 < 2; e2++) {
+                mo[n][e2] = ent[ROWS * D + 8 * n + 2 * t + e2];
+                lo[n][e2] = ent[ROWS * D + ROWS + 8 * n + 2 * t + e2];
+            }
+#pragma unroll
+        for (int n = 0; n < C::NTP; n++)
+#pragma unroll
+            for (int q = 0; q < C::NG; q++) {
+                const int ch = 32 * q + 4 * g, r0 = 8 * n + 2 * t;
+                const float4 R0 = *reinterpret_cast<const float4*>(ent + (size_t)r0 * D + ch);
+                const float4 R1 = *reinterpret_cast<const float4*>(ent + (size_t)(r0 + 1) * D + ch);
+                O[2 * q][n][0] = R0.x;
+                O[2 * q][n][2] = R0.y;
+                O[2 * q + 1][n][0] = R0.z;
+                O[2 * q + 1][n][2] = R0.w;
+                O[2 * q][n][1] = R1.x;
+                O[2 * q][n][3] = R1.y;
+                O[2 * q + 1][n][1] = R1.z;
+                O[2 * q + 1][n][3] = R1.w;
+            }
+    };
+
     for (int i = 0; i < my_chunks; i++) {
         if (i >= 1) {
             bt_store(i + 1, bt_next);
@@ -651,27 +661,28 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
     }
     // a run cut short by the end of the sequence: fold what is left, right to left
     for (int e = n_ent - 1; e >= 0; e--) merge_entry(e);
-    if (my_chunks > 0) write_entry(0);
-    if (lane == 0) flags[warp] = my_chunks > 0 ? 0 : 1;
-    __syncthreads();
 
-    // ---- tree over the W warp results (entry 0 of each warp) -> warp 0's entry 0 ----
+    // ---- tree over the W warp results, in registers: at level s the left warp of
+    // each pair merges its right sibling's entry; a warp that is a right sibling at
+    // the next level publishes its merged result to its entry 0 ----
+    bool have = my_chunks > 0;
+    if (have) write_entry(0);
+    if (lane == 0) flags[warp] = have ? 0 : 1;
+    __syncthreads();
     for (int s = 1; s < W; s <<= 1) {
-        float* dsts[8];
-        const float* srcs[8];
-        int n_m = 0;
-        for (int w = 0; w + s < W; w += 2 * s) {
-            dsts[n_m] = part + (size_t)w * SD * C::PART;
-            srcs[n_m] = part + (size_t)(w + s) * SD * C::PART;
-            n_m++;
+        if ((warp & (2 * s - 1)) == 0 && warp + s < W && flags[warp + s] == 0) {
+            const float* rent = part + (size_t)(warp + s) * SD * C::PART;
+            if (have) {
+                merge_right(rent);
+            } else {
+                load_entry(rent);
+                have = true;
+            }
+            if ((warp & (4 * s - 1)) == 2 * s) {
+                write_entry(0);
+                if (lane == 0) flags[warp] = 0;
+            }
         }
-        if (threadIdx.x < n_m) {
-            flags[16 + threadIdx.x] = flags[threadIdx.x * 2 * s];
-            flags[32 + threadIdx.x] = flags[threadIdx.x * 2 * s + s];
-        }
-        __syncthreads();
-        cta_merge<D, ROWS>(dsts, srcs, n_m, flags + 16, flags + 32, coef);
-        if (threadIdx.x < n_m) flags[threadIdx.x * 2 * s] = flags[16 + threadIdx.x];
         __syncthreads();
     }
     // any warp that gave up on a wait: drain its copies still in flight, then stop
@@ -683,8 +694,9 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
     __syncthreads();
     if (misc[1] == 1) return;
 
-    const float* res = part;
     const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
+    // out = O / l and lse for the real rows of this block; (o_src, m_src, l_src) in the
+    // natural layout (shared memory)
     auto finalize = [&](const float* o_src, const float* m_src, const float* l_src) {
         for (int i = threadIdx.x; i < rows_here * (D / 4); i += blockDim.x) {
             const int rl = i / (D / 4), c4 = i % (D / 4);
@@ -704,16 +716,20 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
         }
     };
 
+    if (warp == 0) write_entry(0);   // the CTA's result, natural layout
+    __syncthreads();
     if (n_splits == 1) {
-        finalize(res, res + ROWS * D, res + ROWS * D + ROWS);
+        finalize(part, part + ROWS * D, part + ROWS * D + ROWS);
         return;
     }
     // ---- publish this CTA's partial; the last CTA completes the tree ----
-    float* go = p.part_o + (pidx * kMaxSplits + sp) * (size_t)(ROWS * D);
-    float* gml = p.part_ml + (pidx * kMaxSplits + sp) * (size_t)(2 * ROWS);
-    for (int i = threadIdx.x; i < ROWS * D / 4; i += blockDim.x)
-        reinterpret_cast<float4*>(go)[i] = reinterpret_cast<const float4*>(res)[i];
-    for (int i = threadIdx.x; i < 2 * ROWS; i += blockDim.x) gml[i] = res[ROWS * D + i];
+    {
+        float* go = p.part_o + (pidx * kMaxSplits + sp) * (size_t)(ROWS * D);
+        float* gml = p.part_ml + (pidx * kMaxSplits + sp) * (size_t)(2 * ROWS);
+        for (int i = threadIdx.x; i < ROWS * D / 4; i += blockDim.x)
+            __stcg(reinterpret_cast<float4*>(go) + i, reinterpret_cast<const float4*>(part)[i]);
+        for (int i = threadIdx.x; i < 2 * ROWS; i += blockDim.x) __stcg(gml + i, part[ROWS * D + i]);
+    }
     __syncthreads();
     // release: this CTA's partial (written by all threads, ordered by the barrier)
     // happens-before the count; acquire: the last CTA sees every other CTA's partial
@@ -755,45 +771,57 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
         }
         __syncthreads();
     }
-    // Elements: binary counter over the leaves, merging at the padded-tree nodes.
+    // Elements: the padded tree evaluated level by level in registers, eight leaves
+    // (an aligned level-3 subtree) at a time, their loads all in flight together.
     float* fin = reinterpret_cast<float*>(smem + S.fin);   // final O [ROWS][D], m, l
     const float* root = hp + (size_t)hidx(H, 0) * ROWS * 4;
+    const int n_groups = (n_splits + 7) >> 3;
     for (int e4 = threadIdx.x; e4 < ROWS * D / 4; e4 += blockDim.x) {
         const int r = (4 * e4) / D;
-        float4 st[kMaxSplits == 64 ? 7 : 12];
-        int lvl[kMaxSplits == 64 ? 7 : 12], beg[kMaxSplits == 64 ? 7 : 12];
-        int n_st = 0;
-        for (int s = 0; s < n_splits; s++) {
-            float4 cur = __ldcg(reinterpret_cast<const float4*>(go0 + (size_t)s * ROWS * D) + e4);
-            int cl = 0, cb = s;
-            while (n_st > 0 && lvl[n_st - 1] == cl) {
-                const int a = beg[n_st - 1];
-                const float* nd = hp + ((size_t)hidx(cl + 1, a >> (cl + 1)) * ROWS + r) * 4;
-                const float4 lf = st[n_st - 1];
-                cur.x = merge_val(lf.x, cur.x, nd[2], nd[3]);
-                cur.y = merge_val(lf.y, cur.y, nd[2], nd[3]);
-                cur.z = merge_val(lf.z, cur.z, nd[2], nd[3]);
-                cur.w = merge_val(lf.w, cur.w, nd[2], nd[3]);
-                cl++;
-                cb = a;
-                n_st--;
+        auto node_merge = [&](float4 lf, float4 rt, int level, int idx) {
+            const float* nd = hp + ((size_t)hidx(level, idx) * ROWS + r) * 4;
+            float4 o;
+            o.x = merge_val(lf.x, rt.x, nd[2], nd[3]);
+            o.y = merge_val(lf.y, rt.y, nd[2], nd[3]);
+            o.z = merge_val(lf.z, rt.z, nd[2], nd[3]);
+            o.w = merge_val(lf.w, rt.w, nd[2], nd[3]);
+            return o;
+        };
+        float4 gv[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            if (j < n_groups) {
+                float4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; u++) {
+                    const int sidx = 8 * j + u;
+                    v[u] = sidx < n_splits ? __ldcg(reinterpret_cast<const float4*>(go0 + (size_t)sidx * ROWS * D) + e4)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int lv = 1; lv <= 3; lv++) {
+#pragma unroll
+                    for (int u = 0; u < (8 >> lv); u++) {
+                        const int idx = ((8 * j) >> lv) + u;           // node (lv, idx)
+                        const bool has_right = (2 * idx + 1) * (1 << (lv - 1)) < n_splits;
+                        if (lv <= H) v[u] = has_right ? node_merge(v[2 * u], v[2 * u + 1], lv, idx) : v[2 * u];
+                    }
+                }
+                gv[j] = v[0];
             }
-            st[n_st] = cur;
-            lvl[n_st] = cl;
-            beg[n_st] = cb;
-            n_st++;
         }
-        float4 acc = st[n_st - 1];
-        for (int i = n_st - 2; i >= 0; i--) {
-            const int a = beg[i], cl = lvl[i];
-            const float* nd = hp + ((size_t)hidx(cl + 1, a >> (cl + 1)) * ROWS + r) * 4;
-            const float4 lf = st[i];
-            acc.x = merge_val(lf.x, acc.x, nd[2], nd[3]);
-            acc.y = merge_val(lf.y, acc.y, nd[2], nd[3]);
-            acc.z = merge_val(lf.z, acc.z, nd[2], nd[3]);
-            acc.w = merge_val(lf.w, acc.w, nd[2], nd[3]);
+        // levels 4 .. H over the group nodes
+#pragma unroll
+        for (int lv = 4; lv <= 6; lv++) {
+#pragma unroll
+            for (int u = 0; u < (64 >> lv); u++) {
+                if (lv <= H && u * (1 << lv) < n_splits) {
+                    const bool has_right = (2 * u + 1) * (1 << (lv - 1)) < n_splits;
+                    gv[u] = has_right ? node_merge(gv[2 * u], gv[2 * u + 1], lv, u) : gv[2 * u];
+                }
+            }
         }
-        reinterpret_cast<float4*>(fin)[e4] = acc;
+        reinterpret_cast<float4*>(fin)[e4] = gv[0];
     }
     float* fml = fin + ROWS * D;
     for (int r = threadIdx.x; r < ROWS; r += blockDim.x) {
