@@ -197,7 +197,9 @@ mq_status mq_kv_append(mq_cache* cache, const void* k, const void* v, mq_dtype d
  * Errors: INVALID_ARG (null pointers, n_seqs < 1 or > 65535, n_q_heads not a
  * multiple of n_kv_heads, total_q < 1, max_q_per_seq < 1, max_seq_len <
  * max_q_per_seq, a non-finite softmax_scale, out not 16-byte aligned), UNSUPPORTED
- * (n_q_heads/n_kv_heads * max_q_per_seq > 64, q dtype), CAPACITY (max_seq_len >
+ * (n_q_heads/n_kv_heads * max_q_per_seq > 64, q dtype, head_dim 256 with
+ * max_seq_len > 524288: the per-warp partial stack no longer fits in shared
+ * memory), CAPACITY (max_seq_len >
  * max_blocks_per_seq * 16), WORKSPACE, CUDA.  A sequence whose L_b / n_b break
  * the bounds above is skipped by the kernel and reported by mq_device_status().
  * ------------------------------------------------------------------------- */

@@ -62,11 +62,10 @@ DevGuard::~DevGuard() {
     if (switched && prev >= 0) cudaSetDevice(prev);
 }
 
-DecodePlan plan_decode(const mq_cache* c, int n_seqs, int n_q_heads, int max_q, int max_seq_len) {
+// The plan for one row class: rows per CTA, launch shape, chunks per CTA.
+static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int rows_total, int max_seq_len) {
     DecodePlan pl{};
-    const int G = n_q_heads / c->n_kv_heads;
-    const int rows_total = G * max_q;
-    pl.cls = rows_class_for(c->head_dim, rows_total);
+    pl.cls = cls;
     pl.rows = rows_class_rows(c->head_dim, pl.cls);
     pl.n_rb = (rows_total + pl.rows - 1) / pl.rows;
     const mq_decode_config cfg = c->cfg[pl.cls];
@@ -92,15 +91,35 @@ DecodePlan plan_decode(const mq_cache* c, int n_seqs, int n_q_heads, int max_q, 
     };
     fit();
     // A configuration that does not fit in shared memory runs with a shallower ring,
-    // then with 4 warps; the arithmetic (and so the output) is the same.
-    while (pl.smem > (size_t)c->max_smem && pl.pages_per_stage > 2) {
-        pl.pages_per_stage--;
+    // then with shorter warp runs (more CTAs per sequence, while the split count stays
+    // within kMaxSplits), then with 4 warps.  The chunk tree is fixed by the chunk
+    // indices alone, so the arithmetic (and so the output) is the same.
+    while (pl.smem > (size_t)c->max_smem) {
+        if (pl.pages_per_stage > 2) {
+            pl.pages_per_stage--;
+        } else if (pl.cpc > pl.warps && (max_chunks + pl.cpc / 2 - 1) / (pl.cpc / 2) <= kMaxSplits) {
+            pl.cpc /= 2;
+            pl.max_splits = (int)std::max<long long>(1, (max_chunks + pl.cpc - 1) / pl.cpc);
+        } else if (pl.warps > 4) {
+            pl.warps = 4;
+        } else {
+            break;
+        }
         fit();
     }
-    if (pl.smem > (size_t)c->max_smem && pl.warps > 4) {
-        pl.warps = 4;
-        fit();
-    }
+    return pl;
+}
+
+DecodePlan plan_decode(const mq_cache* c, int n_seqs, int n_q_heads, int max_q, int max_seq_len) {
+    const int G = n_q_heads / c->n_kv_heads;
+    const int rows_total = G * max_q;
+    // Long histories with many query rows need more partial storage than shared memory
+    // holds; those fall back to a smaller row class (more row blocks, each reading the
+    // pages again).  Every row is computed by the same per-row arithmetic in each class,
+    // so the output does not change.
+    DecodePlan pl = plan_for_class(c, rows_class_for(c->head_dim, rows_total), n_seqs, rows_total, max_seq_len);
+    while (pl.smem > (size_t)c->max_smem && pl.cls > 0)
+        pl = plan_for_class(c, pl.cls - 1, n_seqs, rows_total, max_seq_len);
     return pl;
 }
 
@@ -270,10 +289,15 @@ size_t mq_decode_workspace_bytes(const mq_cache* c, int32_t n_seqs, int32_t n_q_
     const int G = n_q_heads / c->n_kv_heads;
     const int rows_total = G * max_q_per_seq;
     if (rows_total > 64) return 0;
-    const int cls = rows_class_for(c->head_dim, rows_total);
-    const int rows = rows_class_rows(c->head_dim, cls);
-    const int n_rb = (rows_total + rows - 1) / rows;
-    return workspace_bytes_for(c, n_seqs, n_rb, rows);
+    // the planner may fall back to a smaller row class (see plan_decode): size for the
+    // largest of them, so the answer does not depend on the launch configuration
+    size_t need = 0;
+    for (int cls = rows_class_for(c->head_dim, rows_total); cls >= 0; cls--) {
+        const int rows = rows_class_rows(c->head_dim, cls);
+        const int n_rb = (rows_total + rows - 1) / rows;
+        need = std::max(need, workspace_bytes_for(c, n_seqs, n_rb, rows));
+    }
+    return need;
 }
 
 mq_status mq_decode_attn(const mq_cache* c, const void* q, mq_dtype q_dtype, int32_t n_seqs, int32_t n_q_heads,

@@ -664,21 +664,24 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
 
     // ---- tree over the W warp results, in registers: at level s the left warp of
     // each pair merges its right sibling's entry; a warp that is a right sibling at
-    // the next level publishes its merged result to its entry 0 ----
+    // the next level then publishes what it holds to its entry 0 (it may have merged
+    // at lower levels even when its sibling at this level is empty) ----
     bool have = my_chunks > 0;
     if (have) write_entry(0);
     if (lane == 0) flags[warp] = have ? 0 : 1;
     __syncthreads();
     for (int s = 1; s < W; s <<= 1) {
-        if ((warp & (2 * s - 1)) == 0 && warp + s < W && flags[warp + s] == 0) {
-            const float* rent = part + (size_t)(warp + s) * SD * C::PART;
-            if (have) {
-                merge_right(rent);
-            } else {
-                load_entry(rent);
-                have = true;
+        if ((warp & (2 * s - 1)) == 0) {
+            if (warp + s < W && flags[warp + s] == 0) {
+                const float* rent = part + (size_t)(warp + s) * SD * C::PART;
+                if (have) {
+                    merge_right(rent);
+                } else {
+                    load_entry(rent);
+                    have = true;
+                }
             }
-            if ((warp & (4 * s - 1)) == 2 * s) {
+            if ((warp & (4 * s - 1)) == 2 * s && have) {
                 write_entry(0);
                 if (lane == 0) flags[warp] = 0;
             }

@@ -114,11 +114,7 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         !ck(cudaEventCreate(&B.ev[1])))
         return MQ_ERR_CUDA;
     size_t ws_bytes = 0;
-    for (auto& pr : probes) {
-        const int rows_total = G * pr.n_q;
-        const int rows = rows_class_rows(D, rows_class_for(D, rows_total));
-        ws_bytes = std::max(ws_bytes, workspace_bytes_for(cache, 1, (rows_total + rows - 1) / rows, rows));
-    }
+    for (auto& pr : probes) ws_bytes = std::max(ws_bytes, mq_decode_workspace_bytes(cache, 1, Hq, pr.n_q, pr.seq_len));
     const size_t kv_elems = (size_t)max_len * Hkv * D;
     if (!ck(cudaMalloc(&B.pool, copy_bytes * n_copies)) ||
         !ck(cudaMalloc(&B.bt, sizeof(int32_t) * blocks_per_copy * n_copies)) ||

@@ -49,6 +49,34 @@ def test_decode_lengths(L):
     _check(GpuCase(w))
 
 
+@pytest.mark.parametrize("Hq,Hkv,D,L,n", [(8, 2, 128, 262152, 8), (4, 1, 256, 524288, 4)])
+def test_decode_long_history_row_class_fallback(Hq, Hkv, D, L, n):
+    """Histories whose per-warp partial stacks outgrow shared memory in the natural
+    row class (32 rows at D 128, 16 rows at D 256) run in a smaller class with more
+    row blocks; every row stays within tolerance."""
+    _check(GpuCase(wl.Workload("long_fallback", Hq, Hkv, D, [L], [n], [n], shuffle=False)))
+
+
+def test_decode_head_dim_256_beyond_limit_is_unsupported():
+    """head_dim 256 with max_seq_len above 524288 is refused before any launch."""
+    L = 524288 + 128
+    n_blocks = L // 16
+    cache = mq.Cache(1, 256, n_blocks)
+    q = torch.zeros((1, 4, 256), dtype=torch.bfloat16, device="cuda")
+    bt = torch.arange(n_blocks, dtype=torch.int32, device="cuda").view(1, -1)
+    lens = torch.tensor([L], dtype=torch.int32, device="cuda")
+    nq = torch.ones(1, dtype=torch.int32, device="cuda")
+    out = torch.empty((1, 4, 256), dtype=torch.float32, device="cuda")
+    ws_bytes = mq.mq_decode_workspace_bytes(cache.handle, 1, 4, 1, L)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
+    with pytest.raises(mq.MQError) as ei:
+        mq.mq_decode_attn(cache.handle, q, mq.MQ_BF16, 1, 4, 1, 1, L, bt, n_blocks, lens, nq, 0.0625, out, None,
+                          ws, ws.numel())
+    assert ei.value.status == mq.MQ_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert mq.mq_device_status(cache.handle) == mq.MQ_OK
+
+
 def test_single_token_cache_returns_its_value():
     """L = 1: the weight is exactly 1, so out equals the dequantized v_0 exactly."""
     w = wl.long_decode(L=1)
