@@ -185,11 +185,16 @@ mq_status mq_kv_append(mq_cache* cache, const void* k, const void* v, mq_dtype d
  *   lse          fp32 [sum_b n_b][n_q_heads], natural-log log-sum-exp of the
  *                scaled logits; may be NULL
  *   workspace    device scratch of at least mq_decode_workspace_bytes(...)
- *                bytes, 256-byte aligned.  It must be zero-filled before its
- *                first use; every call that completes leaves its counter
- *                region zero again, so it can be reused across calls on the
- *                same stream without clearing.  After MQ_ERR_DEVICE, zero it
+ *                bytes, 256-byte aligned.  Its front 1/512 (rounded up to 256
+ *                bytes) holds per-(sequence, kv-head, row block) counters that
+ *                must be zero before the first call; every call that completes
+ *                leaves them zero again, so the workspace can be reused across
+ *                calls of any shape that fits it without clearing, provided
+ *                every call on it passes the same workspace_bytes (that value
+ *                fixes where the counters sit).  After MQ_ERR_DEVICE, zero it
  *                again.  Calls that share a workspace must not overlap.
+ *   workspace_bytes  its size; a workspace smaller than the query for this
+ *                shape is refused with MQ_ERR_WORKSPACE.
  * Query token j of sequence b (0-based) attends to positions 0 .. L_b - n_b + j:
  * the history plus drafts 0..j (causal among the drafts).  q-head h reads
  * kv-head h / (n_q_heads / n_kv_heads).  The result is bit-identical for every

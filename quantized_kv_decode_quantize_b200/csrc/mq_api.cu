@@ -123,19 +123,23 @@ DecodePlan plan_decode(const mq_cache* c, int n_seqs, int n_q_heads, int max_q, 
     return pl;
 }
 
-size_t workspace_bytes_for(const mq_cache* c, int n_seqs, int n_rb, int rows) {
-    const size_t units = (size_t)n_seqs * c->n_kv_heads * n_rb;
-    size_t off = (units * 4 + 255) / 256 * 256;
-    off += (units * kMaxSplits * rows * 2 * 4 + 255) / 256 * 256;
-    off += units * kMaxSplits * (size_t)rows * c->head_dim * 4;
-    return off;
+static size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t partial_bytes(const mq_cache* c, int n_seqs, const DecodePlan& pl) {
+    const size_t slots = (size_t)n_seqs * c->n_kv_heads * pl.n_rb * pl.max_splits;
+    return al256(slots * pl.rows * 2 * 4) + slots * pl.rows * c->head_dim * 4;
 }
+
+size_t counter_bytes(size_t workspace_bytes) { return al256((workspace_bytes + 511) / 512); }
 
 mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void* q, mq_dtype q_dtype, int n_seqs,
                              int n_q_heads, int total_q, int max_q, const int32_t* block_table, int max_blocks,
                              const int32_t* seq_lens, const int32_t* n_q_per_seq, float softmax_scale, float* out,
-                             float* lse, void* workspace, cudaStream_t st) {
+                             float* lse, void* workspace, size_t workspace_bytes, cudaStream_t st) {
     if (pl.smem == 0 || pl.smem > (size_t)c->max_smem) return MQ_ERR_UNSUPPORTED;
+    const size_t units = (size_t)n_seqs * c->n_kv_heads * pl.n_rb;
+    const size_t cb = counter_bytes(workspace_bytes);
+    if (units * 4 > cb || cb + partial_bytes(c, n_seqs, pl) > workspace_bytes) return MQ_ERR_WORKSPACE;
     cudaError_t e = ensure_decode_smem(c->device, c->head_dim, pl.rows, pl.smem);
     if (e != cudaSuccess) return MQ_ERR_CUDA;
     DecodeParams p{};
@@ -156,13 +160,15 @@ mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void
     p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
     p.out = out;
     p.lse = lse;
-    const size_t units = (size_t)n_seqs * c->n_kv_heads * pl.n_rb;
+    // counters in the fixed front region (the same bytes for every shape that shares
+    // this workspace), then this call's partials with a stride of max_splits per unit
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.counters = reinterpret_cast<unsigned*>(ws);
-    size_t off = (units * 4 + 255) / 256 * 256;
+    size_t off = cb;
     p.part_ml = reinterpret_cast<float*>(ws + off);
-    off += (units * kMaxSplits * pl.rows * 2 * 4 + 255) / 256 * 256;
+    off += al256(units * pl.max_splits * pl.rows * 2 * 4);
     p.part_o = reinterpret_cast<float*>(ws + off);
+    p.split_stride = pl.max_splits;
     p.n_rb = pl.n_rb;
     p.cpc = pl.cpc;
     p.pages_per_stage = pl.pages_per_stage;
@@ -289,13 +295,28 @@ size_t mq_decode_workspace_bytes(const mq_cache* c, int32_t n_seqs, int32_t n_q_
     const int G = n_q_heads / c->n_kv_heads;
     const int rows_total = G * max_q_per_seq;
     if (rows_total > 64) return 0;
-    // the planner may fall back to a smaller row class (see plan_decode): size for the
-    // largest of them, so the answer does not depend on the launch configuration
-    size_t need = 0;
-    for (int cls = rows_class_for(c->head_dim, rows_total); cls >= 0; cls--) {
-        const int rows = rows_class_rows(c->head_dim, cls);
-        const int n_rb = (rows_total + rows - 1) / rows;
-        need = std::max(need, workspace_bytes_for(c, n_seqs, n_rb, rows));
+    // The plan depends on the launch configuration (which mq_tune / mq_set_decode_config
+    // may change after the workspace is sized) and may fall back to a smaller row class:
+    // size the partials for the largest plan over every valid configuration, so the
+    // answer depends on the shape alone.
+    mq_cache probe = *c;
+    size_t part = 0;
+    for (int w = 4; w <= 8; w += 4)
+        for (int r = 2; r <= 4; r++)
+            for (int t = 1; t <= 4; t *= 2) {
+                for (int k = 0; k < 3; k++) probe.cfg[k] = mq_decode_config{w, r, t};
+                const int top = rows_class_for(c->head_dim, rows_total);
+                for (int cls = top; cls >= 0; cls--) {
+                    const DecodePlan pl = plan_for_class(&probe, cls, n_seqs, rows_total, max_seq_len);
+                    part = std::max(part, partial_bytes(c, n_seqs, pl));
+                }
+            }
+    // counters take the front 1/512 of the workspace (rounded up to 256 bytes); a
+    // 256-byte margin keeps any larger workspace valid as well
+    size_t need = part + 256;
+    for (size_t prev = 0; prev != need;) {
+        prev = need;
+        need = part + counter_bytes(need) + 256;
     }
     return need;
 }
@@ -325,7 +346,7 @@ mq_status mq_decode_attn(const mq_cache* c, const void* q, mq_dtype q_dtype, int
     const DecodePlan pl = plan_decode(c, n_seqs, n_q_heads, max_q_per_seq, max_seq_len);
     return launch_decode_plan(c, pl, q, q_dtype, n_seqs, n_q_heads, total_q, max_q_per_seq, block_table,
                               max_blocks_per_seq, seq_lens, n_q_per_seq, softmax_scale, out, lse, workspace,
-                              reinterpret_cast<cudaStream_t>(stream));
+                              workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 mq_status mq_get_decode_config(const mq_cache* c, int32_t cls, mq_decode_config* cfg) {

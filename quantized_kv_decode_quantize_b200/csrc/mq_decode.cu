@@ -727,8 +727,8 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
     }
     // ---- publish this CTA's partial; the last CTA completes the tree ----
     {
-        float* go = p.part_o + (pidx * kMaxSplits + sp) * (size_t)(ROWS * D);
-        float* gml = p.part_ml + (pidx * kMaxSplits + sp) * (size_t)(2 * ROWS);
+        float* go = p.part_o + (pidx * p.split_stride + sp) * (size_t)(ROWS * D);
+        float* gml = p.part_ml + (pidx * p.split_stride + sp) * (size_t)(2 * ROWS);
         for (int i = threadIdx.x; i < ROWS * D / 4; i += blockDim.x)
             __stcg(reinterpret_cast<float4*>(go) + i, reinterpret_cast<const float4*>(part)[i]);
         for (int i = threadIdx.x; i < 2 * ROWS; i += blockDim.x) __stcg(gml + i, part[ROWS * D + i]);
@@ -746,8 +746,8 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
     while ((1 << H) < n_splits) H++;
     float* hp = reinterpret_cast<float*>(smem + S.heap);
     auto hidx = [&](int level, int i) { return (1 << (H - level)) + i; };
-    const float* gml0 = p.part_ml + pidx * kMaxSplits * (size_t)(2 * ROWS);
-    const float* go0 = p.part_o + pidx * kMaxSplits * (size_t)(ROWS * D);
+    const float* gml0 = p.part_ml + pidx * p.split_stride * (size_t)(2 * ROWS);
+    const float* go0 = p.part_o + pidx * p.split_stride * (size_t)(ROWS * D);
     for (int i = threadIdx.x; i < n_splits * ROWS; i += blockDim.x) {
         const int s = i / ROWS, r = i % ROWS;
         float* nd = hp + ((size_t)hidx(0, s) * ROWS + r) * 4;

@@ -43,8 +43,9 @@ struct DecodeParams {
     float* lse;
     // workspace
     unsigned* counters;  // [n_seqs][n_kv_heads][n_rb]
-    float* part_ml;      // [n_seqs][n_kv_heads][n_rb][kMaxSplits][rows][2]
-    float* part_o;       // [n_seqs][n_kv_heads][n_rb][kMaxSplits][rows][D]
+    float* part_ml;      // [n_seqs][n_kv_heads][n_rb][split_stride][rows][2]
+    float* part_o;       // [n_seqs][n_kv_heads][n_rb][split_stride][rows][D]
+    int split_stride;    // partial slots per unit (>= the splits of any unit)
     int n_rb;            // row blocks per kv-head
     int cpc;             // chunks per CTA (power of two >= warps)
     int pages_per_stage; // TMA ring depth per warp

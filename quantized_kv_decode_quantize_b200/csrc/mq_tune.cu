@@ -188,7 +188,7 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         const int32_t* bt = B.bt + (size_t)(rot % n_copies) * blocks_per_copy;
         rot++;
         return launch_decode_plan(&pc, pl, B.q, MQ_BF16, 1, Hq, probes[p].n_q, probes[p].n_q, bt, blocks_per_copy,
-                                  B.lens + p, B.nq + p, 1.0f / std::sqrt((float)D), out, lse, B.ws, B.st);
+                                  B.lens + p, B.nq + p, 1.0f / std::sqrt((float)D), out, lse, B.ws, ws_bytes, B.st);
     };
     const int reps = 7;
     // median device time of `reps` launches (events around each launch)

@@ -77,6 +77,25 @@ def test_decode_head_dim_256_beyond_limit_is_unsupported():
     assert mq.mq_device_status(cache.handle) == mq.MQ_OK
 
 
+def test_workspace_reused_across_shapes():
+    """One workspace, sized for the largest shape and passed with the same size on
+    every call, serves calls of different shapes back to back (few units with many
+    splits, then many units): each output is bit-identical to the same call with a
+    fresh zero-filled workspace of its own."""
+    cases = [GpuCase(wl.FULL["long"]()),
+             GpuCase(wl.Workload("many_units", 32, 8, 128, [600 + 37 * i for i in range(40)], [1] * 40, [1] * 40)),
+             GpuCase(wl.reduced("verify")),
+             GpuCase(wl.reduced("mixed"))]
+    fresh = [c.decode()[0].clone() for c in cases]
+    shared = torch.zeros(max(c.ws.numel() for c in cases), dtype=torch.uint8, device="cuda")
+    for c in cases:
+        c.ws = shared
+    for i in [0, 1, 2, 3, 0, 1, 3, 2, 0]:
+        out = cases[i].decode()[0]
+        assert torch.equal(out, fresh[i]), f"case {i}"
+        assert cases[i].status() == mq.MQ_OK
+
+
 def test_single_token_cache_returns_its_value():
     """L = 1: the weight is exactly 1, so out equals the dequantized v_0 exactly."""
     w = wl.long_decode(L=1)
