@@ -1,6 +1,8 @@
 """Builds the mq CUDA library (libmq.so) in-tree for sm_100a with nvcc.
 
-    python -m quantized_kv_decode_quantize_b200.build [--force] [--verbose]
+    python quantized_kv_decode_quantize_b200/build.py [--force] [--verbose] [--ptxas]
+
+(run as a script: importing the package first would load the library being rebuilt)
 
 Each ``csrc/*.cu`` file is compiled to an object under ``_build/`` and linked with
 the static CUDA runtime into ``quantized_kv_decode_quantize_b200/libmq.so``.  No
