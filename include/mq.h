@@ -218,6 +218,40 @@ mq_status mq_decode_attn(const mq_cache* cache, const void* q, mq_dtype q_dtype,
                          mq_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * mq_decode_attn_static: mq_decode_attn without a caller workspace.
+ *
+ * The method on the pages has no counterpart to this call; it is a convenience
+ * of this library.  It is for callers that cannot give the library a device
+ * allocation when they decode: a server that has reserved nearly all free HBM
+ * for its KV pool, a C host program with no device allocator of its own, or a
+ * decode loop that cannot afford the device synchronization cudaMalloc and
+ * cudaFree may cause.  The call allocates nothing.  Its scratch is one fixed
+ * array of MQ_DECODE_STATIC_SCRATCH_BYTES (16 MiB) per device inside the
+ * library, whose address is looked up on the first call on each device.
+ *
+ * Arguments, layouts, ownership and results are those of mq_decode_attn,
+ * without workspace and workspace_bytes; the outputs equal mq_decode_attn's.
+ * Each call first clears the split counters at the front of the scratch with an
+ * asynchronous memset on `stream`, then launches the decode kernel there.
+ * Make the first call on each device before any stream capture that is to
+ * contain a later call: that first call does the address lookup.
+ * The scratch is shared by every call on a device: calls whose executions may
+ * overlap (different streams or host threads without ordering between them)
+ * race on it and give wrong results.  Order them, or use mq_decode_attn with a
+ * workspace per stream.
+ * Errors: those of mq_decode_attn, and WORKSPACE when the shape needs more than
+ * MQ_DECODE_STATIC_SCRATCH_BYTES of scratch (mq_decode_workspace_bytes() above
+ * that limit); nothing is launched then.
+ * ------------------------------------------------------------------------- */
+#define MQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+
+mq_status mq_decode_attn_static(const mq_cache* cache, const void* q, mq_dtype q_dtype, int32_t n_seqs,
+                                int32_t n_q_heads, int32_t total_q, int32_t max_q_per_seq, int32_t max_seq_len,
+                                const int32_t* block_table, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                const int32_t* n_q_per_seq, float softmax_scale, float* out, float* lse,
+                                mq_stream stream);
+
+/* ---------------------------------------------------------------------------
  * Launch configuration and tuning
  *
  * The decode kernel's arithmetic is fixed: every sequence is cut into chunks of

@@ -5,7 +5,7 @@ integers (device pointers, sizes) and the current CUDA stream through ctypes.
 Torch tensors are accepted wherever the C function takes a device pointer; only
 their ``data_ptr()`` is used.  All computation happens in ``libmq.so``'s CUDA
 kernels; there is no fallback path: if the library is missing this module raises
-ImportError (build it with ``python -m quantized_kv_decode_quantize_b200.build``).
+ImportError (build it with ``python quantized_kv_decode_quantize_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -51,7 +51,7 @@ class MQError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing; build it with `python -m quantized_kv_decode_quantize_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing; build it with `python quantized_kv_decode_quantize_b200/build.py`")
     L = ctypes.CDLL(LIB_PATH)
     P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     sig = {
@@ -65,6 +65,8 @@ def _load():
         "mq_decode_workspace_bytes": ([P, i32, i32, i32, i32], sz),
         "mq_decode_attn": ([P, P, ctypes.c_int, i32, i32, i32, i32, i32, P, i32, P, P, ctypes.c_float, P, P, P, sz, P],
                            ctypes.c_int),
+        "mq_decode_attn_static": ([P, P, ctypes.c_int, i32, i32, i32, i32, i32, P, i32, P, P, ctypes.c_float, P, P,
+                                   P], ctypes.c_int),
         "mq_get_decode_config": ([P, i32, ctypes.POINTER(mq_decode_config)], ctypes.c_int),
         "mq_set_decode_config": ([P, i32, ctypes.POINTER(mq_decode_config)], ctypes.c_int),
         "mq_tune": ([P, ctypes.POINTER(mq_tune_params), ctypes.POINTER(mq_tune_result)], ctypes.c_int),
@@ -150,6 +152,15 @@ def mq_decode_attn(cache: int, q, q_dtype: int, n_seqs: int, n_q_heads: int, tot
                               _ptr(block_table), max_blocks_per_seq, _ptr(seq_lens), _ptr(n_q_per_seq),
                               float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace_bytes,
                               _stream(stream)), "mq_decode_attn")
+
+
+def mq_decode_attn_static(cache: int, q, q_dtype: int, n_seqs: int, n_q_heads: int, total_q: int,
+                          max_q_per_seq: int, max_seq_len: int, block_table, max_blocks_per_seq: int, seq_lens,
+                          n_q_per_seq, softmax_scale: float, out, lse, stream=None) -> None:
+    _check(lib.mq_decode_attn_static(cache, _ptr(q), q_dtype, n_seqs, n_q_heads, total_q, max_q_per_seq, max_seq_len,
+                                     _ptr(block_table), max_blocks_per_seq, _ptr(seq_lens), _ptr(n_q_per_seq),
+                                     float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream)),
+           "mq_decode_attn_static")
 
 
 def mq_get_decode_config(cache: int, rows_class: int) -> tuple:
