@@ -94,18 +94,17 @@ typedef enum mq_dtype { MQ_F32 = 0, MQ_BF16 = 1, MQ_F16 = 2 } mq_dtype;
  * = 25*D + 32 bytes (3232 for D = 128, 6432 for D = 256), against 64*D for
  * fp16 K+V: 0.395x (D = 128) and 0.393x (D = 256) — "more than half" smaller,
  * as the trawling.dev Launch HN page (per-device tuning and performance claims)
- * reports for this codec.  Within each region the bytes are permuted so that
- * the decode kernel's tensor-core fragments load with 16-byte shared-memory
- * reads (lane L = 4g + t, g = 0..7, t = 0..3; NG = D/32 groups):
- *     K code of token tau, channel c: byte (k*32 + L)*16 + (o % 16) with
- *       L = 4*(tau % 8) + c / (D/4), o = c % (D/4), k = (tau / 8)*(D/64) + o/16
- *     K scale of token tau: half-word tau of the K-scale region
- *     V codes: 32-bit word w = 2q + p of lane L sits at ((w/4)*32 + L)*16 +
- *       (w%4)*4 of the V-code region and holds, byte by byte, channels
- *       (c, c+1), (c+2, c+3) of token 8p + 2t, then the same channels of token
- *       8p + 2t + 1, with c = 32q + 4g and the even channel in the low nibble
- *     V scale of token tau, group q: half-word ((t'*NG + q)*2 + tau/8)*2 + tau%2
- *       of the V-scale region, t' = (tau % 8)/2
+ * reports for this codec.  The page is laid out for the decode kernel's tensor
+ * cores as two records of 8 tokens (tokens 0-7 at byte 0, tokens 8-15 at byte
+ * R = 12.5*D + 16; R = 1616 for D = 128, 3216 for D = 256).  In the record of
+ * token tau (tt = tau % 8, NG = D/32 groups):
+ *     K code of (tau, channel c): byte (c/16)*128 + tt*16 + c%16 — 8-row x
+ *       16-byte blocks, so the K codes of consecutive records form one K-major
+ *       int8 matrix operand whose 8-token groups are R bytes apart
+ *     V codes: one 32-bit word per channel c at byte 8*D + 4*c holding the 8
+ *       tokens' 4-bit two's-complement codes, token tt at bit 4*(tt/2) + 16*(tt%2)
+ *     K scale of tau: fp16 at byte 12*D + 2*tt
+ *     V scale of (tau, group g): fp16 at byte 12*D + 16 + 2*(tt*NG + g)
  * The codes and scales themselves are exactly the codec's.
  *
  * A block_table is int32 [n_seqs][max_blocks_per_seq]: entry [b][i] is the
@@ -202,9 +201,7 @@ mq_status mq_kv_append(mq_cache* cache, const void* k, const void* v, mq_dtype d
  * Errors: INVALID_ARG (null pointers, n_seqs < 1 or > 65535, n_q_heads not a
  * multiple of n_kv_heads, total_q < 1, max_q_per_seq < 1, max_seq_len <
  * max_q_per_seq, a non-finite softmax_scale, out not 16-byte aligned), UNSUPPORTED
- * (n_q_heads/n_kv_heads * max_q_per_seq > 64, q dtype, head_dim 256 with
- * max_seq_len > 524288: the per-warp partial stack no longer fits in shared
- * memory), CAPACITY (max_seq_len >
+ * (n_q_heads/n_kv_heads * max_q_per_seq > 64, q dtype), CAPACITY (max_seq_len >
  * max_blocks_per_seq * 16), WORKSPACE, CUDA.  A sequence whose L_b / n_b break
  * the bounds above is skipped by the kernel and reported by mq_device_status().
  * ------------------------------------------------------------------------- */
@@ -254,22 +251,23 @@ mq_status mq_decode_attn_static(const mq_cache* cache, const void* q, mq_dtype q
 /* ---------------------------------------------------------------------------
  * Launch configuration and tuning
  *
- * The decode kernel's arithmetic is fixed: every sequence is cut into chunks of
- * 128 tokens, each chunk is reduced by one warp in token order with an online
- * softmax, and chunk results are combined by one fixed binary tree.  The launch
- * configuration only decides which warp and CTA computes which subtree, so all
- * configurations give bit-identical outputs.
- *   warps_per_cta    4 or 8: chunks a CTA reduces concurrently
- *   pages_per_stage  2 .. 4: pages each warp keeps in flight (TMA ring depth)
- *   ctas_per_sm      1, 2 or 4: target CTAs per SM; fixes how many chunks one
- *                    CTA takes (the split count along the sequence)
+ * The decode kernel cuts every sequence into chunks of 128 tokens; one CTA takes a
+ * contiguous range of chunks of one (sequence, kv-head, row block), accumulates
+ * them in token order, and the CTA partials are combined by one fixed binary
+ * tree over the split index.
+ *   ring_stages    2 .. 4: chunks (8 pages each) a CTA keeps in flight; never
+ *                  changes the output
+ *   splits_per_sm  1, 2 or 4: the split count along the sequence is chosen so
+ *                  that about splits_per_sm x (number of SMs) CTAs run; it sets
+ *                  the chunk ranges and so may change the rounding of the output
+ *                  (the tuner keeps only candidates whose output bytes equal the
+ *                  current configuration's)
  * There is one configuration per row class (query rows per kv-head, padded):
  * rows_class 0 = up to 8 rows, 1 = up to 16, 2 = up to 32.
  * ------------------------------------------------------------------------- */
 typedef struct mq_decode_config {
-    int32_t warps_per_cta;
-    int32_t pages_per_stage;
-    int32_t ctas_per_sm;
+    int32_t ring_stages;
+    int32_t splits_per_sm;
 } mq_decode_config;
 
 mq_status mq_get_decode_config(const mq_cache* cache, int32_t rows_class, mq_decode_config* cfg);

@@ -27,11 +27,10 @@ class mq_cache_desc(ctypes.Structure):
 
 
 class mq_decode_config(ctypes.Structure):
-    _fields_ = [("warps_per_cta", ctypes.c_int32), ("pages_per_stage", ctypes.c_int32),
-                ("ctas_per_sm", ctypes.c_int32)]
+    _fields_ = [("ring_stages", ctypes.c_int32), ("splits_per_sm", ctypes.c_int32)]
 
     def as_tuple(self):
-        return (self.warps_per_cta, self.pages_per_stage, self.ctas_per_sm)
+        return (self.ring_stages, self.splits_per_sm)
 
 
 class mq_tune_params(ctypes.Structure):
@@ -169,9 +168,8 @@ def mq_get_decode_config(cache: int, rows_class: int) -> tuple:
     return c.as_tuple()
 
 
-def mq_set_decode_config(cache: int, rows_class: int, warps_per_cta: int, pages_per_stage: int,
-                         ctas_per_sm: int) -> None:
-    c = mq_decode_config(warps_per_cta, pages_per_stage, ctas_per_sm)
+def mq_set_decode_config(cache: int, rows_class: int, ring_stages: int, splits_per_sm: int) -> None:
+    c = mq_decode_config(ring_stages, splits_per_sm)
     _check(lib.mq_set_decode_config(cache, rows_class, ctypes.byref(c)), "mq_set_decode_config")
 
 

@@ -33,22 +33,17 @@ int rows_class_for(int head_dim, int rows_total) {
 }
 
 mq_decode_config default_config(int head_dim, int cls) {
+    (void)head_dim;
+    (void)cls;
     mq_decode_config c{};
-    if (head_dim == 128) {
-        c.warps_per_cta = cls == 2 ? 4 : 8;
-        c.pages_per_stage = 2;
-        c.ctas_per_sm = cls == 0 ? 2 : 1;
-    } else {
-        c.warps_per_cta = cls == 0 ? 8 : 4;
-        c.pages_per_stage = 2;
-        c.ctas_per_sm = 1;
-    }
+    c.ring_stages = 4;
+    c.splits_per_sm = 1;
     return c;
 }
 
 bool config_valid(const mq_decode_config& c) {
-    return (c.warps_per_cta == 4 || c.warps_per_cta == 8) && c.pages_per_stage >= 2 && c.pages_per_stage <= 4 &&
-           (c.ctas_per_sm == 1 || c.ctas_per_sm == 2 || c.ctas_per_sm == 4);
+    return c.ring_stages >= 2 && c.ring_stages <= 4 &&
+           (c.splits_per_sm == 1 || c.splits_per_sm == 2 || c.splits_per_sm == 4);
 }
 
 DevGuard::DevGuard(int dev) {
@@ -62,50 +57,27 @@ DevGuard::~DevGuard() {
     if (switched && prev >= 0) cudaSetDevice(prev);
 }
 
-// The plan for one row class: rows per CTA, launch shape, chunks per CTA.
+// The plan for one row class: rows per CTA, split count, chunks per CTA, ring depth.
+// The chunk ranges depend only on the shape, the SM count and splits_per_sm.
 static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int rows_total, int max_seq_len) {
     DecodePlan pl{};
     pl.cls = cls;
     pl.rows = rows_class_rows(c->head_dim, pl.cls);
     pl.n_rb = (rows_total + pl.rows - 1) / pl.rows;
     const mq_decode_config cfg = c->cfg[pl.cls];
-    pl.warps = cfg.warps_per_cta;
-    pl.pages_per_stage = cfg.pages_per_stage;
-    const long long max_chunks = (max_seq_len + kChunkTokens - 1) / kChunkTokens;
-    long long cpc = pl.warps;
-    while ((max_chunks + cpc - 1) / cpc > kMaxSplits) cpc *= 2;
+    const long long max_chunks = std::max<long long>(1, (max_seq_len + kChunkTokens - 1) / kChunkTokens);
     const long long units = (long long)n_seqs * c->n_kv_heads * pl.n_rb;
-    const long long target = (long long)cfg.ctas_per_sm * c->n_sm;
-    while (cpc < max_chunks && units * ((max_chunks + cpc - 1) / cpc) > target) cpc *= 2;
+    long long splits = (long long)cfg.splits_per_sm * c->n_sm / units;
+    splits = std::max<long long>(1, std::min<long long>({splits, max_chunks, (long long)kMaxSplits}));
+    const long long cpc = (max_chunks + splits - 1) / splits;
     pl.cpc = (int)cpc;
-    pl.max_splits = (int)std::max<long long>(1, (max_chunks + cpc - 1) / cpc);
-    if (pl.cpc < pl.warps) pl.cpc = pl.warps;
-    auto fit = [&]() {
-        // each warp reduces an aligned run of cpc / warps chunks; its binary counter
-        // keeps at most log2(run) left siblings (at least one entry: its result)
-        const int run = (int)(pl.cpc / pl.warps);
-        int sd = 0;
-        while ((1 << sd) < run) sd++;
-        pl.stack_depth = sd < 1 ? 1 : sd;
-        pl.smem = decode_smem_bytes(c->head_dim, pl.rows, pl.warps, pl.pages_per_stage, pl.stack_depth);
-    };
-    fit();
-    // A configuration that does not fit in shared memory runs with a shallower ring,
-    // then with shorter warp runs (more CTAs per sequence, while the split count stays
-    // within kMaxSplits), then with 4 warps.  The chunk tree is fixed by the chunk
-    // indices alone, so the arithmetic (and so the output) is the same.
-    while (pl.smem > (size_t)c->max_smem) {
-        if (pl.pages_per_stage > 2) {
-            pl.pages_per_stage--;
-        } else if (pl.cpc > pl.warps && (max_chunks + pl.cpc / 2 - 1) / (pl.cpc / 2) <= kMaxSplits) {
-            pl.cpc /= 2;
-            pl.max_splits = (int)std::max<long long>(1, (max_chunks + pl.cpc - 1) / pl.cpc);
-        } else if (pl.warps > 4) {
-            pl.warps = 4;
-        } else {
-            break;
-        }
-        fit();
+    pl.max_splits = (int)((max_chunks + cpc - 1) / cpc);
+    // the ring is shortened (never below 2 stages) until the CTA fits in shared memory
+    pl.stages = cfg.ring_stages;
+    pl.smem = decode_smem_bytes(c->head_dim, pl.rows, pl.stages);
+    while ((pl.smem == 0 || pl.smem > (size_t)c->max_smem) && pl.stages > 2) {
+        pl.stages--;
+        pl.smem = decode_smem_bytes(c->head_dim, pl.rows, pl.stages);
     }
     return pl;
 }
@@ -113,14 +85,7 @@ static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int row
 DecodePlan plan_decode(const mq_cache* c, int n_seqs, int n_q_heads, int max_q, int max_seq_len) {
     const int G = n_q_heads / c->n_kv_heads;
     const int rows_total = G * max_q;
-    // Long histories with many query rows need more partial storage than shared memory
-    // holds; those fall back to a smaller row class (more row blocks, each reading the
-    // pages again).  Every row is computed by the same per-row arithmetic in each class,
-    // so the output does not change.
-    DecodePlan pl = plan_for_class(c, rows_class_for(c->head_dim, rows_total), n_seqs, rows_total, max_seq_len);
-    while (pl.smem > (size_t)c->max_smem && pl.cls > 0)
-        pl = plan_for_class(c, pl.cls - 1, n_seqs, rows_total, max_seq_len);
-    return pl;
+    return plan_for_class(c, rows_class_for(c->head_dim, rows_total), n_seqs, rows_total, max_seq_len);
 }
 
 static size_t al256(size_t x) { return (x + 255) / 256 * 256; }
@@ -171,10 +136,9 @@ mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void
     p.split_stride = pl.max_splits;
     p.n_rb = pl.n_rb;
     p.cpc = pl.cpc;
-    p.pages_per_stage = pl.pages_per_stage;
-    p.stack_depth = pl.stack_depth;
+    p.stages = pl.stages;
     p.err = c->err_word;
-    e = launch_decode(p, c->head_dim, pl.rows, pl.warps, pl.max_splits, pl.smem, st);
+    e = launch_decode(p, c->head_dim, pl.rows, pl.max_splits, pl.smem, st);
     return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
 }
 
@@ -296,21 +260,17 @@ size_t mq_decode_workspace_bytes(const mq_cache* c, int32_t n_seqs, int32_t n_q_
     const int rows_total = G * max_q_per_seq;
     if (rows_total > 64) return 0;
     // The plan depends on the launch configuration (which mq_tune / mq_set_decode_config
-    // may change after the workspace is sized) and may fall back to a smaller row class:
-    // size the partials for the largest plan over every valid configuration, so the
-    // answer depends on the shape alone.
+    // may change after the workspace is sized): size the partials for the largest plan
+    // over every valid configuration, so the answer depends on the shape alone.
     mq_cache probe = *c;
     size_t part = 0;
-    for (int w = 4; w <= 8; w += 4)
-        for (int r = 2; r <= 4; r++)
-            for (int t = 1; t <= 4; t *= 2) {
-                for (int k = 0; k < 3; k++) probe.cfg[k] = mq_decode_config{w, r, t};
-                const int top = rows_class_for(c->head_dim, rows_total);
-                for (int cls = top; cls >= 0; cls--) {
-                    const DecodePlan pl = plan_for_class(&probe, cls, n_seqs, rows_total, max_seq_len);
-                    part = std::max(part, partial_bytes(c, n_seqs, pl));
-                }
-            }
+    for (int r = 2; r <= 4; r++)
+        for (int t = 1; t <= 4; t *= 2) {
+            for (int k = 0; k < 3; k++) probe.cfg[k] = mq_decode_config{r, t};
+            const DecodePlan pl = plan_for_class(&probe, rows_class_for(c->head_dim, rows_total), n_seqs, rows_total,
+                                                 max_seq_len);
+            part = std::max(part, partial_bytes(c, n_seqs, pl));
+        }
     // counters take the front 1/512 of the workspace (rounded up to 256 bytes); a
     // 256-byte margin keeps any larger workspace valid as well
     size_t need = part + 256;

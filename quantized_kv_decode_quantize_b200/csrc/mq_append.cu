@@ -8,8 +8,11 @@
 // Both divisions are IEEE fp32 (__fdiv_rn), rounding is to nearest even, and a
 // zero scale gives code 0.  One warp handles one (token, kv-head): each lane
 // reads D/32 consecutive channels with one vector load, the absmax reductions
-// are warp shuffles (exact: max is order-independent), and each lane stores its
-// codes with one 4- or 8-byte store into the permuted page layout.
+// are warp shuffles (exact: max is order-independent), each lane stores its K
+// codes with one 4- or 8-byte store, and writes its V codes into the channel-major
+// V words of the page (see mq_device.cuh).  A V word holds the codes of eight
+// tokens, so its nibble is replaced with two atomic bit operations (clear, then
+// set): appends of neighbouring tokens in one launch may touch the same word.
 #include "mq_device.cuh"
 #include "mq_kernels.h"
 
@@ -113,7 +116,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     } else {
         *reinterpret_cast<uint2*>(kdst) = make_uint2(kb[0], kb[1]);
     }
-    if (lane == 0) *reinterpret_cast<__half*>(page + k_scale_off(D) + 2 * tau) = sk16;
+    if (lane == 0) *reinterpret_cast<__half*>(page + k_scale_byte(D, tau)) = sk16;
 
     // ---- V: one scale per 32-channel group (LPG lanes) ----
     float av = 0.0f;
@@ -123,14 +126,13 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     for (int o = LPG / 2; o > 0; o >>= 1) av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, o));
     const __half sv16 = __float2half_rn(__fdiv_rn(av, 7.0f));
     const float sv = __half2float(sv16);
+    const int bit = v_nibble_bit(tau);
 #pragma unroll
-    for (int s4 = 0; s4 < CPL / 4; s4++) {   // sets of 4 channels: 2 bytes
-        const int c = c0 + 4 * s4;
-        uint32_t n[4];
-#pragma unroll
-        for (int j = 0; j < 4; j++) n[j] = (uint32_t)quant_code(xv[4 * s4 + j], sv, -8.0f, 7.0f) & 0xFu;
-        const uint16_t two = (uint16_t)((n[0] | (n[1] << 4)) | ((n[2] | (n[3] << 4)) << 8));
-        *reinterpret_cast<uint16_t*>(page + v_code_byte(D, tau, c)) = two;
+    for (int i = 0; i < CPL; i++) {
+        const uint32_t n = (uint32_t)quant_code(xv[i], sv, -8.0f, 7.0f) & 0xFu;
+        unsigned* w = reinterpret_cast<unsigned*>(page + v_word_byte(D, tau, c0 + i));
+        atomicAnd(w, ~(0xFu << bit));
+        atomicOr(w, n << bit);
     }
     if (lane % LPG == 0)
         *reinterpret_cast<__half*>(page + v_scale_byte(D, tau, c0 / 32)) = sv16;

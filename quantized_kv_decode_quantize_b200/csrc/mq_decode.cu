@@ -1,4 +1,5 @@
-// Split-K flash-decode over the K8/V4 paged cache, with draft verification.
+// Split-K flash-decode over the K8/V4 paged cache, with draft verification, on the
+// sm_100a tensor cores (tcgen05 + tensor memory).
 //
 // What it computes (the deep dive on magnitudedev/magnitude at blog.123qwe.co.kr,
 // section 5: the decode attention unit attention_decode_k8v4 over the 8-bit-key /
@@ -8,87 +9,108 @@
 //     z_t = scale * <q, s_k[t] * kcode_t>,  t = 0 .. L_b - n_b + j
 //     out = sum_t softmax(z)_t * (s_v[t, group] * vcode_t),  lse = log sum_t exp z_t
 //
-// How, on sm_100a:
-//  * One CTA takes an aligned block of 128-token chunks of one (sequence, kv-head,
-//    row block); every warp of the CTA takes one chunk per round.  Pages (16
-//    tokens of one kv-head, 3232 or 6432 bytes) stream into a per-warp shared-memory
-//    ring by 1-D bulk TMA copies (cp.async.bulk + mbarrier, L2 evict-first), looked
-//    up through the block table.
-//  * QK^T on the tensor cores in int8: q is held as a 23-bit fixed-point value per
-//    row (q = Q * 2^(E-22), |Q| <= 2^22) split into three 8-bit limbs, so the int8
-//    key codes feed mma.m16n8k32 straight from shared memory with no conversion and
-//    the int32 products are exact; the limbs are combined once per score in fp32.
-//  * P.V on the tensor cores in fp16: the int4 value codes become exact fp16
-//    integers with two LOP3 + one HADD2/HFMA2 per pair; the weights
-//    p * s_v[token, group] are rounded to fp16 (relative error <= 2^-11 per weight).
-//  * Within a chunk one warp keeps an online softmax (running max in log2 units).
-//    Chunk results are combined by ONE fixed binary tree over chunk indices
-//    (warps of a round, rounds of a CTA, CTAs of a sequence), so the output does
-//    not depend on warps per CTA, ring depth or split count.  The last CTA of each
-//    (sequence, kv-head, row block) to finish — found with one atomic counter —
-//    completes the tree over the CTA partials and writes out and lse; there is no
-//    second kernel and no CTA ever waits for another.
+// How.  One CTA (10 warps, one per SM) takes a contiguous range of 128-token chunks of
+// one (sequence, kv-head, row block) and runs a warp-specialised pipeline per chunk:
+//  * warp 0 streams the chunk's 8 pages into a shared-memory ring with one 1-D bulk
+//    TMA copy per page (block-table lookup, L2 evict-first).  The page format makes
+//    the int8 key codes of a chunk one K-major tensor-core operand as they land.
+//  * warp 1 issues the MMAs from one thread.  Scores: S = K q^T with kind::i8, M = 128
+//    tokens, the query rows as the N side, q held as a 23-bit fixed-point value per row
+//    (q = Q * 2^(E-22)) split into three signed 8-bit limbs stacked along N, so the
+//    int32 products are exact; S lands in tensor memory.  Values: O += V^T W with
+//    kind::f16, A = V^T from tensor memory (M = 128 channels, K = tokens), B = the
+//    weights W_g = p * s_v[token, group] for every group g of 32 channels stacked
+//    along N; each channel keeps only its own group's columns.  A second MMA with a
+//    constant all-ones A gives, in every lane, the column sums of W: the per-group
+//    sums that undo the value-code offset, and l = sum_t p from the p columns.
+//  * warps 2-5 turn the int4 value codes into tensor memory as exact fp16 values
+//    u * 2^-24 (u = code + 8 in 0..15, a subnormal) with one mask, shift and flip per
+//    two tokens, a channel per TMEM lane; out = 2^24 * O - 8 * sum_t W_g.
+//  * warps 6-9 (one TMEM lane per token) read S, form z in fp32, take the chunk's row
+//    maxima (redux + a named barrier), keep a lazy running max M per row (moved only
+//    when a chunk max exceeds it by more than kLazy, after rescaling O and the sums in
+//    tensor memory), and write p = 2^(z - M) and the weights W_g (fp16) to shared memory.
+// The CTA partials of a (sequence, kv-head, row block) are combined by one fixed binary
+// tree over the split index; the last CTA to finish (one atomic counter) completes it
+// and writes out and lse.  The chunk ranges depend only on the shape and the SM count,
+// so the result is bit-identical for every ring depth.
 #include <cfloat>
 #include <climits>
 
 #include "mq_device.cuh"
 #include "mq_kernels.h"
+#include "mq_tc.cuh"
 
 namespace mq {
 
 // lazy-max threshold of the online softmax, in log2 units (weights stay <= 2^4)
 constexpr float kLazy = 4.0f;
+constexpr int kThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2-5 values, warps 6-9 softmax
+constexpr int kTmemCols = 512;
 
 template <int D, int ROWS>
-struct Cfg {
+struct Tc {
     static constexpr int PB = page_bytes(D);
-    static constexpr int NG = D / 32;            // V groups (= int8 k-steps of 32 channels)
-    static constexpr int KS = D / 32;
-    static constexpr int MTQ = (ROWS + 15) / 16; // QK m-tiles (16 query rows each)
-    static constexpr int NTP = ROWS / 8;         // PV n-tiles (8 query rows each)
-    static constexpr int MTP = D / 16;           // PV m-tiles (16 channels each)
-    static constexpr int SLOTS = ROWS / 8;       // query rows owned by a lane: 8k + g
-    static constexpr int KCH = D / 32;           // K 16-byte chunks per lane per page
-    static constexpr int VCH = D / 64;           // V code chunks per lane per page
-    static constexpr int SCH = D / 64;           // V scale chunks per lane per page
-    static constexpr bool HI = ROWS > 8;         // rows g+8 of a QK m-tile are real rows
-    static constexpr int PART = ROWS * D + 2 * ROWS;                 // floats of one partial
+    static constexpr int REC = rec_bytes(D);
+    static constexpr int G = D / 32;                              // value groups
+    static constexpr int H = D / 128;                             // 128-channel halves (PV M tiles)
+    static constexpr int NQ = (3 * ROWS + 15) / 16 * 16;          // score MMA N: 3 limbs x rows
+    static constexpr int NO = 4 * ROWS;                           // value MMA N per half
+    static constexpr int NB = ((G + 1) * ROWS + 15) / 16 * 16;    // weight columns: W_0..W_{G-1}, p
+    static constexpr int NSB = (D == 128 && ROWS == 32) ? 1 : 2;  // score buffers in TMEM
+    static constexpr int NVB = (D == 256 && ROWS == 16) ? 1 : 2;  // V^T buffers in TMEM
+    // tensor-memory columns
+    static constexpr int T_S = 0;
+    static constexpr int T_O = NSB * NQ;
+    static constexpr int T_SUM = T_O + H * NO;
+    static constexpr int T_VT = (T_SUM + NB + 31) / 32 * 32;
+    static constexpr int T_END = T_VT + NVB * H * 64;
+    static constexpr int WBYTES = kChunkTokens * NB * 2;          // one weight buffer
+    static constexpr int LBO_W = NB / 8 * 128;                    // its 8-token group stride
+    static constexpr int PART = ROWS * D + 2 * ROWS;              // floats of one partial
+    static_assert(T_END <= kTmemCols, "tensor memory budget");
+    static_assert(NQ <= 256 && NB <= 256 && NO <= 256, "MMA N range");
 };
 
 struct Smem {
-    size_t ring, part, fin, coef, qfrag, flags, mbar, bt, misc, heap, total;
+    size_t ring, wbuf, qlimb, fmat, part, xch, crow, lim, pgbad, mbar, misc, heap, fin, total;
 };
 
-// W warps, R ring slots per warp, SD partial entries per warp (entry 0 holds the warp's
-// result for the CTA tree; the others are left siblings of its binary counter).
+// NS = ring stages (chunks of 8 pages)
 template <int D, int ROWS>
-__host__ __device__ inline Smem smem_layout(int W, int R, int SD) {
-    using C = Cfg<D, ROWS>;
+__host__ __device__ inline Smem smem_layout(int NS) {
+    using T = Tc<D, ROWS>;
     Smem s{};
-    size_t off = 0;
     auto al = [](size_t x, size_t a) { return (x + a - 1) / a * a; };
+    size_t off = 0;
     s.ring = off;
-    off += (size_t)W * R * C::PB;
-    off = al(off, 16);
+    off += (size_t)NS * kChunkPages * T::PB;
+    off = al(off, 128);
+    s.wbuf = off;
+    off += (size_t)2 * T::WBYTES;
+    // the final cross-CTA merge reuses ring + weight buffers (idle by then)
+    s.heap = 0;
+    s.fin = al((size_t)2 * kMaxSplits * ROWS * 16, 16);
+    if (s.fin + (size_t)T::PART * 4 > off) return Smem{};   // does not fit: total = 0
+    off = al(off, 128);
+    s.qlimb = off;
+    off += (size_t)T::NQ * D;
+    off = al(off, 128);
+    s.fmat = off;
+    off += 4096;
     s.part = off;
-    off += (size_t)W * SD * C::PART * 4;
-    s.heap = 0;  // the final merge reuses ring + part
-    const size_t heap_bytes = (size_t)2 * kMaxSplits * ROWS * 4 * 4;
-    if (off < heap_bytes) off = heap_bytes;
-    off = al(off, 16);
-    s.fin = off;                      // the final merge's result (outside the heap)
-    off += (size_t)C::PART * 4;
-    s.coef = off;
-    off += (size_t)8 * ROWS * 2 * 4;  // up to 8 merges per phase
-    s.qfrag = off;
-    off += (size_t)C::MTQ * C::KS * 3 * 32 * 16;
-    s.flags = off;
-    off += 64 * 4;
+    off += (size_t)T::PART * 4;
+    s.xch = off;
+    off += (size_t)2 * ROWS * 4 * 4;
+    s.crow = off;
+    off += (size_t)ROWS * 4;
+    s.lim = off;
+    off += (size_t)ROWS * 4;
+    s.pgbad = off;
+    off += (size_t)NS * kChunkPages * 4;
     off = al(off, 8);
     s.mbar = off;
-    off += (size_t)W * R * 8;
-    s.bt = off;
-    off += (size_t)W * 4 * kChunkPages * 4;
+    off += (size_t)(2 * NS + 12) * 8;
     s.misc = off;
     off += 64;
     s.total = al(off, 128);
@@ -128,14 +150,25 @@ __device__ __forceinline__ float load_q(const DecodeParams& p, size_t i) {
     return ld_f32<__half>(p.q, i);
 }
 
+__device__ __forceinline__ void stsa128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ uint32_t ldsa16(uint32_t a) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float h_bits_to_f32(uint32_t bits) {
+    return __half2float(__ushort_as_half((unsigned short)bits));
+}
+
 template <int D, int ROWS>
-__global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_kernel(const DecodeParams p) {
-    using C = Cfg<D, ROWS>;
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int W = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int R = p.pages_per_stage;
-    const Smem S = smem_layout<D, ROWS>(W, R, p.stack_depth);
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p) {
+    using T = Tc<D, ROWS>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int NS = p.stages;
+    const Smem S = smem_layout<D, ROWS>(NS);
     const int b = blockIdx.z, hk = blockIdx.y / p.n_rb, rb = blockIdx.y % p.n_rb, sp = blockIdx.x;
     const unsigned FULL = 0xffffffffu;
 
@@ -152,19 +185,62 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
     const int n_chunks = (L + kChunkTokens - 1) / kChunkTokens;
     const int c0 = sp * p.cpc;
     if (c0 >= n_chunks) return;
-    const int c1 = min(c0 + p.cpc, n_chunks);
+    const int n_ck = min(c0 + p.cpc, n_chunks) - c0;
     const int n_splits = (n_chunks + p.cpc - 1) / p.cpc;
-    const int n_rounds = (c1 - c0 + W - 1) / W;
 
-    int* misc = reinterpret_cast<int*>(smem + S.misc);
-    int* flags = reinterpret_cast<int*>(smem + S.flags);   // [0..W): warp partial empty
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S.mbar) + warp * R;
-    int* bt = reinterpret_cast<int*>(smem + S.bt) + warp * 4 * kChunkPages;
-    uint8_t* ring = smem + S.ring + (size_t)warp * R * C::PB;
+    int* misc = reinterpret_cast<int*>(smem + S.misc);   // 0 qoff, 1 abort, 2 last CTA, 3 TMEM base
+    volatile int* abort_flag = misc + 1;
     float* part = reinterpret_cast<float*>(smem + S.part);
-    float* coef = reinterpret_cast<float*>(smem + S.coef);
+    float* crow_s = reinterpret_cast<float*>(smem + S.crow);
+    int* lim_s = reinterpret_cast<int*>(smem + S.lim);
+    int* pgbad = reinterpret_cast<int*>(smem + S.pgbad);
+    const uint32_t bar0 = smem_u32(smem + S.mbar);
+    auto full_b = [&](int s) { return bar0 + 8u * (uint32_t)s; };
+    auto empty_b = [&](int s) { return bar0 + 8u * (uint32_t)(NS + s); };
+    const uint32_t sfull_b = bar0 + 8u * (uint32_t)(2 * NS);   // [2] score buffer written
+    const uint32_t sfree_b = sfull_b + 16;                     // [2] score buffer read
+    const uint32_t wfull_b = sfree_b + 16;                     // [2] weights written
+    const uint32_t vfull_b = wfull_b + 16;                     // [2] V^T written
+    const uint32_t pvdone_b = vfull_b + 16;                    // [2] value MMAs of a chunk done
+    const uint32_t xfull_b = pvdone_b + 16;                    // [2] chunk row maxima exchanged
 
-    // ---- query-row offset of this sequence (sum of n_q of earlier sequences) ----
+    // A bounded wait that the whole warp agrees on; a timeout raises the CTA's abort
+    // flag (every role then stops taking new work) and the device error word.
+    auto wait_warp = [&](uint32_t bar, uint32_t parity) -> bool {
+        bool ok = *abort_flag == 0 && mbar_wait_bounded(bar, parity);
+        ok = __all_sync(FULL, ok);
+        if (!ok && lane == 0) {
+            if (*abort_flag == 0) atomicOr(p.err, kErrTimeout);
+            *abort_flag = 1;
+        }
+        return ok;
+    };
+    auto wait_one = [&](uint32_t bar, uint32_t parity) -> bool {   // single thread
+        if (*abort_flag != 0) return false;
+        if (mbar_wait_bounded(bar, parity)) return true;
+        atomicOr(p.err, kErrTimeout);
+        *abort_flag = 1;
+        return false;
+    };
+
+    // ---- set-up: barriers, query-row offset, TMEM, constant operands ----
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; s++) {
+            mbar_init(full_b(s), 1);
+            mbar_init(empty_b(s), 9);   // QK commit + 4 value warps + 4 softmax warps
+        }
+        for (int j = 0; j < 2; j++) {
+            mbar_init(sfull_b + 8 * j, 1);
+            mbar_init(sfree_b + 8 * j, 4);
+            mbar_init(wfull_b + 8 * j, 4);
+            mbar_init(vfull_b + 8 * j, 4);
+            mbar_init(pvdone_b + 8 * j, 1);
+            mbar_init(xfull_b + 8 * j, 4);
+        }
+        mbar_fence_init();
+        misc[1] = 0;
+        misc[2] = 0;
+    }
     if (warp == 0) {
         int s = 0;
         for (int i = lane; i < b; i += 32) s += min(max(__ldg(p.n_q_per_seq + i), 0), p.max_q);
@@ -172,530 +248,420 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
         if (lane == 0) misc[0] = s;
     }
-    if (lane == 0) {
-        for (int s = 0; s < R; s++) mbar_init(smem_u32(&bars[s]), 1);
-        mbar_fence_init();
+    if (warp == 1) {
+        tmem_alloc(smem_u32(misc + 3), kTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
     }
-    if (threadIdx.x == 0) misc[1] = 0;
+    if (warp >= 2 && warp < 6) {
+        // the all-ones A operand of the sum MMA, and the zero padding rows of the limb operand
+        const int tid = threadIdx.x - 64;
+        uint4* f = reinterpret_cast<uint4*>(smem + S.fmat);
+        for (int i = tid; i < 256; i += 128) f[i] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+        uint4* z = reinterpret_cast<uint4*>(smem + S.qlimb + (size_t)3 * ROWS * D);
+        for (int i = tid; i < (T::NQ - 3 * ROWS) * D / 16; i += 128) z[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+    }
     __syncthreads();
     const int qoff = misc[0];
 
-    // ---- q -> three 8-bit limbs of a 23-bit fixed-point value per row ----------
-    // Lane (g, t) owns rows 16*mt + 8*h + g and channels [t*D/4, (t+1)*D/4).  The
-    // A fragment of mma.m16n8k32 for k-step ks holds, for row g (h = 0) and g + 8
-    // (h = 1), channels t*D/4 + 8*ks + {0..3} (regs 0/1) and + {4..7} (regs 2/3).
-    float crow[C::SLOTS];
-    int lim[C::SLOTS];
-    uint32_t* qfrag_s = reinterpret_cast<uint32_t*>(smem + S.qfrag);
+    // ---- q -> three signed 8-bit limbs of a 23-bit fixed-point value per row ----
+    // Q = rint(q * 2^(22 - E)) with |q| < 2^E the row's absmax bound, |Q| <= 2^22, and
+    // Q = l2 * 2^16 + l1 * 2^8 + l0 with l0, l1 in [-128, 127] and |l2| <= 65.  Limb k
+    // of row r is row k * ROWS + r of the N x D (K-major) score operand.
+    if (warp >= 6) {
+        const int tid = threadIdx.x - 192;
+        constexpr int SL = D / 8;   // 8-channel slices of a row
+        for (int it = tid; it < ROWS * SL; it += 128) {
+            const int r = it / SL, sl = it % SL;
+            const bool real = r < rows_here;
+            const int rr = row0 + r, j = real ? rr / p.group : 0, hq = real ? rr % p.group : 0;
+            const long long qrow = (long long)qoff + j;
+            const bool qok = real && qrow < p.total_q;
+            if (real && !qok && sl == 0) atomicOr(p.err, kErrBadRow);
+            const size_t base = ((size_t)qrow * p.n_q_heads + (size_t)hk * p.group + hq) * D + (size_t)8 * sl;
+            float qv[8];
+            float amax = 0.0f;
 #pragma unroll
-    for (int k = 0; k < C::SLOTS; k++) {
-        const int mt = k >> 1, h = k & 1;
-        const int rl = 8 * k + g;  // local row
-        const int r = row0 + rl;
-        const bool real = rl < rows_here;
-        const int j = real ? r / p.group : 0, hq = real ? r % p.group : 0;
-        const long long qrow = (long long)qoff + j;
-        const bool qok = real && qrow < p.total_q;
-        if (real && !qok && t == 0) atomicOr(p.err, kErrBadRow);
-        constexpr int CH = D / 4;
-        float amax = 0.0f;
-        const size_t base = ((size_t)qrow * p.n_q_heads + (size_t)hk * p.group + hq) * D + (size_t)t * CH;
-        // two passes over the lane's channels (max, then limbs) keep few values live
-#pragma unroll 8
-        for (int c = 0; c < CH; c++) amax = fmaxf(amax, fabsf(qok ? load_q(p, base + c) : 0.0f));
-        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
-        int E = 0;
-        if (amax > 0.0f) frexpf(amax, &E);  // amax < 2^E
-        const bool zero_row = !(amax >= 0x1p-100f);
-        const float up = zero_row ? 0.0f : ldexpf(1.0f, 22 - E);
-        crow[k] = zero_row ? 0.0f : ldexpf(p.scale_log2, E - 22);
-        lim[k] = real ? (L - nq + j + 1) : L;
-#pragma unroll
-        for (int ks = 0; ks < C::KS; ks++) {
-            uint32_t w[3][2];
-#pragma unroll
-            for (int half = 0; half < 2; half++) {
-                uint32_t l2 = 0, l1 = 0, l0 = 0;
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    const float qv = qok ? load_q(p, base + 8 * ks + 4 * half + i) : 0.0f;
-                    const int Q = (int)rintf(__fmul_rn(qv, up));
-                    l2 |= (uint32_t)((Q >> 16) & 0xFF) << (8 * i);
-                    l1 |= (uint32_t)((Q >> 8) & 0xFF) << (8 * i);
-                    l0 |= (uint32_t)(Q & 0xFF) << (8 * i);
-                }
-                w[0][half] = l2;
-                w[1][half] = l1;
-                w[2][half] = l0;
+            for (int e = 0; e < 8; e++) {
+                qv[e] = qok ? load_q(p, base + e) : 0.0f;
+                amax = fmaxf(amax, fabsf(qv[e]));
             }
 #pragma unroll
-            for (int lb = 0; lb < 3; lb++) {
-                if (warp == 0) {
-                    uint32_t* f = qfrag_s + ((((size_t)mt * C::KS + ks) * 3 + lb) * 32 + lane) * 4;
-                    if constexpr (C::HI) {
-                        f[h] = w[lb][0];
-                        f[2 + h] = w[lb][1];
-                    } else {   // rows g + 8 are padding: keep regs 0 and 2 only, as 64 bits
-                        f[0] = w[lb][0];
-                        f[1] = w[lb][1];
-                    }
-                }
+            for (int o = 1; o < SL; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
+            int E = 0;
+            if (amax > 0.0f) frexpf(amax, &E);   // amax < 2^E
+            const bool zero_row = !(amax >= 0x1p-100f);
+            const float up = zero_row ? 0.0f : ldexpf(1.0f, 22 - E);
+            if (sl == 0) {
+                crow_s[r] = zero_row ? 0.0f : ldexpf(p.scale_log2, E - 22);
+                lim_s[r] = real ? (L - nq + j + 1) : L;
+            }
+            uint32_t w[3][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}};
+#pragma unroll
+            for (int e = 0; e < 8; e++) {
+                const int Q = (int)rintf(__fmul_rn(qv[e], up));
+                const int l0 = ((Q + 128) & 255) - 128;
+                const int Q1 = (Q - l0) >> 8;
+                const int l1 = ((Q1 + 128) & 255) - 128;
+                const int l2 = (Q1 - l1) >> 8;
+                w[0][e / 4] |= (uint32_t)(l2 & 255) << (8 * (e % 4));
+                w[1][e / 4] |= (uint32_t)(l1 & 255) << (8 * (e % 4));
+                w[2][e / 4] |= (uint32_t)(l0 & 255) << (8 * (e % 4));
+            }
+#pragma unroll
+            for (int k = 0; k < 3; k++) {
+                const int n = k * ROWS + r;
+                const size_t off = (size_t)(n / 8) * (8 * D) + (size_t)(sl / 2) * 128 + (n % 8) * 16 + (sl % 2) * 8;
+                *reinterpret_cast<uint2*>(smem + S.qlimb + off) = make_uint2(w[k][0], w[k][1]);
             }
         }
+        fence_proxy_async_smem();
     }
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)misc[3];
+    const uint32_t ring = smem_u32(smem + S.ring);
 
-    // ---- this warp's chunks: an aligned run [wc0, wc1) of Q = cpc / W chunks ----
-    const uint64_t policy = l2_evict_first_policy();
-    const int Q = p.cpc / W;
-    const int SD = p.stack_depth;                  // partial entries per warp
-    const int wc0 = c0 + warp * Q;
-    const int my_chunks = max(0, min(wc0 + Q, c1) - wc0);
-    const int my_pages = my_chunks > 0 ? min((wc0 + my_chunks) * kChunkPages, n_pages) - wc0 * kChunkPages : 0;
-    // Block-table entries of the run: a ring of four chunks' entries in shared memory,
-    // fetched two chunks ahead into a register, so that no load is ever waited for.
-    constexpr int kUnused = INT_MIN;
-    auto bt_fetch = [&](int i) -> int {   // entry of page `lane` of the run's chunk i (lanes < 8)
-        int blk = kUnused;
-        if (i < my_chunks && lane < kChunkPages) {
-            const int lp = (wc0 + i) * kChunkPages + lane;
-            if (lp < n_pages) blk = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + lp);
-        }
-        return blk;
-    };
-    auto bt_store = [&](int i, int blk) {
-        if (i < my_chunks && lane < kChunkPages) {
-            if (blk != kUnused && (blk < 0 || (long long)blk >= p.n_blocks)) {
-                atomicOr(p.err, kErrBadBlock);
-                blk = -1;
-            }
-            bt[(i & 3) * kChunkPages + lane] = blk == kUnused ? -1 : blk;
-        }
-    };
-    bt_store(0, bt_fetch(0));
-    bt_store(1, bt_fetch(1));
-    int bt_next = bt_fetch(2);
-    __syncwarp();
-    auto issue = [&](int k, int slot) {  // lane 0 only: page k of this warp's run into `slot`
-        const int blk = bt[((k / kChunkPages) & 3) * kChunkPages + (k % kChunkPages)];
-        const uint8_t* src = p.pool + ((long long)(blk < 0 ? 0 : blk) * p.n_kv_heads + hk) * C::PB;
-        mbar_arrive_expect_tx(smem_u32(&bars[slot]), C::PB);
-        tma_load_1d(smem_u32(ring + (size_t)slot * C::PB), src, C::PB, smem_u32(&bars[slot]), policy);
-    };
-    if (lane == 0)
-        for (int k = 0; k < R && k < my_pages; k++) issue(k, k);
-
-    // the smallest visibility limit of the real rows of this row block
-    const int lim_min = L - nq + row0 / p.group + 1;
-    // 32-bit shared-window addresses: ring slot 0 and this lane's q fragments
-    const uint32_t ring_s = smem_u32(ring), lane16 = (uint32_t)lane * 16u;
-    const uint32_t qf_s = smem_u32(qfrag_s) + lane16;
-    float* my_ent = part + (size_t)warp * SD * C::PART;   // this warp's partial entries
-
-    bool aborted = false;
-    int k_abort = 0;       // first page not waited for after a timeout
-    int k_next = 0;        // next page of this warp to consume
-    int slot = 0;          // its ring slot (k_next % R) and mbarrier phase ((k_next / R) & 1)
-    uint32_t phase = 0;
-
-    // The run's result, as (O fragments, m and l of the lane's O rows 8n + 2t + e).
-    float O[C::MTP][C::NTP][4];
-    float mo[C::NTP][2], lo[C::NTP][2];
-    int n_ent = 0;            // binary-counter entries in shared memory (warp-uniform)
-    uint32_t ent_lvl = 0;     // their levels, 4 bits each
-
-    // entry e (left sibling) (+) registers (right sibling) -> registers
-    auto merge_entry = [&](int e) {
-        __syncwarp();
-        const float* ent = my_ent + (size_t)e * C::PART;
-        float ca[C::NTP][2], cb[C::NTP][2];
-#pragma unroll
-        for (int n = 0; n < C::NTP; n++)
-#pragma unroll
-            for (int e2 = 0; e2 < 2; e2++) {
-                const int r = 8 * n + 2 * t + e2;
-                float m, l;
-                merge_coef(ent[ROWS * D + r], ent[ROWS * D + ROWS + r], mo[n][e2], lo[n][e2], m, l, ca[n][e2],
-                           cb[n][e2]);
-                mo[n][e2] = m;
-                lo[n][e2] = l;
-            }
-#pragma unroll
-        for (int n = 0; n < C::NTP; n++)
-#pragma unroll
-            for (int q = 0; q < C::NG; q++) {
-                const int ch = 32 * q + 4 * g, r0 = 8 * n + 2 * t;
-                const float4 L0 = *reinterpret_cast<const float4*>(ent + (size_t)r0 * D + ch);
-                const float4 L1 = *reinterpret_cast<const float4*>(ent + (size_t)(r0 + 1) * D + ch);
-                O[2 * q][n][0] = merge_val(L0.x, O[2 * q][n][0], ca[n][0], cb[n][0]);
-                O[2 * q][n][2] = merge_val(L0.y, O[2 * q][n][2], ca[n][0], cb[n][0]);
-                O[2 * q + 1][n][0] = merge_val(L0.z, O[2 * q + 1][n][0], ca[n][0], cb[n][0]);
-                O[2 * q + 1][n][2] = merge_val(L0.w, O[2 * q + 1][n][2], ca[n][0], cb[n][0]);
-                O[2 * q][n][1] = merge_val(L1.x, O[2 * q][n][1], ca[n][1], cb[n][1]);
-                O[2 * q][n][3] = merge_val(L1.y, O[2 * q][n][3], ca[n][1], cb[n][1]);
-                O[2 * q + 1][n][1] = merge_val(L1.z, O[2 * q + 1][n][1], ca[n][1], cb[n][1]);
-                O[2 * q + 1][n][3] = merge_val(L1.w, O[2 * q + 1][n][3], ca[n][1], cb[n][1]);
-            }
-    };
-    // registers -> entry e (natural layout: O [ROWS][D], m [ROWS], l [ROWS])
-    auto write_entry = [&](int e) {
-        float* ent = my_ent + (size_t)e * C::PART;
-#pragma unroll
-        for (int n = 0; n < C::NTP; n++)
-#pragma unroll
-            for (int q = 0; q < C::NG; q++) {
-                const int ch = 32 * q + 4 * g, r0 = 8 * n + 2 * t;
-                *reinterpret_cast<float4*>(ent + (size_t)r0 * D + ch) =
-                    make_float4(O[2 * q][n][0], O[2 * q][n][2], O[2 * q + 1][n][0], O[2 * q + 1][n][2]);
-                *reinterpret_cast<float4*>(ent + (size_t)(r0 + 1) * D + ch) =
-                    make_float4(O[2 * q][n][1], O[2 * q][n][3], O[2 * q + 1][n][1], O[2 * q + 1][n][3]);
-            }
-        if (g == 0) {
-#pragma unroll
-            for (int n = 0; n < C::NTP; n++)
-#pragma unroll
-                for (int e2 = 0; e2 < 2; e2++) {
-                    ent[ROWS * D + 8 * n + 2 * t + e2] = mo[n][e2];
-                    ent[ROWS * D + ROWS + 8 * n + 2 * t + e2] = lo[n][e2];
+    if (warp == 0) {
+        // ================= TMA producer =================
+        const uint64_t policy = l2_evict_first_policy();
+        int issued = 0;
+        for (int i = 0; i < n_ck; i++) {
+            const int s = i % NS;
+            if (i >= NS && !wait_warp(empty_b(s), (uint32_t)((i - NS) / NS) & 1u)) break;
+            const int c = c0 + i;
+            const int npg = min(kChunkPages, n_pages - c * kChunkPages);
+            int blk = 0;
+            bool bad = true;
+            if (lane < npg) {
+                blk = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + (long long)c * kChunkPages + lane);
+                bad = blk < 0 || (long long)blk >= p.n_blocks;
+                if (bad) {
+                    atomicOr(p.err, kErrBadBlock);
+                    blk = 0;   // read a valid page; its tokens are masked
                 }
+            }
+            if (lane < kChunkPages) pgbad[s * kChunkPages + lane] = bad ? 1 : 0;
+            __syncwarp();
+            if (lane == 0) mbar_arrive_expect_tx(full_b(s), (uint32_t)(npg * T::PB));
+            __syncwarp();
+            if (lane < npg)
+                tma_load_1d(ring + (uint32_t)((s * kChunkPages + lane) * T::PB),
+                            p.pool + ((long long)blk * p.n_kv_heads + hk) * T::PB, T::PB, full_b(s), policy);
+            issued = i + 1;
+        }
+        // after an abort: let copies still in flight land before the CTA leaves
+        if (*abort_flag != 0 && lane == 0)
+            for (int k = max(0, issued - NS); k < issued; k++) mbar_wait_bounded(full_b(k % NS), (uint32_t)(k / NS) & 1u);
+    } else if (warp == 1) {
+        // ================= MMA issuer (one thread) =================
+        if (lane == 0) {
+            const uint32_t wb0 = smem_u32(smem + S.wbuf), ql = smem_u32(smem + S.qlimb);
+            constexpr uint32_t IDQ = instr_desc(2, 1, 1, 0, 0, 128, T::NQ);   // s32 <- s8 x s8, K-major
+            constexpr uint32_t IDO = instr_desc(1, 0, 0, 0, 1, 128, T::NO);   // f32 <- f16 x f16, B MN-major
+            constexpr uint32_t IDS = instr_desc(1, 0, 0, 0, 1, 128, T::NB);
+            const uint64_t fdesc = smem_desc(smem_u32(smem + S.fmat), 128, 256);
+            uint32_t last_bar = 0, last_par = 0;
+            for (int i = 0; i <= n_ck; i++) {
+                if (i < n_ck) {
+                    const int s = i % NS, sb = i % T::NSB;
+                    if (!wait_one(full_b(s), (uint32_t)(i / NS) & 1u)) break;
+                    if (i >= T::NSB && !wait_one(sfree_b + 8 * sb, (uint32_t)((i - T::NSB) / T::NSB) & 1u)) break;
+                    tc_fence_after();
+                    const uint32_t a0 = ring + (uint32_t)(s * kChunkPages * T::PB);
+#pragma unroll
+                    for (int k = 0; k < D / 32; k++)
+                        mma_i8_ss(tmem + T::T_S + sb * T::NQ, smem_desc(a0 + 256 * k, 128, T::REC),
+                                  smem_desc(ql + 256 * k, 128, 8 * D), IDQ, k > 0 ? 1u : 0u);
+                    tc_commit(sfull_b + 8 * sb);
+                    tc_commit(empty_b(s));
+                    last_bar = sfull_b + 8 * sb;
+                    last_par = (uint32_t)(i / T::NSB) & 1u;
+                }
+                if (i >= 1) {
+                    const int j = i - 1, wb = j & 1, vb = j % T::NVB;
+                    if (!wait_one(wfull_b + 8 * wb, (uint32_t)(j >> 1) & 1u)) break;
+                    if (!wait_one(vfull_b + 8 * vb, (uint32_t)(j / T::NVB) & 1u)) break;
+                    tc_fence_after();
+                    const uint32_t w0 = wb0 + (uint32_t)(wb * T::WBYTES);
+#pragma unroll 1
+                    for (int ks = 0; ks < kChunkTokens / 16; ks++) {
+                        const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
+                        const uint32_t wk = w0 + (uint32_t)(ks * 2 * T::LBO_W);
+#pragma unroll
+                        for (int h = 0; h < T::H; h++)
+                            mma_f16_ts(tmem + T::T_O + h * T::NO, tmem + T::T_VT + (vb * T::H + h) * 64 + 8 * ks,
+                                       smem_desc(wk + (uint32_t)(h * 64 * ROWS), T::LBO_W, 128), IDO, acc);
+                        mma_f16_ss(tmem + T::T_SUM, fdesc, smem_desc(wk, T::LBO_W, 128), IDS, acc);
+                    }
+                    tc_commit(pvdone_b + 8 * wb);
+                    last_bar = pvdone_b + 8 * wb;
+                    last_par = (uint32_t)(j >> 1) & 1u;
+                }
+            }
+            // after an abort: the MMAs already issued finish before TMEM is released
+            if (*abort_flag != 0 && last_bar != 0) mbar_wait_bounded(last_bar, last_par);
         }
         __syncwarp();
-    };
-
-    // registers (left sibling) (+) entry (right sibling) -> registers
-    auto merge_right = [&](const float* ent) {
-        float ca[C::NTP][2], cb[C::NTP][2];
+    } else if (warp < 6) {
+        // ================= value codes -> V^T in tensor memory =================
+        const int q = warp & 3;
+        for (int i = 0; i < n_ck; i++) {
+            const int s = i % NS, vb = i % T::NVB;
+            if (!wait_warp(full_b(s), (uint32_t)(i / NS) & 1u)) break;
+            if (i >= T::NVB && !wait_warp(pvdone_b + 8 * ((i - T::NVB) & 1), (uint32_t)((i - T::NVB) >> 1) & 1u))
+                break;
+            tc_fence_after();
+            const uint32_t st = ring + (uint32_t)(s * kChunkPages * T::PB) + rec_v_off(D);
 #pragma unroll
-        for (int n = 0; n < C::NTP; n++)
+            for (int h = 0; h < T::H; h++) {
+                const uint32_t cw = st + 4u * (uint32_t)(128 * h + 32 * q + lane);
 #pragma unroll
-            for (int e2 = 0; e2 < 2; e2++) {
-                const int r = 8 * n + 2 * t + e2;
-                float m, l;
-                merge_coef(mo[n][e2], lo[n][e2], ent[ROWS * D + r], ent[ROWS * D + ROWS + r], m, l, ca[n][e2],
-                           cb[n][e2]);
-                mo[n][e2] = m;
-                lo[n][e2] = l;
+                for (int pp = 0; pp < 2; pp++) {
+                    uint32_t r[32];
+#pragma unroll
+                    for (int p4 = 0; p4 < 4; p4++)
+#pragma unroll
+                        for (int tg = 0; tg < 2; tg++) {
+                            const uint32_t w = ldsa32(cw + (uint32_t)((4 * pp + p4) * T::PB + tg * T::REC));
+                            // tokens (2k, 2k+1) of the group: bits 4k..4k+3 and 16+4k..; flipping
+                            // bit 3 turns the two's-complement code into u = code + 8
+                            r[8 * p4 + 4 * tg + 0] = lop_and_xor(w, 0x000F000Fu, 0x00080008u);
+                            r[8 * p4 + 4 * tg + 1] = lop_and_xor(w >> 4, 0x000F000Fu, 0x00080008u);
+                            r[8 * p4 + 4 * tg + 2] = lop_and_xor(w >> 8, 0x000F000Fu, 0x00080008u);
+                            r[8 * p4 + 4 * tg + 3] = lop_and_xor(w >> 12, 0x000F000Fu, 0x00080008u);
+                        }
+                    tmem_st32(tmem_at(tmem, 32 * q, T::T_VT + (vb * T::H + h) * 64 + 32 * pp), r);
+                }
             }
-#pragma unroll
-        for (int n = 0; n < C::NTP; n++)
-#pragma unroll
-            for (int q = 0; q < C::NG; q++) {
-                const int ch = 32 * q + 4 * g, r0 = 8 * n + 2 * t;
-                const float4 R0 = *reinterpret_cast<const float4*>(ent + (size_t)r0 * D + ch);
-                const float4 R1 = *reinterpret_cast<const float4*>(ent + (size_t)(r0 + 1) * D + ch);
-                O[2 * q][n][0] = merge_val(O[2 * q][n][0], R0.x, ca[n][0], cb[n][0]);
-                O[2 * q][n][2] = merge_val(O[2 * q][n][2], R0.y, ca[n][0], cb[n][0]);
-                O[2 * q + 1][n][0] = merge_val(O[2 * q + 1][n][0], R0.z, ca[n][0], cb[n][0]);
-                O[2 * q + 1][n][2] = merge_val(O[2 * q + 1][n][2], R0.w, ca[n][0], cb[n][0]);
-                O[2 * q][n][1] = merge_val(O[2 * q][n][1], R1.x, ca[n][1], cb[n][1]);
-                O[2 * q][n][3] = merge_val(O[2 * q][n][3], R1.y, ca[n][1], cb[n][1]);
-                O[2 * q + 1][n][1] = merge_val(O[2 * q + 1][n][1], R1.z, ca[n][1], cb[n][1]);
-                O[2 * q + 1][n][3] = merge_val(O[2 * q + 1][n][3], R1.w, ca[n][1], cb[n][1]);
-            }
-    };
-    // entry -> registers
-    auto load_entry = [&](const float* ent) {
-#pragma unroll
-        for (int n = 0; n < C::NTP; n++)
-#pragma unroll
-            for (int e2 = 0; e2 < 2; e2++) {
-                mo[n][e2] = ent[ROWS * D + 8 * n + 2 * t + e2];
-                lo[n][e2] = ent[ROWS * D + ROWS + 8 * n + 2 * t + e2];
-            }
-#pragma unroll
-        for (int n = 0; n < C::NTP; n++)
-#pragma unroll
-            for (int q = 0; q < C::NG; q++) {
-                const int ch = 32 * q + 4 * g, r0 = 8 * n + 2 * t;
-                const float4 R0 = *reinterpret_cast<const float4*>(ent + (size_t)r0 * D + ch);
-                const float4 R1 = *reinterpret_cast<const float4*>(ent + (size_t)(r0 + 1) * D + ch);
-                O[2 * q][n][0] = R0.x;
-                O[2 * q][n][2] = R0.y;
-                O[2 * q + 1][n][0] = R0.z;
-                O[2 * q + 1][n][2] = R0.w;
-                O[2 * q][n][1] = R1.x;
-                O[2 * q][n][3] = R1.y;
-                O[2 * q + 1][n][1] = R1.z;
-                O[2 * q + 1][n][3] = R1.w;
-            }
-    };
-
-    for (int i = 0; i < my_chunks; i++) {
-        if (i >= 1) {
-            bt_store(i + 1, bt_next);
-            bt_next = bt_fetch(i + 2);
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(vfull_b + 8 * vb);
+                mbar_arrive(empty_b(s));
+            }
         }
-        const int c = wc0 + i;
+    } else {
+        // ================= softmax and weights (one TMEM lane = one token) =================
+        const int sw = warp - 6, q = warp & 3, t = 32 * q + lane;
+        const int tp = t / 16, ttg = (t / 8) & 1, tt = t & 7;
+        const uint32_t wb0 = smem_u32(smem + S.wbuf);
+        float* xch = reinterpret_cast<float*>(smem + S.xch);
+        float crow[ROWS], M[ROWS];
+        int lim[ROWS];
 #pragma unroll
-        for (int j = 0; j < C::MTP; j++)
-#pragma unroll
-            for (int n = 0; n < C::NTP; n++)
-#pragma unroll
-                for (int e = 0; e < 4; e++) O[j][n][e] = 0.0f;
-        float mrun[C::SLOTS], lrun[C::SLOTS];
-#pragma unroll
-        for (int k = 0; k < C::SLOTS; k++) {
-            mrun[k] = -INFINITY;
-            lrun[k] = 0.0f;
+        for (int r = 0; r < ROWS; r++) {
+            crow[r] = crow_s[r];
+            lim[r] = lim_s[r];
+            M[r] = -INFINITY;
         }
-        const int pages_here = min(kChunkPages, n_pages - c * kChunkPages);
-        for (int pi = 0; pi < pages_here; pi++, k_next++) {
-            if (!aborted && !mbar_wait_bounded(smem_u32(&bars[slot]), phase)) {
-                aborted = true;
-                k_abort = k_next;
-                if (lane == 0) atomicOr(p.err, kErrTimeout);
-            }
-            const uint32_t pg = ring_s + (uint32_t)slot * C::PB;   // this page
-            const uint32_t pgl = pg + lane16;
-            const int lp = c * kChunkPages + pi;
-            const bool bad = bt[(i & 3) * kChunkPages + pi] < 0;
-            // every token of the page visible to every row: no per-element masking
-            const bool full = !bad && (lp + 1) * kPageTokens <= lim_min;
-
-            // ---- scores: int8 QK^T on the tensor cores ----
-            const float2 skA = __half22float2(u32_as_h2(ldsa32(pg + k_scale_off(D) + 4 * t)));
-            const float2 skB = __half22float2(u32_as_h2(ldsa32(pg + k_scale_off(D) + 16 + 4 * t)));
-            float z[C::SLOTS][2][2];
+        float Mlane = -INFINITY;   // M of row `lane` (lanes < ROWS)
+        const int lim_min = L - nq + row0 / p.group + 1;   // smallest limit of the real rows
+        bool ok = true;
+        for (int i = 0; i < n_ck && ok; i++) {
+            const int s = i % NS, sb = i % T::NSB, wb = i & 1;
+            const int c = c0 + i;
+            ok = wait_warp(sfull_b + 8 * sb, (uint32_t)(i / T::NSB) & 1u) && wait_warp(full_b(s), (uint32_t)(i / NS) & 1u);
+            if (!ok) break;
+            tc_fence_after();
+            // this token's scales and page flag
+            const uint32_t rec = ring + (uint32_t)((s * kChunkPages + tp) * T::PB + ttg * T::REC);
+            const float sk = h_bits_to_f32(ldsa16(rec + rec_ks_off(D) + 2 * tt));
+            float sv[T::G];
+            if constexpr (T::G == 4) {
+                const uint2 v = ldsa64(rec + rec_vs_off(D) + 8 * tt);
+                sv[0] = h_bits_to_f32(v.x & 0xFFFFu);
+                sv[1] = h_bits_to_f32(v.x >> 16);
+                sv[2] = h_bits_to_f32(v.y & 0xFFFFu);
+                sv[3] = h_bits_to_f32(v.y >> 16);
+            } else {
+                const uint4 v = ldsa128(rec + rec_vs_off(D) + 16 * tt);
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int mt = 0; mt < C::MTQ; mt++) {
-                // the lane's key chunks: token g (n-tile 0) and token g + 8 (n-tile 1)
-                uint4 kc[C::KCH];
-#pragma unroll
-                for (int ii = 0; ii < C::KCH; ii++) kc[ii] = ldsa128(pgl + ii * 512);
-                // int32 chains per limb and n-tile (exact, so any order).  The 8-row class
-                // keeps the three limbs apart for ILP; the larger classes, short of
-                // registers, shift the top limb in place before the middle one joins it.
-                constexpr bool SPLIT3 = ROWS == 8;
-                int d2[2][4], d1[SPLIT3 ? 2 : 1][4], d0[2][4];
-#pragma unroll
-                for (int nt = 0; nt < 2; nt++)
-#pragma unroll
-                    for (int ii = 0; ii < 4; ii++) {
-                        d2[nt][ii] = d0[nt][ii] = 0;
-                        if constexpr (SPLIT3) d1[nt][ii] = 0;
-                    }
-#pragma unroll
-                for (int lb = 0; lb < 3; lb++) {
-#pragma unroll
-                    for (int ks = 0; ks < C::KS; ks++) {
-                        uint32_t a[4];
-                        const uint32_t f = qf_s + (((mt * C::KS + ks) * 3 + lb) * 512);
-                        if constexpr (C::HI) {
-                            const uint4 v = ldsa128(f);
-                            a[0] = v.x;
-                            a[1] = v.y;
-                            a[2] = v.z;
-                            a[3] = v.w;
-                        } else {   // rows g + 8 are padding: their fragment registers are zero
-                            const uint2 v = ldsa64(f);
-                            a[0] = v.x;
-                            a[1] = 0u;
-                            a[2] = v.y;
-                            a[3] = 0u;
-                        }
-#pragma unroll
-                        for (int nt = 0; nt < 2; nt++) {
-                            const uint4 ch = kc[nt * (D / 64) + ks / 2];
-                            const uint32_t b0 = (ks & 1) ? ch.z : ch.x;
-                            const uint32_t b1 = (ks & 1) ? ch.w : ch.y;
-                            if (lb == 0) mma_s8s8(d2[nt], a, b0, b1);
-                            else if (lb == 1) {
-                                if constexpr (SPLIT3) mma_u8s8(d1[nt], a, b0, b1);
-                                else mma_u8s8(d2[nt], a, b0, b1);
-                            } else mma_u8s8(d0[nt], a, b0, b1);
-                        }
-                    }
-                    if constexpr (!SPLIT3) {
-                        if (lb == 0) {
-#pragma unroll
-                            for (int nt = 0; nt < 2; nt++)
-#pragma unroll
-                                for (int ii = 0; ii < 4; ii++)
-                                    if (16 * mt + 8 * (ii / 2) < ROWS) d2[nt][ii] <<= 8;
-                        }
-                    }
-                }
-#pragma unroll
-                for (int nt = 0; nt < 2; nt++)
-#pragma unroll
-                    for (int h = 0; h < 2; h++) {
-                        if (16 * mt + 8 * h < ROWS) {
-                            const int k = 2 * mt + h;
-#pragma unroll
-                            for (int e = 0; e < 2; e++) {
-                                int d21;
-                                if constexpr (SPLIT3) d21 = (d2[nt][2 * h + e] << 8) + d1[nt][2 * h + e];
-                                else d21 = d2[nt][2 * h + e];
-                                const float sc = __fmaf_rn((float)d21, 256.0f, (float)d0[nt][2 * h + e]);
-                                const float skv = nt == 0 ? (e == 0 ? skA.x : skA.y) : (e == 0 ? skB.x : skB.y);
-                                z[k][nt][e] = __fmul_rn(__fmul_rn(sc, crow[k]), skv);
-                            }
-                        }
-                    }
-            }
-
-            // ---- online softmax (log2 units) ----
-            const int tok0 = lp * kPageTokens + 2 * t;
-            float pw[C::SLOTS][2][2], alph[C::SLOTS];
-            bool resc = false;
-#pragma unroll
-            for (int k = 0; k < C::SLOTS; k++) {
-                if (!full) {
-#pragma unroll
-                    for (int nt = 0; nt < 2; nt++)
-#pragma unroll
-                        for (int e = 0; e < 2; e++) {
-                            const bool valid = !bad && (tok0 + 8 * nt + e) < lim[k];
-                            z[k][nt][e] = valid ? z[k][nt][e] : -INFINITY;
-                        }
-                }
-                float pm = fmaxf(fmaxf(z[k][0][0], z[k][0][1]), fmaxf(z[k][1][0], z[k][1][1]));
-                pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 1));
-                pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 2));
-                // Lazy reference: the row's reference max moves only when a page max
-                // exceeds it by more than kLazy (log2 units), so p = 2^(z - m) <= 2^kLazy
-                // and a rescale of O is rare.  The first finite page max always moves it
-                // (O is still zero then, so that rescale is skipped).
-                const float mnew = (pm > __fadd_rn(mrun[k], kLazy)) ? pm : mrun[k];
-                alph[k] = (mnew == mrun[k]) ? 1.0f : ex2(__fsub_rn(mrun[k], mnew));
-                resc |= (alph[k] != 1.0f) && (mrun[k] != -INFINITY);
-#pragma unroll
-                for (int nt = 0; nt < 2; nt++)
-#pragma unroll
-                    for (int e = 0; e < 2; e++) {
-                        const float pv = ex2(__fsub_rn(z[k][nt][e], mnew));
-                        pw[k][nt][e] = full ? pv : (z[k][nt][e] == -INFINITY ? 0.0f : pv);
-                    }
-                const float ps = __fadd_rn(__fadd_rn(pw[k][0][0], pw[k][0][1]), __fadd_rn(pw[k][1][0], pw[k][1][1]));
-                lrun[k] = __fadd_rn(__fmul_rn(lrun[k], alph[k]), ps);
-                mrun[k] = mnew;
-            }
-            // rescaling by exactly 1 changes nothing, so it is skipped when no row's
-            // reference moved (the common case)
-            if (__any_sync(FULL, resc)) {
-#pragma unroll
-                for (int n = 0; n < C::NTP; n++) {
-                    const float a0 = __shfl_sync(FULL, alph[n], 8 * t);
-                    const float a1 = __shfl_sync(FULL, alph[n], 8 * t + 4);
-#pragma unroll
-                    for (int j = 0; j < C::MTP; j++) {
-                        O[j][n][0] = __fmul_rn(O[j][n][0], a0);
-                        O[j][n][1] = __fmul_rn(O[j][n][1], a1);
-                        O[j][n][2] = __fmul_rn(O[j][n][2], a0);
-                        O[j][n][3] = __fmul_rn(O[j][n][3], a1);
-                    }
+                for (int k = 0; k < 4; k++) {
+                    sv[2 * k] = h_bits_to_f32(u[k] & 0xFFFFu);
+                    sv[2 * k + 1] = h_bits_to_f32(u[k] >> 16);
                 }
             }
-
-            // ---- P.V: int4 codes as exact fp16, weights p * s_v in fp16 ----
-            uint4 vcw[C::VCH], svw[C::SCH];
+            const int4 bf0 = *reinterpret_cast<const int4*>(pgbad + s * kChunkPages);
+            const int4 bf1 = *reinterpret_cast<const int4*>(pgbad + s * kChunkPages + 4);
+            const bool any_bad = (bf0.x | bf0.y | bf0.z | bf0.w | bf1.x | bf1.y | bf1.z | bf1.w) != 0;
+            const bool my_bad = pgbad[s * kChunkPages + tp] != 0;
+            // ---- scores: the three limb accumulations -> fp32 ----
+            float z[ROWS];
 #pragma unroll
-            for (int ii = 0; ii < C::VCH; ii++) vcw[ii] = ldsa128(pgl + v_code_off(D) + ii * 512);
+            for (int rg = 0; rg < ROWS / 8; rg++) {
+                uint32_t a2[8], a1[8], a0[8];
+                const uint32_t col = T::T_S + sb * T::NQ + 8 * rg;
+                tmem_ld8(tmem_at(tmem, 32 * q, col), a2);
+                tmem_ld8(tmem_at(tmem, 32 * q, col + ROWS), a1);
+                tmem_ld8(tmem_at(tmem, 32 * q, col + 2 * ROWS), a0);
+                tmem_wait_ld();
 #pragma unroll
-            for (int ii = 0; ii < C::SCH; ii++) svw[ii] = ldsa128(pg + v_scale_off(D) + t * (C::NG * 8) + ii * 16);
-#pragma unroll
-            for (int q = 0; q < C::NG; q++) {
-                const float2 s0 = __half22float2(u32_as_h2(comp(svw[(2 * q) / 4], (2 * q) % 4)));
-                const float2 s1 = __half22float2(u32_as_h2(comp(svw[(2 * q + 1) / 4], (2 * q + 1) % 4)));
-                const uint32_t x0 = comp(vcw[(2 * q) / 4], (2 * q) % 4);
-                const uint32_t x1 = comp(vcw[(2 * q + 1) / 4], (2 * q + 1) % 4);
-                const uint32_t y0 = x0 >> 8, y1 = x1 >> 8;
-                const uint32_t A0 = nib_lo_to_h2(x0), A1 = nib_hi_to_h2(x0);
-                const uint32_t A2 = nib_lo_to_h2(x1), A3 = nib_hi_to_h2(x1);
-                const uint32_t B0 = nib_lo_to_h2(y0), B1 = nib_hi_to_h2(y0);
-                const uint32_t B2 = nib_lo_to_h2(y1), B3 = nib_hi_to_h2(y1);
-#pragma unroll
-                for (int n = 0; n < C::NTP; n++) {
-                    float w00 = __fmul_rn(pw[n][0][0], s0.x), w01 = __fmul_rn(pw[n][0][1], s0.y);
-                    float w10 = __fmul_rn(pw[n][1][0], s1.x), w11 = __fmul_rn(pw[n][1][1], s1.y);
-                    if (!full) {  // masked tokens may sit next to unwritten (non-finite) scales
-                        w00 = pw[n][0][0] == 0.0f ? 0.0f : w00;
-                        w01 = pw[n][0][1] == 0.0f ? 0.0f : w01;
-                        w10 = pw[n][1][0] == 0.0f ? 0.0f : w10;
-                        w11 = pw[n][1][1] == 0.0f ? 0.0f : w11;
-                    }
-                    const uint32_t bb0 = pack_h2(w00, w01), bb1 = pack_h2(w10, w11);
-                    mma_f16(O[2 * q][n], A0, A1, A2, A3, bb0, bb1);
-                    mma_f16(O[2 * q + 1][n], B0, B1, B2, B3, bb0, bb1);
+                for (int e = 0; e < 8; e++) {
+                    const int x = (int)a2[e] * 256 + (int)a1[e];   // exact: |x| < 2^30
+                    const float sc = __fmaf_rn((float)x, 256.0f, (float)(int)a0[e]);
+                    z[8 * rg + e] = __fmul_rn(__fmul_rn(sc, crow[8 * rg + e]), sk);
                 }
             }
-            // every lane has consumed the page (its loads fed the math above): refill
-            // the slot.  The reads are complete, so the bulk copy cannot overtake them.
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0 && !aborted && k_next + R < my_pages) issue(k_next + R, slot);
-            if (++slot == R) {
-                slot = 0;
-                phase ^= 1u;
+            if (lane == 0) {
+                mbar_arrive(sfree_b + 8 * sb);
+                mbar_arrive(empty_b(s));
             }
-        }
-        // ---- chunk result: slot form (rows 8k + g) -> O-row form (rows 8n + 2t + e) ----
-        float lrow[C::SLOTS];
+            // ---- visibility: sequence end, causal drafts, unusable pages ----
+            const bool clean = (c + 1) * kChunkTokens <= lim_min && !any_bad;
+            if (!clean) {
+                const int tok = c * kChunkTokens + t;
 #pragma unroll
-        for (int k = 0; k < C::SLOTS; k++) {
-            float l = lrun[k];
-            l = __fadd_rn(l, __shfl_xor_sync(FULL, l, 1));
-            l = __fadd_rn(l, __shfl_xor_sync(FULL, l, 2));
-            lrow[k] = l;
-        }
-#pragma unroll
-        for (int n = 0; n < C::NTP; n++)
-#pragma unroll
-            for (int e2 = 0; e2 < 2; e2++) {
-                mo[n][e2] = __shfl_sync(FULL, mrun[n], 8 * t + 4 * e2);
-                lo[n][e2] = __shfl_sync(FULL, lrow[n], 8 * t + 4 * e2);
+                for (int r = 0; r < ROWS; r++)
+                    if (my_bad || tok >= lim[r]) z[r] = -INFINITY;
             }
-        // ---- binary counter over the run's chunks (aligned, so it closes the subtree) ----
-        int lvl = 0;
-        while (n_ent > 0 && (int)((ent_lvl >> (4 * (n_ent - 1))) & 15u) == lvl) {
-            merge_entry(n_ent - 1);
-            n_ent--;
-            lvl++;
-        }
-        if (i + 1 < my_chunks) {
-            write_entry(n_ent);
-            ent_lvl = (ent_lvl & ~(15u << (4 * n_ent))) | ((uint32_t)lvl << (4 * n_ent));
-            n_ent++;
-        }
-    }
-    // a run cut short by the end of the sequence: fold what is left, right to left
-    for (int e = n_ent - 1; e >= 0; e--) merge_entry(e);
-
-    // ---- tree over the W warp results, in registers: at level s the left warp of
-    // each pair merges its right sibling's entry; a warp that is a right sibling at
-    // the next level then publishes what it holds to its entry 0 (it may have merged
-    // at lower levels even when its sibling at this level is empty) ----
-    bool have = my_chunks > 0;
-    if (have) write_entry(0);
-    if (lane == 0) flags[warp] = have ? 0 : 1;
-    __syncthreads();
-    for (int s = 1; s < W; s <<= 1) {
-        if ((warp & (2 * s - 1)) == 0) {
-            if (warp + s < W && flags[warp + s] == 0) {
-                const float* rent = part + (size_t)(warp + s) * SD * C::PART;
-                if (have) {
-                    merge_right(rent);
-                } else {
-                    load_entry(rent);
-                    have = true;
+            // ---- chunk row maxima over the 128 tokens; lazy running max ----
+            float* xb = xch + (i & 1) * ROWS * 4;
+#pragma unroll
+            for (int r = 0; r < ROWS; r++) {
+                const float m = warp_redux_max(z[r]);
+                if (lane == 0) xb[r * 4 + sw] = m;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xfull_b + 8 * (i & 1));
+            if (!wait_warp(xfull_b + 8 * (i & 1), (uint32_t)(i >> 1) & 1u)) {
+                ok = false;
+                break;
+            }
+            bool need = false;
+            float cm = -INFINITY;
+            if (lane < ROWS) {
+                const float4 v = *reinterpret_cast<const float4*>(xb + lane * 4);
+                cm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+                need = cm > __fadd_rn(Mlane, kLazy);
+            }
+            if (__any_sync(FULL, need)) {
+                const float Mn = need ? cm : Mlane;
+                const float al = (Mn == Mlane) ? 1.0f : ex2(__fsub_rn(Mlane, Mn));
+                Mlane = Mn;
+                float alpha[ROWS];
+#pragma unroll
+                for (int r = 0; r < ROWS; r++) {
+                    M[r] = __shfl_sync(FULL, Mn, r);
+                    alpha[r] = __shfl_sync(FULL, al, r);
+                }
+                if (i > 0) {
+                    // rescale O and the sums (this warp's 32 lanes) once the previous
+                    // chunk's value MMAs are complete
+                    if (!wait_warp(pvdone_b + 8 * ((i - 1) & 1), (uint32_t)((i - 1) >> 1) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int cb = 0; cb < (T::H * T::NO + T::NB) / 8; cb++) {
+                        const int col = cb < T::H * T::NO / 8 ? T::T_O + 8 * cb : T::T_SUM + 8 * cb - T::H * T::NO;
+                        const int r0 = (8 * cb) % ROWS;   // NO and ROWS are multiples of 8
+                        uint32_t v[8];
+                        tmem_ld8(tmem_at(tmem, 32 * q, col), v);
+                        tmem_wait_ld();
+                        float a8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; e++) a8[e] = alpha[0];
+#pragma unroll
+                        for (int r = 0; r < ROWS; r++)
+#pragma unroll
+                            for (int e = 0; e < 8; e++)
+                                if (r == (r0 + e) % ROWS) a8[e] = alpha[r];
+#pragma unroll
+                        for (int e = 0; e < 8; e++) v[e] = __float_as_uint(__fmul_rn(__uint_as_float(v[e]), a8[e]));
+                        tmem_st8(tmem_at(tmem, 32 * q, col), v);
+                    }
+                    tmem_wait_st();
                 }
             }
-            if ((warp & (4 * s - 1)) == 2 * s && have) {
-                write_entry(0);
-                if (lane == 0) flags[warp] = 0;
+            // ---- weights: p = 2^(z - M), W_g = p * s_v[g] (fp16) ----
+            float pw[ROWS];
+#pragma unroll
+            for (int r = 0; r < ROWS; r++) pw[r] = (z[r] == -INFINITY) ? 0.0f : ex2(__fsub_rn(z[r], M[r]));
+            if (i >= 2 && !wait_warp(pvdone_b + 8 * wb, (uint32_t)((i - 2) >> 1) & 1u)) {
+                ok = false;
+                break;
+            }
+            const uint32_t wrow = wb0 + (uint32_t)(wb * T::WBYTES + (t / 8) * T::LBO_W + (t % 8) * 16);
+#pragma unroll
+            for (int g = 0; g < T::G; g++) {
+#pragma unroll
+                for (int rg = 0; rg < ROWS / 8; rg++) {
+                    uint32_t hw[4];
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; e2++) {
+                        const int r = 8 * rg + 2 * e2;
+                        float w0 = __fmul_rn(pw[r], sv[g]), w1 = __fmul_rn(pw[r + 1], sv[g]);
+                        if (!clean) {   // masked tokens may carry unwritten (non-finite) scales
+                            w0 = pw[r] == 0.0f ? 0.0f : w0;
+                            w1 = pw[r + 1] == 0.0f ? 0.0f : w1;
+                        }
+                        hw[e2] = pack_h2(w0, w1);
+                    }
+                    stsa128(wrow + (uint32_t)(((g * ROWS + 8 * rg) / 8) * 128), hw[0], hw[1], hw[2], hw[3]);
+                }
+            }
+#pragma unroll
+            for (int rg = 0; rg < ROWS / 8; rg++)
+                stsa128(wrow + (uint32_t)(((T::G * ROWS + 8 * rg) / 8) * 128), pack_h2(pw[8 * rg], pw[8 * rg + 1]),
+                        pack_h2(pw[8 * rg + 2], pw[8 * rg + 3]), pack_h2(pw[8 * rg + 4], pw[8 * rg + 5]),
+                        pack_h2(pw[8 * rg + 6], pw[8 * rg + 7]));
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(wfull_b + 8 * wb);
+        }
+        // ================= epilogue: the CTA partial in natural layout =================
+        if (ok) ok = wait_warp(pvdone_b + 8 * ((n_ck - 1) & 1), (uint32_t)((n_ck - 1) >> 1) & 1u);
+        if (ok) {
+            tc_fence_after();
+            float lr[ROWS];
+#pragma unroll
+            for (int rg = 0; rg < ROWS / 8; rg++) {
+                uint32_t v[8];
+                tmem_ld8(tmem_at(tmem, 32 * q, T::T_SUM + T::G * ROWS + 8 * rg), v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 8; e++) lr[8 * rg + e] = __uint_as_float(v[e]);
+            }
+#pragma unroll
+            for (int h = 0; h < T::H; h++) {
+                const int ch = 128 * h + 32 * q + lane, g = 4 * h + q;
+#pragma unroll
+                for (int rg = 0; rg < ROWS / 8; rg++) {
+                    uint32_t o[8], sg[8];
+                    tmem_ld8(tmem_at(tmem, 32 * q, T::T_O + h * T::NO + q * ROWS + 8 * rg), o);
+                    tmem_ld8(tmem_at(tmem, 32 * q, T::T_SUM + g * ROWS + 8 * rg), sg);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 8; e++)
+                        part[(8 * rg + e) * D + ch] =
+                            __fmaf_rn(__uint_as_float(o[e]), 16777216.0f, -8.0f * __uint_as_float(sg[e]));
+                }
+            }
+            if (sw == 0 && lane == 0) {
+#pragma unroll
+                for (int r = 0; r < ROWS; r++) {
+                    part[ROWS * D + r] = M[r];
+                    part[ROWS * D + ROWS + r] = lr[r];
+                }
             }
         }
-        __syncthreads();
+        tc_fence_before();
     }
-    // any warp that gave up on a wait: drain its copies still in flight, then stop
-    if (aborted) {
-        for (int k = k_abort; k < my_pages && k < k_abort + R; k++)
-            mbar_wait_bounded(smem_u32(&bars[k % R]), (uint32_t)((k / R) & 1));
-        misc[1] = 1;
-    }
+
     __syncthreads();
-    if (misc[1] == 1) return;
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+    if (*abort_flag != 0) return;
 
     const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
     // out = O / l and lse for the real rows of this block; (o_src, m_src, l_src) in the
@@ -718,9 +684,6 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
                 p.lse[orow] = __fmul_rn(__fadd_rn(m_src[rl], log2f(l)), 0.69314718055994531f);
         }
     };
-
-    if (warp == 0) write_entry(0);   // the CTA's result, natural layout
-    __syncthreads();
     if (n_splits == 1) {
         finalize(part, part + ROWS * D, part + ROWS * D + ROWS);
         return;
@@ -836,9 +799,10 @@ __global__ void __launch_bounds__(256, (D == 128 && ROWS == 8) ? 2 : 1) decode_k
     if (threadIdx.x == 0) p.counters[pidx] = 0u;
 }
 
-size_t decode_smem_bytes(int head_dim, int rows, int warps, int pages_per_stage, int stack_depth) {
+
+size_t decode_smem_bytes(int head_dim, int rows, int stages) {
 #define MQ_SMEM(DD, RR) \
-    if (head_dim == DD && rows == RR) return smem_layout<DD, RR>(warps, pages_per_stage, stack_depth).total;
+    if (head_dim == DD && rows == RR) return smem_layout<DD, RR>(stages).total;
     MQ_SMEM(128, 8) MQ_SMEM(128, 16) MQ_SMEM(128, 32) MQ_SMEM(256, 8) MQ_SMEM(256, 16)
 #undef MQ_SMEM
     return 0;
@@ -858,10 +822,10 @@ cudaError_t decode_prepare(int head_dim, int rows, size_t smem) {
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int warps, int max_splits, size_t smem,
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int max_splits, size_t smem,
                           cudaStream_t st) {
     const dim3 grid((unsigned)max_splits, (unsigned)(p.n_kv_heads * p.n_rb), (unsigned)p.n_seqs);
-    const dim3 block((unsigned)(warps * 32));
+    const dim3 block((unsigned)kThreads);
 #define MQ_LAUNCH(DD, RR) \
     if (head_dim == DD && rows == RR) decode_kernel<DD, RR><<<grid, block, smem, st>>>(p); else
     MQ_LAUNCH(128, 8) MQ_LAUNCH(128, 16) MQ_LAUNCH(128, 32) MQ_LAUNCH(256, 8) MQ_LAUNCH(256, 16)

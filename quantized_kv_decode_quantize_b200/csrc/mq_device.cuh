@@ -1,20 +1,19 @@
 // Device-side helpers shared by the mq kernels: page layout, PTX wrappers for
-// mbarriers, bulk TMA copies and legacy warp-level MMA, and the error word.
+// mbarriers, bulk TMA copies, and the error word.
 //
-// Page layout (one (block, kv-head) page of 16 tokens, head_dim D):
-//   [0, 16D)            K codes, int8, permuted for the QK fragments:
-//                       16-byte chunk c of lane L = 4g + t sits at (c*32 + L)*16 and
-//                       holds channels t*D/4 + 16*(c % (D/64)) .. +15 of token
-//                       g + 8*(c / (D/64)).
-//   [16D, 16D+32)       K scales, fp16, token order.
-//   [16D+32, 24D+32)    V codes, int4 pairs, permuted for the PV fragments:
-//                       32-bit word w = 2*q + tp of lane L = 4g + t sits at
-//                       ((w/4)*32 + L)*16 + (w%4)*4; its bytes are
-//                       [tok A: ch c, c+1][tok A: ch c+2, c+3][tok B: ch c, c+1][tok B: ch c+2, c+3]
-//                       with c = 32q + 4g, tok A = 8*tp + 2t, tok B = tok A + 1,
-//                       and the even channel of a pair in the low nibble.
-//   [24D+32, 25D+32)    V scales, fp16: half index ((t*NG + q)*2 + hi)*2 + par for
-//                       token 8*hi + 2t + par and group q (NG = D/32 groups).
+// Page layout (one (block, kv-head) page of 16 tokens, head_dim D): two token-group
+// records, tokens 0-7 then 8-15, of rec_bytes(D) = 12.5 D + 16 bytes each.  Within a
+// record (token tt = 0..7 of the group):
+//   [0, 8D)               K codes, int8, as 8-row x 16-byte blocks: code (tt, c) at
+//                         byte (c / 16) * 128 + tt * 16 + c % 16.  Consecutive records
+//                         of consecutive pages are then one K-major tensor-core operand
+//                         (tokens x channels) whose 8-token groups sit rec_bytes apart.
+//   [8D, 12D)             V codes, int4 two's complement, channel-major: one 32-bit
+//                         word per channel c at 8D + 4c holding the channel's 8 codes,
+//                         token tt at bit 4 * (tt / 2) + 16 * (tt % 2), so that a mask
+//                         and a shift give two consecutive tokens as the two halves.
+//   [12D, 12D + 16)       K scales, fp16, token order.
+//   [12D + 16, 12.5D + 16) V scales, fp16: (tt, group g) at 12D + 16 + 2 * (tt * D/32 + g).
 #pragma once
 #include <cstdint>
 #include <cuda_fp16.h>
@@ -28,30 +27,26 @@ constexpr int kChunkTokens = kPageTokens * kChunkPages;
 constexpr int kMaxSplits = 64;                  // CTA partials per (sequence, kv-head, row block)
 
 __host__ __device__ constexpr int page_bytes(int D) { return 25 * D + 32; }
-__host__ __device__ constexpr int k_scale_off(int D) { return 16 * D; }
-__host__ __device__ constexpr int v_code_off(int D) { return 16 * D + 32; }
-__host__ __device__ constexpr int v_scale_off(int D) { return 24 * D + 32; }
+__host__ __device__ constexpr int rec_bytes(int D) { return 25 * D / 2 + 16; }
+__host__ __device__ constexpr int rec_v_off(int D) { return 8 * D; }
+__host__ __device__ constexpr int rec_ks_off(int D) { return 12 * D; }
+__host__ __device__ constexpr int rec_vs_off(int D) { return 12 * D + 16; }
 
-// byte offset of K code (token tau, channel c) inside a page
-__host__ __device__ inline int k_code_byte(int D, int tau, int c) {
-    const int t = c / (D / 4), o = c % (D / 4);
-    const int chunk = (tau / 8) * (D / 64) + o / 16;
-    const int lane = 4 * (tau % 8) + t;
-    return (chunk * 32 + lane) * 16 + (o % 16);
+// byte offset inside a page of K code (token tau, channel c)
+__host__ __device__ constexpr int k_code_byte(int D, int tau, int c) {
+    return (tau / 8) * rec_bytes(D) + (c / 16) * 128 + (tau % 8) * 16 + c % 16;
 }
-
-// byte offset (inside a page) of the byte holding V channels (c, c+1) of token
-// tau, for c = 32q + 4g' + 2h (h = 0 or 1)
-__host__ __device__ inline int v_code_byte(int D, int tau, int c) {
-    const int q = c / 32, cg = c % 32, gp = cg / 4, h = (cg % 4) / 2;
-    const int t = (tau % 8) / 2, par = tau % 2, tp = tau / 8;
-    const int lane = 4 * gp + t, w = 2 * q + tp;
-    return v_code_off(D) + ((w / 4) * 32 + lane) * 16 + (w % 4) * 4 + par * 2 + h;
+// byte offset inside a page of the 32-bit V word of channel c for tokens of tau's group,
+// and the bit position of tau's code in it
+__host__ __device__ constexpr int v_word_byte(int D, int tau, int c) {
+    return (tau / 8) * rec_bytes(D) + rec_v_off(D) + 4 * c;
 }
-
-__host__ __device__ inline int v_scale_byte(int D, int tau, int q) {
-    const int NG = D / 32, t = (tau % 8) / 2, hi = tau / 8, par = tau % 2;
-    return v_scale_off(D) + 2 * (((t * NG + q) * 2 + hi) * 2 + par);
+__host__ __device__ constexpr int v_nibble_bit(int tau) { return 4 * ((tau % 8) / 2) + 16 * (tau % 2); }
+__host__ __device__ constexpr int k_scale_byte(int D, int tau) {
+    return (tau / 8) * rec_bytes(D) + rec_ks_off(D) + 2 * (tau % 8);
+}
+__host__ __device__ constexpr int v_scale_byte(int D, int tau, int g) {
+    return (tau / 8) * rec_bytes(D) + rec_vs_off(D) + 2 * ((tau % 8) * (D / 32) + g);
 }
 
 // ---- device error word (one per device) -----------------------------------
@@ -165,38 +160,6 @@ __device__ __forceinline__ uint32_t lds32(const void* p) {
     return v;
 }
 
-// D = A(16x32, s8) * B(32x8, s8) + C, int32 accumulate
-__device__ __forceinline__ void mma_s8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm(
-        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// D = A(16x32, u8) * B(32x8, s8) + C, int32 accumulate
-__device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm(
-        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// D = A(16x16, f16) * B(16x8, f16) + D, fp32 accumulate
-__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                        uint32_t b0, uint32_t b1) {
-    asm(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// (x & mask) | magic in one LOP3
-__device__ __forceinline__ uint32_t lop_and_or(uint32_t x, uint32_t mask, uint32_t magic) {
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(x), "r"(mask), "r"(magic));
-    return d;
-}
-
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
@@ -205,20 +168,6 @@ __device__ __forceinline__ uint32_t lop_and_xor(uint32_t x, uint32_t mask, uint3
     uint32_t d;
     asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(x), "r"(mask), "r"(flip));
     return d;
-}
-
-// Two two's-complement 4-bit codes at bit positions (0..3, 16..19) of x -> fp16x2
-// holding the exact integer codes.  One LOP3 forms 1024 + (n ^ 8) = 1032 + code in
-// each half (0x6400 is 1024; flipping bit 3 turns the two's-complement nibble into
-// code + 8), one HSUB2 removes the 1032.
-__device__ __forceinline__ uint32_t nib_lo_to_h2(uint32_t x) {
-    const uint32_t m = lop_and_xor(x, 0x000F000Fu, 0x64086408u);
-    return h2_as_u32(__hsub2(u32_as_h2(m), u32_as_h2(0x64086408u)));   // - 1032
-}
-// Same for bit positions (4..7, 20..23): 1024 + 16 (code + 8), then /16 - 72.
-__device__ __forceinline__ uint32_t nib_hi_to_h2(uint32_t x) {
-    const uint32_t m = lop_and_xor(x, 0x00F000F0u, 0x64806480u);
-    return h2_as_u32(__hfma2(u32_as_h2(m), u32_as_h2(0x2C002C00u), u32_as_h2(0xD480D480u)));
 }
 
 // 2^x with the SFU instruction (ex2.approx.ftz.f32: relative error ~2^-22, subnormal

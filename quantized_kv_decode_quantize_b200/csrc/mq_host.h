@@ -22,7 +22,7 @@ struct mq_cache {
 namespace mq {
 
 struct DecodePlan {
-    int cls, rows, n_rb, warps, pages_per_stage, cpc, max_splits, stack_depth;
+    int cls, rows, n_rb, stages, cpc, max_splits;
     size_t smem;
 };
 

@@ -47,16 +47,15 @@ struct DecodeParams {
     float* part_o;       // [n_seqs][n_kv_heads][n_rb][split_stride][rows][D]
     int split_stride;    // partial slots per unit (>= the splits of any unit)
     int n_rb;            // row blocks per kv-head
-    int cpc;             // chunks per CTA (power of two >= warps)
-    int pages_per_stage; // TMA ring depth per warp
-    int stack_depth;     // partial entries per warp in shared memory
+    int cpc;             // chunks per CTA
+    int stages;          // TMA ring depth in chunks
     unsigned* err;
 };
 
 // rows: 8, 16 or 32 (padded query rows per kv-head handled by one CTA)
-size_t decode_smem_bytes(int head_dim, int rows, int warps, int pages_per_stage, int stack_depth);
+size_t decode_smem_bytes(int head_dim, int rows, int stages);   // 0: does not fit the layout
 cudaError_t decode_prepare(int head_dim, int rows, size_t smem);  // raises the dynamic smem limit
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int warps, int max_splits, size_t smem,
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int max_splits, size_t smem,
                           cudaStream_t st);
 
 // Fills n values of dtype with a deterministic pseudo-random pattern (uniform in

@@ -221,25 +221,21 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         return MQ_TUNE_BUDGET_EXHAUSTED;
     }
 
-    // ---- candidates: structure (warps, ctas_per_sm) first, then ring depth ----
+    // ---- candidates: structure (splits per SM) first, then ring depth ----
     std::vector<Cand> cands;
     bool class_used[3] = {false, false, false};
     for (auto& pr : probes) class_used[pr.cls] = true;
-    const int Rs[3] = {2, 3, 4};
-    for (int ri = 0; ri < 3; ri++)
-        for (int w : {8, 4})
-            for (int cps : {1, 2, 4})
-                for (int cls = 0; cls < 3; cls++) {
-                    if (!class_used[cls]) continue;
-                    Cand cd;
-                    cd.cfg = mq_decode_config{w, Rs[ri], cps};
-                    cd.cls = cls;
-                    const mq_decode_config& d = cache->cfg[cls];
-                    if (cd.cfg.warps_per_cta == d.warps_per_cta && cd.cfg.pages_per_stage == d.pages_per_stage &&
-                        cd.cfg.ctas_per_sm == d.ctas_per_sm)
-                        continue;
-                    cands.push_back(cd);
-                }
+    for (int r : {4, 3, 2})
+        for (int sps : {1, 2, 4})
+            for (int cls = 0; cls < 3; cls++) {
+                if (!class_used[cls]) continue;
+                Cand cd;
+                cd.cfg = mq_decode_config{r, sps};
+                cd.cls = cls;
+                const mq_decode_config& d = cache->cfg[cls];
+                if (cd.cfg.ring_stages == d.ring_stages && cd.cfg.splits_per_sm == d.splits_per_sm) continue;
+                cands.push_back(cd);
+            }
     bool exhausted = false;
     for (auto& cd : cands) {
         double est = 0;
@@ -334,18 +330,17 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
             for (size_t i = 0; i < cands.size(); i++) {
                 const Cand& cd = cands[i];
                 std::fprintf(f,
-                             "    {\"rows_class\": %d, \"warps_per_cta\": %d, \"pages_per_stage\": %d, \"ctas_per_sm\": %d, "
+                             "    {\"rows_class\": %d, \"ring_stages\": %d, \"splits_per_sm\": %d, "
                              "\"measured\": %s, \"valid\": %s, \"bit_identical\": %s, \"times_us\": [%.3f, %.3f, %.3f]}%s\n",
-                             cd.cls, cd.cfg.warps_per_cta, cd.cfg.pages_per_stage, cd.cfg.ctas_per_sm,
+                             cd.cls, cd.cfg.ring_stages, cd.cfg.splits_per_sm,
                              cd.measured ? "true" : "false", cd.valid ? "true" : "false",
                              cd.identical ? "true" : "false", cd.t[0] * 1e6, cd.t[1] * 1e6, cd.t[2] * 1e6,
                              i + 1 < cands.size() ? "," : "");
             }
             std::fprintf(f, "  ],\n  \"chosen\": [");
             for (int cls = 0; cls < 3; cls++)
-                std::fprintf(f, "%s{\"rows_class\": %d, \"warps_per_cta\": %d, \"pages_per_stage\": %d, \"ctas_per_sm\": %d}",
-                             cls ? ", " : "", cls, res->chosen[cls].warps_per_cta, res->chosen[cls].pages_per_stage,
-                             res->chosen[cls].ctas_per_sm);
+                std::fprintf(f, "%s{\"rows_class\": %d, \"ring_stages\": %d, \"splits_per_sm\": %d}",
+                             cls ? ", " : "", cls, res->chosen[cls].ring_stages, res->chosen[cls].splits_per_sm);
             std::fprintf(f, "],\n  \"cost\": %.4f, \"n_tried\": %d, \"n_rejected\": %d, \"n_skipped\": %d\n}\n", res->cost,
                          res->n_tried, res->n_rejected, res->n_skipped);
             std::fclose(f);

@@ -1,8 +1,11 @@
 """Reads the library's page format back into logical (token, channel) order.
 
-An independent restatement, in numpy, of the byte permutation documented in
-include/mq.h ("Cache layout"); the tests use it to compare the codes and scales the
-CUDA append kernel wrote with the CPU oracle's.  Lane L = 4g + t (g = 0..7, t = 0..3).
+An independent restatement, in numpy, of the page layout documented in include/mq.h
+("Cache layout"); the tests use it to compare the codes and scales the CUDA append
+kernel wrote with the CPU oracle's.  A page holds two records of 8 tokens each
+(tokens 0-7, then 8-15), each record rec_bytes(D) = 12.5 D + 16 bytes:
+K codes as 8 x 16-byte blocks, then one 32-bit V word per channel with the 8 tokens'
+nibbles, then the 8 K scales, then the 8 x D/32 V scales.
 """
 from __future__ import annotations
 
@@ -13,40 +16,42 @@ def page_bytes(D: int) -> int:
     return 25 * D + 32
 
 
+def rec_bytes(D: int) -> int:
+    return 25 * D // 2 + 16
+
+
 def _k_index(D):
+    R = rec_bytes(D)
     idx = np.zeros((16, D), np.int64)
     for tau in range(16):
         for c in range(D):
-            t, o = c // (D // 4), c % (D // 4)
-            chunk = (tau // 8) * (D // 64) + o // 16
-            lane = 4 * (tau % 8) + t
-            idx[tau, c] = (chunk * 32 + lane) * 16 + o % 16
+            idx[tau, c] = (tau // 8) * R + (c // 16) * 128 + (tau % 8) * 16 + c % 16
     return idx
 
 
 def _v_index(D):
-    """byte holding channels (2j, 2j+1) of token tau, for j = 0 .. D/2 - 1"""
-    idx = np.zeros((16, D // 2), np.int64)
-    base = 16 * D + 32
+    """(byte offset of the 32-bit word, bit position of the nibble) of V code (tau, c)"""
+    R = rec_bytes(D)
+    word = np.zeros((16, D), np.int64)
+    bit = np.zeros((16, D), np.int64)
     for tau in range(16):
-        t, par, tp = (tau % 8) // 2, tau % 2, tau // 8
-        for j in range(D // 2):
-            c = 2 * j
-            q, cg = c // 32, c % 32
-            gp, h = cg // 4, (cg % 4) // 2
-            lane = 4 * gp + t
-            w = 2 * q + tp
-            idx[tau, j] = base + ((w // 4) * 32 + lane) * 16 + (w % 4) * 4 + par * 2 + h
-    return idx
+        for c in range(D):
+            word[tau, c] = (tau // 8) * R + 8 * D + 4 * c
+            bit[tau, c] = 4 * ((tau % 8) // 2) + 16 * (tau % 2)
+    return word, bit
+
+
+def _ks_index(D):
+    R = rec_bytes(D)
+    return np.array([(tau // 8) * R + 12 * D + 2 * (tau % 8) for tau in range(16)], np.int64)
 
 
 def _vs_index(D):
-    NG = D // 32
-    idx = np.zeros((16, NG), np.int64)
+    R, G = rec_bytes(D), D // 32
+    idx = np.zeros((16, G), np.int64)
     for tau in range(16):
-        t, hi, par = (tau % 8) // 2, tau // 8, tau % 2
-        for q in range(NG):
-            idx[tau, q] = ((t * NG + q) * 2 + hi) * 2 + par
+        for g in range(G):
+            idx[tau, g] = (tau // 8) * R + 12 * D + 16 + 2 * ((tau % 8) * G + g)
     return idx
 
 
@@ -55,27 +60,42 @@ _CACHE = {}
 
 def _maps(D):
     if D not in _CACHE:
-        _CACHE[D] = (_k_index(D), _v_index(D), _vs_index(D))
+        _CACHE[D] = (_k_index(D), _v_index(D), _ks_index(D), _vs_index(D))
     return _CACHE[D]
 
 
 def check_maps_are_permutations(D):
-    k, v, vs = _maps(D)
-    assert sorted(k.ravel().tolist()) == list(range(16 * D))
-    assert sorted(v.ravel().tolist()) == list(range(16 * D + 32, 24 * D + 32))
-    assert sorted(vs.ravel().tolist()) == list(range(16 * D // 32))
+    """Every byte of a page belongs to exactly one field, every V bit to one code."""
+    k, (vw, vb), ks, vs = _maps(D)
+    owner = np.zeros(page_bytes(D), np.int64)
+    np.add.at(owner, k.ravel(), 1)
+    for off in (0, 1):
+        np.add.at(owner, ks + off, 1)
+        np.add.at(owner, vs.ravel() + off, 1)
+    words = np.unique(vw)
+    for off in range(4):
+        np.add.at(owner, words + off, 1)
+    assert np.all(owner == 1)
+    # each V word holds 8 distinct nibbles
+    bits = {}
+    for w, b in zip(vw.ravel().tolist(), vb.ravel().tolist()):
+        bits.setdefault(w, set()).add(b)
+    assert all(sorted(s) == list(range(0, 32, 4)) for s in bits.values())
 
 
 def decode_pages(pages: np.ndarray, D: int):
     """pages uint8 [n, page_bytes(D)] -> kc int8 [n,16,D], ks u16 [n,16],
-    vp u8 [n,16,D/2] (natural packing), vs u16 [n,16,D/32]."""
+    vp u8 [n,16,D/2] (natural packing: even channel in the low nibble), vs u16 [n,16,D/32]."""
     pages = np.ascontiguousarray(pages)
-    k, v, vs = _maps(D)
+    k, (vw, vb), ks, vs = _maps(D)
     kc = pages[:, k].view(np.int8)
-    ks = np.ascontiguousarray(pages[:, 16 * D: 16 * D + 32]).view(np.uint16)
-    vp = pages[:, v]
-    vsr = np.ascontiguousarray(pages[:, 24 * D + 32: 25 * D + 32]).view(np.uint16)
-    return kc, ks, vp, vsr[:, vs]
+    word = (pages[:, vw].astype(np.uint32) | (pages[:, vw + 1].astype(np.uint32) << 8)
+            | (pages[:, vw + 2].astype(np.uint32) << 16) | (pages[:, vw + 3].astype(np.uint32) << 24))
+    nib = ((word >> vb.astype(np.uint32)) & 0xF).astype(np.uint8)            # [n, 16, D]
+    vp = (nib[:, :, 0::2] | (nib[:, :, 1::2] << 4)).astype(np.uint8)
+    ksv = (pages[:, ks].astype(np.uint16) | (pages[:, ks + 1].astype(np.uint16) << 8))
+    vsv = (pages[:, vs].astype(np.uint16) | (pages[:, vs + 1].astype(np.uint16) << 8))
+    return kc, ksv, vp, vsv
 
 
 def gather_sequence(pool: np.ndarray, n_kv_heads: int, D: int, table: np.ndarray, L: int):

