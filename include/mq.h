@@ -255,8 +255,8 @@ mq_status mq_decode_attn_static(const mq_cache* cache, const void* q, mq_dtype q
  * contiguous range of chunks of one (sequence, kv-head, row block), accumulates
  * them in token order, and the CTA partials are combined by one fixed binary
  * tree over the split index.
- *   ring_stages    2 .. 4: chunks (8 pages each) a CTA keeps in flight; never
- *                  changes the output
+ *   ring_stages    2 .. 8: chunks (8 pages each) a CTA keeps in flight, cut
+ *                  to what fits in shared memory; never changes the output
  *   splits_per_sm  1, 2 or 4: the split count along the sequence is chosen so
  *                  that about splits_per_sm x (number of SMs) CTAs run; it sets
  *                  the chunk ranges and so may change the rounding of the output

@@ -36,13 +36,13 @@ mq_decode_config default_config(int head_dim, int cls) {
     (void)head_dim;
     (void)cls;
     mq_decode_config c{};
-    c.ring_stages = 4;
+    c.ring_stages = 8;   // the planner shortens it to what fits in shared memory
     c.splits_per_sm = 1;
     return c;
 }
 
 bool config_valid(const mq_decode_config& c) {
-    return c.ring_stages >= 2 && c.ring_stages <= 4 &&
+    return c.ring_stages >= 2 && c.ring_stages <= 8 &&
            (c.splits_per_sm == 1 || c.splits_per_sm == 2 || c.splits_per_sm == 4);
 }
 
@@ -67,15 +67,19 @@ static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int row
     const mq_decode_config cfg = c->cfg[pl.cls];
     const long long max_chunks = std::max<long long>(1, (max_seq_len + kChunkTokens - 1) / kChunkTokens);
     const long long units = (long long)n_seqs * c->n_kv_heads * pl.n_rb;
-    long long splits = (long long)cfg.splits_per_sm * c->n_sm / units;
+    const int cps = decode_ctas_per_sm(c->head_dim, pl.rows);
+    long long splits = (long long)cfg.splits_per_sm * cps * c->n_sm / units;
     splits = std::max<long long>(1, std::min<long long>({splits, max_chunks, (long long)kMaxSplits}));
     const long long cpc = (max_chunks + splits - 1) / splits;
     pl.cpc = (int)cpc;
     pl.max_splits = (int)((max_chunks + cpc - 1) / cpc);
-    // the ring is shortened (never below 2 stages) until the CTA fits in shared memory
+    // the ring is shortened (never below 2 stages) until the CTA fits in its share of
+    // the SM's shared memory (1 KB of each CTA's share is reserved by the hardware)
+    const size_t smem_cap = cps == 1 ? (size_t)c->max_smem
+                                     : std::min((size_t)c->max_smem, (size_t)c->smem_per_sm / cps - 1024);
     pl.stages = cfg.ring_stages;
     pl.smem = decode_smem_bytes(c->head_dim, pl.rows, pl.stages);
-    while ((pl.smem == 0 || pl.smem > (size_t)c->max_smem) && pl.stages > 2) {
+    while ((pl.smem == 0 || pl.smem > smem_cap) && pl.stages > 2) {
         pl.stages--;
         pl.smem = decode_smem_bytes(c->head_dim, pl.rows, pl.stages);
     }
@@ -194,9 +198,11 @@ mq_status mq_cache_create(const mq_cache_desc* d, mq_cache** out) {
     if (d->pool_bytes < mq_cache_pool_bytes(d->n_kv_heads, d->head_dim, d->n_blocks)) return MQ_ERR_CAPACITY;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MQ_ERR_CUDA;
-    int n_sm = 0, max_smem = 0;
+    int n_sm = 0, max_smem = 0, smem_per_sm = 0;
     if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MQ_ERR_CUDA;
     if (cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return MQ_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess)
         return MQ_ERR_CUDA;
     unsigned* err = nullptr;
     if (error_word_address(&err) != cudaSuccess) return MQ_ERR_CUDA;
@@ -210,6 +216,7 @@ mq_status mq_cache_create(const mq_cache_desc* d, mq_cache** out) {
     c->device = dev;
     c->n_sm = n_sm;
     c->max_smem = max_smem;
+    c->smem_per_sm = smem_per_sm;
     c->err_word = err;
     for (int k = 0; k < 3; k++) c->cfg[k] = default_config(d->head_dim, k);
     *out = c;
@@ -264,7 +271,7 @@ size_t mq_decode_workspace_bytes(const mq_cache* c, int32_t n_seqs, int32_t n_q_
     // over every valid configuration, so the answer depends on the shape alone.
     mq_cache probe = *c;
     size_t part = 0;
-    for (int r = 2; r <= 4; r++)
+    for (int r = 2; r <= 8; r++)
         for (int t = 1; t <= 4; t *= 2) {
             for (int k = 0; k < 3; k++) probe.cfg[k] = mq_decode_config{r, t};
             const DecodePlan pl = plan_for_class(&probe, rows_class_for(c->head_dim, rows_total), n_seqs, rows_total,

@@ -9,12 +9,12 @@
 //     z_t = scale * <q, s_k[t] * kcode_t>,  t = 0 .. L_b - n_b + j
 //     out = sum_t softmax(z)_t * (s_v[t, group] * vcode_t),  lse = log sum_t exp z_t
 //
-// How.  One CTA (10 warps, one per SM) takes a contiguous range of 128-token chunks of
+// How.  One CTA (11 warps, one per SM) takes a contiguous range of 128-token chunks of
 // one (sequence, kv-head, row block) and runs a warp-specialised pipeline per chunk:
 //  * warp 0 streams the chunk's 8 pages into a shared-memory ring with one 1-D bulk
 //    TMA copy per page (block-table lookup, L2 evict-first).  The page format makes
 //    the int8 key codes of a chunk one K-major tensor-core operand as they land.
-//  * warp 1 issues the MMAs from one thread.  Scores: S = K q^T with kind::i8, M = 128
+//  * warps 1 and 2 issue the MMAs, one thread each (scores, values).  Scores: S = K q^T with kind::i8, M = 128
 //    tokens, the query rows as the N side, q held as a 23-bit fixed-point value per row
 //    (q = Q * 2^(E-22)) split into three signed 8-bit limbs stacked along N, so the
 //    int32 products are exact; S lands in tensor memory.  Values: O += V^T W with
@@ -23,10 +23,10 @@
 //    along N; each channel keeps only its own group's columns.  A second MMA with a
 //    constant all-ones A gives, in every lane, the column sums of W: the per-group
 //    sums that undo the value-code offset, and l = sum_t p from the p columns.
-//  * warps 2-5 turn the int4 value codes into tensor memory as exact fp16 values
+//  * warps 3-6 turn the int4 value codes into tensor memory as exact fp16 values
 //    u * 2^-24 (u = code + 8 in 0..15, a subnormal) with one mask, shift and flip per
 //    two tokens, a channel per TMEM lane; out = 2^24 * O - 8 * sum_t W_g.
-//  * warps 6-9 (one TMEM lane per token) read S, form z in fp32, take the chunk's row
+//  * warps 7-10 (one TMEM lane per token) read S, form z in fp32, take the chunk's row
 //    maxima (redux + a named barrier), keep a lazy running max M per row (moved only
 //    when a chunk max exceeds it by more than kLazy, after rescaling O and the sums in
 //    tensor memory), and write p = 2^(z - M) and the weights W_g (fp16) to shared memory.
@@ -45,8 +45,7 @@ namespace mq {
 
 // lazy-max threshold of the online softmax, in log2 units (weights stay <= 2^4)
 constexpr float kLazy = 4.0f;
-constexpr int kThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2-5 values, warps 6-9 softmax
-constexpr int kTmemCols = 512;
+constexpr int kThreads = 352;   // warp 0 TMA, 1 QK MMA, 2 PV MMA, 3-6 values, 7-10 softmax
 
 template <int D, int ROWS>
 struct Tc {
@@ -57,8 +56,18 @@ struct Tc {
     static constexpr int NQ = (3 * ROWS + 15) / 16 * 16;          // score MMA N: 3 limbs x rows
     static constexpr int NO = 4 * ROWS;                           // value MMA N per half
     static constexpr int NB = ((G + 1) * ROWS + 15) / 16 * 16;    // weight columns: W_0..W_{G-1}, p
-    static constexpr int NSB = (D == 128 && ROWS == 32) ? 1 : 2;  // score buffers in TMEM
-    static constexpr int NVB = (D == 256 && ROWS == 16) ? 1 : 2;  // V^T buffers in TMEM
+    // One CTA per SM owns all of tensor memory.  Every hand-off between the roles is
+    // buffered as deeply as tensor and shared memory allow, so that several chunks are
+    // in flight in each stage and the latency of an MMA (issue to commit) is hidden.
+    // The 8-row D=128 class (grouped-query decode, the common case) runs two CTAs per SM
+    // instead, each with half of tensor memory: two independent pipelines per SM hide
+    // each other's latencies better than deeper buffers in one.
+    static constexpr int CPS = (D == 128 && ROWS == 8) ? 2 : 1;
+    static constexpr int TCOLS = CPS == 2 ? 256 : 512;                           // TMEM columns allocated
+    static constexpr int NSB = CPS == 2 ? 2 : ((D == 128 && ROWS <= 16) ? 4 : (ROWS == 32 ? 1 : 2));   // score buffers (TMEM)
+    static constexpr int NVB = CPS == 2 ? 1 : ((D == 256 && ROWS == 16) ? 1 : 2);  // V^T buffers (TMEM)
+    static constexpr int NWB = CPS == 2 ? 3 : ((ROWS == 32 || (D == 256 && ROWS == 16)) ? 2 : 3);  // weight buffers (smem)
+    static constexpr int NPB = NWB > NVB ? NWB : NVB;                            // value-MMA completion barriers
     // tensor-memory columns
     static constexpr int T_S = 0;
     static constexpr int T_O = NSB * NQ;
@@ -68,7 +77,7 @@ struct Tc {
     static constexpr int WBYTES = kChunkTokens * NB * 2;          // one weight buffer
     static constexpr int LBO_W = NB / 8 * 128;                    // its 8-token group stride
     static constexpr int PART = ROWS * D + 2 * ROWS;              // floats of one partial
-    static_assert(T_END <= kTmemCols, "tensor memory budget");
+    static_assert(T_END <= TCOLS, "tensor memory budget");
     static_assert(NQ <= 256 && NB <= 256 && NO <= 256, "MMA N range");
 };
 
@@ -87,7 +96,7 @@ __host__ __device__ inline Smem smem_layout(int NS) {
     off += (size_t)NS * kChunkPages * T::PB;
     off = al(off, 128);
     s.wbuf = off;
-    off += (size_t)2 * T::WBYTES;
+    off += (size_t)T::NWB * T::WBYTES;
     // the final cross-CTA merge reuses ring + weight buffers (idle by then)
     s.heap = 0;
     s.fin = al((size_t)2 * kMaxSplits * ROWS * 16, 16);
@@ -110,7 +119,7 @@ __host__ __device__ inline Smem smem_layout(int NS) {
     off += (size_t)NS * kChunkPages * 4;
     off = al(off, 8);
     s.mbar = off;
-    off += (size_t)(2 * NS + 12) * 8;
+    off += (size_t)(2 * NS + 2 * T::NSB + T::NWB + T::NVB + T::NPB) * 8;
     s.misc = off;
     off += 64;
     s.total = al(off, 128);
@@ -162,8 +171,37 @@ __device__ __forceinline__ float h_bits_to_f32(uint32_t bits) {
     return __half2float(__ushort_as_half((unsigned short)bits));
 }
 
+template <int ROWS>
+struct AlphaRows {
+    float a[ROWS];
+    __device__ static AlphaRows make(const float (&x)[ROWS]) {
+        AlphaRows r;
+#pragma unroll
+        for (int i = 0; i < ROWS; i++) r.a[i] = x[i];
+        return r;
+    }
+};
+
+// Multiplies this warp's 32 TMEM lanes of the value accumulators (NO columns from t_o)
+// and of the column sums (NS columns from t_sum) by the factor of each column's row
+// (column j holds row j % ROWS).  Out of line: it runs only when a running max moves.
+template <int ROWS, int NO, int NS>
+__device__ __noinline__ void rescale_acc(uint32_t lane_base, int t_o, int t_sum, AlphaRows<ROWS> al) {
+#pragma unroll 1
+    for (int cb = 0; cb < (NO + NS) / 8; cb++) {
+        const int col = cb < NO / 8 ? t_o + 8 * cb : t_sum + 8 * cb - NO;
+        const int r0 = (8 * cb) % ROWS;   // NO, NS and ROWS are multiples of 8
+        uint32_t v[8];
+        tmem_ld8(lane_base + (uint32_t)col, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 8; e++) v[e] = __float_as_uint(__fmul_rn(__uint_as_float(v[e]), al.a[r0 + e]));
+        tmem_st8(lane_base + (uint32_t)col, v);
+    }
+}
+
 template <int D, int ROWS>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(const DecodeParams p) {
     using T = Tc<D, ROWS>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -197,17 +235,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     const uint32_t bar0 = smem_u32(smem + S.mbar);
     auto full_b = [&](int s) { return bar0 + 8u * (uint32_t)s; };
     auto empty_b = [&](int s) { return bar0 + 8u * (uint32_t)(NS + s); };
-    const uint32_t sfull_b = bar0 + 8u * (uint32_t)(2 * NS);   // [2] score buffer written
-    const uint32_t sfree_b = sfull_b + 16;                     // [2] score buffer read
-    const uint32_t wfull_b = sfree_b + 16;                     // [2] weights written
-    const uint32_t vfull_b = wfull_b + 16;                     // [2] V^T written
-    const uint32_t pvdone_b = vfull_b + 16;                    // [2] value MMAs of a chunk done
-    const uint32_t xfull_b = pvdone_b + 16;                    // [2] chunk row maxima exchanged
+    const uint32_t sfull_b = bar0 + 8u * (uint32_t)(2 * NS);   // [NSB] score buffer written
+    const uint32_t sfree_b = sfull_b + 8 * T::NSB;             // [NSB] score buffer read
+    const uint32_t wfull_b = sfree_b + 8 * T::NSB;             // [NWB] weights written
+    const uint32_t vfull_b = wfull_b + 8 * T::NWB;             // [NVB] V^T written
+    const uint32_t pvdone_b = vfull_b + 8 * T::NVB;            // [NPB] value MMAs of a chunk done
+    // completion barrier of chunk j's value MMAs and the parity of that completion
+    auto pv_bar = [&](int j) { return pvdone_b + 8u * (uint32_t)(j % T::NPB); };
+    auto pv_par = [&](int j) { return (uint32_t)(j / T::NPB) & 1u; };
 
     // A bounded wait that the whole warp agrees on; a timeout raises the CTA's abort
-    // flag (every role then stops taking new work) and the device error word.
+    // flag (every role then stops taking new work) and the device error word.  The
+    // softmax warps and the two MMA-issuing threads (the critical path) spin; the other
+    // roles sleep in hardware while they wait, leaving the issue slots to the warps that
+    // compute.
+    const bool spin_waits = warp >= 7;
     auto wait_warp = [&](uint32_t bar, uint32_t parity) -> bool {
-        bool ok = *abort_flag == 0 && mbar_wait_bounded(bar, parity);
+        bool ok = mbar_test_wait(bar, parity);   // fast path: already complete
+        if (!__all_sync(FULL, ok))
+            ok = ok || (*abort_flag == 0 && (spin_waits ? mbar_wait_spin(bar, parity) : mbar_wait_bounded(bar, parity)));
         ok = __all_sync(FULL, ok);
         if (!ok && lane == 0) {
             if (*abort_flag == 0) atomicOr(p.err, kErrTimeout);
@@ -215,9 +261,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
         return ok;
     };
-    auto wait_one = [&](uint32_t bar, uint32_t parity) -> bool {   // single thread
+    auto wait_one = [&](uint32_t bar, uint32_t parity) -> bool {   // single thread (the MMA issuers: spin)
+        if (mbar_test_wait(bar, parity)) return true;
         if (*abort_flag != 0) return false;
-        if (mbar_wait_bounded(bar, parity)) return true;
+        if (mbar_wait_spin(bar, parity)) return true;
         atomicOr(p.err, kErrTimeout);
         *abort_flag = 1;
         return false;
@@ -229,14 +276,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
             mbar_init(full_b(s), 1);
             mbar_init(empty_b(s), 9);   // QK commit + 4 value warps + 4 softmax warps
         }
-        for (int j = 0; j < 2; j++) {
+        for (int j = 0; j < T::NSB; j++) {
             mbar_init(sfull_b + 8 * j, 1);
             mbar_init(sfree_b + 8 * j, 4);
-            mbar_init(wfull_b + 8 * j, 4);
-            mbar_init(vfull_b + 8 * j, 4);
-            mbar_init(pvdone_b + 8 * j, 1);
-            mbar_init(xfull_b + 8 * j, 4);
         }
+        for (int j = 0; j < T::NWB; j++) mbar_init(wfull_b + 8 * j, 4);
+        for (int j = 0; j < T::NVB; j++) mbar_init(vfull_b + 8 * j, 4);
+        for (int j = 0; j < T::NPB; j++) mbar_init(pvdone_b + 8 * j, 1);
         mbar_fence_init();
         misc[1] = 0;
         misc[2] = 0;
@@ -249,13 +295,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         if (lane == 0) misc[0] = s;
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(misc + 3), kTmemCols);
+        tmem_alloc(smem_u32(misc + 3), T::TCOLS);
         tmem_relinquish();
         tc_fence_before();
     }
-    if (warp >= 2 && warp < 6) {
+    if (warp >= 3 && warp < 7) {
         // the all-ones A operand of the sum MMA, and the zero padding rows of the limb operand
-        const int tid = threadIdx.x - 64;
+        const int tid = threadIdx.x - 96;
         uint4* f = reinterpret_cast<uint4*>(smem + S.fmat);
         for (int i = tid; i < 256; i += 128) f[i] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
         uint4* z = reinterpret_cast<uint4*>(smem + S.qlimb + (size_t)3 * ROWS * D);
@@ -269,8 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     // Q = rint(q * 2^(22 - E)) with |q| < 2^E the row's absmax bound, |Q| <= 2^22, and
     // Q = l2 * 2^16 + l1 * 2^8 + l0 with l0, l1 in [-128, 127] and |l2| <= 65.  Limb k
     // of row r is row k * ROWS + r of the N x D (K-major) score operand.
-    if (warp >= 6) {
-        const int tid = threadIdx.x - 192;
+    if (warp >= 7) {
+        const int tid = threadIdx.x - 224;
         constexpr int SL = D / 8;   // 8-channel slices of a row
         for (int it = tid; it < ROWS * SL; it += 128) {
             const int r = it / SL, sl = it % SL;
@@ -318,7 +364,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
         fence_proxy_async_smem();
     }
-    __syncthreads();
+    // the TMA producer starts at once; the other warps wait for the limbs and TMEM
+    if (warp != 0) named_bar_sync(1, kThreads - 32);
     tc_fence_after();
     const uint32_t tmem = (uint32_t)misc[3];
     const uint32_t ring = smem_u32(smem + S.ring);
@@ -326,16 +373,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     if (warp == 0) {
         // ================= TMA producer =================
         const uint64_t policy = l2_evict_first_policy();
+        // block-table entries of chunk i (lanes < 8), loaded one chunk ahead
+        auto bt_load = [&](int i) -> int {
+            const int lp = (c0 + i) * kChunkPages + lane;
+            return (i < n_ck && lane < kChunkPages && lp < n_pages)
+                       ? __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + lp)
+                       : 0;
+        };
+        int blk_next = bt_load(0);
         int issued = 0;
         for (int i = 0; i < n_ck; i++) {
             const int s = i % NS;
             if (i >= NS && !wait_warp(empty_b(s), (uint32_t)((i - NS) / NS) & 1u)) break;
             const int c = c0 + i;
             const int npg = min(kChunkPages, n_pages - c * kChunkPages);
-            int blk = 0;
+            int blk = blk_next;
             bool bad = true;
             if (lane < npg) {
-                blk = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + (long long)c * kChunkPages + lane);
                 bad = blk < 0 || (long long)blk >= p.n_blocks;
                 if (bad) {
                     atomicOr(p.err, kErrBadBlock);
@@ -350,67 +404,74 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
                 tma_load_1d(ring + (uint32_t)((s * kChunkPages + lane) * T::PB),
                             p.pool + ((long long)blk * p.n_kv_heads + hk) * T::PB, T::PB, full_b(s), policy);
             issued = i + 1;
+            blk_next = bt_load(i + 1);
         }
         // after an abort: let copies still in flight land before the CTA leaves
         if (*abort_flag != 0 && lane == 0)
             for (int k = max(0, issued - NS); k < issued; k++) mbar_wait_bounded(full_b(k % NS), (uint32_t)(k / NS) & 1u);
     } else if (warp == 1) {
-        // ================= MMA issuer (one thread) =================
+        // ================= score MMAs (one thread) =================
         if (lane == 0) {
-            const uint32_t wb0 = smem_u32(smem + S.wbuf), ql = smem_u32(smem + S.qlimb);
+            const uint32_t ql = smem_u32(smem + S.qlimb);
             constexpr uint32_t IDQ = instr_desc(2, 1, 1, 0, 0, 128, T::NQ);   // s32 <- s8 x s8, K-major
-            constexpr uint32_t IDO = instr_desc(1, 0, 0, 0, 1, 128, T::NO);   // f32 <- f16 x f16, B MN-major
-            constexpr uint32_t IDS = instr_desc(1, 0, 0, 0, 1, 128, T::NB);
-            const uint64_t fdesc = smem_desc(smem_u32(smem + S.fmat), 128, 256);
             uint32_t last_bar = 0, last_par = 0;
-            for (int i = 0; i <= n_ck; i++) {
-                if (i < n_ck) {
-                    const int s = i % NS, sb = i % T::NSB;
-                    if (!wait_one(full_b(s), (uint32_t)(i / NS) & 1u)) break;
-                    if (i >= T::NSB && !wait_one(sfree_b + 8 * sb, (uint32_t)((i - T::NSB) / T::NSB) & 1u)) break;
-                    tc_fence_after();
-                    const uint32_t a0 = ring + (uint32_t)(s * kChunkPages * T::PB);
+            for (int i = 0; i < n_ck; i++) {
+                const int s = i % NS, sb = i % T::NSB;
+                if (!wait_one(full_b(s), (uint32_t)(i / NS) & 1u)) break;
+                if (i >= T::NSB && !wait_one(sfree_b + 8 * sb, (uint32_t)((i - T::NSB) / T::NSB) & 1u)) break;
+                tc_fence_after();
+                const uint32_t a0 = ring + (uint32_t)(s * kChunkPages * T::PB);
 #pragma unroll
-                    for (int k = 0; k < D / 32; k++)
-                        mma_i8_ss(tmem + T::T_S + sb * T::NQ, smem_desc(a0 + 256 * k, 128, T::REC),
-                                  smem_desc(ql + 256 * k, 128, 8 * D), IDQ, k > 0 ? 1u : 0u);
-                    tc_commit(sfull_b + 8 * sb);
-                    tc_commit(empty_b(s));
-                    last_bar = sfull_b + 8 * sb;
-                    last_par = (uint32_t)(i / T::NSB) & 1u;
-                }
-                if (i >= 1) {
-                    const int j = i - 1, wb = j & 1, vb = j % T::NVB;
-                    if (!wait_one(wfull_b + 8 * wb, (uint32_t)(j >> 1) & 1u)) break;
-                    if (!wait_one(vfull_b + 8 * vb, (uint32_t)(j / T::NVB) & 1u)) break;
-                    tc_fence_after();
-                    const uint32_t w0 = wb0 + (uint32_t)(wb * T::WBYTES);
-#pragma unroll 1
-                    for (int ks = 0; ks < kChunkTokens / 16; ks++) {
-                        const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
-                        const uint32_t wk = w0 + (uint32_t)(ks * 2 * T::LBO_W);
-#pragma unroll
-                        for (int h = 0; h < T::H; h++)
-                            mma_f16_ts(tmem + T::T_O + h * T::NO, tmem + T::T_VT + (vb * T::H + h) * 64 + 8 * ks,
-                                       smem_desc(wk + (uint32_t)(h * 64 * ROWS), T::LBO_W, 128), IDO, acc);
-                        mma_f16_ss(tmem + T::T_SUM, fdesc, smem_desc(wk, T::LBO_W, 128), IDS, acc);
-                    }
-                    tc_commit(pvdone_b + 8 * wb);
-                    last_bar = pvdone_b + 8 * wb;
-                    last_par = (uint32_t)(j >> 1) & 1u;
-                }
+                for (int k = 0; k < D / 32; k++)
+                    mma_i8_ss(tmem + T::T_S + sb * T::NQ, smem_desc(a0 + 256 * k, 128, T::REC),
+                              smem_desc(ql + 256 * k, 128, 8 * D), IDQ, k > 0 ? 1u : 0u);
+                tc_commit(sfull_b + 8 * sb);
+                tc_commit(empty_b(s));
+                last_bar = sfull_b + 8 * sb;
+                last_par = (uint32_t)(i / T::NSB) & 1u;
             }
             // after an abort: the MMAs already issued finish before TMEM is released
             if (*abort_flag != 0 && last_bar != 0) mbar_wait_bounded(last_bar, last_par);
         }
         __syncwarp();
-    } else if (warp < 6) {
+    } else if (warp == 2) {
+        // ================= value MMAs (one thread) =================
+        if (lane == 0) {
+            const uint32_t wb0 = smem_u32(smem + S.wbuf);
+            constexpr uint32_t IDO = instr_desc(1, 0, 0, 0, 1, 128, T::NO);   // f32 <- f16 x f16, B MN-major
+            constexpr uint32_t IDS = instr_desc(1, 0, 0, 0, 1, 128, T::NB);
+            const uint64_t fdesc = smem_desc(smem_u32(smem + S.fmat), 128, 256);
+            uint32_t last_bar = 0, last_par = 0;
+            for (int j = 0; j < n_ck; j++) {
+                const int wb = j % T::NWB, vb = j % T::NVB;
+                if (!wait_one(wfull_b + 8 * wb, (uint32_t)(j / T::NWB) & 1u)) break;
+                if (!wait_one(vfull_b + 8 * vb, (uint32_t)(j / T::NVB) & 1u)) break;
+                tc_fence_after();
+                const uint32_t w0 = wb0 + (uint32_t)(wb * T::WBYTES);
+#pragma unroll 1
+                for (int ks = 0; ks < kChunkTokens / 16; ks++) {
+                    const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
+                    const uint32_t wk = w0 + (uint32_t)(ks * 2 * T::LBO_W);
+#pragma unroll
+                    for (int h = 0; h < T::H; h++)
+                        mma_f16_ts(tmem + T::T_O + h * T::NO, tmem + T::T_VT + (vb * T::H + h) * 64 + 8 * ks,
+                                   smem_desc(wk + (uint32_t)(h * 64 * ROWS), T::LBO_W, 128), IDO, acc);
+                    mma_f16_ss(tmem + T::T_SUM, fdesc, smem_desc(wk, T::LBO_W, 128), IDS, acc);
+                }
+                tc_commit(pv_bar(j));
+                last_bar = pv_bar(j);
+                last_par = pv_par(j);
+            }
+            if (*abort_flag != 0 && last_bar != 0) mbar_wait_bounded(last_bar, last_par);
+        }
+        __syncwarp();
+    } else if (warp < 7) {
         // ================= value codes -> V^T in tensor memory =================
         const int q = warp & 3;
         for (int i = 0; i < n_ck; i++) {
             const int s = i % NS, vb = i % T::NVB;
             if (!wait_warp(full_b(s), (uint32_t)(i / NS) & 1u)) break;
-            if (i >= T::NVB && !wait_warp(pvdone_b + 8 * ((i - T::NVB) & 1), (uint32_t)((i - T::NVB) >> 1) & 1u))
+            if (i >= T::NVB && !wait_warp(pv_bar(i - T::NVB), pv_par(i - T::NVB)))
                 break;
             tc_fence_after();
             const uint32_t st = ring + (uint32_t)(s * kChunkPages * T::PB) + rec_v_off(D);
@@ -445,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
     } else {
         // ================= softmax and weights (one TMEM lane = one token) =================
-        const int sw = warp - 6, q = warp & 3, t = 32 * q + lane;
+        const int sw = warp - 7, q = warp & 3, t = 32 * q + lane;
         const int tp = t / 16, ttg = (t / 8) & 1, tt = t & 7;
         const uint32_t wb0 = smem_u32(smem + S.wbuf);
         float* xch = reinterpret_cast<float*>(smem + S.xch);
@@ -459,166 +520,165 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
         }
         float Mlane = -INFINITY;   // M of row `lane` (lanes < ROWS)
         const int lim_min = L - nq + row0 / p.group + 1;   // smallest limit of the real rows
+        const int nrg4 = (rows_here + 3) / 4;              // 4-row groups holding real rows
+        // A warp whose wait gave up keeps iterating without work, so that the four softmax
+        // warps always meet at the named barrier the same number of times.
         bool ok = true;
-        for (int i = 0; i < n_ck && ok; i++) {
-            const int s = i % NS, sb = i % T::NSB, wb = i & 1;
+        for (int i = 0; i < n_ck; i++) {
+            const int s = i % NS, sb = i % T::NSB, wb = i % T::NWB;
             const int c = c0 + i;
-            ok = wait_warp(sfull_b + 8 * sb, (uint32_t)(i / T::NSB) & 1u) && wait_warp(full_b(s), (uint32_t)(i / NS) & 1u);
-            if (!ok) break;
-            tc_fence_after();
-            // this token's scales and page flag
-            const uint32_t rec = ring + (uint32_t)((s * kChunkPages + tp) * T::PB + ttg * T::REC);
-            const float sk = h_bits_to_f32(ldsa16(rec + rec_ks_off(D) + 2 * tt));
-            float sv[T::G];
-            if constexpr (T::G == 4) {
-                const uint2 v = ldsa64(rec + rec_vs_off(D) + 8 * tt);
-                sv[0] = h_bits_to_f32(v.x & 0xFFFFu);
-                sv[1] = h_bits_to_f32(v.x >> 16);
-                sv[2] = h_bits_to_f32(v.y & 0xFFFFu);
-                sv[3] = h_bits_to_f32(v.y >> 16);
-            } else {
-                const uint4 v = ldsa128(rec + rec_vs_off(D) + 16 * tt);
-                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int k = 0; k < 4; k++) {
-                    sv[2 * k] = h_bits_to_f32(u[k] & 0xFFFFu);
-                    sv[2 * k + 1] = h_bits_to_f32(u[k] >> 16);
-                }
-            }
-            const int4 bf0 = *reinterpret_cast<const int4*>(pgbad + s * kChunkPages);
-            const int4 bf1 = *reinterpret_cast<const int4*>(pgbad + s * kChunkPages + 4);
-            const bool any_bad = (bf0.x | bf0.y | bf0.z | bf0.w | bf1.x | bf1.y | bf1.z | bf1.w) != 0;
-            const bool my_bad = pgbad[s * kChunkPages + tp] != 0;
-            // ---- scores: the three limb accumulations -> fp32 ----
+            // this token's scales and page flags; then the stage is released
+            float sk = 0.0f, sv[T::G];
+            bool any_bad = false, my_bad = false;
             float z[ROWS];
+            if (ok && wait_warp(full_b(s), (uint32_t)(i / NS) & 1u)) {
+                const uint32_t rec = ring + (uint32_t)((s * kChunkPages + tp) * T::PB + ttg * T::REC);
+                sk = h_bits_to_f32(ldsa16(rec + rec_ks_off(D) + 2 * tt));
+                if constexpr (T::G == 4) {
+                    const uint2 v = ldsa64(rec + rec_vs_off(D) + 8 * tt);
+                    sv[0] = h_bits_to_f32(v.x & 0xFFFFu);
+                    sv[1] = h_bits_to_f32(v.x >> 16);
+                    sv[2] = h_bits_to_f32(v.y & 0xFFFFu);
+                    sv[3] = h_bits_to_f32(v.y >> 16);
+                } else {
+                    const uint4 v = ldsa128(rec + rec_vs_off(D) + 16 * tt);
+                    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int rg = 0; rg < ROWS / 8; rg++) {
-                uint32_t a2[8], a1[8], a0[8];
-                const uint32_t col = T::T_S + sb * T::NQ + 8 * rg;
-                tmem_ld8(tmem_at(tmem, 32 * q, col), a2);
-                tmem_ld8(tmem_at(tmem, 32 * q, col + ROWS), a1);
-                tmem_ld8(tmem_at(tmem, 32 * q, col + 2 * ROWS), a0);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 8; e++) {
-                    const int x = (int)a2[e] * 256 + (int)a1[e];   // exact: |x| < 2^30
-                    const float sc = __fmaf_rn((float)x, 256.0f, (float)(int)a0[e]);
-                    z[8 * rg + e] = __fmul_rn(__fmul_rn(sc, crow[8 * rg + e]), sk);
+                    for (int k = 0; k < 4; k++) {
+                        sv[2 * k] = h_bits_to_f32(u[k] & 0xFFFFu);
+                        sv[2 * k + 1] = h_bits_to_f32(u[k] >> 16);
+                    }
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(sfree_b + 8 * sb);
-                mbar_arrive(empty_b(s));
-            }
-            // ---- visibility: sequence end, causal drafts, unusable pages ----
-            const bool clean = (c + 1) * kChunkTokens <= lim_min && !any_bad;
-            if (!clean) {
-                const int tok = c * kChunkTokens + t;
-#pragma unroll
-                for (int r = 0; r < ROWS; r++)
-                    if (my_bad || tok >= lim[r]) z[r] = -INFINITY;
-            }
-            // ---- chunk row maxima over the 128 tokens; lazy running max ----
-            float* xb = xch + (i & 1) * ROWS * 4;
-#pragma unroll
-            for (int r = 0; r < ROWS; r++) {
-                const float m = warp_redux_max(z[r]);
-                if (lane == 0) xb[r * 4 + sw] = m;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(xfull_b + 8 * (i & 1));
-            if (!wait_warp(xfull_b + 8 * (i & 1), (uint32_t)(i >> 1) & 1u)) {
+                const int4 bf0 = *reinterpret_cast<const int4*>(pgbad + s * kChunkPages);
+                const int4 bf1 = *reinterpret_cast<const int4*>(pgbad + s * kChunkPages + 4);
+                any_bad = (bf0.x | bf0.y | bf0.z | bf0.w | bf1.x | bf1.y | bf1.z | bf1.w) != 0;
+                my_bad = pgbad[s * kChunkPages + tp] != 0;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_b(s));
+            } else {
                 ok = false;
-                break;
             }
-            bool need = false;
-            float cm = -INFINITY;
-            if (lane < ROWS) {
-                const float4 v = *reinterpret_cast<const float4*>(xb + lane * 4);
-                cm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
-                need = cm > __fadd_rn(Mlane, kLazy);
-            }
-            if (__any_sync(FULL, need)) {
-                const float Mn = need ? cm : Mlane;
-                const float al = (Mn == Mlane) ? 1.0f : ex2(__fsub_rn(Mlane, Mn));
-                Mlane = Mn;
-                float alpha[ROWS];
+            if (ok && !wait_warp(sfull_b + 8 * sb, (uint32_t)(i / T::NSB) & 1u)) ok = false;
+            const bool clean = (c + 1) * kChunkTokens <= lim_min && !any_bad;
+            float* xb = xch + (i & 1) * ROWS * 4;
+            if (ok) {
+                tc_fence_after();
+                // ---- scores of the real rows: the three limb accumulations -> fp32 ----
 #pragma unroll
-                for (int r = 0; r < ROWS; r++) {
-                    M[r] = __shfl_sync(FULL, Mn, r);
-                    alpha[r] = __shfl_sync(FULL, al, r);
+                for (int rg = 0; rg < ROWS / 4; rg++) {
+                    if (rg < nrg4) {
+                        uint32_t a2[4], a1[4], a0[4];
+                        const uint32_t col = T::T_S + sb * T::NQ + 4 * rg;
+                        tmem_ld4(tmem_at(tmem, 32 * q, col), a2);
+                        tmem_ld4(tmem_at(tmem, 32 * q, col + ROWS), a1);
+                        tmem_ld4(tmem_at(tmem, 32 * q, col + 2 * ROWS), a0);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            const int x = (int)a2[e] * 256 + (int)a1[e];   // exact: |x| < 2^30
+                            const float sc = __fmaf_rn((float)x, 256.0f, (float)(int)a0[e]);
+                            z[4 * rg + e] = __fmul_rn(__fmul_rn(sc, crow[4 * rg + e]), sk);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; e++) z[4 * rg + e] = -INFINITY;
+                    }
                 }
-                if (i > 0) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sfree_b + 8 * sb);
+                // ---- visibility: sequence end, causal drafts, unusable pages ----
+                if (!clean) {
+                    const int tok = c * kChunkTokens + t;
+#pragma unroll
+                    for (int r = 0; r < ROWS; r++)
+                        if (my_bad || tok >= lim[r]) z[r] = -INFINITY;
+                }
+                // ---- chunk row maxima over the 128 tokens ----
+#pragma unroll
+                for (int rg = 0; rg < ROWS / 4; rg++)
+                    if (rg < nrg4) {
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            const float m = warp_redux_max(z[4 * rg + e]);
+                            if (lane == 0) xb[(4 * rg + e) * 4 + sw] = m;
+                        }
+                    }
+            }
+            named_bar_sync(2, 128);
+            if (ok) {
+                // ---- lazy running max: moved only when a chunk max exceeds it by kLazy ----
+                bool need = false;
+                float cm = -INFINITY;
+                if (lane < rows_here) {
+                    const float4 v = *reinterpret_cast<const float4*>(xb + lane * 4);
+                    cm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+                    need = cm > __fadd_rn(Mlane, kLazy);
+                }
+                if (__any_sync(FULL, need)) {
+                    const float Mn = need ? cm : Mlane;
+                    const float al = (Mn == Mlane) ? 1.0f : ex2(__fsub_rn(Mlane, Mn));
+                    Mlane = Mn;
+                    float alpha[ROWS];
+#pragma unroll
+                    for (int r = 0; r < ROWS; r++) {
+                        M[r] = __shfl_sync(FULL, Mn, r);
+                        alpha[r] = __shfl_sync(FULL, al, r);
+                    }
                     // rescale O and the sums (this warp's 32 lanes) once the previous
                     // chunk's value MMAs are complete
-                    if (!wait_warp(pvdone_b + 8 * ((i - 1) & 1), (uint32_t)((i - 1) >> 1) & 1u)) {
+                    if (i > 0 && wait_warp(pv_bar(i - 1), pv_par(i - 1))) {
+                        tc_fence_after();
+                        rescale_acc<ROWS, T::H * T::NO, T::NB>(tmem_at(tmem, 32 * q, 0), T::T_O, T::T_SUM, AlphaRows<ROWS>::make(alpha));
+                        tmem_wait_st();
+                    } else if (i > 0) {
                         ok = false;
-                        break;
                     }
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int cb = 0; cb < (T::H * T::NO + T::NB) / 8; cb++) {
-                        const int col = cb < T::H * T::NO / 8 ? T::T_O + 8 * cb : T::T_SUM + 8 * cb - T::H * T::NO;
-                        const int r0 = (8 * cb) % ROWS;   // NO and ROWS are multiples of 8
-                        uint32_t v[8];
-                        tmem_ld8(tmem_at(tmem, 32 * q, col), v);
-                        tmem_wait_ld();
-                        float a8[8];
-#pragma unroll
-                        for (int e = 0; e < 8; e++) a8[e] = alpha[0];
-#pragma unroll
-                        for (int r = 0; r < ROWS; r++)
-#pragma unroll
-                            for (int e = 0; e < 8; e++)
-                                if (r == (r0 + e) % ROWS) a8[e] = alpha[r];
-#pragma unroll
-                        for (int e = 0; e < 8; e++) v[e] = __float_as_uint(__fmul_rn(__uint_as_float(v[e]), a8[e]));
-                        tmem_st8(tmem_at(tmem, 32 * q, col), v);
-                    }
-                    tmem_wait_st();
                 }
             }
-            // ---- weights: p = 2^(z - M), W_g = p * s_v[g] (fp16) ----
-            float pw[ROWS];
+            if (ok && i >= T::NWB && !wait_warp(pv_bar(i - T::NWB), pv_par(i - T::NWB))) ok = false;
+            if (ok) {
+                // ---- weights of the real rows: p = 2^(z - M), W_g = p * s_v[g] (fp16) ----
+                float pw[ROWS];
 #pragma unroll
-            for (int r = 0; r < ROWS; r++) pw[r] = (z[r] == -INFINITY) ? 0.0f : ex2(__fsub_rn(z[r], M[r]));
-            if (i >= 2 && !wait_warp(pvdone_b + 8 * wb, (uint32_t)((i - 2) >> 1) & 1u)) {
-                ok = false;
-                break;
-            }
-            const uint32_t wrow = wb0 + (uint32_t)(wb * T::WBYTES + (t / 8) * T::LBO_W + (t % 8) * 16);
+                for (int r = 0; r < ROWS; r++)
+                    pw[r] = (r >= rows_here || z[r] == -INFINITY) ? 0.0f : ex2(__fsub_rn(z[r], M[r]));
+                const uint32_t wrow = wb0 + (uint32_t)(wb * T::WBYTES + (t / 8) * T::LBO_W + (t % 8) * 16);
+                auto store_group = [&](uint32_t a, const float* w, bool two) {
+                    // 8 rows of one 8-column group (two = both 4-row halves hold real rows)
+                    const uint32_t h0 = pack_h2(w[0], w[1]), h1 = pack_h2(w[2], w[3]);
+                    if (two) {
+                        stsa128(a, h0, h1, pack_h2(w[4], w[5]), pack_h2(w[6], w[7]));
+                    } else {
+                        asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(a), "r"(h0), "r"(h1) : "memory");
+                    }
+                };
 #pragma unroll
-            for (int g = 0; g < T::G; g++) {
+                for (int rg8 = 0; rg8 < ROWS / 8; rg8++) {
+                    if (2 * rg8 >= nrg4) continue;
+                    const bool two = 2 * rg8 + 1 < nrg4;
 #pragma unroll
-                for (int rg = 0; rg < ROWS / 8; rg++) {
-                    uint32_t hw[4];
+                    for (int g = 0; g < T::G; g++) {
+                        float w[8];
 #pragma unroll
-                    for (int e2 = 0; e2 < 4; e2++) {
-                        const int r = 8 * rg + 2 * e2;
-                        float w0 = __fmul_rn(pw[r], sv[g]), w1 = __fmul_rn(pw[r + 1], sv[g]);
-                        if (!clean) {   // masked tokens may carry unwritten (non-finite) scales
-                            w0 = pw[r] == 0.0f ? 0.0f : w0;
-                            w1 = pw[r + 1] == 0.0f ? 0.0f : w1;
+                        for (int e = 0; e < 8; e++) {
+                            const float pv = pw[8 * rg8 + e];
+                            const float wv = __fmul_rn(pv, sv[g]);
+                            // masked tokens may carry unwritten (non-finite) scales
+                            w[e] = (!clean && pv == 0.0f) ? 0.0f : wv;
                         }
-                        hw[e2] = pack_h2(w0, w1);
+                        store_group(wrow + (uint32_t)(((g * ROWS + 8 * rg8) / 8) * 128), w, two);
                     }
-                    stsa128(wrow + (uint32_t)(((g * ROWS + 8 * rg) / 8) * 128), hw[0], hw[1], hw[2], hw[3]);
+                    store_group(wrow + (uint32_t)(((T::G * ROWS + 8 * rg8) / 8) * 128), pw + 8 * rg8, two);
                 }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(wfull_b + 8 * wb);
             }
-#pragma unroll
-            for (int rg = 0; rg < ROWS / 8; rg++)
-                stsa128(wrow + (uint32_t)(((T::G * ROWS + 8 * rg) / 8) * 128), pack_h2(pw[8 * rg], pw[8 * rg + 1]),
-                        pack_h2(pw[8 * rg + 2], pw[8 * rg + 3]), pack_h2(pw[8 * rg + 4], pw[8 * rg + 5]),
-                        pack_h2(pw[8 * rg + 6], pw[8 * rg + 7]));
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(wfull_b + 8 * wb);
         }
         // ================= epilogue: the CTA partial in natural layout =================
-        if (ok) ok = wait_warp(pvdone_b + 8 * ((n_ck - 1) & 1), (uint32_t)((n_ck - 1) >> 1) & 1u);
+        if (ok) ok = wait_warp(pv_bar(n_ck - 1), pv_par(n_ck - 1));
         if (ok) {
             tc_fence_after();
             float lr[ROWS];
@@ -659,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const DecodeParams 
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, T::TCOLS);
     }
     if (*abort_flag != 0) return;
 
@@ -810,7 +870,15 @@ size_t decode_smem_bytes(int head_dim, int rows, int stages) {
 
 template <int D, int ROWS>
 static cudaError_t set_smem(size_t smem) {
-    return cudaFuncSetAttribute(decode_kernel<D, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // all of the unified L1 / shared-memory array as shared memory, so that the classes
+    // built for two CTAs per SM get both
+    return cudaFuncSetAttribute(decode_kernel<D, ROWS>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+}
+
+int decode_ctas_per_sm(int head_dim, int rows) {
+    return (head_dim == 128 && rows == 8) ? Tc<128, 8>::CPS : 1;
 }
 
 cudaError_t decode_prepare(int head_dim, int rows, size_t smem) {

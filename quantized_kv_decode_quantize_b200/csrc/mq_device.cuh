@@ -87,6 +87,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// One non-blocking test of the phase.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: gives up after ~2^31 cycles (about a second) and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -95,6 +106,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
         if (clock64() - t0 > (1ll << 31)) return false;
     }
     return true;
+}
+
+// Bounded wait for waits on a pipeline's critical path: spins on the non-blocking test
+// (no sleep, so the thread resumes within a few cycles of the phase completing) for
+// ~2^16 cycles, then continues as mbar_wait_bounded.
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity) {
+    if (mbar_test_wait(bar, parity)) return true;   // the common case: already complete
+    const long long t0 = clock64();
+    do {
+        if (mbar_test_wait(bar, parity)) return true;
+    } while (clock64() - t0 < (1ll << 16));
+    return mbar_wait_bounded(bar, parity);
 }
 
 // 1-D bulk copy global -> shared, completion counted on an mbarrier (no multicast).

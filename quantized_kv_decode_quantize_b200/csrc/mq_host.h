@@ -15,6 +15,7 @@ struct mq_cache {
     int device;
     int n_sm;
     int max_smem;
+    int smem_per_sm;
     unsigned* err_word;         // device address of this device's error word
     mq_decode_config cfg[3];    // per rows class
 };

@@ -55,6 +55,7 @@ struct DecodeParams {
 // rows: 8, 16 or 32 (padded query rows per kv-head handled by one CTA)
 size_t decode_smem_bytes(int head_dim, int rows, int stages);   // 0: does not fit the layout
 cudaError_t decode_prepare(int head_dim, int rows, size_t smem);  // raises the dynamic smem limit
+int decode_ctas_per_sm(int head_dim, int rows);                    // CTAs the kernel is built to co-host
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int max_splits, size_t smem,
                           cudaStream_t st);
 

@@ -225,7 +225,7 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
     std::vector<Cand> cands;
     bool class_used[3] = {false, false, false};
     for (auto& pr : probes) class_used[pr.cls] = true;
-    for (int r : {4, 3, 2})
+    for (int r : {8, 6, 4, 3, 2})
         for (int sps : {1, 2, 4})
             for (int cls = 0; cls < 3; cls++) {
                 if (!class_used[cls]) continue;
