@@ -226,7 +226,9 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
     const int n_ck = min(c0 + p.cpc, n_chunks) - c0;
     const int n_splits = (n_chunks + p.cpc - 1) / p.cpc;
 
-    int* misc = reinterpret_cast<int*>(smem + S.misc);   // 0 qoff, 1 abort, 2 last CTA, 3 TMEM base
+    // the dependent merge kernel may be scheduled now; it waits for this grid to complete
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    int* misc = reinterpret_cast<int*>(smem + S.misc);   // 0 qoff, 1 abort, 3 TMEM base
     volatile int* abort_flag = misc + 1;
     float* part = reinterpret_cast<float*>(smem + S.part);
     float* crow_s = reinterpret_cast<float*>(smem + S.crow);
@@ -285,7 +287,6 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
         for (int j = 0; j < T::NPB; j++) mbar_init(pvdone_b + 8 * j, 1);
         mbar_fence_init();
         misc[1] = 0;
-        misc[2] = 0;
     }
     if (warp == 0) {
         int s = 0;
@@ -748,7 +749,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
         finalize(part, part + ROWS * D, part + ROWS * D + ROWS);
         return;
     }
-    // ---- publish this CTA's partial; the last CTA completes the tree ----
+    // ---- publish this CTA's partial; merge_kernel completes the tree ----
     {
         float* go = p.part_o + (pidx * p.split_stride + sp) * (size_t)(ROWS * D);
         float* gml = p.part_ml + (pidx * p.split_stride + sp) * (size_t)(2 * ROWS);
@@ -756,37 +757,76 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
             __stcg(reinterpret_cast<float4*>(go) + i, reinterpret_cast<const float4*>(part)[i]);
         for (int i = threadIdx.x; i < 2 * ROWS; i += blockDim.x) __stcg(gml + i, part[ROWS * D + i]);
     }
-    __syncthreads();
-    // release: this CTA's partial (written by all threads, ordered by the barrier)
-    // happens-before the count; acquire: the last CTA sees every other CTA's partial
-    if (threadIdx.x == 0) misc[2] = (atom_add_acq_rel_gpu(p.counters + pidx, 1u) == (unsigned)(n_splits - 1)) ? 1 : 0;
-    __syncthreads();
-    if (misc[2] == 0) return;
+}
 
-    // Coefficients of every node of the padded tree over the n_splits CTA partials,
-    // heap-indexed (node (level, i) at 2^(H-level) + i), per row: m, l, alpha, beta.
-    int H = 0;
-    while ((1 << H) < n_splits) H++;
-    float* hp = reinterpret_cast<float*>(smem + S.heap);
-    auto hidx = [&](int level, int i) { return (1 << (H - level)) + i; };
+// Completes the fixed binary tree over the CTA partials of every (sequence, kv-head,
+// row block) with more than one split, and writes out and lse.  Launched right after
+// decode_kernel as a programmatic dependent launch: its CTAs may start while the decode
+// CTAs finish, and wait (griddepcontrol.wait) until all of them have completed and
+// their partials are visible.  One CTA covers 128 float4 elements of one unit's
+// [ROWS][D] result; its threads are 128 x (leaf groups of 8 splits): thread (e, j) loads
+// the 8 leaves of group j for element e at once and reduces that aligned level-3 subtree;
+// the group results then meet in shared memory for the levels above.
+template <int D, int ROWS>
+__global__ void __launch_bounds__(1024) merge_kernel(const DecodeParams p) {
+    constexpr int E4 = ROWS * D / 4;   // float4 elements of one partial
+    constexpr int RPC = 512 / D;       // rows covered by one CTA (128 float4)
+    __shared__ float hp[2 * kMaxSplits * RPC * 4];    // tree nodes: m, l, alpha, beta per row of this CTA
+    __shared__ float4 gsm[8][128];                     // group results
+    __shared__ int qoff_s;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int b = blockIdx.z, hk = blockIdx.y / p.n_rb, rb = blockIdx.y % p.n_rb;
+    const int L = __ldg(p.seq_lens + b), nq = __ldg(p.n_q_per_seq + b);
+    if (nq < 1 || nq > p.max_q || nq > L || (long long)L > (long long)p.max_blocks_per_seq * kPageTokens) return;
+    const int rows_b = p.group * nq, row0 = rb * ROWS;
+    if (row0 >= rows_b) return;
+    const int rows_here = min(ROWS, rows_b - row0);
+    const int n_chunks = (L + kChunkTokens - 1) / kChunkTokens;
+    const int n_splits = (n_chunks + p.cpc - 1) / p.cpc;
+    if (n_splits <= 1) return;   // decode_kernel wrote this unit's output itself
+    const int T = blockDim.x, tid = threadIdx.x;
+    const int e = tid & 127, j = tid >> 7;
+    const int e4 = blockIdx.x * 128 + e;
+    const int n_groups = (n_splits + 7) >> 3;
+    const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
     const float* gml0 = p.part_ml + pidx * p.split_stride * (size_t)(2 * ROWS);
     const float* go0 = p.part_o + pidx * p.split_stride * (size_t)(ROWS * D);
-    for (int i = threadIdx.x; i < n_splits * ROWS; i += blockDim.x) {
-        const int s = i / ROWS, r = i % ROWS;
-        float* nd = hp + ((size_t)hidx(0, s) * ROWS + r) * 4;
-        nd[0] = __ldcg(gml0 + (size_t)s * 2 * ROWS + r);
-        nd[1] = __ldcg(gml0 + (size_t)s * 2 * ROWS + ROWS + r);
+    // the 8 leaves of this thread's group, loads in flight together
+    float4 v[8];
+    const bool active = j < n_groups && e4 < E4;
+#pragma unroll
+    for (int u = 0; u < 8; u++) {
+        const int sidx = 8 * j + u;
+        v[u] = (active && sidx < n_splits) ? __ldcg(reinterpret_cast<const float4*>(go0 + (size_t)sidx * ROWS * D) + e4)
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (tid == 0) {
+        int s = 0;
+        for (int i = 0; i < b; i++) s += min(max(__ldg(p.n_q_per_seq + i), 0), p.max_q);
+        qoff_s = s;
+    }
+    // Coefficients of every node of the padded tree, heap-indexed (node (level, i) at
+    // 2^(H-level) + i), per row: m, l, alpha, beta.
+    int H = 0;
+    while ((1 << H) < n_splits) H++;
+    auto hidx = [&](int level, int i) { return (1 << (H - level)) + i; };
+    const int rbase = blockIdx.x * RPC;   // first row of this CTA's elements
+    for (int i = tid; i < n_splits * RPC; i += T) {
+        const int s = i / RPC, r = i % RPC;
+        float* nd = hp + ((size_t)hidx(0, s) * RPC + r) * 4;
+        nd[0] = __ldcg(gml0 + (size_t)s * 2 * ROWS + rbase + r);
+        nd[1] = __ldcg(gml0 + (size_t)s * 2 * ROWS + ROWS + rbase + r);
     }
     __syncthreads();
     for (int lv = 1; lv <= H; lv++) {
         const int n_here = (n_splits + (1 << lv) - 1) >> lv;
-        for (int i = threadIdx.x; i < n_here * ROWS; i += blockDim.x) {
-            const int ni = i / ROWS, r = i % ROWS;
-            float* nd = hp + ((size_t)hidx(lv, ni) * ROWS + r) * 4;
-            const float* lf = hp + ((size_t)hidx(lv - 1, 2 * ni) * ROWS + r) * 4;
+        for (int i = tid; i < n_here * RPC; i += T) {
+            const int ni = i / RPC, r = i % RPC;
+            float* nd = hp + ((size_t)hidx(lv, ni) * RPC + r) * 4;
+            const float* lf = hp + ((size_t)hidx(lv - 1, 2 * ni) * RPC + r) * 4;
             const bool has_right = (2 * ni + 1) * (1 << (lv - 1)) < n_splits;
             if (has_right) {
-                const float* rt = hp + ((size_t)hidx(lv - 1, 2 * ni + 1) * ROWS + r) * 4;
+                const float* rt = hp + ((size_t)hidx(lv - 1, 2 * ni + 1) * RPC + r) * 4;
                 merge_coef(lf[0], lf[1], rt[0], rt[1], nd[0], nd[1], nd[2], nd[3]);
             } else {
                 nd[0] = lf[0];
@@ -797,68 +837,63 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
         }
         __syncthreads();
     }
-    // Elements: the padded tree evaluated level by level in registers, eight leaves
-    // (an aligned level-3 subtree) at a time, their loads all in flight together.
-    float* fin = reinterpret_cast<float*>(smem + S.fin);   // final O [ROWS][D], m, l
-    const float* root = hp + (size_t)hidx(H, 0) * ROWS * 4;
-    const int n_groups = (n_splits + 7) >> 3;
-    for (int e4 = threadIdx.x; e4 < ROWS * D / 4; e4 += blockDim.x) {
-        const int r = (4 * e4) / D;
-        auto node_merge = [&](float4 lf, float4 rt, int level, int idx) {
-            const float* nd = hp + ((size_t)hidx(level, idx) * ROWS + r) * 4;
-            float4 o;
-            o.x = merge_val(lf.x, rt.x, nd[2], nd[3]);
-            o.y = merge_val(lf.y, rt.y, nd[2], nd[3]);
-            o.z = merge_val(lf.z, rt.z, nd[2], nd[3]);
-            o.w = merge_val(lf.w, rt.w, nd[2], nd[3]);
-            return o;
-        };
-        float4 gv[8];
+    const int r = (4 * (e4 < E4 ? e4 : 0)) / D;   // the element's row
+    const int rc = r - rbase;                        // ... within this CTA
+    auto node_merge = [&](float4 lf, float4 rt, int level, int idx) {
+        const float* nd = hp + ((size_t)hidx(level, idx) * RPC + rc) * 4;
+        float4 o;
+        o.x = merge_val(lf.x, rt.x, nd[2], nd[3]);
+        o.y = merge_val(lf.y, rt.y, nd[2], nd[3]);
+        o.z = merge_val(lf.z, rt.z, nd[2], nd[3]);
+        o.w = merge_val(lf.w, rt.w, nd[2], nd[3]);
+        return o;
+    };
+    // levels 1..3 within the group (an aligned subtree of 8 leaves)
+    if (active) {
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-            if (j < n_groups) {
-                float4 v[8];
+        for (int lv = 1; lv <= 3; lv++) {
 #pragma unroll
-                for (int u = 0; u < 8; u++) {
-                    const int sidx = 8 * j + u;
-                    v[u] = sidx < n_splits ? __ldcg(reinterpret_cast<const float4*>(go0 + (size_t)sidx * ROWS * D) + e4)
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int lv = 1; lv <= 3; lv++) {
-#pragma unroll
-                    for (int u = 0; u < (8 >> lv); u++) {
-                        const int idx = ((8 * j) >> lv) + u;           // node (lv, idx)
-                        const bool has_right = (2 * idx + 1) * (1 << (lv - 1)) < n_splits;
-                        if (lv <= H) v[u] = has_right ? node_merge(v[2 * u], v[2 * u + 1], lv, idx) : v[2 * u];
-                    }
-                }
-                gv[j] = v[0];
+            for (int u = 0; u < (8 >> lv); u++) {
+                const int idx = ((8 * j) >> lv) + u;   // node (lv, idx)
+                const bool has_right = (2 * idx + 1) * (1 << (lv - 1)) < n_splits;
+                if (lv <= H) v[u] = has_right ? node_merge(v[2 * u], v[2 * u + 1], lv, idx) : v[2 * u];
             }
         }
-        // levels 4 .. H over the group nodes
-#pragma unroll
-        for (int lv = 4; lv <= 6; lv++) {
-#pragma unroll
-            for (int u = 0; u < (64 >> lv); u++) {
-                if (lv <= H && u * (1 << lv) < n_splits) {
-                    const bool has_right = (2 * u + 1) * (1 << (lv - 1)) < n_splits;
-                    gv[u] = has_right ? node_merge(gv[2 * u], gv[2 * u + 1], lv, u) : gv[2 * u];
-                }
-            }
-        }
-        reinterpret_cast<float4*>(fin)[e4] = gv[0];
-    }
-    float* fml = fin + ROWS * D;
-    for (int r = threadIdx.x; r < ROWS; r += blockDim.x) {
-        fml[r] = root[r * 4 + 0];
-        fml[ROWS + r] = root[r * 4 + 1];
+        gsm[j][e] = v[0];
     }
     __syncthreads();
-    finalize(fin, fml, fml + ROWS);
-    if (threadIdx.x == 0) p.counters[pidx] = 0u;
+    if (j != 0 || e4 >= E4) return;
+    // levels 4 .. H over the group results
+    float4 gv[8];
+#pragma unroll
+    for (int u = 0; u < 8; u++) gv[u] = u < n_groups ? gsm[u][e] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int lv = 4; lv <= 6; lv++) {
+#pragma unroll
+        for (int u = 0; u < (64 >> lv); u++) {
+            if (lv <= H && u * (1 << lv) < n_splits) {
+                const bool has_right = (2 * u + 1) * (1 << (lv - 1)) < n_splits;
+                gv[u] = has_right ? node_merge(gv[2 * u], gv[2 * u + 1], lv, u) : gv[2 * u];
+            }
+        }
+    }
+    // out = O / l and lse for a real row
+    const int rl = r, c4 = e4 % (D / 4);
+    if (rl >= rows_here) return;
+    const int rr = row0 + rl, jq = rr / p.group, hq = rr % p.group;
+    const long long qrow = (long long)qoff_s + jq;
+    if (qrow >= p.total_q) return;
+    const float* root = hp + (size_t)hidx(H, 0) * RPC * 4;
+    const float l = root[rc * 4 + 1], m = root[rc * 4 + 0];
+    float4 o = gv[0];
+    o.x = __fdiv_rn(o.x, l);
+    o.y = __fdiv_rn(o.y, l);
+    o.z = __fdiv_rn(o.z, l);
+    o.w = __fdiv_rn(o.w, l);
+    const size_t orow = (size_t)qrow * p.n_q_heads + (size_t)hk * p.group + hq;
+    reinterpret_cast<float4*>(p.out + orow * D)[c4] = o;
+    if (c4 == 0 && p.lse != nullptr) p.lse[orow] = __fmul_rn(__fadd_rn(m, log2f(l)), 0.69314718055994531f);
 }
-
 
 size_t decode_smem_bytes(int head_dim, int rows, int stages) {
 #define MQ_SMEM(DD, RR) \
@@ -890,16 +925,34 @@ cudaError_t decode_prepare(int head_dim, int rows, size_t smem) {
     return cudaErrorInvalidValue;
 }
 
+// decode_kernel, then (when any unit has several splits) merge_kernel as a programmatic
+// dependent launch on the same stream.
+template <int D, int ROWS>
+static cudaError_t launch_pair(const DecodeParams& p, dim3 grid, size_t smem, int max_splits, cudaStream_t st) {
+    decode_kernel<D, ROWS><<<grid, dim3((unsigned)kThreads), smem, st>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || max_splits <= 1) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)((ROWS * D / 4 + 127) / 128), grid.y, grid.z);
+    cfg.blockDim = dim3((unsigned)(128 * ((max_splits + 7) / 8)));
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, merge_kernel<D, ROWS>, p);
+}
+
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int max_splits, size_t smem,
                           cudaStream_t st) {
     const dim3 grid((unsigned)max_splits, (unsigned)(p.n_kv_heads * p.n_rb), (unsigned)p.n_seqs);
-    const dim3 block((unsigned)kThreads);
 #define MQ_LAUNCH(DD, RR) \
-    if (head_dim == DD && rows == RR) decode_kernel<DD, RR><<<grid, block, smem, st>>>(p); else
+    if (head_dim == DD && rows == RR) return launch_pair<DD, RR>(p, grid, smem, max_splits, st);
     MQ_LAUNCH(128, 8) MQ_LAUNCH(128, 16) MQ_LAUNCH(128, 32) MQ_LAUNCH(256, 8) MQ_LAUNCH(256, 16)
-    return cudaErrorInvalidValue;
 #undef MQ_LAUNCH
-    return cudaGetLastError();
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace mq
