@@ -171,6 +171,27 @@ __device__ __forceinline__ float h_bits_to_f32(uint32_t bits) {
     return __half2float(__ushort_as_half((unsigned short)bits));
 }
 
+// Slow paths of the decode kernel's waits (out of line).  wait_slow_warp: the whole
+// warp; `done` is this lane's result of the first test.  A timeout raises the CTA's
+// abort flag and the device error word.
+__device__ __noinline__ bool wait_slow_warp(uint32_t bar, uint32_t parity, bool spin, bool done,
+                                            volatile int* abort_flag, unsigned* err) {
+    bool ok = done || (*abort_flag == 0 && (spin ? mbar_wait_spin(bar, parity) : mbar_wait_bounded(bar, parity)));
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok && (threadIdx.x & 31) == 0) {
+        if (*abort_flag == 0) atomicOr(err, kErrTimeout);
+        *abort_flag = 1;
+    }
+    return ok;
+}
+__device__ __noinline__ bool wait_slow_one(uint32_t bar, uint32_t parity, volatile int* abort_flag, unsigned* err) {
+    if (*abort_flag != 0) return false;
+    if (mbar_wait_spin(bar, parity)) return true;
+    atomicOr(err, kErrTimeout);
+    *abort_flag = 1;
+    return false;
+}
+
 template <int ROWS>
 struct AlphaRows {
     float a[ROWS];
@@ -250,26 +271,17 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
     // flag (every role then stops taking new work) and the device error word.  The
     // softmax warps and the two MMA-issuing threads (the critical path) spin; the other
     // roles sleep in hardware while they wait, leaving the issue slots to the warps that
-    // compute.
+    // compute.  The fast path (already complete) is one test and a vote; the rest is
+    // out of line, keeping the role loops small in the instruction cache.
     const bool spin_waits = warp >= 7;
     auto wait_warp = [&](uint32_t bar, uint32_t parity) -> bool {
-        bool ok = mbar_test_wait(bar, parity);   // fast path: already complete
-        if (!__all_sync(FULL, ok))
-            ok = ok || (*abort_flag == 0 && (spin_waits ? mbar_wait_spin(bar, parity) : mbar_wait_bounded(bar, parity)));
-        ok = __all_sync(FULL, ok);
-        if (!ok && lane == 0) {
-            if (*abort_flag == 0) atomicOr(p.err, kErrTimeout);
-            *abort_flag = 1;
-        }
-        return ok;
+        const bool done = mbar_test_wait(bar, parity);
+        if (__all_sync(FULL, done)) return true;
+        return wait_slow_warp(bar, parity, spin_waits, done, abort_flag, p.err);
     };
     auto wait_one = [&](uint32_t bar, uint32_t parity) -> bool {   // single thread (the MMA issuers: spin)
         if (mbar_test_wait(bar, parity)) return true;
-        if (*abort_flag != 0) return false;
-        if (mbar_wait_spin(bar, parity)) return true;
-        atomicOr(p.err, kErrTimeout);
-        *abort_flag = 1;
-        return false;
+        return wait_slow_one(bar, parity, abort_flag, p.err);
     };
 
     // ---- set-up: barriers, query-row offset, TMEM, constant operands ----
