@@ -184,14 +184,10 @@ mq_status mq_kv_append(mq_cache* cache, const void* k, const void* v, mq_dtype d
  *   lse          fp32 [sum_b n_b][n_q_heads], natural-log log-sum-exp of the
  *                scaled logits; may be NULL
  *   workspace    device scratch of at least mq_decode_workspace_bytes(...)
- *                bytes, 256-byte aligned.  Its front 1/512 (rounded up to 256
- *                bytes) holds per-(sequence, kv-head, row block) counters that
- *                must be zero before the first call; every call that completes
- *                leaves them zero again, so the workspace can be reused across
- *                calls of any shape that fits it without clearing, provided
- *                every call on it passes the same workspace_bytes (that value
- *                fixes where the counters sit).  After MQ_ERR_DEVICE, zero it
- *                again.  Calls that share a workspace must not overlap.
+ *                bytes, 256-byte aligned, holding the CTA partials of the
+ *                split reduction (see mq_decode_workspace_bytes).  It needs no
+ *                initialization and can be reused by later calls of any shape
+ *                that fits it.  Calls that share a workspace must not overlap.
  *   workspace_bytes  its size; a workspace smaller than the query for this
  *                shape is refused with MQ_ERR_WORKSPACE.
  * Query token j of sequence b (0-based) attends to positions 0 .. L_b - n_b + j:
@@ -228,8 +224,8 @@ mq_status mq_decode_attn(const mq_cache* cache, const void* q, mq_dtype q_dtype,
  *
  * Arguments, layouts, ownership and results are those of mq_decode_attn,
  * without workspace and workspace_bytes; the outputs equal mq_decode_attn's.
- * Each call first clears the split counters at the front of the scratch with an
- * asynchronous memset on `stream`, then launches the decode kernel there.
+ * The call launches the decode kernels on `stream` with the array as their
+ * workspace.
  * Make the first call on each device before any stream capture that is to
  * contain a later call: that first call does the address lookup.
  * The scratch is shared by every call on a device: calls whose executions may

@@ -99,16 +99,13 @@ size_t partial_bytes(const mq_cache* c, int n_seqs, const DecodePlan& pl) {
     return al256(slots * pl.rows * 2 * 4) + slots * pl.rows * c->head_dim * 4;
 }
 
-size_t counter_bytes(size_t workspace_bytes) { return al256((workspace_bytes + 511) / 512); }
-
 mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void* q, mq_dtype q_dtype, int n_seqs,
                              int n_q_heads, int total_q, int max_q, const int32_t* block_table, int max_blocks,
                              const int32_t* seq_lens, const int32_t* n_q_per_seq, float softmax_scale, float* out,
                              float* lse, void* workspace, size_t workspace_bytes, cudaStream_t st) {
     if (pl.smem == 0 || pl.smem > (size_t)c->max_smem) return MQ_ERR_UNSUPPORTED;
     const size_t units = (size_t)n_seqs * c->n_kv_heads * pl.n_rb;
-    const size_t cb = counter_bytes(workspace_bytes);
-    if (units * 4 > cb || cb + partial_bytes(c, n_seqs, pl) > workspace_bytes) return MQ_ERR_WORKSPACE;
+    if (partial_bytes(c, n_seqs, pl) > workspace_bytes) return MQ_ERR_WORKSPACE;
     cudaError_t e = ensure_decode_smem(c->device, c->head_dim, pl.rows, pl.smem);
     if (e != cudaSuccess) return MQ_ERR_CUDA;
     DecodeParams p{};
@@ -129,11 +126,9 @@ mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void
     p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
     p.out = out;
     p.lse = lse;
-    // counters in the fixed front region (the same bytes for every shape that shares
-    // this workspace), then this call's partials with a stride of max_splits per unit
+    // this call's partials: (m, l) then O, with a stride of max_splits per unit
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    p.counters = reinterpret_cast<unsigned*>(ws);
-    size_t off = cb;
+    size_t off = 0;
     p.part_ml = reinterpret_cast<float*>(ws + off);
     off += al256(units * pl.max_splits * pl.rows * 2 * 4);
     p.part_o = reinterpret_cast<float*>(ws + off);
@@ -278,14 +273,7 @@ size_t mq_decode_workspace_bytes(const mq_cache* c, int32_t n_seqs, int32_t n_q_
                                                  max_seq_len);
             part = std::max(part, partial_bytes(c, n_seqs, pl));
         }
-    // counters take the front 1/512 of the workspace (rounded up to 256 bytes); a
-    // 256-byte margin keeps any larger workspace valid as well
-    size_t need = part + 256;
-    for (size_t prev = 0; prev != need;) {
-        prev = need;
-        need = part + counter_bytes(need) + 256;
-    }
-    return need;
+    return part;
 }
 
 mq_status mq_decode_attn(const mq_cache* c, const void* q, mq_dtype q_dtype, int32_t n_seqs, int32_t n_q_heads,

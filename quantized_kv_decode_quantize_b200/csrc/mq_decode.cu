@@ -776,19 +776,55 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
 // decode_kernel as a programmatic dependent launch: its CTAs may start while the decode
 // CTAs finish, and wait (griddepcontrol.wait) until all of them have completed and
 // their partials are visible.  One CTA covers 128 float4 elements of one unit's
-// [ROWS][D] result; its threads are 128 x (leaf groups of 8 splits): thread (e, j) loads
-// the 8 leaves of group j for element e at once and reduces that aligned level-3 subtree;
-// the group results then meet in shared memory for the levels above.
+// [ROWS][D] result; its threads are 128 x (leaf groups of 8 splits).  Thread (e, j)
+// loads the 8 leaves of group j for element e (O, m, l) at once and evaluates that
+// aligned level-3 subtree, coefficients included; the group results meet in shared
+// memory, where thread (e, 0) evaluates the levels above.  Every node is
+// merge(left, right) with merge_coef / merge_val, a node without a right child passes
+// its left child through.
+struct MergeOut {
+    float4 o;
+    float m, l;
+};
+// One tree node: merge(left, right), or the left child passed through.
+__device__ __forceinline__ MergeOut merge_pair(float4 lo, float lm, float ll, float4 ro, float rm, float rl,
+                                               bool has_right) {
+    if (!has_right) return MergeOut{lo, lm, ll};
+    float m, l, a, b;
+    merge_coef(lm, ll, rm, rl, m, l, a, b);
+    return MergeOut{make_float4(merge_val(lo.x, ro.x, a, b), merge_val(lo.y, ro.y, a, b), merge_val(lo.z, ro.z, a, b),
+                                merge_val(lo.w, ro.w, a, b)),
+                    m, l};
+}
+
 template <int D, int ROWS>
 __global__ void __launch_bounds__(1024) merge_kernel(const DecodeParams p) {
     constexpr int E4 = ROWS * D / 4;   // float4 elements of one partial
-    constexpr int RPC = 512 / D;       // rows covered by one CTA (128 float4)
-    __shared__ float hp[2 * kMaxSplits * RPC * 4];    // tree nodes: m, l, alpha, beta per row of this CTA
-    __shared__ float4 gsm[8][128];                     // group results
-    __shared__ int qoff_s;
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float4 g_o[8][128];     // group results: O
+    __shared__ float2 g_ml[8][128];    // group results: m, l
+    // the sequence's bounds: inputs of the launch, readable before the decode grid ends
     const int b = blockIdx.z, hk = blockIdx.y / p.n_rb, rb = blockIdx.y % p.n_rb;
     const int L = __ldg(p.seq_lens + b), nq = __ldg(p.n_q_per_seq + b);
+    const int e = threadIdx.x & 127, j = threadIdx.x >> 7;
+    const int e4 = blockIdx.x * 128 + e;   // < E4: the grid covers E4 exactly
+    const int r = (4 * e4) / D;            // the element's row
+    const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
+    const float* gml0 = p.part_ml + pidx * p.split_stride * (size_t)(2 * ROWS);
+    const float* go0 = p.part_o + pidx * p.split_stride * (size_t)(ROWS * D);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the 8 leaves of this thread's group, loads in flight before the split count is
+    // known (every slot below split_stride exists; unused ones are ignored below)
+    float4 v[8];
+    float vm[8], vl[8];
+#pragma unroll
+    for (int u = 0; u < 8; u++) {
+        const int sidx = 8 * j + u;
+        const bool slot = sidx < p.split_stride;
+        v[u] = slot ? __ldcg(reinterpret_cast<const float4*>(go0 + (size_t)sidx * ROWS * D) + e4)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+        vm[u] = slot ? __ldcg(gml0 + (size_t)sidx * 2 * ROWS + r) : -INFINITY;
+        vl[u] = slot ? __ldcg(gml0 + (size_t)sidx * 2 * ROWS + ROWS + r) : 0.0f;
+    }
     if (nq < 1 || nq > p.max_q || nq > L || (long long)L > (long long)p.max_blocks_per_seq * kPageTokens) return;
     const int rows_b = p.group * nq, row0 = rb * ROWS;
     if (row0 >= rows_b) return;
@@ -796,107 +832,65 @@ __global__ void __launch_bounds__(1024) merge_kernel(const DecodeParams p) {
     const int n_chunks = (L + kChunkTokens - 1) / kChunkTokens;
     const int n_splits = (n_chunks + p.cpc - 1) / p.cpc;
     if (n_splits <= 1) return;   // decode_kernel wrote this unit's output itself
-    const int T = blockDim.x, tid = threadIdx.x;
-    const int e = tid & 127, j = tid >> 7;
-    const int e4 = blockIdx.x * 128 + e;
     const int n_groups = (n_splits + 7) >> 3;
-    const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
-    const float* gml0 = p.part_ml + pidx * p.split_stride * (size_t)(2 * ROWS);
-    const float* go0 = p.part_o + pidx * p.split_stride * (size_t)(ROWS * D);
-    // the 8 leaves of this thread's group, loads in flight together
-    float4 v[8];
-    const bool active = j < n_groups && e4 < E4;
-#pragma unroll
-    for (int u = 0; u < 8; u++) {
-        const int sidx = 8 * j + u;
-        v[u] = (active && sidx < n_splits) ? __ldcg(reinterpret_cast<const float4*>(go0 + (size_t)sidx * ROWS * D) + e4)
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    if (tid == 0) {
-        int s = 0;
-        for (int i = 0; i < b; i++) s += min(max(__ldg(p.n_q_per_seq + i), 0), p.max_q);
-        qoff_s = s;
-    }
-    // Coefficients of every node of the padded tree, heap-indexed (node (level, i) at
-    // 2^(H-level) + i), per row: m, l, alpha, beta.
     int H = 0;
     while ((1 << H) < n_splits) H++;
-    auto hidx = [&](int level, int i) { return (1 << (H - level)) + i; };
-    const int rbase = blockIdx.x * RPC;   // first row of this CTA's elements
-    for (int i = tid; i < n_splits * RPC; i += T) {
-        const int s = i / RPC, r = i % RPC;
-        float* nd = hp + ((size_t)hidx(0, s) * RPC + r) * 4;
-        nd[0] = __ldcg(gml0 + (size_t)s * 2 * ROWS + rbase + r);
-        nd[1] = __ldcg(gml0 + (size_t)s * 2 * ROWS + ROWS + rbase + r);
-    }
-    __syncthreads();
-    for (int lv = 1; lv <= H; lv++) {
-        const int n_here = (n_splits + (1 << lv) - 1) >> lv;
-        for (int i = tid; i < n_here * RPC; i += T) {
-            const int ni = i / RPC, r = i % RPC;
-            float* nd = hp + ((size_t)hidx(lv, ni) * RPC + r) * 4;
-            const float* lf = hp + ((size_t)hidx(lv - 1, 2 * ni) * RPC + r) * 4;
-            const bool has_right = (2 * ni + 1) * (1 << (lv - 1)) < n_splits;
-            if (has_right) {
-                const float* rt = hp + ((size_t)hidx(lv - 1, 2 * ni + 1) * RPC + r) * 4;
-                merge_coef(lf[0], lf[1], rt[0], rt[1], nd[0], nd[1], nd[2], nd[3]);
-            } else {
-                nd[0] = lf[0];
-                nd[1] = lf[1];
-                nd[2] = 1.0f;
-                nd[3] = 0.0f;
-            }
-        }
-        __syncthreads();
-    }
-    const int r = (4 * (e4 < E4 ? e4 : 0)) / D;   // the element's row
-    const int rc = r - rbase;                        // ... within this CTA
-    auto node_merge = [&](float4 lf, float4 rt, int level, int idx) {
-        const float* nd = hp + ((size_t)hidx(level, idx) * RPC + rc) * 4;
-        float4 o;
-        o.x = merge_val(lf.x, rt.x, nd[2], nd[3]);
-        o.y = merge_val(lf.y, rt.y, nd[2], nd[3]);
-        o.z = merge_val(lf.z, rt.z, nd[2], nd[3]);
-        o.w = merge_val(lf.w, rt.w, nd[2], nd[3]);
-        return o;
-    };
-    // levels 1..3 within the group (an aligned subtree of 8 leaves)
-    if (active) {
+    if (j < n_groups) {
+        // levels 1..3 within the group
 #pragma unroll
         for (int lv = 1; lv <= 3; lv++) {
 #pragma unroll
             for (int u = 0; u < (8 >> lv); u++) {
                 const int idx = ((8 * j) >> lv) + u;   // node (lv, idx)
                 const bool has_right = (2 * idx + 1) * (1 << (lv - 1)) < n_splits;
-                if (lv <= H) v[u] = has_right ? node_merge(v[2 * u], v[2 * u + 1], lv, idx) : v[2 * u];
+                const MergeOut mo = merge_pair(v[2 * u], vm[2 * u], vl[2 * u], v[2 * u + 1], vm[2 * u + 1],
+                                               vl[2 * u + 1], has_right);
+                if (lv <= H) {
+                    v[u] = mo.o;
+                    vm[u] = mo.m;
+                    vl[u] = mo.l;
+                }
             }
         }
-        gsm[j][e] = v[0];
+        g_o[j][e] = v[0];
+        g_ml[j][e] = make_float2(vm[0], vl[0]);
     }
     __syncthreads();
-    if (j != 0 || e4 >= E4) return;
+    if (j != 0) return;
     // levels 4 .. H over the group results
     float4 gv[8];
+    float gm[8], gl[8];
 #pragma unroll
-    for (int u = 0; u < 8; u++) gv[u] = u < n_groups ? gsm[u][e] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < 8; u++) {
+        const bool here = u < n_groups;
+        gv[u] = here ? g_o[u][e] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float2 ml = here ? g_ml[u][e] : make_float2(-INFINITY, 0.0f);
+        gm[u] = ml.x;
+        gl[u] = ml.y;
+    }
 #pragma unroll
     for (int lv = 4; lv <= 6; lv++) {
 #pragma unroll
         for (int u = 0; u < (64 >> lv); u++) {
+            const bool has_right = (2 * u + 1) * (1 << (lv - 1)) < n_splits;
+            const MergeOut mo = merge_pair(gv[2 * u], gm[2 * u], gl[2 * u], gv[2 * u + 1], gm[2 * u + 1], gl[2 * u + 1],
+                                           has_right);
             if (lv <= H && u * (1 << lv) < n_splits) {
-                const bool has_right = (2 * u + 1) * (1 << (lv - 1)) < n_splits;
-                gv[u] = has_right ? node_merge(gv[2 * u], gv[2 * u + 1], lv, u) : gv[2 * u];
+                gv[u] = mo.o;
+                gm[u] = mo.m;
+                gl[u] = mo.l;
             }
         }
     }
     // out = O / l and lse for a real row
-    const int rl = r, c4 = e4 % (D / 4);
-    if (rl >= rows_here) return;
-    const int rr = row0 + rl, jq = rr / p.group, hq = rr % p.group;
-    const long long qrow = (long long)qoff_s + jq;
+    const int c4 = e4 % (D / 4);
+    if (r >= rows_here) return;
+    const int rr = row0 + r, jq = rr / p.group, hq = rr % p.group;
+    int qoff = 0;
+    for (int i = 0; i < b; i++) qoff += min(max(__ldg(p.n_q_per_seq + i), 0), p.max_q);
+    const long long qrow = (long long)qoff + jq;
     if (qrow >= p.total_q) return;
-    const float* root = hp + (size_t)hidx(H, 0) * RPC * 4;
-    const float l = root[rc * 4 + 1], m = root[rc * 4 + 0];
+    const float l = gl[0], m = gm[0];
     float4 o = gv[0];
     o.x = __fdiv_rn(o.x, l);
     o.y = __fdiv_rn(o.y, l);

@@ -40,10 +40,8 @@ int rows_class_for(int head_dim, int rows_total);
 mq_decode_config default_config(int head_dim, int cls);
 bool config_valid(const mq_decode_config& c);
 DecodePlan plan_decode(const mq_cache* c, int n_seqs, int n_q_heads, int max_q, int max_seq_len);
-// Bytes of the CTA partials of one plan; bytes of the counter region at the front of a
-// workspace of workspace_bytes (1/512 of it, rounded up to 256).
+// Bytes of the CTA partials of one plan (the decode workspace).
 size_t partial_bytes(const mq_cache* c, int n_seqs, const DecodePlan& pl);
-size_t counter_bytes(size_t workspace_bytes);
 cudaError_t ensure_decode_smem(int device, int head_dim, int rows, size_t smem);
 mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void* q, mq_dtype q_dtype, int n_seqs,
                              int n_q_heads, int total_q, int max_q, const int32_t* block_table, int max_blocks,

@@ -42,7 +42,6 @@ struct DecodeParams {
     float* out;
     float* lse;
     // workspace
-    unsigned* counters;  // [n_seqs][n_kv_heads][n_rb]
     float* part_ml;      // [n_seqs][n_kv_heads][n_rb][split_stride][rows][2]
     float* part_o;       // [n_seqs][n_kv_heads][n_rb][split_stride][rows][D]
     int split_stride;    // partial slots per unit (>= the splits of any unit)

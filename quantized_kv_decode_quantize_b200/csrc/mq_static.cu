@@ -26,9 +26,8 @@ namespace {
 constexpr size_t kScratchBytes = MQ_DECODE_STATIC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
 
-// The scratch itself (one copy per device).  Its front holds the split counters that
-// must be zero when a launch starts; the rest holds CTA partials, written before they
-// are read.
+// The scratch itself (one copy per device): the CTA partials of the split reduction,
+// each written before it is read, so nothing has to start at zero.
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 std::mutex g_scratch_mu;
@@ -64,16 +63,6 @@ extern "C" mq_status mq_decode_attn_static(const mq_cache* c, const void* q, mq_
     void* scratch = nullptr;
     const mq_status st = scratch_address(c->device, &scratch);
     if (st != MQ_OK) return st;
-    if (need > 0) {
-        // The counters of this shape must start at zero.  A completed call leaves them
-        // zero, but one that stopped early (MQ_ERR_DEVICE) may not have, so they are
-        // cleared on the caller's stream before every launch.
-        const int G = n_q_heads / c->n_kv_heads;
-        const size_t max_units = (size_t)n_seqs * c->n_kv_heads * (size_t)((G * max_q_per_seq + 7) / 8);
-        if (cudaMemsetAsync(scratch, 0, max_units * sizeof(unsigned), reinterpret_cast<cudaStream_t>(stream)) !=
-            cudaSuccess)
-            return MQ_ERR_CUDA;
-    }
     return mq_decode_attn(c, q, q_dtype, n_seqs, n_q_heads, total_q, max_q_per_seq, max_seq_len, block_table,
                           max_blocks_per_seq, seq_lens, n_q_per_seq, softmax_scale, out, lse, scratch, kScratchBytes,
                           stream);

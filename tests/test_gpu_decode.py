@@ -179,13 +179,14 @@ def test_every_split_count_within_tolerance(sps):
     _check(case)
 
 
-def test_repeated_calls_reuse_workspace():
-    """The counter region returns to zero: many calls on one workspace agree."""
+def test_workspace_needs_no_initialization():
+    """A workspace full of garbage gives the same bytes as a zeroed one, call after call."""
     case = GpuCase(wl.reduced("verify"))
     ref = case.decode()[0].clone()
-    for _ in range(20):
+    case.ws.fill_(0xFF)
+    for _ in range(5):
         assert torch.equal(case.decode()[0], ref)
-    assert int(case.ws[:64].count_nonzero()) == 0
+    assert case.status() == mq.MQ_OK
 
 
 def test_bad_sequence_is_flagged_not_faulted():
