@@ -64,6 +64,9 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     constexpr int CPL = D / 32;          // channels per lane
     constexpr int LPG = 32 / CPL;        // lanes per 32-channel V group
     const int lane = threadIdx.x & 31;
+    // a decode launched after this append may start its set-up now; it waits for this
+    // grid (griddepcontrol.wait) before it reads any page
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const long long item = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     if (item >= (long long)p.n_tokens * p.n_kv_heads) return;
     const int tok = (int)(item / p.n_kv_heads), h = (int)(item % p.n_kv_heads);

@@ -385,6 +385,11 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
 
     if (warp == 0) {
         // ================= TMA producer =================
+        // The kernel is a programmatic dependent launch: a preceding kernel that allows it
+        // (the append of this step) may still be writing pages.  Wait for it to complete
+        // before the first page is read; everything before this point reads only the
+        // launch's inputs, which no such kernel writes.
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         const uint64_t policy = l2_evict_first_policy();
         // block-table entries of chunk i (lanes < 8), loaded one chunk ahead
         auto bt_load = [&](int i) -> int {
@@ -935,8 +940,17 @@ cudaError_t decode_prepare(int head_dim, int rows, size_t smem) {
 // dependent launch on the same stream.
 template <int D, int ROWS>
 static cudaError_t launch_pair(const DecodeParams& p, dim3 grid, size_t smem, int max_splits, cudaStream_t st) {
-    decode_kernel<D, ROWS><<<grid, dim3((unsigned)kThreads), smem, st>>>(p);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t dc{};
+    dc.gridDim = grid;
+    dc.blockDim = dim3((unsigned)kThreads);
+    dc.dynamicSmemBytes = smem;
+    dc.stream = st;
+    dc.attrs = pdl;
+    dc.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&dc, decode_kernel<D, ROWS>, p);
     if (e != cudaSuccess || max_splits <= 1) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)((ROWS * D / 4 + 127) / 128), grid.y, grid.z);
