@@ -204,6 +204,12 @@ mq_status mq_kv_append(mq_cache* cache, const void* k, const void* v, mq_dtype d
 size_t mq_decode_workspace_bytes(const mq_cache* cache, int32_t n_seqs, int32_t n_q_heads, int32_t max_q_per_seq,
                                  int32_t max_seq_len);
 
+/* Number of kernels one mq_decode_attn call with these bounds launches (1 when no
+ * unit is split across CTAs, else 2: the decode kernel and the merge of the split
+ * partials); 0 for arguments the call would refuse. */
+int32_t mq_decode_kernel_count(const mq_cache* cache, int32_t n_seqs, int32_t n_q_heads, int32_t max_q_per_seq,
+                               int32_t max_seq_len);
+
 mq_status mq_decode_attn(const mq_cache* cache, const void* q, mq_dtype q_dtype, int32_t n_seqs, int32_t n_q_heads,
                          int32_t total_q, int32_t max_q_per_seq, int32_t max_seq_len, const int32_t* block_table,
                          int32_t max_blocks_per_seq, const int32_t* seq_lens, const int32_t* n_q_per_seq,

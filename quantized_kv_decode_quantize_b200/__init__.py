@@ -62,6 +62,7 @@ def _load():
         "mq_cache_destroy": ([P], ctypes.c_int),
         "mq_kv_append": ([P, P, P, ctypes.c_int, i32, i32, P, P, P, i32, P], ctypes.c_int),
         "mq_decode_workspace_bytes": ([P, i32, i32, i32, i32], sz),
+        "mq_decode_kernel_count": ([P, i32, i32, i32, i32], i32),
         "mq_decode_attn": ([P, P, ctypes.c_int, i32, i32, i32, i32, i32, P, i32, P, P, ctypes.c_float, P, P, P, sz, P],
                            ctypes.c_int),
         "mq_decode_attn_static": ([P, P, ctypes.c_int, i32, i32, i32, i32, i32, P, i32, P, P, ctypes.c_float, P, P,
@@ -142,6 +143,10 @@ def mq_kv_append(cache: int, k, v, dtype: int, n_seqs: int, n_tokens: int, cu_ne
 
 def mq_decode_workspace_bytes(cache: int, n_seqs: int, n_q_heads: int, max_q_per_seq: int, max_seq_len: int) -> int:
     return lib.mq_decode_workspace_bytes(cache, n_seqs, n_q_heads, max_q_per_seq, max_seq_len)
+
+
+def mq_decode_kernel_count(cache: int, n_seqs: int, n_q_heads: int, max_q_per_seq: int, max_seq_len: int) -> int:
+    return lib.mq_decode_kernel_count(cache, n_seqs, n_q_heads, max_q_per_seq, max_seq_len)
 
 
 def mq_decode_attn(cache: int, q, q_dtype: int, n_seqs: int, n_q_heads: int, total_q: int, max_q_per_seq: int,

@@ -276,6 +276,13 @@ size_t mq_decode_workspace_bytes(const mq_cache* c, int32_t n_seqs, int32_t n_q_
     return part;
 }
 
+int32_t mq_decode_kernel_count(const mq_cache* c, int32_t n_seqs, int32_t n_q_heads, int32_t max_q_per_seq,
+                               int32_t max_seq_len) {
+    if (c == nullptr || mq_decode_workspace_bytes(c, n_seqs, n_q_heads, max_q_per_seq, max_seq_len) == 0) return 0;
+    const DecodePlan pl = plan_decode(c, n_seqs, n_q_heads, max_q_per_seq, max_seq_len);
+    return pl.max_splits > 1 ? 2 : 1;
+}
+
 mq_status mq_decode_attn(const mq_cache* c, const void* q, mq_dtype q_dtype, int32_t n_seqs, int32_t n_q_heads,
                          int32_t total_q, int32_t max_q_per_seq, int32_t max_seq_len, const int32_t* block_table,
                          int32_t max_blocks_per_seq, const int32_t* seq_lens, const int32_t* n_q_per_seq,
