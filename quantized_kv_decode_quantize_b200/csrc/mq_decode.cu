@@ -528,14 +528,27 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
         const int tp = t / 16, ttg = (t / 8) & 1, tt = t & 7;
         const uint32_t wb0 = smem_u32(smem + S.wbuf);
         float* xch = reinterpret_cast<float*>(smem + S.xch);
-        float crow[ROWS], M[ROWS];
-        int lim[ROWS];
+        // Row factors and visibility limits: registers for the 8-row class, shared memory
+        // (broadcast reads) for the larger ones, which would otherwise run out of registers.
+        constexpr bool kRowRegs = ROWS <= 8;
+        float crow_r[kRowRegs ? ROWS : 1], M[ROWS];
+        int lim_r[kRowRegs ? ROWS : 1];
 #pragma unroll
         for (int r = 0; r < ROWS; r++) {
-            crow[r] = crow_s[r];
-            lim[r] = lim_s[r];
+            if constexpr (kRowRegs) {
+                crow_r[r] = crow_s[r];
+                lim_r[r] = lim_s[r];
+            }
             M[r] = -INFINITY;
         }
+        auto crow = [&](int r) -> float {
+            if constexpr (kRowRegs) return crow_r[r];
+            else return crow_s[r];
+        };
+        auto lim = [&](int r) -> int {
+            if constexpr (kRowRegs) return lim_r[r];
+            else return lim_s[r];
+        };
         float Mlane = -INFINITY;   // M of row `lane` (lanes < ROWS)
         const int lim_min = L - nq + row0 / p.group + 1;   // smallest limit of the real rows
         const int nrg4 = (rows_here + 3) / 4;              // 4-row groups holding real rows
@@ -595,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
                         for (int e = 0; e < 4; e++) {
                             const int x = (int)a2[e] * 256 + (int)a1[e];   // exact: |x| < 2^30
                             const float sc = __fmaf_rn((float)x, 256.0f, (float)(int)a0[e]);
-                            z[4 * rg + e] = __fmul_rn(__fmul_rn(sc, crow[4 * rg + e]), sk);
+                            z[4 * rg + e] = __fmul_rn(__fmul_rn(sc, crow(4 * rg + e)), sk);
                         }
                     } else {
 #pragma unroll
@@ -610,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
                     const int tok = c * kChunkTokens + t;
 #pragma unroll
                     for (int r = 0; r < ROWS; r++)
-                        if (my_bad || tok >= lim[r]) z[r] = -INFINITY;
+                        if (my_bad || tok >= lim(r)) z[r] = -INFINITY;
                 }
                 // ---- chunk row maxima over the 128 tokens ----
 #pragma unroll
@@ -656,11 +669,8 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
             }
             if (ok && i >= T::NWB && !wait_warp(pv_bar(i - T::NWB), pv_par(i - T::NWB))) ok = false;
             if (ok) {
-                // ---- weights of the real rows: p = 2^(z - M), W_g = p * s_v[g] (fp16) ----
-                float pw[ROWS];
-#pragma unroll
-                for (int r = 0; r < ROWS; r++)
-                    pw[r] = (r >= rows_here || z[r] == -INFINITY) ? 0.0f : ex2(__fsub_rn(z[r], M[r]));
+                // ---- weights of the real rows: p = 2^(z - M), W_g = p * s_v[g] (fp16), formed
+                // 8 rows at a time next to their stores ----
                 const uint32_t wrow = wb0 + (uint32_t)(wb * T::WBYTES + (t / 8) * T::LBO_W + (t % 8) * 16);
                 auto store_group = [&](uint32_t a, const float* w, bool two) {
                     // 8 rows of one 8-column group (two = both 4-row halves hold real rows)
@@ -675,19 +685,25 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
                 for (int rg8 = 0; rg8 < ROWS / 8; rg8++) {
                     if (2 * rg8 >= nrg4) continue;
                     const bool two = 2 * rg8 + 1 < nrg4;
+                    float pw[8];
+#pragma unroll
+                    for (int e = 0; e < 8; e++) {
+                        const int r = 8 * rg8 + e;
+                        pw[e] = (r >= rows_here || z[r] == -INFINITY) ? 0.0f : ex2(__fsub_rn(z[r], M[r]));
+                    }
 #pragma unroll
                     for (int g = 0; g < T::G; g++) {
                         float w[8];
 #pragma unroll
                         for (int e = 0; e < 8; e++) {
-                            const float pv = pw[8 * rg8 + e];
+                            const float pv = pw[e];
                             const float wv = __fmul_rn(pv, sv[g]);
                             // masked tokens may carry unwritten (non-finite) scales
                             w[e] = (!clean && pv == 0.0f) ? 0.0f : wv;
                         }
                         store_group(wrow + (uint32_t)(((g * ROWS + 8 * rg8) / 8) * 128), w, two);
                     }
-                    store_group(wrow + (uint32_t)(((T::G * ROWS + 8 * rg8) / 8) * 128), pw + 8 * rg8, two);
+                    store_group(wrow + (uint32_t)(((T::G * ROWS + 8 * rg8) / 8) * 128), pw, two);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
