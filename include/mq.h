@@ -11,6 +11,10 @@
  *                   sequence and merged by log-sum-exp
  *   mq_tune         on-device choice of the decode launch shape under a
  *                   wall-clock budget, accepting only bit-identical candidates
+ *                   (or, on request, candidates within alpha times the output
+ *                   movement of a one-step perturbation of the stored cache),
+ *                   with the choice kept in a store file keyed by the device,
+ *                   driver, toolchain and library build
  *
  * Where the operations come from.  The blog.123qwe.co.kr deep dive on
  * magnitudedev/magnitude, section 5 ("core mechanism 3: speculative decoding,
@@ -21,9 +25,12 @@
  * Its section 3 ("core mechanism 1: the 60 s first-load tuner") describes the
  * tuner: a 60 s wall-clock budget, candidates measured on the device, a cost
  * summed over serving shapes (4k/64k decode, verification width) weighted by
- * their time at the default configuration, and timing passes sized beyond the
- * last-level cache.  The paper-digest.app summary ("Core Mechanics") adds that
- * the tuner keeps only configurations that do not change model output.
+ * their time at the default configuration, timing passes sized beyond the
+ * last-level cache, and results stored and reused by later loads until the
+ * driver or toolchain identity changes.  Its section 4 ("core mechanism 2: the
+ * precision system") gives the alpha = 8 admission rule.  The paper-digest.app
+ * summary ("Core Mechanics") adds that the tuner keeps only configurations that
+ * do not change model output.
  *
  * The codec's arithmetic is this library's fixed reading (the pages name the
  * codec only):
@@ -71,7 +78,8 @@ typedef enum mq_status {
     MQ_ERR_WORKSPACE = 4,       /* workspace null, too small or misaligned                      */
     MQ_ERR_CUDA = 5,            /* a CUDA runtime call or kernel launch failed                   */
     MQ_ERR_DEVICE = 6,          /* a kernel flagged a bad block id/position/length or a timeout  */
-    MQ_TUNE_BUDGET_EXHAUSTED = 7 /* warning: the tuner's budget ran out before every candidate    */
+    MQ_TUNE_BUDGET_EXHAUSTED = 7, /* warning: the tuner's budget ran out before every candidate   */
+    MQ_ERR_IO = 8               /* the tuning store could not be written                        */
 } mq_status;
 
 typedef enum mq_dtype { MQ_F32 = 0, MQ_BF16 = 1, MQ_F16 = 2 } mq_dtype;
@@ -193,7 +201,8 @@ mq_status mq_kv_append(mq_cache* cache, const void* k, const void* v, mq_dtype d
  * Query token j of sequence b (0-based) attends to positions 0 .. L_b - n_b + j:
  * the history plus drafts 0..j (causal among the drafts).  q-head h reads
  * kv-head h / (n_q_heads / n_kv_heads).  The result is bit-identical for every
- * launch configuration the tuner may choose (see mq_tune).
+ * launch configuration the tuner may choose under its default admission rule
+ * (see mq_tune).
  * Errors: INVALID_ARG (null pointers, n_seqs < 1 or > 65535, n_q_heads not a
  * multiple of n_kv_heads, total_q < 1, max_q_per_seq < 1, max_seq_len <
  * max_q_per_seq, a non-finite softmax_scale, out not 16-byte aligned), UNSUPPORTED
@@ -275,28 +284,49 @@ typedef struct mq_decode_config {
 mq_status mq_get_decode_config(const mq_cache* cache, int32_t rows_class, mq_decode_config* cfg);
 mq_status mq_set_decode_config(mq_cache* cache, int32_t rows_class, const mq_decode_config* cfg);
 
+/* Admission rules for tuner candidates. */
+#define MQ_ADMIT_BIT_IDENTICAL 0  /* out and lse bytes equal the default configuration's       */
+#define MQ_ADMIT_ALPHA 1          /* every out and lse point within alpha x storage noise       */
+
 typedef struct mq_tune_params {
     double budget_s;        /* wall-clock budget for everything the tuner does (e.g. 60) */
     int32_t n_q_heads;      /* query heads of the model the cache serves                */
     const char* log_path;   /* host path for the JSON evidence log, or NULL             */
+    const char* store_path; /* host path of the persistent tuning store, or NULL        */
+    int32_t admission;      /* MQ_ADMIT_BIT_IDENTICAL (0) or MQ_ADMIT_ALPHA             */
+    double alpha;           /* the alpha of MQ_ADMIT_ALPHA; <= 0 selects 8              */
 } mq_tune_params;
 
 typedef struct mq_tune_result {
     mq_decode_config chosen[3];   /* per rows_class (unchanged if that class was not probed) */
     double cost;                  /* weighted cost of the chosen set (1.0 = the defaults)   */
     int32_t n_tried;              /* candidates measured                                      */
-    int32_t n_rejected;           /* candidates rejected as not bit-identical                 */
+    int32_t n_rejected;           /* candidates the admission rule rejected                   */
     int32_t n_skipped;            /* candidates not reached inside the budget                 */
     double elapsed_s;
+    int32_t from_store;           /* 1: the choice was read from the store, nothing measured */
 } mq_tune_result;
 
 /* On-device tuner.  Within params->budget_s of wall-clock time (allocation,
  * probe set-up, every measurement included) it measures the candidate launch
  * configurations on three probe shapes built from the cache's geometry and
  * params->n_q_heads — decode at 4K and at 64K tokens, and verification of 8
- * drafts at 64K — rejects any candidate whose output bytes differ from the
- * default configuration's, and keeps the candidate set with the lowest cost
+ * drafts at 64K — admits candidates by params->admission, and keeps the admitted
+ * candidate set with the lowest cost
  *     cost(c) = sum_p median_time(c, p) / median_time(default, p).
+ * The default is the configuration the cache holds when mq_tune is called.
+ *
+ * Admission.  MQ_ADMIT_BIT_IDENTICAL keeps a candidate only if its out and lse
+ * bytes equal the default's on every probe.  MQ_ADMIT_ALPHA keeps it if, at every
+ * point i of out and lse on every probe,
+ *     |candidate_i - default_i| <= alpha * noise_i,
+ * where noise_i, the storage-resolution noise, is how far the default output
+ * moves at i when every stored element of the probe cache moves by one step of
+ * its format (int8 K code and int4 V code by one code, fp16 scales by one unit in
+ * the last place, each in a seeded random direction); noise_i is the larger of
+ * two such perturbations.  The rule uses the stored data and its declared types
+ * only.  A point whose noise is zero must match exactly.
+ *
  * Timed launches read probe caches that together exceed twice the L2 size, so
  * no launch finds its data warm in L2.  The probes use their own device
  * buffers (allocated and freed here; the cache's pool is not touched).  The
@@ -304,8 +334,42 @@ typedef struct mq_tune_result {
  * MQ_TUNE_BUDGET_EXHAUSTED when the budget ended the search early (the best
  * configuration measured so far is kept; the defaults if none).  Synchronizes
  * the device.  Writes a JSON record of every candidate to params->log_path
- * when it is not NULL. */
+ * when it is not NULL.
+ *
+ * Persistence.  With params->store_path set, the tuner first looks up the
+ * identity string of mq_tune_identity() in that store: on a match it applies the
+ * stored choice to the cache, measures nothing, sets result->from_store and
+ * returns MQ_OK.  Otherwise it searches and, when the search completed (MQ_OK),
+ * writes its choice under that identity (a search the budget cut short is not
+ * stored, so a later call with more budget searches again); a store that cannot
+ * be written gives MQ_ERR_IO after the choice has been applied. */
 mq_status mq_tune(mq_cache* cache, const mq_tune_params* params, mq_tune_result* result);
+
+/* The identity a tuning choice is stored under: the GPU's name, SM count and
+ * compute capability, the driver version, the CUDA runtime the library was built
+ * with, the library version and source build id, the cache geometry (head_dim,
+ * n_kv_heads), params->n_q_heads, the admission rule (with alpha), and the
+ * configurations the cache holds (the defaults the candidates are compared with).
+ * Any change to one of them gives another identity, so the choice is searched
+ * again.  Written to buf as a NUL-terminated string of printable characters
+ * without tabs; INVALID_ARG if buf_len is too small (512 bytes always suffice).
+ * Queries the cache's device; launches nothing. */
+mq_status mq_tune_identity(const mq_cache* cache, const mq_tune_params* params, char* buf, size_t buf_len);
+
+/* The tuning store: a text file, one choice per line,
+ *     <identity> TAB <r0>:<s0> <r1>:<s1> <r2>:<s2> TAB <cost>
+ * (ring_stages:splits_per_sm of rows_class 0, 1, 2), after a header line starting
+ * with '#'.  Host-only file access; no GPU is needed.
+ * mq_tune_store_get: *found = 1 and chosen[0..2] set when a well-formed line with
+ *   this identity exists (a line whose configurations are out of range counts as
+ *   absent); *found = 0 otherwise, a missing or unreadable file included.
+ * mq_tune_store_put: writes the file with this identity's line replaced (or
+ *   added), every other line kept, through a temporary file in the same directory
+ *   renamed over the store, so readers never see a partial file.  IO when the file
+ *   cannot be written; INVALID_ARG for an identity holding a tab or newline, or an
+ *   out-of-range configuration. */
+mq_status mq_tune_store_get(const char* path, const char* identity, mq_decode_config chosen[3], int32_t* found);
+mq_status mq_tune_store_put(const char* path, const char* identity, const mq_decode_config chosen[3], double cost);
 
 /* ---------------------------------------------------------------------------
  * Diagnostics

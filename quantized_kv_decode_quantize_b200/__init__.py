@@ -17,6 +17,8 @@ LIB_PATH = os.path.join(_HERE, "libmq.so")
 
 MQ_OK, MQ_ERR_INVALID_ARG, MQ_ERR_UNSUPPORTED, MQ_ERR_CAPACITY = 0, 1, 2, 3
 MQ_ERR_WORKSPACE, MQ_ERR_CUDA, MQ_ERR_DEVICE, MQ_TUNE_BUDGET_EXHAUSTED = 4, 5, 6, 7
+MQ_ERR_IO = 8
+MQ_ADMIT_BIT_IDENTICAL, MQ_ADMIT_ALPHA = 0, 1
 MQ_F32, MQ_BF16, MQ_F16 = 0, 1, 2
 MQ_PAGE_TOKENS = 16
 
@@ -34,12 +36,14 @@ class mq_decode_config(ctypes.Structure):
 
 
 class mq_tune_params(ctypes.Structure):
-    _fields_ = [("budget_s", ctypes.c_double), ("n_q_heads", ctypes.c_int32), ("log_path", ctypes.c_char_p)]
+    _fields_ = [("budget_s", ctypes.c_double), ("n_q_heads", ctypes.c_int32), ("log_path", ctypes.c_char_p),
+                ("store_path", ctypes.c_char_p), ("admission", ctypes.c_int32), ("alpha", ctypes.c_double)]
 
 
 class mq_tune_result(ctypes.Structure):
     _fields_ = [("chosen", mq_decode_config * 3), ("cost", ctypes.c_double), ("n_tried", ctypes.c_int32),
-                ("n_rejected", ctypes.c_int32), ("n_skipped", ctypes.c_int32), ("elapsed_s", ctypes.c_double)]
+                ("n_rejected", ctypes.c_int32), ("n_skipped", ctypes.c_int32), ("elapsed_s", ctypes.c_double),
+                ("from_store", ctypes.c_int32)]
 
 
 class MQError(RuntimeError):
@@ -70,6 +74,11 @@ def _load():
         "mq_get_decode_config": ([P, i32, ctypes.POINTER(mq_decode_config)], ctypes.c_int),
         "mq_set_decode_config": ([P, i32, ctypes.POINTER(mq_decode_config)], ctypes.c_int),
         "mq_tune": ([P, ctypes.POINTER(mq_tune_params), ctypes.POINTER(mq_tune_result)], ctypes.c_int),
+        "mq_tune_identity": ([P, ctypes.POINTER(mq_tune_params), ctypes.c_char_p, sz], ctypes.c_int),
+        "mq_tune_store_get": ([ctypes.c_char_p, ctypes.c_char_p, ctypes.POINTER(mq_decode_config),
+                               ctypes.POINTER(i32)], ctypes.c_int),
+        "mq_tune_store_put": ([ctypes.c_char_p, ctypes.c_char_p, ctypes.POINTER(mq_decode_config), ctypes.c_double],
+                              ctypes.c_int),
         "mq_device_status": ([P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
@@ -178,13 +187,40 @@ def mq_set_decode_config(cache: int, rows_class: int, ring_stages: int, splits_p
     _check(lib.mq_set_decode_config(cache, rows_class, ctypes.byref(c)), "mq_set_decode_config")
 
 
-def mq_tune(cache: int, budget_s: float, n_q_heads: int, log_path: str | None = None) -> dict:
-    p = mq_tune_params(float(budget_s), n_q_heads, log_path.encode() if log_path else None)
+def _tune_params(budget_s, n_q_heads, log_path=None, store_path=None, admission=MQ_ADMIT_BIT_IDENTICAL, alpha=0.0):
+    return mq_tune_params(float(budget_s), n_q_heads, log_path.encode() if log_path else None,
+                          store_path.encode() if store_path else None, admission, float(alpha))
+
+
+def mq_tune(cache: int, budget_s: float, n_q_heads: int, log_path: str | None = None, store_path: str | None = None,
+            admission: int = MQ_ADMIT_BIT_IDENTICAL, alpha: float = 0.0) -> dict:
+    p = _tune_params(budget_s, n_q_heads, log_path, store_path, admission, alpha)
     r = mq_tune_result()
     st = _check(lib.mq_tune(cache, ctypes.byref(p), ctypes.byref(r)), "mq_tune",
                 ok=(MQ_OK, MQ_TUNE_BUDGET_EXHAUSTED))
     return {"status": st, "chosen": [r.chosen[i].as_tuple() for i in range(3)], "cost": r.cost,
-            "n_tried": r.n_tried, "n_rejected": r.n_rejected, "n_skipped": r.n_skipped, "elapsed_s": r.elapsed_s}
+            "n_tried": r.n_tried, "n_rejected": r.n_rejected, "n_skipped": r.n_skipped, "elapsed_s": r.elapsed_s,
+            "from_store": bool(r.from_store)}
+
+
+def mq_tune_identity(cache: int, n_q_heads: int, admission: int = MQ_ADMIT_BIT_IDENTICAL, alpha: float = 0.0) -> str:
+    p = _tune_params(0.0, n_q_heads, admission=admission, alpha=alpha)
+    buf = ctypes.create_string_buffer(512)
+    _check(lib.mq_tune_identity(cache, ctypes.byref(p), buf, len(buf)), "mq_tune_identity")
+    return buf.value.decode()
+
+
+def mq_tune_store_get(path: str, identity: str):
+    """The stored [(ring_stages, splits_per_sm)] * 3 for `identity`, or None."""
+    cfg = (mq_decode_config * 3)()
+    found = ctypes.c_int32(0)
+    _check(lib.mq_tune_store_get(path.encode(), identity.encode(), cfg, ctypes.byref(found)), "mq_tune_store_get")
+    return [cfg[i].as_tuple() for i in range(3)] if found.value else None
+
+
+def mq_tune_store_put(path: str, identity: str, chosen, cost: float) -> None:
+    cfg = (mq_decode_config * 3)(*[mq_decode_config(r, s) for r, s in chosen])
+    _check(lib.mq_tune_store_put(path.encode(), identity.encode(), cfg, float(cost)), "mq_tune_store_put")
 
 
 def mq_device_status(cache: int, stream=None) -> int:

@@ -11,6 +11,7 @@ fast-math: the quantizer relies on IEEE division and round-to-nearest-even.
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import shutil
 import subprocess
@@ -39,6 +40,18 @@ def _deps():
             + [os.path.abspath(__file__)])
 
 
+def build_id() -> str:
+    """First 16 hex digits of a SHA-256 over the library's sources (csrc/ and include/):
+    the library build part of the tuner's store identity."""
+    h = hashlib.sha256()
+    srcs = sorted(glob.glob(os.path.join(CSRC, "*")) + glob.glob(os.path.join(ROOT, "include", "*.h")))
+    for path in srcs:
+        h.update(os.path.basename(path).encode() + b"\0")
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True
@@ -51,9 +64,10 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     objs = []
+    bid = build_id()
     for src in sorted(glob.glob(os.path.join(CSRC, "*.cu"))):
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
-        cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
+        cmd = [nvcc(), *ARCH, *NVCC_FLAGS, f"-DMQ_BUILD_ID=\"{bid}\"", "-c", src, "-o", obj]
         if ptxas_info:
             cmd[1:1] = ["-Xptxas", "-v"]
         if verbose:

@@ -167,6 +167,7 @@ const char* mq_status_string(mq_status s) {
         case MQ_ERR_CUDA: return "CUDA error";
         case MQ_ERR_DEVICE: return "a kernel flagged bad input or a timed-out wait";
         case MQ_TUNE_BUDGET_EXHAUSTED: return "tuning budget exhausted before every candidate was measured";
+        case MQ_ERR_IO: return "the tuning store could not be written";
     }
     return "unknown status";
 }

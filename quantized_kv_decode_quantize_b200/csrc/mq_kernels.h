@@ -67,5 +67,13 @@ cudaError_t launch_fill_random(void* dst, int dtype, long long n, int head_dim, 
 cudaError_t launch_scribble(void* dst, size_t bytes, unsigned v, cudaStream_t st);
 // out[0] = 1 if a[i] != b[i] for some i < n32 (32-bit words), else unchanged.
 cudaError_t launch_compare(const uint32_t* a, const uint32_t* b, long long n32, unsigned* out, cudaStream_t st);
+// one format step of every stored element of n_pages pages (src -> dst, same layout)
+cudaError_t launch_perturb_pages(const void* src, void* dst, long long n_pages, int head_dim,
+                                 unsigned long long seed, cudaStream_t st);
+// noise[i] = max(noise[i], |moved[i] - ref[i]|)
+cudaError_t launch_noise_max(const float* moved, const float* ref, float* noise, long long n, cudaStream_t st);
+// out[0] |= (some |cand - ref| > alpha * noise); out[1] = max ratio as float bits
+cudaError_t launch_alpha_check(const float* cand, const float* ref, const float* noise, long long n, float alpha,
+                               unsigned* out, cudaStream_t st);
 
 }  // namespace mq

@@ -11,12 +11,22 @@
 // last-level cache (here: rotating probe caches that together exceed twice the L2
 // size), so no launch finds its data warm; structurally different candidates are
 // tried before refinements of one; a candidate is started only when the budget
-// left covers its estimated cost.  Admission follows the paper-digest.app summary
-// ("Core Mechanics": only configurations that do not change the output are
-// kept): a candidate's out and lse bytes must equal the default's exactly.
+// left covers its estimated cost; a completed search is stored and reused by the
+// next load with the same device, driver, toolchain and library identity
+// (mq_tune_store.cu).
+//
+// Admission, by default, follows the paper-digest.app summary ("Core Mechanics":
+// only configurations that do not change the output are kept): a candidate's out
+// and lse bytes must equal the default's exactly.  On request it follows the
+// deep dive's section 4 ("core mechanism 2: the precision system") instead, with
+// alpha = 8: at every checked point the candidate may move the default's result by
+// at most alpha times what storage-resolution noise moves it, that noise being the
+// movement of the default output when every stored element of the probe cache
+// takes one step of its format (the larger of two seeded perturbations).
 #include <algorithm>
 #include <chrono>
 #include <cstdio>
+#include <cstring>
 #include <string>
 #include <vector>
 
@@ -40,8 +50,21 @@ struct Cand {
     mq_decode_config cfg;
     int cls;
     double t[3] = {0, 0, 0};
+    double max_ratio = 0;   // largest |candidate - default| / noise over checked points (alpha rule)
     bool identical = true, measured = false, rejected = false, valid = true;
 };
+
+// summary of one probe's storage-resolution noise over its out points
+struct NoiseStats {
+    double min = 0, median = 0, max = 0;
+    long long zero_points = 0;
+};
+
+void json_double(FILE* f, double v) {
+    if (v != v) std::fprintf(f, "NaN");
+    else if (v > 1e300) std::fprintf(f, "Infinity");
+    else std::fprintf(f, "%.6g", v);
+}
 
 double seconds_since(Clock::time_point t0) {
     return std::chrono::duration<double>(Clock::now() - t0).count();
@@ -61,12 +84,16 @@ struct Buffers {
     float* out = nullptr;
     float* lse = nullptr;
     void* ws = nullptr;
-    unsigned* flag = nullptr;
+    unsigned* flag = nullptr;    // [0] bytes differ, [1] alpha rule broken, [2] max ratio (float bits)
+    void* pert = nullptr;        // one perturbed probe cache copy (alpha rule)
+    float* noise_out[3] = {nullptr, nullptr, nullptr};
+    float* noise_lse[3] = {nullptr, nullptr, nullptr};
     cudaEvent_t ev[2] = {nullptr, nullptr};
     cudaStream_t st = nullptr;
     ~Buffers() {
-        void* ptrs[] = {pool, bt, lens, nq, cu, start, kv, q, out, lse, ws, flag,
-                        out_ref[0], out_ref[1], out_ref[2], lse_ref[0], lse_ref[1], lse_ref[2]};
+        void* ptrs[] = {pool, bt, lens, nq, cu, start, kv, q, out, lse, ws, flag, pert,
+                        out_ref[0], out_ref[1], out_ref[2], lse_ref[0], lse_ref[1], lse_ref[2],
+                        noise_out[0], noise_out[1], noise_out[2], noise_lse[0], noise_lse[1], noise_lse[2]};
         for (void* p : ptrs)
             if (p) cudaFree(p);
         for (auto e : ev)
@@ -85,11 +112,45 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
     if (cache == nullptr || prm == nullptr || res == nullptr) return MQ_ERR_INVALID_ARG;
     if (!(prm->budget_s >= 0.0) || prm->n_q_heads < 1 || prm->n_q_heads % cache->n_kv_heads != 0)
         return MQ_ERR_INVALID_ARG;
+    if (prm->admission != MQ_ADMIT_BIT_IDENTICAL && prm->admission != MQ_ADMIT_ALPHA) return MQ_ERR_INVALID_ARG;
+    if (!(prm->alpha <= 0.0 || prm->alpha < 1e30)) return MQ_ERR_INVALID_ARG;   // NaN or absurd alpha
+    const bool alpha_rule = prm->admission == MQ_ADMIT_ALPHA;
+    const double alpha = prm->alpha > 0.0 ? prm->alpha : 8.0;
     const int Hkv = cache->n_kv_heads, D = cache->head_dim, Hq = prm->n_q_heads, G = Hq / Hkv;
     if (G > 64) return MQ_ERR_UNSUPPORTED;
     *res = mq_tune_result{};
     for (int k = 0; k < 3; k++) res->chosen[k] = cache->cfg[k];
     res->cost = 1.0;
+
+    // ---- the store: a stored choice for this identity is applied without measuring ----
+    char identity[512] = {0};
+    if (prm->store_path != nullptr) {
+        mq_status s = mq_tune_identity(cache, prm, identity, sizeof identity);
+        if (s != MQ_OK) return s;
+        mq_decode_config got[3];
+        int32_t found = 0;
+        if ((s = mq_tune_store_get(prm->store_path, identity, got, &found)) != MQ_OK) return s;
+        if (found) {
+            for (int k = 0; k < 3; k++) cache->cfg[k] = res->chosen[k] = got[k];
+            res->from_store = 1;
+            res->elapsed_s = seconds_since(t0);
+            if (prm->log_path != nullptr) {
+                FILE* f = std::fopen(prm->log_path, "w");
+                if (f != nullptr) {
+                    std::fprintf(f, "{\n  \"from_store\": true, \"identity\": \"%s\", \"elapsed_s\": %.6f,\n", identity,
+                                 res->elapsed_s);
+                    std::fprintf(f, "  \"chosen\": [");
+                    for (int cls = 0; cls < 3; cls++)
+                        std::fprintf(f, "%s{\"rows_class\": %d, \"ring_stages\": %d, \"splits_per_sm\": %d}",
+                                     cls ? ", " : "", cls, got[cls].ring_stages, got[cls].splits_per_sm);
+                    std::fprintf(f, "],\n  \"n_tried\": 0\n}\n");
+                    std::fclose(f);
+                }
+            }
+            return MQ_OK;
+        }
+    }
+
     if (prm->budget_s < 0.5) {   // not even the probe set-up fits: keep the defaults
         res->elapsed_s = seconds_since(t0);
         return MQ_TUNE_BUDGET_EXHAUSTED;
@@ -122,7 +183,7 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         !ck(cudaMalloc(&B.cu, sizeof(int32_t) * 2)) || !ck(cudaMalloc(&B.start, sizeof(int32_t))) ||
         !ck(cudaMalloc(&B.kv, kv_elems * 2 * 2)) || !ck(cudaMalloc(&B.q, (size_t)8 * Hq * D * 2)) ||
         !ck(cudaMalloc(&B.out, (size_t)8 * Hq * D * 4)) || !ck(cudaMalloc(&B.lse, (size_t)8 * Hq * 4)) ||
-        !ck(cudaMalloc(&B.ws, ws_bytes)) || !ck(cudaMalloc(&B.flag, sizeof(unsigned))))
+        !ck(cudaMalloc(&B.ws, ws_bytes)) || !ck(cudaMalloc(&B.flag, 3 * sizeof(unsigned))))
         return MQ_ERR_CUDA;
     for (int p = 0; p < P; p++)
         if (!ck(cudaMalloc(&B.out_ref[p], (size_t)8 * Hq * D * 4)) || !ck(cudaMalloc(&B.lse_ref[p], (size_t)8 * Hq * 4)))
@@ -181,12 +242,19 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
 
     int rot = 0;
     // one launch of probe p with configuration cfg on copy `rot`; returns status
-    auto launch = [&](int p, const mq_decode_config& cfg, float* out, float* lse) -> mq_status {
+    // (with `pool` set: on that single copy instead, e.g. the perturbed one)
+    auto launch = [&](int p, const mq_decode_config& cfg, float* out, float* lse, void* pool = nullptr) -> mq_status {
         mq_cache pc = probe_cache;
         pc.cfg[probes[p].cls] = cfg;
-        const DecodePlan pl = plan_decode(&pc, 1, Hq, probes[p].n_q, probes[p].seq_len);
         const int32_t* bt = B.bt + (size_t)(rot % n_copies) * blocks_per_copy;
         rot++;
+        if (pool != nullptr) {
+            pc.pool = pool;
+            pc.pool_bytes = copy_bytes;
+            pc.n_blocks = blocks_per_copy;
+            bt = B.bt;   // the first copy's table: blocks 0 .. blocks_per_copy - 1
+        }
+        const DecodePlan pl = plan_decode(&pc, 1, Hq, probes[p].n_q, probes[p].seq_len);
         return launch_decode_plan(&pc, pl, B.q, MQ_BF16, 1, Hq, probes[p].n_q, probes[p].n_q, bt, blocks_per_copy,
                                   B.lens + p, B.nq + p, 1.0f / std::sqrt((float)D), out, lse, B.ws, ws_bytes, B.st);
     };
@@ -216,6 +284,42 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         if ((s = time_probe(p, cache->cfg[probes[p].cls], &probes[p].t_default)) != MQ_OK) return s;
     }
     if (!ck(cudaStreamSynchronize(B.st))) return MQ_ERR_CUDA;
+
+    // ---- storage-resolution noise of the default output (alpha rule only) ----
+    NoiseStats nstat[3];
+    if (alpha_rule) {
+        if (!ck(cudaMalloc(&B.pert, copy_bytes))) return MQ_ERR_CUDA;
+        for (int p = 0; p < P; p++) {
+            const size_t n_out = (size_t)probes[p].n_q * Hq * D, n_lse = (size_t)probes[p].n_q * Hq;
+            if (!ck(cudaMalloc(&B.noise_out[p], n_out * 4)) || !ck(cudaMalloc(&B.noise_lse[p], n_lse * 4)) ||
+                !ck(cudaMemsetAsync(B.noise_out[p], 0, n_out * 4, B.st)) ||
+                !ck(cudaMemsetAsync(B.noise_lse[p], 0, n_lse * 4, B.st)))
+                return MQ_ERR_CUDA;
+        }
+        const long long n_pages = (long long)blocks_per_copy * Hkv;
+        for (unsigned long long seed : {0x5354455031ull, 0x5354455032ull}) {
+            if (!ck(launch_perturb_pages(B.pool, B.pert, n_pages, D, seed, B.st))) return MQ_ERR_CUDA;
+            for (int p = 0; p < P; p++) {
+                const long long n_out = (long long)probes[p].n_q * Hq * D, n_lse = (long long)probes[p].n_q * Hq;
+                mq_status s = launch(p, cache->cfg[probes[p].cls], B.out, B.lse, B.pert);
+                if (s != MQ_OK) return s;
+                if (!ck(launch_noise_max(B.out, B.out_ref[p], B.noise_out[p], n_out, B.st)) ||
+                    !ck(launch_noise_max(B.lse, B.lse_ref[p], B.noise_lse[p], n_lse, B.st)))
+                    return MQ_ERR_CUDA;
+            }
+        }
+        for (int p = 0; p < P; p++) {
+            std::vector<float> h((size_t)probes[p].n_q * Hq * D);
+            if (!ck(cudaMemcpyAsync(h.data(), B.noise_out[p], h.size() * 4, cudaMemcpyDeviceToHost, B.st)) ||
+                !ck(cudaStreamSynchronize(B.st)))
+                return MQ_ERR_CUDA;
+            for (float v : h) nstat[p].zero_points += v == 0.0f;
+            std::sort(h.begin(), h.end());
+            nstat[p].min = h.front();
+            nstat[p].median = h[h.size() / 2];
+            nstat[p].max = h.back();
+        }
+    }
     if (seconds_since(t0) > prm->budget_s) {
         res->elapsed_s = seconds_since(t0);
         return MQ_TUNE_BUDGET_EXHAUSTED;
@@ -257,21 +361,28 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
                 ok = false;
                 break;
             }
-            // admission: bit-identical out and lse
+            // admission: the bytes are compared always (evidence), the alpha rule on request
             if (launch(p, cd.cfg, B.out, B.lse) != MQ_OK) return MQ_ERR_CUDA;
-            if (!ck(cudaMemsetAsync(B.flag, 0, sizeof(unsigned), B.st))) return MQ_ERR_CUDA;
+            if (!ck(cudaMemsetAsync(B.flag, 0, 3 * sizeof(unsigned), B.st))) return MQ_ERR_CUDA;
             const long long n_out = (long long)probes[p].n_q * Hq * D, n_lse = (long long)probes[p].n_q * Hq;
             if (!ck(launch_compare(reinterpret_cast<const uint32_t*>(B.out), reinterpret_cast<const uint32_t*>(B.out_ref[p]),
                                    n_out, B.flag, B.st)) ||
                 !ck(launch_compare(reinterpret_cast<const uint32_t*>(B.lse), reinterpret_cast<const uint32_t*>(B.lse_ref[p]),
                                    n_lse, B.flag, B.st)))
                 return MQ_ERR_CUDA;
-            unsigned differ = 0;
-            if (!ck(cudaMemcpyAsync(&differ, B.flag, sizeof differ, cudaMemcpyDeviceToHost, B.st)) ||
+            if (alpha_rule &&
+                (!ck(launch_alpha_check(B.out, B.out_ref[p], B.noise_out[p], n_out, (float)alpha, B.flag + 1, B.st)) ||
+                 !ck(launch_alpha_check(B.lse, B.lse_ref[p], B.noise_lse[p], n_lse, (float)alpha, B.flag + 1, B.st))))
+                return MQ_ERR_CUDA;
+            unsigned fl[3] = {0, 0, 0};
+            if (!ck(cudaMemcpyAsync(fl, B.flag, sizeof fl, cudaMemcpyDeviceToHost, B.st)) ||
                 !ck(cudaStreamSynchronize(B.st)))
                 return MQ_ERR_CUDA;
-            if (differ) {
-                cd.identical = false;
+            float ratio = 0.0f;
+            std::memcpy(&ratio, &fl[2], sizeof ratio);
+            cd.max_ratio = std::max(cd.max_ratio, (double)ratio);
+            if (fl[0]) cd.identical = false;
+            if (alpha_rule ? fl[1] != 0 : fl[0] != 0) {
                 cd.rejected = true;
                 res->n_rejected++;
                 ok = false;
@@ -314,6 +425,12 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         n_terms += terms;
     }
     res->cost = n_terms ? total / n_terms : 1.0;
+    mq_status status = exhausted ? MQ_TUNE_BUDGET_EXHAUSTED : MQ_OK;
+    bool stored = false;
+    if (prm->store_path != nullptr && status == MQ_OK) {
+        if (mq_tune_store_put(prm->store_path, identity, res->chosen, res->cost) != MQ_OK) status = MQ_ERR_IO;
+        else stored = true;
+    }
     res->elapsed_s = seconds_since(t0);
 
     if (prm->log_path != nullptr) {
@@ -321,6 +438,18 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         if (f != nullptr) {
             std::fprintf(f, "{\n  \"budget_s\": %.3f, \"elapsed_s\": %.3f, \"n_copies\": %d, \"l2_bytes\": %d,\n",
                          prm->budget_s, res->elapsed_s, n_copies, l2);
+            std::fprintf(f, "  \"from_store\": false, \"stored\": %s, \"identity\": \"%s\",\n", stored ? "true" : "false",
+                         identity);
+            std::fprintf(f, "  \"admission\": \"%s\", \"alpha\": %.6g,\n", alpha_rule ? "alpha" : "bit_identical", alpha);
+            if (alpha_rule) {
+                std::fprintf(f, "  \"noise\": [");
+                for (int p = 0; p < P; p++)
+                    std::fprintf(f, "%s{\"probe\": \"%s\", \"out_min\": %.6g, \"out_median\": %.6g, \"out_max\": %.6g, "
+                                 "\"out_zero_points\": %lld}",
+                                 p ? ", " : "", probes[p].name, nstat[p].min, nstat[p].median, nstat[p].max,
+                                 nstat[p].zero_points);
+                std::fprintf(f, "],\n");
+            }
             std::fprintf(f, "  \"probes\": [");
             for (int p = 0; p < P; p++)
                 std::fprintf(f, "%s{\"name\": \"%s\", \"seq_len\": %d, \"n_q\": %d, \"rows_class\": %d, \"default_us\": %.3f}",
@@ -331,11 +460,14 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
                 const Cand& cd = cands[i];
                 std::fprintf(f,
                              "    {\"rows_class\": %d, \"ring_stages\": %d, \"splits_per_sm\": %d, "
-                             "\"measured\": %s, \"valid\": %s, \"bit_identical\": %s, \"times_us\": [%.3f, %.3f, %.3f]}%s\n",
+                             "\"measured\": %s, \"valid\": %s, \"bit_identical\": %s, \"admitted\": %s, "
+                             "\"times_us\": [%.3f, %.3f, %.3f], \"max_ratio\": ",
                              cd.cls, cd.cfg.ring_stages, cd.cfg.splits_per_sm,
                              cd.measured ? "true" : "false", cd.valid ? "true" : "false",
-                             cd.identical ? "true" : "false", cd.t[0] * 1e6, cd.t[1] * 1e6, cd.t[2] * 1e6,
-                             i + 1 < cands.size() ? "," : "");
+                             cd.identical ? "true" : "false", (cd.measured && !cd.rejected) ? "true" : "false",
+                             cd.t[0] * 1e6, cd.t[1] * 1e6, cd.t[2] * 1e6);
+                json_double(f, cd.max_ratio);
+                std::fprintf(f, "}%s\n", i + 1 < cands.size() ? "," : "");
             }
             std::fprintf(f, "  ],\n  \"chosen\": [");
             for (int cls = 0; cls < 3; cls++)
@@ -346,5 +478,5 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
             std::fclose(f);
         }
     }
-    return exhausted ? MQ_TUNE_BUDGET_EXHAUSTED : MQ_OK;
+    return status;
 }

@@ -55,7 +55,7 @@ def test_sizes():
 
 
 def test_status_strings():
-    for s in range(8):
+    for s in range(9):
         assert mq.mq_status_string(s) and mq.mq_status_string(s) != "unknown status"
     assert mq.mq_status_string(99) == "unknown status"
     assert mq.mq_version() >= 10000
