@@ -9,8 +9,9 @@
 //     z_t = scale * <q, s_k[t] * kcode_t>,  t = 0 .. L_b - n_b + j
 //     out = sum_t softmax(z)_t * (s_v[t, group] * vcode_t),  lse = log sum_t exp z_t
 //
-// How.  One CTA (11 warps, one per SM) takes a contiguous range of 128-token chunks of
-// one (sequence, kv-head, row block) and runs a warp-specialised pipeline per chunk:
+// How.  One CTA (11 warps; two per SM for the 8-row D=128 class, one per SM otherwise)
+// takes a contiguous range of 128-token chunks of one (sequence, kv-head, row block) and
+// runs a warp-specialised pipeline per chunk:
 //  * warp 0 streams the chunk's 8 pages into a shared-memory ring with one 1-D bulk
 //    TMA copy per page (block-table lookup, L2 evict-first).  The page format makes
 //    the int8 key codes of a chunk one K-major tensor-core operand as they land.
@@ -31,9 +32,10 @@
 //    when a chunk max exceeds it by more than kLazy, after rescaling O and the sums in
 //    tensor memory), and write p = 2^(z - M) and the weights W_g (fp16) to shared memory.
 // The CTA partials of a (sequence, kv-head, row block) are combined by one fixed binary
-// tree over the split index; the last CTA to finish (one atomic counter) completes it
-// and writes out and lse.  The chunk ranges depend only on the shape and the SM count,
-// so the result is bit-identical for every ring depth.
+// tree over the split index in merge_kernel, launched right after this kernel as a
+// programmatic dependent launch; it writes out and lse.  A unit that is not split writes
+// them here.  The chunk ranges depend only on the shape, the SM count and the configured
+// splits per SM, so the result is bit-identical for every ring depth.
 #include <cfloat>
 #include <climits>
 
@@ -64,9 +66,11 @@ struct Tc {
     // each other's latencies better than deeper buffers in one.
     static constexpr int CPS = (D == 128 && ROWS == 8) ? 2 : 1;
     static constexpr int TCOLS = CPS == 2 ? 256 : 512;                           // TMEM columns allocated
-    static constexpr int NSB = CPS == 2 ? 2 : ((D == 128 && ROWS <= 16) ? 4 : (ROWS == 32 ? 1 : 2));   // score buffers (TMEM)
-    static constexpr int NVB = CPS == 2 ? 1 : ((D == 256 && ROWS == 16) ? 1 : 2);  // V^T buffers (TMEM)
-    static constexpr int NWB = CPS == 2 ? 3 : ((ROWS == 32 || (D == 256 && ROWS == 16)) ? 2 : 3);  // weight buffers (smem)
+    // With two CTAs per SM (256 columns each) one score buffer leaves room for two V^T
+    // buffers, so that converting chunk i + 1 overlaps the value MMAs of chunk i.
+    static constexpr int NSB = CPS == 2 ? 1 : ((D == 128 && ROWS <= 16) ? 4 : (ROWS == 32 ? 1 : 2));   // score buffers (TMEM)
+    static constexpr int NVB = CPS == 2 ? 2 : ((D == 256 && ROWS == 16) ? 1 : 2);  // V^T buffers (TMEM)
+    static constexpr int NWB = CPS == 2 ? 2 : ((ROWS == 32 || (D == 256 && ROWS == 16)) ? 2 : 3);  // weight buffers (smem)
     static constexpr int NPB = NWB > NVB ? NWB : NVB;                            // value-MMA completion barriers
     // tensor-memory columns
     static constexpr int T_S = 0;
@@ -82,7 +86,7 @@ struct Tc {
 };
 
 struct Smem {
-    size_t ring, wbuf, qlimb, fmat, part, xch, crow, lim, pgbad, mbar, misc, heap, fin, total;
+    size_t ring, wbuf, qlimb, fmat, part, xch, crow, lim, pgbad, mbar, misc, total;
 };
 
 // NS = ring stages (chunks of 8 pages)
@@ -97,18 +101,16 @@ __host__ __device__ inline Smem smem_layout(int NS) {
     off = al(off, 128);
     s.wbuf = off;
     off += (size_t)T::NWB * T::WBYTES;
-    // the final cross-CTA merge reuses ring + weight buffers (idle by then)
-    s.heap = 0;
-    s.fin = al((size_t)2 * kMaxSplits * ROWS * 16, 16);
-    if (s.fin + (size_t)T::PART * 4 > off) return Smem{};   // does not fit: total = 0
+    // the CTA partial is written after the last chunk's value MMAs are complete: every
+    // page copy has landed and every role is done with the ring, so it reuses the ring
+    s.part = s.ring;
+    if ((size_t)T::PART * 4 > (size_t)NS * kChunkPages * T::PB) return Smem{};   // does not fit: total = 0
     off = al(off, 128);
     s.qlimb = off;
     off += (size_t)T::NQ * D;
     off = al(off, 128);
     s.fmat = off;
     off += 4096;
-    s.part = off;
-    off += (size_t)T::PART * 4;
     s.xch = off;
     off += (size_t)2 * ROWS * 4 * 4;
     s.crow = off;
@@ -246,6 +248,15 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
     if (c0 >= n_chunks) return;
     const int n_ck = min(c0 + p.cpc, n_chunks) - c0;
     const int n_splits = (n_chunks + p.cpc - 1) / p.cpc;
+
+    // block-table entries of the first chunk (warp 0, lanes < 8), loaded before the set-up:
+    // the table is an input of the launch that no preceding append writes
+    int blk_first = 0;
+    if (warp == 0) {
+        const int lp = c0 * kChunkPages + lane;
+        if (lane < kChunkPages && lp < n_pages)
+            blk_first = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + lp);
+    }
 
     // the dependent merge kernel may be scheduled now; it waits for this grid to complete
     if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -398,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
                        ? __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + lp)
                        : 0;
         };
-        int blk_next = bt_load(0);
+        int blk_next = blk_first;
         int issued = 0;
         for (int i = 0; i < n_ck; i++) {
             const int s = i % NS;
@@ -832,6 +843,10 @@ __global__ void __launch_bounds__(1024) merge_kernel(const DecodeParams p) {
     const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
     const float* gml0 = p.part_ml + pidx * p.split_stride * (size_t)(2 * ROWS);
     const float* go0 = p.part_o + pidx * p.split_stride * (size_t)(ROWS * D);
+    // the next kernel on the stream may be scheduled now: a decode kernel there reads no
+    // page and writes no partial before its own griddepcontrol.wait, which returns only
+    // once this grid has completed
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // the 8 leaves of this thread's group, loads in flight before the split count is
     // known (every slot below split_stride exists; unused ones are ignored below)
