@@ -120,10 +120,12 @@ def load_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the decode kernel's own sources (the kernel, its device helpers and its
+    parameter block): DRAM counters taken on another version of them are stale."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "quantized_kv_decode_quantize_b200", "csrc")
-    for n in sorted(os.listdir(d)):
+    for n in ("mq_decode.cu", "mq_device.cuh", "mq_tc.cuh", "mq_kernels.h"):
         with open(os.path.join(d, n), "rb") as f:
             h.update(n.encode() + f.read())
     return h.hexdigest()[:16]

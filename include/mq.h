@@ -198,6 +198,13 @@ mq_status mq_kv_append(mq_cache* cache, const void* k, const void* v, mq_dtype d
  *                that fits it.  Calls that share a workspace must not overlap.
  *   workspace_bytes  its size; a workspace smaller than the query for this
  *                shape is refused with MQ_ERR_WORKSPACE.
+ * Stream order: the kernels are launched as programmatic dependent launches and
+ * let the kernel after them start its set-up early.  Every page read and every
+ * write waits until the preceding kernel on the stream has completed, but the set-up
+ * reads q, block_table, seq_lens and n_q_per_seq before that wait.  When the
+ * preceding work on the stream is another mq_decode_attn or mq_kv_append call, these
+ * four inputs must not be that call's outputs (e.g. its out used as this call's q).
+ * Any other kernel in between restores plain stream order.
  * Query token j of sequence b (0-based) attends to positions 0 .. L_b - n_b + j:
  * the history plus drafts 0..j (causal among the drafts).  q-head h reads
  * kv-head h / (n_q_heads / n_kv_heads).  The result is bit-identical for every
