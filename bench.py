@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tune", type=float, default=0.0, help="run mq_tune with this budget (s) first")
+    ap.add_argument("--cascade", action="store_true",
+                    help="decode with mq_decode_attn_cascade over the workload's shared prefix")
     return ap.parse_args()
 
 
@@ -330,7 +332,12 @@ def run_mq(args, rank, world, local):
     n_q = torch.tensor(w.n_q, **i32)
     out = torch.empty((w.total_q, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
     lse = torch.empty((w.total_q, w.n_q_heads), dtype=torch.float32, device=dev)
-    ws_bytes = mq.mq_decode_workspace_bytes(cache.handle, w.n_seqs, w.n_q_heads, w.max_q, w.max_seq_len)
+    cascade = bool(args.cascade and w.shared_prefix)
+    if cascade:
+        ws_bytes = mq.mq_decode_cascade_workspace_bytes(cache.handle, w.n_seqs, w.n_q_heads, w.total_q, w.max_q,
+                                                        w.max_seq_len, w.shared_prefix)
+    else:
+        ws_bytes = mq.mq_decode_workspace_bytes(cache.handle, w.n_seqs, w.n_q_heads, w.max_q, w.max_seq_len)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
     scale = 1.0 / math.sqrt(w.head_dim)
     tab_c = [tabs[c] for c in range(copies)]
@@ -342,8 +349,13 @@ def run_mq(args, rank, world, local):
             return
         if ev is not None:
             ev[0].record(stream)
-        mq.mq_decode_attn(cache.handle, q, dt_code, w.n_seqs, w.n_q_heads, w.total_q, w.max_q, w.max_seq_len,
-                          tab_c[c], w.max_blocks(), seq_lens, n_q, scale, out, lse, ws, ws_bytes, stream)
+        if cascade:
+            mq.mq_decode_attn_cascade(cache.handle, q, dt_code, w.n_seqs, w.n_q_heads, w.total_q, w.max_q,
+                                      w.max_seq_len, tab_c[c], w.max_blocks(), seq_lens, n_q, w.shared_prefix, scale,
+                                      out, lse, ws, ws_bytes, stream)
+        else:
+            mq.mq_decode_attn(cache.handle, q, dt_code, w.n_seqs, w.n_q_heads, w.total_q, w.max_q, w.max_seq_len,
+                              tab_c[c], w.max_blocks(), seq_lens, n_q, scale, out, lse, ws, ws_bytes, stream)
         if ev is not None:
             ev[1].record(stream)
 
@@ -423,7 +435,12 @@ def run_mq(args, rank, world, local):
         xs = sorted(xs)
         return xs[min(len(xs) - 1, int(round(q * (len(xs) - 1))))] if xs else None
 
-    n_decode_kernels = mq.mq_decode_kernel_count(cache.handle, w.n_seqs, w.n_q_heads, w.max_q, w.max_seq_len)
+    if cascade:   # prefix pass + suffix pass + the two-way merge
+        n_decode_kernels = (mq.mq_decode_kernel_count(cache.handle, 1, w.n_q_heads, w.total_q, w.shared_prefix)
+                            + mq.mq_decode_kernel_count(cache.handle, w.n_seqs, w.n_q_heads, w.max_q,
+                                                        w.max_seq_len - w.shared_prefix) + 1)
+    else:
+        n_decode_kernels = mq.mq_decode_kernel_count(cache.handle, w.n_seqs, w.n_q_heads, w.max_q, w.max_seq_len)
 
     # ---- e2e through the C ABI from pinned host buffers ----
     e2e = None
@@ -474,7 +491,8 @@ def run_mq(args, rank, world, local):
                        "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
                        "l2_policy": f"inputs larger than L2: {copies} rotating cache copies "
                                     f"({copies * copy_bytes / 1e6:.0f} MB, L2 {l2 / 1e6:.0f} MB)",
-                       "parallelism": f"replica x{world}", "step": "mq_kv_append + mq_decode_attn",
+                       "parallelism": f"replica x{world}",
+                       "step": "mq_kv_append + " + ("mq_decode_attn_cascade" if cascade else "mq_decode_attn"),
                        "decode_config": cfg, "us_per_step": elapsed_ms / args.steps * 1e3,
                        "pct_of_8TBps": 100 * value / world / 8000.0,
                        "decode_bytes_logical": dec_bytes,
@@ -489,7 +507,9 @@ def run_mq(args, rank, world, local):
                          "kernel_us_median": statistics.median(kern_ms) * 1e3 if kern_ms else None,
                          "kernel_us_p10": pct(kern_ms, 0.1) * 1e3 if kern_ms else None,
                          "kernel_us_p90": pct(kern_ms, 0.9) * 1e3 if kern_ms else None,
-                         "kernels_timed": "decode_kernel + merge_kernel" if n_decode_kernels == 2 else "decode_kernel"},
+                         "kernels_timed": ("cascade: two decode passes + merge_two_kernel" if cascade else
+                                           "decode_kernel + merge_kernel" if n_decode_kernels == 2 else
+                                           "decode_kernel")},
             "e2e": e2e,
             "gpu_launches": (1 + n_decode_kernels) * args.steps,
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],

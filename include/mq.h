@@ -9,6 +9,8 @@
  *                   n > 1 = verification of n speculative draft tokens, causal
  *                   among the drafts) against the cache, split over the
  *                   sequence and merged by log-sum-exp
+ *   mq_decode_attn_cascade  the same for sessions sharing a cached prefix: the
+ *                   shared pages are read once for all of them
  *   mq_tune         on-device choice of the decode launch shape under a
  *                   wall-clock budget, accepting only bit-identical candidates
  *                   (or, on request, candidates within alpha times the output
@@ -265,6 +267,47 @@ mq_status mq_decode_attn_static(const mq_cache* cache, const void* q, mq_dtype q
                                 const int32_t* block_table, int32_t max_blocks_per_seq, const int32_t* seq_lens,
                                 const int32_t* n_q_per_seq, float softmax_scale, float* out, float* lse,
                                 mq_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * mq_decode_attn_cascade: mq_decode_attn for sessions that share a cached prefix,
+ * reading the shared pages once.
+ *
+ * The pages report concurrent sessions sharing one prefix cache (the deep dive,
+ * section 5; trawling.dev "Launch HN: Magnitude", per-device kernel tuning).  With
+ * mq_decode_attn every session reads the shared pages again.  Here the step is
+ *   1. one pass over the prefix pages for the query tokens of every session together
+ *      (no causal mask: every query token of a session already sees its whole prefix),
+ *   2. the plain decode over each session's own pages after the prefix, causal among
+ *      its drafts as in mq_decode_attn,
+ *   3. a merge of the two results per (query token, q-head) by their log-sum-exps:
+ *      out = (o1 e^lse1 + o2 e^lse2) / (e^lse1 + e^lse2), lse = log(e^lse1 + e^lse2).
+ * The result equals mq_decode_attn's within fp32 rounding (not bit-identical: the
+ * summation order differs).
+ *
+ * Arguments are those of mq_decode_attn plus
+ *   prefix_len   tokens of the shared prefix, a positive multiple of 16.  Every
+ *                sequence's block table starts with the same prefix_len / 16 blocks
+ *                (the caller's promise; the prefix pages are read through row 0), and
+ *                every sequence has L_b - n_b >= prefix_len (its queries lie after the
+ *                prefix; a sequence that breaks this is skipped and reported by
+ *                mq_device_status()).
+ *   workspace    at least mq_decode_cascade_workspace_bytes(...) bytes, 256-byte
+ *                aligned, no initialization needed; it holds both passes' CTA partials
+ *                and the prefix pass's out and lse.
+ * Errors: those of mq_decode_attn; INVALID_ARG also for a prefix_len that is not a
+ * positive multiple of 16, total_q > prefix_len, max_seq_len - prefix_len <
+ * max_q_per_seq, or total_q < max_q_per_seq; UNSUPPORTED when (n_q_heads / n_kv_heads)
+ * x total_q > 64 (the prefix pass's query rows per kv-head).
+ * Launches: the two decode passes (one or two kernels each) and one merge kernel.
+ * ------------------------------------------------------------------------- */
+size_t mq_decode_cascade_workspace_bytes(const mq_cache* cache, int32_t n_seqs, int32_t n_q_heads, int32_t total_q,
+                                         int32_t max_q_per_seq, int32_t max_seq_len, int32_t prefix_len);
+
+mq_status mq_decode_attn_cascade(const mq_cache* cache, const void* q, mq_dtype q_dtype, int32_t n_seqs,
+                                 int32_t n_q_heads, int32_t total_q, int32_t max_q_per_seq, int32_t max_seq_len,
+                                 const int32_t* block_table, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                 const int32_t* n_q_per_seq, int32_t prefix_len, float softmax_scale, float* out,
+                                 float* lse, void* workspace, size_t workspace_bytes, mq_stream stream);
 
 /* ---------------------------------------------------------------------------
  * Launch configuration and tuning

@@ -71,6 +71,9 @@ def _load():
                            ctypes.c_int),
         "mq_decode_attn_static": ([P, P, ctypes.c_int, i32, i32, i32, i32, i32, P, i32, P, P, ctypes.c_float, P, P,
                                    P], ctypes.c_int),
+        "mq_decode_cascade_workspace_bytes": ([P, i32, i32, i32, i32, i32, i32], sz),
+        "mq_decode_attn_cascade": ([P, P, ctypes.c_int, i32, i32, i32, i32, i32, P, i32, P, P, i32, ctypes.c_float,
+                                    P, P, P, sz, P], ctypes.c_int),
         "mq_get_decode_config": ([P, i32, ctypes.POINTER(mq_decode_config)], ctypes.c_int),
         "mq_set_decode_config": ([P, i32, ctypes.POINTER(mq_decode_config)], ctypes.c_int),
         "mq_tune": ([P, ctypes.POINTER(mq_tune_params), ctypes.POINTER(mq_tune_result)], ctypes.c_int),
@@ -174,6 +177,22 @@ def mq_decode_attn_static(cache: int, q, q_dtype: int, n_seqs: int, n_q_heads: i
                                      _ptr(block_table), max_blocks_per_seq, _ptr(seq_lens), _ptr(n_q_per_seq),
                                      float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream)),
            "mq_decode_attn_static")
+
+
+def mq_decode_cascade_workspace_bytes(cache: int, n_seqs: int, n_q_heads: int, total_q: int, max_q_per_seq: int,
+                                      max_seq_len: int, prefix_len: int) -> int:
+    return lib.mq_decode_cascade_workspace_bytes(cache, n_seqs, n_q_heads, total_q, max_q_per_seq, max_seq_len,
+                                                 prefix_len)
+
+
+def mq_decode_attn_cascade(cache: int, q, q_dtype: int, n_seqs: int, n_q_heads: int, total_q: int,
+                           max_q_per_seq: int, max_seq_len: int, block_table, max_blocks_per_seq: int, seq_lens,
+                           n_q_per_seq, prefix_len: int, softmax_scale: float, out, lse, workspace,
+                           workspace_bytes: int, stream=None) -> None:
+    _check(lib.mq_decode_attn_cascade(cache, _ptr(q), q_dtype, n_seqs, n_q_heads, total_q, max_q_per_seq,
+                                      max_seq_len, _ptr(block_table), max_blocks_per_seq, _ptr(seq_lens),
+                                      _ptr(n_q_per_seq), prefix_len, float(softmax_scale), _ptr(out), _ptr(lse),
+                                      _ptr(workspace), workspace_bytes, _stream(stream)), "mq_decode_attn_cascade")
 
 
 def mq_get_decode_config(cache: int, rows_class: int) -> tuple:

@@ -102,7 +102,8 @@ size_t partial_bytes(const mq_cache* c, int n_seqs, const DecodePlan& pl) {
 mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void* q, mq_dtype q_dtype, int n_seqs,
                              int n_q_heads, int total_q, int max_q, const int32_t* block_table, int max_blocks,
                              const int32_t* seq_lens, const int32_t* n_q_per_seq, float softmax_scale, float* out,
-                             float* lse, void* workspace, size_t workspace_bytes, cudaStream_t st) {
+                             float* lse, void* workspace, size_t workspace_bytes, cudaStream_t st,
+                             const DecodeView& view) {
     if (pl.smem == 0 || pl.smem > (size_t)c->max_smem) return MQ_ERR_UNSUPPORTED;
     const size_t units = (size_t)n_seqs * c->n_kv_heads * pl.n_rb;
     if (partial_bytes(c, n_seqs, pl) > workspace_bytes) return MQ_ERR_WORKSPACE;
@@ -137,6 +138,11 @@ mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void
     p.cpc = pl.cpc;
     p.stages = pl.stages;
     p.err = c->err_word;
+    p.causal = view.causal;
+    p.len_offset = view.len_offset;
+    p.bt_col = view.bt_col;
+    p.fixed_len = view.fixed_len;
+    p.fixed_nq = view.fixed_nq;
     e = launch_decode(p, c->head_dim, pl.rows, pl.max_splits, pl.smem, st);
     return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
 }

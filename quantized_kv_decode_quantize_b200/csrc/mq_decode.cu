@@ -234,8 +234,9 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
     const unsigned FULL = 0xffffffffu;
 
     // ---- sequence bounds (uniform per CTA) ----
-    const int L = __ldg(p.seq_lens + b), nq = __ldg(p.n_q_per_seq + b);
-    if (nq < 1 || nq > p.max_q || nq > L || (long long)L > (long long)p.max_blocks_per_seq * kPageTokens) {
+    const int L = seq_len_of(p, b), nq = seq_nq_of(p, b);
+    if (nq < 1 || nq > p.max_q || nq > L ||
+        (long long)L + (long long)p.bt_col * kPageTokens > (long long)p.max_blocks_per_seq * kPageTokens) {
         if (sp == 0 && rb == 0 && hk == 0 && threadIdx.x == 0) atomicOr(p.err, kErrBadSeq);
         return;
     }
@@ -255,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
     if (warp == 0) {
         const int lp = c0 * kChunkPages + lane;
         if (lane < kChunkPages && lp < n_pages)
-            blk_first = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + lp);
+            blk_first = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + p.bt_col + lp);
     }
 
     // the dependent merge kernel may be scheduled now; it waits for this grid to complete
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
     }
     if (warp == 0) {
         int s = 0;
-        for (int i = lane; i < b; i += 32) s += min(max(__ldg(p.n_q_per_seq + i), 0), p.max_q);
+        for (int i = lane; i < b; i += 32) s += min(max(seq_nq_of(p, i), 0), p.max_q);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(FULL, s, o);
         if (lane == 0) misc[0] = s;
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
             const float up = zero_row ? 0.0f : ldexpf(1.0f, 22 - E);
             if (sl == 0) {
                 crow_s[r] = zero_row ? 0.0f : ldexpf(p.scale_log2, E - 22);
-                lim_s[r] = real ? (L - nq + j + 1) : L;
+                lim_s[r] = (real && p.causal) ? (L - nq + j + 1) : L;
             }
             uint32_t w[3][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}};
 #pragma unroll
@@ -406,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
         auto bt_load = [&](int i) -> int {
             const int lp = (c0 + i) * kChunkPages + lane;
             return (i < n_ck && lane < kChunkPages && lp < n_pages)
-                       ? __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + lp)
+                       ? __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + p.bt_col + lp)
                        : 0;
         };
         int blk_next = blk_first;
@@ -561,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
             else return lim_s[r];
         };
         float Mlane = -INFINITY;   // M of row `lane` (lanes < ROWS)
-        const int lim_min = L - nq + row0 / p.group + 1;   // smallest limit of the real rows
+        const int lim_min = p.causal ? L - nq + row0 / p.group + 1 : L;   // smallest limit of the real rows
         const int nrg4 = (rows_here + 3) / 4;              // 4-row groups holding real rows
         // A warp whose wait gave up keeps iterating without work, so that the four softmax
         // warps always meet at the named barrier the same number of times.
@@ -836,7 +837,7 @@ __global__ void __launch_bounds__(1024) merge_kernel(const DecodeParams p) {
     __shared__ float2 g_ml[8][128];    // group results: m, l
     // the sequence's bounds: inputs of the launch, readable before the decode grid ends
     const int b = blockIdx.z, hk = blockIdx.y / p.n_rb, rb = blockIdx.y % p.n_rb;
-    const int L = __ldg(p.seq_lens + b), nq = __ldg(p.n_q_per_seq + b);
+    const int L = seq_len_of(p, b), nq = seq_nq_of(p, b);
     const int e = threadIdx.x & 127, j = threadIdx.x >> 7;
     const int e4 = blockIdx.x * 128 + e;   // < E4: the grid covers E4 exactly
     const int r = (4 * e4) / D;            // the element's row
@@ -861,7 +862,9 @@ __global__ void __launch_bounds__(1024) merge_kernel(const DecodeParams p) {
         vm[u] = slot ? __ldcg(gml0 + (size_t)sidx * 2 * ROWS + r) : -INFINITY;
         vl[u] = slot ? __ldcg(gml0 + (size_t)sidx * 2 * ROWS + ROWS + r) : 0.0f;
     }
-    if (nq < 1 || nq > p.max_q || nq > L || (long long)L > (long long)p.max_blocks_per_seq * kPageTokens) return;
+    if (nq < 1 || nq > p.max_q || nq > L ||
+        (long long)L + (long long)p.bt_col * kPageTokens > (long long)p.max_blocks_per_seq * kPageTokens)
+        return;
     const int rows_b = p.group * nq, row0 = rb * ROWS;
     if (row0 >= rows_b) return;
     const int rows_here = min(ROWS, rows_b - row0);
@@ -923,7 +926,7 @@ __global__ void __launch_bounds__(1024) merge_kernel(const DecodeParams p) {
     if (r >= rows_here) return;
     const int rr = row0 + r, jq = rr / p.group, hq = rr % p.group;
     int qoff = 0;
-    for (int i = 0; i < b; i++) qoff += min(max(__ldg(p.n_q_per_seq + i), 0), p.max_q);
+    for (int i = 0; i < b; i++) qoff += min(max(seq_nq_of(p, i), 0), p.max_q);
     const long long qrow = (long long)qoff + jq;
     if (qrow >= p.total_q) return;
     const float l = gl[0], m = gm[0];

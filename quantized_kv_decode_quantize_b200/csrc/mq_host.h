@@ -43,9 +43,20 @@ DecodePlan plan_decode(const mq_cache* c, int n_seqs, int n_q_heads, int max_q, 
 // Bytes of the CTA partials of one plan (the decode workspace).
 size_t partial_bytes(const mq_cache* c, int n_seqs, const DecodePlan& pl);
 cudaError_t ensure_decode_smem(int device, int head_dim, int rows, size_t smem);
+// How one decode launch sees its sequences (see DecodeParams): the defaults are a plain
+// causal decode over seq_lens and n_q_per_seq.
+struct DecodeView {
+    int causal = 1;
+    int len_offset = 0;
+    int bt_col = 0;
+    int fixed_len = 0;
+    int fixed_nq = 0;
+};
+
 mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void* q, mq_dtype q_dtype, int n_seqs,
                              int n_q_heads, int total_q, int max_q, const int32_t* block_table, int max_blocks,
                              const int32_t* seq_lens, const int32_t* n_q_per_seq, float softmax_scale, float* out,
-                             float* lse, void* workspace, size_t workspace_bytes, cudaStream_t st);
+                             float* lse, void* workspace, size_t workspace_bytes, cudaStream_t st,
+                             const DecodeView& view = DecodeView{});
 
 }  // namespace mq

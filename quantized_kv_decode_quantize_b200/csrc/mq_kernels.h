@@ -49,7 +49,24 @@ struct DecodeParams {
     int cpc;             // chunks per CTA
     int stages;          // TMA ring depth in chunks
     unsigned* err;
+    // How the launch sees each sequence (the cascade's two passes use these; a plain
+    // decode has causal 1 and the rest 0).
+    int causal;          // 1: query j of n sees positions <= L - n + j; 0: every query sees all L
+    int len_offset;      // L = seq_lens[b] - len_offset
+    int bt_col;          // block-table column of the sequence's first page
+    int fixed_len;       // > 0: L = fixed_len for every sequence (seq_lens not read)
+    int fixed_nq;        // > 0: n = fixed_nq for every sequence (n_q_per_seq not read)
 };
+
+// Cached tokens and query tokens of sequence b as a launch sees them.
+#ifdef __CUDACC__
+__device__ __forceinline__ int seq_len_of(const DecodeParams& p, int b) {
+    return p.fixed_len > 0 ? p.fixed_len : __ldg(p.seq_lens + b) - p.len_offset;
+}
+__device__ __forceinline__ int seq_nq_of(const DecodeParams& p, int b) {
+    return p.fixed_nq > 0 ? p.fixed_nq : __ldg(p.n_q_per_seq + b);
+}
+#endif
 
 // rows: 8, 16 or 32 (padded query rows per kv-head handled by one CTA)
 size_t decode_smem_bytes(int head_dim, int rows, int stages);   // 0: does not fit the layout

@@ -67,6 +67,21 @@ class GpuCase:
                           self.lse if with_lse else None, self.ws, self.ws.numel())
         return self.out, self.lse
 
+    def decode_cascade(self, prefix_len=None, copy=0, scale=None, with_lse=True):
+        """mq_decode_attn_cascade over the workload's shared prefix (or prefix_len)."""
+        w = self.w
+        prefix_len = w.shared_prefix if prefix_len is None else prefix_len
+        scale = 1.0 / math.sqrt(w.head_dim) if scale is None else scale
+        need = mq.mq_decode_cascade_workspace_bytes(self.cache.handle, w.n_seqs, w.n_q_heads, w.total_q, w.max_q,
+                                                    w.max_seq_len, prefix_len)
+        if self.ws.numel() < need:   # need == 0: the call itself refuses the arguments
+            self.ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+        mq.mq_decode_attn_cascade(self.cache.handle, self.q, DT[w.dtype], w.n_seqs, w.n_q_heads, w.total_q, w.max_q,
+                                  w.max_seq_len, self.tabs[copy], w.max_blocks(), self.seq_lens, self.n_q,
+                                  prefix_len, scale, self.out, self.lse if with_lse else None, self.ws,
+                                  self.ws.numel())
+        return self.out, self.lse
+
     def status(self):
         return mq.mq_device_status(self.cache.handle)
 

@@ -91,6 +91,9 @@ def test_null_arguments_rejected_before_cuda():
     assert mq.lib.mq_decode_attn(None, 1, 1, 1, 8, 1, 1, 16, 1, 1, 1, 1, 0.1, 16, None, 256, 1 << 20, None) \
         == mq.MQ_ERR_INVALID_ARG
     assert mq.lib.mq_decode_workspace_bytes(None, 1, 8, 1, 16) == 0
+    assert mq.lib.mq_decode_cascade_workspace_bytes(None, 1, 8, 1, 1, 64, 16) == 0
+    assert mq.lib.mq_decode_attn_cascade(None, 1, 1, 1, 8, 1, 1, 64, 1, 4, 1, 1, 16, 0.1, 16, None, 256, 1 << 20,
+                                         None) == mq.MQ_ERR_INVALID_ARG
     assert mq.lib.mq_device_status(None, None) == mq.MQ_ERR_INVALID_ARG
     cfg = mq.mq_decode_config()
     assert mq.lib.mq_get_decode_config(None, 0, ctypes.byref(cfg)) == mq.MQ_ERR_INVALID_ARG
