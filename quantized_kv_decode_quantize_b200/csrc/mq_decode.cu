@@ -47,7 +47,6 @@ namespace mq {
 
 // lazy-max threshold of the online softmax, in log2 units (weights stay <= 2^4)
 constexpr float kLazy = 4.0f;
-constexpr int kThreads = 352;   // warp 0 TMA, 1 QK MMA, 2 PV MMA, 3-6 values, 7-10 softmax
 
 template <int D, int ROWS>
 struct Tc {
@@ -72,6 +71,13 @@ struct Tc {
     static constexpr int NVB = CPS == 2 ? 2 : ((D == 256 && ROWS == 16) ? 1 : 2);  // V^T buffers (TMEM)
     static constexpr int NWB = CPS == 2 ? 2 : ((ROWS == 32 || (D == 256 && ROWS == 16)) ? 2 : 3);  // weight buffers (smem)
     static constexpr int NPB = NWB > NVB ? NWB : NVB;                            // value-MMA completion barriers
+    // Softmax warp groups: the 32-row class splits its rows over two groups of four warps
+    // (one warp per TMEM lane quadrant each); rows interact only through the chunk maximum
+    // of each row, which a group exchanges on its own named barrier.
+    static constexpr int NSG = ROWS == 32 ? 2 : 1;
+    static constexpr int RPG = ROWS / NSG;                                       // rows per group
+    // warp 0 TMA, 1 QK MMA, 2 PV MMA, 3-6 values, 7.. softmax
+    static constexpr int THREADS = 224 + 128 * NSG;
     // tensor-memory columns
     static constexpr int T_S = 0;
     static constexpr int T_O = NSB * NQ;
@@ -207,13 +213,15 @@ struct AlphaRows {
 
 // Multiplies this warp's 32 TMEM lanes of the value accumulators (NO columns from t_o)
 // and of the column sums (NS columns from t_sum) by the factor of each column's row
-// (column j holds row j % ROWS).  Out of line: it runs only when a running max moves.
-template <int ROWS, int NO, int NS>
-__device__ __noinline__ void rescale_acc(uint32_t lane_base, int t_o, int t_sum, AlphaRows<ROWS> al) {
+// (column j holds row j % ROWS), for the RPG rows from row rlo (a softmax warp group's
+// rows; al holds their factors).  Out of line: it runs only when a running max moves.
+template <int ROWS, int RPG, int NO, int NS>
+__device__ __noinline__ void rescale_acc(uint32_t lane_base, int t_o, int t_sum, int rlo, AlphaRows<RPG> al) {
 #pragma unroll 1
     for (int cb = 0; cb < (NO + NS) / 8; cb++) {
         const int col = cb < NO / 8 ? t_o + 8 * cb : t_sum + 8 * cb - NO;
-        const int r0 = (8 * cb) % ROWS;   // NO, NS and ROWS are multiples of 8
+        const int r0 = (8 * cb) % ROWS - rlo;   // NO, NS, ROWS and rlo are multiples of 8
+        if (r0 < 0 || r0 >= RPG) continue;      // another group's rows
         uint32_t v[8];
         tmem_ld8(lane_base + (uint32_t)col, v);
         tmem_wait_ld();
@@ -224,7 +232,7 @@ __device__ __noinline__ void rescale_acc(uint32_t lane_base, int t_o, int t_sum,
 }
 
 template <int D, int ROWS>
-__global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode_kernel(const DecodeParams p) {
     using T = Tc<D, ROWS>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -300,13 +308,13 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; s++) {
             mbar_init(full_b(s), 1);
-            mbar_init(empty_b(s), 9);   // QK commit + 4 value warps + 4 softmax warps
+            mbar_init(empty_b(s), 5 + 4 * T::NSG);   // QK commit + 4 value warps + the softmax warps
         }
         for (int j = 0; j < T::NSB; j++) {
             mbar_init(sfull_b + 8 * j, 1);
-            mbar_init(sfree_b + 8 * j, 4);
+            mbar_init(sfree_b + 8 * j, 4 * T::NSG);
         }
-        for (int j = 0; j < T::NWB; j++) mbar_init(wfull_b + 8 * j, 4);
+        for (int j = 0; j < T::NWB; j++) mbar_init(wfull_b + 8 * j, 4 * T::NSG);
         for (int j = 0; j < T::NVB; j++) mbar_init(vfull_b + 8 * j, 4);
         for (int j = 0; j < T::NPB; j++) mbar_init(pvdone_b + 8 * j, 1);
         mbar_fence_init();
@@ -343,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
     if (warp >= 7) {
         const int tid = threadIdx.x - 224;
         constexpr int SL = D / 8;   // 8-channel slices of a row
-        for (int it = tid; it < ROWS * SL; it += 128) {
+        for (int it = tid; it < ROWS * SL; it += 128 * T::NSG) {
             const int r = it / SL, sl = it % SL;
             const bool real = r < rows_here;
             const int rr = row0 + r, j = real ? rr / p.group : 0, hq = real ? rr % p.group : 0;
@@ -390,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
         fence_proxy_async_smem();
     }
     // the TMA producer starts at once; the other warps wait for the limbs and TMEM
-    if (warp != 0) named_bar_sync(1, kThreads - 32);
+    if (warp != 0) named_bar_sync(1, T::THREADS - 32);
     tc_fence_after();
     const uint32_t tmem = (uint32_t)misc[3];
     const uint32_t ring = smem_u32(smem + S.ring);
@@ -536,36 +544,41 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
         }
     } else {
         // ================= softmax and weights (one TMEM lane = one token) =================
-        const int sw = warp - 7, q = warp & 3, t = 32 * q + lane;
+        // warp 7 + 4 * sg + k: lane quadrant (warp & 3), rows r0g .. r0g + RPG - 1
+        constexpr int RPG = T::RPG;
+        const int sw = warp - 7, sw4 = sw & 3, sg = sw >> 2, q = warp & 3, t = 32 * q + lane;
+        const int r0g = sg * RPG;
         const int tp = t / 16, ttg = (t / 8) & 1, tt = t & 7;
         const uint32_t wb0 = smem_u32(smem + S.wbuf);
         float* xch = reinterpret_cast<float*>(smem + S.xch);
         // Row factors and visibility limits: registers for the 8-row class, shared memory
         // (broadcast reads) for the larger ones, which would otherwise run out of registers.
+        // Below, rows are indexed within the group (0 .. RPG - 1).
         constexpr bool kRowRegs = ROWS <= 8;
-        float crow_r[kRowRegs ? ROWS : 1], M[ROWS];
-        int lim_r[kRowRegs ? ROWS : 1];
+        float crow_r[kRowRegs ? RPG : 1], M[RPG];
+        int lim_r[kRowRegs ? RPG : 1];
 #pragma unroll
-        for (int r = 0; r < ROWS; r++) {
+        for (int r = 0; r < RPG; r++) {
             if constexpr (kRowRegs) {
-                crow_r[r] = crow_s[r];
-                lim_r[r] = lim_s[r];
+                crow_r[r] = crow_s[r0g + r];
+                lim_r[r] = lim_s[r0g + r];
             }
             M[r] = -INFINITY;
         }
         auto crow = [&](int r) -> float {
             if constexpr (kRowRegs) return crow_r[r];
-            else return crow_s[r];
+            else return crow_s[r0g + r];
         };
         auto lim = [&](int r) -> int {
             if constexpr (kRowRegs) return lim_r[r];
-            else return lim_s[r];
+            else return lim_s[r0g + r];
         };
-        float Mlane = -INFINITY;   // M of row `lane` (lanes < ROWS)
+        float Mlane = -INFINITY;   // M of the group's row `lane` (lanes < RPG)
         const int lim_min = p.causal ? L - nq + row0 / p.group + 1 : L;   // smallest limit of the real rows
-        const int nrg4 = (rows_here + 3) / 4;              // 4-row groups holding real rows
-        // A warp whose wait gave up keeps iterating without work, so that the four softmax
-        // warps always meet at the named barrier the same number of times.
+        const int rh = max(0, min(RPG, rows_here - r0g));                 // the group's real rows
+        const int nrg4 = (rh + 3) / 4;                                    // 4-row groups holding real rows
+        // A warp whose wait gave up keeps iterating without work, so that the four warps
+        // of a group always meet at their named barrier the same number of times.
         bool ok = true;
         for (int i = 0; i < n_ck; i++) {
             const int s = i % NS, sb = i % T::NSB, wb = i % T::NWB;
@@ -573,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
             // this token's scales and page flags; then the stage is released
             float sk = 0.0f, sv[T::G];
             bool any_bad = false, my_bad = false;
-            float z[ROWS];
+            float z[RPG];
             if (ok && wait_warp(full_b(s), (uint32_t)(i / NS) & 1u)) {
                 const uint32_t rec = ring + (uint32_t)((s * kChunkPages + tp) * T::PB + ttg * T::REC);
                 sk = h_bits_to_f32(ldsa16(rec + rec_ks_off(D) + 2 * tt));
@@ -608,10 +621,10 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
                 tc_fence_after();
                 // ---- scores of the real rows: the three limb accumulations -> fp32 ----
 #pragma unroll
-                for (int rg = 0; rg < ROWS / 4; rg++) {
+                for (int rg = 0; rg < RPG / 4; rg++) {
                     if (rg < nrg4) {
                         uint32_t a2[4], a1[4], a0[4];
-                        const uint32_t col = T::T_S + sb * T::NQ + 4 * rg;
+                        const uint32_t col = T::T_S + sb * T::NQ + r0g + 4 * rg;
                         tmem_ld4(tmem_at(tmem, 32 * q, col), a2);
                         tmem_ld4(tmem_at(tmem, 32 * q, col + ROWS), a1);
                         tmem_ld4(tmem_at(tmem, 32 * q, col + 2 * ROWS), a0);
@@ -634,27 +647,27 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
                 if (!clean) {
                     const int tok = c * kChunkTokens + t;
 #pragma unroll
-                    for (int r = 0; r < ROWS; r++)
+                    for (int r = 0; r < RPG; r++)
                         if (my_bad || tok >= lim(r)) z[r] = -INFINITY;
                 }
                 // ---- chunk row maxima over the 128 tokens ----
 #pragma unroll
-                for (int rg = 0; rg < ROWS / 4; rg++)
+                for (int rg = 0; rg < RPG / 4; rg++)
                     if (rg < nrg4) {
 #pragma unroll
                         for (int e = 0; e < 4; e++) {
                             const float m = warp_redux_max(z[4 * rg + e]);
-                            if (lane == 0) xb[(4 * rg + e) * 4 + sw] = m;
+                            if (lane == 0) xb[(r0g + 4 * rg + e) * 4 + sw4] = m;
                         }
                     }
             }
-            named_bar_sync(2, 128);
+            named_bar_sync(2 + sg, 128);
             if (ok) {
                 // ---- lazy running max: moved only when a chunk max exceeds it by kLazy ----
                 bool need = false;
                 float cm = -INFINITY;
-                if (lane < rows_here) {
-                    const float4 v = *reinterpret_cast<const float4*>(xb + lane * 4);
+                if (lane < rh) {
+                    const float4 v = *reinterpret_cast<const float4*>(xb + (r0g + lane) * 4);
                     cm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
                     need = cm > __fadd_rn(Mlane, kLazy);
                 }
@@ -662,17 +675,18 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
                     const float Mn = need ? cm : Mlane;
                     const float al = (Mn == Mlane) ? 1.0f : ex2(__fsub_rn(Mlane, Mn));
                     Mlane = Mn;
-                    float alpha[ROWS];
+                    float alpha[RPG];
 #pragma unroll
-                    for (int r = 0; r < ROWS; r++) {
+                    for (int r = 0; r < RPG; r++) {
                         M[r] = __shfl_sync(FULL, Mn, r);
                         alpha[r] = __shfl_sync(FULL, al, r);
                     }
-                    // rescale O and the sums (this warp's 32 lanes) once the previous
-                    // chunk's value MMAs are complete
+                    // rescale O and the sums (this warp's 32 lanes, this group's rows) once
+                    // the previous chunk's value MMAs are complete
                     if (i > 0 && wait_warp(pv_bar(i - 1), pv_par(i - 1))) {
                         tc_fence_after();
-                        rescale_acc<ROWS, T::H * T::NO, T::NB>(tmem_at(tmem, 32 * q, 0), T::T_O, T::T_SUM, AlphaRows<ROWS>::make(alpha));
+                        rescale_acc<ROWS, RPG, T::H * T::NO, T::NB>(tmem_at(tmem, 32 * q, 0), T::T_O, T::T_SUM, r0g,
+                                                                     AlphaRows<RPG>::make(alpha));
                         tmem_wait_st();
                     } else if (i > 0) {
                         ok = false;
@@ -694,14 +708,14 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
                     }
                 };
 #pragma unroll
-                for (int rg8 = 0; rg8 < ROWS / 8; rg8++) {
+                for (int rg8 = 0; rg8 < RPG / 8; rg8++) {
                     if (2 * rg8 >= nrg4) continue;
                     const bool two = 2 * rg8 + 1 < nrg4;
                     float pw[8];
 #pragma unroll
                     for (int e = 0; e < 8; e++) {
                         const int r = 8 * rg8 + e;
-                        pw[e] = (r >= rows_here || z[r] == -INFINITY) ? 0.0f : ex2(__fsub_rn(z[r], M[r]));
+                        pw[e] = (r >= rh || z[r] == -INFINITY) ? 0.0f : ex2(__fsub_rn(z[r], M[r]));
                     }
 #pragma unroll
                     for (int g = 0; g < T::G; g++) {
@@ -713,9 +727,9 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
                             // masked tokens may carry unwritten (non-finite) scales
                             w[e] = (!clean && pv == 0.0f) ? 0.0f : wv;
                         }
-                        store_group(wrow + (uint32_t)(((g * ROWS + 8 * rg8) / 8) * 128), w, two);
+                        store_group(wrow + (uint32_t)(((g * ROWS + r0g + 8 * rg8) / 8) * 128), w, two);
                     }
-                    store_group(wrow + (uint32_t)(((T::G * ROWS + 8 * rg8) / 8) * 128), pw, two);
+                    store_group(wrow + (uint32_t)(((T::G * ROWS + r0g + 8 * rg8) / 8) * 128), pw, two);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -727,11 +741,11 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
         if (ok) ok = wait_warp(pv_bar(n_ck - 1), pv_par(n_ck - 1));
         if (ok) {
             tc_fence_after();
-            float lr[ROWS];
+            float lr[RPG];
 #pragma unroll
-            for (int rg = 0; rg < ROWS / 8; rg++) {
+            for (int rg = 0; rg < RPG / 8; rg++) {
                 uint32_t v[8];
-                tmem_ld8(tmem_at(tmem, 32 * q, T::T_SUM + T::G * ROWS + 8 * rg), v);
+                tmem_ld8(tmem_at(tmem, 32 * q, T::T_SUM + T::G * ROWS + r0g + 8 * rg), v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 8; e++) lr[8 * rg + e] = __uint_as_float(v[e]);
@@ -740,22 +754,22 @@ __global__ void __launch_bounds__(kThreads, Tc<D, ROWS>::CPS) decode_kernel(cons
             for (int h = 0; h < T::H; h++) {
                 const int ch = 128 * h + 32 * q + lane, g = 4 * h + q;
 #pragma unroll
-                for (int rg = 0; rg < ROWS / 8; rg++) {
-                    uint32_t o[8], sg[8];
-                    tmem_ld8(tmem_at(tmem, 32 * q, T::T_O + h * T::NO + q * ROWS + 8 * rg), o);
-                    tmem_ld8(tmem_at(tmem, 32 * q, T::T_SUM + g * ROWS + 8 * rg), sg);
+                for (int rg = 0; rg < RPG / 8; rg++) {
+                    uint32_t o[8], sgm[8];
+                    tmem_ld8(tmem_at(tmem, 32 * q, T::T_O + h * T::NO + q * ROWS + r0g + 8 * rg), o);
+                    tmem_ld8(tmem_at(tmem, 32 * q, T::T_SUM + g * ROWS + r0g + 8 * rg), sgm);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 8; e++)
-                        part[(8 * rg + e) * D + ch] =
-                            __fmaf_rn(__uint_as_float(o[e]), 16777216.0f, -8.0f * __uint_as_float(sg[e]));
+                        part[(r0g + 8 * rg + e) * D + ch] =
+                            __fmaf_rn(__uint_as_float(o[e]), 16777216.0f, -8.0f * __uint_as_float(sgm[e]));
                 }
             }
-            if (sw == 0 && lane == 0) {
+            if (sw4 == 0 && lane == 0) {
 #pragma unroll
-                for (int r = 0; r < ROWS; r++) {
-                    part[ROWS * D + r] = M[r];
-                    part[ROWS * D + ROWS + r] = lr[r];
+                for (int r = 0; r < RPG; r++) {
+                    part[ROWS * D + r0g + r] = M[r];
+                    part[ROWS * D + ROWS + r0g + r] = lr[r];
                 }
             }
         }
@@ -979,7 +993,7 @@ static cudaError_t launch_pair(const DecodeParams& p, dim3 grid, size_t smem, in
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t dc{};
     dc.gridDim = grid;
-    dc.blockDim = dim3((unsigned)kThreads);
+    dc.blockDim = dim3((unsigned)Tc<D, ROWS>::THREADS);
     dc.dynamicSmemBytes = smem;
     dc.stream = st;
     dc.attrs = pdl;
