@@ -165,10 +165,16 @@ mq_status mq_cache_destroy(mq_cache* cache);
  * block_table[b][pos / 16], slot pos % 16.  Two calls (or two tokens) that
  * write the same position race; writing a position of a shared block changes
  * it for every sequence that names the block.
- * Errors: INVALID_ARG (null pointers, n_seqs < 1, n_tokens < 0, dtype),
- * CUDA.  n_tokens == 0 launches nothing.  A position beyond
- * max_blocks_per_seq*16 or a block id outside [0, n_blocks) is skipped by the
- * kernel and reported through mq_device_status() as MQ_ERR_DEVICE.
+ * Work: one warp per (8-token half page, kv-head) the new tokens touch.  A half
+ * page the call covers entirely is written with plain stores; the others (the
+ * ragged ends of each sequence's range) replace each 4-bit code with atomic bit
+ * operations, so appends split over several calls give the same pages as one.
+ * Errors: INVALID_ARG (null pointers, n_seqs < 1 or > 65535, n_tokens < 0,
+ * dtype), CUDA.  n_tokens == 0 launches nothing.  A position outside
+ * [0, max_blocks_per_seq*16) or a block id outside [0, n_blocks) is skipped by
+ * the kernel, and a sequence whose cu_new range leaves [0, n_tokens] is skipped
+ * whole (none of its K/V is read); both are reported through mq_device_status()
+ * as MQ_ERR_DEVICE.
  * ------------------------------------------------------------------------- */
 mq_status mq_kv_append(mq_cache* cache, const void* k, const void* v, mq_dtype dtype, int32_t n_seqs,
                        int32_t n_tokens, const int32_t* cu_new, const int32_t* start_pos,

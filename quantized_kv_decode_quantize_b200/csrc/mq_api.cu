@@ -233,7 +233,8 @@ mq_status mq_cache_destroy(mq_cache* c) {
 mq_status mq_kv_append(mq_cache* c, const void* k, const void* v, mq_dtype dtype, int32_t n_seqs, int32_t n_tokens,
                        const int32_t* cu_new, const int32_t* start_pos, const int32_t* block_table,
                        int32_t max_blocks_per_seq, mq_stream stream) {
-    if (c == nullptr || n_seqs < 1 || n_tokens < 0 || max_blocks_per_seq < 1) return MQ_ERR_INVALID_ARG;
+    if (c == nullptr || n_seqs < 1 || n_seqs > 65535 || n_tokens < 0 || max_blocks_per_seq < 1)
+        return MQ_ERR_INVALID_ARG;
     if (dtype != MQ_F32 && dtype != MQ_BF16 && dtype != MQ_F16) return MQ_ERR_INVALID_ARG;
     if (n_tokens == 0) return MQ_OK;
     if (k == nullptr || v == nullptr || cu_new == nullptr || start_pos == nullptr || block_table == nullptr)

@@ -6,13 +6,22 @@
 //   K per (token, kv-head):        s = fp16_rn(max|x| / 127), code = clamp(rne(x / s), -127, 127)
 //   V per (token, kv-head, 32 ch): s = fp16_rn(max|x| / 7),   code = clamp(rne(x / s), -8, 7)
 // Both divisions are IEEE fp32 (__fdiv_rn), rounding is to nearest even, and a
-// zero scale gives code 0.  One warp handles one (token, kv-head): each lane
-// reads D/32 consecutive channels with one vector load, the absmax reductions
-// are warp shuffles (exact: max is order-independent), each lane stores its K
-// codes with one 4- or 8-byte store, and writes its V codes into the channel-major
-// V words of the page (see mq_device.cuh).  A V word holds the codes of eight
-// tokens, so its nibble is replaced with two atomic bit operations (clear, then
-// set): appends of neighbouring tokens in one launch may touch the same word.
+// zero scale gives code 0.
+//
+// Work split: one warp per (8-position record, kv-head) that a sequence's new tokens
+// touch; the grid is (x, sequence, kv-head) and the warps of a (sequence, kv-head)
+// stride over its records.  Per token the warp quantizes as follows: each lane reads
+// D/32 consecutive channels with one vector load, the absmax reductions are warp
+// shuffles (exact: max is order-independent), each lane stores its K codes with one
+// 4- or 8-byte store.  A V word of the page holds one channel's codes for the 8
+// tokens of a record (see mq_device.cuh): when the append covers the whole record, the
+// warp assembles every word in registers and writes it with a plain store; otherwise
+// (the ragged ends of an append, single-token appends) each nibble is replaced with
+// two atomic bit operations (clear, then set), since another launch may have written
+// the record's other tokens.
+
+#include <algorithm>
+
 #include "mq_device.cuh"
 #include "mq_kernels.h"
 
@@ -59,98 +68,151 @@ __device__ __forceinline__ int quant_code(float x, float s, float lo, float hi) 
     return static_cast<int>(r);
 }
 
+// One token's codes, quantized by a whole warp (lane: channels CPL * lane ..).
+template <int D>
+struct TokenCodes {
+    static constexpr int CPL = D / 32;
+    uint32_t kb[CPL / 4];   // this lane's K codes, 4 per word
+    __half sk16;            // K scale (every lane)
+    uint32_t vn[CPL];       // this lane's V codes as 4-bit two's complement
+    __half sv16;            // V scale of this lane's 32-channel group
+};
+
 template <int D, typename T>
-__global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
+__device__ __forceinline__ void quantize_token(const AppendParams& p, long long tok, int h, int lane,
+                                               TokenCodes<D>& out) {
     constexpr int CPL = D / 32;          // channels per lane
     constexpr int LPG = 32 / CPL;        // lanes per 32-channel V group
-    const int lane = threadIdx.x & 31;
-    // a decode launched after this append may start its set-up now; it waits for this
-    // grid (griddepcontrol.wait) before it reads any page
-    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const long long item = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-    if (item >= (long long)p.n_tokens * p.n_kv_heads) return;
-    const int tok = (int)(item / p.n_kv_heads), h = (int)(item % p.n_kv_heads);
-
-    // sequence of this token: last b with cu_new[b] <= tok (binary search)
-    int lo = 0, hi = p.n_seqs - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(p.cu_new + mid) <= tok) lo = mid; else hi = mid - 1;
-    }
-    const int b = lo;
-    const long long pos = (long long)__ldg(p.start_pos + b) + (tok - __ldg(p.cu_new + b));
-    if (pos < 0 || pos >= (long long)p.max_blocks_per_seq * kPageTokens) {
-        if (lane == 0) atomicOr(p.err, kErrBadPosition);
-        return;
-    }
-    const int blk = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + pos / kPageTokens);
-    if (blk < 0 || (long long)blk >= p.n_blocks) {
-        if (lane == 0) atomicOr(p.err, kErrBadBlock);
-        return;
-    }
-    const int tau = (int)(pos % kPageTokens);
-    uint8_t* page = p.pool + ((long long)blk * p.n_kv_heads + h) * page_bytes(D);
-
     const size_t vec = ((size_t)tok * p.n_kv_heads + h) * D + (size_t)lane * CPL;
     float xk[CPL], xv[CPL];
     load_vec<T, CPL>(reinterpret_cast<const T*>(p.k) + vec, xk);
     load_vec<T, CPL>(reinterpret_cast<const T*>(p.v) + vec, xv);
-
     // ---- K: one scale over all D channels ----
     float a = 0.0f;
 #pragma unroll
     for (int i = 0; i < CPL; i++) a = fmaxf(a, fabsf(xk[i]));
     a = warp_max(a);
-    const __half sk16 = __float2half_rn(__fdiv_rn(a, 127.0f));
-    const float sk = __half2float(sk16);
-    uint32_t kb[CPL / 4];
+    out.sk16 = __float2half_rn(__fdiv_rn(a, 127.0f));
+    const float sk = __half2float(out.sk16);
 #pragma unroll
     for (int w = 0; w < CPL / 4; w++) {
         uint32_t word = 0;
 #pragma unroll
         for (int j = 0; j < 4; j++)
             word |= (uint32_t)(quant_code(xk[4 * w + j], sk, -127.0f, 127.0f) & 0xFF) << (8 * j);
-        kb[w] = word;
+        out.kb[w] = word;
     }
-    const int c0 = lane * CPL;
-    uint8_t* kdst = page + k_code_byte(D, tau, c0);
-    if constexpr (CPL == 4) {
-        *reinterpret_cast<uint32_t*>(kdst) = kb[0];
-    } else {
-        *reinterpret_cast<uint2*>(kdst) = make_uint2(kb[0], kb[1]);
-    }
-    if (lane == 0) *reinterpret_cast<__half*>(page + k_scale_byte(D, tau)) = sk16;
-
     // ---- V: one scale per 32-channel group (LPG lanes) ----
     float av = 0.0f;
 #pragma unroll
     for (int i = 0; i < CPL; i++) av = fmaxf(av, fabsf(xv[i]));
 #pragma unroll
     for (int o = LPG / 2; o > 0; o >>= 1) av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, o));
-    const __half sv16 = __float2half_rn(__fdiv_rn(av, 7.0f));
-    const float sv = __half2float(sv16);
-    const int bit = v_nibble_bit(tau);
+    out.sv16 = __float2half_rn(__fdiv_rn(av, 7.0f));
+    const float sv = __half2float(out.sv16);
 #pragma unroll
-    for (int i = 0; i < CPL; i++) {
-        const uint32_t n = (uint32_t)quant_code(xv[i], sv, -8.0f, 7.0f) & 0xFu;
-        unsigned* w = reinterpret_cast<unsigned*>(page + v_word_byte(D, tau, c0 + i));
-        atomicAnd(w, ~(0xFu << bit));
-        atomicOr(w, n << bit);
+    for (int i = 0; i < CPL; i++) out.vn[i] = (uint32_t)quant_code(xv[i], sv, -8.0f, 7.0f) & 0xFu;
+}
+
+// K codes, K scale and V scale of one token at slot tau of a page.
+template <int D>
+__device__ __forceinline__ void store_token_kscales(uint8_t* page, int tau, int lane, const TokenCodes<D>& tc) {
+    constexpr int CPL = D / 32, LPG = 32 / CPL;
+    const int c0 = lane * CPL;
+    uint8_t* kdst = page + k_code_byte(D, tau, c0);
+    if constexpr (CPL == 4) {
+        *reinterpret_cast<uint32_t*>(kdst) = tc.kb[0];
+    } else {
+        *reinterpret_cast<uint2*>(kdst) = make_uint2(tc.kb[0], tc.kb[1]);
     }
-    if (lane % LPG == 0)
-        *reinterpret_cast<__half*>(page + v_scale_byte(D, tau, c0 / 32)) = sv16;
+    if (lane == 0) *reinterpret_cast<__half*>(page + k_scale_byte(D, tau)) = tc.sk16;
+    if (lane % LPG == 0) *reinterpret_cast<__half*>(page + v_scale_byte(D, tau, c0 / 32)) = tc.sv16;
+}
+
+template <int D, typename T>
+__global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
+    constexpr int CPL = D / 32;
+    const int lane = threadIdx.x & 31;
+    // a decode launched after this append may start its set-up now; it waits for this
+    // grid (griddepcontrol.wait) before it reads any page
+    if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int b = blockIdx.y, h = blockIdx.z;
+    const int tok0 = __ldg(p.cu_new + b), tok1 = __ldg(p.cu_new + b + 1);
+    if (tok0 < 0 || tok1 < tok0 || tok1 > p.n_tokens) {   // inconsistent cu_new: nothing is read
+        if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(p.err, kErrBadSeq);
+        return;
+    }
+    if (tok1 == tok0) return;
+    const long long start = __ldg(p.start_pos + b), end = start + (tok1 - tok0);   // positions [start, end)
+    const long long limit = (long long)p.max_blocks_per_seq * kPageTokens;
+    const long long r_lo = start >= 0 ? start / 8 : -((-start + 7) / 8);             // floor(start / 8)
+    const long long r_hi = (end - 1) >= 0 ? (end - 1) / 8 : -((-(end - 1) + 7) / 8);
+    const int wpb = blockDim.x / 32;
+    for (long long r = r_lo + (long long)blockIdx.x * wpb + (threadIdx.x >> 5); r <= r_hi;
+         r += (long long)gridDim.x * wpb) {
+        // a record lies wholly inside or wholly outside [0, limit): limit is a multiple of 16
+        if (8 * r < 0 || 8 * r >= limit) {
+            if (lane == 0) atomicOr(p.err, kErrBadPosition);
+            continue;
+        }
+        const int blk = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + (8 * r) / kPageTokens);
+        if (blk < 0 || (long long)blk >= p.n_blocks) {
+            if (lane == 0) atomicOr(p.err, kErrBadBlock);
+            continue;
+        }
+        uint8_t* page = p.pool + ((long long)blk * p.n_kv_heads + h) * page_bytes(D);
+        const int tau0 = (int)((8 * r) % kPageTokens);   // 0 or 8: the record within the page
+        const long long p0 = 8 * r > start ? 8 * r : start, p1 = 8 * r + 8 < end ? 8 * r + 8 : end;
+        const int c0 = lane * CPL;
+        if (p1 - p0 == 8) {
+            // the whole record: V words assembled in registers, plain stores
+            uint32_t vw[CPL];
+#pragma unroll
+            for (int i = 0; i < CPL; i++) vw[i] = 0u;
+#pragma unroll 2
+            for (int tt = 0; tt < 8; tt++) {
+                TokenCodes<D> tc;
+                quantize_token<D, T>(p, tok0 + (8 * r + tt - start), h, lane, tc);
+                store_token_kscales<D>(page, tau0 + tt, lane, tc);
+                const int bit = v_nibble_bit(tt);
+#pragma unroll
+                for (int i = 0; i < CPL; i++) vw[i] |= tc.vn[i] << bit;
+            }
+#pragma unroll
+            for (int i = 0; i < CPL; i++) *reinterpret_cast<uint32_t*>(page + v_word_byte(D, tau0, c0 + i)) = vw[i];
+        } else {
+            // part of the record: each nibble replaced atomically
+            for (long long pos = p0; pos < p1; pos++) {
+                const int tau = (int)(pos % kPageTokens);
+                TokenCodes<D> tc;
+                quantize_token<D, T>(p, tok0 + (pos - start), h, lane, tc);
+                store_token_kscales<D>(page, tau, lane, tc);
+                const int bit = v_nibble_bit(tau);
+#pragma unroll
+                for (int i = 0; i < CPL; i++) {
+                    unsigned* w = reinterpret_cast<unsigned*>(page + v_word_byte(D, tau, c0 + i));
+                    atomicAnd(w, ~(0xFu << bit));
+                    atomicOr(w, tc.vn[i] << bit);
+                }
+            }
+        }
+    }
 }
 
 template <int D>
 static cudaError_t launch_append_d(const AppendParams& p, cudaStream_t st) {
-    const long long warps = (long long)p.n_tokens * p.n_kv_heads;
+    if (p.n_seqs > 65535 || p.n_kv_heads > 65535) return cudaErrorInvalidConfiguration;
     const int wpb = 8;
-    const long long blocks = (warps + wpb - 1) / wpb;
-    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    // records of one sequence: at most n_tokens / 8 + 2; about 8 warps per SM in all
+    const long long per_seq = ((long long)p.n_tokens / 8 + 2 + wpb - 1) / wpb;
+    const long long units = (long long)p.n_seqs * p.n_kv_heads;
+    const long long fill = (148LL * 8 + units - 1) / units;
+    const long long gx = std::max<long long>(1, std::min(per_seq, fill));
+    const dim3 grid((unsigned)gx, (unsigned)p.n_seqs, (unsigned)p.n_kv_heads);
     switch (p.dtype) {
-        case 0: append_kernel<D, float><<<(unsigned)blocks, wpb * 32, 0, st>>>(p); break;
-        case 1: append_kernel<D, __nv_bfloat16><<<(unsigned)blocks, wpb * 32, 0, st>>>(p); break;
-        default: append_kernel<D, __half><<<(unsigned)blocks, wpb * 32, 0, st>>>(p); break;
+        case 0: append_kernel<D, float><<<grid, wpb * 32, 0, st>>>(p); break;
+        case 1: append_kernel<D, __nv_bfloat16><<<grid, wpb * 32, 0, st>>>(p); break;
+        default: append_kernel<D, __half><<<grid, wpb * 32, 0, st>>>(p); break;
     }
     return cudaGetLastError();
 }

@@ -546,7 +546,9 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
         // ================= softmax and weights (one TMEM lane = one token) =================
         // warp 7 + 4 * sg + k: lane quadrant (warp & 3), rows r0g .. r0g + RPG - 1
         constexpr int RPG = T::RPG;
-        const int sw = warp - 7, sw4 = sw & 3, sg = sw >> 2, q = warp & 3, t = 32 * q + lane;
+        // (with one group the group index is the constant 0, so the row offsets fold away)
+        const int sw = warp - 7, sw4 = T::NSG == 1 ? sw : (sw & 3), sg = T::NSG == 1 ? 0 : (sw >> 2);
+        const int q = warp & 3, t = 32 * q + lane;
         const int r0g = sg * RPG;
         const int tp = t / 16, ttg = (t / 8) & 1, tt = t & 7;
         const uint32_t wb0 = smem_u32(smem + S.wbuf);

@@ -144,3 +144,41 @@ def test_append_bad_position_and_block_are_flagged():
                     tab[:, :1].contiguous(), 1)
     assert mq.mq_device_status(cache.handle) == mq.MQ_ERR_DEVICE
     assert mq.mq_device_status(cache.handle) == mq.MQ_OK     # the word was cleared
+
+
+@pytest.mark.parametrize("cuts", [[13, 40, 41, 77], [1, 2, 8, 9, 24, 77], [77]])
+def test_append_split_launches_equal_bulk(cuts):
+    """Appends cut at arbitrary positions (records completed across launches, partly
+    with whole-record stores, partly with atomic nibble updates) write the same pages as
+    one bulk append."""
+    w = wl.reduced("long")
+    w.seq_lens = [77]
+    inp = wl.make_inputs(w)
+    bulk = GpuCase(w, inp)
+    inc = mq.Cache(w.n_kv_heads, w.head_dim, bulk.cache.n_blocks)
+    lo = 0
+    for hi in cuts:
+        mq.mq_kv_append(inc.handle, inp.own_k[0][lo:hi].cuda(), inp.own_v[0][lo:hi].cuda(), mq.MQ_BF16, 1, hi - lo,
+                        torch.tensor([0, hi - lo], dtype=torch.int32, device="cuda"),
+                        torch.tensor([lo], dtype=torch.int32, device="cuda"), bulk.tabs[0], w.max_blocks())
+        lo = hi
+    assert mq.mq_device_status(inc.handle) == mq.MQ_OK
+    a = pagelayout.gather_sequence(bulk.cache.pool.cpu().numpy(), w.n_kv_heads, w.head_dim, bulk.tabs_np[0, 0], 77)
+    b = pagelayout.gather_sequence(inc.pool.cpu().numpy(), w.n_kv_heads, w.head_dim, bulk.tabs_np[0, 0], 77)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_append_inconsistent_cu_new_and_negative_position_are_flagged():
+    cache = mq.Cache(1, 128, 2)
+    k = torch.zeros((2, 1, 128), dtype=torch.bfloat16, device="cuda")
+    tab = torch.tensor([[0, 1]], dtype=torch.int32, device="cuda")
+    # cu_new claims 5 tokens where the launch has 2: refused before any K/V is read
+    mq.mq_kv_append(cache.handle, k, k, mq.MQ_BF16, 1, 2, torch.tensor([0, 5], dtype=torch.int32, device="cuda"),
+                    torch.tensor([0], dtype=torch.int32, device="cuda"), tab, 2)
+    assert mq.mq_device_status(cache.handle) == mq.MQ_ERR_DEVICE
+    # positions -1 and 0: the first is flagged, the second written
+    mq.mq_kv_append(cache.handle, k, k, mq.MQ_BF16, 1, 2, torch.tensor([0, 2], dtype=torch.int32, device="cuda"),
+                    torch.tensor([-1], dtype=torch.int32, device="cuda"), tab, 2)
+    assert mq.mq_device_status(cache.handle) == mq.MQ_ERR_DEVICE
+    assert mq.mq_device_status(cache.handle) == mq.MQ_OK
