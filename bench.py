@@ -123,13 +123,18 @@ def load_peaks():
 
 def kernel_source_hash():
     """Hash of the decode kernel's own sources (the kernel, its device helpers and its
-    parameter block): DRAM counters taken on another version of them are stale."""
+    parameter block) without comments and blank space: DRAM counters taken on another
+    version of the code are stale, an edited comment does not change the kernel."""
     import hashlib
+    import re
     h = hashlib.sha256()
     d = os.path.join(ROOT, "quantized_kv_decode_quantize_b200", "csrc")
     for n in ("mq_decode.cu", "mq_device.cuh", "mq_tc.cuh", "mq_kernels.h"):
-        with open(os.path.join(d, n), "rb") as f:
-            h.update(n.encode() + f.read())
+        with open(os.path.join(d, n)) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)   # block comments
+        src = re.sub(r"//[^\n]*", " ", src)                 # line comments
+        h.update(n.encode() + " ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

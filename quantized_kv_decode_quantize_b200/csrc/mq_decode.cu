@@ -9,9 +9,9 @@
 //     z_t = scale * <q, s_k[t] * kcode_t>,  t = 0 .. L_b - n_b + j
 //     out = sum_t softmax(z)_t * (s_v[t, group] * vcode_t),  lse = log sum_t exp z_t
 //
-// How.  One CTA (11 warps; two per SM for the 8-row D=128 class, one per SM otherwise)
-// takes a contiguous range of 128-token chunks of one (sequence, kv-head, row block) and
-// runs a warp-specialised pipeline per chunk:
+// How.  One CTA (11 warps, 15 for the 32-row class; two CTAs per SM for the 8-row D=128
+// class, one per SM otherwise) takes a contiguous range of 128-token chunks of one
+// (sequence, kv-head, row block) and runs a warp-specialised pipeline per chunk:
 //  * warp 0 streams the chunk's 8 pages into a shared-memory ring with one 1-D bulk
 //    TMA copy per page (block-table lookup, L2 evict-first).  The page format makes
 //    the int8 key codes of a chunk one K-major tensor-core operand as they land.
@@ -27,8 +27,9 @@
 //  * warps 3-6 turn the int4 value codes into tensor memory as exact fp16 values
 //    u * 2^-24 (u = code + 8 in 0..15, a subnormal) with one mask, shift and flip per
 //    two tokens, a channel per TMEM lane; out = 2^24 * O - 8 * sum_t W_g.
-//  * warps 7-10 (one TMEM lane per token) read S, form z in fp32, take the chunk's row
-//    maxima (redux + a named barrier), keep a lazy running max M per row (moved only
+//  * warps 7-10 (one TMEM lane per token; 7-14 in two row groups for the 32-row class)
+//    read S, form z in fp32, take the chunk's row maxima (redux + a named barrier),
+//    keep a lazy running max M per row (moved only
 //    when a chunk max exceeds it by more than kLazy, after rescaling O and the sums in
 //    tensor memory), and write p = 2^(z - M) and the weights W_g (fp16) to shared memory.
 // The CTA partials of a (sequence, kv-head, row block) are combined by one fixed binary
