@@ -11,6 +11,9 @@
  *                   sequence and merged by log-sum-exp
  *   mq_decode_attn_cascade  the same for sessions sharing a cached prefix: the
  *                   shared pages are read once for all of them
+ *   mq_draft_ngram  history-based drafts (the tokens that followed the latest
+ *                   earlier occurrence of a sequence's last n tokens), to verify
+ *                   with mq_decode_attn
  *   mq_tune         on-device choice of the decode launch shape under a
  *                   wall-clock budget, accepting only bit-identical candidates
  *                   (or, on request, candidates within alpha times the output
@@ -314,6 +317,32 @@ mq_status mq_decode_attn_cascade(const mq_cache* cache, const void* q, mq_dtype 
                                  const int32_t* block_table, int32_t max_blocks_per_seq, const int32_t* seq_lens,
                                  const int32_t* n_q_per_seq, int32_t prefix_len, float softmax_scale, float* out,
                                  float* lse, void* workspace, size_t workspace_bytes, mq_stream stream);
+
+/* ---------------------------------------------------------------------------
+ * mq_draft_ngram: history-based drafting (speculative decoding).
+ *
+ * The deep dive (section 5, the drafting guarantees) lists history-based drafters
+ * among those whose draft step costs only the bytes they read; the drafts are then
+ * verified by one mq_decode_attn launch (n_q_per_seq = 1 + the number of drafts).
+ * The pages give no algorithm; this library's reading: for each sequence b with
+ * history tokens[b][0 .. L_b), find the most recent earlier occurrence of its last
+ * `ngram` tokens,
+ *   i* = max { i : 0 <= i < L_b - ngram, tokens[b][i + j] == tokens[b][L_b - ngram + j]
+ *              for every j < ngram },
+ * and propose the tokens that followed it:
+ *   drafts[b][j] = tokens[b][i* + ngram + j],  j < n_drafts[b] = min(max_draft, L_b - i* - ngram).
+ *   tokens     int32 [n_seqs][max_len] (device), token ids compared as int32 values
+ *   seq_lens   int32 [n_seqs] (device), L_b
+ *   drafts     int32 [n_seqs][max_draft] (device); entries at or past n_drafts[b]
+ *              are not written
+ *   n_drafts   int32 [n_seqs] (device): the count, 0 when nothing matches or
+ *              L_b <= ngram, -1 when L_b is outside [0, max_len]
+ * Runs one kernel on `stream` (the current device); reads each history once.
+ * Errors: INVALID_ARG (null pointers, max_len < 1, n_seqs < 1, ngram outside
+ * [1, 64], max_draft < 1), CUDA.
+ * ------------------------------------------------------------------------- */
+mq_status mq_draft_ngram(const int32_t* tokens, int32_t max_len, const int32_t* seq_lens, int32_t n_seqs,
+                         int32_t ngram, int32_t max_draft, int32_t* drafts, int32_t* n_drafts, mq_stream stream);
 
 /* ---------------------------------------------------------------------------
  * Launch configuration and tuning

@@ -14,6 +14,10 @@ header: the blog.123qwe.co.kr deep dive on magnitudedev/magnitude, section 5
 scale); the pages give no formula, so the exact arithmetic is a fixed reading
 of them, stated in the C file's header.
 
+``draft_ngram`` (history-based drafting, the deep dive's section 5 drafting
+guarantees) is pinned by hand-worked cases and a cross-check against Python's
+``bytes.rfind``.
+
 Parity status: quantization and dequantized attention are pinned by
 ``tests/test_oracle_*.py`` (hand-worked cases, brute force, closed forms,
 invariants, a library cross-check).  The error against unquantized attention is
@@ -71,6 +75,8 @@ class OracleLib:
         L.mqo_dequantize_v.argtypes = [P, P, i64, i32, P]
         L.mqo_attention_f64.argtypes = [P, P, P, i32, i32, i32, i32, i64, dbl, P, P, P, i32]
         L.mqo_attention_quant_f64.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i64, dbl, P, P, i32]
+        L.mqo_draft_ngram.argtypes = [P, i32, i32, i32, P]
+        L.mqo_draft_ngram.restype = i32
         L.mqo_max_threads.restype = i32
         for f in ("mqo_quantize_k", "mqo_quantize_v", "mqo_dequantize_k", "mqo_dequantize_v",
                   "mqo_attention_f64", "mqo_attention_quant_f64"):
@@ -163,6 +169,14 @@ class OracleLib:
                                        _p(out), _p(lse), int(n_threads))
         return out, lse
 
+    def draft_ngram(self, tokens, n: int, k: int) -> np.ndarray:
+        """History-based drafts: the up to k tokens that followed the most recent
+        earlier occurrence of the last n tokens of `tokens` (int32 [L])."""
+        t = _c(np.asarray(tokens), np.int32)
+        out = np.zeros(max(int(k), 1), np.int32)
+        cnt = self.L.mqo_draft_ngram(_p(t), int(t.shape[0]), int(n), int(k), _p(out))
+        return out[:cnt].copy()
+
     def max_threads(self) -> int:
         return int(self.L.mqo_max_threads())
 
@@ -219,6 +233,10 @@ def attention(q, k, v, scale, n_threads=1, return_weights=False):
 
 def attention_quant(q, kc, ks, vp, vs, scale, n_threads=1):
     return lib().attention_quant(q, kc, ks, vp, vs, scale, n_threads)
+
+
+def draft_ngram(tokens, n, k):
+    return lib().draft_ngram(tokens, n, k)
 
 
 def max_threads() -> int:

@@ -260,3 +260,26 @@ int mqo_max_threads(void) {
     return 1;
 #endif
 }
+
+/* ---- history-based drafting (n-gram lookup over the token history) -------------
+ * The deep dive (section 5, the drafting guarantees) lists history-based drafters
+ * among the drafters whose step costs only the bytes they read; it gives no
+ * algorithm.  Reading: propose the tokens that followed the most recent earlier
+ * occurrence of the history's last n tokens.
+ *   match i: 0 <= i < L - n and tokens[i + j] == tokens[L - n + j] for j < n
+ *   i* = the largest match; drafts[j] = tokens[i* + n + j] for j < min(k, L - i* - n)
+ * Returns the number of drafts (0 when L <= n or nothing matches).  Written as the
+ * definition: candidates from the latest down, the first full match wins.          */
+int mqo_draft_ngram(const int32_t* tokens, int32_t L, int32_t n, int32_t k, int32_t* drafts) {
+    if (L <= n || n < 1 || k < 1) return 0;
+    for (int32_t i = L - n - 1; i >= 0; i--) {
+        int same = 1;
+        for (int32_t j = 0; j < n && same; j++) same = tokens[i + j] == tokens[L - n + j];
+        if (!same) continue;
+        int32_t cnt = L - i - n;
+        if (cnt > k) cnt = k;
+        for (int32_t j = 0; j < cnt; j++) drafts[j] = tokens[i + n + j];
+        return cnt;
+    }
+    return 0;
+}

@@ -74,6 +74,7 @@ def _load():
         "mq_decode_cascade_workspace_bytes": ([P, i32, i32, i32, i32, i32, i32], sz),
         "mq_decode_attn_cascade": ([P, P, ctypes.c_int, i32, i32, i32, i32, i32, P, i32, P, P, i32, ctypes.c_float,
                                     P, P, P, sz, P], ctypes.c_int),
+        "mq_draft_ngram": ([P, i32, P, i32, i32, i32, P, P, P], ctypes.c_int),
         "mq_get_decode_config": ([P, i32, ctypes.POINTER(mq_decode_config)], ctypes.c_int),
         "mq_set_decode_config": ([P, i32, ctypes.POINTER(mq_decode_config)], ctypes.c_int),
         "mq_tune": ([P, ctypes.POINTER(mq_tune_params), ctypes.POINTER(mq_tune_result)], ctypes.c_int),
@@ -193,6 +194,12 @@ def mq_decode_attn_cascade(cache: int, q, q_dtype: int, n_seqs: int, n_q_heads: 
                                       max_seq_len, _ptr(block_table), max_blocks_per_seq, _ptr(seq_lens),
                                       _ptr(n_q_per_seq), prefix_len, float(softmax_scale), _ptr(out), _ptr(lse),
                                       _ptr(workspace), workspace_bytes, _stream(stream)), "mq_decode_attn_cascade")
+
+
+def mq_draft_ngram(tokens, max_len: int, seq_lens, n_seqs: int, ngram: int, max_draft: int, drafts, n_drafts,
+                   stream=None) -> None:
+    _check(lib.mq_draft_ngram(_ptr(tokens), max_len, _ptr(seq_lens), n_seqs, ngram, max_draft, _ptr(drafts),
+                              _ptr(n_drafts), _stream(stream)), "mq_draft_ngram")
 
 
 def mq_get_decode_config(cache: int, rows_class: int) -> tuple:

@@ -429,3 +429,47 @@ QUANT_CHECKS = [check_f16_hand, check_f16_vs_numpy, check_bf16_hand, check_k_han
 ATTN_CHECKS = [check_attn_single_token, check_attn_two_token_closed_form, check_attn_constant_v,
                check_attn_weights, check_attn_dominant_key, check_attn_torch, check_attn_causal,
                check_attn_gqa, check_attn_permutation, check_attn_quant_form]
+
+
+# ---- history-based drafting ------------------------------------------------------
+DRAFT_GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "draft_ngram_cases.json")
+
+
+def check_draft_hand(O):
+    """The hand-worked cases of tests/golden/draft_ngram_cases.json."""
+    with open(DRAFT_GOLDEN) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        got = O.draft_ngram(np.array(c["tokens"], np.int32), c["n"], c["k"]).tolist()
+        assert got == c["drafts"], (c, got)
+
+
+def _rfind_drafts(tokens, n, k):
+    """The same drafts found with bytes.rfind: each token (0 <= t < 250) is the 4-byte
+    word 0xFF t 0xFE 0xFD, so a byte match can only start on a token boundary; the
+    window must end before the last token, i.e. inside bytes [0, 4 (L - 1))."""
+    L = len(tokens)
+    if L <= n:
+        return []
+    enc = b"".join(bytes([0xFF, int(t), 0xFE, 0xFD]) for t in tokens)
+    at = enc.rfind(enc[4 * (L - n):], 0, 4 * (L - 1))
+    if at < 0:
+        return []
+    assert at % 4 == 0
+    i = at // 4
+    return [int(t) for t in tokens[i + n: min(i + n + k, L)]]
+
+
+def check_draft_rfind(O, trials=300, seed=11):
+    """Random short-alphabet histories (many repeats) against the bytes.rfind search."""
+    rng = np.random.default_rng(seed)
+    for _ in range(trials):
+        L = int(rng.integers(1, 200))
+        alpha = int(rng.integers(2, 6))
+        t = rng.integers(0, alpha, L).astype(np.int32)
+        n = int(rng.integers(1, 6))
+        k = int(rng.integers(1, 9))
+        assert O.draft_ngram(t, n, k).tolist() == _rfind_drafts(t, n, k), (t.tolist(), n, k)
+
+
+DRAFT_CHECKS = [check_draft_hand, check_draft_rfind]

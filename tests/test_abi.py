@@ -92,6 +92,10 @@ def test_null_arguments_rejected_before_cuda():
         == mq.MQ_ERR_INVALID_ARG
     assert mq.lib.mq_decode_workspace_bytes(None, 1, 8, 1, 16) == 0
     assert mq.lib.mq_decode_cascade_workspace_bytes(None, 1, 8, 1, 1, 64, 16) == 0
+    for bad in ((None, 8, 1, 1, 2, 1, 1), (1, 0, 1, 1, 2, 1, 1), (1, 8, 1, 0, 2, 1, 1), (1, 8, 1, 1, 0, 1, 1),
+                (1, 8, 1, 1, 65, 1, 1), (1, 8, 1, 1, 2, 0, 1)):
+        t, ml, sl, ns, n, k, d = bad
+        assert mq.lib.mq_draft_ngram(t, ml, sl, ns, n, k, d, 1, None) == mq.MQ_ERR_INVALID_ARG
     assert mq.lib.mq_decode_attn_cascade(None, 1, 1, 1, 8, 1, 1, 64, 1, 4, 1, 1, 16, 0.1, 16, None, 256, 1 << 20,
                                          None) == mq.MQ_ERR_INVALID_ARG
     assert mq.lib.mq_device_status(None, None) == mq.MQ_ERR_INVALID_ARG

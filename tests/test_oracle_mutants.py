@@ -36,6 +36,11 @@ MUTANTS = [
     ("lse_without_max", "lse[r] = m + log(l);\n        free(z);\n    }\n}\n\n/* Same attention",
      "lse[r] = log(l);\n        free(z);\n    }\n}\n\n/* Same attention"),
     ("absmax_signed", "float m = fabsf(x[c]);", "float m = x[c];"),
+    ("draft_earliest_match", "for (int32_t i = L - n - 1; i >= 0; i--) {", "for (int32_t i = 0; i < L - n; i++) {"),
+    ("draft_suffix_matches_itself", "for (int32_t i = L - n - 1; i >= 0; i--) {", "for (int32_t i = L - n; i >= 0; i--) {"),
+    ("draft_count_off_by_one", "int32_t cnt = L - i - n;", "int32_t cnt = L - i - n - 1;"),
+    ("draft_last_token_only", "for (int32_t j = 0; j < n && same; j++) same = tokens[i + j] == tokens[L - n + j];",
+     "same = tokens[i + n - 1] == tokens[L - 1];"),
 ]
 
 
@@ -44,7 +49,8 @@ def _checks():
     order = [P.check_k_hand, P.check_v_hand, P.check_dequant_hand, P.check_memory_claim,
              P.check_attn_single_token, P.check_attn_two_token_closed_form, P.check_attn_weights,
              P.check_attn_gqa, P.check_attn_causal, P.check_attn_torch, P.check_attn_quant_form,
-             P.check_roundtrip, P.check_tiny_scales, P.check_near_ties, P.check_k_bruteforce, P.check_v_bruteforce]
+             P.check_roundtrip, P.check_tiny_scales, P.check_near_ties, P.check_k_bruteforce, P.check_v_bruteforce,
+             P.check_draft_hand, P.check_draft_rfind]
     return order
 
 

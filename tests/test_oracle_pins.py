@@ -19,3 +19,8 @@ def test_quantization_pins(O, check):
 @pytest.mark.parametrize("check", P.ATTN_CHECKS, ids=lambda f: f.__name__)
 def test_attention_pins(O, check):
     check(O)
+
+
+@pytest.mark.parametrize("check", P.DRAFT_CHECKS, ids=lambda f: f.__name__)
+def test_drafting_pins(O, check):
+    check(O)
