@@ -23,7 +23,9 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("mq_cache_create", "mq_cache_destroy", "mq_kv_append", "mq_decode_attn", "mq_tune",
-              "mq_decode_workspace_bytes", "mq_status_string", "mq_device_status"):
+              "mq_decode_workspace_bytes", "mq_status_string", "mq_device_status", "mq_decode_attn_static",
+              "mq_decode_attn_cascade", "mq_decode_cascade_workspace_bytes", "mq_draft_ngram", "mq_tune_identity",
+              "mq_tune_store_get", "mq_tune_store_put", "mq_decode_kernel_count"):
         assert n in names
 
 
