@@ -423,12 +423,35 @@ def check_attn_quant_form(O):
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
+def check_attn_prefix_split(O):
+    """Attention over a whole cache equals the log-sum-exp merge of attention over a
+    prefix (every query sees all of it) and over the rest (causal among the drafts):
+    the identity the shared-prefix cascade rests on, and a pin on lse, which carries
+    the merge weights."""
+    rng = np.random.default_rng(23)
+    L, P, Hkv, D, n = 90, 48, 2, 128, 3
+    x = _x_data(24, L * Hkv, D).reshape(L, Hkv, D)
+    y = _x_data(25, L * Hkv, D).reshape(L, Hkv, D)
+    kc, ks = O.quantize_k(x)
+    vp, vs = O.quantize_v(y)
+    q = rng.standard_normal((n, 4, D))
+    o, l = O.attention_quant(q, kc, ks, vp, vs, 1 / math.sqrt(D))
+    o2, l2 = O.attention_quant(q, kc[P:], ks[P:], vp[P:], vs[P:], 1 / math.sqrt(D))
+    for j in range(n):
+        o1, l1 = O.attention_quant(q[j:j + 1], kc[:P], ks[:P], vp[:P], vs[:P], 1 / math.sqrt(D))
+        m = np.maximum(l1[0], l2[j])
+        w1, w2 = np.exp(l1[0] - m), np.exp(l2[j] - m)
+        om = (o1[0] * w1[:, None] + o2[j] * w2[:, None]) / (w1 + w2)[:, None]
+        lm = m + np.log(w1 + w2)
+        assert np.max(np.abs(om - o[j])) < 1e-12 and np.max(np.abs(lm - l[j])) < 1e-12
+
+
 QUANT_CHECKS = [check_f16_hand, check_f16_vs_numpy, check_bf16_hand, check_k_hand, check_v_hand,
                 check_dequant_hand, check_k_bruteforce, check_v_bruteforce, check_tiny_scales,
                 check_near_ties, check_roundtrip, check_memory_claim]
 ATTN_CHECKS = [check_attn_single_token, check_attn_two_token_closed_form, check_attn_constant_v,
                check_attn_weights, check_attn_dominant_key, check_attn_torch, check_attn_causal,
-               check_attn_gqa, check_attn_permutation, check_attn_quant_form]
+               check_attn_gqa, check_attn_permutation, check_attn_quant_form, check_attn_prefix_split]
 
 
 # ---- history-based drafting ------------------------------------------------------
