@@ -1,0 +1,53 @@
+"""bench.py's host logic without a GPU: the validity hash of the committed DRAM
+counters (comments and blank space do not count, code does) and the lookup that
+turns a stale or missing record into null."""
+import json
+import os
+import shutil
+
+import bench
+
+FILES = ("mq_decode.cu", "mq_device.cuh", "mq_tc.cuh", "mq_kernels.h")
+
+
+def _tree(tmp_path):
+    root = tmp_path / "repo"
+    d = root / "quantized_kv_decode_quantize_b200" / "csrc"
+    d.mkdir(parents=True)
+    for n in FILES:
+        shutil.copy(os.path.join(bench.ROOT, "quantized_kv_decode_quantize_b200", "csrc", n), d / n)
+    (root / "profiles").mkdir()
+    return root, d
+
+
+def test_hash_ignores_comments_and_blank_space(tmp_path, monkeypatch):
+    root, d = _tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    h0 = bench.kernel_source_hash()
+    p = d / "mq_decode.cu"
+    src = p.read_text()
+    p.write_text("// a new comment line\n/* and a block\n comment */\n" + src.replace("\n", "\n\n", 5))
+    assert bench.kernel_source_hash() == h0
+    p.write_text(src.replace("constexpr float kLazy = 4.0f;", "constexpr float kLazy = 5.0f;"))
+    assert bench.kernel_source_hash() != h0
+
+
+def test_traffic_record_is_null_when_stale_or_missing(tmp_path, monkeypatch):
+    root, d = _tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.ncu_traffic("long_decode_64k") is None                  # no record file
+    rec = {"long_decode_64k": {"dram_bytes_per_launch": 123, "kernel_source_hash": bench.kernel_source_hash()}}
+    (root / "profiles" / "ncu_traffic.json").write_text(json.dumps(rec))
+    assert bench.ncu_traffic("long_decode_64k") == 123
+    assert bench.ncu_traffic("tiny_decode_4k") is None                   # another workload
+    p = d / "mq_tc.cuh"
+    p.write_text(p.read_text() + "\nnamespace mq { constexpr int kChanged = 1; }\n")
+    assert bench.ncu_traffic("long_decode_64k") is None                  # the kernel changed
+
+
+def test_committed_record_names_the_bench_workload():
+    with open(os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")) as f:
+        rec = json.load(f)
+    e = rec["long_decode_64k"]
+    assert e["dram_bytes_per_launch"] == e["dram_bytes_read"] + e["dram_bytes_write"]
+    assert "--clock-control none" in e["command"]
