@@ -153,6 +153,15 @@ def ncu_traffic(workload_name: str):
 
 
 # ---------------------------------------------------------------------------------
+def graph_steps(copies: int, steps: int, override: int = 0) -> int:
+    """Steps captured in one CUDA graph: a whole number of rotations over the cache
+    copies (about 24 steps), but never more than the timed steps, so that the timed
+    region holds at least one replay and the events recorded around each decode call
+    inside it give the kernel duration at any --steps."""
+    S = override or copies * max(1, math.ceil(24 / copies))
+    return max(1, min(S, steps))
+
+
 def max_over_ranks(x: float, device) -> float:
     """The max of x over all ranks (identity without a process group)."""
     import torch
@@ -194,7 +203,7 @@ def run_reference(args, rank, world):
     import torch
 
     import oracle
-    from quantized_kv_decode_quantize_b200 import workloads as wl
+    import workloads as wl
 
     if rank != 0:
         return
@@ -245,9 +254,15 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(w, inp, steps_budget_s=20.0):
+def cpu_baseline(w, inp, gpu_out=None, gpu_lse=None, steps_budget_s=20.0):
     """The oracle as it stands, on all host cores: full decode steps of the workload
-    (every sequence, every head) until ~steps_budget_s of work; GB/s of KV read."""
+    (every sequence, every head) until ~steps_budget_s of work; GB/s of KV read.
+
+    The first step's oracle outputs also give the accuracy figures of the GPU result
+    (`gpu_out`, `gpu_lse`: numpy copies of the bench's last decode): max-abs error
+    against the oracle's fp64 attention over the same quantized cache (the parity
+    bar, 1e-3), and max-abs / relative-L2 error against fp64 attention over the
+    original, unquantized K/V (reported, not gated).  Returns (baseline, accuracy)."""
     import numpy as np
 
     import oracle
@@ -262,19 +277,41 @@ def cpu_baseline(w, inp, steps_budget_s=20.0):
     q = inp.q.float().numpy().astype(np.float64)
     qoff = np.concatenate([[0], np.cumsum(w.n_q)]).astype(int)
     scale = 1.0 / math.sqrt(w.head_dim)
+    ref_out = np.empty((w.total_q, w.n_q_heads, w.head_dim))
+    ref_lse = np.empty((w.total_q, w.n_q_heads))
     n = 0
     t0 = time.perf_counter()
     while True:
         for b in range(w.n_seqs):
-            oracle.attention_quant(q[qoff[b]: qoff[b + 1]], *codes[b], scale, cores)
+            o, l = oracle.attention_quant(q[qoff[b]: qoff[b + 1]], *codes[b], scale, cores)
+            if n == 0:
+                ref_out[qoff[b]: qoff[b + 1]], ref_lse[qoff[b]: qoff[b + 1]] = o, l
         n += 1
         if time.perf_counter() - t0 > steps_budget_s or n >= 50:
             break
     dt = time.perf_counter() - t0
-    return {"value": sum(w.seq_lens) * w.n_kv_heads * bpt * n / dt / 1e9, "unit": "GB/s", "cores": cores,
+    base = {"value": sum(w.seq_lens) * w.n_kv_heads * bpt * n / dt / 1e9, "unit": "GB/s", "cores": cores,
             "kind": "oracle",
             "sample": f"{n} full decode step(s) of {w.name} (all sequences and heads, fp64 attention over the "
                       f"quantized cache), {dt:.1f} s"}
+    acc = None
+    if gpu_out is not None:
+        unq = np.empty_like(ref_out)
+        for b in range(w.n_seqs):
+            o, _ = oracle.attention(q[qoff[b]: qoff[b + 1]], inp.seq_k(b).float().numpy(),
+                                    inp.seq_v(b).float().numpy(), scale, cores)
+            unq[qoff[b]: qoff[b + 1]] = o
+        d_q = np.abs(gpu_out - ref_out)
+        d_u = gpu_out - unq
+        acc = {"vs_oracle_quantized": {"max_abs_out": float(d_q.max()),
+                                       "max_abs_lse": float(np.abs(gpu_lse - ref_lse).max()),
+                                       "tolerance": 1e-3},
+               "vs_unquantized_fp64": {"max_abs_out": float(np.abs(d_u).max()),
+                                       "rel_l2_out": float(np.linalg.norm(d_u) / np.linalg.norm(unq)),
+                                       "note": "reported, not gated: K int8 / V int4 quantization error"},
+               "sample": f"every output of the bench's last decode step ({w.total_q} query token(s) x "
+                         f"{w.n_q_heads} q-heads x {w.head_dim})"}
+    return base, acc
 
 
 def run_mq(args, rank, world, local):
@@ -283,7 +320,7 @@ def run_mq(args, rank, world, local):
     import torch.distributed as dist
 
     import quantized_kv_decode_quantize_b200 as mq
-    from quantized_kv_decode_quantize_b200 import workloads as wl
+    import workloads as wl
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -365,7 +402,7 @@ def run_mq(args, rank, world, local):
             ev[1].record(stream)
 
     # ---- capture S steps (one rotation over the copies, or more) in a graph ----
-    S = args.graph_steps or copies * max(1, math.ceil(24 / copies))
+    S = graph_steps(copies, args.steps, args.graph_steps)
     stream = torch.cuda.Stream(dev)
     evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
            for _ in range(S)]
@@ -522,7 +559,9 @@ def run_mq(args, rank, world, local):
             "wall_s": wall1 - wall0,
         }
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(w, inp)
+            torch.cuda.synchronize(dev)
+            line["cpu_baseline"], line["accuracy"] = cpu_baseline(w, inp, out.cpu().numpy().astype(np.float64),
+                                                                  lse.cpu().numpy().astype(np.float64))
         print(json.dumps(line), flush=True)
     del g
     if world > 1:

@@ -5,6 +5,7 @@
  * inference engine whose KV cache stores keys as int8 and values as int4:
  *
  *   mq_kv_append    quantize-on-append of new K/V tokens into a paged cache
+ *   mq_kv_export    cached tokens read back in the codec's canonical packing
  *   mq_decode_attn  attention of a few query tokens per sequence (1 = decode,
  *                   n > 1 = verification of n speculative draft tokens, causal
  *                   among the drafts) against the cache, split over the
@@ -43,8 +44,11 @@
  *     IEEE fp32 division then rounded to fp16; code = clamp(rne(x / s), -127,
  *     127) with an IEEE fp32 division; s == 0 gives code 0.
  *   V, per (token, kv-head, 32 consecutive channels): s = fp16_rn(max|x| / 7),
- *     code = clamp(rne(x / s), -8, 7); two codes per byte, the even channel in
- *     the low nibble, two's complement nibbles.
+ *     code = clamp(rne(x / s), -8, 7), stored as 4-bit two's complement nibbles,
+ *     two per byte.  Which two codes share a byte is the page layout's choice
+ *     (below: the codes of one channel for two tokens); mq_kv_export writes the
+ *     codec's canonical packing, channel 2j in the low nibble of byte j and
+ *     channel 2j + 1 in the high nibble.
  *   Symmetric (no zero point).  NaN inputs give code 0; scales that overflow
  *     fp16 become +inf and give code 0 (inputs beyond 65504*127 for K or
  *     65504*7 for V are outside the codec's domain).
@@ -184,6 +188,38 @@ mq_status mq_kv_append(mq_cache* cache, const void* k, const void* v, mq_dtype d
                        const int32_t* block_table, int32_t max_blocks_per_seq, mq_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * mq_kv_export — cached tokens read back in the codec's canonical form
+ *
+ * The codec (deep dive, section 5: "Key 8-bit, Value 4-bit, group 32, f16
+ * scale") packs V codes two per byte; the page layout above groups them by
+ * channel for the decode kernel.  This call reads tokens back with V packed
+ * channel by channel, as the codec paragraph at the top of this header defines
+ * it, and copies codes and scales unchanged (no arithmetic on values): for
+ * offloading or inspecting a cache, and for checking it byte for byte.
+ *   cu_tok       int32 [n_seqs + 1], exclusive prefix sum of the tokens read per
+ *                sequence (like mq_kv_append's cu_new)
+ *   start_pos    int32 [n_seqs], position of sequence b's first token read
+ *   block_table  int32 [n_seqs][max_blocks_per_seq]
+ *   k_codes      out int8   [n_tokens][n_kv_heads][head_dim]
+ *   k_scales     out uint16 [n_tokens][n_kv_heads]          (fp16 bits)
+ *   v_packed     out uint8  [n_tokens][n_kv_heads][head_dim / 2]: byte j =
+ *                (code[2j] & 15) | (code[2j + 1] & 15) << 4
+ *   v_scales     out uint16 [n_tokens][n_kv_heads][head_dim / 32] (fp16 bits)
+ * All pointers are device pointers owned by the caller; asynchronous on
+ * `stream`.  Token i of sequence b is position start_pos[b] + i.  Reading a
+ * position no append has written returns whatever the pool holds there.
+ * Errors: INVALID_ARG (null pointers, n_seqs < 1 or > 65535, n_tokens < 0,
+ * max_blocks_per_seq < 1), CUDA.  n_tokens == 0 launches nothing.  A token
+ * outside its sequence's cu_tok range, a position outside [0,
+ * max_blocks_per_seq*16) or a block id outside [0, n_blocks) is not read: its
+ * outputs are zero and mq_device_status() reports MQ_ERR_DEVICE.
+ * ------------------------------------------------------------------------- */
+mq_status mq_kv_export(const mq_cache* cache, int32_t n_seqs, int32_t n_tokens, const int32_t* cu_tok,
+                       const int32_t* start_pos, const int32_t* block_table, int32_t max_blocks_per_seq,
+                       int8_t* k_codes, uint16_t* k_scales, uint8_t* v_packed, uint16_t* v_scales,
+                       mq_stream stream);
+
+/* ---------------------------------------------------------------------------
  * mq_decode_attn — attention of n_q_per_seq[b] query tokens of every sequence
  * against its quantized cache
  *
@@ -260,7 +296,9 @@ mq_status mq_decode_attn(const mq_cache* cache, const void* q, mq_dtype q_dtype,
  * The call launches the decode kernels on `stream` with the array as their
  * workspace.
  * Make the first call on each device before any stream capture that is to
- * contain a later call: that first call does the address lookup.
+ * contain a later call: that first call does the address lookup.  The lookup is
+ * repeated when the device's context has changed since (after cudaDeviceReset),
+ * so make the first call after a reset outside a capture too.
  * The scratch is shared by every call on a device: calls whose executions may
  * overlap (different streams or host threads without ordering between them)
  * race on it and give wrong results.  Order them, or use mq_decode_attn with a

@@ -65,6 +65,7 @@ def _load():
         "mq_cache_create": ([ctypes.POINTER(mq_cache_desc), ctypes.POINTER(P)], ctypes.c_int),
         "mq_cache_destroy": ([P], ctypes.c_int),
         "mq_kv_append": ([P, P, P, ctypes.c_int, i32, i32, P, P, P, i32, P], ctypes.c_int),
+        "mq_kv_export": ([P, i32, i32, P, P, P, i32, P, P, P, P, P], ctypes.c_int),
         "mq_decode_workspace_bytes": ([P, i32, i32, i32, i32], sz),
         "mq_decode_kernel_count": ([P, i32, i32, i32, i32], i32),
         "mq_decode_attn": ([P, P, ctypes.c_int, i32, i32, i32, i32, i32, P, i32, P, P, ctypes.c_float, P, P, P, sz, P],
@@ -152,6 +153,13 @@ def mq_kv_append(cache: int, k, v, dtype: int, n_seqs: int, n_tokens: int, cu_ne
                  max_blocks_per_seq: int, stream=None) -> None:
     _check(lib.mq_kv_append(cache, _ptr(k), _ptr(v), dtype, n_seqs, n_tokens, _ptr(cu_new), _ptr(start_pos),
                             _ptr(block_table), max_blocks_per_seq, _stream(stream)), "mq_kv_append")
+
+
+def mq_kv_export(cache: int, n_seqs: int, n_tokens: int, cu_tok, start_pos, block_table, max_blocks_per_seq: int,
+                 k_codes, k_scales, v_packed, v_scales, stream=None) -> None:
+    _check(lib.mq_kv_export(cache, n_seqs, n_tokens, _ptr(cu_tok), _ptr(start_pos), _ptr(block_table),
+                            max_blocks_per_seq, _ptr(k_codes), _ptr(k_scales), _ptr(v_packed), _ptr(v_scales),
+                            _stream(stream)), "mq_kv_export")
 
 
 def mq_decode_workspace_bytes(cache: int, n_seqs: int, n_q_heads: int, max_q_per_seq: int, max_seq_len: int) -> int:

@@ -261,6 +261,36 @@ mq_status mq_kv_append(mq_cache* c, const void* k, const void* v, mq_dtype dtype
                                                                                                : MQ_ERR_CUDA;
 }
 
+mq_status mq_kv_export(const mq_cache* c, int32_t n_seqs, int32_t n_tokens, const int32_t* cu_tok,
+                       const int32_t* start_pos, const int32_t* block_table, int32_t max_blocks_per_seq,
+                       int8_t* k_codes, uint16_t* k_scales, uint8_t* v_packed, uint16_t* v_scales,
+                       mq_stream stream) {
+    if (c == nullptr || n_seqs < 1 || n_seqs > 65535 || n_tokens < 0 || max_blocks_per_seq < 1)
+        return MQ_ERR_INVALID_ARG;
+    if (n_tokens == 0) return MQ_OK;
+    if (cu_tok == nullptr || start_pos == nullptr || block_table == nullptr || k_codes == nullptr ||
+        k_scales == nullptr || v_packed == nullptr || v_scales == nullptr)
+        return MQ_ERR_INVALID_ARG;
+    DevGuard guard(c->device);
+    ExportParams p{};
+    p.pool = static_cast<const uint8_t*>(c->pool);
+    p.n_kv_heads = c->n_kv_heads;
+    p.n_blocks = c->n_blocks;
+    p.n_seqs = n_seqs;
+    p.n_tokens = n_tokens;
+    p.cu_tok = cu_tok;
+    p.start_pos = start_pos;
+    p.block_table = block_table;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.k_codes = k_codes;
+    p.k_scales = k_scales;
+    p.v_packed = v_packed;
+    p.v_scales = v_scales;
+    p.err = c->err_word;
+    return launch_export(p, c->head_dim, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MQ_OK
+                                                                                               : MQ_ERR_CUDA;
+}
+
 size_t mq_decode_workspace_bytes(const mq_cache* c, int32_t n_seqs, int32_t n_q_heads, int32_t max_q_per_seq,
                                  int32_t max_seq_len) {
     if (c == nullptr || n_seqs < 1 || n_q_heads < 1 || n_q_heads % c->n_kv_heads != 0 || max_q_per_seq < 1 ||

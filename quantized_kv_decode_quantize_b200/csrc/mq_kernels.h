@@ -23,6 +23,25 @@ struct AppendParams {
 
 cudaError_t launch_append(const AppendParams& p, int head_dim, cudaStream_t st);
 
+struct ExportParams {
+    const uint8_t* pool;
+    int n_kv_heads;
+    long long n_blocks;
+    int n_seqs;
+    int n_tokens;
+    const int32_t* cu_tok;
+    const int32_t* start_pos;
+    const int32_t* block_table;
+    int max_blocks_per_seq;
+    int8_t* k_codes;
+    uint16_t* k_scales;
+    uint8_t* v_packed;
+    uint16_t* v_scales;
+    unsigned* err;
+};
+
+cudaError_t launch_export(const ExportParams& p, int head_dim, cudaStream_t st);
+
 struct DecodeParams {
     const uint8_t* pool;
     int n_kv_heads;

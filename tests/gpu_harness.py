@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import quantized_kv_decode_quantize_b200 as mq
-from quantized_kv_decode_quantize_b200 import workloads as wl
+import workloads as wl
 from tests import pagelayout
 
 DT = {"f32": mq.MQ_F32, "bf16": mq.MQ_BF16}

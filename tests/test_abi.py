@@ -25,7 +25,7 @@ def test_header_declares_the_entry_points():
     for n in ("mq_cache_create", "mq_cache_destroy", "mq_kv_append", "mq_decode_attn", "mq_tune",
               "mq_decode_workspace_bytes", "mq_status_string", "mq_device_status", "mq_decode_attn_static",
               "mq_decode_attn_cascade", "mq_decode_cascade_workspace_bytes", "mq_draft_ngram", "mq_tune_identity",
-              "mq_tune_store_get", "mq_tune_store_put", "mq_decode_kernel_count"):
+              "mq_tune_store_get", "mq_tune_store_put", "mq_decode_kernel_count", "mq_kv_export"):
         assert n in names
 
 
@@ -90,6 +90,7 @@ def test_null_arguments_rejected_before_cuda():
     assert mq.lib.mq_cache_create(None, None) == mq.MQ_ERR_INVALID_ARG
     assert mq.lib.mq_cache_destroy(None) == mq.MQ_OK
     assert mq.lib.mq_kv_append(None, 1, 1, 1, 1, 1, 1, 1, 1, 1, None) == mq.MQ_ERR_INVALID_ARG
+    assert mq.lib.mq_kv_export(None, 1, 1, 1, 1, 1, 1, 1, 1, 1, 1, None) == mq.MQ_ERR_INVALID_ARG
     assert mq.lib.mq_decode_attn(None, 1, 1, 1, 8, 1, 1, 16, 1, 1, 1, 1, 0.1, 16, None, 256, 1 << 20, None) \
         == mq.MQ_ERR_INVALID_ARG
     assert mq.lib.mq_decode_workspace_bytes(None, 1, 8, 1, 16) == 0

@@ -51,3 +51,17 @@ def test_committed_record_names_the_bench_workload():
     e = rec["long_decode_64k"]
     assert e["dram_bytes_per_launch"] == e["dram_bytes_read"] + e["dram_bytes_write"]
     assert "--clock-control none" in e["command"]
+
+
+def test_graph_never_longer_than_the_timed_steps():
+    """The kernel events live inside graph replays: at any --steps the timed region
+    must hold at least one whole replay (the driver times 20 steps against a default
+    graph of 24)."""
+    for copies in (2, 3, 6, 8):
+        for steps in (1, 3, 5, 20, 23, 24, 25, 200, 20000):
+            S = bench.graph_steps(copies, steps)
+            assert 1 <= S <= steps
+            assert divmod(steps, S)[0] >= 1
+    assert bench.graph_steps(6, 20000) == 24
+    assert bench.graph_steps(6, 20) == 20
+    assert bench.graph_steps(6, 20000, override=12) == 12

@@ -1,11 +1,13 @@
-"""mq_kv_append (CUDA) against the CPU oracle: codes and scales must match bit for bit."""
+"""mq_kv_append (CUDA) against the CPU oracle: codes and scales must match bit for bit,
+and so must the packed V bytes in the codec's canonical packing (read back through
+mq_kv_export)."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import quantized_kv_decode_quantize_b200 as mq
-from quantized_kv_decode_quantize_b200 import workloads as wl
+import workloads as wl
 from tests import oracle_pins, pagelayout
 from tests.gpu_harness import GpuCase, oracle_codes
 
@@ -19,6 +21,60 @@ def _assert_seq_equal(case, b):
     assert np.array_equal(ks, eks), "K scales differ"
     assert np.array_equal(vp, evp), "V codes differ"
     assert np.array_equal(vs, evs), "V scales differ"
+
+
+def export_sequence(case, b, copy=0):
+    """Every token of sequence b through mq_kv_export (one call, one sequence)."""
+    w = case.w
+    L = w.seq_lens[b]
+    H, D = w.n_kv_heads, w.head_dim
+    i32 = dict(dtype=torch.int32, device="cuda")
+    kc = torch.empty((L, H, D), dtype=torch.int8, device="cuda")
+    ks = torch.empty((L, H), dtype=torch.int16, device="cuda")
+    vp = torch.empty((L, H, D // 2), dtype=torch.uint8, device="cuda")
+    vs = torch.empty((L, H, D // 32), dtype=torch.int16, device="cuda")
+    mq.mq_kv_export(case.cache.handle, 1, L, torch.tensor([0, L], **i32), torch.tensor([0], **i32),
+                    case.tabs[copy][b:b + 1].contiguous(), w.max_blocks(), kc, ks, vp, vs)
+    return (kc.cpu().numpy(), ks.cpu().numpy().view(np.uint16), vp.cpu().numpy(),
+            vs.cpu().numpy().view(np.uint16))
+
+
+def _assert_export_equal(case, b):
+    kc, ks, vp, vs = export_sequence(case, b)
+    ekc, eks, evp, evs = oracle_codes(case.inp, b)
+    assert np.array_equal(kc, ekc), "exported K codes differ"
+    assert np.array_equal(ks, eks), "exported K scales differ"
+    assert np.array_equal(vp, evp), "exported packed V bytes differ from the oracle's packing"
+    assert np.array_equal(vs, evs), "exported V scales differ"
+
+
+@pytest.mark.parametrize("name", ["tiny", "long", "prefix", "verify", "mixed"])
+def test_export_packed_bytes_bit_exact(name):
+    """The codec's byte contract end to end: quantize-on-append, then the packed bytes
+    read back in the canonical packing equal the oracle's packed bytes."""
+    w = wl.reduced(name)
+    case = GpuCase(w)
+    for b in range(w.n_seqs):
+        _assert_export_equal(case, b)
+    assert case.status() == mq.MQ_OK
+
+
+def test_export_bad_position_is_flagged_and_zeroed():
+    w = wl.reduced("long")
+    case = GpuCase(w)
+    i32 = dict(dtype=torch.int32, device="cuda")
+    H, D = w.n_kv_heads, w.head_dim
+    kc = torch.full((2, H, D), 7, dtype=torch.int8, device="cuda")
+    ks = torch.full((2, H), 7, dtype=torch.int16, device="cuda")
+    vp = torch.full((2, H, D // 2), 7, dtype=torch.uint8, device="cuda")
+    vs = torch.full((2, H, D // 32), 7, dtype=torch.int16, device="cuda")
+    mq.mq_kv_export(case.cache.handle, 1, 2, torch.tensor([0, 2], **i32),
+                    torch.tensor([w.max_blocks() * 16 - 1], **i32), case.tabs[0][:1].contiguous(), w.max_blocks(),
+                    kc, ks, vp, vs)
+    assert case.status() == mq.MQ_ERR_DEVICE
+    # the first token is in range, the second is not: zeros there
+    assert int(kc[1].abs().sum()) == 0 and int(vp[1].sum()) == 0 and int(ks[1].abs().sum()) == 0
+    assert int(vs[1].abs().sum()) == 0
 
 
 @pytest.mark.parametrize("name", ["tiny", "long", "prefix", "verify", "mixed"])
@@ -40,6 +96,7 @@ def test_append_full_size_bit_exact(name):
     seqs = range(w.n_seqs) if name == "long" else range(0, w.n_seqs, 3)
     for b in seqs:
         _assert_seq_equal(case, b)
+        _assert_export_equal(case, b)
 
 
 @pytest.mark.parametrize("D", [128, 256])

@@ -8,7 +8,7 @@ import torch
 
 import oracle
 import quantized_kv_decode_quantize_b200 as mq
-from quantized_kv_decode_quantize_b200 import workloads as wl
+import workloads as wl
 from tests.gpu_harness import GpuCase, oracle_outputs
 
 pytestmark = pytest.mark.gpu

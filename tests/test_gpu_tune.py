@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import quantized_kv_decode_quantize_b200 as mq
-from quantized_kv_decode_quantize_b200 import workloads as wl
+import workloads as wl
 from tests.gpu_harness import GpuCase
 
 pytestmark = pytest.mark.gpu

@@ -2,7 +2,7 @@
 import numpy as np
 import torch
 
-from quantized_kv_decode_quantize_b200 import workloads as wl
+import workloads as wl
 
 
 def test_inputs_are_deterministic_and_shaped():
