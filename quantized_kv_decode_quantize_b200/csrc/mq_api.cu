@@ -62,7 +62,9 @@ DevGuard::~DevGuard() {
 static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int rows_total, int max_seq_len) {
     DecodePlan pl{};
     pl.cls = cls;
-    pl.rows = rows_class_rows(c->head_dim, pl.cls);
+    // class 0 runs 4-row blocks when every block holds at most 4 real rows (grouped-query
+    // decode at GQA <= 4 with one query token)
+    pl.rows = (cls == 0 && rows_total <= 4) ? 4 : rows_class_rows(c->head_dim, pl.cls);
     pl.n_rb = (rows_total + pl.rows - 1) / pl.rows;
     const mq_decode_config cfg = c->cfg[pl.cls];
     const long long max_chunks = std::max<long long>(1, (max_seq_len + kChunkTokens - 1) / kChunkTokens);
@@ -149,8 +151,9 @@ mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void
 
 cudaError_t ensure_decode_smem(int device, int head_dim, int rows, size_t smem) {
     // raised limit per (device, kernel variant); the attribute only grows
-    static size_t done[64][2][3] = {};
-    const int di = device & 63, hi = head_dim == 128 ? 0 : 1, ri = rows == 8 ? 0 : (rows == 16 ? 1 : 2);
+    static size_t done[64][2][4] = {};
+    const int di = device & 63, hi = head_dim == 128 ? 0 : 1;
+    const int ri = rows == 4 ? 0 : (rows == 8 ? 1 : (rows == 16 ? 2 : 3));
     if (done[di][hi][ri] >= smem) return cudaSuccess;
     cudaError_t e = decode_prepare(head_dim, rows, smem);
     if (e == cudaSuccess) done[di][hi][ri] = smem;

@@ -37,12 +37,7 @@
 // programmatic dependent launch; it writes out and lse.  A unit that is not split writes
 // them here.  The chunk ranges depend only on the shape, the SM count and the configured
 // splits per SM, so the result is bit-identical for every ring depth.
-#include <cfloat>
-#include <climits>
-
-#include "mq_device.cuh"
-#include "mq_kernels.h"
-#include "mq_tc.cuh"
+#include "mq_decode_common.cuh"
 
 namespace mq {
 
@@ -57,7 +52,7 @@ struct Tc {
     static constexpr int H = D / 128;                             // 128-channel halves (PV M tiles)
     static constexpr int NQ = (3 * ROWS + 15) / 16 * 16;          // score MMA N: 3 limbs x rows
     static constexpr int NO = 4 * ROWS;                           // value MMA N per half
-    static constexpr int NB = ((G + 1) * ROWS + 15) / 16 * 16;    // weight columns: W_0..W_{G-1}, p
+    static constexpr int NB = G * ROWS;                           // weight columns: W_0 .. W_{G-1}
     // One CTA per SM owns all of tensor memory.  Every hand-off between the roles is
     // buffered as deeply as tensor and shared memory allow, so that several chunks are
     // in flight in each stage and the latency of an MMA (issue to commit) is hidden.
@@ -66,11 +61,12 @@ struct Tc {
     // each other's latencies better than deeper buffers in one.
     static constexpr int CPS = (D == 128 && ROWS == 8) ? 2 : 1;
     static constexpr int TCOLS = CPS == 2 ? 256 : 512;                           // TMEM columns allocated
-    // With two CTAs per SM (256 columns each) one score buffer leaves room for two V^T
-    // buffers, so that converting chunk i + 1 overlaps the value MMAs of chunk i.
-    static constexpr int NSB = CPS == 2 ? 1 : ((D == 128 && ROWS <= 16) ? 4 : (ROWS == 32 ? 1 : 2));   // score buffers (TMEM)
-    static constexpr int NVB = CPS == 2 ? 2 : ((D == 256 && ROWS == 16) ? 1 : 2);  // V^T buffers (TMEM)
-    static constexpr int NWB = CPS == 2 ? 2 : ((ROWS == 32 || (D == 256 && ROWS == 16)) ? 2 : 3);  // weight buffers (smem)
+    // Two score buffers let the score MMAs of chunk i + 1 run while the softmax still
+    // reads chunk i; two V^T buffers let the conversion of chunk i + 1 overlap the value
+    // MMAs of chunk i.
+    static constexpr int NSB = CPS == 2 ? 2 : ((D == 128 && ROWS <= 16) ? 4 : 2);   // score buffers (TMEM)
+    static constexpr int NVB = 2;                                                // V^T buffers (TMEM)
+    static constexpr int NWB = CPS == 2 ? 2 : 3;                                 // weight buffers (smem)
     static constexpr int NPB = NWB > NVB ? NWB : NVB;                            // value-MMA completion barriers
     // Softmax warp groups: the 32-row class splits its rows over two groups of four warps
     // (one warp per TMEM lane quadrant each); rows interact only through the chunk maximum
@@ -82,18 +78,17 @@ struct Tc {
     // tensor-memory columns
     static constexpr int T_S = 0;
     static constexpr int T_O = NSB * NQ;
-    static constexpr int T_SUM = T_O + H * NO;
-    static constexpr int T_VT = (T_SUM + NB + 31) / 32 * 32;
+    static constexpr int T_VT = (T_O + H * NO + 31) / 32 * 32;
     static constexpr int T_END = T_VT + NVB * H * 64;
     static constexpr int WBYTES = kChunkTokens * NB * 2;          // one weight buffer
     static constexpr int LBO_W = NB / 8 * 128;                    // its 8-token group stride
     static constexpr int PART = ROWS * D + 2 * ROWS;              // floats of one partial
     static_assert(T_END <= TCOLS, "tensor memory budget");
-    static_assert(NQ <= 256 && NB <= 256 && NO <= 256, "MMA N range");
+    static_assert(NQ <= 256 && NO <= 256, "MMA N range");
 };
 
 struct Smem {
-    size_t ring, wbuf, qlimb, fmat, part, xch, crow, lim, pgbad, mbar, misc, total;
+    size_t ring, wbuf, qlimb, part, xch, xsv, crow, lim, pgbad, mbar, misc, total;
 };
 
 // NS = ring stages (chunks of 8 pages)
@@ -115,11 +110,11 @@ __host__ __device__ inline Smem smem_layout(int NS) {
     off = al(off, 128);
     s.qlimb = off;
     off += (size_t)T::NQ * D;
-    off = al(off, 128);
-    s.fmat = off;
-    off += 4096;
-    s.xch = off;
-    off += (size_t)2 * ROWS * 4 * 4;
+    off = al(off, 16);
+    s.xch = off;                            // [3][ROWS][4 warps] chunk row maxima (2), row sums of p
+    off += (size_t)3 * ROWS * 4 * 4;
+    s.xsv = off;                            // [2][groups][4 warps] chunk V-scale maxima
+    off += (size_t)2 * 2 * 4 * 4;
     s.crow = off;
     off += (size_t)ROWS * 4;
     s.lim = off;
@@ -135,72 +130,6 @@ __host__ __device__ inline Smem smem_layout(int NS) {
     return s;
 }
 
-// ---- merge of two partial results (one binary-tree node) ------------------
-__device__ __forceinline__ void merge_coef(float ml, float ll, float mr, float lr, float& m, float& l, float& a,
-                                           float& b) {
-    m = fmaxf(ml, mr);
-    a = (ml == m) ? 1.0f : ex2(__fsub_rn(ml, m));
-    b = (mr == m) ? 1.0f : ex2(__fsub_rn(mr, m));
-    l = __fadd_rn(__fmul_rn(ll, a), __fmul_rn(lr, b));
-}
-__device__ __forceinline__ float merge_val(float ol, float orr, float a, float b) {
-    return __fadd_rn(__fmul_rn(ol, a), __fmul_rn(orr, b));
-}
-
-template <typename T>
-__device__ __forceinline__ float ld_f32(const void* base, size_t i);
-template <>
-__device__ __forceinline__ float ld_f32<float>(const void* base, size_t i) {
-    return __ldg(reinterpret_cast<const float*>(base) + i);
-}
-template <>
-__device__ __forceinline__ float ld_f32<__nv_bfloat16>(const void* base, size_t i) {
-    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
-}
-template <>
-__device__ __forceinline__ float ld_f32<__half>(const void* base, size_t i) {
-    return __half2float(reinterpret_cast<const __half*>(base)[i]);
-}
-
-__device__ __forceinline__ float load_q(const DecodeParams& p, size_t i) {
-    if (p.q_dtype == 0) return ld_f32<float>(p.q, i);
-    if (p.q_dtype == 1) return ld_f32<__nv_bfloat16>(p.q, i);
-    return ld_f32<__half>(p.q, i);
-}
-
-__device__ __forceinline__ void stsa128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
-}
-__device__ __forceinline__ uint32_t ldsa16(uint32_t a) {
-    unsigned short v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ float h_bits_to_f32(uint32_t bits) {
-    return __half2float(__ushort_as_half((unsigned short)bits));
-}
-
-// Slow paths of the decode kernel's waits (out of line).  wait_slow_warp: the whole
-// warp; `done` is this lane's result of the first test.  A timeout raises the CTA's
-// abort flag and the device error word.
-__device__ __noinline__ bool wait_slow_warp(uint32_t bar, uint32_t parity, bool spin, bool done,
-                                            volatile int* abort_flag, unsigned* err) {
-    bool ok = done || (*abort_flag == 0 && (spin ? mbar_wait_spin(bar, parity) : mbar_wait_bounded(bar, parity)));
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok && (threadIdx.x & 31) == 0) {
-        if (*abort_flag == 0) atomicOr(err, kErrTimeout);
-        *abort_flag = 1;
-    }
-    return ok;
-}
-__device__ __noinline__ bool wait_slow_one(uint32_t bar, uint32_t parity, volatile int* abort_flag, unsigned* err) {
-    if (*abort_flag != 0) return false;
-    if (mbar_wait_spin(bar, parity)) return true;
-    atomicOr(err, kErrTimeout);
-    *abort_flag = 1;
-    return false;
-}
-
 template <int ROWS>
 struct AlphaRows {
     float a[ROWS];
@@ -213,15 +142,15 @@ struct AlphaRows {
 };
 
 // Multiplies this warp's 32 TMEM lanes of the value accumulators (NO columns from t_o)
-// and of the column sums (NS columns from t_sum) by the factor of each column's row
-// (column j holds row j % ROWS), for the RPG rows from row rlo (a softmax warp group's
-// rows; al holds their factors).  Out of line: it runs only when a running max moves.
-template <int ROWS, int RPG, int NO, int NS>
-__device__ __noinline__ void rescale_acc(uint32_t lane_base, int t_o, int t_sum, int rlo, AlphaRows<RPG> al) {
+// by the factor of each column's row (column j holds row j % ROWS), for the RPG rows
+// from row rlo (a softmax warp group's rows; al holds their factors).  Out of line: it
+// runs only when a running max moves.
+template <int ROWS, int RPG, int NO>
+__device__ __noinline__ void rescale_acc(uint32_t lane_base, int t_o, int rlo, AlphaRows<RPG> al) {
 #pragma unroll 1
-    for (int cb = 0; cb < (NO + NS) / 8; cb++) {
-        const int col = cb < NO / 8 ? t_o + 8 * cb : t_sum + 8 * cb - NO;
-        const int r0 = (8 * cb) % ROWS - rlo;   // NO, NS, ROWS and rlo are multiples of 8
+    for (int cb = 0; cb < NO / 8; cb++) {
+        const int col = t_o + 8 * cb;
+        const int r0 = (8 * cb) % ROWS - rlo;   // NO, ROWS and rlo are multiples of 8
         if (r0 < 0 || r0 >= RPG) continue;      // another group's rows
         uint32_t v[8];
         tmem_ld8(lane_base + (uint32_t)col, v);
@@ -290,21 +219,16 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
 
     // A bounded wait that the whole warp agrees on; a timeout raises the CTA's abort
     // flag (every role then stops taking new work) and the device error word.  The
-    // softmax warps and the two MMA-issuing threads (the critical path) spin; the other
+    // softmax warps and the two MMA-issuing warps (the critical path) spin; the other
     // roles sleep in hardware while they wait, leaving the issue slots to the warps that
     // compute.  The fast path (already complete) is one test and a vote; the rest is
     // out of line, keeping the role loops small in the instruction cache.
-    const bool spin_waits = warp >= 7;
+    const bool spin_waits = warp >= 7 || warp == 1 || warp == 2;
     auto wait_warp = [&](uint32_t bar, uint32_t parity) -> bool {
         const bool done = mbar_test_wait(bar, parity);
         if (__all_sync(FULL, done)) return true;
         return wait_slow_warp(bar, parity, spin_waits, done, abort_flag, p.err);
     };
-    auto wait_one = [&](uint32_t bar, uint32_t parity) -> bool {   // single thread (the MMA issuers: spin)
-        if (mbar_test_wait(bar, parity)) return true;
-        return wait_slow_one(bar, parity, abort_flag, p.err);
-    };
-
     // ---- set-up: barriers, query-row offset, TMEM, constant operands ----
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; s++) {
@@ -333,69 +257,13 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
         tmem_relinquish();
         tc_fence_before();
     }
-    if (warp >= 3 && warp < 7) {
-        // the all-ones A operand of the sum MMA, and the zero padding rows of the limb operand
-        const int tid = threadIdx.x - 96;
-        uint4* f = reinterpret_cast<uint4*>(smem + S.fmat);
-        for (int i = tid; i < 256; i += 128) f[i] = make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
-        uint4* z = reinterpret_cast<uint4*>(smem + S.qlimb + (size_t)3 * ROWS * D);
-        for (int i = tid; i < (T::NQ - 3 * ROWS) * D / 16; i += 128) z[i] = make_uint4(0u, 0u, 0u, 0u);
-        fence_proxy_async_smem();
-    }
     __syncthreads();
     const int qoff = misc[0];
 
-    // ---- q -> three signed 8-bit limbs of a 23-bit fixed-point value per row ----
-    // Q = rint(q * 2^(22 - E)) with |q| < 2^E the row's absmax bound, |Q| <= 2^22, and
-    // Q = l2 * 2^16 + l1 * 2^8 + l0 with l0, l1 in [-128, 127] and |l2| <= 65.  Limb k
-    // of row r is row k * ROWS + r of the N x D (K-major) score operand.
+    // ---- q -> three signed 8-bit limbs per row (the score MMA's B operand) ----
     if (warp >= 7) {
-        const int tid = threadIdx.x - 224;
-        constexpr int SL = D / 8;   // 8-channel slices of a row
-        for (int it = tid; it < ROWS * SL; it += 128 * T::NSG) {
-            const int r = it / SL, sl = it % SL;
-            const bool real = r < rows_here;
-            const int rr = row0 + r, j = real ? rr / p.group : 0, hq = real ? rr % p.group : 0;
-            const long long qrow = (long long)qoff + j;
-            const bool qok = real && qrow < p.total_q;
-            if (real && !qok && sl == 0) atomicOr(p.err, kErrBadRow);
-            const size_t base = ((size_t)qrow * p.n_q_heads + (size_t)hk * p.group + hq) * D + (size_t)8 * sl;
-            float qv[8];
-            float amax = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 8; e++) {
-                qv[e] = qok ? load_q(p, base + e) : 0.0f;
-                amax = fmaxf(amax, fabsf(qv[e]));
-            }
-#pragma unroll
-            for (int o = 1; o < SL; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
-            int E = 0;
-            if (amax > 0.0f) frexpf(amax, &E);   // amax < 2^E
-            const bool zero_row = !(amax >= 0x1p-100f);
-            const float up = zero_row ? 0.0f : ldexpf(1.0f, 22 - E);
-            if (sl == 0) {
-                crow_s[r] = zero_row ? 0.0f : ldexpf(p.scale_log2, E - 22);
-                lim_s[r] = (real && p.causal) ? (L - nq + j + 1) : L;
-            }
-            uint32_t w[3][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}};
-#pragma unroll
-            for (int e = 0; e < 8; e++) {
-                const int Q = (int)rintf(__fmul_rn(qv[e], up));
-                const int l0 = ((Q + 128) & 255) - 128;
-                const int Q1 = (Q - l0) >> 8;
-                const int l1 = ((Q1 + 128) & 255) - 128;
-                const int l2 = (Q1 - l1) >> 8;
-                w[0][e / 4] |= (uint32_t)(l2 & 255) << (8 * (e % 4));
-                w[1][e / 4] |= (uint32_t)(l1 & 255) << (8 * (e % 4));
-                w[2][e / 4] |= (uint32_t)(l0 & 255) << (8 * (e % 4));
-            }
-#pragma unroll
-            for (int k = 0; k < 3; k++) {
-                const int n = k * ROWS + r;
-                const size_t off = (size_t)(n / 8) * (8 * D) + (size_t)(sl / 2) * 128 + (n % 8) * 16 + (sl % 2) * 8;
-                *reinterpret_cast<uint2*>(smem + S.qlimb + off) = make_uint2(w[k][0], w[k][1]);
-            }
-        }
+        q_to_limbs<D, ROWS, T::NQ>(p, smem + S.qlimb, crow_s, lim_s, threadIdx.x - 224, 128 * T::NSG, row0, rows_here,
+                                   qoff, L, nq, hk);
         fence_proxy_async_smem();
     }
     // the TMA producer starts at once; the other warps wait for the limbs and TMEM
@@ -449,60 +317,66 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
         if (*abort_flag != 0 && lane == 0)
             for (int k = max(0, issued - NS); k < issued; k++) mbar_wait_bounded(full_b(k % NS), (uint32_t)(k / NS) & 1u);
     } else if (warp == 1) {
-        // ================= score MMAs (one thread) =================
-        if (lane == 0) {
-            const uint32_t ql = smem_u32(smem + S.qlimb);
-            constexpr uint32_t IDQ = instr_desc(2, 1, 1, 0, 0, 128, T::NQ);   // s32 <- s8 x s8, K-major
-            uint32_t last_bar = 0, last_par = 0;
-            for (int i = 0; i < n_ck; i++) {
-                const int s = i % NS, sb = i % T::NSB;
-                if (!wait_one(full_b(s), (uint32_t)(i / NS) & 1u)) break;
-                if (i >= T::NSB && !wait_one(sfree_b + 8 * sb, (uint32_t)((i - T::NSB) / T::NSB) & 1u)) break;
-                tc_fence_after();
-                const uint32_t a0 = ring + (uint32_t)(s * kChunkPages * T::PB);
+        // ================= score MMAs (whole warp; one elected lane issues) =================
+        // The loop runs in step on all 32 lanes and every operand is computed the same way
+        // on each, so that the MMAs issue back to back (a single-lane loop waits about two
+        // hundred cycles per MMA).
+        const uint32_t ql = smem_u32(smem + S.qlimb);
+        constexpr uint32_t IDQ = instr_desc(2, 1, 1, 0, 0, 128, T::NQ);   // s32 <- s8 x s8, K-major
+        const uint64_t dq = smem_desc(ql, 128, 8 * D);
+        uint32_t last_bar = 0, last_par = 0;
+        int s = 0;
+        uint32_t ph = 0;   // ring stage of chunk i and the parity of its fill
+        for (int i = 0; i < n_ck; i++) {
+            const int sb = i % T::NSB;
+            if (!wait_warp(full_b(s), ph)) break;
+            if (i >= T::NSB && !wait_warp(sfree_b + 8 * sb, (uint32_t)((i - T::NSB) / T::NSB) & 1u)) break;
+            tc_fence_after();
+            const uint64_t da = smem_desc(ring + (uint32_t)(s * kChunkPages * T::PB), 128, T::REC);
+            const uint32_t dst = tmem + T::T_S + sb * T::NQ;
 #pragma unroll
-                for (int k = 0; k < D / 32; k++)
-                    mma_i8_ss(tmem + T::T_S + sb * T::NQ, smem_desc(a0 + 256 * k, 128, T::REC),
-                              smem_desc(ql + 256 * k, 128, 8 * D), IDQ, k > 0 ? 1u : 0u);
-                tc_commit(sfull_b + 8 * sb);
-                tc_commit(empty_b(s));
-                last_bar = sfull_b + 8 * sb;
-                last_par = (uint32_t)(i / T::NSB) & 1u;
+            for (int k = 0; k < D / 32; k++) mma_i8_ss_w(dst, da + 16 * k, dq + 16 * k, IDQ, k > 0 ? 1u : 0u);
+            tc_commit_w(sfull_b + 8 * sb);
+            tc_commit_w(empty_b(s));
+            last_bar = sfull_b + 8 * sb;
+            last_par = (uint32_t)(i / T::NSB) & 1u;
+            if (++s == NS) {
+                s = 0;
+                ph ^= 1u;
             }
-            // after an abort: the MMAs already issued finish before TMEM is released
-            if (*abort_flag != 0 && last_bar != 0) mbar_wait_bounded(last_bar, last_par);
         }
+        // after an abort: the MMAs already issued finish before TMEM is released
+        if (lane == 0 && *abort_flag != 0 && last_bar != 0) mbar_wait_bounded(last_bar, last_par);
         __syncwarp();
     } else if (warp == 2) {
-        // ================= value MMAs (one thread) =================
-        if (lane == 0) {
-            const uint32_t wb0 = smem_u32(smem + S.wbuf);
-            constexpr uint32_t IDO = instr_desc(1, 0, 0, 0, 1, 128, T::NO);   // f32 <- f16 x f16, B MN-major
-            constexpr uint32_t IDS = instr_desc(1, 0, 0, 0, 1, 128, T::NB);
-            const uint64_t fdesc = smem_desc(smem_u32(smem + S.fmat), 128, 256);
-            uint32_t last_bar = 0, last_par = 0;
-            for (int j = 0; j < n_ck; j++) {
-                const int wb = j % T::NWB, vb = j % T::NVB;
-                if (!wait_one(wfull_b + 8 * wb, (uint32_t)(j / T::NWB) & 1u)) break;
-                if (!wait_one(vfull_b + 8 * vb, (uint32_t)(j / T::NVB) & 1u)) break;
-                tc_fence_after();
-                const uint32_t w0 = wb0 + (uint32_t)(wb * T::WBYTES);
-#pragma unroll 1
-                for (int ks = 0; ks < kChunkTokens / 16; ks++) {
-                    const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
-                    const uint32_t wk = w0 + (uint32_t)(ks * 2 * T::LBO_W);
+        // ================= value MMAs (whole warp; one elected lane issues) =================
+        const uint32_t wb0 = smem_u32(smem + S.wbuf);
+        constexpr uint32_t IDO = instr_desc(1, 0, 0, 0, 1, 128, T::NO);   // f32 <- f16 x f16, B MN-major
+        uint32_t last_bar = 0, last_par = 0;
+        for (int j = 0; j < n_ck; j++) {
+            const int wb = j % T::NWB, vb = j % T::NVB;
+            if (!wait_warp(wfull_b + 8 * wb, (uint32_t)(j / T::NWB) & 1u)) break;
+            if (!wait_warp(vfull_b + 8 * vb, (uint32_t)(j / T::NVB) & 1u)) break;
+            tc_fence_after();
+            // descriptors of the chunk's weight buffer; each k-step adds a constant offset
+            // (the 14-bit address field never carries: shared addresses stay below 2^18)
+            const uint64_t dw = smem_desc(wb0 + (uint32_t)(wb * T::WBYTES), T::LBO_W, 128);
+            const uint32_t vt = tmem + T::T_VT + vb * T::H * 64;
+            const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-                    for (int h = 0; h < T::H; h++)
-                        mma_f16_ts(tmem + T::T_O + h * T::NO, tmem + T::T_VT + (vb * T::H + h) * 64 + 8 * ks,
-                                   smem_desc(wk + (uint32_t)(h * 64 * ROWS), T::LBO_W, 128), IDO, acc);
-                    mma_f16_ss(tmem + T::T_SUM, fdesc, smem_desc(wk, T::LBO_W, 128), IDS, acc);
-                }
-                tc_commit(pv_bar(j));
-                last_bar = pv_bar(j);
-                last_par = pv_par(j);
+            for (int ks = 0; ks < kChunkTokens / 16; ks++) {
+                const uint32_t acc = ks > 0 ? 1u : acc0;
+                const uint64_t dk = dw + (uint64_t)((ks * 2 * T::LBO_W) >> 4);
+#pragma unroll
+                for (int h = 0; h < T::H; h++)
+                    mma_f16_ts_w(tmem + T::T_O + h * T::NO, vt + h * 64 + 8 * ks,
+                                 dk + (uint64_t)((h * 64 * ROWS) >> 4), IDO, acc);
             }
-            if (*abort_flag != 0 && last_bar != 0) mbar_wait_bounded(last_bar, last_par);
+            tc_commit_w(pv_bar(j));
+            last_bar = pv_bar(j);
+            last_par = pv_par(j);
         }
+        if (lane == 0 && *abort_flag != 0 && last_bar != 0) mbar_wait_bounded(last_bar, last_par);
         __syncwarp();
     } else if (warp < 7) {
         // ================= value codes -> V^T in tensor memory =================
@@ -526,11 +400,13 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
                         for (int tg = 0; tg < 2; tg++) {
                             const uint32_t w = ldsa32(cw + (uint32_t)((4 * pp + p4) * T::PB + tg * T::REC));
                             // tokens (2k, 2k+1) of the group: bits 4k..4k+3 and 16+4k..; flipping
-                            // bit 3 turns the two's-complement code into u = code + 8
-                            r[8 * p4 + 4 * tg + 0] = lop_and_xor(w, 0x000F000Fu, 0x00080008u);
-                            r[8 * p4 + 4 * tg + 1] = lop_and_xor(w >> 4, 0x000F000Fu, 0x00080008u);
-                            r[8 * p4 + 4 * tg + 2] = lop_and_xor(w >> 8, 0x000F000Fu, 0x00080008u);
-                            r[8 * p4 + 4 * tg + 3] = lop_and_xor(w >> 12, 0x000F000Fu, 0x00080008u);
+                            // bit 3 turns the two's-complement code into u = code + 8, and the
+                            // exponent bits 0x6400 make the fp16 value 1024 + u; subtracting
+                            // 1032 leaves the code itself, exactly
+                            r[8 * p4 + 4 * tg + 0] = code_pair(w);
+                            r[8 * p4 + 4 * tg + 1] = code_pair(w >> 4);
+                            r[8 * p4 + 4 * tg + 2] = code_pair(w >> 8);
+                            r[8 * p4 + 4 * tg + 3] = code_pair(w >> 12);
                         }
                     tmem_st32(tmem_at(tmem, 32 * q, T::T_VT + (vb * T::H + h) * 64 + 32 * pp), r);
                 }
@@ -554,6 +430,7 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
         const int tp = t / 16, ttg = (t / 8) & 1, tt = t & 7;
         const uint32_t wb0 = smem_u32(smem + S.wbuf);
         float* xch = reinterpret_cast<float*>(smem + S.xch);
+        float* xsv = reinterpret_cast<float*>(smem + S.xsv);
         // Row factors and visibility limits: registers for the 8-row class, shared memory
         // (broadcast reads) for the larger ones, which would otherwise run out of registers.
         // Below, rows are indexed within the group (0 .. RPG - 1).
@@ -583,6 +460,9 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
         // A warp whose wait gave up keeps iterating without work, so that the four warps
         // of a group always meet at their named barrier the same number of times.
         bool ok = true;
+        float lsum[RPG];   // this token's share of l = sum_t p_t, per row
+#pragma unroll
+        for (int r = 0; r < RPG; r++) lsum[r] = 0.0f;
         for (int i = 0; i < n_ck; i++) {
             const int s = i % NS, sb = i % T::NSB, wb = i % T::NWB;
             const int c = c0 + i;
@@ -620,6 +500,7 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
             if (ok && !wait_warp(sfull_b + 8 * sb, (uint32_t)(i / T::NSB) & 1u)) ok = false;
             const bool clean = (c + 1) * kChunkTokens <= lim_min && !any_bad;
             float* xb = xch + (i & 1) * ROWS * 4;
+            float* xs = xsv + (i & 1) * 8 + 4 * sg;
             if (ok) {
                 tc_fence_after();
                 // ---- scores of the real rows: the three limb accumulations -> fp32 ----
@@ -653,7 +534,9 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
                     for (int r = 0; r < RPG; r++)
                         if (my_bad || tok >= lim(r)) z[r] = -INFINITY;
                 }
-                // ---- chunk row maxima over the 128 tokens ----
+                // ---- chunk row maxima over the 128 tokens, and the chunk's largest V scale
+                // (tokens some row sees; a non-finite scale is outside the codec's domain and
+                // is left out) ----
 #pragma unroll
                 for (int rg = 0; rg < RPG / 4; rg++)
                     if (rg < nrg4) {
@@ -663,19 +546,33 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
                             if (lane == 0) xb[(r0g + 4 * rg + e) * 4 + sw4] = m;
                         }
                     }
+                float svm = 0.0f;
+                if (!my_bad && c * kChunkTokens + t < L) {
+#pragma unroll
+                    for (int g = 0; g < T::G; g++) svm = fmaxf(svm, sv[g]);
+                }
+                if (!(svm <= 65504.0f)) svm = 0.0f;
+                svm = warp_redux_max(svm);
+                if (lane == 0) xs[sw4] = svm;
             }
             named_bar_sync(2 + sg, 128);
             if (ok) {
-                // ---- lazy running max: moved only when a chunk max exceeds it by kLazy ----
+                // ---- running max, moved lazily: only when a chunk max exceeds it by kLazy
+                // (p <= 2^kLazy), or when a weight p * s_v could pass 2^15 (the fp16 weights
+                // hold up to 65504): then it is raised to cm + log2(smax) - 15 ----
                 bool need = false;
-                float cm = -INFINITY;
+                float Mn = Mlane;
                 if (lane < rh) {
                     const float4 v = *reinterpret_cast<const float4*>(xb + (r0g + lane) * 4);
-                    cm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
-                    need = cm > __fadd_rn(Mlane, kLazy);
+                    const float4 w4 = *reinterpret_cast<const float4*>(xs);
+                    const float cm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+                    const float smax = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
+                    // weights of the chunk are at most 2^(cm - M) * smax = 2^(cm - M + B + 15)
+                    const float B = smax > 2048.0f ? __fsub_rn(log2f(smax), 15.0f) : -INFINITY;
+                    need = cm > __fadd_rn(Mlane, kLazy) || Mlane < __fadd_rn(cm, B);
+                    if (need) Mn = __fadd_rn(cm, fmaxf(B, 0.0f));
                 }
                 if (__any_sync(FULL, need)) {
-                    const float Mn = need ? cm : Mlane;
                     const float al = (Mn == Mlane) ? 1.0f : ex2(__fsub_rn(Mlane, Mn));
                     Mlane = Mn;
                     float alpha[RPG];
@@ -683,13 +580,14 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
                     for (int r = 0; r < RPG; r++) {
                         M[r] = __shfl_sync(FULL, Mn, r);
                         alpha[r] = __shfl_sync(FULL, al, r);
+                        lsum[r] = __fmul_rn(lsum[r], alpha[r]);
                     }
-                    // rescale O and the sums (this warp's 32 lanes, this group's rows) once
-                    // the previous chunk's value MMAs are complete
+                    // rescale O (this warp's 32 lanes, this group's rows) once the previous
+                    // chunk's value MMAs are complete
                     if (i > 0 && wait_warp(pv_bar(i - 1), pv_par(i - 1))) {
                         tc_fence_after();
-                        rescale_acc<ROWS, RPG, T::H * T::NO, T::NB>(tmem_at(tmem, 32 * q, 0), T::T_O, T::T_SUM, r0g,
-                                                                     AlphaRows<RPG>::make(alpha));
+                        rescale_acc<ROWS, RPG, T::H * T::NO>(tmem_at(tmem, 32 * q, 0), T::T_O, r0g,
+                                                             AlphaRows<RPG>::make(alpha));
                         tmem_wait_st();
                     } else if (i > 0) {
                         ok = false;
@@ -719,6 +617,7 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
                     for (int e = 0; e < 8; e++) {
                         const int r = 8 * rg8 + e;
                         pw[e] = (r >= rh || z[r] == -INFINITY) ? 0.0f : ex2(__fsub_rn(z[r], M[r]));
+                        lsum[r] = __fadd_rn(lsum[r], pw[e]);
                     }
 #pragma unroll
                     for (int g = 0; g < T::G; g++) {
@@ -732,7 +631,6 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
                         }
                         store_group(wrow + (uint32_t)(((g * ROWS + r0g + 8 * rg8) / 8) * 128), w, two);
                     }
-                    store_group(wrow + (uint32_t)(((T::G * ROWS + r0g + 8 * rg8) / 8) * 128), pw, two);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -741,39 +639,39 @@ __global__ void __launch_bounds__(Tc<D, ROWS>::THREADS, Tc<D, ROWS>::CPS) decode
             }
         }
         // ================= epilogue: the CTA partial in natural layout =================
+        // l per row: the group's 128 tokens' shares, summed in a fixed order (warp
+        // butterfly, then the four warps in index order)
+        float* xl = xch + 2 * ROWS * 4;
+#pragma unroll
+        for (int r = 0; r < RPG; r++) {
+            float v = lsum[r];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(FULL, v, o));
+            if (lane == 0) xl[(r0g + r) * 4 + sw4] = v;
+        }
+        named_bar_sync(2 + sg, 128);
         if (ok) ok = wait_warp(pv_bar(n_ck - 1), pv_par(n_ck - 1));
         if (ok) {
             tc_fence_after();
-            float lr[RPG];
-#pragma unroll
-            for (int rg = 0; rg < RPG / 8; rg++) {
-                uint32_t v[8];
-                tmem_ld8(tmem_at(tmem, 32 * q, T::T_SUM + T::G * ROWS + r0g + 8 * rg), v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 8; e++) lr[8 * rg + e] = __uint_as_float(v[e]);
-            }
 #pragma unroll
             for (int h = 0; h < T::H; h++) {
-                const int ch = 128 * h + 32 * q + lane, g = 4 * h + q;
+                const int ch = 128 * h + 32 * q + lane;
 #pragma unroll
                 for (int rg = 0; rg < RPG / 8; rg++) {
-                    uint32_t o[8], sgm[8];
+                    uint32_t o[8];
                     tmem_ld8(tmem_at(tmem, 32 * q, T::T_O + h * T::NO + q * ROWS + r0g + 8 * rg), o);
-                    tmem_ld8(tmem_at(tmem, 32 * q, T::T_SUM + g * ROWS + r0g + 8 * rg), sgm);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 8; e++)
-                        part[(r0g + 8 * rg + e) * D + ch] =
-                            __fmaf_rn(__uint_as_float(o[e]), 16777216.0f, -8.0f * __uint_as_float(sgm[e]));
+                    for (int e = 0; e < 8; e++) part[(r0g + 8 * rg + e) * D + ch] = __uint_as_float(o[e]);
                 }
+            }
+            if (sw4 == 0 && lane < RPG) {
+                const float4 v = *reinterpret_cast<const float4*>(xl + (r0g + lane) * 4);
+                part[ROWS * D + ROWS + r0g + lane] = __fadd_rn(__fadd_rn(__fadd_rn(v.x, v.y), v.z), v.w);
             }
             if (sw4 == 0 && lane == 0) {
 #pragma unroll
-                for (int r = 0; r < RPG; r++) {
-                    part[ROWS * D + r0g + r] = M[r];
-                    part[ROWS * D + ROWS + r0g + r] = lr[r];
-                }
+                for (int r = 0; r < RPG; r++) part[ROWS * D + r0g + r] = M[r];
             }
         }
         tc_fence_before();
@@ -958,9 +856,10 @@ __global__ void __launch_bounds__(1024) merge_kernel(const DecodeParams p) {
 }
 
 size_t decode_smem_bytes(int head_dim, int rows, int stages) {
+    if (rows <= 8) return small_smem_bytes(head_dim, rows, stages);
 #define MQ_SMEM(DD, RR) \
     if (head_dim == DD && rows == RR) return smem_layout<DD, RR>(stages).total;
-    MQ_SMEM(128, 8) MQ_SMEM(128, 16) MQ_SMEM(128, 32) MQ_SMEM(256, 8) MQ_SMEM(256, 16)
+    MQ_SMEM(128, 16) MQ_SMEM(128, 32) MQ_SMEM(256, 16)
 #undef MQ_SMEM
     return 0;
 }
@@ -975,34 +874,21 @@ static cudaError_t set_smem(size_t smem) {
 }
 
 int decode_ctas_per_sm(int head_dim, int rows) {
-    return (head_dim == 128 && rows == 8) ? Tc<128, 8>::CPS : 1;
+    return rows <= 8 ? small_ctas_per_sm(head_dim, rows) : 1;
 }
 
 cudaError_t decode_prepare(int head_dim, int rows, size_t smem) {
-    if (head_dim == 128 && rows == 8) return set_smem<128, 8>(smem);
+    if (rows <= 8) return small_prepare(head_dim, rows, smem);
     if (head_dim == 128 && rows == 16) return set_smem<128, 16>(smem);
     if (head_dim == 128 && rows == 32) return set_smem<128, 32>(smem);
-    if (head_dim == 256 && rows == 8) return set_smem<256, 8>(smem);
     if (head_dim == 256 && rows == 16) return set_smem<256, 16>(smem);
     return cudaErrorInvalidValue;
 }
 
-// decode_kernel, then (when any unit has several splits) merge_kernel as a programmatic
-// dependent launch on the same stream.
+// merge_kernel as a programmatic dependent launch on the same stream (after a decode
+// launch in which some unit has several splits).
 template <int D, int ROWS>
-static cudaError_t launch_pair(const DecodeParams& p, dim3 grid, size_t smem, int max_splits, cudaStream_t st) {
-    cudaLaunchAttribute pdl[1];
-    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t dc{};
-    dc.gridDim = grid;
-    dc.blockDim = dim3((unsigned)Tc<D, ROWS>::THREADS);
-    dc.dynamicSmemBytes = smem;
-    dc.stream = st;
-    dc.attrs = pdl;
-    dc.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&dc, decode_kernel<D, ROWS>, p);
-    if (e != cudaSuccess || max_splits <= 1) return e;
+static cudaError_t launch_merge(const DecodeParams& p, dim3 grid, int max_splits, cudaStream_t st) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)((ROWS * D / 4 + 127) / 128), grid.y, grid.z);
     cfg.blockDim = dim3((unsigned)(128 * ((max_splits + 7) / 8)));
@@ -1016,13 +902,37 @@ static cudaError_t launch_pair(const DecodeParams& p, dim3 grid, size_t smem, in
     return cudaLaunchKernelEx(&cfg, merge_kernel<D, ROWS>, p);
 }
 
+// decode_kernel of the 16- and 32-row classes as a programmatic dependent launch
+template <int D, int ROWS>
+static cudaError_t launch_wide(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t st) {
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t dc{};
+    dc.gridDim = grid;
+    dc.blockDim = dim3((unsigned)Tc<D, ROWS>::THREADS);
+    dc.dynamicSmemBytes = smem;
+    dc.stream = st;
+    dc.attrs = pdl;
+    dc.numAttrs = 1;
+    return cudaLaunchKernelEx(&dc, decode_kernel<D, ROWS>, p);
+}
+
+// The decode kernel of the row class, then (when any unit has several splits) the merge.
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int max_splits, size_t smem,
                           cudaStream_t st) {
     const dim3 grid((unsigned)max_splits, (unsigned)(p.n_kv_heads * p.n_rb), (unsigned)p.n_seqs);
-#define MQ_LAUNCH(DD, RR) \
-    if (head_dim == DD && rows == RR) return launch_pair<DD, RR>(p, grid, smem, max_splits, st);
-    MQ_LAUNCH(128, 8) MQ_LAUNCH(128, 16) MQ_LAUNCH(128, 32) MQ_LAUNCH(256, 8) MQ_LAUNCH(256, 16)
-#undef MQ_LAUNCH
+    cudaError_t e = cudaErrorInvalidValue;
+    if (rows <= 8) e = small_launch(p, head_dim, rows, grid, smem, st);
+    else if (head_dim == 128 && rows == 16) e = launch_wide<128, 16>(p, grid, smem, st);
+    else if (head_dim == 128 && rows == 32) e = launch_wide<128, 32>(p, grid, smem, st);
+    else if (head_dim == 256 && rows == 16) e = launch_wide<256, 16>(p, grid, smem, st);
+    if (e != cudaSuccess || max_splits <= 1) return e;
+#define MQ_MERGE(DD, RR) \
+    if (head_dim == DD && rows == RR) return launch_merge<DD, RR>(p, grid, max_splits, st);
+    MQ_MERGE(128, 4) MQ_MERGE(128, 8) MQ_MERGE(128, 16) MQ_MERGE(128, 32) MQ_MERGE(256, 4) MQ_MERGE(256, 8)
+    MQ_MERGE(256, 16)
+#undef MQ_MERGE
     return cudaErrorInvalidValue;
 }
 

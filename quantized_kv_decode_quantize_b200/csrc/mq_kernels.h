@@ -87,7 +87,13 @@ __device__ __forceinline__ int seq_nq_of(const DecodeParams& p, int b) {
 }
 #endif
 
-// rows: 8, 16 or 32 (padded query rows per kv-head handled by one CTA)
+// The small row classes (4 and 8 rows, mq_decode_small.cu).
+size_t small_smem_bytes(int head_dim, int rows, int stages);
+int small_ctas_per_sm(int head_dim, int rows);
+cudaError_t small_prepare(int head_dim, int rows, size_t smem);
+cudaError_t small_launch(const DecodeParams& p, int head_dim, int rows, dim3 grid, size_t smem, cudaStream_t st);
+
+// rows: 4, 8, 16 or 32 (padded query rows per kv-head handled by one CTA)
 size_t decode_smem_bytes(int head_dim, int rows, int stages);   // 0: does not fit the layout
 cudaError_t decode_prepare(int head_dim, int rows, size_t smem);  // raises the dynamic smem limit
 int decode_ctas_per_sm(int head_dim, int rows);                    // CTAs the kernel is built to co-host

@@ -216,3 +216,32 @@ def test_error_against_unquantized_is_reported():
     rel = float(np.linalg.norm(o - eo) / np.linalg.norm(eo))
     print(f"\nvs unquantized fp64 attention: max-abs {err:.3e}, relative L2 {rel:.3e}")
     assert np.isfinite(err)
+
+
+@pytest.mark.parametrize("vmax", [1e4, 3e4, 1e5, 4.5e5])
+@pytest.mark.parametrize("name", ["long", "verify"])
+def test_large_values_up_to_the_codec_domain(name, vmax):
+    """Values whose V scales reach the top of fp16 (a scale is max|x| / 7, so |V| up to
+    65504 * 7 = 458,528 is inside the codec's domain).  The weights p * s_v are fp16
+    operands of the value MMAs; the running max is raised where they could overflow.
+    Attention is linear in V, so the bar is the unit-scale bar on out / vmax (here
+    |V| <= vmax, against |V| of about 5 in the unit workloads); lse does not depend on
+    V and keeps the absolute bar.  Mixed magnitudes: every 7th token is unscaled and
+    every 5th at a third of the rest."""
+    w = wl.reduced(name)
+    inp = wl.make_inputs(w)
+    v = inp.own_v[0].float()
+    f = torch.full((v.shape[0], 1, 1), 1.0)
+    f[::5] = 1.0 / 3.0
+    f[::7] = 1.0 / vmax
+    inp.own_v[0] = (v / v.abs().amax() * vmax * f).to(inp.own_v[0].dtype)
+    case = GpuCase(w, inputs=inp)
+    out, lse = case.decode()
+    assert case.status() == mq.MQ_OK
+    eo, el = oracle_outputs(w, inp)
+    o, l = out.cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(o)), "non-finite output: a weight overflowed fp16"
+    err = float(np.max(np.abs(o - eo))) / vmax
+    lerr = float(np.max(np.abs(l - el)))
+    assert err <= TOL, f"max-abs error / vmax {err:.3e}"
+    assert lerr <= TOL_LSE, f"lse error {lerr:.3e}"
