@@ -10,6 +10,8 @@
  *                   n > 1 = verification of n speculative draft tokens, causal
  *                   among the drafts) against the cache, split over the
  *                   sequence and merged by log-sum-exp
+ *   mq_prefill_attn attention of many query tokens per sequence (a prompt or a
+ *                   prompt chunk), causal, in tiles of 128 query rows
  *   mq_decode_attn_cascade  the same for sessions sharing a cached prefix: the
  *                   shared pages are read once for all of them
  *   mq_draft_ngram  history-based drafts (the tokens that followed the latest
@@ -280,6 +282,37 @@ mq_status mq_decode_attn(const mq_cache* cache, const void* q, mq_dtype q_dtype,
                          mq_stream stream);
 
 /* ---------------------------------------------------------------------------
+ * mq_prefill_attn — attention of a prompt's query tokens against the quantized
+ * cache (prefill, or a chunk of it)
+ *
+ * The deep dive (section 3, the first-load tuner) counts 4k and 64k prompt
+ * prefill among the serving terms the tuner weighs; the stork.ai page quotes
+ * prefill rates.  The arithmetic is mq_decode_attn's, for any number of query
+ * tokens per sequence: query token j of sequence b (0-based, n_b of them) attends
+ * to positions 0 .. L_b - n_b + j, where L_b counts the prompt's own tokens, whose
+ * K/V must already be appended (mq_kv_append).  n_b = L_b is a whole prompt; a
+ * smaller n_b is a prompt chunk after a cached history.
+ *   q, seq_lens, n_q_per_seq, total_q, block_table, softmax_scale, out, lse
+ *                as mq_decode_attn (q packed by sequence; out fp32, lse may be NULL)
+ *   max_q_per_seq, max_seq_len   host bounds on n_b and L_b
+ * No workspace: one CTA takes a tile of 128 query rows (query token, q-head of a
+ * kv-head) over every key its rows see.  Keys enter the tensor cores as exact
+ * fp16 codes, q as fp16 scaled by a power of two per row (exact for the BF16 and
+ * F16 q this call accepts), values as two fp16 parts hi + lo of code * s_v (about
+ * 22 significant bits), the softmax weights as fp16 with l summed from the same
+ * rounded weights.  Asynchronous on `stream`, launched as a programmatic
+ * dependent launch like mq_decode_attn (see its stream-order note).
+ * Errors: those of mq_decode_attn's host checks; UNSUPPORTED for F32 q, head_dim
+ * other than 128, or a group size n_q_heads / n_kv_heads that does not divide 128.  A
+ * sequence whose L_b / n_b break the bounds is skipped and reported by
+ * mq_device_status(), as are unusable block ids (their tokens are masked).
+ * ------------------------------------------------------------------------- */
+mq_status mq_prefill_attn(const mq_cache* cache, const void* q, mq_dtype q_dtype, int32_t n_seqs, int32_t n_q_heads,
+                          int32_t total_q, int32_t max_q_per_seq, int32_t max_seq_len, const int32_t* block_table,
+                          int32_t max_blocks_per_seq, const int32_t* seq_lens, const int32_t* n_q_per_seq,
+                          float softmax_scale, float* out, float* lse, mq_stream stream);
+
+/* ---------------------------------------------------------------------------
  * mq_decode_attn_static: mq_decode_attn without a caller workspace.
  *
  * The method on the pages has no counterpart to this call; it is a convenience
@@ -433,10 +466,14 @@ typedef struct mq_tune_result {
 /* On-device tuner.  Within params->budget_s of wall-clock time (allocation,
  * probe set-up, every measurement included) it measures the candidate launch
  * configurations on three probe shapes built from the cache's geometry and
- * params->n_q_heads — decode at 4K and at 64K tokens, and verification of 8
- * drafts at 64K — admits candidates by params->admission, and keeps the admitted
- * candidate set with the lowest cost
- *     cost(c) = sum_p median_time(c, p) / median_time(default, p).
+ * params->n_q_heads — decode at 4K and at 64K tokens, and a speculative step: one
+ * mq_draft_ngram launch over a 64K-token history followed by the verification of
+ * 8 drafts at 64K — admits candidates by params->admission, and keeps the admitted
+ * candidate set with the lowest cost (the deep dive's service cost)
+ *     cost(c) = sum_p weight(p) * median_time(c, p),
+ *     weight(p) = sum_t launches(t, p) / time_at_defaults(t)
+ * over the terms t (decode 4K, decode 64K, the drafter launch, verification of 8
+ * drafts), each of weight 1; reported relative to the defaults' cost.
  * The default is the configuration the cache holds when mq_tune is called.
  *
  * Admission.  MQ_ADMIT_BIT_IDENTICAL keeps a candidate only if its out and lse

@@ -70,6 +70,8 @@ def _load():
         "mq_decode_kernel_count": ([P, i32, i32, i32, i32], i32),
         "mq_decode_attn": ([P, P, ctypes.c_int, i32, i32, i32, i32, i32, P, i32, P, P, ctypes.c_float, P, P, P, sz, P],
                            ctypes.c_int),
+        "mq_prefill_attn": ([P, P, ctypes.c_int, i32, i32, i32, i32, i32, P, i32, P, P, ctypes.c_float, P, P, P],
+                            ctypes.c_int),
         "mq_decode_attn_static": ([P, P, ctypes.c_int, i32, i32, i32, i32, i32, P, i32, P, P, ctypes.c_float, P, P,
                                    P], ctypes.c_int),
         "mq_decode_cascade_workspace_bytes": ([P, i32, i32, i32, i32, i32, i32], sz),
@@ -177,6 +179,14 @@ def mq_decode_attn(cache: int, q, q_dtype: int, n_seqs: int, n_q_heads: int, tot
                               _ptr(block_table), max_blocks_per_seq, _ptr(seq_lens), _ptr(n_q_per_seq),
                               float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace_bytes,
                               _stream(stream)), "mq_decode_attn")
+
+
+def mq_prefill_attn(cache: int, q, q_dtype: int, n_seqs: int, n_q_heads: int, total_q: int, max_q_per_seq: int,
+                    max_seq_len: int, block_table, max_blocks_per_seq: int, seq_lens, n_q_per_seq, softmax_scale: float,
+                    out, lse, stream=None) -> None:
+    _check(lib.mq_prefill_attn(cache, _ptr(q), q_dtype, n_seqs, n_q_heads, total_q, max_q_per_seq, max_seq_len,
+                               _ptr(block_table), max_blocks_per_seq, _ptr(seq_lens), _ptr(n_q_per_seq),
+                               float(softmax_scale), _ptr(out), _ptr(lse), _stream(stream)), "mq_prefill_attn")
 
 
 def mq_decode_attn_static(cache: int, q, q_dtype: int, n_seqs: int, n_q_heads: int, total_q: int,

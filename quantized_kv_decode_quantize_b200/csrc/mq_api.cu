@@ -352,6 +352,52 @@ mq_status mq_decode_attn(const mq_cache* c, const void* q, mq_dtype q_dtype, int
                               workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
+mq_status mq_prefill_attn(const mq_cache* c, const void* q, mq_dtype q_dtype, int32_t n_seqs, int32_t n_q_heads,
+                          int32_t total_q, int32_t max_q_per_seq, int32_t max_seq_len, const int32_t* block_table,
+                          int32_t max_blocks_per_seq, const int32_t* seq_lens, const int32_t* n_q_per_seq,
+                          float softmax_scale, float* out, float* lse, mq_stream stream) {
+    if (c == nullptr || q == nullptr || block_table == nullptr || seq_lens == nullptr || n_q_per_seq == nullptr ||
+        out == nullptr)
+        return MQ_ERR_INVALID_ARG;
+    if (n_seqs < 1 || n_seqs > 65535 || n_q_heads < 1 || n_q_heads % c->n_kv_heads != 0) return MQ_ERR_INVALID_ARG;
+    if (max_q_per_seq < 1 || max_seq_len < max_q_per_seq || total_q < 1 || max_blocks_per_seq < 1)
+        return MQ_ERR_INVALID_ARG;
+    if (!(std::isfinite(softmax_scale))) return MQ_ERR_INVALID_ARG;
+    // q enters the tensor cores as fp16, exactly for BF16 and F16 input (F32 would lose bits)
+    if (q_dtype != MQ_BF16 && q_dtype != MQ_F16) return MQ_ERR_UNSUPPORTED;
+    const int G = n_q_heads / c->n_kv_heads;
+    if (c->head_dim != 128 || G > 128 || 128 % G != 0) return MQ_ERR_UNSUPPORTED;
+    if ((long long)max_seq_len > (long long)max_blocks_per_seq * MQ_PAGE_TOKENS) return MQ_ERR_CAPACITY;
+    if (c->n_kv_heads > 65535) return MQ_ERR_UNSUPPORTED;
+    if (prefill_smem_bytes() > (size_t)c->max_smem) return MQ_ERR_UNSUPPORTED;
+    DevGuard guard(c->device);
+    DecodeParams p{};
+    p.pool = static_cast<const uint8_t*>(c->pool);
+    p.n_kv_heads = c->n_kv_heads;
+    p.n_blocks = c->n_blocks;
+    p.q = q;
+    p.q_dtype = (int)q_dtype;
+    p.n_q_heads = n_q_heads;
+    p.group = G;
+    p.total_q = total_q;
+    p.max_q = max_q_per_seq;
+    p.n_seqs = n_seqs;
+    p.block_table = block_table;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.seq_lens = seq_lens;
+    p.n_q_per_seq = n_q_per_seq;
+    p.scale_log2 = (float)((double)softmax_scale * 1.4426950408889634);
+    p.out = out;
+    p.lse = lse;
+    p.err = c->err_word;
+    p.causal = 1;
+    const int tq = 128 / G;   // query tokens per tile
+    const long long tiles = ((long long)max_q_per_seq + tq - 1) / tq;
+    if (tiles > 0x7fffffffLL) return MQ_ERR_UNSUPPORTED;
+    return launch_prefill(p, (int)tiles, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MQ_OK
+                                                                                              : MQ_ERR_CUDA;
+}
+
 mq_status mq_get_decode_config(const mq_cache* c, int32_t cls, mq_decode_config* cfg) {
     if (c == nullptr || cfg == nullptr || cls < 0 || cls > 2) return MQ_ERR_INVALID_ARG;
     *cfg = c->cfg[cls];

@@ -93,6 +93,10 @@ int small_ctas_per_sm(int head_dim, int rows);
 cudaError_t small_prepare(int head_dim, int rows, size_t smem);
 cudaError_t small_launch(const DecodeParams& p, int head_dim, int rows, dim3 grid, size_t smem, cudaStream_t st);
 
+// Prefill attention (mq_prefill.cu): head_dim 128, tiles of 128 query rows.
+size_t prefill_smem_bytes();
+cudaError_t launch_prefill(const DecodeParams& p, int max_tiles, cudaStream_t st);
+
 // rows: 4, 8, 16 or 32 (padded query rows per kv-head handled by one CTA)
 size_t decode_smem_bytes(int head_dim, int rows, int stages);   // 0: does not fit the layout
 cudaError_t decode_prepare(int head_dim, int rows, size_t smem);  // raises the dynamic smem limit

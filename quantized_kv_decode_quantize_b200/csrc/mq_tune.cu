@@ -4,10 +4,13 @@
 // magnitudedev/magnitude, section 3 ("core mechanism 1: the 60 s first-load
 // tuner"): one wall-clock budget covers everything (probe set-up, every launch,
 // every comparison); candidates are measured on the device over serving shapes
-// (decode at 4k and 64k history, the verification width), and the cost of a
-// configuration c is
-//     cost(c) = sum_p weight(p) * median_time(c, p),  weight(p) = 1 / median_time(default, p)
-// (each probe is one launch of its term); timing passes read data sized beyond the
+// (decode at 4k and 64k history, and a speculative step: one drafter launch, then the
+// verification of 8 drafts), and the cost of a configuration c is
+//     cost(c) = sum_p weight(p) * median_time(c, p),
+//     weight(p) = sum_t term_weight(t) * launches(t, p) / time_at_defaults(t)
+// over the terms t = decode_4k, decode_64k, draft_64k (mq_draft_ngram over a 64K-token
+// history) and verify8_64k, each of weight 1 (the speculative-step probe holds one
+// launch of each of its two terms); timing passes read data sized beyond the
 // last-level cache (here: rotating probe caches that together exceed twice the L2
 // size), so no launch finds its data warm; structurally different candidates are
 // tried before refinements of one; a candidate is started only when the budget
@@ -43,7 +46,9 @@ using Clock = std::chrono::steady_clock;
 struct Probe {
     const char* name;
     int seq_len, n_q, cls;
+    bool with_draft;        // a drafter launch precedes the decode launch
     double t_default = 0;   // median seconds at the default configuration
+    double weight = 0;      // sum over its terms of launches / time_at_defaults (1/s)
 };
 
 struct Cand {
@@ -77,6 +82,9 @@ struct Buffers {
     int32_t* nq = nullptr;
     int32_t* cu = nullptr;
     int32_t* start = nullptr;
+    int32_t* tokens = nullptr;   // the drafter's 64K-token history
+    int32_t* drafts = nullptr;
+    int32_t* n_drafts = nullptr;
     void* kv = nullptr;          // staging for K and V
     void* q = nullptr;
     float* out_ref[3] = {nullptr, nullptr, nullptr};
@@ -91,7 +99,7 @@ struct Buffers {
     cudaEvent_t ev[2] = {nullptr, nullptr};
     cudaStream_t st = nullptr;
     ~Buffers() {
-        void* ptrs[] = {pool, bt, lens, nq, cu, start, kv, q, out, lse, ws, flag, pert,
+        void* ptrs[] = {pool, bt, lens, nq, cu, start, tokens, drafts, n_drafts, kv, q, out, lse, ws, flag, pert,
                         out_ref[0], out_ref[1], out_ref[2], lse_ref[0], lse_ref[1], lse_ref[2],
                         noise_out[0], noise_out[1], noise_out[2], noise_lse[0], noise_lse[1], noise_lse[2]};
         for (void* p : ptrs)
@@ -157,10 +165,11 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
     }
     DevGuard guard(cache->device);
 
-    std::vector<Probe> probes = {{"decode_4k", 4096, 1, rows_class_for(D, G)},
-                                 {"decode_64k", 65536, 1, rows_class_for(D, G)}};
-    if (G * 8 <= 64) probes.push_back({"verify8_64k", 65544, 8, rows_class_for(D, G * 8)});
+    std::vector<Probe> probes = {{"decode_4k", 4096, 1, rows_class_for(D, G), false},
+                                 {"decode_64k", 65536, 1, rows_class_for(D, G), false}};
+    if (G * 8 <= 64) probes.push_back({"draft_verify8_64k", 65544, 8, rows_class_for(D, G * 8), true});
     const int P = (int)probes.size();
+    constexpr int kDraftLen = 65536, kDraftN = 4, kDraftK = 8;   // drafter term: history, n-gram, drafts
 
     // ---- probe caches: enough rotating copies to exceed 2x L2 ----
     int l2 = 0;
@@ -183,7 +192,9 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         !ck(cudaMalloc(&B.cu, sizeof(int32_t) * 2)) || !ck(cudaMalloc(&B.start, sizeof(int32_t))) ||
         !ck(cudaMalloc(&B.kv, kv_elems * 2 * 2)) || !ck(cudaMalloc(&B.q, (size_t)8 * Hq * D * 2)) ||
         !ck(cudaMalloc(&B.out, (size_t)8 * Hq * D * 4)) || !ck(cudaMalloc(&B.lse, (size_t)8 * Hq * 4)) ||
-        !ck(cudaMalloc(&B.ws, ws_bytes)) || !ck(cudaMalloc(&B.flag, 3 * sizeof(unsigned))))
+        !ck(cudaMalloc(&B.ws, ws_bytes)) || !ck(cudaMalloc(&B.flag, 3 * sizeof(unsigned))) ||
+        !ck(cudaMalloc(&B.tokens, sizeof(int32_t) * (kDraftLen + 1))) ||
+        !ck(cudaMalloc(&B.drafts, sizeof(int32_t) * kDraftK)) || !ck(cudaMalloc(&B.n_drafts, sizeof(int32_t))))
         return MQ_ERR_CUDA;
     for (int p = 0; p < P; p++)
         if (!ck(cudaMalloc(&B.out_ref[p], (size_t)8 * Hq * D * 4)) || !ck(cudaMalloc(&B.lse_ref[p], (size_t)8 * Hq * 4)))
@@ -204,6 +215,13 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         }
         if (!ck(cudaMemcpy(B.lens, lens, sizeof(int32_t) * P, cudaMemcpyHostToDevice)) ||
             !ck(cudaMemcpy(B.nq, nq, sizeof(int32_t) * P, cudaMemcpyHostToDevice)))
+            return MQ_ERR_CUDA;
+        // the drafter's history: a token stream with repeats (a 4093-token cycle with a
+        // few edits), and its length at the end of the buffer
+        std::vector<int32_t> tok(kDraftLen + 1);
+        for (int i = 0; i < kDraftLen; i++) tok[i] = (int32_t)((i % 4093) * 7 % 32000 + (i % 9973 == 0 ? 1 : 0));
+        tok[kDraftLen] = kDraftLen;
+        if (!ck(cudaMemcpy(B.tokens, tok.data(), sizeof(int32_t) * tok.size(), cudaMemcpyHostToDevice)))
             return MQ_ERR_CUDA;
     }
     // random K/V for one copy, quantized by the append kernel, then replicated
@@ -258,13 +276,20 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         return launch_decode_plan(&pc, pl, B.q, MQ_BF16, 1, Hq, probes[p].n_q, probes[p].n_q, bt, blocks_per_copy,
                                   B.lens + p, B.nq + p, 1.0f / std::sqrt((float)D), out, lse, B.ws, ws_bytes, B.st);
     };
+    // one drafter launch over the 64K-token history
+    auto launch_draft = [&]() -> mq_status {
+        return mq_draft_ngram(B.tokens, kDraftLen, B.tokens + kDraftLen, 1, kDraftN, kDraftK, B.drafts, B.n_drafts,
+                              reinterpret_cast<mq_stream>(B.st));
+    };
     const int reps = 7;
-    // median device time of `reps` launches (events around each launch)
+    // median device time of `reps` launches of probe p (events around the probe's
+    // launches: the drafter's, when it has one, then the decode)
     auto time_probe = [&](int p, const mq_decode_config& cfg, double* out_t) -> mq_status {
         std::vector<float> ts;
         for (int r = 0; r < reps; r++) {
             cudaEventRecord(B.ev[0], B.st);
-            mq_status s = launch(p, cfg, B.out, B.lse);
+            mq_status s = probes[p].with_draft ? launch_draft() : MQ_OK;
+            if (s == MQ_OK) s = launch(p, cfg, B.out, B.lse);
             if (s != MQ_OK) return s;
             cudaEventRecord(B.ev[1], B.st);
             if (!ck(cudaEventSynchronize(B.ev[1]))) return MQ_ERR_CUDA;
@@ -277,11 +302,38 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         return MQ_OK;
     };
 
-    // ---- defaults: reference outputs and times ----
+    // ---- defaults: reference outputs and times; each term's time at the defaults ----
     for (int p = 0; p < P; p++) {
         mq_status s = launch(p, cache->cfg[probes[p].cls], B.out_ref[p], B.lse_ref[p]);
         if (s != MQ_OK) return s;
         if ((s = time_probe(p, cache->cfg[probes[p].cls], &probes[p].t_default)) != MQ_OK) return s;
+    }
+    // the drafter term alone (median of `reps` launches)
+    double t_draft_default = 0;
+    {
+        std::vector<float> ts;
+        for (int r = 0; r < reps; r++) {
+            cudaEventRecord(B.ev[0], B.st);
+            if (launch_draft() != MQ_OK) return MQ_ERR_CUDA;
+            cudaEventRecord(B.ev[1], B.st);
+            if (!ck(cudaEventSynchronize(B.ev[1]))) return MQ_ERR_CUDA;
+            float ms = 0;
+            cudaEventElapsedTime(&ms, B.ev[0], B.ev[1]);
+            ts.push_back(ms);
+        }
+        std::sort(ts.begin(), ts.end());
+        t_draft_default = ts[ts.size() / 2] * 1e-3;
+    }
+    // weight(p) = sum_t launches(t, p) / time_at_defaults(t): a probe with a drafter holds
+    // one launch of the drafter term and one of its decode term, whose time at the
+    // defaults is the probe's time less the drafter's
+    for (int p = 0; p < P; p++) {
+        if (probes[p].with_draft) {
+            const double t_dec = std::max(probes[p].t_default - t_draft_default, 1e-9);
+            probes[p].weight = 1.0 / std::max(t_draft_default, 1e-9) + 1.0 / t_dec;
+        } else {
+            probes[p].weight = 1.0 / std::max(probes[p].t_default, 1e-9);
+        }
     }
     if (!ck(cudaStreamSynchronize(B.st))) return MQ_ERR_CUDA;
 
@@ -401,19 +453,21 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
     int n_terms = 0;
     for (int cls = 0; cls < 3; cls++) {
         if (!class_used[cls]) continue;
-        double best = 0;
+        // cost(c) = sum_p weight(p) * time(c, p), relative to the defaults' cost
+        double base = 0;
         int terms = 0;
         for (int p = 0; p < P; p++)
             if (probes[p].cls == cls) {
-                best += 1.0;
+                base += probes[p].weight * probes[p].t_default;
                 terms++;
             }
+        double best = 1.0;
         mq_decode_config pick = cache->cfg[cls];
         for (auto& cd : cands) {
             if (cd.cls != cls || !cd.measured || cd.rejected || !cd.valid) continue;
             double cost = 0;
             for (int p = 0; p < P; p++)
-                if (probes[p].cls == cls) cost += cd.t[p] / probes[p].t_default;
+                if (probes[p].cls == cls) cost += probes[p].weight * cd.t[p] / base;
             if (cost < best) {
                 best = cost;
                 pick = cd.cfg;
@@ -421,7 +475,7 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         }
         res->chosen[cls] = pick;
         cache->cfg[cls] = pick;
-        total += best;
+        total += best * terms;
         n_terms += terms;
     }
     res->cost = n_terms ? total / n_terms : 1.0;
@@ -450,11 +504,21 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
                                  nstat[p].zero_points);
                 std::fprintf(f, "],\n");
             }
-            std::fprintf(f, "  \"probes\": [");
+            std::fprintf(f, "  \"terms\": [{\"name\": \"decode_4k\", \"default_us\": %.3f}, "
+                         "{\"name\": \"decode_64k\", \"default_us\": %.3f}",
+                         probes[0].t_default * 1e6, probes[1].t_default * 1e6);
+            if (P > 2)
+                std::fprintf(f, ", {\"name\": \"draft_64k\", \"default_us\": %.3f, \"ngram\": %d, \"max_draft\": %d}, "
+                             "{\"name\": \"verify8_64k\", \"default_us\": %.3f}",
+                             t_draft_default * 1e6, kDraftN, kDraftK,
+                             std::max(probes[2].t_default - t_draft_default, 0.0) * 1e6);
+            std::fprintf(f, "],\n  \"probes\": [");
             for (int p = 0; p < P; p++)
-                std::fprintf(f, "%s{\"name\": \"%s\", \"seq_len\": %d, \"n_q\": %d, \"rows_class\": %d, \"default_us\": %.3f}",
+                std::fprintf(f, "%s{\"name\": \"%s\", \"seq_len\": %d, \"n_q\": %d, \"rows_class\": %d, "
+                             "\"launches\": \"%s\", \"default_us\": %.3f, \"weight_per_s\": %.6g}",
                              p ? ", " : "", probes[p].name, probes[p].seq_len, probes[p].n_q, probes[p].cls,
-                             probes[p].t_default * 1e6);
+                             probes[p].with_draft ? "draft_64k + verify8_64k" : probes[p].name,
+                             probes[p].t_default * 1e6, probes[p].weight);
             std::fprintf(f, "],\n  \"candidates\": [\n");
             for (size_t i = 0; i < cands.size(); i++) {
                 const Cand& cd = cands[i];

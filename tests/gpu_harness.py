@@ -18,7 +18,8 @@ DT = {"f32": mq.MQ_F32, "bf16": mq.MQ_BF16}
 class GpuCase:
     """A workload populated into a device cache through mq_kv_append."""
 
-    def __init__(self, w: wl.Workload, inputs: wl.Inputs | None = None, copies: int = 1, config=None):
+    def __init__(self, w: wl.Workload, inputs: wl.Inputs | None = None, copies: int = 1, config=None,
+                 workspace: bool = True):
         self.w = w
         self.inp = inputs if inputs is not None else wl.make_inputs(w)
         tabs, n_blocks = wl.block_tables(w, copies=copies)
@@ -34,9 +35,10 @@ class GpuCase:
         self.seq_lens = torch.tensor(w.seq_lens, dtype=torch.int32, device="cuda")
         self.n_q = torch.tensor(w.n_q, dtype=torch.int32, device="cuda")
         self.q = self.inp.q.cuda()
-        ws_bytes = mq.mq_decode_workspace_bytes(self.cache.handle, w.n_seqs, w.n_q_heads, w.max_q, w.max_seq_len)
-        assert ws_bytes > 0
-        self.ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
+        if workspace:   # decode calls (prefill needs none)
+            ws_bytes = mq.mq_decode_workspace_bytes(self.cache.handle, w.n_seqs, w.n_q_heads, w.max_q, w.max_seq_len)
+            assert ws_bytes > 0
+            self.ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
         self.out = torch.empty((w.total_q, w.n_q_heads, w.head_dim), dtype=torch.float32, device="cuda")
         self.lse = torch.empty((w.total_q, w.n_q_heads), dtype=torch.float32, device="cuda")
 

@@ -33,6 +33,17 @@ def test_tune_within_budget_and_output_unchanged(tmp_path):
     assert r["cost"] <= 1.0 + 1e-9
     d = json.load(open(log))
     assert d["candidates"] and any(c["measured"] and c["bit_identical"] for c in d["candidates"])
+    # the service cost's terms, the drafter launch among them, and the probe weights
+    # weight(p) = sum_t launches(t, p) / time_at_defaults(t)
+    terms = {t["name"]: t["default_us"] for t in d["terms"]}
+    assert set(terms) == {"decode_4k", "decode_64k", "draft_64k", "verify8_64k"}
+    assert all(v > 0 for v in terms.values())
+    probes = {p["name"]: p for p in d["probes"]}
+    spec = probes["draft_verify8_64k"]
+    assert spec["launches"] == "draft_64k + verify8_64k"
+    assert abs(spec["weight_per_s"] - 1e6 * (1 / terms["draft_64k"] + 1 / terms["verify8_64k"])) \
+        <= 1e-3 * spec["weight_per_s"]
+    assert abs(probes["decode_64k"]["weight_per_s"] - 1e6 / terms["decode_64k"]) <= 1e-3 * 1e6 / terms["decode_64k"]
     # ring depth never changes the bytes, so those candidates are all admitted
     assert all(c["bit_identical"] for c in d["candidates"] if c["measured"] and c["splits_per_sm"] == 1)
     # the tuned configuration gives the same bytes as the defaults
