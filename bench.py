@@ -49,7 +49,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=500)
     ap.add_argument("--impl", default="mq", choices=["mq", "reference"])
-    ap.add_argument("--workload", default="long", choices=["tiny", "long", "prefix", "verify", "mixed"])
+    ap.add_argument("--workload", default="long",
+                    choices=["tiny", "long", "prefix", "verify", "mixed", "prefill_4k", "prefill_64k"])
     ap.add_argument("--graph-steps", type=int, default=0, help="steps per captured graph (0: one rotation)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -121,6 +122,122 @@ def load_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def load_tensor_peak():
+    """Dense bf16 (= fp16) tensor TFLOP/s: the measured burst figure, else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def prefill_flops(seq_lens, n_q, n_q_heads, head_dim):
+    """Algorithmic FLOPs of causal prefill attention: query j of n sees L - n + j + 1
+    keys; 2 * D flops for its score and 2 * D for its share of the output per key."""
+    vis = sum(n * (L - n) + n * (n + 1) // 2 for L, n in zip(seq_lens, n_q))
+    return 4 * head_dim * n_q_heads * vis
+
+
+def run_prefill(args, rank, world, local):
+    """Prompt prefill over the quantized cache (mq_prefill_attn): a whole 4K- or
+    64K-token prompt per rank, timed like the decode step (CUDA graph of launches,
+    events around the timed region); algorithmic TFLOP/s against the tensor peak."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import quantized_kv_decode_quantize_b200 as mq
+    import workloads as wl
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    L = 4096 if args.workload == "prefill_4k" else 65536
+    w = wl.Workload(args.workload, 32, 8, 128, [L], [L], [L],
+                    note=f"one {L}-token prompt, 32 q / 8 kv heads (GQA 4), D 128, bf16, shuffled 16-token blocks")
+    inp = wl.make_inputs(w)
+    tabs_np, n_blocks = wl.block_tables(w)
+    cache = mq.Cache(w.n_kv_heads, w.head_dim, n_blocks)
+    tab = torch.from_numpy(tabs_np[0]).to(dev)
+    i32 = dict(dtype=torch.int32, device=dev)
+    mq.mq_kv_append(cache.handle, inp.own_k[0].to(dev), inp.own_v[0].to(dev), mq.MQ_BF16, 1, L,
+                    torch.tensor([0, L], **i32), torch.tensor([0], **i32), tab, w.max_blocks())
+    q = inp.q.to(dev).contiguous()
+    lens = torch.tensor([L], **i32)
+    out = torch.empty((L, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    lse = torch.empty((L, w.n_q_heads), dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(w.head_dim)
+
+    def call(stream):
+        mq.mq_prefill_attn(cache.handle, q, mq.MQ_BF16, 1, w.n_q_heads, L, L, L, tab, w.max_blocks(), lens, lens,
+                           scale, out, lse, stream)
+
+    stream = torch.cuda.Stream(dev)
+    S = max(1, min(args.steps, 4))
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            call(stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(S):
+            call(stream)
+    sampler = ClockSampler(local)
+    sampler.start()
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, math.ceil(args.warmup / S))):
+            g.replay()
+    torch.cuda.synchronize(dev)
+    reps, rem = divmod(args.steps, S)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        for _ in range(rem):
+            call(stream)
+        t1.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1), dev)
+    assert mq.mq_device_status(cache.handle) == mq.MQ_OK
+    flops = prefill_flops(w.seq_lens, w.n_q, w.n_q_heads, w.head_dim)
+    tflops = world * flops * args.steps / (ms * 1e-3) / 1e12
+    peak, kind = load_tensor_peak()
+    if rank == 0:
+        clocks = sampler.summary()
+        print(json.dumps({
+            "metric": "prefill attention over the K8/V4 cache: algorithmic TFLOP/s", "value": tflops,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp16 tensor-core operands (exact bf16 q, exact key codes, values hi + lo), fp32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": w.name, "note": w.note, "prompt_tokens": L, "flops_per_step": flops,
+                       "parallelism": f"replica x{world}"},
+            "roofline": {"bound": "tensor", "achieved": tflops / world, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / world / peak, "peak_kind": peak_kind_note(kind),
+                         "traffic": None, "kernel": "mq::prefill_kernel"},
+            "gpu_launches": args.steps,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
+                       "samples": clocks["samples"]},
+        }), flush=True)
+    del g
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def peak_kind_note(kind):
+    return (f"{kind} dense bf16 (fp16 runs at the same rate); the kernel issues 1.5x the algorithmic "
+            f"MMA work (values as hi + lo)")
 
 
 def kernel_source_hash():
@@ -209,6 +326,9 @@ def run_reference(args, rank, world):
 
     if rank != 0:
         return
+    if args.workload.startswith("prefill"):
+        run_reference_prefill(args, world)
+        return
     w = wl.FULL[args.workload]()
     inp = wl.make_inputs(w)
     cores = oracle.max_threads()
@@ -254,6 +374,49 @@ def run_reference(args, rank, world):
         "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def run_reference_prefill(args, world):
+    """The reference arm of the prefill workloads: the oracle's fp64 attention over the
+    quantized cache for a bounded sample of the prompt's query rows (the last query
+    tokens, which see the whole prompt) on the host cores; algorithmic TFLOP/s."""
+    import numpy as np
+
+    import oracle
+    import workloads as wl
+
+    L = 4096 if args.workload == "prefill_4k" else 65536
+    w = wl.Workload(args.workload, 32, 8, 128, [L], [L], [L])
+    inp = wl.make_inputs(w)
+    cores = oracle.max_threads()
+    kc, ks = oracle.quantize_k(inp.own_k[0].float().numpy())
+    vp, vs = oracle.quantize_v(inp.own_v[0].float().numpy())
+    scale = 1.0 / math.sqrt(w.head_dim)
+    n_s = 4 if L > 8192 else 32          # sampled query tokens per step (all 32 heads each)
+    q = inp.q[L - n_s:].float().numpy().astype(np.float64)
+
+    def step():
+        oracle.attention_quant(q, kc, ks, vp, vs, scale, cores)
+
+    for _ in range(min(args.warmup, 1)):
+        step()
+    steps = max(1, min(args.steps, 5))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    dt = time.perf_counter() - t0
+    flops = prefill_flops([L], [n_s], w.n_q_heads, w.head_dim)
+    val = flops * steps / dt / 1e12
+    sample = (f"per step: fp64 attention of the last {n_s} query tokens (32 q-heads each) of the {L}-token "
+              f"prompt over the quantized cache, {steps} step(s)")
+    print(json.dumps({
+        "metric": "prefill attention over the K8/V4 cache: algorithmic TFLOP/s", "value": val, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": steps, "warmup": args.warmup, "ms_per_step": dt / steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference", "config": {"workload": w.name, "prompt_tokens": L},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
 
 
 def cpu_baseline(w, inp, gpu_out=None, gpu_lse=None, steps_budget_s=20.0):
@@ -596,6 +759,9 @@ def main():
     rank, world, local = dist_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.workload.startswith("prefill"):
+        run_prefill(args, rank, world, local)
         return
     run_mq(args, rank, world, local)
 

@@ -473,7 +473,10 @@ typedef struct mq_tune_result {
  *     cost(c) = sum_p weight(p) * median_time(c, p),
  *     weight(p) = sum_t launches(t, p) / time_at_defaults(t)
  * over the terms t (decode 4K, decode 64K, the drafter launch, verification of 8
- * drafts), each of weight 1; reported relative to the defaults' cost.
+ * drafts, and prompt prefill of 4K and 64K tokens through mq_prefill_attn when the
+ * geometry allows it), each of weight 1; reported relative to the defaults' cost.
+ * No candidate changes the drafter or prefill launches: their terms are measured
+ * once and enter every candidate's cost at that time.
  * The default is the configuration the cache holds when mq_tune is called.
  *
  * Admission.  MQ_ADMIT_BIT_IDENTICAL keeps a candidate only if its out and lse

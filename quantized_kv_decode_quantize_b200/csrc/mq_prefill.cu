@@ -39,7 +39,7 @@ constexpr int kPNS = 2;                      // ring stages (chunks of 8 pages)
 constexpr int kPNK = 2;                      // fp16 key buffers
 constexpr int kPNV = 1;                      // value buffers (each an fp16 pair hi + lo)
 constexpr int kPNSB = 2;                     // score buffers (TMEM)
-constexpr int kPNP = 1;                      // P buffers (TMEM)
+constexpr int kPNP = 2;                      // P buffers (TMEM)
 constexpr float kPLazy = 8.0f;               // lazy-max threshold (log2 units): p <= 256
 constexpr int kPOpBytes = kChunkTokens * kPD * 2;   // one fp16 operand tile (128 x 128)
 // tensor memory: S buffers (128 fp32 columns each), O (D columns), P (64 columns)

@@ -9,8 +9,11 @@
 //     cost(c) = sum_p weight(p) * median_time(c, p),
 //     weight(p) = sum_t term_weight(t) * launches(t, p) / time_at_defaults(t)
 // over the terms t = decode_4k, decode_64k, draft_64k (mq_draft_ngram over a 64K-token
-// history) and verify8_64k, each of weight 1 (the speculative-step probe holds one
-// launch of each of its two terms); timing passes read data sized beyond the
+// history), verify8_64k, and the 4k and 64k prompt prefill (mq_prefill_attn), each of
+// weight 1 (the speculative-step probe holds one launch of each of its two terms).  No
+// candidate changes how the drafter or the prefill launch, so their terms are measured
+// once at the defaults and enter every candidate's cost at that time; timing passes
+// read data sized beyond the
 // last-level cache (here: rotating probe caches that together exceed twice the L2
 // size), so no launch finds its data warm; structurally different candidates are
 // tried before refinements of one; a candidate is started only when the budget
@@ -83,6 +86,9 @@ struct Buffers {
     int32_t* cu = nullptr;
     int32_t* start = nullptr;
     int32_t* tokens = nullptr;   // the drafter's 64K-token history
+    void* q_pf = nullptr;        // prefill probes: q of a 64K-token prompt, and its out
+    float* out_pf = nullptr;
+    int32_t* pf_lens = nullptr;  // [2]: 4096, 65536
     int32_t* drafts = nullptr;
     int32_t* n_drafts = nullptr;
     void* kv = nullptr;          // staging for K and V
@@ -99,7 +105,8 @@ struct Buffers {
     cudaEvent_t ev[2] = {nullptr, nullptr};
     cudaStream_t st = nullptr;
     ~Buffers() {
-        void* ptrs[] = {pool, bt, lens, nq, cu, start, tokens, drafts, n_drafts, kv, q, out, lse, ws, flag, pert,
+        void* ptrs[] = {pool, bt, lens, nq, cu, start, tokens, drafts, n_drafts, q_pf, out_pf, pf_lens, kv, q, out, lse,
+                        ws, flag, pert,
                         out_ref[0], out_ref[1], out_ref[2], lse_ref[0], lse_ref[1], lse_ref[2],
                         noise_out[0], noise_out[1], noise_out[2], noise_lse[0], noise_lse[1], noise_lse[2]};
         for (void* p : ptrs)
@@ -324,6 +331,36 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         std::sort(ts.begin(), ts.end());
         t_draft_default = ts[ts.size() / 2] * 1e-3;
     }
+    // the prompt-prefill terms (4k and 64k prompts over the probe cache; head_dim 128 and
+    // a group size dividing 128, else not part of the cost)
+    double t_pf[2] = {0, 0};
+    const bool with_prefill = D == 128 && G <= 128 && 128 % G == 0;
+    if (with_prefill) {
+        const size_t pf_q = (size_t)65536 * Hq * D;
+        int32_t pl[2] = {4096, 65536};
+        if (!ck(cudaMalloc(&B.q_pf, pf_q * 2)) || !ck(cudaMalloc(&B.out_pf, pf_q * 4)) ||
+            !ck(cudaMalloc(&B.pf_lens, sizeof pl)) ||
+            !ck(cudaMemcpy(B.pf_lens, pl, sizeof pl, cudaMemcpyHostToDevice)) ||
+            !ck(launch_fill_random(B.q_pf, 1, (long long)pf_q, D, 0x7066ull, B.st)))
+            return MQ_ERR_CUDA;
+        for (int k = 0; k < 2; k++) {
+            std::vector<float> ts;
+            for (int r = 0; r < (k == 0 ? reps : 3); r++) {
+                cudaEventRecord(B.ev[0], B.st);
+                if (mq_prefill_attn(&probe_cache, B.q_pf, MQ_BF16, 1, Hq, pl[k], pl[k], pl[k], B.bt, blocks_per_copy,
+                                    B.pf_lens + k, B.pf_lens + k, 1.0f / std::sqrt((float)D), B.out_pf, nullptr,
+                                    reinterpret_cast<mq_stream>(B.st)) != MQ_OK)
+                    return MQ_ERR_CUDA;
+                cudaEventRecord(B.ev[1], B.st);
+                if (!ck(cudaEventSynchronize(B.ev[1]))) return MQ_ERR_CUDA;
+                float ms = 0;
+                cudaEventElapsedTime(&ms, B.ev[0], B.ev[1]);
+                ts.push_back(ms);
+            }
+            std::sort(ts.begin(), ts.end());
+            t_pf[k] = ts[ts.size() / 2] * 1e-3;
+        }
+    }
     // weight(p) = sum_t launches(t, p) / time_at_defaults(t): a probe with a drafter holds
     // one launch of the drafter term and one of its decode term, whose time at the
     // defaults is the probe's time less the drafter's
@@ -478,6 +515,11 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         total += best * terms;
         n_terms += terms;
     }
+    // the prefill terms: the same time for every candidate, weight 1 / time each
+    if (with_prefill) {
+        total += 2.0;
+        n_terms += 2;
+    }
     res->cost = n_terms ? total / n_terms : 1.0;
     mq_status status = exhausted ? MQ_TUNE_BUDGET_EXHAUSTED : MQ_OK;
     bool stored = false;
@@ -512,6 +554,10 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
                              "{\"name\": \"verify8_64k\", \"default_us\": %.3f}",
                              t_draft_default * 1e6, kDraftN, kDraftK,
                              std::max(probes[2].t_default - t_draft_default, 0.0) * 1e6);
+            if (with_prefill)
+                std::fprintf(f, ", {\"name\": \"prefill_4k\", \"default_us\": %.3f, \"prompt_tokens\": 4096}, "
+                             "{\"name\": \"prefill_64k\", \"default_us\": %.3f, \"prompt_tokens\": 65536}",
+                             t_pf[0] * 1e6, t_pf[1] * 1e6);
             std::fprintf(f, "],\n  \"probes\": [");
             for (int p = 0; p < P; p++)
                 std::fprintf(f, "%s{\"name\": \"%s\", \"seq_len\": %d, \"n_q\": %d, \"rows_class\": %d, "
