@@ -856,7 +856,7 @@ __global__ void __launch_bounds__(1024) merge_kernel(const DecodeParams p) {
 }
 
 size_t decode_smem_bytes(int head_dim, int rows, int stages) {
-    if (rows <= 8) return small_smem_bytes(head_dim, rows, stages);
+    return small_smem_bytes(head_dim, rows, stages);
 #define MQ_SMEM(DD, RR) \
     if (head_dim == DD && rows == RR) return smem_layout<DD, RR>(stages).total;
     MQ_SMEM(128, 16) MQ_SMEM(128, 32) MQ_SMEM(256, 16)
@@ -874,11 +874,11 @@ static cudaError_t set_smem(size_t smem) {
 }
 
 int decode_ctas_per_sm(int head_dim, int rows) {
-    return rows <= 8 ? small_ctas_per_sm(head_dim, rows) : 1;
+    return small_ctas_per_sm(head_dim, rows);
 }
 
 cudaError_t decode_prepare(int head_dim, int rows, size_t smem) {
-    if (rows <= 8) return small_prepare(head_dim, rows, smem);
+    return small_prepare(head_dim, rows, smem);
     if (head_dim == 128 && rows == 16) return set_smem<128, 16>(smem);
     if (head_dim == 128 && rows == 32) return set_smem<128, 32>(smem);
     if (head_dim == 256 && rows == 16) return set_smem<256, 16>(smem);
@@ -922,11 +922,7 @@ static cudaError_t launch_wide(const DecodeParams& p, dim3 grid, size_t smem, cu
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int max_splits, size_t smem,
                           cudaStream_t st) {
     const dim3 grid((unsigned)max_splits, (unsigned)(p.n_kv_heads * p.n_rb), (unsigned)p.n_seqs);
-    cudaError_t e = cudaErrorInvalidValue;
-    if (rows <= 8) e = small_launch(p, head_dim, rows, grid, smem, st);
-    else if (head_dim == 128 && rows == 16) e = launch_wide<128, 16>(p, grid, smem, st);
-    else if (head_dim == 128 && rows == 32) e = launch_wide<128, 32>(p, grid, smem, st);
-    else if (head_dim == 256 && rows == 16) e = launch_wide<256, 16>(p, grid, smem, st);
+    const cudaError_t e = small_launch(p, head_dim, rows, grid, smem, st);
     if (e != cudaSuccess || max_splits <= 1) return e;
 #define MQ_MERGE(DD, RR) \
     if (head_dim == DD && rows == RR) return launch_merge<DD, RR>(p, grid, max_splits, st);

@@ -74,6 +74,12 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t x) {
     const uint32_t biased = lop_and_xor(x, 0x000F000Fu, 0x64086408u);   // fp16 (1024 + code + 8) x 2
     return h2_as_u32(__hsub2(u32_as_h2(biased), u32_as_h2(0x64086408u)));
 }
+// The same for the codes in bits 4-7 and 20-23, read in place: under exponent 2^6 the
+// nibble is the mantissa's bits 4-7 (steps of 1/16 x 16 = 1), so the pair is 64 + code + 8.
+__device__ __forceinline__ uint32_t code_pair_hi(uint32_t x) {
+    const uint32_t biased = lop_and_xor(x, 0x00F000F0u, 0x54805480u);   // fp16 (64 + code + 8) x 2
+    return h2_as_u32(__hsub2(u32_as_h2(biased), u32_as_h2(0x54805480u)));
+}
 
 
 // ---- q -> three signed 8-bit limbs of a 23-bit fixed-point value per row ----------------

@@ -48,26 +48,32 @@ struct Sm {
     // each with half of tensor memory and of the registers), one for the others
     static constexpr int CPS = (D == 128 && ROWS == 4) ? 2 : 1;
     static constexpr int TCOLS = CPS == 2 ? 256 : 512;      // tensor-memory columns per CTA
-    static constexpr int NSB = 4;                           // score buffers
+    // buffer depths that fill tensor memory for each class
+    static constexpr int NSB = ROWS == 32 ? 1 : ((D == 256 && ROWS == 16) ? 2 : 4);   // score buffers
     static constexpr int NOB = 2;                           // per-chunk value accumulators
-    static constexpr int NVB = 2;                           // V^T buffers
+    static constexpr int NVB = (D == 256 && ROWS == 16) ? 1 : 2;   // V^T buffers
     static constexpr int NWB = 2;                           // weight buffers (shared memory)
     static constexpr int NPB = 2;                           // value-MMA completion barriers
-    static constexpr int NML = NWB + NOB;                   // slots of the chunk maxima and sums
-    static constexpr int THREADS = 352;                     // 0 TMA, 1 QK, 2 PV, 3-6 values, 7-10 softmax
+    static constexpr int NML = NWB + NOB;                   // slots of the chunk maxima
+    // softmax warp groups: 32-row blocks split their rows over two groups of four warps
+    // (one warp per TMEM lane quadrant each); rows meet only through the chunk maximum of
+    // each row, which a group exchanges on its own named barrier
+    static constexpr int NSG = ROWS == 32 ? 2 : 1;
+    static constexpr int RPG = ROWS / NSG;                  // rows per group
+    static constexpr int THREADS = 224 + 128 * NSG;         // 0 TMA, 1 QK, 2 PV, 3-6 values, 7.. softmax
     static constexpr int T_S = 0;
     static constexpr int T_O = NSB * NQ;
     static constexpr int T_VT = (T_O + NOB * H * NO + 31) / 32 * 32;
     static constexpr int T_END = T_VT + NVB * H * 64;
     static constexpr int WBYTES = kChunkTokens * NB * 2;    // one weight buffer
     static constexpr int LBO_W = NB / 8 * 128;              // its 8-token group stride
-    static_assert(ROWS == 4 || ROWS == 8, "row class");
+    static_assert(ROWS == 4 || ROWS == 8 || ROWS == 16 || ROWS == 32, "row class");
     static_assert(T_END <= TCOLS, "tensor memory budget");
     static_assert(NPB >= NOB && NPB >= NVB && NPB >= NWB, "completion barriers");
 };
 
 struct SmallSmem {
-    size_t ring, wbuf, qlimb, xch, xm, xl, crow, lim, pgbad, mbar, misc, total;
+    size_t ring, wbuf, qlimb, xch, xm, lp, xl, crow, lim, pgbad, mbar, misc, total;
 };
 
 // NS = ring stages (chunks of 8 pages)
@@ -87,10 +93,12 @@ __host__ __device__ inline SmallSmem small_layout(int NS) {
     off += (size_t)T::NQ * D;
     s.xch = off;                                  // [2][ROWS][4 warps] chunk row maxima
     off += (size_t)2 * ROWS * 4 * 4;
-    s.xm = off;                                   // [NML][ROWS] chunk row maxima (merged)
-    off += (size_t)T::NML * ROWS * 4;
-    s.xl = off;                                   // [4 warps][ROWS] the softmax warps' shares of l
-    off += (size_t)4 * ROWS * 4;
+    s.xm = off;                                   // [NML][ROWS] merge factors (a, b) of each chunk
+    off += (size_t)T::NML * ROWS * 8;
+    s.lp = off;                                   // [2][4 warps][ROWS] chunk sums of p (fixed point)
+    off += (size_t)2 * 4 * ROWS * 4;
+    s.xl = off;                                   // [2][ROWS] the CTA's row maxima and l
+    off += (size_t)2 * ROWS * 4;
     s.crow = off;
     off += (size_t)ROWS * 4;
     s.lim = off;
@@ -150,8 +158,9 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
     int* lim_s = reinterpret_cast<int*>(smem + S.lim);
     int* pgbad = reinterpret_cast<int*>(smem + S.pgbad);
     float* xch = reinterpret_cast<float*>(smem + S.xch);
-    float* xm = reinterpret_cast<float*>(smem + S.xm);
-    float* xlf = reinterpret_cast<float*>(smem + S.xl);   // [4 softmax warps][ROWS] shares of l
+    float2* xm = reinterpret_cast<float2*>(smem + S.xm);
+    uint32_t* lpart = reinterpret_cast<uint32_t*>(smem + S.lp);
+    float* xlf = reinterpret_cast<float*>(smem + S.xl);   // [ROWS] maxima, then [ROWS] l
     const uint32_t bar0 = smem_u32(smem + S.mbar);
     auto full_b = [&](int s) { return bar0 + 8u * (uint32_t)s; };
     auto empty_b = [&](int s) { return bar0 + 8u * (uint32_t)(NS + s); };
@@ -180,17 +189,17 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; s++) {
             mbar_init(full_b(s), 1);
-            mbar_init(empty_b(s), 9);   // QK commit + 4 value warps + 4 softmax warps
+            mbar_init(empty_b(s), 5 + 4 * T::NSG);   // QK commit + 4 value warps + the softmax warps
         }
         for (int j = 0; j < T::NSB; j++) {
             mbar_init(sfull_b + 8 * j, 1);
-            mbar_init(sfree_b + 8 * j, 4);
+            mbar_init(sfree_b + 8 * j, 4 * T::NSG);
         }
-        for (int j = 0; j < T::NWB; j++) mbar_init(wfull_b + 8 * j, 4);
+        for (int j = 0; j < T::NWB; j++) mbar_init(wfull_b + 8 * j, 4 * T::NSG);
         for (int j = 0; j < T::NVB; j++) mbar_init(vfull_b + 8 * j, 4);
         for (int j = 0; j < T::NPB; j++) mbar_init(pvdone_b + 8 * j, 1);
         for (int j = 0; j < T::NOB; j++) mbar_init(ofree_b + 8 * j, 4);
-        for (int j = 0; j < T::NML; j++) mbar_init(mready_b + 8 * j, 4);
+        for (int j = 0; j < T::NML; j++) mbar_init(mready_b + 8 * j, 4 * T::NSG);
         mbar_fence_init();
         misc[1] = 0;
     }
@@ -209,8 +218,8 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
     __syncthreads();
     const int qoff = misc[0];
     if (warp >= 7) {
-        q_to_limbs<D, ROWS, T::NQ>(p, smem + S.qlimb, crow_s, lim_s, threadIdx.x - 224, 128, row0, rows_here, qoff, L,
-                                   nq, hk);
+        q_to_limbs<D, ROWS, T::NQ>(p, smem + S.qlimb, crow_s, lim_s, threadIdx.x - 224, 128 * T::NSG, row0, rows_here,
+                                   qoff, L, nq, hk);
         fence_proxy_async_smem();
     }
     // the TMA producer starts at once; the other warps wait for the limbs and TMEM
@@ -219,15 +228,12 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
     const uint32_t tmem = (uint32_t)misc[3];
     const uint32_t ring = smem_u32(smem + S.ring);
 
-    // the CTA's running result, held by the value warps (lane = channel of each half)
-    float Or[T::H][ROWS], Mr[ROWS], lr[ROWS];
+    // the CTA's running output, held by the value warps (lane = channel of each half)
+    float Or[T::H][ROWS];
 #pragma unroll
-    for (int r = 0; r < ROWS; r++) {
-        Mr[r] = -INFINITY;
-        lr[r] = 0.0f;
+    for (int r = 0; r < ROWS; r++)
 #pragma unroll
         for (int h = 0; h < T::H; h++) Or[h][r] = 0.0f;
-    }
 
     if (warp == 0) {
         // ================= TMA producer =================
@@ -339,46 +345,44 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
     } else if (warp < 7) {
         // ============ value codes -> V^T in tensor memory; merge of the chunk results ============
         const int q = warp & 3;
-        // Chunk j's value accumulator, row maxima and sums of p, merged into the running
-        // result by log-sum-exp (merge_coef / merge_val: the merge kernel's arithmetic).
+        // Chunk j's value accumulator, merged into the running output with the chunk's
+        // log-sum-exp factors (a, b) per row, which the softmax computed once per row
+        // (merge_val: the merge kernel's arithmetic).
         auto merge_chunk = [&](int j) -> bool {
             if (!wait_warp(pv_bar(j), pv_par(j))) return false;
             const int slot = j % T::NML;
             if (!wait_warp(mready_b + 8 * slot, (uint32_t)(j / T::NML) & 1u)) return false;
-            // this chunk's row maxima, read before the accumulator is released (its release
-            // lets the softmax reach chunk j + NML, which reuses the slot)
-            float mj[ROWS];
-#pragma unroll
-            for (int r = 0; r < ROWS; r++) mj[r] = xm[slot * ROWS + r];
+            // Row groups of up to 16: each reads its factors (before the accumulator is
+            // released: the release lets the softmax reach chunk j + NML, which reuses the
+            // slot) and its accumulator columns, and merges them.
+            constexpr int RG = ROWS < 16 ? ROWS : 16;
             tc_fence_after();
-            float o[T::H][ROWS];
 #pragma unroll
-            for (int h = 0; h < T::H; h++) {
-                const uint32_t col = T::T_O + (j % T::NOB) * T::H * T::NO + h * T::NO + q * ROWS;
-                if constexpr (ROWS == 4) {
-                    uint32_t v[4];
-                    tmem_ld4(tmem_at(tmem, 32 * q, col), v);
+            for (int g0 = 0; g0 < ROWS; g0 += RG) {
+                float2 f[RG];
+#pragma unroll
+                for (int r = 0; r < RG; r++) f[r] = xm[slot * ROWS + g0 + r];
+                float o[T::H][RG];
+#pragma unroll
+                for (int h = 0; h < T::H; h++) {
+                    const uint32_t col = T::T_O + (j % T::NOB) * T::H * T::NO + h * T::NO + q * ROWS + g0;
+                    uint32_t v[RG];
+                    if constexpr (RG == 4) tmem_ld4(tmem_at(tmem, 32 * q, col), v);
+                    else if constexpr (RG == 8) tmem_ld8(tmem_at(tmem, 32 * q, col), v);
+                    else tmem_ld16(tmem_at(tmem, 32 * q, col), v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int r = 0; r < 4; r++) o[h][r] = __uint_as_float(v[r]);
-                } else {
-                    uint32_t v[8];
-                    tmem_ld8(tmem_at(tmem, 32 * q, col), v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int r = 0; r < 8; r++) o[h][r] = __uint_as_float(v[r]);
+                    for (int r = 0; r < RG; r++) o[h][r] = __uint_as_float(v[r]);
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(ofree_b + 8 * (j % T::NOB));
+                if (g0 + RG == ROWS) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(ofree_b + 8 * (j % T::NOB));
+                }
 #pragma unroll
-            for (int r = 0; r < ROWS; r++) {
-                float m, l, a, bc;
-                merge_coef(Mr[r], 0.0f, mj[r], 0.0f, m, l, a, bc);
+                for (int r = 0; r < RG; r++)
 #pragma unroll
-                for (int h = 0; h < T::H; h++) Or[h][r] = merge_val(Or[h][r], o[h][r], a, bc);
-                Mr[r] = m;
+                    for (int h = 0; h < T::H; h++) Or[h][g0 + r] = merge_val(Or[h][g0 + r], o[h][r], f[r].x, f[r].y);
             }
             return true;
         };
@@ -387,8 +391,11 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
         uint32_t ph = 0;   // ring stage of chunk i and the parity of its fill
         for (int i = 0; i < n_ck && ok; i++) {
             const int vb = i % T::NVB;
-            // the V^T buffer of chunk i - 2 is free: its value MMAs were waited for when
-            // chunk i - 2 was merged (in iteration i - 1)
+            // the V^T buffer of chunk i - NVB is free: its value MMAs were waited for when
+            // that chunk was merged (in iteration i - 1, or just below with one buffer)
+            if constexpr (T::NVB == 1) {
+                if (i > 0 && !(ok = merge_chunk(i - 1))) break;
+            }
             if (!wait_warp(full_b(s), ph)) {
                 ok = false;
                 break;
@@ -408,9 +415,9 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
                             const uint32_t w = ldsa32(cw + (uint32_t)((4 * pp + p4) * T::PB + tg * T::REC));
                             // tokens (2k, 2k+1) of the record: bits 4k..4k+3 and 16+4k..
                             r[8 * p4 + 4 * tg + 0] = code_pair(w);
-                            r[8 * p4 + 4 * tg + 1] = code_pair(w >> 4);
+                            r[8 * p4 + 4 * tg + 1] = code_pair_hi(w);
                             r[8 * p4 + 4 * tg + 2] = code_pair(w >> 8);
-                            r[8 * p4 + 4 * tg + 3] = code_pair(w >> 12);
+                            r[8 * p4 + 4 * tg + 3] = code_pair_hi(w >> 8);
                         }
                     tmem_st32(tmem_at(tmem, 32 * q, T::T_VT + (vb * T::H + h) * 64 + 32 * pp), r);
                 }
@@ -426,32 +433,49 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
                 s = 0;
                 ph ^= 1u;
             }
-            if (i > 0) ok = merge_chunk(i - 1);
+            if constexpr (T::NVB > 1) {
+                if (i > 0) ok = merge_chunk(i - 1);
+            }
         }
         if (ok) ok = merge_chunk(n_ck - 1);
         tc_fence_before();
     } else {
         // ================= softmax and weights (one TMEM lane = one token) =================
-        const int sw = warp - 7, q = warp & 3, t = 32 * q + lane;
+        // group sg takes rows r0g .. r0g + RPG - 1; its warp k reads TMEM lane quadrant q
+        constexpr int RPG = T::RPG;
+        const int sg = (warp - 7) >> 2, sw = (warp - 7) & 3, q = warp & 3, t = 32 * q + lane;
+        const int r0g = sg * RPG;
         const int tp = t / 16, ttg = (t / 8) & 1, tt = t & 7;
         const uint32_t wb0 = smem_u32(smem + S.wbuf);
-        float crow[ROWS];
-        int lim[ROWS];
+        // row factors and limits: registers for up to 8 rows, shared memory beyond
+        constexpr bool RREG = RPG <= 8;
+        float crow[RREG ? RPG : 1];
+        int lim[RREG ? RPG : 1];
+        if constexpr (RREG) {
 #pragma unroll
-        for (int r = 0; r < ROWS; r++) {
-            crow[r] = crow_s[r];
-            lim[r] = lim_s[r];
+            for (int r = 0; r < RPG; r++) {
+                crow[r] = crow_s[r0g + r];
+                lim[r] = lim_s[r0g + r];
+            }
         }
+        auto crow_of = [&](int r) { if constexpr (RREG) return crow[r]; else return crow_s[r0g + r]; };
+        auto lim_of = [&](int r) { if constexpr (RREG) return lim[r]; else return lim_s[r0g + r]; };
         const int lim_min = p.causal ? L - nq + row0 / p.group + 1 : L;   // smallest limit of the real rows
-        // The running row maxima over the chunks so far (the same in every softmax warp: they
-        // see the same chunk maxima) and this token's share of l = sum_t 2^(z_t - max), kept
-        // relative to them; the shares are summed once, after the last chunk.
-        float Mrun[ROWS], lt[ROWS];
+        // Row state, one lane per row: lane r < RPG of the group's warp 0 keeps row
+        // r0g + r's running maximum M and l = sum_t 2^(z_t - M) over the chunks so far.  Per
+        // chunk it forms the merge factors a = 2^(M_old - M), b = 2^(m_chunk - M) for the
+        // value warps, and folds in the chunk's sum of p one chunk late (the four warps'
+        // sums of chunk i are in shared memory once the group meets for chunk i + 1).
+        const bool leader = sw == 0 && lane < RPG;
+        float Mrow = -INFINITY, lrow = 0.0f, a_last = 1.0f, b_last = 0.0f;
+        // l of the chunk whose sums of p sit in buffer pb: the four warps' sums of
+        // bits(1 + p_t), less 128 x bits(1.0), are sum_t round(p_t * 2^23) < 2^31
+        auto fold_l = [&](int pb) {
+            uint32_t u = 0u - 128u * 0x3F800000u;
 #pragma unroll
-        for (int r = 0; r < ROWS; r++) {
-            Mrun[r] = -INFINITY;
-            lt[r] = 0.0f;
-        }
+            for (int k = 0; k < 4; k++) u += lpart[(pb * 4 + k) * ROWS + r0g + lane];
+            lrow = __fadd_rn(__fmul_rn(lrow, a_last), __fmul_rn(__fmul_rn((float)u, 0x1p-23f), b_last));
+        };
         // A warp whose wait gave up keeps iterating without work, so that the four warps
         // always meet at their named barrier the same number of times.
         bool ok = true;
@@ -460,25 +484,26 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
         for (int i = 0; i < n_ck; i++) {
             const int sb = i % T::NSB, wb = i % T::NWB, slot = i % T::NML;
             const int c = c0 + i;
-            float sk = 0.0f, sv[T::G];
+            float sk = 0.0f;
+            uint32_t sv2[T::G];   // the token's value scales as fp16 pairs (s_v[g], s_v[g])
             bool any_bad = false, my_bad = false;
-            float z[ROWS];
+            float z[RPG];
             if (ok && wait_warp(full_b(s), ph)) {
                 const uint32_t rec = ring + (uint32_t)((s * kChunkPages + tp) * T::PB + ttg * T::REC);
                 sk = h_bits_to_f32(ldsa16(rec + rec_ks_off(D) + 2 * tt));
                 if constexpr (T::G == 4) {
                     const uint2 v = ldsa64(rec + rec_vs_off(D) + 8 * tt);
-                    sv[0] = h_bits_to_f32(v.x & 0xFFFFu);
-                    sv[1] = h_bits_to_f32(v.x >> 16);
-                    sv[2] = h_bits_to_f32(v.y & 0xFFFFu);
-                    sv[3] = h_bits_to_f32(v.y >> 16);
+                    sv2[0] = __byte_perm(v.x, 0u, 0x1010);
+                    sv2[1] = __byte_perm(v.x, 0u, 0x3232);
+                    sv2[2] = __byte_perm(v.y, 0u, 0x1010);
+                    sv2[3] = __byte_perm(v.y, 0u, 0x3232);
                 } else {
                     const uint4 v = ldsa128(rec + rec_vs_off(D) + 16 * tt);
                     const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int k = 0; k < 4; k++) {
-                        sv[2 * k] = h_bits_to_f32(u[k] & 0xFFFFu);
-                        sv[2 * k + 1] = h_bits_to_f32(u[k] >> 16);
+                        sv2[2 * k] = __byte_perm(u[k], 0u, 0x1010);
+                        sv2[2 * k + 1] = __byte_perm(u[k], 0u, 0x3232);
                     }
                 }
                 const int4 bf0 = *reinterpret_cast<const int4*>(pgbad + s * kChunkPages);
@@ -492,13 +517,26 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
             }
             if (ok && !wait_warp(sfull_b + 8 * sb, (uint32_t)(i / T::NSB) & 1u)) ok = false;
             const bool clean = (c + 1) * kChunkTokens <= lim_min && !any_bad;
-            float* xb = xch + (i & 1) * ROWS * 4;
+            float* xb = xch + (i & 1) * ROWS * 4 + r0g * 4;
             if (ok) {
                 tc_fence_after();
                 // ---- scores: the three limb accumulations of each row -> fp32 ----
-                uint32_t a[3 * ROWS];
+                uint32_t a[3 * RPG];
                 const uint32_t col = T::T_S + sb * T::NQ;
-                if constexpr (ROWS == 4) {
+                if constexpr (RPG == 16) {
+                    // limb l of row r sits in column l * ROWS + r
+                    uint32_t v0[16], v1[16], v2[16];
+                    tmem_ld16(tmem_at(tmem, 32 * q, col + r0g), v0);
+                    tmem_ld16(tmem_at(tmem, 32 * q, col + ROWS + r0g), v1);
+                    tmem_ld16(tmem_at(tmem, 32 * q, col + 2 * ROWS + r0g), v2);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 16; k++) {
+                        a[k] = v0[k];
+                        a[16 + k] = v1[k];
+                        a[32 + k] = v2[k];
+                    }
+                } else if constexpr (ROWS == 4) {
                     uint32_t v[16];
                     tmem_ld16(tmem_at(tmem, 32 * q, col), v);
                     tmem_wait_ld();
@@ -518,87 +556,112 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
                 __syncwarp();
                 if (lane == 0) mbar_arrive(sfree_b + 8 * sb);
 #pragma unroll
-                for (int r = 0; r < ROWS; r++) {
-                    const int x = (int)a[r] * 256 + (int)a[ROWS + r];   // exact: |x| < 2^30
-                    const float sc = __fmaf_rn((float)x, 256.0f, (float)(int)a[2 * ROWS + r]);
-                    z[r] = r < rows_here ? __fmul_rn(__fmul_rn(sc, crow[r]), sk) : -INFINITY;
+                for (int r = 0; r < RPG; r++) {
+                    // every limb sum is below 2^22 in magnitude: exact as fp32 through the
+                    // 1.5 x 2^23 bias (integer add, float subtract)
+                    const float f0 = __fsub_rn(__int_as_float((int)a[r] + 0x4B400000), 12582912.0f);
+                    const float f1 = __fsub_rn(__int_as_float((int)a[RPG + r] + 0x4B400000), 12582912.0f);
+                    const float f2 = __fsub_rn(__int_as_float((int)a[2 * RPG + r] + 0x4B400000), 12582912.0f);
+                    const float sc = __fmaf_rn(f0, 65536.0f, __fmaf_rn(f1, 256.0f, f2));
+                    z[r] = r0g + r < rows_here ? __fmul_rn(__fmul_rn(sc, crow_of(r)), sk) : -INFINITY;
                 }
                 // ---- visibility: sequence end, causal drafts, unusable pages ----
                 if (!clean) {
                     const int tok = c * kChunkTokens + t;
 #pragma unroll
-                    for (int r = 0; r < ROWS; r++)
-                        if (my_bad || tok >= lim[r]) z[r] = -INFINITY;
+                    for (int r = 0; r < RPG; r++)
+                        if (my_bad || tok >= lim_of(r)) z[r] = -INFINITY;
                 }
                 // ---- chunk row maxima over the 128 tokens ----
+                // (the reductions are issued back to back: their latencies overlap)
+                float mx[RPG];
 #pragma unroll
-                for (int r = 0; r < ROWS; r++) {
-                    const float m = warp_redux_max(z[r]);
-                    if (lane == 0) xb[r * 4 + sw] = m;
+                for (int r = 0; r < RPG; r++) mx[r] = warp_redux_max(z[r]);
+                if (lane == 0) {
+#pragma unroll
+                    for (int r = 0; r < RPG; r++) xb[r * 4 + sw] = mx[r];
                 }
             }
-            named_bar_sync(2, 128);
+            named_bar_sync(2 + sg, 128);
             if (ok && i >= T::NWB && !wait_warp(pv_bar(i - T::NWB), pv_par(i - T::NWB))) ok = false;
             if (ok) {
-                // ---- p = 2^(z - chunk max) <= 1, this token's share of l, weights W_g = p * s_v[g] ----
-                float pw[ROWS];
+                // ---- p = 2^(z - chunk max) <= 1, the warp's sums of p, weights W_g = p * s_v[g] ----
+                float pw[RPG];
+                uint32_t* lp = lpart + ((i & 1) * 4 + sw) * ROWS + r0g;
 #pragma unroll
-                for (int r = 0; r < ROWS; r++) {
+                for (int r = 0; r < RPG; r++) {
                     const float4 v = *reinterpret_cast<const float4*>(xb + r * 4);
                     const float cm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
                     pw[r] = z[r] == -INFINITY ? 0.0f : ex2(__fsub_rn(z[r], cm));
-                    const float mn = fmaxf(Mrun[r], cm);
-                    const float al = Mrun[r] == mn ? 1.0f : ex2(__fsub_rn(Mrun[r], mn));
-                    const float be = cm == mn ? 1.0f : ex2(__fsub_rn(cm, mn));
-                    lt[r] = __fadd_rn(__fmul_rn(lt[r], al), __fmul_rn(pw[r], be));
-                    Mrun[r] = mn;
                 }
-                // the chunk's row maxima for the merge of its value accumulator
-                if (sw == 0 && lane < ROWS) {
-                    const float4 v = *reinterpret_cast<const float4*>(xb + lane * 4);
-                    xm[slot * ROWS + lane] = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+                // 1 + p in [1, 2]: its bits are bits(1.0) + round(p * 2^23)
+                uint32_t psum[RPG];
+#pragma unroll
+                for (int r = 0; r < RPG; r++) psum[r] = warp_redux_add(__float_as_uint(__fadd_rn(pw[r], 1.0f)));
+                if (lane == 0) {
+#pragma unroll
+                    for (int r = 0; r < RPG; r++) lp[r] = psum[r];
                 }
                 const uint32_t wrow = wb0 + (uint32_t)(wb * T::WBYTES + (t / 8) * T::LBO_W + (t % 8) * 16);
-                float w[T::G][ROWS];
+                // W_g = fp16(p) * s_v[g], two rows per fp16 pair multiply.  A token that no row
+                // sees (past the sequence end, or on an unusable page) may carry unwritten,
+                // non-finite scales: its scales are taken as 0 (its p is 0 in every row).
+                if (!clean && (my_bad || c * kChunkTokens + t >= L)) {
 #pragma unroll
-                for (int g = 0; g < T::G; g++)
+                    for (int g = 0; g < T::G; g++) sv2[g] = 0u;
+                }
+                uint32_t ph[(RPG + 1) / 2];
 #pragma unroll
-                    for (int r = 0; r < ROWS; r++) {
-                        // masked tokens may carry unwritten (non-finite) scales
-                        w[g][r] = (!clean && pw[r] == 0.0f) ? 0.0f : __fmul_rn(pw[r], sv[g]);
-                    }
-                if constexpr (ROWS == 4) {
+                for (int k = 0; k < RPG / 2; k++) ph[k] = pack_h2(pw[2 * k], pw[2 * k + 1]);
+                auto wpair = [&](int k, int g) { return h2_as_u32(__hmul2(u32_as_h2(ph[k]), u32_as_h2(sv2[g]))); };
+                if constexpr (ROWS > 8) {
+                    // column g * ROWS + r0g + 8k + (0..7) of the weights: one 8-column group each
+#pragma unroll
+                    for (int g = 0; g < T::G; g++)
+#pragma unroll
+                        for (int k = 0; k < RPG / 8; k++)
+                            stsa128(wrow + 128u * (uint32_t)((g * ROWS + r0g) / 8 + k), wpair(4 * k, g),
+                                    wpair(4 * k + 1, g), wpair(4 * k + 2, g), wpair(4 * k + 3, g));
+                } else if constexpr (ROWS == 4) {
                     // column group cg holds groups 2cg and 2cg + 1, rows 0-3 each
 #pragma unroll
                     for (int cg = 0; cg < T::G / 2; cg++)
-                        stsa128(wrow + 128u * cg, pack_h2(w[2 * cg][0], w[2 * cg][1]), pack_h2(w[2 * cg][2], w[2 * cg][3]),
-                                pack_h2(w[2 * cg + 1][0], w[2 * cg + 1][1]), pack_h2(w[2 * cg + 1][2], w[2 * cg + 1][3]));
+                        stsa128(wrow + 128u * cg, wpair(0, 2 * cg), wpair(1, 2 * cg), wpair(0, 2 * cg + 1),
+                                wpair(1, 2 * cg + 1));
                 } else {
 #pragma unroll
                     for (int g = 0; g < T::G; g++)
-                        stsa128(wrow + 128u * g, pack_h2(w[g][0], w[g][1]), pack_h2(w[g][2], w[g][3]),
-                                pack_h2(w[g][4], w[g][5]), pack_h2(w[g][6], w[g][7]));
+                        stsa128(wrow + 128u * g, wpair(0, g), wpair(1, g), wpair(2, g), wpair(3, g));
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(wfull_b + 8 * wb);
-                    mbar_arrive(mready_b + 8 * slot);
+                if (lane == 0) mbar_arrive(wfull_b + 8 * wb);
+                // the row state, after the weights are out: the previous chunk's l, this
+                // chunk's merge factors
+                if (leader) {
+                    if (i > 0) fold_l((i - 1) & 1);
+                    const float4 v = *reinterpret_cast<const float4*>(xb + lane * 4);
+                    const float cm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+                    const float mn = fmaxf(Mrow, cm);
+                    a_last = Mrow == mn ? 1.0f : ex2(__fsub_rn(Mrow, mn));
+                    b_last = cm == mn ? 1.0f : ex2(__fsub_rn(cm, mn));
+                    Mrow = mn;
+                    xm[slot * ROWS + r0g + lane] = make_float2(a_last, b_last);
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(mready_b + 8 * slot);
             }
             if (++s == NS) {
                 s = 0;
                 ph ^= 1u;
             }
         }
-        // l per row: the 128 tokens' shares, summed in a fixed order (warp butterfly, then
-        // the four warps in index order by the value warps after the final barrier)
-#pragma unroll
-        for (int r = 0; r < ROWS; r++) {
-            float v = lt[r];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(FULL, v, o));
-            if (lane == 0) xlf[sw * ROWS + r] = v;
+        // the last chunk's sums of p, then the rows' maxima and l for the epilogue
+        named_bar_sync(2 + sg, 128);
+        if (leader) {
+            if (ok && n_ck > 0) fold_l((n_ck - 1) & 1);
+            xlf[r0g + lane] = Mrow;
+            xlf[ROWS + r0g + lane] = lrow;
         }
     }
 
@@ -611,9 +674,8 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
 
     // ---- the value warps write the CTA's result from registers (lane = channel) ----
     const int q = warp & 3;
-#pragma unroll
-    for (int r = 0; r < ROWS; r++)
-        lr[r] = __fadd_rn(__fadd_rn(__fadd_rn(xlf[r], xlf[ROWS + r]), xlf[2 * ROWS + r]), xlf[3 * ROWS + r]);
+    const float* Mr = xlf;
+    const float* lr = xlf + ROWS;
     const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
     if (n_splits == 1) {
         // out = O / l and lse for the real rows of this block
@@ -639,22 +701,18 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
 #pragma unroll
         for (int h = 0; h < T::H; h++) __stcg(go + r * D + 128 * h + 32 * q + lane, Or[h][r]);
     if (q == 3 && lane < ROWS) {
-        float m = Mr[0], l = lr[0];
-#pragma unroll
-        for (int r = 1; r < ROWS; r++)
-            if (lane == r) {
-                m = Mr[r];
-                l = lr[r];
-            }
-        __stcg(gml + lane, m);
-        __stcg(gml + ROWS + lane, l);
+        __stcg(gml + lane, Mr[lane]);
+        __stcg(gml + ROWS + lane, lr[lane]);
     }
 }
+
+// every row class: head_dim 128 with 4, 8, 16 or 32 rows; head_dim 256 with 4, 8 or 16
+#define MQ_SMALL_CLASSES(X) X(128, 4) X(128, 8) X(128, 16) X(128, 32) X(256, 4) X(256, 8) X(256, 16)
 
 size_t small_smem_bytes(int head_dim, int rows, int stages) {
 #define MQ_SMEM(DD, RR) \
     if (head_dim == DD && rows == RR) return small_layout<DD, RR>(stages).total;
-    MQ_SMEM(128, 4) MQ_SMEM(128, 8) MQ_SMEM(256, 4) MQ_SMEM(256, 8)
+    MQ_SMALL_CLASSES(MQ_SMEM)
 #undef MQ_SMEM
     return 0;
 }
@@ -671,29 +729,34 @@ static cudaError_t small_set_smem(size_t smem) {
 }
 
 cudaError_t small_prepare(int head_dim, int rows, size_t smem) {
-    if (head_dim == 128 && rows == 4) return small_set_smem<128, 4>(smem);
-    if (head_dim == 128 && rows == 8) return small_set_smem<128, 8>(smem);
-    if (head_dim == 256 && rows == 4) return small_set_smem<256, 4>(smem);
-    if (head_dim == 256 && rows == 8) return small_set_smem<256, 8>(smem);
+#define MQ_PREP(DD, RR) \
+    if (head_dim == DD && rows == RR) return small_set_smem<DD, RR>(smem);
+    MQ_SMALL_CLASSES(MQ_PREP)
+#undef MQ_PREP
     return cudaErrorInvalidValue;
 }
 
-// The decode kernel of the small row classes, as a programmatic dependent launch.
-cudaError_t small_launch(const DecodeParams& p, int head_dim, int rows, dim3 grid, size_t smem, cudaStream_t st) {
+template <int D, int ROWS>
+static cudaError_t small_launch_t(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t st) {
     cudaLaunchAttribute pdl[1];
     pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t dc{};
     dc.gridDim = grid;
-    dc.blockDim = dim3(352);
+    dc.blockDim = dim3((unsigned)Sm<D, ROWS>::THREADS);
     dc.dynamicSmemBytes = smem;
     dc.stream = st;
     dc.attrs = pdl;
     dc.numAttrs = 1;
-    if (head_dim == 128 && rows == 4) return cudaLaunchKernelEx(&dc, decode_small_kernel<128, 4>, p);
-    if (head_dim == 128 && rows == 8) return cudaLaunchKernelEx(&dc, decode_small_kernel<128, 8>, p);
-    if (head_dim == 256 && rows == 4) return cudaLaunchKernelEx(&dc, decode_small_kernel<256, 4>, p);
-    if (head_dim == 256 && rows == 8) return cudaLaunchKernelEx(&dc, decode_small_kernel<256, 8>, p);
+    return cudaLaunchKernelEx(&dc, decode_small_kernel<D, ROWS>, p);
+}
+
+// The decode kernel of the row class, as a programmatic dependent launch.
+cudaError_t small_launch(const DecodeParams& p, int head_dim, int rows, dim3 grid, size_t smem, cudaStream_t st) {
+#define MQ_LAUNCH(DD, RR) \
+    if (head_dim == DD && rows == RR) return small_launch_t<DD, RR>(p, grid, smem, st);
+    MQ_SMALL_CLASSES(MQ_LAUNCH)
+#undef MQ_LAUNCH
     return cudaErrorInvalidValue;
 }
 
