@@ -248,7 +248,8 @@ def kernel_source_hash():
     import re
     h = hashlib.sha256()
     d = os.path.join(ROOT, "quantized_kv_decode_quantize_b200", "csrc")
-    for n in ("mq_decode.cu", "mq_device.cuh", "mq_tc.cuh", "mq_kernels.h"):
+    for n in ("mq_decode_small.cu", "mq_decode_common.cuh", "mq_decode.cu", "mq_device.cuh", "mq_tc.cuh",
+              "mq_kernels.h"):
         with open(os.path.join(d, n)) as f:
             src = f.read()
         src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)   # block comments
@@ -724,7 +725,7 @@ def run_mq(args, rank, world, local):
                        "append_GBps": app_bytes / (app_avg * 1e-3) / 1e9 if app_avg else None},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": (achieved / peak) if achieved else None, "peak_kind": peak_kind,
-                         "traffic": ncu_traffic(w.name), "kernel": "mq::decode_kernel",
+                         "traffic": ncu_traffic(w.name), "kernel": "mq::decode_small_kernel",
                          "bytes_per_launch": dec_unique, "kernel_us_mean": kern_avg * 1e3 if kern_avg else None,
                          "kernel_us_median": statistics.median(kern_ms) * 1e3 if kern_ms else None,
                          "kernel_us_p10": pct(kern_ms, 0.1) * 1e3 if kern_ms else None,

@@ -57,8 +57,15 @@ DevGuard::~DevGuard() {
     if (switched && prev >= 0) cudaSetDevice(prev);
 }
 
-// The plan for one row class: rows per CTA, split count, chunks per CTA, ring depth.
-// The chunk ranges depend only on the shape, the SM count and splits_per_sm.
+// The plan for one row class: rows per CTA, split count, chunks per CTA, merge-tree leaf,
+// ring depth.  The chunk ranges depend only on the shape, the SM count and splits_per_sm.
+// For the classes whose CTAs build a node of the fixed merge tree (up to 8 rows: one query
+// token per sequence at GQA <= 8; small_leaf_kmax > 0), the leaf is a fixed run of chunks
+// that depends on the shape alone (at most 2^kmax leaves per unit), every CTA holds an
+// aligned power-of-two run of leaves, and the split count follows from that run: whatever
+// the configured splits per SM, the CTAs and the merge kernel evaluate the same tree, so
+// the output is bit-identical across split counts and ring depths.  The wider classes (draft verification) split into any
+// number of equal ranges, one leaf each (a power of two would idle SMs there).
 static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int rows_total, int max_seq_len) {
     DecodePlan pl{};
     pl.cls = cls;
@@ -72,9 +79,27 @@ static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int row
     const int cps = decode_ctas_per_sm(c->head_dim, pl.rows);
     long long splits = (long long)cfg.splits_per_sm * cps * c->n_sm / units;
     splits = std::max<long long>(1, std::min<long long>({splits, max_chunks, (long long)kMaxSplits}));
-    const long long cpc = (max_chunks + splits - 1) / splits;
-    pl.cpc = (int)cpc;
-    pl.max_splits = (int)((max_chunks + cpc - 1) / cpc);
+    const int kmax = small_leaf_kmax(c->head_dim, pl.rows);
+    if (kmax > 0) {
+        // 2^kmax leaf slots per unit, each leaf ceil(max_chunks / 2^kmax) chunks: the unit
+        // fills the slots up to less than one chunk per slot, so aligned power-of-two CTA
+        // ranges of leaves stay balanced whatever max_chunks is
+        const long long slots = 1LL << kmax;
+        const long long leaf = (max_chunks + slots - 1) / slots;
+        const long long leaves = (max_chunks + leaf - 1) / leaf;
+        long long p2 = 1;
+        while (p2 * 2 <= std::min(splits, leaves)) p2 *= 2;
+        long long lpc = slots / p2;   // leaves per CTA, a power of two
+        while (lpc > 1 && (leaves + lpc / 2 - 1) / (lpc / 2) <= p2) lpc /= 2;
+        pl.node_chunks = (int)leaf;
+        pl.cpc = (int)(lpc * leaf);
+    } else {
+        const long long cpc = (max_chunks + splits - 1) / splits;
+        pl.cpc = (int)cpc;
+        pl.node_chunks = (int)cpc;
+    }
+    pl.max_splits = (int)((max_chunks + pl.cpc - 1) / pl.cpc);
+    pl.merge = pl.max_splits > 1;
     // the ring is shortened (never below 2 stages) until the CTA fits in its share of
     // the SM's shared memory (1 KB of each CTA's share is reserved by the hardware)
     const size_t smem_cap = cps == 1 ? (size_t)c->max_smem
@@ -138,6 +163,7 @@ mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void
     p.split_stride = pl.max_splits;
     p.n_rb = pl.n_rb;
     p.cpc = pl.cpc;
+    p.node_chunks = pl.node_chunks;
     p.stages = pl.stages;
     p.err = c->err_word;
     p.causal = view.causal;
@@ -145,7 +171,7 @@ mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void
     p.bt_col = view.bt_col;
     p.fixed_len = view.fixed_len;
     p.fixed_nq = view.fixed_nq;
-    e = launch_decode(p, c->head_dim, pl.rows, pl.max_splits, pl.smem, st);
+    e = launch_decode(p, c->head_dim, pl.rows, pl.max_splits, pl.merge, pl.smem, st);
     return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
 }
 
@@ -321,7 +347,7 @@ int32_t mq_decode_kernel_count(const mq_cache* c, int32_t n_seqs, int32_t n_q_he
                                int32_t max_seq_len) {
     if (c == nullptr || mq_decode_workspace_bytes(c, n_seqs, n_q_heads, max_q_per_seq, max_seq_len) == 0) return 0;
     const DecodePlan pl = plan_decode(c, n_seqs, n_q_heads, max_q_per_seq, max_seq_len);
-    return pl.max_splits > 1 ? 2 : 1;
+    return pl.merge ? 2 : 1;
 }
 
 mq_status mq_decode_attn(const mq_cache* c, const void* q, mq_dtype q_dtype, int32_t n_seqs, int32_t n_q_heads,

@@ -1,5 +1,5 @@
-// Device helpers shared by the decode kernels (mq_decode.cu: query-row classes of 16 and
-// 32 rows; mq_decode_small.cu: classes of 4 and 8 rows) and the merge kernel.
+// Device helpers shared by the decode kernel (mq_decode_small.cu), the merge kernel
+// (mq_decode.cu) and the prefill kernel (mq_prefill.cu).
 #pragma once
 #include <cfloat>
 #include <climits>
@@ -81,6 +81,36 @@ __device__ __forceinline__ uint32_t code_pair_hi(uint32_t x) {
     return h2_as_u32(__hsub2(u32_as_h2(biased), u32_as_h2(0x54805480u)));
 }
 
+
+// ---- the merge tree over a unit's leaves -----------------------------------------------
+// A unit's leaves are runs of node_chunks chunks; the tree over them is fixed: node (k, i)
+// covers leaves [i 2^k, (i + 1) 2^k), merges nodes (k - 1, 2i) and (k - 1, 2i + 1), and is
+// its left child when the right one starts past the last leaf.  Where the split count is
+// free (the classes of up to 8 rows), a CTA holds an aligned power-of-two run of leaves,
+// i.e. one node of that tree, which it builds with a binary counter (pending left children
+// in slots by level) and publishes as its partial; the merge kernel's tree over the CTAs
+// is the same tree's upper part.  TreeStep is what the CTA does when leaf li is complete.
+struct TreeStep {
+    uint32_t merge_mask;   // slots merged into the new node, in increasing level
+    int level;             // the node's level after the carry
+    bool push;             // kept in slot `level`; else (the CTA's last leaf) it is the CTA's node
+};
+__device__ __forceinline__ TreeStep tree_step(int li, int l0, bool last, uint32_t occ, int kmax) {
+    TreeStep st{};
+    int t = 0, idx = li;
+    // carry: a right child whose left sibling (in this CTA) waits in slot t
+    while (t < kmax && (idx & 1) && ((idx - 1) << t) >= l0) {
+        st.merge_mask |= 1u << t;
+        idx >>= 1;
+        t++;
+    }
+    st.level = t;
+    st.push = !last;
+    // the CTA's last leaf: its right edge, the remaining left children in increasing level
+    // (their right parts lie past the sequence's last leaf)
+    if (last) st.merge_mask |= occ & ~st.merge_mask;
+    return st;
+}
 
 // ---- q -> three signed 8-bit limbs of a 23-bit fixed-point value per row ----------------
 // Q = rint(q * 2^(22 - E)) with |q| < 2^E the row's absmax bound, |Q| <= 2^22, and

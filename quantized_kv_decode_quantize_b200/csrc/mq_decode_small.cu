@@ -54,7 +54,12 @@ struct Sm {
     static constexpr int NVB = (D == 256 && ROWS == 16) ? 1 : 2;   // V^T buffers
     static constexpr int NWB = 2;                           // weight buffers (shared memory)
     static constexpr int NPB = 2;                           // value-MMA completion barriers
-    static constexpr int NML = NWB + NOB;                   // slots of the chunk maxima
+    static constexpr int NML = NWB + NOB;                   // slots of the merge factors
+    // levels of the merge-tree node a CTA builds from its leaves (the classes whose split
+    // count is free: up to 8 rows, where tensor memory has room for the pending children);
+    // 0 for the others, whose leaf is the CTA's range
+    static constexpr int KMAX = (ROWS <= 8 && !(D == 256 && ROWS == 8)) ? 6 : 0;
+    static constexpr int XS = 1 + KMAX;                     // factor pairs per row and chunk
     // softmax warp groups: 32-row blocks split their rows over two groups of four warps
     // (one warp per TMEM lane quadrant each); rows meet only through the chunk maximum of
     // each row, which a group exchanges on its own named barrier
@@ -64,7 +69,8 @@ struct Sm {
     static constexpr int T_S = 0;
     static constexpr int T_O = NSB * NQ;
     static constexpr int T_VT = (T_O + NOB * H * NO + 31) / 32 * 32;
-    static constexpr int T_END = T_VT + NVB * H * 64;
+    static constexpr int T_STK = T_VT + NVB * H * 64;       // pending left children: KMAX x (H x ROWS)
+    static constexpr int T_END = T_STK + KMAX * H * ROWS;
     static constexpr int WBYTES = kChunkTokens * NB * 2;    // one weight buffer
     static constexpr int LBO_W = NB / 8 * 128;              // its 8-token group stride
     static_assert(ROWS == 4 || ROWS == 8 || ROWS == 16 || ROWS == 32, "row class");
@@ -91,12 +97,12 @@ __host__ __device__ inline SmallSmem small_layout(int NS) {
     off = al(off, 128);
     s.qlimb = off;
     off += (size_t)T::NQ * D;
-    s.xch = off;                                  // [2][ROWS][4 warps] chunk row maxima
-    off += (size_t)2 * ROWS * 4 * 4;
-    s.xm = off;                                   // [NML][ROWS] merge factors (a, b) of each chunk
-    off += (size_t)T::NML * ROWS * 8;
-    s.lp = off;                                   // [2][4 warps][ROWS] chunk sums of p (fixed point)
-    off += (size_t)2 * 4 * ROWS * 4;
+    s.xch = off;                                  // [4][ROWS][4 warps] chunk row maxima
+    off += (size_t)4 * ROWS * 4 * 4;
+    s.xm = off;                                   // [NML][XS][ROWS] merge factors (a, b): the chunk's, then its leaf's
+    off += (size_t)T::NML * T::XS * ROWS * 8;
+    s.lp = off;                                   // [4][4 warps][ROWS] chunk sums of p (fixed point)
+    off += (size_t)4 * 4 * ROWS * 4;
     s.xl = off;                                   // [2][ROWS] the CTA's row maxima and l
     off += (size_t)2 * ROWS * 4;
     s.crow = off;
@@ -139,7 +145,14 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
     const int c0 = sp * p.cpc;
     if (c0 >= n_chunks) return;
     const int n_ck = min(c0 + p.cpc, n_chunks) - c0;
-    const int n_splits = (n_chunks + p.cpc - 1) / p.cpc;
+    // The merge tree's leaves are runs of node_chunks chunks, folded in order; the CTA's
+    // range is whole leaves, and its partial is the tree node over them (see tree_step).
+    // The unit's only CTA writes out and lse; otherwise merge_kernel combines the partials.
+    const int node_ch = p.node_chunks;
+    const int l0 = c0 / node_ch, l1 = (c0 + n_ck + node_ch - 1) / node_ch;   // this CTA's leaves
+    const bool direct = (n_chunks + p.cpc - 1) / p.cpc == 1;                // the unit's only CTA
+    const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
+    auto leaf_end = [&](int c) { return c % node_ch == node_ch - 1 || c == n_chunks - 1; };
 
     // block-table entries of the first chunk (warp 0, lanes < 8), loaded before the set-up:
     // the table is an input of the launch that no preceding append writes
@@ -199,7 +212,7 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
         for (int j = 0; j < T::NVB; j++) mbar_init(vfull_b + 8 * j, 4);
         for (int j = 0; j < T::NPB; j++) mbar_init(pvdone_b + 8 * j, 1);
         for (int j = 0; j < T::NOB; j++) mbar_init(ofree_b + 8 * j, 4);
-        for (int j = 0; j < T::NML; j++) mbar_init(mready_b + 8 * j, 4 * T::NSG);
+        for (int j = 0; j < T::NML; j++) mbar_init(mready_b + 8 * j, 1);
         mbar_fence_init();
         misc[1] = 0;
     }
@@ -228,8 +241,10 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
     const uint32_t tmem = (uint32_t)misc[3];
     const uint32_t ring = smem_u32(smem + S.ring);
 
-    // the CTA's running output, held by the value warps (lane = channel of each half)
+    // the CTA's running output, held by the value warps (lane = channel of each half); the
+    // pending left children of its tree node wait in tensor memory
     float Or[T::H][ROWS];
+    uint32_t occ_v = 0u;
 #pragma unroll
     for (int r = 0; r < ROWS; r++)
 #pragma unroll
@@ -316,6 +331,66 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
         // ================= value MMAs (whole warp; one elected lane issues) =================
         const uint32_t wb0 = smem_u32(smem + S.wbuf);
         constexpr uint32_t IDO = instr_desc(1, 0, 0, 0, 1, 128, T::NO);   // f32 <- f16 x f16, B MN-major
+        // The row state, lane r = row r of the block, kept here once the chunk's value MMAs
+        // are issued (off the softmax warps' path): the current leaf's running maximum M
+        // and l = sum_t 2^(z_t - M), and the (M, l) of the pending left children of the
+        // CTA's merge subtrees.  Per chunk it forms the log-sum-exp factors (a, b) for the
+        // value warps' merges: the chunk's into the leaf, then the leaf's into the subtrees.
+        float Mrow = -INFINITY, lrow = 0.0f;
+        float Ms[T::KMAX > 0 ? T::KMAX : 1], ls[T::KMAX > 0 ? T::KMAX : 1];
+        uint32_t occ = 0u;
+        auto row_step = [&](int j) {
+            const int c = c0 + j, xbuf = j & 3;
+            // the chunk's row maximum (the four softmax warps' maxima) and l: their sums of
+            // bits(1 + p_t), less 128 x bits(1.0), are sum_t round(p_t * 2^23) < 2^31
+            const float4 v = *reinterpret_cast<const float4*>(xch + (xbuf * ROWS + lane) * 4);
+            const float cm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+            uint32_t u = 0u - 128u * 0x3F800000u;
+#pragma unroll
+            for (int k = 0; k < 4; k++) u += lpart[(xbuf * 4 + k) * ROWS + lane];
+            const float lc = __fmul_rn((float)u, 0x1p-23f);
+            const float mn = fmaxf(Mrow, cm);
+            const float a = Mrow == mn ? 1.0f : ex2(__fsub_rn(Mrow, mn));
+            const float bb = cm == mn ? 1.0f : ex2(__fsub_rn(cm, mn));
+            Mrow = mn;
+            lrow = __fadd_rn(__fmul_rn(lrow, a), __fmul_rn(lc, bb));
+            float2* xf = xm + (size_t)(j % T::NML) * T::XS * ROWS + lane;
+            xf[0] = make_float2(a, bb);
+            if (!leaf_end(c)) return;
+            // the leaf's merges into the CTA's tree node
+            const int li = c / node_ch;
+            const bool last = li == l1 - 1;
+            const TreeStep st = tree_step(li, l0, last, occ, T::KMAX);
+            int k = 1;
+#pragma unroll
+            for (int t = 0; t < T::KMAX; t++)
+                if ((st.merge_mask >> t) & 1u) {
+                    float m, l, fa, fb;
+                    merge_coef(Ms[t], ls[t], Mrow, lrow, m, l, fa, fb);
+                    xf[k * ROWS] = make_float2(fa, fb);
+                    Mrow = m;
+                    lrow = l;
+                    k++;
+                }
+            if (st.push) {
+#pragma unroll
+                for (int t = 0; t < T::KMAX; t++)
+                    if (t == st.level) {
+                        Ms[t] = Mrow;
+                        ls[t] = lrow;
+                    }
+                occ = (occ & ~st.merge_mask) | (1u << st.level);
+                Mrow = -INFINITY;   // the next leaf starts afresh
+                lrow = 0.0f;
+            } else if (!direct) {
+                float* gml = p.part_ml + (pidx * p.split_stride + sp) * (size_t)(2 * ROWS);
+                __stcg(gml + lane, Mrow);
+                __stcg(gml + ROWS + lane, lrow);
+            } else {
+                xlf[lane] = Mrow;   // the unit's root, for the epilogue
+                xlf[ROWS + lane] = lrow;
+            }
+        };
         uint32_t last_bar = 0, last_par = 0;
         for (int j = 0; j < n_ck; j++) {
             const int wb = j % T::NWB, vb = j % T::NVB, ob = j % T::NOB;
@@ -339,6 +414,11 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
             tc_commit_w(pv_bar(j));
             last_bar = pv_bar(j);
             last_par = pv_par(j);
+            // the chunk's maxima and sums of p are complete (the softmax warps wrote them
+            // before their arrival on wfull)
+            if (lane < ROWS) row_step(j);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(mready_b + 8 * (j % T::NML));
         }
         if (lane == 0 && *abort_flag != 0 && last_bar != 0) mbar_wait_bounded(last_bar, last_par);
         __syncwarp();
@@ -347,21 +427,23 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
         const int q = warp & 3;
         // Chunk j's value accumulator, merged into the running output with the chunk's
         // log-sum-exp factors (a, b) per row, which the softmax computed once per row
-        // (merge_val: the merge kernel's arithmetic).
+        // (merge_val: the merge kernel's arithmetic); at a leaf's end, the leaf's merges
+        // into the CTA's subtrees with the factors that follow.
         auto merge_chunk = [&](int j) -> bool {
             if (!wait_warp(pv_bar(j), pv_par(j))) return false;
             const int slot = j % T::NML;
             if (!wait_warp(mready_b + 8 * slot, (uint32_t)(j / T::NML) & 1u)) return false;
-            // Row groups of up to 16: each reads its factors (before the accumulator is
-            // released: the release lets the softmax reach chunk j + NML, which reuses the
-            // slot) and its accumulator columns, and merges them.
+            // Row groups of up to 16: each reads its factors and its accumulator columns, and
+            // merges them.  (The factor slot stays valid after the accumulator's release: it
+            // is rewritten for chunk j + NML, whose value MMAs wait for the release of chunk
+            // j + NWB's accumulator, i.e. for this warp to be past chunk j.)
             constexpr int RG = ROWS < 16 ? ROWS : 16;
             tc_fence_after();
 #pragma unroll
             for (int g0 = 0; g0 < ROWS; g0 += RG) {
                 float2 f[RG];
 #pragma unroll
-                for (int r = 0; r < RG; r++) f[r] = xm[slot * ROWS + g0 + r];
+                for (int r = 0; r < RG; r++) f[r] = xm[slot * T::XS * ROWS + g0 + r];
                 float o[T::H][RG];
 #pragma unroll
                 for (int h = 0; h < T::H; h++) {
@@ -383,6 +465,57 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
                 for (int r = 0; r < RG; r++)
 #pragma unroll
                     for (int h = 0; h < T::H; h++) Or[h][g0 + r] = merge_val(Or[h][g0 + r], o[h][r], f[r].x, f[r].y);
+            }
+            const int c = c0 + j;
+            if (leaf_end(c)) {
+                const int li = c / node_ch;
+                const bool last = li == l1 - 1;
+                const TreeStep st = tree_step(li, l0, last, occ_v, T::KMAX);
+                const float2* xf = xm + (size_t)slot * T::XS * ROWS;
+                constexpr int HR = T::H * ROWS;
+                if constexpr (T::KMAX > 0) {
+                    int k = 1;
+#pragma unroll 1
+                    for (int t = 0; t < T::KMAX; t++) {
+                        if (!((st.merge_mask >> t) & 1u)) continue;
+                        uint32_t sv[HR];
+                        if constexpr (HR == 4) tmem_ld4(tmem_at(tmem, 32 * q, T::T_STK + t * HR), sv);
+                        else tmem_ld8(tmem_at(tmem, 32 * q, T::T_STK + t * HR), sv);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int r = 0; r < ROWS; r++) {
+                            const float2 fk = xf[k * ROWS + r];
+#pragma unroll
+                            for (int h = 0; h < T::H; h++)
+                                Or[h][r] = merge_val(__uint_as_float(sv[h * ROWS + r]), Or[h][r], fk.x, fk.y);
+                        }
+                        k++;
+                    }
+                }
+                if (st.push) {
+                    if constexpr (T::KMAX > 0) {
+                        uint32_t sv[HR];
+#pragma unroll
+                        for (int h = 0; h < T::H; h++)
+#pragma unroll
+                            for (int r = 0; r < ROWS; r++) sv[h * ROWS + r] = __float_as_uint(Or[h][r]);
+                        if constexpr (HR == 4) tmem_st4(tmem_at(tmem, 32 * q, T::T_STK + st.level * HR), sv);
+                        else tmem_st8(tmem_at(tmem, 32 * q, T::T_STK + st.level * HR), sv);
+                        tmem_wait_st();
+                    }
+#pragma unroll
+                    for (int r = 0; r < ROWS; r++)
+#pragma unroll
+                        for (int h = 0; h < T::H; h++) Or[h][r] = 0.0f;
+                    occ_v = (occ_v & ~st.merge_mask) | (1u << st.level);
+                } else if (!direct) {
+                    // the CTA's node: its partial (lane = channel)
+                    float* go = p.part_o + (pidx * p.split_stride + sp) * (size_t)(ROWS * D);
+#pragma unroll
+                    for (int r = 0; r < ROWS; r++)
+#pragma unroll
+                        for (int h = 0; h < T::H; h++) __stcg(go + r * D + 128 * h + 32 * q + lane, Or[h][r]);
+                }
             }
             return true;
         };
@@ -461,21 +594,6 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
         auto crow_of = [&](int r) { if constexpr (RREG) return crow[r]; else return crow_s[r0g + r]; };
         auto lim_of = [&](int r) { if constexpr (RREG) return lim[r]; else return lim_s[r0g + r]; };
         const int lim_min = p.causal ? L - nq + row0 / p.group + 1 : L;   // smallest limit of the real rows
-        // Row state, one lane per row: lane r < RPG of the group's warp 0 keeps row
-        // r0g + r's running maximum M and l = sum_t 2^(z_t - M) over the chunks so far.  Per
-        // chunk it forms the merge factors a = 2^(M_old - M), b = 2^(m_chunk - M) for the
-        // value warps, and folds in the chunk's sum of p one chunk late (the four warps'
-        // sums of chunk i are in shared memory once the group meets for chunk i + 1).
-        const bool leader = sw == 0 && lane < RPG;
-        float Mrow = -INFINITY, lrow = 0.0f, a_last = 1.0f, b_last = 0.0f;
-        // l of the chunk whose sums of p sit in buffer pb: the four warps' sums of
-        // bits(1 + p_t), less 128 x bits(1.0), are sum_t round(p_t * 2^23) < 2^31
-        auto fold_l = [&](int pb) {
-            uint32_t u = 0u - 128u * 0x3F800000u;
-#pragma unroll
-            for (int k = 0; k < 4; k++) u += lpart[(pb * 4 + k) * ROWS + r0g + lane];
-            lrow = __fadd_rn(__fmul_rn(lrow, a_last), __fmul_rn(__fmul_rn((float)u, 0x1p-23f), b_last));
-        };
         // A warp whose wait gave up keeps iterating without work, so that the four warps
         // always meet at their named barrier the same number of times.
         bool ok = true;
@@ -517,7 +635,7 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
             }
             if (ok && !wait_warp(sfull_b + 8 * sb, (uint32_t)(i / T::NSB) & 1u)) ok = false;
             const bool clean = (c + 1) * kChunkTokens <= lim_min && !any_bad;
-            float* xb = xch + (i & 1) * ROWS * 4 + r0g * 4;
+            float* xb = xch + (i & 3) * ROWS * 4 + r0g * 4;
             if (ok) {
                 tc_fence_after();
                 // ---- scores: the three limb accumulations of each row -> fp32 ----
@@ -587,7 +705,7 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
             if (ok) {
                 // ---- p = 2^(z - chunk max) <= 1, the warp's sums of p, weights W_g = p * s_v[g] ----
                 float pw[RPG];
-                uint32_t* lp = lpart + ((i & 1) * 4 + sw) * ROWS + r0g;
+                uint32_t* lp = lpart + ((i & 3) * 4 + sw) * ROWS + r0g;
 #pragma unroll
                 for (int r = 0; r < RPG; r++) {
                     const float4 v = *reinterpret_cast<const float4*>(xb + r * 4);
@@ -636,32 +754,12 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(wfull_b + 8 * wb);
-                // the row state, after the weights are out: the previous chunk's l, this
-                // chunk's merge factors
-                if (leader) {
-                    if (i > 0) fold_l((i - 1) & 1);
-                    const float4 v = *reinterpret_cast<const float4*>(xb + lane * 4);
-                    const float cm = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
-                    const float mn = fmaxf(Mrow, cm);
-                    a_last = Mrow == mn ? 1.0f : ex2(__fsub_rn(Mrow, mn));
-                    b_last = cm == mn ? 1.0f : ex2(__fsub_rn(cm, mn));
-                    Mrow = mn;
-                    xm[slot * ROWS + r0g + lane] = make_float2(a_last, b_last);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(mready_b + 8 * slot);
+
             }
             if (++s == NS) {
                 s = 0;
                 ph ^= 1u;
             }
-        }
-        // the last chunk's sums of p, then the rows' maxima and l for the epilogue
-        named_bar_sync(2 + sg, 128);
-        if (leader) {
-            if (ok && n_ck > 0) fold_l((n_ck - 1) & 1);
-            xlf[r0g + lane] = Mrow;
-            xlf[ROWS + r0g + lane] = lrow;
         }
     }
 
@@ -676,33 +774,19 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
     const int q = warp & 3;
     const float* Mr = xlf;
     const float* lr = xlf + ROWS;
-    const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
-    if (n_splits == 1) {
-        // out = O / l and lse for the real rows of this block
+    if (!direct) return;   // the leaves are published; the merge kernel writes the output
+    // out = O / l and lse for the real rows of this block
 #pragma unroll
-        for (int r = 0; r < ROWS; r++) {
-            if (r >= rows_here) break;
-            const int rr = row0 + r, j = rr / p.group, hq = rr % p.group;
-            const long long qrow = (long long)qoff + j;
-            if (qrow >= p.total_q) continue;
-            const size_t orow = (size_t)qrow * p.n_q_heads + (size_t)hk * p.group + hq;
+    for (int r = 0; r < ROWS; r++) {
+        if (r >= rows_here) break;
+        const int rr = row0 + r, j = rr / p.group, hq = rr % p.group;
+        const long long qrow = (long long)qoff + j;
+        if (qrow >= p.total_q) continue;
+        const size_t orow = (size_t)qrow * p.n_q_heads + (size_t)hk * p.group + hq;
 #pragma unroll
-            for (int h = 0; h < T::H; h++) p.out[orow * D + 128 * h + 32 * q + lane] = __fdiv_rn(Or[h][r], lr[r]);
-            if (q == 3 && lane == 0 && p.lse != nullptr)
-                p.lse[orow] = __fmul_rn(__fadd_rn(Mr[r], log2f(lr[r])), 0.69314718055994531f);
-        }
-        return;
-    }
-    // ---- publish this CTA's partial; merge_kernel completes the tree ----
-    float* go = p.part_o + (pidx * p.split_stride + sp) * (size_t)(ROWS * D);
-    float* gml = p.part_ml + (pidx * p.split_stride + sp) * (size_t)(2 * ROWS);
-#pragma unroll
-    for (int r = 0; r < ROWS; r++)
-#pragma unroll
-        for (int h = 0; h < T::H; h++) __stcg(go + r * D + 128 * h + 32 * q + lane, Or[h][r]);
-    if (q == 3 && lane < ROWS) {
-        __stcg(gml + lane, Mr[lane]);
-        __stcg(gml + ROWS + lane, lr[lane]);
+        for (int h = 0; h < T::H; h++) p.out[orow * D + 128 * h + 32 * q + lane] = __fdiv_rn(Or[h][r], lr[r]);
+        if (q == 3 && lane == 0 && p.lse != nullptr)
+            p.lse[orow] = __fmul_rn(__fadd_rn(Mr[r], log2f(lr[r])), 0.69314718055994531f);
     }
 }
 
@@ -718,6 +802,14 @@ size_t small_smem_bytes(int head_dim, int rows, int stages) {
 }
 
 int small_ctas_per_sm(int head_dim, int rows) { return (head_dim == 128 && rows == 4) ? 2 : 1; }
+
+int small_leaf_kmax(int head_dim, int rows) {
+#define MQ_KMAX(DD, RR) \
+    if (head_dim == DD && rows == RR) return Sm<DD, RR>::KMAX;
+    MQ_SMALL_CLASSES(MQ_KMAX)
+#undef MQ_KMAX
+    return 0;
+}
 
 template <int D, int ROWS>
 static cudaError_t small_set_smem(size_t smem) {

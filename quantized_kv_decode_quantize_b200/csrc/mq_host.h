@@ -24,6 +24,8 @@ namespace mq {
 
 struct DecodePlan {
     int cls, rows, n_rb, stages, cpc, max_splits;
+    int node_chunks;               // merge-tree leaf (chunks)
+    bool merge;                    // some unit has several CTAs (merge_kernel completes the tree)
     size_t smem;
 };
 

@@ -61,11 +61,12 @@ struct DecodeParams {
     float* out;
     float* lse;
     // workspace
-    float* part_ml;      // [n_seqs][n_kv_heads][n_rb][split_stride][rows][2]
+    float* part_ml;      // [n_seqs][n_kv_heads][n_rb][split_stride][2][rows]: m then l per CTA
     float* part_o;       // [n_seqs][n_kv_heads][n_rb][split_stride][rows][D]
-    int split_stride;    // partial slots per unit (>= the splits of any unit)
+    int split_stride;    // partial slots per unit (>= the CTAs of any unit)
     int n_rb;            // row blocks per kv-head
-    int cpc;             // chunks per CTA
+    int cpc;             // chunks per CTA (a multiple of node_chunks)
+    int node_chunks;     // chunks per merge-tree leaf
     int stages;          // TMA ring depth in chunks
     unsigned* err;
     // How the launch sees each sequence (the cascade's two passes use these; a plain
@@ -90,6 +91,7 @@ __device__ __forceinline__ int seq_nq_of(const DecodeParams& p, int b) {
 // The small row classes (4 and 8 rows, mq_decode_small.cu).
 size_t small_smem_bytes(int head_dim, int rows, int stages);
 int small_ctas_per_sm(int head_dim, int rows);
+int small_leaf_kmax(int head_dim, int rows);
 cudaError_t small_prepare(int head_dim, int rows, size_t smem);
 cudaError_t small_launch(const DecodeParams& p, int head_dim, int rows, dim3 grid, size_t smem, cudaStream_t st);
 
@@ -101,7 +103,7 @@ cudaError_t launch_prefill(const DecodeParams& p, int max_tiles, cudaStream_t st
 size_t decode_smem_bytes(int head_dim, int rows, int stages);   // 0: does not fit the layout
 cudaError_t decode_prepare(int head_dim, int rows, size_t smem);  // raises the dynamic smem limit
 int decode_ctas_per_sm(int head_dim, int rows);                    // CTAs the kernel is built to co-host
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int max_splits, size_t smem,
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int max_splits, bool merge, size_t smem,
                           cudaStream_t st);
 
 // Fills n values of dtype with a deterministic pseudo-random pattern (uniform in

@@ -7,7 +7,7 @@ import shutil
 
 import bench
 
-FILES = ("mq_decode.cu", "mq_device.cuh", "mq_tc.cuh", "mq_kernels.h")
+FILES = ("mq_decode_small.cu", "mq_decode_common.cuh", "mq_decode.cu", "mq_device.cuh", "mq_tc.cuh", "mq_kernels.h")
 
 
 def _tree(tmp_path):
@@ -24,11 +24,12 @@ def test_hash_ignores_comments_and_blank_space(tmp_path, monkeypatch):
     root, d = _tree(tmp_path)
     monkeypatch.setattr(bench, "ROOT", str(root))
     h0 = bench.kernel_source_hash()
-    p = d / "mq_decode.cu"
+    p = d / "mq_decode_small.cu"
     src = p.read_text()
     p.write_text("// a new comment line\n/* and a block\n comment */\n" + src.replace("\n", "\n\n", 5))
     assert bench.kernel_source_hash() == h0
-    p.write_text(src.replace("constexpr float kLazy = 4.0f;", "constexpr float kLazy = 5.0f;"))
+    assert "static constexpr int NWB = 2;" in src
+    p.write_text(src.replace("static constexpr int NWB = 2;", "static constexpr int NWB = 3;"))
     assert bench.kernel_source_hash() != h0
 
 

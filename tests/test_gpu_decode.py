@@ -169,6 +169,33 @@ def test_ring_depth_bit_identical(name):
             assert torch.equal(base[0], ref[0]) and torch.equal(base[1], ref[1])
 
 
+@pytest.mark.parametrize("shape", ["long", "tiny", "mixed", "gqa8", "ragged"])
+def test_split_count_bit_identical_for_decode_classes(shape):
+    """One query token per sequence at GQA <= 8 (row classes of 4 and 8 rows): every split
+    count and ring depth gives the same output bytes, because the merge-tree leaves are
+    fixed runs of chunks that do not depend on the split count."""
+    if shape == "long":
+        w = wl.long_decode(L=20000)
+    elif shape == "tiny":
+        w = wl.tiny(L=4096)
+    elif shape == "mixed":
+        w = wl.reduced("mixed")
+    elif shape == "gqa8":
+        w = wl.Workload("gqa8", 32, 4, 128, [33000, 5000], [1, 1], [1, 1])
+    else:
+        w = wl.Workload("ragged", 8, 2, 256, [70000, 129, 16385], [1, 1, 1], [1, 1, 1])
+    case = GpuCase(w)
+    ref = [t.clone() for t in case.decode()]
+    assert case.status() == mq.MQ_OK
+    for sps in SPLITS_PER_SM:
+        for r in RING_STAGES:
+            mq.mq_set_decode_config(case.cache.handle, 0, r, sps)
+            out, lse = case.decode()
+            assert case.status() == mq.MQ_OK
+            assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1]), (sps, r)
+    _check(case)
+
+
 @pytest.mark.parametrize("sps", SPLITS_PER_SM)
 def test_every_split_count_within_tolerance(sps):
     """Every split count the tuner may try stays within the tolerance of the oracle."""

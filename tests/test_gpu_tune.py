@@ -44,8 +44,12 @@ def test_tune_within_budget_and_output_unchanged(tmp_path):
     assert abs(spec["weight_per_s"] - 1e6 * (1 / terms["draft_64k"] + 1 / terms["verify8_64k"])) \
         <= 1e-3 * spec["weight_per_s"]
     assert abs(probes["decode_64k"]["weight_per_s"] - 1e6 / terms["decode_64k"]) <= 1e-3 * 1e6 / terms["decode_64k"]
-    # ring depth never changes the bytes, so those candidates are all admitted
+    # ring depth never changes the bytes, and for the decode class (one query token at
+    # GQA <= 8) neither does the split count: those candidates are all admitted
     assert all(c["bit_identical"] for c in d["candidates"] if c["measured"] and c["splits_per_sm"] == 1)
+    decode_class = [c for c in d["candidates"] if c["measured"] and c["rows_class"] == 0]
+    assert any(c["splits_per_sm"] != 1 for c in decode_class)
+    assert all(c["bit_identical"] and c["admitted"] for c in decode_class)
     # the tuned configuration gives the same bytes as the defaults
     out, lse = case.decode()
     assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1])
