@@ -419,22 +419,32 @@ mq_status mq_draft_ngram(const int32_t* tokens, int32_t max_len, const int32_t* 
  * Launch configuration and tuning
  *
  * The decode kernel cuts every sequence into chunks of 128 tokens; one CTA takes a
- * contiguous range of chunks of one (sequence, kv-head, row block), accumulates
- * them in token order, and the CTA partials are combined by one fixed binary
- * tree over the split index.
+ * contiguous range of chunks of one (sequence, kv-head, row block) and the CTA
+ * partials are combined by one fixed binary tree over the split index.
  *   ring_stages    2 .. 8: chunks (8 pages each) a CTA keeps in flight, cut
  *                  to what fits in shared memory; never changes the output
  *   splits_per_sm  1, 2 or 4: the split count along the sequence is chosen so
- *                  that about splits_per_sm x (number of SMs) CTAs run; it sets
- *                  the chunk ranges and so may change the rounding of the output
- *                  (the tuner keeps only candidates whose output bytes equal the
- *                  current configuration's)
+ *                  that about splits_per_sm x (number of SMs) CTAs run.  Row
+ *                  blocks of up to 8 rows (one query token per sequence at GQA
+ *                  <= 8, head_dim 128; GQA <= 4 at head_dim 256) merge fixed runs
+ *                  of chunks over one fixed binary tree whose shape depends on the
+ *                  sequence length alone, a CTA taking an aligned power-of-two run
+ *                  of them: there the split count never changes the output.  The
+ *                  wider blocks (draft verification) accumulate each CTA's range in
+ *                  token order, so there it sets the rounding of the output.
+ *   softmax_warps  4 or 8: warps that turn one chunk's scores into weights; with
+ *                  8, a block's rows are split over two groups of four (each row's
+ *                  arithmetic is the same in either case, so this never changes
+ *                  the output).  32-row blocks always use 8 and 4-row blocks 4.
+ * The tuner keeps only candidates whose output bytes equal the current
+ * configuration's (or, on request, within the alpha rule; see mq_tune).
  * There is one configuration per row class (query rows per kv-head, padded):
  * rows_class 0 = up to 8 rows, 1 = up to 16, 2 = up to 32.
  * ------------------------------------------------------------------------- */
 typedef struct mq_decode_config {
     int32_t ring_stages;
     int32_t splits_per_sm;
+    int32_t softmax_warps;
 } mq_decode_config;
 
 mq_status mq_get_decode_config(const mq_cache* cache, int32_t rows_class, mq_decode_config* cfg);

@@ -29,10 +29,10 @@ class mq_cache_desc(ctypes.Structure):
 
 
 class mq_decode_config(ctypes.Structure):
-    _fields_ = [("ring_stages", ctypes.c_int32), ("splits_per_sm", ctypes.c_int32)]
+    _fields_ = [("ring_stages", ctypes.c_int32), ("splits_per_sm", ctypes.c_int32), ("softmax_warps", ctypes.c_int32)]
 
     def as_tuple(self):
-        return (self.ring_stages, self.splits_per_sm)
+        return (self.ring_stages, self.splits_per_sm, self.softmax_warps)
 
 
 class mq_tune_params(ctypes.Structure):
@@ -226,8 +226,12 @@ def mq_get_decode_config(cache: int, rows_class: int) -> tuple:
     return c.as_tuple()
 
 
-def mq_set_decode_config(cache: int, rows_class: int, ring_stages: int, splits_per_sm: int) -> None:
-    c = mq_decode_config(ring_stages, splits_per_sm)
+def mq_set_decode_config(cache: int, rows_class: int, ring_stages: int, splits_per_sm: int,
+                         softmax_warps: int | None = None) -> None:
+    """softmax_warps None keeps the class's current value."""
+    if softmax_warps is None:
+        softmax_warps = mq_get_decode_config(cache, rows_class)[2]
+    c = mq_decode_config(ring_stages, splits_per_sm, softmax_warps)
     _check(lib.mq_set_decode_config(cache, rows_class, ctypes.byref(c)), "mq_set_decode_config")
 
 
@@ -263,7 +267,7 @@ def mq_tune_store_get(path: str, identity: str):
 
 
 def mq_tune_store_put(path: str, identity: str, chosen, cost: float) -> None:
-    cfg = (mq_decode_config * 3)(*[mq_decode_config(r, s) for r, s in chosen])
+    cfg = (mq_decode_config * 3)(*[mq_decode_config(*c) for c in chosen])
     _check(lib.mq_tune_store_put(path.encode(), identity.encode(), cfg, float(cost)), "mq_tune_store_put")
 
 

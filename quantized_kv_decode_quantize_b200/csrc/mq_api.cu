@@ -34,16 +34,17 @@ int rows_class_for(int head_dim, int rows_total) {
 
 mq_decode_config default_config(int head_dim, int cls) {
     (void)head_dim;
-    (void)cls;
     mq_decode_config c{};
     c.ring_stages = 8;   // the planner shortens it to what fits in shared memory
     c.splits_per_sm = 1;
+    c.softmax_warps = cls == 2 ? 8 : 4;
     return c;
 }
 
 bool config_valid(const mq_decode_config& c) {
     return c.ring_stages >= 2 && c.ring_stages <= 8 &&
-           (c.splits_per_sm == 1 || c.splits_per_sm == 2 || c.splits_per_sm == 4);
+           (c.splits_per_sm == 1 || c.splits_per_sm == 2 || c.splits_per_sm == 4) &&
+           (c.softmax_warps == 4 || c.softmax_warps == 8);
 }
 
 DevGuard::DevGuard(int dev) {
@@ -74,6 +75,8 @@ static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int row
     pl.rows = (cls == 0 && rows_total <= 4) ? 4 : rows_class_rows(c->head_dim, pl.cls);
     pl.n_rb = (rows_total + pl.rows - 1) / pl.rows;
     const mq_decode_config cfg = c->cfg[pl.cls];
+    // softmax warp groups: 32-row blocks need two, 4-row blocks have one
+    pl.groups = pl.rows == 32 ? 2 : (pl.rows == 4 ? 1 : cfg.softmax_warps / 4);
     const long long max_chunks = std::max<long long>(1, (max_seq_len + kChunkTokens - 1) / kChunkTokens);
     const long long units = (long long)n_seqs * c->n_kv_heads * pl.n_rb;
     const int cps = decode_ctas_per_sm(c->head_dim, pl.rows);
@@ -105,10 +108,10 @@ static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int row
     const size_t smem_cap = cps == 1 ? (size_t)c->max_smem
                                      : std::min((size_t)c->max_smem, (size_t)c->smem_per_sm / cps - 1024);
     pl.stages = cfg.ring_stages;
-    pl.smem = decode_smem_bytes(c->head_dim, pl.rows, pl.stages);
+    pl.smem = decode_smem_bytes(c->head_dim, pl.rows, pl.groups, pl.stages);
     while ((pl.smem == 0 || pl.smem > smem_cap) && pl.stages > 2) {
         pl.stages--;
-        pl.smem = decode_smem_bytes(c->head_dim, pl.rows, pl.stages);
+        pl.smem = decode_smem_bytes(c->head_dim, pl.rows, pl.groups, pl.stages);
     }
     return pl;
 }
@@ -134,7 +137,7 @@ mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void
     if (pl.smem == 0 || pl.smem > (size_t)c->max_smem) return MQ_ERR_UNSUPPORTED;
     const size_t units = (size_t)n_seqs * c->n_kv_heads * pl.n_rb;
     if (partial_bytes(c, n_seqs, pl) > workspace_bytes) return MQ_ERR_WORKSPACE;
-    cudaError_t e = ensure_decode_smem(c->device, c->head_dim, pl.rows, pl.smem);
+    cudaError_t e = ensure_decode_smem(c->device, c->head_dim, pl.rows, pl.groups, pl.smem);
     if (e != cudaSuccess) return MQ_ERR_CUDA;
     DecodeParams p{};
     p.pool = static_cast<const uint8_t*>(c->pool);
@@ -171,18 +174,19 @@ mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void
     p.bt_col = view.bt_col;
     p.fixed_len = view.fixed_len;
     p.fixed_nq = view.fixed_nq;
-    e = launch_decode(p, c->head_dim, pl.rows, pl.max_splits, pl.merge, pl.smem, st);
+    e = launch_decode(p, c->head_dim, pl.rows, pl.groups, pl.max_splits, pl.merge, pl.smem, st);
     return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
 }
 
-cudaError_t ensure_decode_smem(int device, int head_dim, int rows, size_t smem) {
+cudaError_t ensure_decode_smem(int device, int head_dim, int rows, int groups, size_t smem) {
     // raised limit per (device, kernel variant); the attribute only grows
-    static size_t done[64][2][4] = {};
+    static size_t done[64][2][4][2] = {};
     const int di = device & 63, hi = head_dim == 128 ? 0 : 1;
     const int ri = rows == 4 ? 0 : (rows == 8 ? 1 : (rows == 16 ? 2 : 3));
-    if (done[di][hi][ri] >= smem) return cudaSuccess;
-    cudaError_t e = decode_prepare(head_dim, rows, smem);
-    if (e == cudaSuccess) done[di][hi][ri] = smem;
+    const int gi = groups == 2 ? 1 : 0;
+    if (done[di][hi][ri][gi] >= smem) return cudaSuccess;
+    cudaError_t e = decode_prepare(head_dim, rows, groups, smem);
+    if (e == cudaSuccess) done[di][hi][ri][gi] = smem;
     return e;
 }
 
@@ -335,7 +339,7 @@ size_t mq_decode_workspace_bytes(const mq_cache* c, int32_t n_seqs, int32_t n_q_
     size_t part = 0;
     for (int r = 2; r <= 8; r++)
         for (int t = 1; t <= 4; t *= 2) {
-            for (int k = 0; k < 3; k++) probe.cfg[k] = mq_decode_config{r, t};
+            for (int k = 0; k < 3; k++) probe.cfg[k] = mq_decode_config{r, t, k == 2 ? 8 : 4};
             const DecodePlan pl = plan_for_class(&probe, rows_class_for(c->head_dim, rows_total), n_seqs, rows_total,
                                                  max_seq_len);
             part = std::max(part, partial_bytes(c, n_seqs, pl));

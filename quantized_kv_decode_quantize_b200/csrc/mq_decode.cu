@@ -150,11 +150,15 @@ __global__ void __launch_bounds__(1024) merge_kernel(const DecodeParams p) {
     if (c4 == 0 && p.lse != nullptr) p.lse[orow] = __fmul_rn(__fadd_rn(m, log2f(l)), 0.69314718055994531f);
 }
 
-size_t decode_smem_bytes(int head_dim, int rows, int stages) { return small_smem_bytes(head_dim, rows, stages); }
+size_t decode_smem_bytes(int head_dim, int rows, int groups, int stages) {
+    return small_smem_bytes(head_dim, rows, groups, stages);
+}
 
 int decode_ctas_per_sm(int head_dim, int rows) { return small_ctas_per_sm(head_dim, rows); }
 
-cudaError_t decode_prepare(int head_dim, int rows, size_t smem) { return small_prepare(head_dim, rows, smem); }
+cudaError_t decode_prepare(int head_dim, int rows, int groups, size_t smem) {
+    return small_prepare(head_dim, rows, groups, smem);
+}
 
 // merge_kernel as a programmatic dependent launch on the same stream (after a decode
 // launch in which some unit's tree is not finished by one CTA).
@@ -174,11 +178,11 @@ static cudaError_t launch_merge(const DecodeParams& p, dim3 grid, int max_splits
 }
 
 // The decode kernel of the row class, then (when some unit needs it) the merge.
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int max_splits, bool merge, size_t smem,
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int groups, int max_splits, bool merge, size_t smem,
                           cudaStream_t st) {
     if (max_splits < 1 || max_splits > kMaxSplits || p.split_stride < max_splits) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)max_splits, (unsigned)(p.n_kv_heads * p.n_rb), (unsigned)p.n_seqs);
-    const cudaError_t e = small_launch(p, head_dim, rows, grid, smem, st);
+    const cudaError_t e = small_launch(p, head_dim, rows, groups, grid, smem, st);
     if (e != cudaSuccess || !merge) return e;
 #define MQ_MERGE(DD, RR) \
     if (head_dim == DD && rows == RR) return launch_merge<DD, RR>(p, grid, max_splits, st);

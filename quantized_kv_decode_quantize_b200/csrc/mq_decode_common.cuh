@@ -43,6 +43,9 @@ __device__ __forceinline__ float load_q(const DecodeParams& p, size_t i) {
     return ld_f32<__half>(p.q, i);
 }
 
+__device__ __forceinline__ void stsa64(uint32_t a, uint32_t x, uint32_t y) {
+    asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(a), "r"(x), "r"(y) : "memory");
+}
 __device__ __forceinline__ void stsa128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }

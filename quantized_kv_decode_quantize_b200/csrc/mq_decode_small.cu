@@ -35,7 +35,12 @@
 
 namespace mq {
 
-template <int D, int ROWS>
+// Levels of the merge-tree node a CTA builds from its leaves: the classes whose split count
+// is free (up to 8 rows, where tensor memory has room for the pending children; 64 leaves
+// per unit at most); 0 for the others, whose leaf is the CTA's range.
+constexpr int tree_levels(int D, int ROWS) { return (ROWS <= 8 && !(D == 256 && ROWS == 8)) ? 6 : 0; }
+
+template <int D, int ROWS, int NSG_>
 struct Sm {
     static constexpr int PB = page_bytes(D);
     static constexpr int REC = rec_bytes(D);
@@ -55,15 +60,12 @@ struct Sm {
     static constexpr int NWB = 2;                           // weight buffers (shared memory)
     static constexpr int NPB = 2;                           // value-MMA completion barriers
     static constexpr int NML = NWB + NOB;                   // slots of the merge factors
-    // levels of the merge-tree node a CTA builds from its leaves (the classes whose split
-    // count is free: up to 8 rows, where tensor memory has room for the pending children);
-    // 0 for the others, whose leaf is the CTA's range
-    static constexpr int KMAX = (ROWS <= 8 && !(D == 256 && ROWS == 8)) ? 6 : 0;
+    static constexpr int KMAX = tree_levels(D, ROWS);
     static constexpr int XS = 1 + KMAX;                     // factor pairs per row and chunk
-    // softmax warp groups: 32-row blocks split their rows over two groups of four warps
-    // (one warp per TMEM lane quadrant each); rows meet only through the chunk maximum of
-    // each row, which a group exchanges on its own named barrier
-    static constexpr int NSG = ROWS == 32 ? 2 : 1;
+    // softmax warp groups: a block's rows split over NSG groups of four warps (one warp
+    // per TMEM lane quadrant each); rows meet only through the chunk maximum of each row,
+    // which a group exchanges on its own named barrier
+    static constexpr int NSG = NSG_;
     static constexpr int RPG = ROWS / NSG;                  // rows per group
     static constexpr int THREADS = 224 + 128 * NSG;         // 0 TMA, 1 QK, 2 PV, 3-6 values, 7.. softmax
     static constexpr int T_S = 0;
@@ -74,6 +76,9 @@ struct Sm {
     static constexpr int WBYTES = kChunkTokens * NB * 2;    // one weight buffer
     static constexpr int LBO_W = NB / 8 * 128;              // its 8-token group stride
     static_assert(ROWS == 4 || ROWS == 8 || ROWS == 16 || ROWS == 32, "row class");
+    static_assert(NSG == 1 || NSG == 2, "softmax groups");
+    static_assert(RPG >= 4 && RPG <= 16, "rows per softmax group");
+    static_assert(CPS == 1 || NSG == 1, "two CTAs per SM with one softmax group");
     static_assert(T_END <= TCOLS, "tensor memory budget");
     static_assert(NPB >= NOB && NPB >= NVB && NPB >= NWB, "completion barriers");
 };
@@ -83,9 +88,9 @@ struct SmallSmem {
 };
 
 // NS = ring stages (chunks of 8 pages)
-template <int D, int ROWS>
+template <int D, int ROWS, int NSG>
 __host__ __device__ inline SmallSmem small_layout(int NS) {
-    using T = Sm<D, ROWS>;
+    using T = Sm<D, ROWS, NSG>;
     SmallSmem s{};
     auto al = [](size_t x, size_t a) { return (x + a - 1) / a * a; };
     size_t off = 0;
@@ -120,13 +125,14 @@ __host__ __device__ inline SmallSmem small_layout(int NS) {
     return s;
 }
 
-template <int D, int ROWS>
-__global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode_small_kernel(const DecodeParams p) {
-    using T = Sm<D, ROWS>;
+template <int D, int ROWS, int NSG>
+__global__ void __launch_bounds__(Sm<D, ROWS, NSG>::THREADS, Sm<D, ROWS, NSG>::CPS)
+    decode_small_kernel(const DecodeParams p) {
+    using T = Sm<D, ROWS, NSG>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NS = p.stages;
-    const SmallSmem S = small_layout<D, ROWS>(NS);
+    const SmallSmem S = small_layout<D, ROWS, NSG>(NS);
     const int b = blockIdx.z, hk = blockIdx.y / p.n_rb, rb = blockIdx.y % p.n_rb, sp = blockIdx.x;
     const unsigned FULL = 0xffffffffu;
 
@@ -641,18 +647,28 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
                 // ---- scores: the three limb accumulations of each row -> fp32 ----
                 uint32_t a[3 * RPG];
                 const uint32_t col = T::T_S + sb * T::NQ;
-                if constexpr (RPG == 16) {
-                    // limb l of row r sits in column l * ROWS + r
-                    uint32_t v0[16], v1[16], v2[16];
-                    tmem_ld16(tmem_at(tmem, 32 * q, col + r0g), v0);
-                    tmem_ld16(tmem_at(tmem, 32 * q, col + ROWS + r0g), v1);
-                    tmem_ld16(tmem_at(tmem, 32 * q, col + 2 * ROWS + r0g), v2);
+                if constexpr (RPG == 16 || T::NSG > 1) {
+                    // limb l of row r sits in column l * ROWS + r: the group's rows of each limb
+                    uint32_t v0[RPG], v1[RPG], v2[RPG];
+                    if constexpr (RPG == 16) {
+                        tmem_ld16(tmem_at(tmem, 32 * q, col + r0g), v0);
+                        tmem_ld16(tmem_at(tmem, 32 * q, col + ROWS + r0g), v1);
+                        tmem_ld16(tmem_at(tmem, 32 * q, col + 2 * ROWS + r0g), v2);
+                    } else if constexpr (RPG == 8) {
+                        tmem_ld8(tmem_at(tmem, 32 * q, col + r0g), v0);
+                        tmem_ld8(tmem_at(tmem, 32 * q, col + ROWS + r0g), v1);
+                        tmem_ld8(tmem_at(tmem, 32 * q, col + 2 * ROWS + r0g), v2);
+                    } else {
+                        tmem_ld4(tmem_at(tmem, 32 * q, col + r0g), v0);
+                        tmem_ld4(tmem_at(tmem, 32 * q, col + ROWS + r0g), v1);
+                        tmem_ld4(tmem_at(tmem, 32 * q, col + 2 * ROWS + r0g), v2);
+                    }
                     tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 16; k++) {
+                    for (int k = 0; k < RPG; k++) {
                         a[k] = v0[k];
-                        a[16 + k] = v1[k];
-                        a[32 + k] = v2[k];
+                        a[RPG + k] = v1[k];
+                        a[2 * RPG + k] = v2[k];
                     }
                 } else if constexpr (ROWS == 4) {
                     uint32_t v[16];
@@ -740,6 +756,10 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
                         for (int k = 0; k < RPG / 8; k++)
                             stsa128(wrow + 128u * (uint32_t)((g * ROWS + r0g) / 8 + k), wpair(4 * k, g),
                                     wpair(4 * k + 1, g), wpair(4 * k + 2, g), wpair(4 * k + 3, g));
+                } else if constexpr (T::NSG > 1) {
+                    // 8 rows in two groups of 4: this group's half of each 8-column group
+#pragma unroll
+                    for (int g = 0; g < T::G; g++) stsa64(wrow + 128u * g + 2u * r0g, wpair(0, g), wpair(1, g));
                 } else if constexpr (ROWS == 4) {
                     // column group cg holds groups 2cg and 2cg + 1, rows 0-3 each
 #pragma unroll
@@ -790,12 +810,16 @@ __global__ void __launch_bounds__(Sm<D, ROWS>::THREADS, Sm<D, ROWS>::CPS) decode
     }
 }
 
-// every row class: head_dim 128 with 4, 8, 16 or 32 rows; head_dim 256 with 4, 8 or 16
-#define MQ_SMALL_CLASSES(X) X(128, 4) X(128, 8) X(128, 16) X(128, 32) X(256, 4) X(256, 8) X(256, 16)
+// every (head_dim, rows, softmax groups) built: head_dim 128 with 4, 8, 16 or 32 rows and
+// head_dim 256 with 4, 8 or 16; one group of four softmax warps, or two for blocks of 8 and
+// more rows (two for 32)
+#define MQ_SMALL_CLASSES(X)                                                                         \
+    X(128, 4, 1) X(128, 8, 1) X(128, 8, 2) X(128, 16, 1) X(128, 16, 2) X(128, 32, 2) X(256, 4, 1) \
+    X(256, 8, 1) X(256, 8, 2) X(256, 16, 1) X(256, 16, 2)
 
-size_t small_smem_bytes(int head_dim, int rows, int stages) {
-#define MQ_SMEM(DD, RR) \
-    if (head_dim == DD && rows == RR) return small_layout<DD, RR>(stages).total;
+size_t small_smem_bytes(int head_dim, int rows, int groups, int stages) {
+#define MQ_SMEM(DD, RR, GG) \
+    if (head_dim == DD && rows == RR && groups == GG) return small_layout<DD, RR, GG>(stages).total;
     MQ_SMALL_CLASSES(MQ_SMEM)
 #undef MQ_SMEM
     return 0;
@@ -803,50 +827,46 @@ size_t small_smem_bytes(int head_dim, int rows, int stages) {
 
 int small_ctas_per_sm(int head_dim, int rows) { return (head_dim == 128 && rows == 4) ? 2 : 1; }
 
-int small_leaf_kmax(int head_dim, int rows) {
-#define MQ_KMAX(DD, RR) \
-    if (head_dim == DD && rows == RR) return Sm<DD, RR>::KMAX;
-    MQ_SMALL_CLASSES(MQ_KMAX)
-#undef MQ_KMAX
-    return 0;
-}
+int small_leaf_kmax(int head_dim, int rows) { return tree_levels(head_dim, rows); }
 
-template <int D, int ROWS>
+template <int D, int ROWS, int NSG>
 static cudaError_t small_set_smem(size_t smem) {
-    cudaError_t e =
-        cudaFuncSetAttribute(decode_small_kernel<D, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(decode_small_kernel<D, ROWS, NSG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     // all of the unified L1 / shared-memory array as shared memory, so that two CTAs fit
-    return cudaFuncSetAttribute(decode_small_kernel<D, ROWS>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return cudaFuncSetAttribute(decode_small_kernel<D, ROWS, NSG>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                100);
 }
 
-cudaError_t small_prepare(int head_dim, int rows, size_t smem) {
-#define MQ_PREP(DD, RR) \
-    if (head_dim == DD && rows == RR) return small_set_smem<DD, RR>(smem);
+cudaError_t small_prepare(int head_dim, int rows, int groups, size_t smem) {
+#define MQ_PREP(DD, RR, GG) \
+    if (head_dim == DD && rows == RR && groups == GG) return small_set_smem<DD, RR, GG>(smem);
     MQ_SMALL_CLASSES(MQ_PREP)
 #undef MQ_PREP
     return cudaErrorInvalidValue;
 }
 
-template <int D, int ROWS>
+template <int D, int ROWS, int NSG>
 static cudaError_t small_launch_t(const DecodeParams& p, dim3 grid, size_t smem, cudaStream_t st) {
     cudaLaunchAttribute pdl[1];
     pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t dc{};
     dc.gridDim = grid;
-    dc.blockDim = dim3((unsigned)Sm<D, ROWS>::THREADS);
+    dc.blockDim = dim3((unsigned)Sm<D, ROWS, NSG>::THREADS);
     dc.dynamicSmemBytes = smem;
     dc.stream = st;
     dc.attrs = pdl;
     dc.numAttrs = 1;
-    return cudaLaunchKernelEx(&dc, decode_small_kernel<D, ROWS>, p);
+    return cudaLaunchKernelEx(&dc, decode_small_kernel<D, ROWS, NSG>, p);
 }
 
 // The decode kernel of the row class, as a programmatic dependent launch.
-cudaError_t small_launch(const DecodeParams& p, int head_dim, int rows, dim3 grid, size_t smem, cudaStream_t st) {
-#define MQ_LAUNCH(DD, RR) \
-    if (head_dim == DD && rows == RR) return small_launch_t<DD, RR>(p, grid, smem, st);
+cudaError_t small_launch(const DecodeParams& p, int head_dim, int rows, int groups, dim3 grid, size_t smem,
+                         cudaStream_t st) {
+#define MQ_LAUNCH(DD, RR, GG) \
+    if (head_dim == DD && rows == RR && groups == GG) return small_launch_t<DD, RR, GG>(p, grid, smem, st);
     MQ_SMALL_CLASSES(MQ_LAUNCH)
 #undef MQ_LAUNCH
     return cudaErrorInvalidValue;

@@ -23,7 +23,7 @@ struct mq_cache {
 namespace mq {
 
 struct DecodePlan {
-    int cls, rows, n_rb, stages, cpc, max_splits;
+    int cls, rows, groups, n_rb, stages, cpc, max_splits;
     int node_chunks;               // merge-tree leaf (chunks)
     bool merge;                    // some unit has several CTAs (merge_kernel completes the tree)
     size_t smem;
@@ -44,7 +44,7 @@ bool config_valid(const mq_decode_config& c);
 DecodePlan plan_decode(const mq_cache* c, int n_seqs, int n_q_heads, int max_q, int max_seq_len);
 // Bytes of the CTA partials of one plan (the decode workspace).
 size_t partial_bytes(const mq_cache* c, int n_seqs, const DecodePlan& pl);
-cudaError_t ensure_decode_smem(int device, int head_dim, int rows, size_t smem);
+cudaError_t ensure_decode_smem(int device, int head_dim, int rows, int groups, size_t smem);
 // How one decode launch sees its sequences (see DecodeParams): the defaults are a plain
 // causal decode over seq_lens and n_q_per_seq.
 struct DecodeView {

@@ -89,21 +89,22 @@ __device__ __forceinline__ int seq_nq_of(const DecodeParams& p, int b) {
 #endif
 
 // The small row classes (4 and 8 rows, mq_decode_small.cu).
-size_t small_smem_bytes(int head_dim, int rows, int stages);
+size_t small_smem_bytes(int head_dim, int rows, int groups, int stages);
 int small_ctas_per_sm(int head_dim, int rows);
 int small_leaf_kmax(int head_dim, int rows);
-cudaError_t small_prepare(int head_dim, int rows, size_t smem);
-cudaError_t small_launch(const DecodeParams& p, int head_dim, int rows, dim3 grid, size_t smem, cudaStream_t st);
+cudaError_t small_prepare(int head_dim, int rows, int groups, size_t smem);
+cudaError_t small_launch(const DecodeParams& p, int head_dim, int rows, int groups, dim3 grid, size_t smem,
+                         cudaStream_t st);
 
 // Prefill attention (mq_prefill.cu): head_dim 128, tiles of 128 query rows.
 size_t prefill_smem_bytes();
 cudaError_t launch_prefill(const DecodeParams& p, int max_tiles, cudaStream_t st);
 
 // rows: 4, 8, 16 or 32 (padded query rows per kv-head handled by one CTA)
-size_t decode_smem_bytes(int head_dim, int rows, int stages);   // 0: does not fit the layout
-cudaError_t decode_prepare(int head_dim, int rows, size_t smem);  // raises the dynamic smem limit
+size_t decode_smem_bytes(int head_dim, int rows, int groups, int stages);   // 0: not built / does not fit
+cudaError_t decode_prepare(int head_dim, int rows, int groups, size_t smem);  // raises the dynamic smem limit
 int decode_ctas_per_sm(int head_dim, int rows);                    // CTAs the kernel is built to co-host
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int max_splits, bool merge, size_t smem,
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int groups, int max_splits, bool merge, size_t smem,
                           cudaStream_t st);
 
 // Fills n values of dtype with a deterministic pseudo-random pattern (uniform in

@@ -156,8 +156,11 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
                                  res->elapsed_s);
                     std::fprintf(f, "  \"chosen\": [");
                     for (int cls = 0; cls < 3; cls++)
-                        std::fprintf(f, "%s{\"rows_class\": %d, \"ring_stages\": %d, \"splits_per_sm\": %d}",
-                                     cls ? ", " : "", cls, got[cls].ring_stages, got[cls].splits_per_sm);
+                        std::fprintf(f,
+                                     "%s{\"rows_class\": %d, \"ring_stages\": %d, \"splits_per_sm\": %d, "
+                                     "\"softmax_warps\": %d}",
+                                     cls ? ", " : "", cls, got[cls].ring_stages, got[cls].splits_per_sm,
+                                     got[cls].softmax_warps);
                     std::fprintf(f, "],\n  \"n_tried\": 0\n}\n");
                     std::fclose(f);
                 }
@@ -414,21 +417,31 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         return MQ_TUNE_BUDGET_EXHAUSTED;
     }
 
-    // ---- candidates: structure (splits per SM) first, then ring depth ----
+    // ---- candidates: structure (splits per SM, softmax warps) first, then ring depth ----
     std::vector<Cand> cands;
     bool class_used[3] = {false, false, false};
-    for (auto& pr : probes) class_used[pr.cls] = true;
+    int class_rows[3] = {0, 0, 0};   // the row block the class's probes run
+    for (auto& pr : probes) {
+        class_used[pr.cls] = true;
+        class_rows[pr.cls] = plan_decode(&probe_cache, 1, Hq, pr.n_q, pr.seq_len).rows;
+    }
     for (int r : {8, 6, 4, 3, 2})
         for (int sps : {1, 2, 4})
-            for (int cls = 0; cls < 3; cls++) {
-                if (!class_used[cls]) continue;
-                Cand cd;
-                cd.cfg = mq_decode_config{r, sps};
-                cd.cls = cls;
-                const mq_decode_config& d = cache->cfg[cls];
-                if (cd.cfg.ring_stages == d.ring_stages && cd.cfg.splits_per_sm == d.splits_per_sm) continue;
-                cands.push_back(cd);
-            }
+            for (int w : {4, 8})
+                for (int cls = 0; cls < 3; cls++) {
+                    if (!class_used[cls]) continue;
+                    // 32-row blocks always run 8 softmax warps and 4-row blocks 4: the other
+                    // value would repeat a candidate
+                    if ((class_rows[cls] == 32 && w == 4) || (class_rows[cls] == 4 && w == 8)) continue;
+                    Cand cd;
+                    cd.cfg = mq_decode_config{r, sps, w};
+                    cd.cls = cls;
+                    const mq_decode_config& d = cache->cfg[cls];
+                    if (cd.cfg.ring_stages == d.ring_stages && cd.cfg.splits_per_sm == d.splits_per_sm &&
+                        cd.cfg.softmax_warps == d.softmax_warps)
+                        continue;
+                    cands.push_back(cd);
+                }
     bool exhausted = false;
     for (auto& cd : cands) {
         double est = 0;
@@ -570,9 +583,10 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
                 const Cand& cd = cands[i];
                 std::fprintf(f,
                              "    {\"rows_class\": %d, \"ring_stages\": %d, \"splits_per_sm\": %d, "
+                             "\"softmax_warps\": %d, "
                              "\"measured\": %s, \"valid\": %s, \"bit_identical\": %s, \"admitted\": %s, "
                              "\"times_us\": [%.3f, %.3f, %.3f], \"max_ratio\": ",
-                             cd.cls, cd.cfg.ring_stages, cd.cfg.splits_per_sm,
+                             cd.cls, cd.cfg.ring_stages, cd.cfg.splits_per_sm, cd.cfg.softmax_warps,
                              cd.measured ? "true" : "false", cd.valid ? "true" : "false",
                              cd.identical ? "true" : "false", (cd.measured && !cd.rejected) ? "true" : "false",
                              cd.t[0] * 1e6, cd.t[1] * 1e6, cd.t[2] * 1e6);
@@ -581,8 +595,11 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
             }
             std::fprintf(f, "  ],\n  \"chosen\": [");
             for (int cls = 0; cls < 3; cls++)
-                std::fprintf(f, "%s{\"rows_class\": %d, \"ring_stages\": %d, \"splits_per_sm\": %d}",
-                             cls ? ", " : "", cls, res->chosen[cls].ring_stages, res->chosen[cls].splits_per_sm);
+                std::fprintf(f,
+                             "%s{\"rows_class\": %d, \"ring_stages\": %d, \"splits_per_sm\": %d, "
+                             "\"softmax_warps\": %d}",
+                             cls ? ", " : "", cls, res->chosen[cls].ring_stages, res->chosen[cls].splits_per_sm,
+                             res->chosen[cls].softmax_warps);
             std::fprintf(f, "],\n  \"cost\": %.4f, \"n_tried\": %d, \"n_rejected\": %d, \"n_skipped\": %d\n}\n", res->cost,
                          res->n_tried, res->n_rejected, res->n_skipped);
             std::fclose(f);

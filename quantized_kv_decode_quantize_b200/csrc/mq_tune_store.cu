@@ -7,7 +7,8 @@
 // key=value fields (device, SM count, compute capability, driver, CUDA runtime,
 // library version and build, cache geometry, query heads, admission rule, the
 // default configurations), and the store is a text file with one line per identity:
-//     <identity> TAB <r0>:<s0> <r1>:<s1> <r2>:<s2> TAB <cost>
+//     <identity> TAB <r0>:<s0>:<w0> <r1>:<s1>:<w1> <r2>:<s2>:<w2> TAB <cost>
+// (ring stages, splits per SM and softmax warps of each row class).
 // Reading and writing the file is plain host code: no CUDA call is made there.
 #include <cctype>
 #include <cstdio>
@@ -29,7 +30,7 @@
 namespace mq {
 namespace {
 
-const char* const kStoreHeader = "# mq tuning store v1: identity<TAB>r0:s0 r1:s1 r2:s2<TAB>cost";
+const char* const kStoreHeader = "# mq tuning store v2: identity<TAB>r0:s0:w0 r1:s1:w1 r2:s2:w2<TAB>cost";
 
 bool identity_ok(const char* id) {
     if (id == nullptr || *id == '\0') return false;
@@ -48,16 +49,16 @@ std::string token(const char* s) {
     return o.empty() ? std::string("_") : o;
 }
 
-// Parses "<r0>:<s0> <r1>:<s1> <r2>:<s2>"; false unless all three are in range.
+// Parses "<r0>:<s0>:<w0> <r1>:<s1>:<w1> <r2>:<s2>:<w2>"; false unless all three are in range.
 bool parse_configs(const std::string& f, mq_decode_config out[3]) {
     std::istringstream in(f);
     for (int k = 0; k < 3; k++) {
         std::string item;
         if (!(in >> item)) return false;
-        int r = 0, s = 0;
+        int r = 0, s = 0, w = 0;
         char tail = 0;
-        if (std::sscanf(item.c_str(), "%d:%d%c", &r, &s, &tail) != 2) return false;
-        out[k] = mq_decode_config{r, s};
+        if (std::sscanf(item.c_str(), "%d:%d:%d%c", &r, &s, &w, &tail) != 3) return false;
+        out[k] = mq_decode_config{r, s, w};
         if (!config_valid(out[k])) return false;
     }
     std::string extra;
@@ -95,7 +96,8 @@ extern "C" mq_status mq_tune_identity(const mq_cache* c, const mq_tune_params* p
       << prop.minor << ";driver=" << drv << ";runtime=" << rt << ";lib=" << mq_version() << "+" << MQ_BUILD_ID
       << ";D=" << c->head_dim << ";Hkv=" << c->n_kv_heads << ";Hq=" << prm->n_q_heads << ";admit=" << admit
       << ";base=";
-    for (int k = 0; k < 3; k++) o << (k ? "," : "") << c->cfg[k].ring_stages << ":" << c->cfg[k].splits_per_sm;
+    for (int k = 0; k < 3; k++)
+        o << (k ? "," : "") << c->cfg[k].ring_stages << ":" << c->cfg[k].splits_per_sm << ":" << c->cfg[k].softmax_warps;
     const std::string s = o.str();
     if (s.size() + 1 > buf_len) return MQ_ERR_INVALID_ARG;
     std::memcpy(buf, s.c_str(), s.size() + 1);
@@ -136,8 +138,9 @@ extern "C" mq_status mq_tune_store_put(const char* path, const char* identity, c
         }
     }
     char entry[64];
-    std::snprintf(entry, sizeof entry, "%d:%d %d:%d %d:%d", chosen[0].ring_stages, chosen[0].splits_per_sm,
-                  chosen[1].ring_stages, chosen[1].splits_per_sm, chosen[2].ring_stages, chosen[2].splits_per_sm);
+    std::snprintf(entry, sizeof entry, "%d:%d:%d %d:%d:%d %d:%d:%d", chosen[0].ring_stages, chosen[0].splits_per_sm,
+                  chosen[0].softmax_warps, chosen[1].ring_stages, chosen[1].splits_per_sm, chosen[1].softmax_warps,
+                  chosen[2].ring_stages, chosen[2].splits_per_sm, chosen[2].softmax_warps);
     char cbuf[32];
     std::snprintf(cbuf, sizeof cbuf, "%.6f", cost);
     keep.push_back(std::string(identity) + "\t" + entry + "\t" + cbuf);

@@ -196,6 +196,27 @@ def test_split_count_bit_identical_for_decode_classes(shape):
     _check(case)
 
 
+@pytest.mark.parametrize("shape", ["gqa8", "drafts4", "d256_gqa8", "d256_drafts4"])
+def test_softmax_warps_bit_identical(shape):
+    """Splitting a row block over two groups of softmax warps never changes the output."""
+    w = {"gqa8": wl.Workload("gqa8", 32, 4, 128, [20000, 3000], [1, 1], [1, 1]),
+         "drafts4": wl.Workload("drafts4", 16, 4, 128, [9000, 700], [4, 3], [4, 3]),
+         "d256_gqa8": wl.Workload("d256_gqa8", 16, 2, 256, [12000], [1], [1]),
+         "d256_drafts4": wl.Workload("d256_drafts4", 16, 4, 256, [5000, 300], [4, 2], [4, 2])}[shape]
+    case = GpuCase(w)
+    cls = 0 if max(w.n_q) * w.n_q_heads // w.n_kv_heads <= 8 else 1
+    mq.mq_set_decode_config(case.cache.handle, cls, 4, 1, 4)
+    ref = [t.clone() for t in case.decode()]
+    assert case.status() == mq.MQ_OK
+    for r, sps in ((4, 1), (3, 2)):
+        mq.mq_set_decode_config(case.cache.handle, cls, r, sps, 8)
+        out, lse = case.decode()
+        assert case.status() == mq.MQ_OK
+        if sps == 1 or cls == 0 and shape != "d256_gqa8":
+            assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1]), (r, sps)
+    _check(case)
+
+
 @pytest.mark.parametrize("sps", SPLITS_PER_SM)
 def test_every_split_count_within_tolerance(sps):
     """Every split count the tuner may try stays within the tolerance of the oracle."""

@@ -18,7 +18,7 @@ import quantized_kv_decode_quantize_b200 as mq
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 ID_A = ("dev=NVIDIA_B200;sm=148;cc=10.0;driver=12090;runtime=12090;lib=10000+0123456789abcdef;"
-        "D=128;Hkv=8;Hq=32;admit=bit;base=8:1,8:1,8:1")
+        "D=128;Hkv=8;Hq=32;admit=bit;base=8:1:4,8:1:4,8:1:8")
 
 
 def _lines(path):
@@ -31,25 +31,25 @@ def test_missing_store_is_empty(tmp_path):
 
 def test_round_trip(tmp_path):
     p = str(tmp_path / "store.tsv")
-    mq.mq_tune_store_put(p, ID_A, [(6, 2), (8, 1), (4, 4)], 0.93)
-    assert mq.mq_tune_store_get(p, ID_A) == [(6, 2), (8, 1), (4, 4)]
+    mq.mq_tune_store_put(p, ID_A, [(6, 2, 4), (8, 1, 8), (4, 4, 8)], 0.93)
+    assert mq.mq_tune_store_get(p, ID_A) == [(6, 2, 4), (8, 1, 8), (4, 4, 8)]
     text = open(p).read()
-    assert text.startswith("# mq tuning store v1")
-    assert _lines(p) == [ID_A + "\t6:2 8:1 4:4\t0.930000"]
+    assert text.startswith("# mq tuning store v2")
+    assert _lines(p) == [ID_A + "\t6:2:4 8:1:8 4:4:8\t0.930000"]
 
 
 def test_put_replaces_the_identity_and_keeps_the_rest(tmp_path):
     p = str(tmp_path / "store.tsv")
     other = ID_A.replace("Hq=32", "Hq=64")
-    mq.mq_tune_store_put(p, ID_A, [(8, 1)] * 3, 1.0)
-    mq.mq_tune_store_put(p, other, [(2, 4)] * 3, 0.5)
-    mq.mq_tune_store_put(p, ID_A, [(3, 2)] * 3, 0.8)
+    mq.mq_tune_store_put(p, ID_A, [(8, 1, 4)] * 3, 1.0)
+    mq.mq_tune_store_put(p, other, [(2, 4, 8)] * 3, 0.5)
+    mq.mq_tune_store_put(p, ID_A, [(3, 2, 4)] * 3, 0.8)
     lines = _lines(p)
     assert len(lines) == 2
-    assert mq.mq_tune_store_get(p, ID_A) == [(3, 2)] * 3
-    assert mq.mq_tune_store_get(p, other) == [(2, 4)] * 3
+    assert mq.mq_tune_store_get(p, ID_A) == [(3, 2, 4)] * 3
+    assert mq.mq_tune_store_get(p, other) == [(2, 4, 8)] * 3
     # one header line, however many rewrites
-    assert sum(l.startswith("# mq tuning store v1") for l in open(p).read().splitlines()) == 1
+    assert sum(l.startswith("# mq tuning store v2") for l in open(p).read().splitlines()) == 1
 
 
 @pytest.mark.parametrize("field,new", [
@@ -58,11 +58,12 @@ def test_put_replaces_the_identity_and_keeps_the_rest(tmp_path):
     ("lib=10000+0123456789abcdef", "lib=10000+fedcba9876543210"),   # a rebuilt library
     ("dev=NVIDIA_B200", "dev=NVIDIA_H100"),
     ("admit=bit", "admit=alpha8"),
-    ("base=8:1,8:1,8:1", "base=4:1,8:1,8:1"),
+    ("base=8:1:4,8:1:4,8:1:8", "base=4:1:4,8:1:4,8:1:8"),
+    ("base=8:1:4,8:1:4,8:1:8", "base=8:1:8,8:1:4,8:1:8"),
 ])
 def test_changed_identity_finds_nothing(tmp_path, field, new):
     p = str(tmp_path / "store.tsv")
-    mq.mq_tune_store_put(p, ID_A, [(6, 2)] * 3, 0.9)
+    mq.mq_tune_store_put(p, ID_A, [(6, 2, 4)] * 3, 0.9)
     assert field in ID_A
     assert mq.mq_tune_store_get(p, ID_A.replace(field, new)) is None
     # a prefix of a stored identity is a different identity
@@ -73,31 +74,33 @@ def test_malformed_or_out_of_range_lines_are_absent(tmp_path):
     p = str(tmp_path / "store.tsv")
     with open(p, "w") as f:
         f.write("# some header\n")
-        f.write(ID_A + "\t9:1 8:1 8:1\t1.0\n")        # ring_stages 9 is out of range
-        f.write(ID_A.replace("Hq=32", "Hq=8") + "\t8:3 8:1 8:1\t1.0\n")   # splits 3 not allowed
-        f.write(ID_A.replace("Hq=32", "Hq=16") + "\t8:1 8:1\t1.0\n")      # two configs only
-        f.write(ID_A.replace("Hq=32", "Hq=24") + "\t8:1 8:1 8:1 8:1\t1.0\n")
+        f.write(ID_A + "\t9:1:4 8:1:4 8:1:8\t1.0\n")        # ring_stages 9 is out of range
+        f.write(ID_A.replace("Hq=32", "Hq=8") + "\t8:3:4 8:1:4 8:1:8\t1.0\n")   # splits 3 not allowed
+        f.write(ID_A.replace("Hq=32", "Hq=16") + "\t8:1:4 8:1:4\t1.0\n")        # two configs only
+        f.write(ID_A.replace("Hq=32", "Hq=24") + "\t8:1:4 8:1:4 8:1:8 8:1:4\t1.0\n")
+        f.write(ID_A.replace("Hq=32", "Hq=40") + "\t8:1:6 8:1:4 8:1:8\t1.0\n")  # 6 softmax warps
+        f.write(ID_A.replace("Hq=32", "Hq=48") + "\t8:1 8:1 8:1\t1.0\n")        # the two-field format
         f.write("garbage line without tabs\n")
-    for hq in ("Hq=32", "Hq=8", "Hq=16", "Hq=24"):
+    for hq in ("Hq=32", "Hq=8", "Hq=16", "Hq=24", "Hq=40", "Hq=48"):
         assert mq.mq_tune_store_get(p, ID_A.replace("Hq=32", hq)) is None
     # put keeps foreign lines and replaces only its own identity
-    mq.mq_tune_store_put(p, ID_A, [(2, 1), (2, 2), (2, 4)], 0.7)
-    assert mq.mq_tune_store_get(p, ID_A) == [(2, 1), (2, 2), (2, 4)]
+    mq.mq_tune_store_put(p, ID_A, [(2, 1, 4), (2, 2, 8), (2, 4, 8)], 0.7)
+    assert mq.mq_tune_store_get(p, ID_A) == [(2, 1, 4), (2, 2, 8), (2, 4, 8)]
     text = open(p).read()
     assert "garbage line without tabs" in text and "# some header" in text
-    assert "9:1 8:1 8:1" not in text
+    assert "9:1:4 8:1:4 8:1:8" not in text
 
 
 def test_invalid_arguments(tmp_path):
     p = str(tmp_path / "store.tsv")
     for bad in ("a\tb", "a\nb", ""):
         with pytest.raises(mq.MQError) as e:
-            mq.mq_tune_store_put(p, bad, [(8, 1)] * 3, 1.0)
+            mq.mq_tune_store_put(p, bad, [(8, 1, 4)] * 3, 1.0)
         assert e.value.status == mq.MQ_ERR_INVALID_ARG
         with pytest.raises(mq.MQError):
             mq.mq_tune_store_get(p, bad)
     with pytest.raises(mq.MQError) as e:
-        mq.mq_tune_store_put(p, ID_A, [(8, 1), (8, 1), (1, 1)], 1.0)   # 1 stage is below the range
+        mq.mq_tune_store_put(p, ID_A, [(8, 1, 4), (8, 1, 4), (1, 1, 8)], 1.0)   # 1 stage is below the range
     assert e.value.status == mq.MQ_ERR_INVALID_ARG
     assert not os.path.exists(p)
 
@@ -105,14 +108,14 @@ def test_invalid_arguments(tmp_path):
 def test_unwritable_store_is_an_io_error(tmp_path):
     p = str(tmp_path / "no_such_dir" / "store.tsv")
     with pytest.raises(mq.MQError) as e:
-        mq.mq_tune_store_put(p, ID_A, [(8, 1)] * 3, 1.0)
+        mq.mq_tune_store_put(p, ID_A, [(8, 1, 4)] * 3, 1.0)
     assert e.value.status == mq.MQ_ERR_IO
 
 
 def test_rewrite_leaves_no_temporary_files(tmp_path):
     p = str(tmp_path / "store.tsv")
     for i in range(5):
-        mq.mq_tune_store_put(p, ID_A.replace("Hq=32", f"Hq={8 * (i + 1)}"), [(8, 1)] * 3, 1.0)
+        mq.mq_tune_store_put(p, ID_A.replace("Hq=32", f"Hq={8 * (i + 1)}"), [(8, 1, 4)] * 3, 1.0)
     assert sorted(os.listdir(tmp_path)) == ["store.tsv"]
     assert len(_lines(p)) == 5
 
