@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--tune", type=float, default=0.0, help="run mq_tune with this budget (s) first")
+    ap.add_argument("--decode-config", default="",
+                    help="ring_stages,splits_per_sm,softmax_warps for every row class (before --tune)")
     ap.add_argument("--cascade", action="store_true",
                     help="decode with mq_decode_attn_cascade over the workload's shared prefix")
     return ap.parse_args()
@@ -527,6 +529,10 @@ def run_mq(args, rank, world, local):
     torch.cuda.synchronize(dev)
     assert mq.mq_device_status(cache.handle) == mq.MQ_OK
 
+    if args.decode_config:
+        r_, s_, w_ = (int(x) for x in args.decode_config.split(","))
+        for k in range(3):
+            mq.mq_set_decode_config(cache.handle, k, r_, s_, 8 if k == 2 else w_)
     if args.tune > 0:
         mq.mq_tune(cache.handle, args.tune, w.n_q_heads)
 
@@ -703,7 +709,9 @@ def run_mq(args, rank, world, local):
                "d2h_bytes_per_step": d2h, "steps": K2, "ms_per_step": e_dt / K2 * 1e3}
 
     if rank == 0:
-        cfg = mq.mq_get_decode_config(cache.handle, 0)
+        rows_total = w.n_q_heads // w.n_kv_heads * w.max_q
+        cls = 0 if rows_total <= 8 else (1 if rows_total <= 16 or w.head_dim == 256 else 2)
+        cfg = mq.mq_get_decode_config(cache.handle, cls)
         clocks = sampler.summary()
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,

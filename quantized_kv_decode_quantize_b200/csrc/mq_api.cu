@@ -290,7 +290,7 @@ mq_status mq_kv_append(mq_cache* c, const void* k, const void* v, mq_dtype dtype
     p.block_table = block_table;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.err = c->err_word;
-    return launch_append(p, c->head_dim, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MQ_OK
+    return launch_append(p, c->head_dim, c->n_sm, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MQ_OK
                                                                                                : MQ_ERR_CUDA;
 }
 

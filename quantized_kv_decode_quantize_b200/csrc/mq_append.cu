@@ -9,16 +9,18 @@
 // zero scale gives code 0.
 //
 // Work split: one warp per (8-position record, kv-head) that a sequence's new tokens
-// touch; the grid is (x, sequence, kv-head) and the warps of a (sequence, kv-head)
-// stride over its records.  Per token the warp quantizes as follows: each lane reads
-// D/32 consecutive channels with one vector load, the absmax reductions are warp
-// shuffles (exact: max is order-independent), each lane stores its K codes with one
-// 4- or 8-byte store.  A V word of the page holds one channel's codes for the 8
+// touch; the grid is (x, sequence, kv-head), sized from the device's SM count, and the
+// warps of a (sequence, kv-head) stride over its records.  A token's head vector is read
+// with 16-byte loads, one per lane (two per lane for fp32 at head_dim 256): LPT = min(32,
+// D x element size / 16) lanes per token, so at head_dim 128 with 2-byte inputs a warp
+// quantizes two tokens at once, one per half-warp.  The absmax reductions are shuffles
+// within a token's lanes (exact: max is order-independent); each lane stores its K codes
+// with one 4- or 8-byte store.  A V word of the page holds one channel's codes for the 8
 // tokens of a record (see mq_device.cuh): when the append covers the whole record, the
 // warp assembles every word in registers and writes it with a plain store; otherwise
-// (the ragged ends of an append, single-token appends) each nibble is replaced with
-// two atomic bit operations (clear, then set), since another launch may have written
-// the record's other tokens.
+// (the ragged ends of an append, single-token appends) each nibble is replaced with two
+// atomic bit operations (clear, then set), since another launch may have written the
+// record's other tokens.
 
 #include <algorithm>
 
@@ -68,10 +70,19 @@ __device__ __forceinline__ int quant_code(float x, float s, float lo, float hi) 
     return static_cast<int>(r);
 }
 
-// One token's codes, quantized by a whole warp (lane: channels CPL * lane ..).
-template <int D>
+// Lanes per token: 16 bytes of the token's head vector per lane, at most a warp.
+template <int D, typename T>
+struct Lanes {
+    static constexpr int LPT = (D * (int)sizeof(T) / 16) < 32 ? D * (int)sizeof(T) / 16 : 32;
+    static constexpr int TPW = 32 / LPT;   // tokens per warp
+    static constexpr int CPL = D / LPT;    // channels per lane
+    static constexpr int LPG = 32 / CPL;   // lanes per 32-channel V group
+    static_assert(LPT == 16 || LPT == 32, "lanes per token");
+};
+
+// One token's codes, quantized by its LPT lanes (lane l: channels CPL * l ..).
+template <int CPL>
 struct TokenCodes {
-    static constexpr int CPL = D / 32;
     uint32_t kb[CPL / 4];   // this lane's K codes, 4 per word
     __half sk16;            // K scale (every lane)
     uint32_t vn[CPL];       // this lane's V codes as 4-bit two's complement
@@ -79,19 +90,20 @@ struct TokenCodes {
 };
 
 template <int D, typename T>
-__device__ __forceinline__ void quantize_token(const AppendParams& p, long long tok, int h, int lane,
-                                               TokenCodes<D>& out) {
-    constexpr int CPL = D / 32;          // channels per lane
-    constexpr int LPG = 32 / CPL;        // lanes per 32-channel V group
-    const size_t vec = ((size_t)tok * p.n_kv_heads + h) * D + (size_t)lane * CPL;
+__device__ __forceinline__ void quantize_token(const AppendParams& p, long long tok, int h, int l,
+                                               TokenCodes<Lanes<D, T>::CPL>& out) {
+    using LN = Lanes<D, T>;
+    constexpr int CPL = LN::CPL, LPG = LN::LPG;
+    const size_t vec = ((size_t)tok * p.n_kv_heads + h) * D + (size_t)l * CPL;
     float xk[CPL], xv[CPL];
     load_vec<T, CPL>(reinterpret_cast<const T*>(p.k) + vec, xk);
     load_vec<T, CPL>(reinterpret_cast<const T*>(p.v) + vec, xv);
-    // ---- K: one scale over all D channels ----
+    // ---- K: one scale over all D channels (the token's LPT lanes) ----
     float a = 0.0f;
 #pragma unroll
     for (int i = 0; i < CPL; i++) a = fmaxf(a, fabsf(xk[i]));
-    a = warp_max(a);
+#pragma unroll
+    for (int o = LN::LPT / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     out.sk16 = __float2half_rn(__fdiv_rn(a, 127.0f));
     const float sk = __half2float(out.sk16);
 #pragma unroll
@@ -114,25 +126,28 @@ __device__ __forceinline__ void quantize_token(const AppendParams& p, long long 
     for (int i = 0; i < CPL; i++) out.vn[i] = (uint32_t)quant_code(xv[i], sv, -8.0f, 7.0f) & 0xFu;
 }
 
-// K codes, K scale and V scale of one token at slot tau of a page.
-template <int D>
-__device__ __forceinline__ void store_token_kscales(uint8_t* page, int tau, int lane, const TokenCodes<D>& tc) {
-    constexpr int CPL = D / 32, LPG = 32 / CPL;
-    const int c0 = lane * CPL;
+// K codes, K scale and V scale of one token at slot tau of a page (lane l of the token).
+template <int D, int CPL>
+__device__ __forceinline__ void store_token_kscales(uint8_t* page, int tau, int l, const TokenCodes<CPL>& tc) {
+    constexpr int LPG = 32 / CPL;
+    const int c0 = l * CPL;
     uint8_t* kdst = page + k_code_byte(D, tau, c0);
+    static_assert(CPL == 4 || CPL == 8, "channels per lane");
     if constexpr (CPL == 4) {
         *reinterpret_cast<uint32_t*>(kdst) = tc.kb[0];
     } else {
-        *reinterpret_cast<uint2*>(kdst) = make_uint2(tc.kb[0], tc.kb[1]);
+        *reinterpret_cast<uint2*>(kdst) = make_uint2(tc.kb[0], tc.kb[1]);   // within one 16-channel group
     }
-    if (lane == 0) *reinterpret_cast<__half*>(page + k_scale_byte(D, tau)) = tc.sk16;
-    if (lane % LPG == 0) *reinterpret_cast<__half*>(page + v_scale_byte(D, tau, c0 / 32)) = tc.sv16;
+    if (l == 0) *reinterpret_cast<__half*>(page + k_scale_byte(D, tau)) = tc.sk16;
+    if (l % LPG == 0) *reinterpret_cast<__half*>(page + v_scale_byte(D, tau, c0 / 32)) = tc.sv16;
 }
 
 template <int D, typename T>
 __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
-    constexpr int CPL = D / 32;
+    using LN = Lanes<D, T>;
+    constexpr int CPL = LN::CPL, TPW = LN::TPW;
     const int lane = threadIdx.x & 31;
+    const int sub = lane / LN::LPT, l = lane % LN::LPT;   // this lane's token of the warp's TPW, its lane there
     // a decode launched after this append may start its set-up now; it waits for this
     // grid (griddepcontrol.wait) before it reads any page
     if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -163,30 +178,44 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
         uint8_t* page = p.pool + ((long long)blk * p.n_kv_heads + h) * page_bytes(D);
         const int tau0 = (int)((8 * r) % kPageTokens);   // 0 or 8: the record within the page
         const long long p0 = 8 * r > start ? 8 * r : start, p1 = 8 * r + 8 < end ? 8 * r + 8 : end;
-        const int c0 = lane * CPL;
+        const int c0 = l * CPL;
         if (p1 - p0 == 8) {
-            // the whole record: V words assembled in registers, plain stores
+            // the whole record: V words assembled in registers (the TPW tokens of each step
+            // in separate lanes, combined below), plain stores
             uint32_t vw[CPL];
 #pragma unroll
             for (int i = 0; i < CPL; i++) vw[i] = 0u;
 #pragma unroll 2
-            for (int tt = 0; tt < 8; tt++) {
-                TokenCodes<D> tc;
-                quantize_token<D, T>(p, tok0 + (8 * r + tt - start), h, lane, tc);
-                store_token_kscales<D>(page, tau0 + tt, lane, tc);
+            for (int t2 = 0; t2 < 8; t2 += TPW) {
+                const int tt = t2 + sub;
+                TokenCodes<CPL> tc;
+                quantize_token<D, T>(p, tok0 + (8 * r + tt - start), h, l, tc);
+                store_token_kscales<D, CPL>(page, tau0 + tt, l, tc);
                 const int bit = v_nibble_bit(tt);
 #pragma unroll
                 for (int i = 0; i < CPL; i++) vw[i] |= tc.vn[i] << bit;
             }
+            if constexpr (TPW == 2) {
 #pragma unroll
-            for (int i = 0; i < CPL; i++) *reinterpret_cast<uint32_t*>(page + v_word_byte(D, tau0, c0 + i)) = vw[i];
+                for (int i = 0; i < CPL; i++) vw[i] |= __shfl_xor_sync(0xffffffffu, vw[i], 16);
+            }
+            if (sub == 0) {
+#pragma unroll
+                for (int i = 0; i < CPL; i++)
+                    *reinterpret_cast<uint32_t*>(page + v_word_byte(D, tau0, c0 + i)) = vw[i];
+            }
         } else {
-            // part of the record: each nibble replaced atomically
-            for (long long pos = p0; pos < p1; pos++) {
+            // part of the record: each nibble replaced atomically (TPW positions at a time)
+            for (long long q0 = p0; q0 < p1; q0 += TPW) {
+                const long long pos = q0 + sub;
+                const bool here = pos < p1;
+                TokenCodes<CPL> tc;
+                // lanes past the record's end quantize the record's first position again
+                // (their shuffles must run) and store nothing
+                quantize_token<D, T>(p, tok0 + ((here ? pos : p0) - start), h, l, tc);
+                if (!here) continue;
                 const int tau = (int)(pos % kPageTokens);
-                TokenCodes<D> tc;
-                quantize_token<D, T>(p, tok0 + (pos - start), h, lane, tc);
-                store_token_kscales<D>(page, tau, lane, tc);
+                store_token_kscales<D, CPL>(page, tau, l, tc);
                 const int bit = v_nibble_bit(tau);
 #pragma unroll
                 for (int i = 0; i < CPL; i++) {
@@ -200,13 +229,13 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
 }
 
 template <int D>
-static cudaError_t launch_append_d(const AppendParams& p, cudaStream_t st) {
+static cudaError_t launch_append_d(const AppendParams& p, int n_sm, cudaStream_t st) {
     if (p.n_seqs > 65535 || p.n_kv_heads > 65535) return cudaErrorInvalidConfiguration;
     const int wpb = 8;
-    // records of one sequence: at most n_tokens / 8 + 2; about 8 warps per SM in all
+    // records of one sequence: at most n_tokens / 8 + 2; about 8 CTAs per SM in all
     const long long per_seq = ((long long)p.n_tokens / 8 + 2 + wpb - 1) / wpb;
     const long long units = (long long)p.n_seqs * p.n_kv_heads;
-    const long long fill = (148LL * 8 + units - 1) / units;
+    const long long fill = ((long long)n_sm * 8 + units - 1) / units;
     const long long gx = std::max<long long>(1, std::min(per_seq, fill));
     const dim3 grid((unsigned)gx, (unsigned)p.n_seqs, (unsigned)p.n_kv_heads);
     switch (p.dtype) {
@@ -217,8 +246,8 @@ static cudaError_t launch_append_d(const AppendParams& p, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_append(const AppendParams& p, int head_dim, cudaStream_t st) {
-    return head_dim == 128 ? launch_append_d<128>(p, st) : launch_append_d<256>(p, st);
+cudaError_t launch_append(const AppendParams& p, int head_dim, int n_sm, cudaStream_t st) {
+    return head_dim == 128 ? launch_append_d<128>(p, n_sm, st) : launch_append_d<256>(p, n_sm, st);
 }
 
 }  // namespace mq

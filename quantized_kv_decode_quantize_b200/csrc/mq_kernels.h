@@ -21,7 +21,7 @@ struct AppendParams {
     unsigned* err;
 };
 
-cudaError_t launch_append(const AppendParams& p, int head_dim, cudaStream_t st);
+cudaError_t launch_append(const AppendParams& p, int head_dim, int n_sm, cudaStream_t st);
 
 struct ExportParams {
     const uint8_t* pool;

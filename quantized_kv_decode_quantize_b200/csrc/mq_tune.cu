@@ -260,7 +260,7 @@ extern "C" mq_status mq_tune(mq_cache* cache, const mq_tune_params* prm, mq_tune
         ap.block_table = B.bt;
         ap.max_blocks_per_seq = blocks_per_copy;
         ap.err = cache->err_word;
-        if (!ck(launch_append(ap, D, B.st))) return MQ_ERR_CUDA;
+        if (!ck(launch_append(ap, D, cache->n_sm, B.st))) return MQ_ERR_CUDA;
         for (int i = 1; i < n_copies; i++)
             if (!ck(cudaMemcpyAsync(static_cast<uint8_t*>(B.pool) + copy_bytes * i, B.pool, copy_bytes,
                                     cudaMemcpyDeviceToDevice, B.st)))
