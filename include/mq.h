@@ -530,9 +530,9 @@ mq_status mq_tune(mq_cache* cache, const mq_tune_params* params, mq_tune_result*
 mq_status mq_tune_identity(const mq_cache* cache, const mq_tune_params* params, char* buf, size_t buf_len);
 
 /* The tuning store: a text file, one choice per line,
- *     <identity> TAB <r0>:<s0> <r1>:<s1> <r2>:<s2> TAB <cost>
- * (ring_stages:splits_per_sm of rows_class 0, 1, 2), after a header line starting
- * with '#'.  Host-only file access; no GPU is needed.
+ *     <identity> TAB <r0>:<s0>:<w0> <r1>:<s1>:<w1> <r2>:<s2>:<w2> TAB <cost>
+ * (ring_stages:splits_per_sm:softmax_warps of rows_class 0, 1, 2), after a header
+ * line starting with '#'.  Host-only file access; no GPU is needed.
  * mq_tune_store_get: *found = 1 and chosen[0..2] set when a well-formed line with
  *   this identity exists (a line whose configurations are out of range counts as
  *   absent); *found = 0 otherwise, a missing or unreadable file included.

@@ -1,36 +1,41 @@
-// Split-K flash-decode for blocks of 4 or 8 query rows per kv-head (grouped-query decode:
-// GQA 4 with one query token is 4 rows), on the sm_100a tensor cores.
+// Split-K flash-decode over the K8/V4 paged cache, with draft verification, on the sm_100a
+// tensor cores: one warp-specialised kernel for every row class (4, 8, 16 or 32 query rows
+// per kv-head; grouped-query decode at GQA 4 with one query token is 4 rows).
 //
-// What it computes is mq_decode.cu's (the deep dive on magnitudedev/magnitude at
-// blog.123qwe.co.kr, section 5: the decode attention unit attention_decode_k8v4 over the
-// 8-bit-key / 4-bit-value cache): for query token j of sequence b and q-head h,
+// What it computes (the deep dive on magnitudedev/magnitude at blog.123qwe.co.kr, section
+// 5: the decode attention unit attention_decode_k8v4 over the 8-bit-key / 4-bit-value
+// cache, and the guarantee that verifying several draft tokens is one launch against the
+// cache): for query token j of sequence b (n_b query tokens, L_b cached tokens including
+// the drafts) and q-head h,
 //     z_t = scale * <q, s_k[t] * kcode_t>,  t = 0 .. L_b - n_b + j
 //     out = sum_t softmax(z)_t * (s_v[t, group] * vcode_t),  lse = log sum_t exp z_t
 //
-// How.  One CTA (11 warps; two CTAs per SM for 4 rows of head_dim 128) takes a contiguous range of
-// 128-token chunks of one (sequence, kv-head, row block).  Every chunk is a small
-// attention problem of its own, solved with the chunk's exact row maxima, and the
-// per-chunk results are merged by log-sum-exp in registers:
+// How.  One CTA (11 warps, 15 with two softmax groups; two CTAs per SM for 4 rows of
+// head_dim 128) takes a contiguous range of 128-token chunks of one (sequence, kv-head,
+// row block).  Every chunk is a small attention problem of its own, solved with the
+// chunk's exact row maxima, and the per-chunk results are merged by log-sum-exp:
 //  * warp 0 streams the chunk's 8 pages into a shared-memory ring, one 1-D bulk TMA copy
 //    per page (block-table lookup, L2 evict-first);
 //  * warp 1 issues the score MMAs (kind::i8, M = 128 tokens, q as three signed 8-bit
 //    limbs per row along N, exact int32 products in tensor memory);
-//  * warps 7-10 (one TMEM lane = one token) form z in fp32, take the chunk's row maxima
-//    (redux + one named barrier), and write p = 2^(z - max) <= 1 and the fp16 weights
-//    W_g = p * s_v[token, g] to shared memory; each thread keeps its token's share of
-//    l = sum_t p_t relative to the running row maxima, summed over the CTA at the end;
+//  * the softmax warps (one or two groups of four; one TMEM lane = one token) form z in
+//    fp32, take the chunk's row maxima (redux + one named barrier per group), and write
+//    p = 2^(z - max) <= 1, the warp's exact integer sums of p per row, and the fp16
+//    weights W_g = fp16(p) * s_v[token, g] to shared memory;
 //  * warp 2 issues the value MMAs (kind::f16, A = V^T in tensor memory, B = the weights,
 //    every group of 32 channels using its own columns) into a fresh accumulator per
-//    chunk (two alternate);
+//    chunk (two alternate), then keeps the row state, one lane per row: the chunk's
+//    maximum and l, the running (M, l), and every log-sum-exp factor the merges use;
 //  * warps 3-6 turn the chunk's int4 value codes into V^T in tensor memory as exact fp16
-//    values (one channel per lane), and then merge the previous chunk's accumulator into
-//    the CTA's running (max, sum, output) held in registers, lane = channel.
+//    values (one channel per lane), then merge the previous chunk's accumulator into the
+//    CTA's running output in registers (lane = channel) with warp 2's factors.
 // The weights never exceed the fp16 range (p <= 1 and s_v <= 65504), no accumulator is
 // ever rescaled in tensor memory, and the chunk steps of the softmax do not wait for one
-// another.  The CTA partials of a unit are combined by merge_kernel (mq_decode.cu) over a
-// fixed binary tree; a unit that is not split writes out and lse here.  The chunk ranges
-// depend only on the shape, the SM count and the configured splits per SM, so the result
-// is bit-identical for every ring depth.
+// another.  The chunks of a merge-tree leaf (node_chunks chunks) fold in order; for the
+// classes of up to 8 rows a CTA holds an aligned power-of-two run of leaves and combines
+// it into that node of a fixed binary tree (see tree_step; pending children in tensor
+// memory), otherwise its range is one leaf.  The CTA's partial goes to the workspace and
+// merge_kernel (mq_decode.cu) finishes the tree; a unit of one CTA writes out and lse here.
 #include "mq_decode_common.cuh"
 
 namespace mq {

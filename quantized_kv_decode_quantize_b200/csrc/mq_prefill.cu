@@ -1,6 +1,6 @@
 // Prefill (prompt) attention over the K8/V4 paged cache on the sm_100a tensor cores.
 //
-// What it computes is the decode attention of mq_decode.cu for many query tokens at
+// What it computes is the decode attention of mq_decode_small.cu for many query tokens at
 // once: for query token j of sequence b (n_b queries, L_b cached tokens including the
 // prompt's own, already appended) and q-head h,
 //     z_t = scale * <q, s_k[t] * kcode_t>,  t = 0 .. L_b - n_b + j
