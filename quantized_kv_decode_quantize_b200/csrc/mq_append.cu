@@ -163,8 +163,14 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     const long long r_lo = start >= 0 ? start / 8 : -((-start + 7) / 8);             // floor(start / 8)
     const long long r_hi = (end - 1) >= 0 ? (end - 1) / 8 : -((-(end - 1) + 7) / 8);
     const int wpb = blockDim.x / 32;
-    for (long long r = r_lo + (long long)blockIdx.x * wpb + (threadIdx.x >> 5); r <= r_hi;
-         r += (long long)gridDim.x * wpb) {
+    // work items: (record, slice); with several slices a record's 8 positions are shared by
+    // that many warps (small appends, which would leave most of the GPU idle), each taking
+    // its positions through the atomic path
+    const int slices = p.slices, per_slice = 8 / slices;
+    for (long long item = r_lo * slices + (long long)blockIdx.x * wpb + (threadIdx.x >> 5); item <= r_hi * slices + slices - 1;
+         item += (long long)gridDim.x * wpb) {
+        const long long r = item >= 0 ? item / slices : -((-item + slices - 1) / slices);
+        const int slice = (int)(item - r * slices);
         // a record lies wholly inside or wholly outside [0, limit): limit is a multiple of 16
         if (8 * r < 0 || 8 * r >= limit) {
             if (lane == 0) atomicOr(p.err, kErrBadPosition);
@@ -177,16 +183,22 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
         }
         uint8_t* page = p.pool + ((long long)blk * p.n_kv_heads + h) * page_bytes(D);
         const int tau0 = (int)((8 * r) % kPageTokens);   // 0 or 8: the record within the page
-        const long long p0 = 8 * r > start ? 8 * r : start, p1 = 8 * r + 8 < end ? 8 * r + 8 : end;
+        long long p0 = 8 * r > start ? 8 * r : start, p1 = 8 * r + 8 < end ? 8 * r + 8 : end;
+        if (slices > 1) {
+            const long long s0 = 8 * r + slice * per_slice, s1 = s0 + per_slice;
+            p0 = p0 > s0 ? p0 : s0;
+            p1 = p1 < s1 ? p1 : s1;
+            if (p0 >= p1) continue;
+        }
         const int c0 = l * CPL;
-        if (p1 - p0 == 8) {
+        if (slices == 1 && p1 - p0 == 8) {
             // the whole record: V words assembled in registers (the TPW tokens of each step
             // in separate lanes, combined below), plain stores
             uint32_t vw[CPL];
 #pragma unroll
             for (int i = 0; i < CPL; i++) vw[i] = 0u;
-#pragma unroll 2
-            for (int t2 = 0; t2 < 8; t2 += TPW) {
+#pragma unroll
+            for (int t2 = 0; t2 < 8; t2 += TPW) {   // unrolled: every token's loads in flight at once
                 const int tt = t2 + sub;
                 TokenCodes<CPL> tc;
                 quantize_token<D, T>(p, tok0 + (8 * r + tt - start), h, l, tc);
@@ -232,16 +244,19 @@ template <int D>
 static cudaError_t launch_append_d(const AppendParams& p, int n_sm, cudaStream_t st) {
     if (p.n_seqs > 65535 || p.n_kv_heads > 65535) return cudaErrorInvalidConfiguration;
     const int wpb = 8;
-    // records of one sequence: at most n_tokens / 8 + 2; about 8 CTAs per SM in all
-    const long long per_seq = ((long long)p.n_tokens / 8 + 2 + wpb - 1) / wpb;
+    // records of one sequence: at most n_tokens / 8 + 2; about 8 CTAs per SM in all.  A small
+    // append (its records x 4 within 16 warps per SM) splits every record over 4 warps.
     const long long units = (long long)p.n_seqs * p.n_kv_heads;
+    AppendParams q = p;
+    q.slices = ((long long)p.n_tokens / 8 + p.n_seqs) * p.n_kv_heads * 4 <= (long long)n_sm * 16 ? 4 : 1;
+    const long long per_seq = (((long long)p.n_tokens / 8 + 2) * q.slices + wpb - 1) / wpb;
     const long long fill = ((long long)n_sm * 8 + units - 1) / units;
     const long long gx = std::max<long long>(1, std::min(per_seq, fill));
     const dim3 grid((unsigned)gx, (unsigned)p.n_seqs, (unsigned)p.n_kv_heads);
     switch (p.dtype) {
-        case 0: append_kernel<D, float><<<grid, wpb * 32, 0, st>>>(p); break;
-        case 1: append_kernel<D, __nv_bfloat16><<<grid, wpb * 32, 0, st>>>(p); break;
-        default: append_kernel<D, __half><<<grid, wpb * 32, 0, st>>>(p); break;
+        case 0: append_kernel<D, float><<<grid, wpb * 32, 0, st>>>(q); break;
+        case 1: append_kernel<D, __nv_bfloat16><<<grid, wpb * 32, 0, st>>>(q); break;
+        default: append_kernel<D, __half><<<grid, wpb * 32, 0, st>>>(q); break;
     }
     return cudaGetLastError();
 }

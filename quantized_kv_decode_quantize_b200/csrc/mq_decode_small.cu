@@ -266,7 +266,19 @@ __global__ void __launch_bounds__(Sm<D, ROWS, NSG>::THREADS, Sm<D, ROWS, NSG>::C
         // The kernel is a programmatic dependent launch: a preceding kernel that allows it
         // (the append of this step) may still be writing pages.  Wait for it to complete
         // before the first page is read; everything before this point reads only the
-        // launch's inputs, which no such kernel writes.
+        // launch's inputs, which no such kernel writes.  Meanwhile the pages of the first
+        // ring-full of chunks are brought into L2 (a prefetch moves no data to the SM and
+        // has no effect on what a later read returns: a page the append rewrites is read
+        // from L2 after the wait like any other).
+        {
+            // lane = page (lane % 8) of chunk lane / 8: up to four chunks in one round of loads
+            const int i = lane / kChunkPages, lp = (c0 + i) * kChunkPages + lane % kChunkPages;
+            if (i < NS && i < n_ck && lp < n_pages) {
+                const int blk = __ldg(p.block_table + (long long)b * p.max_blocks_per_seq + p.bt_col + lp);
+                if (blk >= 0 && (long long)blk < p.n_blocks)
+                    bulk_prefetch_l2(p.pool + ((long long)blk * p.n_kv_heads + hk) * T::PB, T::PB);
+            }
+        }
         asm volatile("griddepcontrol.wait;" ::: "memory");
         const uint64_t policy = l2_evict_first_policy();
         auto bt_load = [&](int i) -> int {

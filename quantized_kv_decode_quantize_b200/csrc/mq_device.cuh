@@ -130,6 +130,12 @@ __device__ __forceinline__ void tma_load_1d(uint32_t dst, const void* src, uint3
         : "memory");
 }
 
+// A hint that brings [src, src + bytes) into L2 (16-byte multiple); no data moves to the
+// SM and nothing waits on it.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

@@ -19,6 +19,7 @@ struct AppendParams {
     const int32_t* block_table;
     int max_blocks_per_seq;
     unsigned* err;
+    int slices;   // warps per 8-position record (1, or 4 for small appends; set by the launch)
 };
 
 cudaError_t launch_append(const AppendParams& p, int head_dim, int n_sm, cudaStream_t st);
