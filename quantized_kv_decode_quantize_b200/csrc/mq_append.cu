@@ -142,6 +142,12 @@ __device__ __forceinline__ void store_token_kscales(uint8_t* page, int tau, int 
     if (l % LPG == 0) *reinterpret_cast<__half*>(page + v_scale_byte(D, tau, c0 / 32)) = tc.sv16;
 }
 
+// The kernel is a programmatic dependent launch: the preceding kernel on the stream may
+// still run (a decode or merge of the previous step, which may read the pages written
+// here).  The new tokens are read and quantized at once; each thread waits for that
+// kernel to complete before its first page write.
+__device__ __forceinline__ void grid_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 template <int D, typename T>
 __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     using LN = Lanes<D, T>;
@@ -197,11 +203,12 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
             uint32_t vw[CPL];
 #pragma unroll
             for (int i = 0; i < CPL; i++) vw[i] = 0u;
-#pragma unroll
-            for (int t2 = 0; t2 < 8; t2 += TPW) {   // unrolled: every token's loads in flight at once
+#pragma unroll 2
+            for (int t2 = 0; t2 < 8; t2 += TPW) {
                 const int tt = t2 + sub;
                 TokenCodes<CPL> tc;
                 quantize_token<D, T>(p, tok0 + (8 * r + tt - start), h, l, tc);
+                if (t2 == 0) grid_wait();
                 store_token_kscales<D, CPL>(page, tau0 + tt, l, tc);
                 const int bit = v_nibble_bit(tt);
 #pragma unroll
@@ -226,6 +233,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
                 // (their shuffles must run) and store nothing
                 quantize_token<D, T>(p, tok0 + ((here ? pos : p0) - start), h, l, tc);
                 if (!here) continue;
+                grid_wait();
                 const int tau = (int)(pos % kPageTokens);
                 store_token_kscales<D, CPL>(page, tau, l, tc);
                 const int bit = v_nibble_bit(tau);
@@ -253,12 +261,20 @@ static cudaError_t launch_append_d(const AppendParams& p, int n_sm, cudaStream_t
     const long long fill = ((long long)n_sm * 8 + units - 1) / units;
     const long long gx = std::max<long long>(1, std::min(per_seq, fill));
     const dim3 grid((unsigned)gx, (unsigned)p.n_seqs, (unsigned)p.n_kv_heads);
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(wpb * 32);
+    cfg.stream = st;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
     switch (p.dtype) {
-        case 0: append_kernel<D, float><<<grid, wpb * 32, 0, st>>>(q); break;
-        case 1: append_kernel<D, __nv_bfloat16><<<grid, wpb * 32, 0, st>>>(q); break;
-        default: append_kernel<D, __half><<<grid, wpb * 32, 0, st>>>(q); break;
+        case 0: return cudaLaunchKernelEx(&cfg, append_kernel<D, float>, q);
+        case 1: return cudaLaunchKernelEx(&cfg, append_kernel<D, __nv_bfloat16>, q);
+        default: return cudaLaunchKernelEx(&cfg, append_kernel<D, __half>, q);
     }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_append(const AppendParams& p, int head_dim, int n_sm, cudaStream_t st) {
