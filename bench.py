@@ -532,7 +532,7 @@ def run_mq(args, rank, world, local):
     if args.decode_config:
         r_, s_, w_ = (int(x) for x in args.decode_config.split(","))
         for k in range(3):
-            mq.mq_set_decode_config(cache.handle, k, r_, s_, 8 if k == 2 else w_)
+            mq.mq_set_decode_config(cache.handle, k, r_, s_, max(w_, 8) if k == 2 else min(w_, 8))
     if args.tune > 0:
         mq.mq_tune(cache.handle, args.tune, w.n_q_heads)
 
