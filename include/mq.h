@@ -429,7 +429,12 @@ mq_status mq_draft_ngram(const int32_t* tokens, int32_t max_len, const int32_t* 
  *                  <= 8, head_dim 128; GQA <= 4 at head_dim 256) merge fixed runs
  *                  of chunks over one fixed binary tree whose shape depends on the
  *                  sequence length alone, a CTA taking an aligned power-of-two run
- *                  of them: there the split count never changes the output.  The
+ *                  of them: there the split count never changes the output.  With
+ *                  several sequences in such a call the CTAs are one flat grid of
+ *                  about splits_per_sm x (CTAs per SM) x (number of SMs): the
+ *                  device reads every sequence's length and gives each (sequence,
+ *                  kv-head) CTAs in proportion to its own length (the run of
+ *                  chunks per CTA is the smallest power of two whose CTAs fit).  The
  *                  wider blocks (draft verification) accumulate each CTA's range in
  *                  token order, so there it sets the rounding of the output.
  *   softmax_warps  4 or 8: warps that turn one chunk's scores into weights; with

@@ -84,24 +84,35 @@ static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int row
     splits = std::max<long long>(1, std::min<long long>({splits, max_chunks, (long long)kMaxSplits}));
     const int kmax = small_leaf_kmax(c->head_dim, pl.rows);
     if (kmax > 0) {
-        // 2^kmax leaf slots per unit, each leaf ceil(max_chunks / 2^kmax) chunks: the unit
-        // fills the slots up to less than one chunk per slot, so aligned power-of-two CTA
-        // ranges of leaves stay balanced whatever max_chunks is
+        // at most 2^kmax leaves per unit, each ceil(max_chunks / 2^kmax) chunks (the unit
+        // fills its leaves up to less than one chunk per leaf).  Every CTA takes an aligned
+        // power-of-two run of leaves (lpc): the smallest lpc whose CTAs fit splits_per_sm x
+        // (CTAs per SM) x (number of SMs).  With several sequences the grid is flat and the
+        // CTAs find lpc and their unit on the device from every sequence's length (each
+        // unit takes CTAs in proportion to its own length: flat_lpc / flat_locate); one
+        // sequence takes the run for max_seq_len on a (split, unit) grid.
         const long long slots = 1LL << kmax;
         const long long leaf = (max_chunks + slots - 1) / slots;
         const long long leaves = (max_chunks + leaf - 1) / leaf;
-        long long p2 = 1;
-        while (p2 * 2 <= std::min(splits, leaves)) p2 *= 2;
-        long long lpc = slots / p2;   // leaves per CTA, a power of two
-        while (lpc > 1 && (leaves + lpc / 2 - 1) / (lpc / 2) <= p2) lpc /= 2;
+        const long long budget = std::min<long long>((long long)cfg.splits_per_sm * cps * c->n_sm, 1LL << 30);
         pl.node_chunks = (int)leaf;
-        pl.cpc = (int)(lpc * leaf);
+        if (n_seqs > 1) {
+            pl.cpc = 0;
+            pl.cta_budget = (int)budget;
+            pl.flat_ctas = (int)std::max<long long>(budget, units);
+            pl.max_splits = (int)leaves;   // partial slots per unit: at most one CTA per leaf
+        } else {
+            long long lpc = 1;
+            while (lpc < 64 && units * ((leaves + lpc - 1) / lpc) > budget) lpc *= 2;
+            pl.cpc = (int)(lpc * leaf);
+            pl.max_splits = (int)((leaves + lpc - 1) / lpc);
+        }
     } else {
         const long long cpc = (max_chunks + splits - 1) / splits;
         pl.cpc = (int)cpc;
         pl.node_chunks = (int)cpc;
+        pl.max_splits = (int)((max_chunks + pl.cpc - 1) / pl.cpc);
     }
-    pl.max_splits = (int)((max_chunks + pl.cpc - 1) / pl.cpc);
     pl.merge = pl.max_splits > 1;
     // the ring is shortened (never below 2 stages) until the CTA fits in its share of
     // the SM's shared memory (1 KB of each CTA's share is reserved by the hardware)
@@ -163,6 +174,7 @@ mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void
     p.part_ml = reinterpret_cast<float*>(ws + off);
     off += al256(units * pl.max_splits * pl.rows * 2 * 4);
     p.part_o = reinterpret_cast<float*>(ws + off);
+    p.cta_budget = pl.cta_budget;
     p.split_stride = pl.max_splits;
     p.n_rb = pl.n_rb;
     p.cpc = pl.cpc;
@@ -174,7 +186,7 @@ mq_status launch_decode_plan(const mq_cache* c, const DecodePlan& pl, const void
     p.bt_col = view.bt_col;
     p.fixed_len = view.fixed_len;
     p.fixed_nq = view.fixed_nq;
-    e = launch_decode(p, c->head_dim, pl.rows, pl.groups, pl.max_splits, pl.merge, pl.smem, st);
+    e = launch_decode(p, c->head_dim, pl.rows, pl.groups, pl.max_splits, pl.flat_ctas, pl.merge, pl.smem, st);
     return e == cudaSuccess ? MQ_OK : MQ_ERR_CUDA;
 }
 

@@ -85,6 +85,90 @@ __device__ __forceinline__ uint32_t code_pair_hi(uint32_t x) {
 }
 
 
+// ---- balanced split counts (a flat grid) -------------------------------------------------
+// Where the split count is free (the decode classes), a launch with p.cta_budget > 0 gives
+// every unit of sequence b ceil(n_leaves_b / lpc) CTAs of lpc leaves each, lpc the smallest
+// power of two (at most 64, the leaves of the longest unit) whose total fits the budget:
+// short and long sequences then take work in proportion to their length, and every CTA
+// still holds an aligned power-of-two run of leaves (the fixed merge tree).  One warp
+// computes it (all 32 lanes call), reading every sequence's length.
+struct SeqShape {
+    int units, leaves;   // row blocks x kv-heads of the sequence, merge-tree leaves of each
+};
+__device__ __forceinline__ SeqShape seq_shape(const DecodeParams& p, int b, int rows_per_block) {
+    SeqShape sh{0, 0};
+    const int L = seq_len_of(p, b), nq = seq_nq_of(p, b);
+    if (nq < 1 || nq > p.max_q || nq > L ||
+        (long long)L + (long long)p.bt_col * kPageTokens > (long long)p.max_blocks_per_seq * kPageTokens)
+        return sh;
+    const int n_chunks = (L + kChunkTokens - 1) / kChunkTokens;
+    sh.leaves = (n_chunks + p.node_chunks - 1) / p.node_chunks;
+    sh.units = p.n_kv_heads * ((p.group * nq + rows_per_block - 1) / rows_per_block);
+    return sh;
+}
+// A flat grid's leaves per CTA (lpc): the smallest power of two (at most 64) for which
+// every unit's CTAs, sum over units of ceil(leaves / lpc), fit p.cta_budget.  One warp (all
+// 32 lanes call; lane = sequence, in rounds of 32); `first` returns the lane's shape from
+// the first round for flat_locate.
+__device__ __forceinline__ int flat_lpc(const DecodeParams& p, int rows_per_block, SeqShape& first) {
+    const unsigned FULL = 0xffffffffu;
+    const int lane = threadIdx.x & 31;
+    first = lane < p.n_seqs ? seq_shape(p, lane, rows_per_block) : SeqShape{0, 0};
+    long long need[7] = {0, 0, 0, 0, 0, 0, 0};
+    for (int b0 = 0; b0 < p.n_seqs; b0 += 32) {
+        SeqShape sh = first;
+        if (b0 > 0) sh = b0 + lane < p.n_seqs ? seq_shape(p, b0 + lane, rows_per_block) : SeqShape{0, 0};
+#pragma unroll
+        for (int k = 0; k < 7; k++) need[k] += (long long)sh.units * ((sh.leaves + (1 << k) - 1) >> k);
+    }
+#pragma unroll
+    for (int k = 0; k < 7; k++)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) need[k] += __shfl_xor_sync(FULL, need[k], o);
+    int lpc = 64;
+#pragma unroll
+    for (int k = 6; k >= 0; k--)
+        if (need[k] <= p.cta_budget) lpc = 1 << k;
+    return lpc;
+}
+// CTA `cta` of a flat grid: its sequence b, kv-head hk, row block rb and split sp (CTAs are
+// numbered unit by unit, sequences in order, each unit's splits consecutive); false when
+// the index is past the launch's work.  One warp, after flat_lpc.
+__device__ __forceinline__ bool flat_locate(const DecodeParams& p, int rows_per_block, int lpc, SeqShape first,
+                                            int cta, int& b, int& hk, int& rb, int& sp) {
+    const unsigned FULL = 0xffffffffu;
+    const int lane = threadIdx.x & 31;
+    long long base = 0;
+    for (int b0 = 0; b0 < p.n_seqs; b0 += 32) {
+        SeqShape sh = first;
+        if (b0 > 0) sh = b0 + lane < p.n_seqs ? seq_shape(p, b0 + lane, rows_per_block) : SeqShape{0, 0};
+        const int per_unit = (sh.leaves + lpc - 1) / lpc;
+        const long long cnt = (long long)sh.units * per_unit;
+        long long incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long v = __shfl_up_sync(FULL, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const long long excl = base + incl - cnt;
+        const unsigned who = __ballot_sync(FULL, cnt > 0 && cta >= excl && cta < excl + cnt);
+        if (who != 0u) {
+            const int src = __ffs(who) - 1;
+            const int local = (int)(cta - __shfl_sync(FULL, excl, src));
+            const int pu = __shfl_sync(FULL, per_unit, src);
+            const int nrb = __shfl_sync(FULL, sh.units, src) / p.n_kv_heads;
+            b = b0 + src;
+            const int unit = local / pu;
+            sp = local % pu;
+            hk = unit / nrb;
+            rb = unit % nrb;
+            return true;
+        }
+        base += __shfl_sync(FULL, incl, 31);
+    }
+    return false;
+}
+
 // ---- the merge tree over a unit's leaves -----------------------------------------------
 // A unit's leaves are runs of node_chunks chunks; the tree over them is fixed: node (k, i)
 // covers leaves [i 2^k, (i + 1) 2^k), merges nodes (k - 1, 2i) and (k - 1, 2i + 1), and is

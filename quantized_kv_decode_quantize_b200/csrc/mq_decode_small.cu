@@ -138,8 +138,49 @@ __global__ void __launch_bounds__(Sm<D, ROWS, NSG>::THREADS, Sm<D, ROWS, NSG>::C
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int NS = p.stages;
     const SmallSmem S = small_layout<D, ROWS, NSG>(NS);
-    const int b = blockIdx.z, hk = blockIdx.y / p.n_rb, rb = blockIdx.y % p.n_rb, sp = blockIdx.x;
     const unsigned FULL = 0xffffffffu;
+    int* misc = reinterpret_cast<int*>(smem + S.misc);   // 0 qoff, 1 abort, 3 TMEM base, 5-9 flat plan
+
+    // ---- this CTA's unit (sequence, kv-head, row block) and split ----
+    int b, hk, rb, sp, cpc;
+    bool flat = false;
+    if constexpr (T::KMAX > 0) flat = p.cta_budget > 0;   // only the fixed-tree classes run flat grids
+    if (flat) {
+        // a flat grid: warp 0 finds the launch's leaves per CTA and this CTA's unit
+        if (warp == 0) {
+            SeqShape first;
+            const int lpc = flat_lpc(p, ROWS, first);
+            int fb = -1, fh = 0, fr = 0, fs = 0;
+            if (!flat_locate(p, ROWS, lpc, first, blockIdx.x, fb, fh, fr, fs)) fb = -1;
+            if (lane == 0) {
+                misc[5] = fb;
+                misc[6] = fh;
+                misc[7] = fr;
+                misc[8] = fs;
+                misc[9] = lpc;
+            }
+            if (blockIdx.x == 0)   // sequences with bad bounds take no CTA: flagged here
+                for (int bb = lane; bb < p.n_seqs; bb += 32) {
+                    const int Lb = seq_len_of(p, bb), nb = seq_nq_of(p, bb);
+                    if (nb < 1 || nb > p.max_q || nb > Lb ||
+                        (long long)Lb + (long long)p.bt_col * kPageTokens > (long long)p.max_blocks_per_seq * kPageTokens)
+                        atomicOr(p.err, kErrBadSeq);
+                }
+        }
+        __syncthreads();
+        if (misc[5] < 0) return;   // past the launch's work
+        b = misc[5];
+        hk = misc[6];
+        rb = misc[7];
+        sp = misc[8];
+        cpc = misc[9] * p.node_chunks;
+    } else {
+        b = blockIdx.z;
+        hk = blockIdx.y / p.n_rb;
+        rb = blockIdx.y % p.n_rb;
+        sp = blockIdx.x;
+        cpc = p.cpc;
+    }
 
     // ---- sequence bounds (uniform per CTA) ----
     const int L = seq_len_of(p, b), nq = seq_nq_of(p, b);
@@ -153,15 +194,15 @@ __global__ void __launch_bounds__(Sm<D, ROWS, NSG>::THREADS, Sm<D, ROWS, NSG>::C
     const int rows_here = min(ROWS, rows_b - row0);
     const int n_pages = (L + kPageTokens - 1) / kPageTokens;
     const int n_chunks = (L + kChunkTokens - 1) / kChunkTokens;
-    const int c0 = sp * p.cpc;
+    const int c0 = sp * cpc;
     if (c0 >= n_chunks) return;
-    const int n_ck = min(c0 + p.cpc, n_chunks) - c0;
+    const int n_ck = min(c0 + cpc, n_chunks) - c0;
     // The merge tree's leaves are runs of node_chunks chunks, folded in order; the CTA's
     // range is whole leaves, and its partial is the tree node over them (see tree_step).
     // The unit's only CTA writes out and lse; otherwise merge_kernel combines the partials.
     const int node_ch = p.node_chunks;
     const int l0 = c0 / node_ch, l1 = (c0 + n_ck + node_ch - 1) / node_ch;   // this CTA's leaves
-    const bool direct = (n_chunks + p.cpc - 1) / p.cpc == 1;                // the unit's only CTA
+    const bool direct = (n_chunks + cpc - 1) / cpc == 1;                    // the unit's only CTA
     const size_t pidx = ((size_t)(b * p.n_kv_heads + hk) * p.n_rb + rb);
     auto leaf_end = [&](int c) { return c % node_ch == node_ch - 1 || c == n_chunks - 1; };
 
@@ -176,7 +217,6 @@ __global__ void __launch_bounds__(Sm<D, ROWS, NSG>::THREADS, Sm<D, ROWS, NSG>::C
 
     // the dependent merge kernel may be scheduled now; it waits for this grid to complete
     if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    int* misc = reinterpret_cast<int*>(smem + S.misc);   // 0 qoff, 1 abort, 3 TMEM base
     volatile int* abort_flag = misc + 1;
     float* crow_s = reinterpret_cast<float*>(smem + S.crow);
     int* lim_s = reinterpret_cast<int*>(smem + S.lim);

@@ -25,6 +25,7 @@ namespace mq {
 struct DecodePlan {
     int cls, rows, groups, n_rb, stages, cpc, max_splits;
     int node_chunks;               // merge-tree leaf (chunks)
+    int cta_budget, flat_ctas;     // > 0: a flat grid of flat_ctas CTAs, balanced on the device
     bool merge;                    // some unit has several CTAs (merge_kernel completes the tree)
     size_t smem;
 };

@@ -66,8 +66,9 @@ struct DecodeParams {
     float* part_o;       // [n_seqs][n_kv_heads][n_rb][split_stride][rows][D]
     int split_stride;    // partial slots per unit (>= the CTAs of any unit)
     int n_rb;            // row blocks per kv-head
-    int cpc;             // chunks per CTA (a multiple of node_chunks)
+    int cpc;             // chunks per CTA (a multiple of node_chunks); with cta_budget, set per launch on the device
     int node_chunks;     // chunks per merge-tree leaf
+    int cta_budget;      // > 0: a flat grid whose units take CTAs by their own length (flat_lpc, flat_locate)
     int stages;          // TMA ring depth in chunks
     unsigned* err;
     // How the launch sees each sequence (the cascade's two passes use these; a plain
@@ -105,7 +106,7 @@ cudaError_t launch_prefill(const DecodeParams& p, int max_tiles, cudaStream_t st
 size_t decode_smem_bytes(int head_dim, int rows, int groups, int stages);   // 0: not built / does not fit
 cudaError_t decode_prepare(int head_dim, int rows, int groups, size_t smem);  // raises the dynamic smem limit
 int decode_ctas_per_sm(int head_dim, int rows);                    // CTAs the kernel is built to co-host
-cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int groups, int max_splits, bool merge, size_t smem,
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, int rows, int groups, int max_splits, int flat_ctas, bool merge, size_t smem,
                           cudaStream_t st);
 
 // Fills n values of dtype with a deterministic pseudo-random pattern (uniform in

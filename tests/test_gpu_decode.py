@@ -196,6 +196,43 @@ def test_split_count_bit_identical_for_decode_classes(shape):
     _check(case)
 
 
+def test_flat_grid_many_sequences_of_very_different_lengths():
+    """36 sequences (more than one warp's worth: the device planner reads their lengths in
+    two rounds) from 1 token to 40000: the units take CTAs in proportion to their own
+    lengths, chosen on the device; every split budget and ring depth gives the same bytes,
+    within tolerance of the oracle."""
+    rng = np.random.default_rng(5)
+    lens = [1, 40000, 16, 17, 2048] + np.floor(np.exp(rng.uniform(0.0, math.log(40000), 31))).astype(int).tolist()
+    w = wl.Workload("flat_many", 32, 8, 128, lens, [1] * len(lens), [1] * len(lens))
+    case = GpuCase(w)
+    ref = [t.clone() for t in case.decode()]
+    assert case.status() == mq.MQ_OK
+    for sps in SPLITS_PER_SM:
+        for r in (2, 4):
+            mq.mq_set_decode_config(case.cache.handle, 0, r, sps)
+            out, lse = case.decode()
+            assert case.status() == mq.MQ_OK
+            assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1]), (sps, r)
+    _check(case)
+
+
+def test_flat_grid_bad_sequence_is_flagged_and_the_others_unchanged():
+    """A sequence with an out-of-range length in a batch: the device error word is set, the
+    sequence takes no CTA, and every other sequence's output keeps its bytes."""
+    w = wl.Workload("flat_bad", 32, 8, 128, [20000, 3000, 9000, 500], [1] * 4, [1] * 4)
+    case = GpuCase(w)
+    ref = [t.clone() for t in case.decode()]
+    assert case.status() == mq.MQ_OK
+    bad = case.seq_lens.clone()
+    bad[1] = w.max_blocks() * 16 + 5
+    mq.mq_decode_attn(case.cache.handle, case.q, mq.MQ_BF16, w.n_seqs, w.n_q_heads, w.total_q, w.max_q,
+                      w.max_seq_len, case.tabs[0], w.max_blocks(), bad, case.n_q, 1.0 / math.sqrt(w.head_dim),
+                      case.out, case.lse, case.ws, case.ws.numel())
+    assert case.status() == mq.MQ_ERR_DEVICE
+    keep = [0, 2, 3]   # one query row per sequence
+    assert torch.equal(case.out[keep], ref[0][keep]) and torch.equal(case.lse[keep], ref[1][keep])
+
+
 @pytest.mark.parametrize("shape", ["gqa8", "drafts4", "d256_gqa8", "d256_drafts4"])
 def test_softmax_warps_bit_identical(shape):
     """Splitting a row block over two groups of softmax warps never changes the output."""
