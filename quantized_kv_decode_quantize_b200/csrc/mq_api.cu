@@ -86,15 +86,20 @@ static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int row
     if (kmax > 0) {
         // at most 2^kmax leaves per unit, each ceil(max_chunks / 2^kmax) chunks (the unit
         // fills its leaves up to less than one chunk per leaf).  Every CTA takes an aligned
-        // power-of-two run of leaves (lpc): the smallest lpc whose CTAs fit splits_per_sm x
-        // (CTAs per SM) x (number of SMs).  With several sequences the grid is flat and the
+        // power-of-two run of leaves (lpc): the smallest lpc whose CTAs fit the CTA budget
+        // below.  With several sequences the grid is flat and the
         // CTAs find lpc and their unit on the device from every sequence's length (each
         // unit takes CTAs in proportion to its own length: flat_lpc / flat_locate); one
         // sequence takes the run for max_seq_len on a (split, unit) grid.
         const long long slots = 1LL << kmax;
         const long long leaf = (max_chunks + slots - 1) / slots;
         const long long leaves = (max_chunks + leaf - 1) / leaf;
-        const long long budget = std::min<long long>((long long)cfg.splits_per_sm * cps * c->n_sm, 1LL << 30);
+        // the CTA budget: splits_per_sm x (CTAs per SM) x (number of SMs), and with several
+        // sequences at least 4 CTAs per unit on average (with about one CTA slot per unit,
+        // the power-of-two run that fits is too coarse for lengths that differ widely: the
+        // longest sequence's units would each go to one CTA)
+        long long budget = std::min<long long>((long long)cfg.splits_per_sm * cps * c->n_sm, 1LL << 30);
+        if (n_seqs > 1) budget = std::min<long long>(std::max<long long>(budget, 4 * units), 1LL << 30);
         pl.node_chunks = (int)leaf;
         if (n_seqs > 1) {
             pl.cpc = 0;
