@@ -20,9 +20,9 @@ replayed right after the timed region.  Multi-GPU (torchrun): every rank runs it
 replica (the work shards over independent sessions; no collective on the data path),
 the time is the max over ranks, and the value is the whole job's bytes / that time.
 
-`e2e` times the same step through the C ABI from pinned HOST buffers: per step an
-H2D copy of q and the new K/V, the two calls, a D2H copy of out and lse, and a
-stream synchronize.  `--impl reference` runs the CPU oracle (the reference arm) on
+`e2e` times the same step through the C ABI from pinned HOST buffers: per step one
+H2D copy of the step's inputs (q and the new K/V, packed in one buffer), the two
+calls, one D2H copy of the results (out and lse, packed), and a stream synchronize.  `--impl reference` runs the CPU oracle (the reference arm) on
 a bounded sample of the same workload on the host cores.
 """
 from __future__ import annotations
@@ -240,6 +240,25 @@ def run_prefill(args, rank, world, local):
 def peak_kind_note(kind):
     return (f"{kind} dense bf16 (fp16 runs at the same rate); the kernel issues 1.5x the algorithmic "
             f"MMA work (values as hi + lo)")
+
+
+def packed_buffer(specs, device):
+    """One byte buffer holding tensors of the given (shape, dtype), each at a 256-byte
+    aligned offset (pinned when on the host); returns the buffer and the views."""
+    import torch
+    offs, off = [], 0
+    for shape, dt in specs:
+        offs.append(off)
+        n = math.prod(shape) * torch.empty((), dtype=dt).element_size()
+        off = (off + n + 255) // 256 * 256
+    buf = torch.zeros(off, dtype=torch.uint8, device=device)
+    if device == "cpu":
+        buf = buf.pin_memory()
+    views = []
+    for (shape, dt), o in zip(specs, offs):
+        n = math.prod(shape) * torch.empty((), dtype=dt).element_size()
+        views.append(buf[o: o + n].view(dt).view(shape))
+    return buf, views
 
 
 def kernel_source_hash():
@@ -537,15 +556,21 @@ def run_mq(args, rank, world, local):
         mq.mq_tune(cache.handle, args.tune, w.n_q_heads)
 
     n_new = [int(x.shape[0]) for x in step_k]
-    new_k = torch.cat(step_k).to(dev).contiguous()
-    new_v = torch.cat(step_v).to(dev).contiguous()
+    # the step's inputs (q, new K, new V) share one device buffer and its results (out,
+    # lse) another, so that a step from host memory is one copy each way
+    h_k_src, h_v_src = torch.cat(step_k).contiguous(), torch.cat(step_v).contiguous()
+    in_specs = [(tuple(inp.q.shape), inp.q.dtype), (tuple(h_k_src.shape), h_k_src.dtype),
+                (tuple(h_v_src.shape), h_v_src.dtype)]
+    res_specs = [((w.total_q, w.n_q_heads, w.head_dim), torch.float32), ((w.total_q, w.n_q_heads), torch.float32)]
+    d_in, (q, new_k, new_v) = packed_buffer(in_specs, dev)
+    d_res, (out, lse) = packed_buffer(res_specs, dev)
+    q.copy_(inp.q.to(dev))
+    new_k.copy_(h_k_src.to(dev))
+    new_v.copy_(h_v_src.to(dev))
     cu_new = torch.tensor(np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32), device=dev)
     start = torch.tensor([L - a for L, a in zip(w.seq_lens, w.n_append)], **i32)
-    q = inp.q.to(dev).contiguous()
     seq_lens = torch.tensor(w.seq_lens, **i32)
     n_q = torch.tensor(w.n_q, **i32)
-    out = torch.empty((w.total_q, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
-    lse = torch.empty((w.total_q, w.n_q_heads), dtype=torch.float32, device=dev)
     cascade = bool(args.cascade and w.shared_prefix)
     if cascade:
         ws_bytes = mq.mq_decode_cascade_workspace_bytes(cache.handle, w.n_seqs, w.n_q_heads, w.total_q, w.max_q,
@@ -674,37 +699,31 @@ def run_mq(args, rank, world, local):
     # ---- e2e through the C ABI from pinned host buffers ----
     e2e = None
     if not args.no_e2e:
-        h_q = inp.q.contiguous().pin_memory()
-        h_k = torch.cat(step_k).contiguous().pin_memory()
-        h_v = torch.cat(step_v).contiguous().pin_memory()
-        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h_in, (hq_, hk_, hv_) = packed_buffer(in_specs, "cpu")
+        hq_.copy_(inp.q)
+        hk_.copy_(h_k_src)
+        hv_.copy_(h_v_src)
+        h_res, _ = packed_buffer(res_specs, "cpu")
         K2 = min(args.steps, 2000)
         with torch.cuda.stream(stream):
             for i in range(min(args.warmup, 50)):
-                q.copy_(h_q, non_blocking=True)
-                new_k.copy_(h_k, non_blocking=True)
-                new_v.copy_(h_v, non_blocking=True)
+                d_in.copy_(h_in, non_blocking=True)
                 step(i % copies, stream)
-                h_out.copy_(out, non_blocking=True)
-                h_lse.copy_(lse, non_blocking=True)
+                h_res.copy_(d_res, non_blocking=True)
                 stream.synchronize()
             if world > 1:
                 dist.barrier()
             torch.cuda.synchronize(dev)
             e0 = time.perf_counter()
             for i in range(K2):
-                q.copy_(h_q, non_blocking=True)
-                new_k.copy_(h_k, non_blocking=True)
-                new_v.copy_(h_v, non_blocking=True)
+                d_in.copy_(h_in, non_blocking=True)
                 step(i % copies, stream)
-                h_out.copy_(out, non_blocking=True)
-                h_lse.copy_(lse, non_blocking=True)
+                h_res.copy_(d_res, non_blocking=True)
                 stream.synchronize()
             e_dt = time.perf_counter() - e0
         e_dt = max_over_ranks(e_dt, dev)
-        h2d = h_q.numel() * h_q.element_size() + h_k.numel() * h_k.element_size() * 2
-        d2h = h_out.numel() * 4 + h_lse.numel() * 4
+        h2d = h_in.numel()
+        d2h = h_res.numel()
         e2e = {"value": world * step_bytes * K2 / e_dt / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": K2, "ms_per_step": e_dt / K2 * 1e3}
 
