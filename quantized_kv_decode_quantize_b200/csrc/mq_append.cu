@@ -5,8 +5,9 @@
 // scale"), with this library's symmetric reading:
 //   K per (token, kv-head):        s = fp16_rn(max|x| / 127), code = clamp(rne(x / s), -127, 127)
 //   V per (token, kv-head, 32 ch): s = fp16_rn(max|x| / 7),   code = clamp(rne(x / s), -8, 7)
-// Both divisions are IEEE fp32 (__fdiv_rn), rounding is to nearest even, and a
-// zero scale gives code 0.
+// Both divisions are IEEE fp32 (x / s is decided by a multiply with 1/s except next to
+// a tie, where __fdiv_rn decides: quant_code), rounding is to nearest even, and a zero
+// scale gives code 0.
 //
 // Work split: one warp per (8-position record, kv-head) that a sequence's new tokens
 // touch; the grid is (x, sequence, kv-head), sized from the device's SM count, and the
@@ -62,10 +63,19 @@ __device__ __forceinline__ void load_vec(const T* p, float (&x)[N]) {
     }
 }
 
-__device__ __forceinline__ int quant_code(float x, float s, float lo, float hi) {
+// code = clamp(rne(x / s)) with x / s the IEEE fp32 quotient.  inv = 1/s and q = x * inv
+// (both correctly rounded) put q within |x / s| * 2^-22.4 of that quotient, under 2^-14
+// while |x / s| <= 256 (the scales make |x / s| at most ~127.1, and anything past 127.5
+// clamps the same way on both sides); so q and the quotient round to the same integer
+// unless q lies within 2^-14 of a half-integer, and only such elements (and NaN) take
+// the division.
+__device__ __forceinline__ int quant_code(float x, float s, float inv, float lo, float hi) {
     if (s == 0.0f) return 0;
-    float r = rintf(__fdiv_rn(x, s));   // IEEE division, round half to even
-    if (r != r) return 0;               // NaN input
+    float q = __fmul_rn(x, inv);
+    const float h = fabsf(__fsub_rn(__fsub_rn(q, floorf(q)), 0.5f));
+    if (!(h > 0x1p-14f)) q = __fdiv_rn(x, s);   // near a tie: the IEEE division decides
+    float r = rintf(q);                         // round half to even
+    if (r != r) return 0;                       // NaN input
     r = fminf(fmaxf(r, lo), hi);
     return static_cast<int>(r);
 }
@@ -105,13 +115,13 @@ __device__ __forceinline__ void quantize_token(const AppendParams& p, long long 
 #pragma unroll
     for (int o = LN::LPT / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     out.sk16 = __float2half_rn(__fdiv_rn(a, 127.0f));
-    const float sk = __half2float(out.sk16);
+    const float sk = __half2float(out.sk16), ik = __frcp_rn(sk);
 #pragma unroll
     for (int w = 0; w < CPL / 4; w++) {
         uint32_t word = 0;
 #pragma unroll
         for (int j = 0; j < 4; j++)
-            word |= (uint32_t)(quant_code(xk[4 * w + j], sk, -127.0f, 127.0f) & 0xFF) << (8 * j);
+            word |= (uint32_t)(quant_code(xk[4 * w + j], sk, ik, -127.0f, 127.0f) & 0xFF) << (8 * j);
         out.kb[w] = word;
     }
     // ---- V: one scale per 32-channel group (LPG lanes) ----
@@ -121,9 +131,9 @@ __device__ __forceinline__ void quantize_token(const AppendParams& p, long long 
 #pragma unroll
     for (int o = LPG / 2; o > 0; o >>= 1) av = fmaxf(av, __shfl_xor_sync(0xffffffffu, av, o));
     out.sv16 = __float2half_rn(__fdiv_rn(av, 7.0f));
-    const float sv = __half2float(out.sv16);
+    const float sv = __half2float(out.sv16), iv = __frcp_rn(sv);
 #pragma unroll
-    for (int i = 0; i < CPL; i++) out.vn[i] = (uint32_t)quant_code(xv[i], sv, -8.0f, 7.0f) & 0xFu;
+    for (int i = 0; i < CPL; i++) out.vn[i] = (uint32_t)quant_code(xv[i], sv, iv, -8.0f, 7.0f) & 0xFu;
 }
 
 // K codes, K scale and V scale of one token at slot tau of a page (lane l of the token).

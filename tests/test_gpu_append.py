@@ -132,6 +132,50 @@ def test_append_edge_vectors(D, dtype):
     assert np.array_equal(vp, evp) and np.array_equal(vs, evs)
 
 
+def _near_ties(rng, n_tok, D, group, div, n_lo, n_hi):
+    """Tokens whose elements sit at and a few ulps around (n + 1/2) * s, s the scale the
+    token's (or group's) first element sets: every code is decided next to a tie."""
+    x = np.zeros((n_tok, D), dtype=np.float32)
+    for t in range(n_tok):
+        for g0 in range(0, D, group):
+            m = np.float32(10.0 ** rng.uniform(-3, 3))
+            s = np.float32(np.float16(m / np.float32(div)))
+            n = rng.integers(n_lo, n_hi + 1, group).astype(np.float32)
+            v = ((n + np.float32(0.5)) * s).astype(np.float32)
+            k = rng.integers(-3, 4, group)
+            for _ in range(3):
+                step = np.where(k > 0, np.float32(np.inf), np.float32(-np.inf))
+                v = np.where(k != 0, np.nextafter(v, step), v).astype(np.float32)
+                k = k - np.sign(k)
+            v[0] = m
+            x[t, g0:g0 + group] = v
+    return x
+
+
+@pytest.mark.parametrize("D", [128, 256])
+def test_append_codes_next_to_ties_bit_exact(D):
+    """Every K and V element at, or up to 3 ulps from, a half-integer multiple of its
+    scale: the codes equal the oracle's IEEE-division codes bit for bit."""
+    rng = np.random.default_rng(11)
+    n = 64
+    xk = _near_ties(rng, n, D, D, 127.0, -126, 125)
+    xv = _near_ties(rng, n, D, 32, 7.0, -7, 5)
+    kt = torch.from_numpy(np.stack([xk, xk[::-1]], 1).copy())
+    vt = torch.from_numpy(np.stack([xv, xv[::-1]], 1).copy())
+    cache = mq.Cache(2, D, 4)
+    tab = torch.tensor([[1, 3, 0, 2]], dtype=torch.int32, device="cuda")
+    cu = torch.tensor([0, n], dtype=torch.int32, device="cuda")
+    sp = torch.tensor([0], dtype=torch.int32, device="cuda")
+    mq.mq_kv_append(cache.handle, kt.cuda(), vt.cuda(), 0, 1, n, cu, sp, tab, 4)
+    assert mq.mq_device_status(cache.handle) == mq.MQ_OK
+    kc, ks, vp, vs = pagelayout.gather_sequence(cache.pool.cpu().numpy(), 2, D, tab.cpu().numpy()[0], n)
+    ekc, eks = oracle.quantize_k(kt.numpy())
+    evp, evs = oracle.quantize_v(vt.numpy())
+    assert np.array_equal(ks, eks) and np.array_equal(vs, evs)
+    assert np.array_equal(kc, ekc), f"K codes differ at {np.argwhere(kc != ekc)[:4].tolist()}"
+    assert np.array_equal(vp, evp), f"V codes differ at {np.argwhere(vp != evp)[:4].tolist()}"
+
+
 def test_append_hand_worked_cases():
     """The hand-derived cases of tests/golden/quant_hand_cases.json, through the GPU."""
     g = oracle_pins.golden()
