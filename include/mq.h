@@ -430,9 +430,10 @@ mq_status mq_draft_ngram(const int32_t* tokens, int32_t max_len, const int32_t* 
  *                  of chunks over one fixed binary tree whose shape depends on the
  *                  sequence length alone, a CTA taking an aligned power-of-two run
  *                  of them: there the split count never changes the output.  With
- *                  several sequences in such a call the CTAs are one flat grid of
+ *                  2 to 64 sequences in such a call the CTAs are one flat grid of
  *                  about splits_per_sm x (CTAs per SM) x (number of SMs), and at
- *                  least 4 per (sequence, kv-head) on average: the
+ *                  least 4 per (sequence, kv-head) on average (up to 4 per
+ *                  CTA slot): the
  *                  device reads every sequence's length and gives each (sequence,
  *                  kv-head) CTAs in proportion to its own length (the run of
  *                  chunks per CTA is the smallest power of two whose CTAs fit).  The

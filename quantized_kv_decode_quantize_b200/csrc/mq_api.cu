@@ -90,18 +90,23 @@ static DecodePlan plan_for_class(const mq_cache* c, int cls, int n_seqs, int row
         // below.  With several sequences the grid is flat and the
         // CTAs find lpc and their unit on the device from every sequence's length (each
         // unit takes CTAs in proportion to its own length: flat_lpc / flat_locate); one
-        // sequence takes the run for max_seq_len on a (split, unit) grid.
+        // sequence, or more than kFlatMaxSeqs, takes the run for max_seq_len on a (split,
+        // unit) grid.
         const long long slots = 1LL << kmax;
         const long long leaf = (max_chunks + slots - 1) / slots;
         const long long leaves = (max_chunks + leaf - 1) / leaf;
-        // the CTA budget: splits_per_sm x (CTAs per SM) x (number of SMs), and with several
-        // sequences at least 4 CTAs per unit on average (with about one CTA slot per unit,
+        // the CTA budget: splits_per_sm x (CTAs per SM) x (number of SMs), and on a flat
+        // grid at least 4 CTAs per unit on average (with about one CTA slot per unit,
         // the power-of-two run that fits is too coarse for lengths that differ widely: the
         // longest sequence's units would each go to one CTA)
+        // Each CTA of a flat grid reads every sequence's length (rounds of 32), so flat
+        // grids are kept to batches of up to kFlatMaxSeqs sequences (two rounds); larger
+        // batches take the (split, unit) grid.  The floor is capped at 4 CTAs per slot.
+        const bool flat = n_seqs > 1 && n_seqs <= kFlatMaxSeqs;
         long long budget = std::min<long long>((long long)cfg.splits_per_sm * cps * c->n_sm, 1LL << 30);
-        if (n_seqs > 1) budget = std::min<long long>(std::max<long long>(budget, 4 * units), 1LL << 30);
+        if (flat) budget = std::max<long long>(budget, std::min<long long>(4 * units, 4LL * cps * c->n_sm));
         pl.node_chunks = (int)leaf;
-        if (n_seqs > 1) {
+        if (flat) {
             pl.cpc = 0;
             pl.cta_budget = (int)budget;
             pl.flat_ctas = (int)std::max<long long>(budget, units);

@@ -216,6 +216,23 @@ def test_flat_grid_many_sequences_of_very_different_lengths():
     _check(case)
 
 
+def test_batch_past_the_flat_grid_limit():
+    """80 sequences (more than a flat grid takes: the (split, unit) grid sized by the
+    longest): bit-identical for every split budget, within tolerance of the oracle."""
+    rng = np.random.default_rng(8)
+    lens = [9000, 1] + rng.integers(16, 3000, 78).tolist()
+    w = wl.Workload("past_flat", 16, 4, 128, lens, [1] * len(lens), [1] * len(lens))
+    case = GpuCase(w)
+    ref = [t.clone() for t in case.decode()]
+    assert case.status() == mq.MQ_OK
+    for sps in SPLITS_PER_SM:
+        mq.mq_set_decode_config(case.cache.handle, 0, 3, sps)
+        out, lse = case.decode()
+        assert case.status() == mq.MQ_OK
+        assert torch.equal(out, ref[0]) and torch.equal(lse, ref[1]), sps
+    _check(case)
+
+
 def test_flat_grid_bad_sequence_is_flagged_and_the_others_unchanged():
     """A sequence with an out-of-range length in a batch: the device error word is set, the
     sequence takes no CTA, and every other sequence's output keeps its bytes."""
