@@ -25,7 +25,6 @@ constexpr int kPageTokens = 16;
 constexpr int kChunkPages = 8;                  // tokens per canonical chunk = 128
 constexpr int kChunkTokens = kPageTokens * kChunkPages;
 constexpr int kMaxSplits = 64;                  // CTAs per (sequence, kv-head, row block)
-constexpr int kFlatMaxSeqs = 64;                // sequences of a call planned on the device (flat grid)
 
 __host__ __device__ constexpr int page_bytes(int D) { return 25 * D + 32; }
 __host__ __device__ constexpr int rec_bytes(int D) { return 25 * D / 2 + 16; }

@@ -22,6 +22,10 @@ struct mq_cache {
 
 namespace mq {
 
+// sequences of a call whose CTAs the device plans (a flat grid: every CTA reads every
+// sequence's length, in rounds of 32)
+constexpr int kFlatMaxSeqs = 64;
+
 struct DecodePlan {
     int cls, rows, groups, n_rb, stages, cpc, max_splits;
     int node_chunks;               // merge-tree leaf (chunks)
