@@ -685,6 +685,41 @@ def run_mq(args, rank, world, local):
                 app_ms.append(a0.elapsed_time(a1))
     app_avg = statistics.median(app_ms) if app_ms else None
 
+    # ---- verification against one decode step of the same sequences (several query
+    # tokens per sequence): each sequence's last query token alone, on the same caches;
+    # decode + merge by CUDA events, each call on a copy no recent call has read ----
+    verify_vs_decode = None
+    if w.max_q > 1 and not cascade:
+        last = torch.as_tensor(np.cumsum(w.n_q) - 1, dtype=torch.long, device=dev)
+        q1 = q[last].contiguous()
+        nq1 = torch.ones(w.n_seqs, **i32)
+        out1 = torch.empty((w.n_seqs, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+        lse1 = torch.empty((w.n_seqs, w.n_q_heads), dtype=torch.float32, device=dev)
+        ws1_bytes = mq.mq_decode_workspace_bytes(cache.handle, w.n_seqs, w.n_q_heads, 1, w.max_seq_len)
+        ws1 = torch.zeros(max(ws1_bytes, 256), dtype=torch.uint8, device=dev)
+        v_ms, d_ms = [], []
+        with torch.cuda.stream(stream):
+            for i in range(24):
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                e[0].record(stream)
+                mq.mq_decode_attn(cache.handle, q, dt_code, w.n_seqs, w.n_q_heads, w.total_q, w.max_q, w.max_seq_len,
+                                  tab_c[(2 * i) % copies], w.max_blocks(), seq_lens, n_q, scale, out, lse, ws,
+                                  ws_bytes, stream)
+                e[1].record(stream)
+                mq.mq_decode_attn(cache.handle, q1, dt_code, w.n_seqs, w.n_q_heads, w.n_seqs, 1, w.max_seq_len,
+                                  tab_c[(2 * i + 1) % copies], w.max_blocks(), seq_lens, nq1, scale, out1, lse1, ws1,
+                                  ws1_bytes, stream)
+                e[2].record(stream)
+                e[2].synchronize()
+                if i >= 4:
+                    v_ms.append(e[0].elapsed_time(e[1]))
+                    d_ms.append(e[1].elapsed_time(e[2]))
+        assert mq.mq_device_status(cache.handle, stream) == mq.MQ_OK
+        v_med, d_med = statistics.median(v_ms), statistics.median(d_ms)
+        verify_vs_decode = {"verify_us": v_med * 1e3, "decode_us": d_med * 1e3, "ratio": v_med / d_med,
+                            "decode": "the same sequences and caches, each sequence's last query token alone "
+                                      "(one decode step); decode + merge kernels by CUDA events, 20 calls each"}
+
     def pct(xs, q):
         xs = sorted(xs)
         return xs[min(len(xs) - 1, int(round(q * (len(xs) - 1))))] if xs else None
@@ -749,7 +784,8 @@ def run_mq(args, rank, world, local):
                        "decode_bytes_unique": dec_unique,
                        "append_bytes": app_bytes,
                        "append_us_median": app_avg * 1e3 if app_avg else None,
-                       "append_GBps": app_bytes / (app_avg * 1e-3) / 1e9 if app_avg else None},
+                       "append_GBps": app_bytes / (app_avg * 1e-3) / 1e9 if app_avg else None,
+                       **({"verify_vs_decode": verify_vs_decode} if verify_vs_decode else {})},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": (achieved / peak) if achieved else None, "peak_kind": peak_kind,
                          "traffic": ncu_traffic(w.name), "kernel": "mq::decode_small_kernel",
