@@ -242,9 +242,10 @@ def peak_kind_note(kind):
             f"MMA work (values as hi + lo)")
 
 
-def packed_buffer(specs, device):
+def packed_buffer(specs, device, pin=None):
     """One byte buffer holding tensors of the given (shape, dtype), each at a 256-byte
-    aligned offset (pinned when on the host); returns the buffer and the views."""
+    aligned offset (pinned when on the host, unless pin is False); returns the buffer and
+    the views."""
     import torch
     offs, off = [], 0
     for shape, dt in specs:
@@ -252,7 +253,7 @@ def packed_buffer(specs, device):
         n = math.prod(shape) * torch.empty((), dtype=dt).element_size()
         off = (off + n + 255) // 256 * 256
     buf = torch.zeros(off, dtype=torch.uint8, device=device)
-    if device == "cpu":
+    if (device == "cpu") if pin is None else pin:
         buf = buf.pin_memory()
     views = []
     for (shape, dt), o in zip(specs, offs):

@@ -66,3 +66,22 @@ def test_graph_never_longer_than_the_timed_steps():
     assert bench.graph_steps(6, 20000) == 24
     assert bench.graph_steps(6, 20) == 20
     assert bench.graph_steps(6, 20000, override=12) == 12
+
+
+def test_packed_buffer_views_are_aligned_and_disjoint():
+    """The e2e step's inputs and results each live in one buffer (one copy each way): every
+    view starts on a 256-byte boundary, views do not overlap, and writes land in place."""
+    import torch
+    import bench
+    specs = [((3, 32, 128), torch.bfloat16), ((5, 8, 128), torch.float32), ((7,), torch.float16)]
+    buf, views = bench.packed_buffer(specs, "cpu", pin=False)
+    spans = []
+    for (shape, dt), v in zip(specs, views):
+        off = v.data_ptr() - buf.data_ptr()
+        assert off % 256 == 0 and tuple(v.shape) == shape and v.dtype == dt and v.is_contiguous()
+        spans.append((off, off + v.numel() * v.element_size()))
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:])) and spans[-1][1] <= buf.numel()
+    for i, v in enumerate(views):
+        v.fill_(i + 1)
+    for i, v in enumerate(views):
+        assert bool((v == i + 1).all())
